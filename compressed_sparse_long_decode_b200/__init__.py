@@ -1,0 +1,241 @@
+"""Python binding of libcsld.so -- the hybrid compressed-attention (CSA + HCA) decode path on
+B200 (sm_100a).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels behind the C ABI
+declared in include/csld.h.  PyTorch provides device memory and streams.  There is no CPU
+fallback: if the shared library is missing, importing this package raises.
+
+Functions keep the C names (csa_compress, hca_compress, indexer_topk,
+hybrid_decode_attention, kv_cache_append, kv_cache_prefill) and take torch tensors on the
+current CUDA device; results are written into caller-provided tensors or freshly allocated
+ones, on torch's current stream.
+"""
+import ctypes as C
+import os
+
+import torch
+
+__all__ = [
+    "csa_compress", "hca_compress", "compress", "indexer_topk", "hybrid_decode_attention",
+    "kv_cache_append", "kv_cache_prefill", "LayerCache", "CsldError", "lib", "ENTRY_BYTES",
+    "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace",
+]
+
+DIM = 512
+DIM_NOPE = 448
+ENTRY_BYTES = 576
+IKEY_BYTES = 32
+HEADS = 16
+IDX_HEADS = 4
+IDX_DIM = 64
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsld.so")
+
+
+class CsldError(RuntimeError):
+    pass
+
+
+class _Cache(C.Structure):
+    _fields_ = [
+        ("ratio", C.c_int32), ("window", C.c_int32), ("batch", C.c_int32), ("has_indexer", C.c_int32),
+        ("capacity", C.c_int64), ("comp_kv", C.c_void_p), ("ikeys", C.c_void_p),
+        ("iscales", C.c_void_p), ("win_kv", C.c_void_p), ("tail_kv", C.c_void_p),
+        ("tail_gate", C.c_void_p), ("seq_len", C.c_void_p), ("pos_bias", C.c_void_p),
+        ("w_idx", C.c_void_p),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libcsld.so not found at {LIB_PATH}; build it with "
+                          "`python compressed_sparse_long_decode_b200/build.py`")
+    L = C.CDLL(LIB_PATH)
+    P, I, I64, F, S = C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_size_t
+    L.csld_abi_version.restype = I
+    L.csld_last_error.restype = C.c_char_p
+    L.csld_status_string.restype = C.c_char_p
+    L.csld_status_string.argtypes = [I]
+    L.csld_compress.argtypes = [P, P, P, I, P, I64, P, P, P, P]
+    L.csa_compress.argtypes = [P, P, P, P, I64, P, P, P, P]
+    L.hca_compress.argtypes = [P, P, P, I64, P, P]
+    L.kv_cache_append.argtypes = [C.POINTER(_Cache), P, P, P, P]
+    L.kv_cache_prefill.argtypes = [C.POINTER(_Cache), P, P, I64, P]
+    L.csld_indexer_workspace_size.restype = S
+    L.csld_indexer_workspace_size.argtypes = [I, I64, I]
+    L.indexer_topk.argtypes = [P, P, I64, P, I, P, P, I, I, P, P, S, P, P]
+    L.csld_attention_workspace_size.restype = S
+    L.csld_attention_workspace_size.argtypes = [I, I, I64, I, I]
+    L.hybrid_decode_attention.argtypes = [P, I, P, I64, I, P, I, P, I, P, I, F, P, P, P, S, P, P]
+    for fn in ("csld_compress", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
+               "indexer_topk", "hybrid_decode_attention"):
+        getattr(L, fn).restype = I
+    return L
+
+
+lib = _load()
+
+
+def _check(status, what):
+    if status != 0:
+        msg = lib.csld_last_error().decode()
+        raise CsldError(f"{what}: {lib.csld_status_string(status).decode()} ({msg})")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _need(t, dtype, name):
+    if t is None:
+        raise CsldError(f"{name} is required")
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise CsldError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {t.dtype} "
+                        f"{'cuda' if t.is_cuda else 'cpu'} contiguous={t.is_contiguous()}")
+    return t
+
+
+def _bits(t, name):
+    """bf16 tensor -> the same memory viewed as raw 16-bit patterns (no copy)."""
+    _need(t, torch.bfloat16, name)
+    return t
+
+
+# ---- compression ------------------------------------------------------------------------
+def compress(raw, gate, pos_bias, ratio, w_idx=None, kv_out=None, ikey_out=None, iscale_out=None):
+    """Prefill compression of one sequence: raw [T,512] bf16, gate [T] f32, pos_bias [ratio]."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    _need(pos_bias, torch.float32, "pos_bias")
+    T = raw.shape[0]
+    E = T // ratio
+    dev = raw.device
+    if kv_out is None:
+        kv_out = torch.empty((E, ENTRY_BYTES), dtype=torch.uint8, device=dev)
+    if w_idx is not None:
+        _need(w_idx, torch.float32, "w_idx")
+        if ikey_out is None:
+            ikey_out = torch.empty((E, IKEY_BYTES), dtype=torch.uint8, device=dev)
+        if iscale_out is None:
+            iscale_out = torch.empty((E, 2), dtype=torch.float32, device=dev)
+    _check(lib.csld_compress(_ptr(raw), _ptr(gate), _ptr(pos_bias), ratio, _ptr(w_idx), T,
+                             _ptr(kv_out), _ptr(ikey_out), _ptr(iscale_out), _stream()), "csld_compress")
+    return (kv_out, ikey_out, iscale_out) if w_idx is not None else kv_out
+
+
+def csa_compress(raw, gate, pos_bias, w_idx, kv_out=None, ikey_out=None, iscale_out=None):
+    return compress(raw, gate, pos_bias, 4, w_idx, kv_out, ikey_out, iscale_out)
+
+
+def hca_compress(raw, gate, pos_bias, kv_out=None):
+    return compress(raw, gate, pos_bias, 128, None, kv_out)
+
+
+# ---- cache state ------------------------------------------------------------------------
+class LayerCache:
+    """One layer's cache state for B sequences, in device memory owned by torch."""
+
+    def __init__(self, batch, capacity, ratio, window, pos_bias, w_idx=None, device="cuda"):
+        if w_idx is not None and capacity % 2:
+            capacity += 1
+        self.batch, self.capacity, self.ratio, self.window = batch, capacity, ratio, window
+        dev = torch.device(device)
+        self.comp_kv = torch.zeros((batch, capacity, ENTRY_BYTES), dtype=torch.uint8, device=dev)
+        self.has_indexer = w_idx is not None
+        self.ikeys = torch.zeros((batch, capacity, IKEY_BYTES), dtype=torch.uint8, device=dev) if self.has_indexer else None
+        self.iscales = torch.zeros((batch, capacity, 2), dtype=torch.float32, device=dev) if self.has_indexer else None
+        self.win_kv = torch.zeros((batch, max(window, 1), ENTRY_BYTES), dtype=torch.uint8, device=dev)
+        self.tail_kv = torch.zeros((batch, ratio, DIM), dtype=torch.bfloat16, device=dev)
+        self.tail_gate = torch.zeros((batch, ratio), dtype=torch.float32, device=dev)
+        self.seq_len = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.pos_bias = _need(pos_bias.to(dev).contiguous(), torch.float32, "pos_bias")
+        self.w_idx = _need(w_idx.to(dev).contiguous(), torch.float32, "w_idx") if self.has_indexer else None
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def struct(self):
+        return _Cache(self.ratio, self.window, self.batch, int(self.has_indexer), self.capacity,
+                      _ptr(self.comp_kv), _ptr(self.ikeys), _ptr(self.iscales), _ptr(self.win_kv),
+                      _ptr(self.tail_kv), _ptr(self.tail_gate), _ptr(self.seq_len),
+                      _ptr(self.pos_bias), _ptr(self.w_idx))
+
+
+def kv_cache_append(cache: LayerCache, kv_new, gate_new, err=None):
+    """Append one token per sequence: kv_new [B,512] bf16, gate_new [B] f32."""
+    _bits(kv_new, "kv_new")
+    _need(gate_new, torch.float32, "gate_new")
+    s = cache.struct()
+    _check(lib.kv_cache_append(C.byref(s), _ptr(kv_new), _ptr(gate_new),
+                               _ptr(cache.err if err is None else err), _stream()), "kv_cache_append")
+
+
+def kv_cache_prefill(cache: LayerCache, raw, gate):
+    """Prefill all sequences with T tokens: raw [B,T,512] bf16, gate [B,T] f32."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    s = cache.struct()
+    _check(lib.kv_cache_prefill(C.byref(s), _ptr(raw), _ptr(gate), raw.shape[1], _stream()),
+           "kv_cache_prefill")
+
+
+# ---- indexer ------------------------------------------------------------------------------
+def indexer_workspace(B, cap, k, device="cuda"):
+    n = lib.csld_indexer_workspace_size(B, cap, k)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def indexer_topk(ikeys, iscales, seq_len, ratio, q_idx, head_w, k, out=None, ws=None, err=None):
+    """ikeys [B,cap,32] u8, iscales [B,cap,2] f32, seq_len [B] i32, q_idx [B,4,64] f32,
+    head_w [B,4] f32 -> top-k entry indices [B,k] i32 (ascending, -1 padded)."""
+    _need(ikeys, torch.uint8, "ikeys")
+    _need(iscales, torch.float32, "iscales")
+    _need(seq_len, torch.int32, "seq_len")
+    _need(q_idx, torch.float32, "q_idx")
+    _need(head_w, torch.float32, "head_w")
+    B, cap = ikeys.shape[0], ikeys.shape[1]
+    if out is None:
+        out = torch.empty((B, k), dtype=torch.int32, device=ikeys.device)
+    if ws is None:
+        ws = indexer_workspace(B, cap, k, ikeys.device)
+    _check(lib.indexer_topk(_ptr(ikeys), _ptr(iscales), cap, _ptr(seq_len), ratio, _ptr(q_idx),
+                            _ptr(head_w), B, k, _ptr(out), _ptr(ws), ws.numel(), _ptr(err), _stream()),
+           "indexer_topk")
+    return out
+
+
+# ---- attention ----------------------------------------------------------------------------
+def attention_workspace(B, cap, k, W, device="cuda"):
+    n = lib.csld_attention_workspace_size(B, HEADS, cap, k, W)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def hybrid_decode_attention(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, out=None,
+                            lse=None, ws=None, err=None):
+    """q [B,16,512] bf16; comp_kv [B,cap,576] u8; topk [B,k] i32 or None (dense); win_kv
+    [B,W,576] u8; seq_len [B] i32 -> (out [B,16,512] f32, lse [B,16] f32)."""
+    _bits(q, "q")
+    _need(comp_kv, torch.uint8, "comp_kv")
+    _need(seq_len, torch.int32, "seq_len")
+    B, H = q.shape[0], q.shape[1]
+    cap = comp_kv.shape[1]
+    k = 0
+    if topk is not None:
+        _need(topk, torch.int32, "topk")
+        k = topk.shape[1]
+    if W > 0:
+        _need(win_kv, torch.uint8, "win_kv")
+    if out is None:
+        out = torch.empty((B, H, DIM), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = attention_workspace(B, cap, max(k, 1), W, q.device)
+    _check(lib.hybrid_decode_attention(_ptr(q), H, _ptr(comp_kv), cap, ratio, _ptr(topk), k,
+                                       _ptr(win_kv) if W > 0 else None, W, _ptr(seq_len), B,
+                                       float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                       _ptr(err), _stream()), "hybrid_decode_attention")
+    return out, lse

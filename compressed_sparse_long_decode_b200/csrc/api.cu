@@ -1,0 +1,202 @@
+// extern "C" entry points of libcsld: host-side validation, workspace sizing and launches.
+// Every check happens before anything is enqueued; a failed check launches nothing.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "csld_internal.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+csld_status fail(csld_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+csld_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(CSLD_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+csld_status check_cache(const csld_layer_cache* c) {
+    if (!c) return fail(CSLD_ERR_ARG, "cache is NULL");
+    if (c->ratio < 1 || c->ratio > CSLD_MAX_RATIO)
+        return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", c->ratio, CSLD_MAX_RATIO);
+    if (c->window < 0 || c->window > CSLD_MAX_WINDOW)
+        return fail(CSLD_ERR_ARG, "window %d outside 0..%d", c->window, CSLD_MAX_WINDOW);
+    if (c->batch < 1 || c->batch > 65535) return fail(CSLD_ERR_ARG, "batch %d outside 1..65535", c->batch);
+    if (c->capacity < 1 || c->capacity > (int64_t)INT32_MAX)
+        return fail(CSLD_ERR_ARG, "capacity %lld outside 1..2^31-1", (long long)c->capacity);
+    if (!c->comp_kv || !c->tail_kv || !c->tail_gate || !c->seq_len || !c->pos_bias)
+        return fail(CSLD_ERR_ARG, "a required cache pointer is NULL");
+    if (c->window > 0 && !c->win_kv) return fail(CSLD_ERR_ARG, "win_kv is NULL with window > 0");
+    if (c->has_indexer && (!c->ikeys || !c->iscales || !c->w_idx))
+        return fail(CSLD_ERR_ARG, "indexer arrays are NULL with has_indexer set");
+    if (c->has_indexer && (c->capacity & 1))
+        return fail(CSLD_ERR_ALIGN, "capacity must be even when the cache keeps indexer keys");
+    if (!aligned16(c->comp_kv) || (c->win_kv && !aligned16(c->win_kv)) || !aligned16(c->tail_kv) ||
+        (c->ikeys && !aligned16(c->ikeys)) || (c->iscales && !aligned16(c->iscales)))
+        return fail(CSLD_ERR_ALIGN, "cache arrays must be 16-byte aligned");
+    return CSLD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csld_abi_version(void) { return CSLD_ABI_VERSION; }
+
+const char* csld_last_error(void) { return g_msg; }
+
+const char* csld_status_string(csld_status s) {
+    switch (s) {
+        case CSLD_OK: return "ok";
+        case CSLD_ERR_ARG: return "invalid argument";
+        case CSLD_ERR_SHAPE: return "inconsistent shape";
+        case CSLD_ERR_ALIGN: return "misaligned pointer or stride";
+        case CSLD_ERR_CAPACITY: return "size exceeds a maximum or the cache capacity";
+        case CSLD_ERR_CUDA: return "CUDA error";
+        case CSLD_ERR_UNSUPPORTED: return "unsupported shape";
+        case CSLD_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+csld_status csld_compress(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
+                          const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
+                          float* iscale_out, void* stream) {
+    if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
+    if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
+    if (T / ratio == 0) return CSLD_OK;
+    if (!raw || !gate || !pos_bias || !kv_out) return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (w_idx && (!ikey_out || !iscale_out)) return fail(CSLD_ERR_ARG, "ikey_out / iscale_out NULL with w_idx");
+    if (!aligned16(raw) || !aligned16(kv_out) || (ikey_out && !aligned16(ikey_out)))
+        return fail(CSLD_ERR_ALIGN, "raw, kv_out and ikey_out must be 16-byte aligned");
+    cudaError_t e = csld::launch_compress(raw, gate, pos_bias, ratio, w_idx, T, 1, T / ratio, kv_out,
+                                          ikey_out, iscale_out, num_sms(), as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "csld_compress");
+    return CSLD_OK;
+}
+
+csld_status csa_compress(const uint16_t* raw, const float* gate, const float* pos_bias,
+                         const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
+                         float* iscale_out, void* stream) {
+    if (!w_idx) return fail(CSLD_ERR_ARG, "csa_compress needs w_idx");
+    return csld_compress(raw, gate, pos_bias, 4, w_idx, T, kv_out, ikey_out, iscale_out, stream);
+}
+
+csld_status hca_compress(const uint16_t* raw, const float* gate, const float* pos_bias, int64_t T,
+                         uint8_t* kv_out, void* stream) {
+    return csld_compress(raw, gate, pos_bias, 128, nullptr, T, kv_out, nullptr, nullptr, stream);
+}
+
+csld_status kv_cache_append(const csld_layer_cache* cache, const uint16_t* kv_new,
+                            const float* gate_new, int32_t* err, void* stream) {
+    csld_status s = check_cache(cache);
+    if (s != CSLD_OK) return s;
+    if (!kv_new || !gate_new) return fail(CSLD_ERR_ARG, "kv_new / gate_new is NULL");
+    if (!aligned16(kv_new)) return fail(CSLD_ERR_ALIGN, "kv_new must be 16-byte aligned");
+    cudaError_t e = csld::launch_append(*cache, kv_new, gate_new, err, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kv_cache_append");
+    return CSLD_OK;
+}
+
+csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
+                             int64_t T, void* stream) {
+    csld_status s = check_cache(cache);
+    if (s != CSLD_OK) return s;
+    if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
+    if (T > 0 && (!raw || !gate)) return fail(CSLD_ERR_ARG, "raw / gate is NULL");
+    if (T > 0 && !aligned16(raw)) return fail(CSLD_ERR_ALIGN, "raw must be 16-byte aligned");
+    if (T / cache->ratio > cache->capacity)
+        return fail(CSLD_ERR_CAPACITY, "T/ratio = %lld entries exceed capacity %lld",
+                    (long long)(T / cache->ratio), (long long)cache->capacity);
+    const cudaStream_t st = as_stream(stream);
+    cudaError_t e = csld::launch_compress(raw, gate, cache->pos_bias, cache->ratio,
+                                          cache->has_indexer ? cache->w_idx : nullptr, T, cache->batch,
+                                          cache->capacity, cache->comp_kv, cache->ikeys,
+                                          cache->iscales, num_sms(), st);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_cache_prefill (compress)");
+    e = csld::launch_prefill_state(raw, gate, T, cache->ratio, cache->window, cache->batch,
+                                   cache->win_kv, cache->tail_kv, cache->tail_gate, cache->seq_len, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_cache_prefill (state)");
+    return CSLD_OK;
+}
+
+size_t csld_indexer_workspace_size(int B, int64_t cap, int k) {
+    if (B < 1 || cap < 1 || k < 1) return 0;
+    return csld::indexer_plan(B, cap, k, num_sms()).ws_bytes;
+}
+
+csld_status indexer_topk(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                         const int32_t* seq_len, int ratio, const float* q_idx, const float* head_w,
+                         int B, int k, int32_t* topk_out, void* ws, size_t ws_bytes, int32_t* err,
+                         void* stream) {
+    if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
+    if (k < 1 || k > CSLD_MAX_TOPK) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
+    if (cap < 1 || cap > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^31-1", (long long)cap);
+    if (cap & 1) return fail(CSLD_ERR_ALIGN, "cap must be even");
+    if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
+    if (!ikeys || !iscales || !seq_len || !q_idx || !head_w || !topk_out)
+        return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (!aligned16(ikeys) || !aligned16(iscales)) return fail(CSLD_ERR_ALIGN, "ikeys / iscales must be 16-byte aligned");
+    const csld::IndexerPlan plan = csld::indexer_plan(B, cap, k, num_sms());
+    if (!plan.levels_ok) return fail(CSLD_ERR_CAPACITY, "cap %lld too large for the merge tree", (long long)cap);
+    if (!ws || ws_bytes < plan.ws_bytes)
+        return fail(CSLD_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, plan.ws_bytes);
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CSLD_ERR_ALIGN, "workspace must be 256-byte aligned");
+    cudaError_t e = csld::launch_indexer(ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, B, k,
+                                         topk_out, ws, plan, err, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "indexer_topk");
+    return CSLD_OK;
+}
+
+size_t csld_attention_workspace_size(int B, int heads, int64_t cap, int k, int W) {
+    if (B < 1 || heads != CSLD_HEADS || cap < 1 || W < 0) return 0;
+    const csld::AttentionPlan pd = csld::attention_plan(B, cap, k, false, W, num_sms());
+    const csld::AttentionPlan ps = csld::attention_plan(B, cap, k > 0 ? k : 1, true, W, num_sms());
+    return pd.ws_bytes > ps.ws_bytes ? pd.ws_bytes : ps.ws_bytes;
+}
+
+csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t* comp_kv, int64_t cap,
+                                    int ratio, const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                                    const int32_t* seq_len, int B, float scale, float* out, float* lse_out,
+                                    void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+    if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; this build implements %d", heads, CSLD_HEADS);
+    if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
+    if (cap < 1 || cap > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^31-1", (long long)cap);
+    if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
+    if (W < 0 || W > CSLD_MAX_WINDOW) return fail(CSLD_ERR_ARG, "W %d outside 0..%d", W, CSLD_MAX_WINDOW);
+    if (topk && (k < 1 || k > CSLD_MAX_TOPK)) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
+    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return fail(CSLD_ERR_ARG, "scale is not finite");
+    if (!q || !comp_kv || !seq_len || !out) return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (W > 0 && !win_kv) return fail(CSLD_ERR_ARG, "win_kv is NULL with W > 0");
+    if (!aligned16(q) || !aligned16(comp_kv) || (win_kv && !aligned16(win_kv)) || !aligned16(out))
+        return fail(CSLD_ERR_ALIGN, "q, comp_kv, win_kv and out must be 16-byte aligned");
+    const csld::AttentionPlan plan = csld::attention_plan(B, cap, k, topk != nullptr, W, num_sms());
+    if (!ws || ws_bytes < plan.ws_bytes)
+        return fail(CSLD_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, plan.ws_bytes);
+    if (!aligned16(ws)) return fail(CSLD_ERR_ALIGN, "workspace must be 16-byte aligned");
+    cudaError_t e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, seq_len, B,
+                                           scale, out, lse_out, ws, plan, err, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention");
+    return CSLD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,463 @@
+// Hybrid decode attention over FP8/bf16 compressed entries plus a sliding window.
+//
+// Source: "DeepSeek-V4: a million-token context that agents can actually use" -- CSA paragraph
+// and Figure 3 caption (each query attends to its top-k compressed blocks; a sliding-window
+// branch covers the most recent uncompressed tokens), HCA paragraph and Figure 4 caption
+// (every query attends densely to all compressed blocks; the same window branch), storage
+// paragraph (entries FP8 except the RoPE dims in bf16); velog.io paper review, core
+// techniques 1-2.  Keys and values are the same decoded 512-d entry (one KV head); 16 query
+// heads share it; one softmax runs over {selected or all visible entries} + {window tokens}.
+//
+// Kernel design (one CTA = one split of one sequence's key list; 8 warps):
+//  - The split's key list is walked in tiles of 64 entries.  Warp 0 gathers each entry's 576
+//    bytes into shared memory with a 1-D bulk copy (3-stage mbarrier ring; sparse mode reads
+//    the top-k index, dense mode the position, the window part the ring slot); empty slots
+//    are zero-filled so they contribute exact zeros.
+//  - QK (tensor cores, mma.sync m16n8k16, fp32 accumulate): warp w computes the logits of
+//    entries 8w..8w+7 for all 16 heads.  The E4M3 dims are widened in registers with
+//    cvt.rn.f16x2.e4m3x2 (exact) and multiplied with the query in f16; the query of head h is
+//    pre-scaled by a power of two alpha_h so that max|alpha_h q_h| <= 2^14 (exact in f16 for
+//    the bf16 inputs); the 64 RoPE dims stay bf16 and use the bf16 MMA on the same accumulator.
+//  - Online softmax in the log2 domain with per-tile maxima exchanged through shared memory;
+//    P is written to shared memory (f16 for the E4M3 dims, bf16 for the RoPE dims).
+//  - PV: warp w owns output dims 64w..64w+63 for all heads; V fragments are read from the
+//    staged bytes (pairs of entries per dim), widened, and multiplied with P.
+//  - Each split writes unnormalised O, the running max m (log2 units) and the sum l; a second
+//    kernel merges the splits (log-sum-exp) into out and lse.
+#include "csld_internal.cuh"
+#include "kernels.cuh"
+
+namespace csld {
+
+constexpr int kAttnThreads = 256;
+constexpr int kAT = 64;                 // entries per tile
+constexpr int kAStages = 3;
+constexpr int kEStride = 592;           // staged bytes per entry (576 + 16: conflict-free PV reads)
+constexpr int kPStride = kAT + 8;       // P row stride in 16-bit elements (144 bytes)
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct AttnSmem {
+    uint8_t stage[kAStages][kAT * kEStride];
+    uint16_t p16[kHeads * kPStride];    // P as f16 [head][entry]
+    uint16_t pbf[kHeads * kPStride];    // P as bf16
+    float tmax[8][kHeads];
+    float lsum[8][kHeads];
+    uint64_t valid[kAStages];           // bit e set: slot e of the stage holds an entry
+    uint64_t full[kAStages];
+};
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_bf162(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
+    const uint16_t* __restrict__ q, const uint8_t* __restrict__ comp_kv, int64_t cap, int ratio,
+    const int32_t* __restrict__ topk, int k, const uint8_t* __restrict__ win_kv, int W,
+    const int32_t* __restrict__ seq_len, float scale, int splits, float* __restrict__ opart,
+    float2* __restrict__ mlpart, int32_t* err) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, cq = lane & 3;
+    const int b = blockIdx.y, split = blockIdx.x;
+
+    // ---- the key list of sequence b and this split's tile range ----------------------------
+    int32_t n = seq_len[b];
+    if (n < 0) {
+        if (tid == 0 && split == 0) dev_error(err, CSLD_DEVERR_SEQ_LEN);
+        n = 0;
+    }
+    const int64_t n_vis = min64(n / ratio, cap);
+    const bool sparse = topk != nullptr;
+    const int64_t n_comp = sparse ? (int64_t)k : n_vis;            // list slots of the compressed part
+    const int n_win = W > 0 ? min(W, n) : 0;
+    const int64_t L = n_comp + n_win;
+    const int64_t n_tiles_all = (L + kAT - 1) / kAT;
+    const int64_t t_begin = n_tiles_all * split / splits;
+    const int64_t t_end = n_tiles_all * (split + 1) / splits;
+    const int n_tiles = static_cast<int>(t_end - t_begin);
+
+    const size_t part = (size_t)b * splits + split;
+    if (n_tiles <= 0) {
+        if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
+        return;
+    }
+
+    // ---- query fragments (A operand, 32 k-steps x 4 registers) ------------------------------
+    // k-step s < 28 (E4M3 dims): a0/a1 = dims 112*cq + 4s + {0,1} of heads g / g+8,
+    // a2/a3 = dims 112*cq + 4s + {2,3}.  k-step 28+s' (RoPE): dims 448 + 16*cq + 4s' + ...
+    uint32_t qa[32][4];
+    float c2[2];  // log2-domain logit factor for heads g and g+8
+    {
+        const uint16_t* qh[2] = {q + ((size_t)b * kHeads + g) * kDim, q + ((size_t)b * kHeads + g + 8) * kDim};
+        float amax[2] = {0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            for (int i = 0; i < 14; ++i) {
+                const uint4 v = *reinterpret_cast<const uint4*>(qh[r] + 112 * cq + 8 * i);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    amax[r] = fmaxf(amax[r], fmaxf(fabsf(bf16_bits_to_f32(w[j])), fabsf(bf16_bits_to_f32(w[j] >> 16))));
+            }
+            for (int i = 0; i < 2; ++i) {
+                const uint4 v = *reinterpret_cast<const uint4*>(qh[r] + kNope + 16 * cq + 8 * i);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    amax[r] = fmaxf(amax[r], fmaxf(fabsf(bf16_bits_to_f32(w[j])), fabsf(bf16_bits_to_f32(w[j] >> 16))));
+            }
+            amax[r] = fmaxf(amax[r], __shfl_xor_sync(0xffffffffu, amax[r], 1));
+            amax[r] = fmaxf(amax[r], __shfl_xor_sync(0xffffffffu, amax[r], 2));
+        }
+        float alpha[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            int e2 = 0;
+            if (amax[r] > 0.f) frexpf(amax[r], &e2);      // amax < 2^e2
+            e2 = max(e2, -100);                           // keep alpha finite for tiny queries
+            alpha[r] = ldexpf(1.f, 14 - e2);              // alpha * amax < 2^14
+            c2[r] = scale * kLog2e / alpha[r];
+        }
+#pragma unroll
+        for (int s = 0; s < 28; ++s) {
+            const int d = 112 * cq + 4 * s;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint2 v = *reinterpret_cast<const uint2*>(qh[r] + d);
+                qa[s][r] = pack_half2(alpha[r] * bf16_bits_to_f32(v.x), alpha[r] * bf16_bits_to_f32(v.x >> 16));
+                qa[s][2 + r] = pack_half2(alpha[r] * bf16_bits_to_f32(v.y), alpha[r] * bf16_bits_to_f32(v.y >> 16));
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const int d = kNope + 16 * cq + 4 * s;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint2 v = *reinterpret_cast<const uint2*>(qh[r] + d);
+                qa[28 + s][r] = pack_bf162(alpha[r] * bf16_bits_to_f32(v.x), alpha[r] * bf16_bits_to_f32(v.x >> 16));
+                qa[28 + s][2 + r] = pack_bf162(alpha[r] * bf16_bits_to_f32(v.y), alpha[r] * bf16_bits_to_f32(v.y >> 16));
+            }
+        }
+    }
+
+    if (tid == 0) {
+        for (int s = 0; s < kAStages; ++s) mbar_init(&sm.full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    // ---- producer (warp 0): gather tile `it` (0-based within the split) into its stage ------
+    const uint8_t* comp_b = comp_kv + (size_t)b * cap * kEntry;
+    const uint8_t* win_b = win_kv ? win_kv + (size_t)b * W * kEntry : nullptr;
+    const int32_t* topk_b = sparse ? topk + (size_t)b * k : nullptr;
+    auto produce = [&](int it) {
+        const int st = it % kAStages;
+        const int64_t slot0 = (t_begin + it) * kAT;
+        const uint8_t* src[2];
+        bool val[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = lane + 32 * h;
+            const int64_t i = slot0 + e;
+            src[h] = nullptr;
+            if (i < L) {
+                if (i < n_comp) {
+                    int64_t v = i;
+                    if (sparse) {
+                        v = topk_b[i];
+                        if (v >= n_vis) {
+                            dev_error(err, CSLD_DEVERR_BAD_INDEX);
+                            v = -1;
+                        }
+                    }
+                    if (v >= 0) src[h] = comp_b + (size_t)v * kEntry;
+                } else {
+                    const int64_t t = (int64_t)n - n_win + (i - n_comp);
+                    src[h] = win_b + (size_t)(t % W) * kEntry;
+                }
+            }
+            val[h] = src[h] != nullptr;
+            if (!val[h]) {
+                uint4* dst = reinterpret_cast<uint4*>(sm.stage[st] + e * kEStride);
+                for (int j = 0; j < kEntry / 16; ++j) dst[j] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        const uint32_t m0 = __ballot_sync(0xffffffffu, val[0]);
+        const uint32_t m1 = __ballot_sync(0xffffffffu, val[1]);
+        if (lane == 0) sm.valid[st] = (uint64_t)m0 | ((uint64_t)m1 << 32);
+        const uint32_t bytes = (uint32_t)(__popc(m0) + __popc(m1)) * kEntry;
+        // zero-fills and the valid mask are ordered before the arrive (release)
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&sm.full[st], bytes);
+        __syncwarp();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            if (val[h]) bulk_g2s(sm.stage[st] + (lane + 32 * h) * kEStride, src[h], kEntry, &sm.full[st]);
+    };
+    if (warp == 0)
+        for (int it = 0; it < min(n_tiles, kAStages); ++it) produce(it);
+
+    // ---- consumer state ---------------------------------------------------------------------
+    float m_run[2] = {-INFINITY, -INFINITY};   // heads g, g+8 (identical in every warp)
+    float l_run[2] = {0.f, 0.f};               // this thread's share of the row sums
+    float o[8][4];                             // O[heads][64 dims of this warp], 8 n-tiles
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    const bool rope_warp = (warp == 7);
+
+    int consumed = 0;
+    bool ok = true;
+    for (int it = 0; it < n_tiles; ++it) {
+        const int st = it % kAStages;
+        const bool landed = mbar_wait(&sm.full[st], (it / kAStages) & 1);
+        if (__syncthreads_or(!landed)) {
+            ok = false;
+            break;
+        }
+        consumed = it + 1;
+        const uint8_t* stg = sm.stage[st];
+        const uint64_t vmask = sm.valid[st];
+
+        // -- QK: entries 8*warp + g --
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const uint8_t* ent = stg + (8 * warp + g) * kEStride;
+#pragma unroll
+            for (int i = 0; i < 7; ++i) {
+                const uint4 v = *reinterpret_cast<const uint4*>(ent + 112 * cq + 16 * i);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int s = 4 * i + j;
+                    mma_f16(s4, qa[s][0], qa[s][1], qa[s][2], qa[s][3], e4m3x2_to_f16x2(w[j] & 0xFFFFu),
+                            e4m3x2_to_f16x2(w[j] >> 16));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const uint4 v = *reinterpret_cast<const uint4*>(ent + kNope + 32 * cq + 16 * i);
+                mma_bf16(s4, qa[28 + 2 * i][0], qa[28 + 2 * i][1], qa[28 + 2 * i][2], qa[28 + 2 * i][3], v.x, v.y);
+                mma_bf16(s4, qa[29 + 2 * i][0], qa[29 + 2 * i][1], qa[29 + 2 * i][2], qa[29 + 2 * i][3], v.z, v.w);
+            }
+        }
+        // s4: (head g, entries e0, e0+1), (head g+8, entries e0, e0+1) with e0 = 8w + 2cq
+        const int e0 = 8 * warp + 2 * cq;
+        const bool v0 = (vmask >> e0) & 1ull, v1 = (vmask >> (e0 + 1)) & 1ull;
+        float x[4];
+        x[0] = v0 ? s4[0] * c2[0] : -INFINITY;
+        x[1] = v1 ? s4[1] * c2[0] : -INFINITY;
+        x[2] = v0 ? s4[2] * c2[1] : -INFINITY;
+        x[3] = v1 ? s4[3] * c2[1] : -INFINITY;
+        float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        if (cq == 0) {
+            sm.tmax[warp][g] = mx0;
+            sm.tmax[warp][g + 8] = mx1;
+        }
+        __syncthreads();
+        float tm0 = sm.tmax[0][g], tm1 = sm.tmax[0][g + 8];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) {
+            tm0 = fmaxf(tm0, sm.tmax[w][g]);
+            tm1 = fmaxf(tm1, sm.tmax[w][g + 8]);
+        }
+        const float mn0 = fmaxf(m_run[0], tm0), mn1 = fmaxf(m_run[1], tm1);
+        // a row with no key yet keeps m = -inf; its p's are 0 and nothing is rescaled
+        const float corr0 = (mn0 == -INFINITY) ? 1.f : exp2f(m_run[0] - mn0);
+        const float corr1 = (mn1 == -INFINITY) ? 1.f : exp2f(m_run[1] - mn1);
+        const float p0 = (mn0 == -INFINITY) ? 0.f : exp2f(x[0] - mn0);
+        const float p1 = (mn0 == -INFINITY) ? 0.f : exp2f(x[1] - mn0);
+        const float p2 = (mn1 == -INFINITY) ? 0.f : exp2f(x[2] - mn1);
+        const float p3 = (mn1 == -INFINITY) ? 0.f : exp2f(x[3] - mn1);
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+        l_run[0] = l_run[0] * corr0 + (p0 + p1);
+        l_run[1] = l_run[1] * corr1 + (p2 + p3);
+        *reinterpret_cast<uint32_t*>(&sm.p16[g * kPStride + e0]) = pack_half2(p0, p1);
+        *reinterpret_cast<uint32_t*>(&sm.p16[(g + 8) * kPStride + e0]) = pack_half2(p2, p3);
+        *reinterpret_cast<uint32_t*>(&sm.pbf[g * kPStride + e0]) = pack_bf162(p0, p1);
+        *reinterpret_cast<uint32_t*>(&sm.pbf[(g + 8) * kPStride + e0]) = pack_bf162(p2, p3);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            o[j][0] *= corr0;
+            o[j][1] *= corr0;
+            o[j][2] *= corr1;
+            o[j][3] *= corr1;
+        }
+        __syncthreads();
+
+        // -- PV: this warp's 64 output dims; n-tile j, column g <-> dim base + 8g + j --
+        const uint16_t* P = rope_warp ? sm.pbf : sm.p16;
+#pragma unroll
+        for (int t = 0; t < kAT / 16; ++t) {
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a0, a1, a2, a3, P + (lane & 15) * kPStride + 16 * t + ((lane >> 4) << 3));
+            const int ea = 16 * t + 2 * cq;   // entries ea, ea+1 (b0) and ea+8, ea+9 (b1)
+            if (!rope_warp) {
+                const int off = 64 * warp + 8 * g;
+                const uint2 A = *reinterpret_cast<const uint2*>(stg + (ea)*kEStride + off);
+                const uint2 Bv = *reinterpret_cast<const uint2*>(stg + (ea + 1) * kEStride + off);
+                const uint2 C = *reinterpret_cast<const uint2*>(stg + (ea + 8) * kEStride + off);
+                const uint2 D = *reinterpret_cast<const uint2*>(stg + (ea + 9) * kEStride + off);
+                uint32_t bb0[8], bb1[8];
+#pragma unroll
+                for (int hw = 0; hw < 2; ++hw) {
+                    const uint32_t xa = hw ? A.y : A.x, xb = hw ? Bv.y : Bv.x;
+                    const uint32_t xc = hw ? C.y : C.x, xd = hw ? D.y : D.x;
+                    const uint32_t lo01 = prmt(xa, xb, 0x5140u), hi23 = prmt(xa, xb, 0x7362u);
+                    const uint32_t clo = prmt(xc, xd, 0x5140u), chi = prmt(xc, xd, 0x7362u);
+                    bb0[4 * hw + 0] = e4m3x2_to_f16x2(lo01 & 0xFFFFu);
+                    bb0[4 * hw + 1] = e4m3x2_to_f16x2(lo01 >> 16);
+                    bb0[4 * hw + 2] = e4m3x2_to_f16x2(hi23 & 0xFFFFu);
+                    bb0[4 * hw + 3] = e4m3x2_to_f16x2(hi23 >> 16);
+                    bb1[4 * hw + 0] = e4m3x2_to_f16x2(clo & 0xFFFFu);
+                    bb1[4 * hw + 1] = e4m3x2_to_f16x2(clo >> 16);
+                    bb1[4 * hw + 2] = e4m3x2_to_f16x2(chi & 0xFFFFu);
+                    bb1[4 * hw + 3] = e4m3x2_to_f16x2(chi >> 16);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mma_f16(o[j], a0, a1, a2, a3, bb0[j], bb1[j]);
+            } else {
+                const int off = kNope + 16 * g;   // bf16 elements 8g..8g+7 of the RoPE part
+                const uint4 A = *reinterpret_cast<const uint4*>(stg + (ea)*kEStride + off);
+                const uint4 Bv = *reinterpret_cast<const uint4*>(stg + (ea + 1) * kEStride + off);
+                const uint4 C = *reinterpret_cast<const uint4*>(stg + (ea + 8) * kEStride + off);
+                const uint4 D = *reinterpret_cast<const uint4*>(stg + (ea + 9) * kEStride + off);
+                const uint32_t wa[4] = {A.x, A.y, A.z, A.w}, wb[4] = {Bv.x, Bv.y, Bv.z, Bv.w};
+                const uint32_t wc[4] = {C.x, C.y, C.z, C.w}, wd[4] = {D.x, D.y, D.z, D.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+                    mma_bf16(o[j], a0, a1, a2, a3, prmt(wa[j >> 1], wb[j >> 1], sel),
+                             prmt(wc[j >> 1], wd[j >> 1], sel));
+                }
+            }
+        }
+        __syncthreads();   // stage and P buffers free
+        if (warp == 0 && it + kAStages < n_tiles) produce(it + kAStages);
+    }
+    if (!ok) {
+        if (tid == 0) {
+            dev_error(err, CSLD_DEVERR_TIMEOUT);
+            for (int t = consumed; t < min(n_tiles, consumed + kAStages); ++t)
+                (void)mbar_wait(&sm.full[t % kAStages], (t / kAStages) & 1);
+        }
+        if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
+        return;
+    }
+
+    // ---- row sums across the 4 lanes of a group and the 8 warps ----------------------------
+    float ls0 = l_run[0], ls1 = l_run[1];
+    ls0 += __shfl_xor_sync(0xffffffffu, ls0, 1);
+    ls0 += __shfl_xor_sync(0xffffffffu, ls0, 2);
+    ls1 += __shfl_xor_sync(0xffffffffu, ls1, 1);
+    ls1 += __shfl_xor_sync(0xffffffffu, ls1, 2);
+    if (cq == 0) {
+        sm.lsum[warp][g] = ls0;
+        sm.lsum[warp][g + 8] = ls1;
+    }
+    __syncthreads();
+    if (warp == 0 && cq == 0) {
+        float t0 = 0.f, t1 = 0.f;
+        for (int w = 0; w < 8; ++w) {
+            t0 += sm.lsum[w][g];
+            t1 += sm.lsum[w][g + 8];
+        }
+        mlpart[part * kHeads + g] = make_float2(m_run[0], t0);
+        mlpart[part * kHeads + g + 8] = make_float2(m_run[1], t1);
+    }
+    // ---- unnormalised O of this split ------------------------------------------------------
+    float* ob = opart + part * kHeads * kDim;
+    const int base = 64 * warp;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int d0 = base + 8 * (2 * cq) + j, d1 = base + 8 * (2 * cq + 1) + j;
+        ob[g * kDim + d0] = o[j][0];
+        ob[g * kDim + d1] = o[j][1];
+        ob[(g + 8) * kDim + d0] = o[j][2];
+        ob[(g + 8) * kDim + d1] = o[j][3];
+    }
+}
+
+// Merge the splits of one (sequence, head): out = sum_j 2^(m_j - M) O_j / L,
+// lse = ln 2 * (M + log2 L) with L = sum_j 2^(m_j - M) l_j.
+__global__ void __launch_bounds__(128) attention_merge_kernel(const float* __restrict__ opart,
+                                                              const float2* __restrict__ mlpart,
+                                                              int splits, float* __restrict__ out,
+                                                              float* __restrict__ lse_out) {
+    const int b = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    float M = -INFINITY;
+    for (int j = 0; j < splits; ++j) {
+        const float2 ml = mlpart[((size_t)b * splits + j) * kHeads + h];
+        if (ml.y > 0.f) M = fmaxf(M, ml.x);
+    }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Lsum = 0.f;
+    if (M != -INFINITY) {
+        for (int j = 0; j < splits; ++j) {
+            const float2 ml = mlpart[((size_t)b * splits + j) * kHeads + h];
+            if (!(ml.y > 0.f)) continue;
+            const float f = exp2f(ml.x - M);
+            Lsum += f * ml.y;
+            const float4 v = reinterpret_cast<const float4*>(opart + (((size_t)b * splits + j) * kHeads + h) * kDim)[tid];
+            acc.x += f * v.x;
+            acc.y += f * v.y;
+            acc.z += f * v.z;
+            acc.w += f * v.w;
+        }
+        const float inv = 1.f / Lsum;
+        acc.x *= inv;
+        acc.y *= inv;
+        acc.z *= inv;
+        acc.w *= inv;
+    }
+    reinterpret_cast<float4*>(out + ((size_t)b * kHeads + h) * kDim)[tid] = acc;
+    if (lse_out && tid == 0)
+        lse_out[(size_t)b * kHeads + h] = (M == -INFINITY) ? -INFINITY : (M + log2f(Lsum)) * 0.69314718055994531f;
+}
+
+AttentionPlan attention_plan(int B, int64_t cap, int k, bool sparse, int W, int num_sms) {
+    AttentionPlan p;
+    const int64_t L = (sparse ? (int64_t)k : cap) + W;
+    const int64_t tiles = (L + kAT - 1) / kAT;
+    int64_t s = num_sms / (B > 0 ? B : 1);
+    if (s < 1) s = 1;
+    if (s > tiles) s = tiles;
+    if (s < 1) s = 1;
+    if (s > 256) s = 256;
+    p.splits = static_cast<int>(s);
+    p.ws_bytes = (size_t)B * p.splits * kHeads * (kDim * sizeof(float) + sizeof(float2));
+    return p;
+}
+
+cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
+                             const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                             const int32_t* seq_len, int B, float scale, float* out,
+                             float* lse_out, void* ws, const AttentionPlan& plan, int32_t* err,
+                             cudaStream_t stream) {
+    float* opart = static_cast<float*>(ws);
+    float2* mlpart = reinterpret_cast<float2*>(opart + (size_t)B * plan.splits * kHeads * kDim);
+    const size_t smem = sizeof(AttnSmem);
+    cudaError_t e = set_smem_once(attention_partial_kernel, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(plan.splits, B);
+    attention_partial_kernel<<<grid, kAttnThreads, smem, stream>>>(q, comp_kv, cap, ratio, topk, k,
+                                                                   win_kv, W, seq_len, scale,
+                                                                   plan.splits, opart, mlpart, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attention_merge_kernel<<<dim3(B, kHeads), 128, 0, stream>>>(opart, mlpart, plan.splits, out, lse_out);
+    return cudaGetLastError();
+}
+
+}  // namespace csld

@@ -1,0 +1,205 @@
+// Internal device helpers of libcsld (sm_100a).  Not part of the ABI.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csld.h"
+
+namespace csld {
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+constexpr int kDim = CSLD_DIM;
+constexpr int kNope = CSLD_DIM_NOPE;
+constexpr int kRope = CSLD_DIM_ROPE;
+constexpr int kEntry = CSLD_ENTRY_BYTES;
+constexpr int kHeads = CSLD_HEADS;
+constexpr int kIdxHeads = CSLD_IDX_HEADS;
+constexpr int kIdxDim = CSLD_IDX_DIM;
+constexpr int kIkey = CSLD_IKEY_BYTES;
+
+// ------------------------------------------------------------------------------------------
+// Shared-memory addressing, mbarriers and bulk (TMA) copies.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+// Make initialised barriers visible to the async (bulk-copy) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false if the phase did not complete within the
+// limit (about a second); callers then record CSLD_DEVERR_TIMEOUT and stop issuing work.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        __nanosleep(256);
+        if (mbar_try_wait(bar, parity)) return true;
+    }
+    return false;
+}
+
+// 1-D bulk copy global -> shared, completing `bytes` on the mbarrier.  src, dst 16-byte
+// aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------------------------------------
+// Warp-level tensor-core MMAs (legacy mma.sync path; fragments in registers).
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                            const void* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// ------------------------------------------------------------------------------------------
+// Number formats.  E4M3 / bf16 conversions use the hardware round-to-nearest-even converts;
+// E2M1 (FP4) is written out below from the grid {0, .5, 1, 1.5, 2, 3, 4, 6}.
+// ------------------------------------------------------------------------------------------
+// Two E4M3 bytes (low byte = first element) -> f16x2 (low half = first element); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+    uint32_t r;
+    asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n"
+        : "=r"(r)
+        : "r"(two_bytes));
+    return r;
+}
+
+// fp32 -> E4M3 byte: round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float x) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(x)));
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
+    return __uint_as_float((h & 0xFFFFu) << 16);
+}
+
+// E2M1 code of v (|v| <= 6 expected; larger saturates): nearest grid value, ties to the even
+// mantissa (0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4).  Bit 3 = sign.
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+    const float a = fabsf(v);
+    uint32_t m;
+    if (a <= 0.25f) m = 0;
+    else if (a < 0.75f) m = 1;
+    else if (a <= 1.25f) m = 2;
+    else if (a < 1.75f) m = 3;
+    else if (a <= 2.5f) m = 4;
+    else if (a < 3.5f) m = 5;
+    else if (a <= 5.0f) m = 6;
+    else m = 7;
+    return (signbit(v) ? 8u : 0u) | m;
+}
+
+// Twice the value of an E2M1 magnitude index 0..7 (an integer): 0,1,2,3,4,6,8,12.
+constexpr uint32_t kTwiceE2M1Lo = 0x03020100u;  // indices 0..3
+constexpr uint32_t kTwiceE2M1Hi = 0x0C080604u;  // indices 4..7
+
+// Smallest power of two sigma with amax <= 6*sigma; 1 when amax == 0.  Exact: with
+// 2^e0 <= amax < 2^(e0+1), sigma is 2^(e0-2) if amax <= 1.5*2^e0, else 2^(e0-1).
+__device__ __forceinline__ float fp4_group_scale(float amax) {
+    if (!(amax > 0.f)) return 1.f;
+    const int e0 = ilogbf(amax);
+    return (amax <= ldexpf(1.5f, e0)) ? ldexpf(1.f, e0 - 2) : ldexpf(1.f, e0 - 1);
+}
+
+// Order-preserving 32-bit key of an fp32 score (-0 and +0 map to the same key).
+__device__ __forceinline__ uint32_t score_key(float s) {
+    uint32_t u = __float_as_uint(s);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Opt a kernel into its dynamic shared-memory size once per process (a function attribute,
+// not a stream operation, so later calls may be captured into CUDA graphs).
+template <typename K>
+inline cudaError_t set_smem_once(K kernel, size_t bytes) {
+    static int done = 0;
+    if (done) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(bytes));
+    if (e == cudaSuccess) done = 1;
+    return e;
+}
+
+__device__ __forceinline__ void dev_error(int32_t* err, uint32_t flag) {
+    if (err) atomicOr(reinterpret_cast<unsigned int*>(err), flag);
+}
+
+}  // namespace csld

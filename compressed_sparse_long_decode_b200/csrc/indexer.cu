@@ -1,0 +1,496 @@
+// Lightning indexer + exact top-k.
+//
+// Source: "DeepSeek-V4: a million-token context that agents can actually use" -- CSA paragraph
+// (the lightning indexer, an FP4 ReLU-scored multi-head dot product, picks the top-k
+// compressed blocks for each query) and Figure 3 caption; velog.io paper review, "core
+// technique 1: CSA" (the indexer scores which compressed entries the query should read).
+//
+// Score of entry s for one query (4 heads, 64 dims, one key per entry shared by the heads):
+//   e_s = sum_h w_h * ReLU(q_h . k_s), q and k both FP4 (E2M1 codes, power-of-two scale / 32).
+// The two 32-element group dots of every (entry, head) are exact integers (codes doubled are
+// the integers {0,1,2,3,4,6,8,12} with sign), computed on the tensor cores with
+// mma.sync.m16n8k32 s8 x s8 -> s32.  A key nibble is turned into its doubled magnitude by one
+// PRMT lookup: the code's sign bit is PRMT's sign-replicate flag, so negative codes yield 0;
+// the same lookup on the nibbles with flipped signs yields the negative codes' magnitudes, and
+// dot = pos . q - neg . q = pos . q + neg . (-q).  B columns 0..3 hold the query heads over
+// group 0 and columns 4..7 over group 1, so one accumulator holds both group dots.
+// The fp32 score then follows a fixed operation order (see the ABI header), so the selection
+// is reproducible bit for bit; order key = (score, -index).
+//
+// One kernel (indexer_topk_kernel), grid (chunk, sequence): each CTA streams `chunk` entries
+// of keys through shared memory with 1-D bulk copies (4-stage mbarrier ring), scores them into
+// 32-bit order keys held in shared memory, and radix-selects its chunk's top min(k, chunk),
+// written as a run in index order.  The runs are then merged by a tree inside the same kernel:
+// the last CTA of a group of G runs to finish (an atomic arrival counter; nothing ever waits)
+// loads the group's runs, selects their top min(k, ...) and publishes one run for the next
+// level; the last run is the answer, written in ascending index order and -1 padded.
+// Selecting the top k of a union of per-part top-k sets is exact under the total order
+// (score desc, index asc), because every global top-k entry is in its part's top k.
+#include "csld_internal.cuh"
+#include "kernels.cuh"
+
+namespace csld {
+
+constexpr int kIdxThreads = 256;
+constexpr int kIdxTile = 256;          // entries per pipeline stage (32 per warp)
+constexpr int kIdxStages = 4;
+constexpr int kIdxMaxChunk = 8192;
+
+constexpr int kIdxMaxGroup = 64;       // runs merged by one CTA
+constexpr int kIdxMaxLevels = 4;
+
+struct IdxSmem {
+    uint8_t codes[kIdxStages][kIdxTile * kIkey];
+    float scales[kIdxStages][kIdxTile * 2];
+    uint32_t keys[kIdxMaxChunk];       // order keys of the chunk, or of the runs being merged
+    int32_t idx[kIdxMaxChunk];         // their entry indices
+    uint32_t hist[256];
+    uint32_t scan[32];
+    int32_t offs[kIdxMaxGroup + 1];
+    float qscale[8];                   // [group*4 + head]
+    uint64_t full[kIdxStages];
+    uint32_t sel[4];
+    int32_t last;
+};
+
+// --- block-wide helpers (256 threads) ----------------------------------------------------
+
+// Exclusive scan of one value per thread over the block; returns the thread's prefix and the
+// total through *total.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* buf, uint32_t* total) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nw = blockDim.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    __syncthreads();
+    if (lane == 31) buf[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = lane < nw ? buf[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < nw) buf[lane] = w;   // inclusive warp totals
+    }
+    __syncthreads();
+    const uint32_t before = (warp > 0 ? buf[warp - 1] : 0u) + x - v;
+    *total = buf[nw - 1];
+    __syncthreads();
+    return before;
+}
+
+// Radix select over n keys (read through `get(i)`): the largest `want` keys, ties on the
+// threshold resolved by lower position.  Returns the threshold key and, through *take_eq, how
+// many keys equal to it are selected (the lowest-position ones).  hist: 256 words of smem,
+// sel: 4 words.  All threads must call.
+template <typename Get>
+__device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint32_t* sel,
+                                 uint32_t* take_eq) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t prefix = 0u, mask = 0u;
+    uint32_t remaining = static_cast<uint32_t>(want);
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0u;
+        __syncthreads();
+        const int n_round = (n + 31) & ~31;
+        for (int i = tid; i < n_round; i += blockDim.x) {
+            uint32_t d = 256u;
+            if (i < n) {
+                const uint32_t key = get(i);
+                if (((key ^ prefix) & mask) == 0u) d = (key >> shift) & 0xFFu;
+            }
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+        }
+        __syncthreads();
+        if (tid < 32) {
+            // lane l owns digits 255-8l .. 248-8l (descending)
+            uint32_t cnt[8], tot = 0u;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                cnt[q] = hist[255 - 8 * lane - q];
+                tot += cnt[q];
+            }
+            uint32_t incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const uint32_t excl = incl - tot;
+            const uint32_t hit = __ballot_sync(0xffffffffu, incl >= remaining && excl < remaining);
+            if (lane == __ffs(hit) - 1) {
+                uint32_t run = excl;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    if (run + cnt[q] >= remaining) {
+                        sel[0] = 255u - 8u * lane - q;    // the digit
+                        sel[1] = remaining - run;         // still wanted inside that digit
+                        break;
+                    }
+                    run += cnt[q];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= sel[0] << shift;
+        mask |= 0xFFu << shift;
+        remaining = sel[1];
+        __syncthreads();
+    }
+    *take_eq = remaining;
+    return prefix;
+}
+
+// Writes, in position order, the positions selected by (key > thr) or (key == thr and among
+// the first take_eq such positions).  Each thread owns a contiguous segment.  emit(pos, i).
+template <typename Get, typename Emit>
+__device__ void select_compact(Get get, int n, uint32_t thr, uint32_t take_eq, uint32_t* buf,
+                               Emit emit) {
+    const int tid = threadIdx.x;
+    const int seg = (n + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
+    uint32_t gt = 0u, eq = 0u;
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t key = get(i);
+        gt += key > thr;
+        eq += key == thr;
+    }
+    uint32_t tot;
+    const uint32_t eq_before = block_exclusive_scan(eq, buf, &tot);
+    const uint32_t eq_take = eq_before >= take_eq ? 0u : min(eq, take_eq - eq_before);
+    uint32_t pos = block_exclusive_scan(gt + eq_take, buf, &tot);
+    uint32_t eq_left = eq_take;
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t key = get(i);
+        bool take = key > thr;
+        if (!take && key == thr && eq_left > 0u) {
+            take = true;
+            --eq_left;
+        }
+        if (take) emit(pos++, i);
+    }
+}
+
+
+// ------------------------------------------------------------------------------------------
+// Workspace layout of the merge tree.
+// ------------------------------------------------------------------------------------------
+struct IdxTree {
+    int levels;                        // run levels that are stored (the final run is not)
+    int n_runs[kIdxMaxLevels + 1];     // runs per sequence at each level (level 0 = chunks)
+    uint32_t* keys[kIdxMaxLevels];     // [B][n_runs[l]][kc]
+    int32_t* idx[kIdxMaxLevels];
+    int32_t* cnt[kIdxMaxLevels];       // [B][n_runs[l]]
+    int32_t* ctr[kIdxMaxLevels + 1];   // arrival counters of level l runs, [B][n_runs[l]]
+    int group;
+};
+
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static IdxTree tree_layout(int B, int n_chunks, int kc, int group, uint8_t* base, size_t* bytes) {
+    IdxTree t{};
+    t.group = group;
+    t.n_runs[0] = n_chunks;
+    int l = 0;
+    while (t.n_runs[l] > 1 && l < kIdxMaxLevels) {
+        t.n_runs[l + 1] = (t.n_runs[l] + group - 1) / group;
+        ++l;
+    }
+    t.levels = l;  // levels 0..l-1 store runs; level l has exactly one run (the answer)
+    size_t off = 0;
+    for (int i = 0; i < t.levels; ++i) {
+        const size_t slots = (size_t)B * t.n_runs[i] * kc;
+        t.keys[i] = reinterpret_cast<uint32_t*>(base ? base + off : nullptr);
+        off += up256(slots * 4);
+        t.idx[i] = reinterpret_cast<int32_t*>(base ? base + off : nullptr);
+        off += up256(slots * 4);
+        t.cnt[i] = reinterpret_cast<int32_t*>(base ? base + off : nullptr);
+        off += up256((size_t)B * t.n_runs[i] * 4);
+    }
+    for (int i = 1; i <= t.levels; ++i) {
+        t.ctr[i] = reinterpret_cast<int32_t*>(base ? base + off : nullptr);
+        off += up256((size_t)B * t.n_runs[i] * 4);
+    }
+    *bytes = off;
+    return t;
+}
+
+// ------------------------------------------------------------------------------------------
+// The kernel.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
+    const uint8_t* __restrict__ ikeys, const float* __restrict__ iscales, int64_t cap,
+    const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
+    const float* __restrict__ head_w, int chunk, int kc, int k, IdxTree tree,
+    int32_t* __restrict__ topk_out, int32_t* err) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    IdxSmem& sm = *reinterpret_cast<IdxSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, cq = lane & 3;
+    const int b = blockIdx.y, ch = blockIdx.x;
+
+    int64_t n_b = seq_len[b];
+    n_b = n_b < 0 ? 0 : n_b / ratio;
+    if (n_b > cap) n_b = cap;
+    const int64_t c0 = (int64_t)ch * chunk;
+    const int cn = static_cast<int>(max64(0, min64(chunk, n_b - c0)));
+
+    bool chunk_ok = true;
+    if (cn > 0) {
+        // --- query: FP4 codes doubled as int8, in the MMA's B layout ----------------------
+        // B column n (= g): n < 4 -> head n over group 0; n >= 4 -> head n-4 over group 1.
+        // K order inside a group: MMA k = 4c+i <-> dim 8c+i, k = 16+4c+i <-> dim 8c+4+i.
+        uint32_t bq0, bq1;
+        {
+            const int h = g & 3, grp = g >> 2;
+            const float* qv = q_idx + ((size_t)b * kIdxHeads + h) * kIdxDim + 32 * grp;
+            float amax = 0.f;
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[i]));
+            const float sg = fp4_group_scale(amax);
+            const float inv = 1.0f / sg;   // exact: a power of two
+            if (cq == 0) sm.qscale[grp * 4 + h] = sg;
+            uint32_t w0 = 0u, w1 = 0u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t c_lo = e2m1_code(qv[8 * cq + i] * inv);
+                const uint32_t c_hi = e2m1_code(qv[8 * cq + 4 + i] * inv);
+                const int v_lo = static_cast<int>(prmt(kTwiceE2M1Lo, kTwiceE2M1Hi, c_lo & 7u) & 0xFFu) *
+                                 ((c_lo & 8u) ? -1 : 1);
+                const int v_hi = static_cast<int>(prmt(kTwiceE2M1Lo, kTwiceE2M1Hi, c_hi & 7u) & 0xFFu) *
+                                 ((c_hi & 8u) ? -1 : 1);
+                w0 |= (static_cast<uint32_t>(v_lo) & 0xFFu) << (8 * i);
+                w1 |= (static_cast<uint32_t>(v_hi) & 0xFFu) << (8 * i);
+            }
+            bq0 = w0;
+            bq1 = w1;
+        }
+        // group-0 MMAs see columns 0..3 only, group-1 MMAs columns 4..7 only
+        const bool col_grp1 = g >= 4;
+        const uint32_t b00 = col_grp1 ? 0u : bq0, b01 = col_grp1 ? 0u : bq1;
+        const uint32_t b10 = col_grp1 ? bq0 : 0u, b11 = col_grp1 ? bq1 : 0u;
+        auto neg4 = [](uint32_t v) -> uint32_t {   // bytewise negation (|values| <= 12)
+            uint32_t r = 0u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) r |= ((0u - ((v >> (8 * i)) & 0xFFu)) & 0xFFu) << (8 * i);
+            return r;
+        };
+        const uint32_t n00 = neg4(b00), n01 = neg4(b01), n10 = neg4(b10), n11 = neg4(b11);
+        const float w0 = head_w[b * kIdxHeads + 0], w1 = head_w[b * kIdxHeads + 1];
+        const float w2 = head_w[b * kIdxHeads + 2], w3 = head_w[b * kIdxHeads + 3];
+
+        if (tid == 0) {
+            for (int s = 0; s < kIdxStages; ++s) mbar_init(&sm.full[s], 1);
+            fence_barrier_init();
+        }
+        __syncthreads();
+
+        const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
+        const uint8_t* kbase = ikeys + ((size_t)b * cap + (size_t)c0) * kIkey;
+        const float* sbase = iscales + ((size_t)b * cap + (size_t)c0) * 2;
+        auto issue = [&](int tile) {
+            const int s = tile % kIdxStages;
+            const int nt = min(kIdxTile, cn - tile * kIdxTile);
+            const int nt2 = (nt + 1) & ~1;   // scales copy: a multiple of 16 bytes (cap is even)
+            const uint32_t cb = static_cast<uint32_t>(nt) * kIkey;
+            const uint32_t sb = static_cast<uint32_t>(nt2) * 8u;
+            mbar_arrive_expect_tx(&sm.full[s], cb + sb);
+            bulk_g2s(sm.codes[s], kbase + (size_t)tile * kIdxTile * kIkey, cb, &sm.full[s]);
+            bulk_g2s(sm.scales[s], sbase + (size_t)tile * kIdxTile * 2, sb, &sm.full[s]);
+        };
+        if (tid == 0)
+            for (int t = 0; t < min(n_tiles, kIdxStages); ++t) issue(t);
+
+        int consumed = 0;
+        bool ok = true;
+        for (int tile = 0; tile < n_tiles; ++tile) {
+            const int s = tile % kIdxStages;
+            const bool landed = mbar_wait(&sm.full[s], (tile / kIdxStages) & 1);
+            if (__syncthreads_or(!landed)) {
+                ok = false;
+                break;
+            }
+            consumed = tile + 1;
+            const uint8_t* cs = sm.codes[s];
+            const float* ss = sm.scales[s];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int rA = 32 * warp + 16 * half + g, rB = rA + 8;
+                const uint32_t kA0 = *reinterpret_cast<const uint32_t*>(cs + rA * kIkey + 4 * cq);
+                const uint32_t kB0 = *reinterpret_cast<const uint32_t*>(cs + rB * kIkey + 4 * cq);
+                const uint32_t kA1 = *reinterpret_cast<const uint32_t*>(cs + rA * kIkey + 16 + 4 * cq);
+                const uint32_t kB1 = *reinterpret_cast<const uint32_t*>(cs + rB * kIkey + 16 + 4 * cq);
+                int acc[4] = {0, 0, 0, 0};
+                auto lut = [](uint32_t sel) { return prmt(kTwiceE2M1Lo, kTwiceE2M1Hi, sel); };
+                mma_s8(acc, lut(kA0), lut(kB0), lut(kA0 >> 16), lut(kB0 >> 16), b00, b01);
+                {
+                    const uint32_t nA = kA0 ^ 0x88888888u, nB = kB0 ^ 0x88888888u;
+                    mma_s8(acc, lut(nA), lut(nB), lut(nA >> 16), lut(nB >> 16), n00, n01);
+                }
+                mma_s8(acc, lut(kA1), lut(kB1), lut(kA1 >> 16), lut(kB1 >> 16), b10, b11);
+                {
+                    const uint32_t nA = kA1 ^ 0x88888888u, nB = kB1 ^ 0x88888888u;
+                    mma_s8(acc, lut(nA), lut(nB), lut(nA >> 16), lut(nB >> 16), n10, n11);
+                }
+                // acc: (row g, cols 2cq, 2cq+1), (row g+8, same).  cq < 2: group-0 dots of
+                // heads 2cq, 2cq+1; cq >= 2: group-1 dots of heads 2(cq-2), 2(cq-2)+1.
+                const bool lo = cq < 2;
+                const int send0 = lo ? acc[2] : acc[0], send1 = lo ? acc[3] : acc[1];
+                const int got0 = __shfl_xor_sync(0xffffffffu, send0, 2);
+                const int got1 = __shfl_xor_sync(0xffffffffu, send1, 2);
+                const int row = lo ? rA : rB;
+                const int hp = (cq & 1) * 2;
+                const int i0a = lo ? acc[0] : got0, i0b = lo ? acc[1] : got1;
+                const int i1a = lo ? got0 : acc[2], i1b = lo ? got1 : acc[3];
+                const float ks0 = ss[2 * row], ks1 = ss[2 * row + 1];
+                float r[2];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int h = hp + q;
+                    const float s0 = __fmul_rn(__fmul_rn(sm.qscale[h], ks0), 0.25f);
+                    const float s1 = __fmul_rn(__fmul_rn(sm.qscale[4 + h], ks1), 0.25f);
+                    const int I0 = q ? i0b : i0a, I1 = q ? i1b : i1a;
+                    const float d = __fmaf_rn(static_cast<float>(I1), s1,
+                                              __fmul_rn(static_cast<float>(I0), s0));
+                    r[q] = d > 0.f ? d : 0.f;
+                }
+                const float r2 = __shfl_xor_sync(0xffffffffu, r[0], 1);
+                const float r3 = __shfl_xor_sync(0xffffffffu, r[1], 1);
+                if ((cq & 1) == 0) {
+                    float e = __fmul_rn(w0, r[0]);
+                    e = __fmaf_rn(w1, r[1], e);
+                    e = __fmaf_rn(w2, r2, e);
+                    e = __fmaf_rn(w3, r3, e);
+                    const int li = tile * kIdxTile + row;
+                    if (li < cn) {
+                        sm.keys[li] = score_key(e);
+                        sm.idx[li] = static_cast<int32_t>(c0 + li);
+                    }
+                }
+            }
+            __syncthreads();   // stage s fully consumed
+            if (tid == 0 && tile + kIdxStages < n_tiles) issue(tile + kIdxStages);
+        }
+        chunk_ok = ok;
+        if (!ok) {
+            // A copy did not land in time: record it, drain what is in flight (bounded), and
+            // publish this chunk as empty so the merge tree still completes.
+            if (tid == 0) {
+                dev_error(err, CSLD_DEVERR_TIMEOUT);
+                for (int t = consumed; t < min(n_tiles, consumed + kIdxStages); ++t)
+                    (void)mbar_wait(&sm.full[t % kIdxStages], (t / kIdxStages) & 1);
+            }
+            __syncthreads();
+        }
+        // (the stage barriers are not reused after this point)
+    }
+
+    // --- selection and the merge tree ------------------------------------------------------
+    int n = (cn > 0 && chunk_ok) ? cn : 0;   // a timed-out chunk publishes nothing
+    int level = 0, run = ch;
+    for (;;) {
+        const int n_runs = tree.n_runs[level];
+        const bool final_run = (n_runs == 1);
+        const int want = min(final_run ? k : kc, n);
+        uint32_t thr = 0u, take_eq = static_cast<uint32_t>(n);
+        if (want < n) thr = radix_select([&](int i) { return sm.keys[i]; }, n, want, sm.hist, sm.sel, &take_eq);
+        if (final_run) {
+            int32_t* out = topk_out + (size_t)b * k;
+            select_compact([&](int i) { return sm.keys[i]; }, n, thr, take_eq, sm.scan,
+                           [&](uint32_t pos, int i) { out[pos] = sm.idx[i]; });
+            for (int i = want + tid; i < k; i += blockDim.x) out[i] = -1;
+            return;
+        }
+        const size_t rb = ((size_t)b * n_runs + run) * kc;
+        uint32_t* okeys = tree.keys[level] + rb;
+        int32_t* oidx = tree.idx[level] + rb;
+        select_compact([&](int i) { return sm.keys[i]; }, n, thr, take_eq, sm.scan,
+                       [&](uint32_t pos, int i) {
+                           okeys[pos] = sm.keys[i];
+                           oidx[pos] = sm.idx[i];
+                       });
+        if (tid == 0) tree.cnt[level][(size_t)b * n_runs + run] = want;
+        // arrive at the parent; the last child to arrive carries on with the merge
+        const int parent = run / tree.group;
+        const int n_par = tree.n_runs[level + 1];
+        const int children = min(tree.group, n_runs - parent * tree.group);
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            int32_t* ctr = tree.ctr[level + 1] + (size_t)b * n_par + parent;
+            const int old = atomicAdd(ctr, 1);
+            sm.last = (old == children - 1);
+            if (sm.last) {
+                *ctr = 0;          // leave the counter ready for the next call
+                __threadfence();
+            }
+        }
+        __syncthreads();
+        if (!sm.last) return;
+        // load the children runs (published by other CTAs: read through L2)
+        if (tid == 0) {
+            int acc = 0;
+            for (int c = 0; c < children; ++c) {
+                sm.offs[c] = acc;
+                acc += __ldcg(tree.cnt[level] + (size_t)b * n_runs + parent * tree.group + c);
+            }
+            sm.offs[children] = acc;
+        }
+        __syncthreads();
+        for (int c = 0; c < children; ++c) {
+            const int cc = sm.offs[c + 1] - sm.offs[c];
+            const size_t src = ((size_t)b * n_runs + parent * tree.group + c) * kc;
+            for (int i = tid; i < cc; i += blockDim.x) {
+                sm.keys[sm.offs[c] + i] = __ldcg(tree.keys[level] + src + i);
+                sm.idx[sm.offs[c] + i] = __ldcg(tree.idx[level] + src + i);
+            }
+        }
+        n = sm.offs[children];
+        __syncthreads();
+        ++level;
+        run = parent;
+    }
+}
+
+IndexerPlan indexer_plan(int B, int64_t cap, int k, int num_sms) {
+    IndexerPlan p;
+    int chunk = kIdxMaxChunk;
+    while (chunk > 1024 && (int64_t)B * ((cap + chunk - 1) / chunk) < num_sms) chunk >>= 1;
+    p.chunk = chunk;
+    const int64_t nc = (cap + chunk - 1) / chunk;
+    p.n_chunks = static_cast<int>(nc < 1 ? 1 : nc);
+    p.kc = k < chunk ? k : chunk;
+    int group = kIdxMaxChunk / p.kc;
+    if (group > kIdxMaxGroup) group = kIdxMaxGroup;
+    if (group < 2) group = 2;
+    p.group = group;
+    size_t bytes = 0;
+    IdxTree t = tree_layout(B, p.n_chunks, p.kc, group, nullptr, &bytes);
+    p.levels_ok = (t.n_runs[t.levels] == 1);
+    p.ws_bytes = bytes;
+    return p;
+}
+
+cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                           const int32_t* seq_len, int ratio, const float* q_idx,
+                           const float* head_w, int B, int k, int32_t* topk_out, void* ws,
+                           const IndexerPlan& plan, int32_t* err, cudaStream_t stream) {
+    size_t bytes = 0;
+    IdxTree tree = tree_layout(B, plan.n_chunks, plan.kc, plan.group, static_cast<uint8_t*>(ws), &bytes);
+    const size_t smem = sizeof(IdxSmem);
+    cudaError_t e = set_smem_once(indexer_topk_kernel, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(plan.n_chunks, B);
+    indexer_topk_kernel<<<grid, kIdxThreads, smem, stream>>>(ikeys, iscales, cap, seq_len, ratio,
+                                                             q_idx, head_w, plan.chunk, plan.kc, k,
+                                                             tree, topk_out, err);
+    return cudaGetLastError();
+}
+
+}  // namespace csld

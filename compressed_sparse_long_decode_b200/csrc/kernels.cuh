@@ -1,0 +1,50 @@
+// Launchers of the libcsld kernels (host side, internal).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csld.h"
+
+namespace csld {
+
+cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float* bias, int m,
+                            const float* w_idx, int64_t T, int B, int64_t out_seq_stride,
+                            uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, int num_sms,
+                            cudaStream_t stream);
+size_t compress_index_smem_bytes();
+
+cudaError_t launch_prefill_state(const uint16_t* raw, const float* gate, int64_t T, int m, int W,
+                                 int B, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
+                                 int32_t* seq_len, cudaStream_t stream);
+
+cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
+                          const float* gate_new, int32_t* err, cudaStream_t stream);
+
+// Lightning indexer + top-k.
+struct IndexerPlan {
+    int chunk;          // entries per scoring CTA (multiple of 256)
+    int n_chunks;       // chunks per sequence (over the capacity)
+    int kc;             // candidates kept per chunk = min(k, chunk)
+    int group;          // runs merged by one CTA in the merge tree
+    bool levels_ok;     // the merge tree reaches one run within its level limit
+    size_t ws_bytes;    // workspace bytes (must be zero-filled before first use)
+};
+IndexerPlan indexer_plan(int B, int64_t cap, int k, int num_sms);
+cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                           const int32_t* seq_len, int ratio, const float* q_idx,
+                           const float* head_w, int B, int k, int32_t* topk_out, void* ws,
+                           const IndexerPlan& plan, int32_t* err, cudaStream_t stream);
+
+// Hybrid decode attention.
+struct AttentionPlan {
+    int splits;         // CTAs per sequence
+    size_t ws_bytes;
+};
+AttentionPlan attention_plan(int B, int64_t cap, int k, bool sparse, int W, int num_sms);
+cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
+                             const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                             const int32_t* seq_len, int B, float scale, float* out,
+                             float* lse_out, void* ws, const AttentionPlan& plan, int32_t* err,
+                             cudaStream_t stream);
+
+}  // namespace csld

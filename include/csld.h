@@ -1,0 +1,204 @@
+/*
+ * csld.h -- C ABI of libcsld.so: the decode hot path of hybrid compressed attention
+ * (CSA + HCA) on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the pages about DeepSeek-V4:
+ *  [HF]  "DeepSeek-V4: a million-token context that agents can actually use" (Korean rendering
+ *        of the Hugging Face blog): CSA paragraph and Figure 3 caption (4x softmax-gated pooling
+ *        with a learned positional bias; FP4 ReLU-scored multi-head lightning indexer; top-k
+ *        compressed blocks per query; sliding-window branch), HCA paragraph and Figure 4 caption
+ *        (128x compression, dense attention over the compressed stream, same window branch),
+ *        storage paragraph (KV mostly FP8, RoPE dims BF16, indexer FP4).
+ *  [VEL] velog.io "DeepSeek V4 paper review": "core technique 1: CSA", "core technique 2: HCA",
+ *        and the KV-cache-layout section (compressed caches, a separate sliding-window state,
+ *        a separately kept uncompressed tail).
+ *
+ * Conventions for every call:
+ *  - All array pointers are DEVICE pointers owned by the caller; the library allocates nothing.
+ *    Scratch ("workspace") is caller-provided; its size comes from the *_workspace_size query.
+ *  - bf16 values are passed as their raw 16-bit patterns (uint16_t).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Every
+ *    call only enqueues work on `stream` and returns; nothing synchronises the host.
+ *  - Arguments are validated on the host before anything is launched; on a bad argument the
+ *    call returns a non-zero csld_status, launches nothing and leaves a message in
+ *    csld_last_error() (thread-local).  A failed launch returns CSLD_ERR_CUDA.
+ *  - Conditions only the device can see (a top-k index that is not a visible entry, a full
+ *    compressed cache) are never turned into traps: the kernel skips the offending item and
+ *    ORs a flag into the caller's device error word `err` (may be NULL), see CSLD_DEVERR_*.
+ *  - Shapes fixed by the format: D = 512 (448 "nope" dims stored E4M3 + 64 RoPE dims stored
+ *    bf16, one shared KV head whose 512-d entry is both key and value), 16 query heads per KV
+ *    head in the decode kernel, 4 indexer heads x 64 dims.
+ */
+#ifndef CSLD_H
+#define CSLD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSLD_API __attribute__((visibility("default")))
+#else
+#define CSLD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSLD_ABI_VERSION 1
+
+#define CSLD_DIM 512            /* entry / head dimension */
+#define CSLD_DIM_NOPE 448       /* dims 0..447 stored as E4M3 (scale 1, RNE, saturating) */
+#define CSLD_DIM_ROPE 64        /* dims 448..511 stored as bf16 */
+#define CSLD_ENTRY_BYTES 576    /* 448 E4M3 bytes followed by 64 little-endian bf16 */
+#define CSLD_HEADS 16           /* query heads sharing the KV head (decode kernel) */
+#define CSLD_IDX_HEADS 4        /* lightning-indexer heads */
+#define CSLD_IDX_DIM 64         /* lightning-indexer dims per head (one key shared by the heads) */
+#define CSLD_IKEY_BYTES 32      /* 64 E2M1 codes, element 2i in the low nibble of byte i */
+#define CSLD_IKEY_SCALES 2      /* fp32 power-of-two scale per group of 32 codes */
+#define CSLD_MAX_RATIO 128      /* tokens per compressed entry: 1..128 (CSA 4, HCA 128) */
+#define CSLD_MAX_WINDOW 1024    /* sliding-window length in raw tokens: 0..1024 */
+#define CSLD_MAX_TOPK 2048      /* indexer top-k: 1..2048 */
+
+typedef enum csld_status {
+    CSLD_OK = 0,
+    CSLD_ERR_ARG = 1,          /* null pointer or out-of-range scalar */
+    CSLD_ERR_SHAPE = 2,        /* inconsistent sizes */
+    CSLD_ERR_ALIGN = 3,        /* a pointer or stride is not 16-byte aligned */
+    CSLD_ERR_CAPACITY = 4,     /* a size exceeds a stated maximum or the cache capacity */
+    CSLD_ERR_CUDA = 5,         /* a CUDA runtime error (launch failure, no device, ...) */
+    CSLD_ERR_UNSUPPORTED = 6,  /* a shape this build does not implement (e.g. heads != 16) */
+    CSLD_ERR_WORKSPACE = 7     /* workspace pointer NULL or smaller than required */
+} csld_status;
+
+/* Device error word flags (ORed into `err` by kernels). */
+#define CSLD_DEVERR_CAPACITY 1u     /* kv_cache_append: entry index >= capacity; token dropped */
+#define CSLD_DEVERR_BAD_INDEX 2u    /* hybrid_decode_attention: a top-k index was not visible */
+#define CSLD_DEVERR_SEQ_LEN 4u      /* a seq_len < 0; that sequence was treated as empty */
+#define CSLD_DEVERR_TIMEOUT 8u      /* a bounded wait for an asynchronous copy gave up */
+
+CSLD_API int csld_abi_version(void);
+CSLD_API const char* csld_last_error(void);
+CSLD_API const char* csld_status_string(csld_status s);
+
+/* ----------------------------------------------------------------------------------------
+ * Prefill compression ([HF] CSA paragraph, Figure 3; HCA paragraph, Figure 4).
+ * For one sequence of T raw tokens, block s = tokens s*m .. s*m+m-1 becomes entry s:
+ *   a_j = gate[s*m+j] + pos_bias[j];  w = softmax(a);  c = sum_j w_j * raw[s*m+j]   (fp32)
+ *   kv_out[s]  = E4M3(c[0:448]) || bf16(c[448:512])                                 (RNE)
+ * and, when w_idx != NULL (CSA layers), the lightning-indexer key
+ *   u = c . W_I  (bf16 operands, fp32 accumulation),  ikey_out[s] = E2M1 codes of u / sigma_g,
+ *   iscale_out[s][g] = sigma_g = smallest power of two with max|u in group g| <= 6 sigma_g.
+ * The trailing T mod m tokens form no entry.
+ *   raw        [T][512] bf16     gate [T] f32     pos_bias [m] f32     w_idx [512][64] f32
+ *   kv_out     [T/m][576] u8     ikey_out [T/m][32] u8     iscale_out [T/m][2] f32
+ * raw, kv_out, ikey_out must be 16-byte aligned.  1 <= ratio <= 128.
+ * csa_compress = csld_compress with ratio 4 and the indexer key; hca_compress = ratio 128
+ * without it.
+ * -------------------------------------------------------------------------------------- */
+CSLD_API csld_status csld_compress(const uint16_t* raw, const float* gate, const float* pos_bias,
+                          int ratio, const float* w_idx, int64_t T, uint8_t* kv_out,
+                          uint8_t* ikey_out, float* iscale_out, void* stream);
+CSLD_API csld_status csa_compress(const uint16_t* raw, const float* gate, const float* pos_bias,
+                         const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
+                         float* iscale_out, void* stream);
+CSLD_API csld_status hca_compress(const uint16_t* raw, const float* gate, const float* pos_bias,
+                         int64_t T, uint8_t* kv_out, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * One layer's KV-cache state for B sequences ([VEL] KV-cache-layout section: compressed
+ * cache, separate sliding-window state, separately kept uncompressed tail).  A host struct of
+ * device pointers; the caller owns all of it.
+ *   comp_kv   [B][capacity][576]  compressed entries (entry s = tokens s*m .. s*m+m-1)
+ *   ikeys     [B][capacity][32]   indexer key codes     (has_indexer != 0; else NULL)
+ *   iscales   [B][capacity][2]    indexer key scales    (has_indexer != 0; else NULL)
+ *   win_kv    [B][window][576]    ring of the last `window` raw tokens, token t at slot t mod W
+ *   tail_kv   [B][ratio][512]     bf16 raw tokens of the block being filled, token t at t mod m
+ *   tail_gate [B][ratio]          their gate logits
+ *   seq_len   [B]                 raw tokens so far (int32, device)
+ *   pos_bias  [ratio]             positional bias of the pooling
+ *   w_idx     [512][64]           indexer projection (has_indexer != 0)
+ * capacity must be even (16-byte alignment of the per-sequence scale arrays).
+ * -------------------------------------------------------------------------------------- */
+typedef struct csld_layer_cache {
+    int32_t ratio;
+    int32_t window;
+    int32_t batch;
+    int32_t has_indexer;
+    int64_t capacity;
+    uint8_t* comp_kv;
+    uint8_t* ikeys;
+    float* iscales;
+    uint8_t* win_kv;
+    uint16_t* tail_kv;
+    float* tail_gate;
+    int32_t* seq_len;
+    const float* pos_bias;
+    const float* w_idx;
+} csld_layer_cache;
+
+/* Decode-time append of ONE raw token per sequence ([VEL] KV-cache layout; [HF] Figures 3-4).
+ * For sequence b with t = seq_len[b]:  window slot t mod W <- entry(kv_new[b]);
+ * tail slot t mod m <- (kv_new[b], gate_new[b]);  when (t+1) mod m == 0 the m tail tokens are
+ * pooled (same arithmetic as csld_compress) into entry t/m (+ indexer key);  seq_len[b] = t+1.
+ * If entry t/m would not fit in capacity, nothing of sequence b changes and
+ * CSLD_DEVERR_CAPACITY is ORed into *err.
+ *   kv_new [B][512] bf16, gate_new [B] f32, err: device int32 or NULL. */
+CSLD_API csld_status kv_cache_append(const csld_layer_cache* cache, const uint16_t* kv_new,
+                            const float* gate_new, int32_t* err, void* stream);
+
+/* Prefill of all B sequences with T raw tokens each (raw [B][T][512], gate [B][T]): writes
+ * entries 0..T/m-1 (+ keys), the window ring with the last min(W, T) tokens, the tail with the
+ * last T mod m tokens, and sets seq_len[b] = T.  Equivalent to T calls of kv_cache_append on
+ * an empty cache.  Requires T/m <= capacity. */
+CSLD_API csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint16_t* raw,
+                             const float* gate, int64_t T, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Lightning indexer + top-k ([HF] CSA paragraph: "FP4, ReLU-scored multi-head dot product"
+ * picks the top-k compressed blocks per query; [VEL] core technique 1).
+ * For sequence b, the visible entries are s < n_b = min(seq_len[b] / ratio, cap).  The query
+ * q_idx[b][h] (fp32) is quantised to FP4 exactly like the keys (E2M1, power-of-two scale per
+ * 32); per entry and head the two FP4 vectors give an exact dot d; the score is
+ *   e_s = sum_h head_w[b][h] * max(d_h, 0)
+ * formed in fp32 in the fixed order  e = w0*r0; e = fma(w1,r1,e); e = fma(w2,r2,e);
+ * e = fma(w3,r3,e)  with  d_h = fma(I1, s1, I0*s0),  I_g the integer group dots (x4) and
+ * s_g = (qscale_g * kscale_g) * 0.25.  The min(k, n_b) entries with the largest (score,
+ * -index) are written to topk_out[b] in ascending index order, followed by -1 padding.
+ *   ikeys [B][cap][32] u8, iscales [B][cap][2] f32, seq_len [B] i32, q_idx [B][4][64] f32,
+ *   head_w [B][4] f32, topk_out [B][k] i32.  cap even; ikeys 16-byte aligned; 1 <= k <= 2048.
+ * Workspace: csld_indexer_workspace_size(B, cap, k) bytes, 256-byte aligned, zero-filled once
+ * before its first use (it holds arrival counters that every call leaves at zero again); calls
+ * that share one workspace must not overlap on the GPU.  err: device error word or NULL. */
+CSLD_API size_t csld_indexer_workspace_size(int B, int64_t cap, int k);
+CSLD_API csld_status indexer_topk(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                         const int32_t* seq_len, int ratio, const float* q_idx,
+                         const float* head_w, int B, int k, int32_t* topk_out, void* ws,
+                         size_t ws_bytes, int32_t* err, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Hybrid decode attention ([HF] CSA paragraph + Figure 3: attention over the selected entries
+ * plus a sliding-window branch; HCA paragraph + Figure 4: dense attention over every
+ * compressed entry plus the same window branch).
+ * For sequence b (n = seq_len[b], n_vis = min(n / ratio, cap)) the key set is
+ *   { comp_kv[b][s] : s in topk[b], s >= 0 }   (sparse mode, topk != NULL), or
+ *   { comp_kv[b][s] : s < n_vis }                (dense mode, topk == NULL),
+ * together with { win_kv[b][t mod W] : max(0, n-W) <= t < n }.  Keys = values = the decoded
+ * 512-vectors; for each head h: out[b][h] = softmax(scale * q[b][h] . K^T) V, one joint
+ * softmax over the union; lse_out[b][h] = natural log of the softmax denominator in logit
+ * units.  An empty key set gives out = 0 and lse = -inf.
+ *   q [B][heads][512] bf16 (heads == 16), comp_kv [B][cap][576], topk [B][k] i32 or NULL,
+ *   win_kv [B][W][576], seq_len [B] i32, out [B][heads][512] f32, lse_out [B][heads] f32 or NULL.
+ * comp_kv, win_kv must be 16-byte aligned.  Workspace: csld_attention_workspace_size(...).
+ * -------------------------------------------------------------------------------------- */
+CSLD_API size_t csld_attention_workspace_size(int B, int heads, int64_t cap, int k, int W);
+CSLD_API csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t* comp_kv,
+                                    int64_t cap, int ratio, const int32_t* topk, int k,
+                                    const uint8_t* win_kv, int W, const int32_t* seq_len, int B,
+                                    float scale, float* out, float* lse_out, void* ws,
+                                    size_t ws_bytes, int32_t* err, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSLD_H */

@@ -1,0 +1,147 @@
+"""Comparison helpers shared by the GPU parity tests (tolerances as stated for the path).
+
+- compressed entries: E4M3 codes within one code step of the float64 oracle's; bf16 RoPE
+  values within one bf16 ulp of the oracle's plus the error bound of the GPU's fp32 weighted
+  sum of m tokens, (m+2) 2^-24 max|x| (pool_slack) -- a value produced by cancellation near
+  zero cannot be resolved to a bf16 ulp by an fp32 sum; the stated bar for the cache, one FP8
+  ulp, is far looser than this;
+- FP4 indexer keys: equal scales and codes within one grid step, except groups whose oracle
+  amax/6 lies within 2^-8 (relative) of a power of two, where the scale may differ by one
+  binade (the GPU forms the projection from bf16 operands);
+- top-k sets: bit-exact; pairs of entries whose float64 scores differ by < 1e-6 relative are
+  exempt when the float64 order is used;
+- attention: |gpu - oracle| <= 2e-2 + 1e-2 |oracle| elementwise, for out and lse.
+"""
+import math
+
+import numpy as np
+
+ATOL = 2e-2
+RTOL = 1e-2
+
+
+def e4m3_ordinal(codes):
+    c = np.asarray(codes).astype(np.int32)
+    mag = c & 0x7F
+    return np.where(c & 0x80, -mag, mag)
+
+
+def bf16_ordinal(bits):
+    b = np.asarray(bits).astype(np.int64)
+    mag = b & 0x7FFF
+    return np.where(b & 0x8000, -mag, mag)
+
+
+def bf16_values(bits):
+    b = np.asarray(bits, np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def bf16_ulp(vals):
+    """Spacing of bf16 values at |vals| (the fp32 spacing times 2^16)."""
+    return np.spacing(np.abs(vals).astype(np.float32)).astype(np.float64) * 65536.0
+
+
+def pool_slack(raw_bf16, m):
+    """fp32 error bound of an m-term convex combination of the given bf16 tokens."""
+    x = np.abs(np.asarray(raw_bf16.float().cpu().numpy() if hasattr(raw_bf16, "float") else raw_bf16))
+    return (m + 2) * 2.0 ** -24 * float(x.max(initial=0.0))
+
+
+def entry_distance(gpu, ref):
+    """(max E4M3 code distance, max bf16 |difference| in units of the oracle's ulp)."""
+    gpu = np.asarray(gpu, np.uint8).reshape(-1, 576)
+    ref = np.asarray(ref, np.uint8).reshape(-1, 576)
+    d8 = np.abs(e4m3_ordinal(gpu[:, :448]) - e4m3_ordinal(ref[:, :448])).max(initial=0)
+    g = bf16_values(gpu[:, 448:].copy().view(np.uint16))
+    r = bf16_values(ref[:, 448:].copy().view(np.uint16))
+    return int(d8), g, r
+
+
+def assert_entries_close(gpu, ref, what="entries", abs_slack=0.0):
+    d8, g, r = entry_distance(gpu, ref)
+    assert d8 <= 1, f"{what}: E4M3 code distance {d8}"
+    err = np.abs(g - r)
+    bound = bf16_ulp(r) + abs_slack
+    assert np.all(err <= bound), f"{what}: bf16 error {float((err - bound).max()):.3g} above bound"
+    gb = np.asarray(gpu, np.uint8).reshape(-1)
+    rb = np.asarray(ref, np.uint8).reshape(-1)
+    return float((gb == rb).mean())
+
+
+def _fp4_ord(codes):
+    c = np.asarray(codes).astype(np.int32)
+    return np.where(c & 8, -(c & 7), c & 7)
+
+
+def unpack_fp4(keys):
+    k = np.asarray(keys, np.uint8)
+    lo = k & 0xF
+    hi = k >> 4
+    out = np.empty(k.shape[:-1] + (k.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def assert_fp4_keys_close(gkeys, gscales, rkeys, rscales, ramax=None):
+    """gkeys/rkeys [E,32] u8, gscales/rscales [E,2] f32; ramax [E,2] oracle group amax (or None)."""
+    gc = unpack_fp4(gkeys).reshape(-1, 2, 32)
+    rc = unpack_fp4(rkeys).reshape(-1, 2, 32)
+    gs = np.asarray(gscales, np.float32).reshape(-1, 2)
+    rs = np.asarray(rscales, np.float32).reshape(-1, 2)
+    same = gs == rs
+    d = np.abs(_fp4_ord(gc) - _fp4_ord(rc)).max(axis=2)
+    assert np.all(d[same] <= 1), f"FP4 codes differ by {d[same].max()} steps at equal scales"
+    if not np.all(same):
+        bad = np.argwhere(~same)
+        assert ramax is not None, "scales differ and no oracle amax was given"
+        for e, g in bad:
+            ratio = gs[e, g] / rs[e, g]
+            assert ratio in (0.5, 2.0), f"scale ratio {ratio}"
+            a6 = float(ramax[e, g]) / 6.0
+            near = abs(a6 / 2.0 ** round(math.log2(a6)) - 1.0) < 2.0 ** -8
+            assert near, f"scales differ away from a power-of-two boundary (amax/6={a6})"
+    return float(same.mean())
+
+
+def assert_attention_close(gout, glse, rout, rlse, what="attention"):
+    gout = np.asarray(gout, np.float64)
+    rout = np.asarray(rout, np.float64)
+    err = np.abs(gout - rout)
+    bound = ATOL + RTOL * np.abs(rout)
+    worst = float((err - bound).max(initial=-1.0))
+    assert np.all(err <= bound), f"{what}: out exceeds tolerance by {worst:.3g} (max abs err {err.max():.3g})"
+    if glse is not None:
+        glse = np.asarray(glse, np.float64)
+        rlse = np.asarray(rlse, np.float64)
+        fin = np.isfinite(rlse)
+        assert np.array_equal(np.isfinite(glse), fin), f"{what}: lse finiteness differs"
+        le = np.abs(glse[fin] - rlse[fin])
+        assert np.all(le <= ATOL + RTOL * np.abs(rlse[fin])), f"{what}: lse error {le.max():.3g}"
+    return float(err.max(initial=0.0))
+
+
+def assert_topk_equal(gpu, ref, score64=None):
+    gpu = np.asarray(gpu)
+    ref = np.asarray(ref)
+    assert gpu.shape == ref.shape
+    if np.array_equal(gpu, ref):
+        return
+    bad = np.argwhere(np.any(gpu != ref, axis=-1)).ravel() if gpu.ndim == 2 else [None]
+    raise AssertionError(f"top-k sets differ (rows {list(bad)[:8]})")
+
+
+def near_tie_only(set_a, set_b, score64, rel=1e-6):
+    """True if every entry in the symmetric difference of two selections has a partner on the
+    other side whose float64 score is within rel of its own (the exemption for near-ties)."""
+    a = set(int(x) for x in set_a if x >= 0)
+    b = set(int(x) for x in set_b if x >= 0)
+    only_a, only_b = a - b, b - a
+    if not only_a and not only_b:
+        return True
+    if len(only_a) != len(only_b):
+        return False
+    sa = sorted(score64[i] for i in only_a)
+    sb = sorted(score64[i] for i in only_b)
+    return all(abs(x - y) <= rel * max(abs(x), abs(y), 1e-300) for x, y in zip(sa, sb))

@@ -1,0 +1,86 @@
+"""End-to-end parity of the tiny single-layer-pair decode workload: 4080 prefill tokens then 16
+decode steps (each: append to the CSA and HCA layers, indexer top-k 128 on the CSA layer,
+sparse CSA attention and dense HCA attention, both with a 128-token window), ending at 4096
+tokens = 1024 CSA and 32 HCA entries.  Each stage is also checked on identical input bytes:
+the GPU indexer on the oracle's keys must reproduce the oracle's selection bit for bit, and
+the GPU attention on the oracle's cache must match the oracle's output."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+SCALE = 1.0 / math.sqrt(512.0)
+
+
+@pytest.fixture(scope="module")
+def csld():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import compressed_sparse_long_decode_b200 as m
+    return m
+
+
+def test_tiny_decode_workload(csld, orc):
+    T0, steps, W, k = 4080, 16, 128, 128
+    inp = synth.prefill_inputs(T0 + steps, seed=0)
+    raw, gate = inp["raw"], inp["gate"]
+    bits = synth.bits16(raw)[None]
+    gates = gate.numpy()[None]
+    # GPU layers
+    csa = csld.LayerCache(1, 1030, 4, W, inp["bias4"], inp["w_idx"])
+    hca = csld.LayerCache(1, 34, 128, W, inp["bias128"])
+    csld.kv_cache_prefill(csa, raw[None, :T0].contiguous().cuda(), gate[None, :T0].contiguous().cuda())
+    csld.kv_cache_prefill(hca, raw[None, :T0].contiguous().cuda(), gate[None, :T0].contiguous().cuda())
+    # oracle layers
+    ocsa = orc.LayerState(1, csa.capacity, 4, W, True)
+    ohca = orc.LayerState(1, hca.capacity, 128, W, False)
+    for t in range(T0):
+        orc.append_batch(ocsa, inp["bias4"].numpy(), inp["w_idx"].numpy(), bits[:, t].copy(), gates[:, t].copy())
+        orc.append_batch(ohca, inp["bias128"].numpy(), None, bits[:, t].copy(), gates[:, t].copy())
+    overlap = []
+    for step in range(steps):
+        t = T0 + step
+        qs = synth.decode_queries(1, seed=100 + step)
+        x = raw[t:t + 1].contiguous().cuda()
+        z = gate[t:t + 1].contiguous().cuda()
+        csld.kv_cache_append(csa, x, z)
+        csld.kv_cache_append(hca, x, z)
+        orc.append_batch(ocsa, inp["bias4"].numpy(), inp["w_idx"].numpy(), bits[:, t].copy(), gates[:, t].copy())
+        orc.append_batch(ohca, inp["bias128"].numpy(), None, bits[:, t].copy(), gates[:, t].copy())
+        sel = csld.indexer_topk(csa.ikeys, csa.iscales, csa.seq_len, 4, qs["q_idx"].cuda(), qs["head_w"].cuda(), k)
+        o_csa, l_csa = csld.hybrid_decode_attention(qs["q"].cuda(), csa.comp_kv, 4, sel, csa.win_kv, W,
+                                                    csa.seq_len, SCALE)
+        o_hca, l_hca = csld.hybrid_decode_attention(qs["q"].cuda(), hca.comp_kv, 128, None, hca.win_kv, W,
+                                                    hca.seq_len, SCALE)
+        torch.cuda.synchronize()
+        # oracle pipeline on its own state
+        osel = orc.indexer_topk_batch(ocsa.ikeys, ocsa.iscales, ocsa.seq_len, 4, qs["q_idx"].numpy(),
+                                      qs["head_w"].numpy(), k)
+        qb = synth.bits16(qs["q"])
+        ro_csa, rl_csa = orc.attention_batch(qb, ocsa.comp_kv, 4, osel, ocsa.win_kv, ocsa.seq_len, SCALE)
+        ro_hca, rl_hca = orc.attention_batch(qb, ohca.comp_kv, 128, None, ohca.win_kv, ohca.seq_len, SCALE)
+        H.assert_attention_close(o_hca.cpu().numpy(), l_hca.cpu().numpy(), ro_hca, rl_hca, f"HCA step {step}")
+        H.assert_attention_close(o_csa.cpu().numpy(), l_csa.cpu().numpy(), ro_csa, rl_csa, f"CSA step {step}")
+        gsel = sel.cpu().numpy()
+        overlap.append(len(set(gsel[0]) & set(osel[0])) / k)
+        # stage checks on identical bytes: the oracle's keys -> GPU indexer; the oracle's cache -> GPU attention
+        sel_o = csld.indexer_topk(torch.from_numpy(ocsa.ikeys).cuda(), torch.from_numpy(ocsa.iscales).cuda(),
+                                  torch.from_numpy(ocsa.seq_len).cuda(), 4, qs["q_idx"].cuda(),
+                                  qs["head_w"].cuda(), k)
+        H.assert_topk_equal(sel_o.cpu().numpy(), osel)
+        o2, l2 = csld.hybrid_decode_attention(qs["q"].cuda(), torch.from_numpy(ocsa.comp_kv).cuda(), 4,
+                                              torch.from_numpy(osel).cuda(), torch.from_numpy(ocsa.win_kv).cuda(),
+                                              W, torch.from_numpy(ocsa.seq_len).cuda(), SCALE)
+        H.assert_attention_close(o2.cpu().numpy(), l2.cpu().numpy(), ro_csa, rl_csa, f"CSA step {step} (same bytes)")
+    assert csa.seq_len.item() == 4096 and hca.seq_len.item() == 4096
+    assert int(csa.seq_len.item()) // 4 == 1024 and int(hca.seq_len.item()) // 128 == 32
+    H.assert_entries_close(csa.comp_kv[:, :1024].cpu().numpy(), ocsa.comp_kv[:, :1024], "CSA cache",
+                            H.pool_slack(raw, 4))
+    H.assert_entries_close(hca.comp_kv[:, :32].cpu().numpy(), ohca.comp_kv[:, :32], "HCA cache",
+                            H.pool_slack(raw, 128))
+    # GPU and oracle keys differ by at most one FP4 step; their selections nearly coincide
+    assert min(overlap) >= 0.95, overlap

@@ -1,0 +1,95 @@
+"""GPU parity of the lightning indexer + top-k: the selected index sets must equal the oracle's
+bit for bit (both take the selection in fp32 with the same operation order), at small sizes
+and at the full decode workloads, including ties, padding and ragged lengths."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def csld():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import compressed_sparse_long_decode_b200 as m
+    return m
+
+
+def _run(csld, orc, ikeys, iscales, seq_len, q_idx, head_w, k, ratio=4):
+    dev = [t.cuda() for t in (ikeys, iscales, seq_len, q_idx, head_w)]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = csld.indexer_topk(*dev[:3], ratio, dev[3], dev[4], k, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref = orc.indexer_topk_batch(ikeys.numpy(), iscales.numpy(), seq_len.numpy(), ratio,
+                                 q_idx.numpy(), head_w.numpy(), k)
+    return out.cpu().numpy(), ref
+
+
+def _inputs(B, cap, n_valid, seed, heavy=0.0):
+    g = synth.gen(seed)
+    ik, isc = synth.random_ikeys(B, cap, g, heavy_frac=heavy, n_valid=n_valid)
+    qs = synth.decode_queries(B, seed=seed + 1)
+    return ik, isc, qs["q_idx"], qs["head_w"]
+
+
+@pytest.mark.parametrize("B,n_c,k", [(1, 1024, 128), (3, 5000, 256), (2, 300, 512), (1, 8192 * 2 + 77, 1024),
+                                     (4, 20000, 1), (2, 9000, 2048)])
+def test_indexer_topk_matches_oracle(csld, orc, B, n_c, k):
+    cap = n_c + (n_c & 1) + 64
+    ik, isc, q, w = _inputs(B, cap, n_c, seed=B * 1000 + k)
+    seq = torch.full((B,), 4 * n_c + 3, dtype=torch.int32)
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, k)
+    H.assert_topk_equal(got, ref)
+
+
+def test_indexer_ragged_lengths_and_padding(csld, orc):
+    B, cap, k = 6, 4096, 200
+    ik, isc, q, w = _inputs(B, cap, cap, seed=5)
+    seq = torch.tensor([0, 3, 4, 4 * 150 + 1, 4 * 4000, 4 * 5000], dtype=torch.int32)  # last: > cap
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, k)
+    H.assert_topk_equal(got, ref)
+    assert np.all(got[0] == -1) and np.all(got[1] == -1)
+    assert got[2, 0] == 0 and np.all(got[2, 1:] == -1)
+    assert np.array_equal(got[3, :150], np.arange(150)) and np.all(got[3, 150:] == -1)
+
+
+def test_indexer_exact_ties_go_to_lower_index(csld, orc):
+    B, cap, k = 2, 6000, 300
+    ik = torch.zeros((B, cap, 32), dtype=torch.uint8)
+    ik[:, :, :] = 0x22                                   # every code +1.0: identical keys
+    ik[0, 4000:4100, :] = 0x44                           # 100 keys with code +2.0 on seq 0
+    isc = torch.ones((B, cap, 2), dtype=torch.float32)
+    q = torch.ones((B, 4, 64))
+    w = torch.ones((B, 4))
+    seq = torch.full((B,), 4 * cap, dtype=torch.int32)
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, k)
+    H.assert_topk_equal(got, ref)
+    assert np.array_equal(got[1], np.arange(k))
+    assert np.array_equal(got[0], np.concatenate([np.arange(200), np.arange(4000, 4100)]))
+
+
+def test_indexer_negative_weights_and_relu(csld, orc):
+    B, cap, k = 2, 2048, 64
+    ik, isc, q, w = _inputs(B, cap, cap, seed=9)
+    w[0] = torch.tensor([1.0, -2.0, 0.5, -0.25])
+    w[1] = torch.tensor([-1.0, -1.0, -1.0, -1.0])       # all scores <= 0: ties at zero
+    seq = torch.full((B,), 4 * cap, dtype=torch.int32)
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, k)
+    H.assert_topk_equal(got, ref)
+
+
+@pytest.mark.parametrize("name", ["decode128k", "decode1m"])
+def test_indexer_full_workloads(csld, orc, name):
+    wl = synth.WORKLOADS[name]
+    ik, isc, q, w = _inputs(wl.batch, wl.csa_cap, wl.csa_entries, seed=11, heavy=wl.heavy_frac)
+    seq = torch.full((wl.batch,), wl.context, dtype=torch.int32)
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, wl.topk)
+    H.assert_topk_equal(got, ref)
+    # the fp32 decision agrees with the float64 one up to near-ties
+    s32, s64 = orc.indexer_scores(ik[0, :wl.csa_entries].numpy(), isc[0, :wl.csa_entries].numpy(),
+                                  q[0].numpy(), w[0].numpy())
+    assert H.near_tie_only(ref[0], orc.topk64(s64, wl.topk), s64)
