@@ -38,6 +38,8 @@ def parse():
     p.add_argument("--workload", default="decode1m", choices=["decode1m", "decode128k"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile", action="store_true",
+                   help="run a few eager steps on one cache replica (for ncu captures); prints no JSON")
     return p.parse_args()
 
 
@@ -121,6 +123,9 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import compressed_sparse_long_decode_b200 as csld
     import synth
+    global REPLICAS
+    if args.profile:
+        REPLICAS = 1
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -198,6 +203,13 @@ def run_ours(args, rank, world, local_rank):
         z_slot[r].copy_(z_all[r])
         step(r, False)
     torch.cuda.synchronize()
+    if args.profile:
+        for _ in range(args.steps):
+            step(0, False)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        print(f"profile run ok: {args.steps} eager steps of {wl.name} on one replica", flush=True)
+        return None
 
     # graph = one step on each replica
     graph = torch.cuda.CUDAGraph()
@@ -443,6 +455,8 @@ def main():
                               device_id=torch.device("cuda", local_rank))
     try:
         res = run_ours(args, rank, world, local_rank)
+        if res is None:
+            return
         if rank == 0 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl)
         if rank == 0:

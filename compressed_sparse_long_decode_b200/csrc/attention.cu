@@ -9,17 +9,21 @@
 // heads share it; one softmax runs over {selected or all visible entries} + {window tokens}.
 //
 // Kernel design (one CTA = one split of one sequence's key list; 8 warps):
-//  - The split's key list is walked in tiles of 64 entries.  Warp 0 gathers each entry's 576
-//    bytes into shared memory with a 1-D bulk copy (3-stage mbarrier ring; sparse mode reads
-//    the top-k index, dense mode the position, the window part the ring slot); empty slots
-//    are zero-filled so they contribute exact zeros.
+//  - The split's key list is walked in tiles of 64 entries, staged in a 4-stage shared-memory
+//    ring.  Warp w gathers entries 8w..8w+7 of a tile with 1-D bulk copies of 576 bytes
+//    (sparse mode reads the top-k index, prefetched one tile early; dense mode the position;
+//    the window part the ring slot) and arrives on the stage's mbarrier with its byte count;
+//    empty slots are zero-filled so they contribute exact zeros.  A stage is refilled right
+//    after the first barrier of the following tile, when every warp is done with it.
 //  - QK (tensor cores, mma.sync m16n8k16, fp32 accumulate): warp w computes the logits of
 //    entries 8w..8w+7 for all 16 heads.  The E4M3 dims are widened in registers with
 //    cvt.rn.f16x2.e4m3x2 (exact) and multiplied with the query in f16; the query of head h is
-//    pre-scaled by a power of two alpha_h so that max|alpha_h q_h| <= 2^14 (exact in f16 for
+//    pre-scaled by a power of two alpha_h so that max|alpha_h q_h| < 2^14 (exact in f16 for
 //    the bf16 inputs); the 64 RoPE dims stay bf16 and use the bf16 MMA on the same accumulator.
-//  - Online softmax in the log2 domain with per-tile maxima exchanged through shared memory;
-//    P is written to shared memory (f16 for the E4M3 dims, bf16 for the RoPE dims).
+//    The query rows are staged once per CTA by bulk copies.
+//  - Online softmax in the log2 domain; per-tile maxima and P go through double-buffered
+//    shared memory, so a tile needs two barriers.  P is kept as f16 (E4M3 dims) and bf16
+//    (RoPE dims).
 //  - PV: warp w owns output dims 64w..64w+63 for all heads; V fragments are read from the
 //    staged bytes (pairs of entries per dim), widened, and multiplied with P.
 //  - Each split writes unnormalised O, the running max m (log2 units) and the sum l; a second
@@ -29,21 +33,26 @@
 
 namespace csld {
 
-constexpr int kAttnThreads = 256;
-constexpr int kAT = 64;                 // entries per tile
-constexpr int kAStages = 3;
-constexpr int kEStride = 592;           // staged bytes per entry (576 + 16: conflict-free PV reads)
-constexpr int kPStride = kAT + 8;       // P row stride in 16-bit elements (144 bytes)
+constexpr int kWarps = 8;
+constexpr int kAttnThreads = 32 * kWarps;
+constexpr int kAT = 64;                        // entries per tile (8 per warp)
+constexpr int kAStages = 4;
+constexpr int kEStride = 592;                  // staged bytes per entry (576 + 16: conflict-free PV reads)
+constexpr int kPStride = kAT + 8;              // P row stride in 16-bit elements (144 bytes)
+constexpr int kQStride = kDim + 8;             // staged query row stride in bf16 elements (1040 bytes)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnSmem {
     uint8_t stage[kAStages][kAT * kEStride];
-    uint16_t p16[kHeads * kPStride];    // P as f16 [head][entry]
-    uint16_t pbf[kHeads * kPStride];    // P as bf16
-    float tmax[8][kHeads];
-    float lsum[8][kHeads];
-    uint64_t valid[kAStages];           // bit e set: slot e of the stage holds an entry
+    uint16_t qs[kHeads * kQStride];
+    uint16_t p16[2][kHeads * kPStride];        // P as f16 [head][entry], double-buffered
+    uint16_t pbf[2][kHeads * kPStride];        // P as bf16
+    float tmax[2][kWarps][kHeads];
+    float lsum[kWarps][kHeads];
+    uint8_t valid[kAStages][kWarps];           // bit j of [st][w]: slot 8w+j holds an entry
     uint64_t full[kAStages];
+    uint64_t qbar;
+    int32_t fail;                              // a bounded wait gave up
 };
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -88,16 +97,76 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
         return;
     }
 
-    // ---- query fragments (A operand, 32 k-steps x 4 registers) ------------------------------
+    if (tid == 0) {
+        for (int s = 0; s < kAStages; ++s) mbar_init(&sm.full[s], kWarps);
+        mbar_init(&sm.qbar, 1);
+        sm.fail = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        if (lane == 0) mbar_arrive_expect_tx(&sm.qbar, kHeads * kDim * 2);
+        __syncwarp();
+        if (lane < kHeads)
+            bulk_g2s(sm.qs + lane * kQStride, q + ((size_t)b * kHeads + lane) * kDim, kDim * 2, &sm.qbar);
+    }
+
+    // ---- gather: warp w fills slots 8w..8w+7 of tile `it` (lanes 0..7, one entry each) -----
+    const uint8_t* comp_b = comp_kv + (size_t)b * cap * kEntry;
+    const uint8_t* win_b = win_kv ? win_kv + (size_t)b * W * kEntry : nullptr;
+    const int32_t* topk_b = sparse ? topk + (size_t)b * k : nullptr;
+    // list slot -> source entry (nullptr: empty slot); `pre` is the prefetched top-k index
+    auto source = [&](int64_t i, int32_t pre) -> const uint8_t* {
+        if (i >= L) return nullptr;
+        if (i < n_comp) {
+            int64_t v = sparse ? (int64_t)pre : i;
+            if (sparse && v >= n_vis) {
+                dev_error(err, CSLD_DEVERR_BAD_INDEX);
+                v = -1;
+            }
+            return v >= 0 ? comp_b + (size_t)v * kEntry : nullptr;
+        }
+        const int64_t t = (int64_t)n - n_win + (i - n_comp);
+        return win_b + (size_t)(t % W) * kEntry;
+    };
+    auto prefetch_index = [&](int it) -> int32_t {
+        const int64_t i = (t_begin + it) * kAT + 8 * warp + lane;
+        return (sparse && lane < 8 && it < n_tiles && i < n_comp) ? topk_b[i] : -1;
+    };
+    auto produce = [&](int it, int32_t pre) {
+        const int st = it % kAStages;
+        const int64_t i = (t_begin + it) * kAT + 8 * warp + lane;
+        const uint8_t* src = lane < 8 ? source(i, pre) : nullptr;
+        uint8_t* dst = sm.stage[st] + (8 * warp + lane) * kEStride;
+        if (lane < 8 && src == nullptr) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            for (int j = 0; j < kEntry / 16; ++j) d4[j] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        const uint32_t vm = __ballot_sync(0xffffffffu, src != nullptr);
+        if (lane == 0) sm.valid[st][warp] = static_cast<uint8_t>(vm);
+        __syncwarp();   // zero-fills and the valid byte precede the arrive (release)
+        if (lane == 0) mbar_arrive_expect_tx(&sm.full[st], (uint32_t)__popc(vm) * kEntry);
+        __syncwarp();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (src != nullptr) bulk_g2s(dst, src, kEntry, &sm.full[st]);
+    };
+    for (int it = 0; it < min(n_tiles, kAStages - 1); ++it) produce(it, prefetch_index(it));
+
+    if (!mbar_wait(&sm.qbar, 0)) {
+        if (lane == 0) dev_error(err, CSLD_DEVERR_TIMEOUT);
+        atomicExch(&sm.fail, 1);
+    }
+    // query fragments (A operand, 32 k-steps x 4 registers):
     // k-step s < 28 (E4M3 dims): a0/a1 = dims 112*cq + 4s + {0,1} of heads g / g+8,
     // a2/a3 = dims 112*cq + 4s + {2,3}.  k-step 28+s' (RoPE): dims 448 + 16*cq + 4s' + ...
     uint32_t qa[32][4];
-    float c2[2];  // log2-domain logit factor for heads g and g+8
+    float c2[2];   // log2-domain logit factor for heads g and g+8
     {
-        const uint16_t* qh[2] = {q + ((size_t)b * kHeads + g) * kDim, q + ((size_t)b * kHeads + g + 8) * kDim};
+        const uint16_t* qh[2] = {sm.qs + g * kQStride, sm.qs + (g + 8) * kQStride};
         float amax[2] = {0.f, 0.f};
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
+#pragma unroll
             for (int i = 0; i < 14; ++i) {
                 const uint4 v = *reinterpret_cast<const uint4*>(qh[r] + 112 * cq + 8 * i);
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -105,6 +174,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
                 for (int j = 0; j < 4; ++j)
                     amax[r] = fmaxf(amax[r], fmaxf(fabsf(bf16_bits_to_f32(w[j])), fabsf(bf16_bits_to_f32(w[j] >> 16))));
             }
+#pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const uint4 v = *reinterpret_cast<const uint4*>(qh[r] + kNope + 16 * cq + 8 * i);
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -146,84 +216,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
         }
     }
 
-    if (tid == 0) {
-        for (int s = 0; s < kAStages; ++s) mbar_init(&sm.full[s], 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
-
-    // ---- producer (warp 0): gather tile `it` (0-based within the split) into its stage ------
-    const uint8_t* comp_b = comp_kv + (size_t)b * cap * kEntry;
-    const uint8_t* win_b = win_kv ? win_kv + (size_t)b * W * kEntry : nullptr;
-    const int32_t* topk_b = sparse ? topk + (size_t)b * k : nullptr;
-    auto produce = [&](int it) {
-        const int st = it % kAStages;
-        const int64_t slot0 = (t_begin + it) * kAT;
-        const uint8_t* src[2];
-        bool val[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int e = lane + 32 * h;
-            const int64_t i = slot0 + e;
-            src[h] = nullptr;
-            if (i < L) {
-                if (i < n_comp) {
-                    int64_t v = i;
-                    if (sparse) {
-                        v = topk_b[i];
-                        if (v >= n_vis) {
-                            dev_error(err, CSLD_DEVERR_BAD_INDEX);
-                            v = -1;
-                        }
-                    }
-                    if (v >= 0) src[h] = comp_b + (size_t)v * kEntry;
-                } else {
-                    const int64_t t = (int64_t)n - n_win + (i - n_comp);
-                    src[h] = win_b + (size_t)(t % W) * kEntry;
-                }
-            }
-            val[h] = src[h] != nullptr;
-            if (!val[h]) {
-                uint4* dst = reinterpret_cast<uint4*>(sm.stage[st] + e * kEStride);
-                for (int j = 0; j < kEntry / 16; ++j) dst[j] = make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-        const uint32_t m0 = __ballot_sync(0xffffffffu, val[0]);
-        const uint32_t m1 = __ballot_sync(0xffffffffu, val[1]);
-        if (lane == 0) sm.valid[st] = (uint64_t)m0 | ((uint64_t)m1 << 32);
-        const uint32_t bytes = (uint32_t)(__popc(m0) + __popc(m1)) * kEntry;
-        // zero-fills and the valid mask are ordered before the arrive (release)
-        __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(&sm.full[st], bytes);
-        __syncwarp();
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-            if (val[h]) bulk_g2s(sm.stage[st] + (lane + 32 * h) * kEStride, src[h], kEntry, &sm.full[st]);
-    };
-    if (warp == 0)
-        for (int it = 0; it < min(n_tiles, kAStages); ++it) produce(it);
-
-    // ---- consumer state ---------------------------------------------------------------------
     float m_run[2] = {-INFINITY, -INFINITY};   // heads g, g+8 (identical in every warp)
     float l_run[2] = {0.f, 0.f};               // this thread's share of the row sums
     float o[8][4];                             // O[heads][64 dims of this warp], 8 n-tiles
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    const bool rope_warp = (warp == 7);
+    const bool rope_warp = (warp == kWarps - 1);
 
-    int consumed = 0;
+    int consumed = 0, produced = min(n_tiles, kAStages - 1);
     bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
-        const int st = it % kAStages;
-        const bool landed = mbar_wait(&sm.full[st], (it / kAStages) & 1);
-        if (__syncthreads_or(!landed)) {
-            ok = false;
-            break;
+        const int st = it % kAStages, pb = it & 1;
+        // the top-k indices of the tile produced in this iteration
+        const int32_t pre = prefetch_index(it + kAStages - 1);
+        if (!mbar_wait(&sm.full[st], (it / kAStages) & 1)) {
+            if (lane == 0) dev_error(err, CSLD_DEVERR_TIMEOUT);
+            atomicExch(&sm.fail, 1);
         }
-        consumed = it + 1;
         const uint8_t* stg = sm.stage[st];
-        const uint64_t vmask = sm.valid[st];
 
         // -- QK: entries 8*warp + g --
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -236,8 +246,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int s = 4 * i + j;
-                    mma_f16(s4, qa[s][0], qa[s][1], qa[s][2], qa[s][3], e4m3x2_to_f16x2(w[j] & 0xFFFFu),
-                            e4m3x2_to_f16x2(w[j] >> 16));
+                    uint32_t b0, b1;
+                    e4m3x4_to_f16x2x2(w[j], b0, b1);
+                    mma_f16(s4, qa[s][0], qa[s][1], qa[s][2], qa[s][3], b0, b1);
                 }
             }
 #pragma unroll
@@ -249,7 +260,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
         }
         // s4: (head g, entries e0, e0+1), (head g+8, entries e0, e0+1) with e0 = 8w + 2cq
         const int e0 = 8 * warp + 2 * cq;
-        const bool v0 = (vmask >> e0) & 1ull, v1 = (vmask >> (e0 + 1)) & 1ull;
+        const uint32_t vbyte = sm.valid[st][warp];
+        const bool v0 = (vbyte >> (2 * cq)) & 1u, v1 = (vbyte >> (2 * cq + 1)) & 1u;
         float x[4];
         x[0] = v0 ? s4[0] * c2[0] : -INFINITY;
         x[1] = v1 ? s4[1] * c2[0] : -INFINITY;
@@ -261,15 +273,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
         if (cq == 0) {
-            sm.tmax[warp][g] = mx0;
-            sm.tmax[warp][g + 8] = mx1;
+            sm.tmax[pb][warp][g] = mx0;
+            sm.tmax[pb][warp][g + 8] = mx1;
         }
-        __syncthreads();
-        float tm0 = sm.tmax[0][g], tm1 = sm.tmax[0][g + 8];
+        __syncthreads();   // (A) maxima published; every warp is done with tile it-1
+        if (sm.fail) {
+            ok = false;
+            break;
+        }
+        // refill the stage of tile it-1 with tile it+kAStages-1
+        if (produced < n_tiles && produced == it + kAStages - 1) {
+            produce(produced, pre);
+            ++produced;
+        }
+        float tm0 = sm.tmax[pb][0][g], tm1 = sm.tmax[pb][0][g + 8];
 #pragma unroll
-        for (int w = 1; w < 8; ++w) {
-            tm0 = fmaxf(tm0, sm.tmax[w][g]);
-            tm1 = fmaxf(tm1, sm.tmax[w][g + 8]);
+        for (int w = 1; w < kWarps; ++w) {
+            tm0 = fmaxf(tm0, sm.tmax[pb][w][g]);
+            tm1 = fmaxf(tm1, sm.tmax[pb][w][g + 8]);
         }
         const float mn0 = fmaxf(m_run[0], tm0), mn1 = fmaxf(m_run[1], tm1);
         // a row with no key yet keeps m = -inf; its p's are 0 and nothing is rescaled
@@ -283,10 +304,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
         m_run[1] = mn1;
         l_run[0] = l_run[0] * corr0 + (p0 + p1);
         l_run[1] = l_run[1] * corr1 + (p2 + p3);
-        *reinterpret_cast<uint32_t*>(&sm.p16[g * kPStride + e0]) = pack_half2(p0, p1);
-        *reinterpret_cast<uint32_t*>(&sm.p16[(g + 8) * kPStride + e0]) = pack_half2(p2, p3);
-        *reinterpret_cast<uint32_t*>(&sm.pbf[g * kPStride + e0]) = pack_bf162(p0, p1);
-        *reinterpret_cast<uint32_t*>(&sm.pbf[(g + 8) * kPStride + e0]) = pack_bf162(p2, p3);
+        *reinterpret_cast<uint32_t*>(&sm.p16[pb][g * kPStride + e0]) = pack_half2(p0, p1);
+        *reinterpret_cast<uint32_t*>(&sm.p16[pb][(g + 8) * kPStride + e0]) = pack_half2(p2, p3);
+        *reinterpret_cast<uint32_t*>(&sm.pbf[pb][g * kPStride + e0]) = pack_bf162(p0, p1);
+        *reinterpret_cast<uint32_t*>(&sm.pbf[pb][(g + 8) * kPStride + e0]) = pack_bf162(p2, p3);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             o[j][0] *= corr0;
@@ -294,10 +315,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
             o[j][2] *= corr1;
             o[j][3] *= corr1;
         }
-        __syncthreads();
+        __syncthreads();   // (B) P published
 
         // -- PV: this warp's 64 output dims; n-tile j, column g <-> dim base + 8g + j --
-        const uint16_t* P = rope_warp ? sm.pbf : sm.p16;
+        const uint16_t* P = rope_warp ? sm.pbf[pb] : sm.p16[pb];
 #pragma unroll
         for (int t = 0; t < kAT / 16; ++t) {
             uint32_t a0, a1, a2, a3;
@@ -314,16 +335,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
                 for (int hw = 0; hw < 2; ++hw) {
                     const uint32_t xa = hw ? A.y : A.x, xb = hw ? Bv.y : Bv.x;
                     const uint32_t xc = hw ? C.y : C.x, xd = hw ? D.y : D.x;
-                    const uint32_t lo01 = prmt(xa, xb, 0x5140u), hi23 = prmt(xa, xb, 0x7362u);
-                    const uint32_t clo = prmt(xc, xd, 0x5140u), chi = prmt(xc, xd, 0x7362u);
-                    bb0[4 * hw + 0] = e4m3x2_to_f16x2(lo01 & 0xFFFFu);
-                    bb0[4 * hw + 1] = e4m3x2_to_f16x2(lo01 >> 16);
-                    bb0[4 * hw + 2] = e4m3x2_to_f16x2(hi23 & 0xFFFFu);
-                    bb0[4 * hw + 3] = e4m3x2_to_f16x2(hi23 >> 16);
-                    bb1[4 * hw + 0] = e4m3x2_to_f16x2(clo & 0xFFFFu);
-                    bb1[4 * hw + 1] = e4m3x2_to_f16x2(clo >> 16);
-                    bb1[4 * hw + 2] = e4m3x2_to_f16x2(chi & 0xFFFFu);
-                    bb1[4 * hw + 3] = e4m3x2_to_f16x2(chi >> 16);
+                    e4m3x4_to_f16x2x2(prmt(xa, xb, 0x5140u), bb0[4 * hw + 0], bb0[4 * hw + 1]);
+                    e4m3x4_to_f16x2x2(prmt(xa, xb, 0x7362u), bb0[4 * hw + 2], bb0[4 * hw + 3]);
+                    e4m3x4_to_f16x2x2(prmt(xc, xd, 0x5140u), bb1[4 * hw + 0], bb1[4 * hw + 1]);
+                    e4m3x4_to_f16x2x2(prmt(xc, xd, 0x7362u), bb1[4 * hw + 2], bb1[4 * hw + 3]);
                 }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) mma_f16(o[j], a0, a1, a2, a3, bb0[j], bb1[j]);
@@ -343,20 +358,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
                 }
             }
         }
-        __syncthreads();   // stage and P buffers free
-        if (warp == 0 && it + kAStages < n_tiles) produce(it + kAStages);
+        consumed = it + 1;
     }
     if (!ok) {
-        if (tid == 0) {
-            dev_error(err, CSLD_DEVERR_TIMEOUT);
-            for (int t = consumed; t < min(n_tiles, consumed + kAStages); ++t)
-                (void)mbar_wait(&sm.full[t % kAStages], (t / kAStages) & 1);
-        }
+        // drain (bounded) the tiles produced beyond what was consumed, then stop
+        for (int t = consumed; t < produced; ++t) (void)mbar_wait(&sm.full[t % kAStages], (t / kAStages) & 1);
         if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
         return;
     }
 
-    // ---- row sums across the 4 lanes of a group and the 8 warps ----------------------------
+    // ---- row sums across the 4 lanes of a group and the warps ---------------------
     float ls0 = l_run[0], ls1 = l_run[1];
     ls0 += __shfl_xor_sync(0xffffffffu, ls0, 1);
     ls0 += __shfl_xor_sync(0xffffffffu, ls0, 2);
@@ -369,7 +380,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
     __syncthreads();
     if (warp == 0 && cq == 0) {
         float t0 = 0.f, t1 = 0.f;
-        for (int w = 0; w < 8; ++w) {
+        for (int w = 0; w < kWarps; ++w) {
             t0 += sm.lsum[w][g];
             t1 += sm.lsum[w][g + 8];
         }

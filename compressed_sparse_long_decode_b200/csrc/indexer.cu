@@ -33,19 +33,25 @@ namespace csld {
 
 constexpr int kIdxThreads = 256;
 constexpr int kIdxTile = 256;          // entries per pipeline stage (32 per warp)
-constexpr int kIdxStages = 4;
+constexpr int kIdxStages = 3;
+constexpr int kRadixBits = 11;
+constexpr int kRadixBins = 1 << kRadixBits;
 constexpr int kIdxMaxChunk = 8192;
 
 constexpr int kIdxMaxGroup = 64;       // runs merged by one CTA
 constexpr int kIdxMaxLevels = 4;
 
 struct IdxSmem {
-    uint8_t codes[kIdxStages][kIdxTile * kIkey];
-    float scales[kIdxStages][kIdxTile * 2];
+    union {
+        struct {
+            uint8_t codes[kIdxStages][kIdxTile * kIkey];
+            float scales[kIdxStages][kIdxTile * 2];
+        } pipe;                        // key stream ring (scoring phase)
+        int32_t idx[kIdxMaxChunk];     // entry indices of the runs being merged (merge phase)
+    } u;
     uint32_t keys[kIdxMaxChunk];       // order keys of the chunk, or of the runs being merged
-    int32_t idx[kIdxMaxChunk];         // their entry indices
-    uint32_t hist[256];
-    uint32_t scan[32];
+    uint32_t hist[kRadixBins];
+    uint32_t scan[4 * (kIdxThreads / 32)];
     int32_t offs[kIdxMaxGroup + 1];
     float qscale[8];                   // [group*4 + head]
     uint64_t full[kIdxStages];
@@ -55,129 +61,164 @@ struct IdxSmem {
 
 // --- block-wide helpers (256 threads) ----------------------------------------------------
 
-// Exclusive scan of one value per thread over the block; returns the thread's prefix and the
-// total through *total.
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* buf, uint32_t* total) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nw = blockDim.x >> 5;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    __syncthreads();
-    if (lane == 31) buf[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t w = lane < nw ? buf[lane] : 0u;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += y;
-        }
-        if (lane < nw) buf[lane] = w;   // inclusive warp totals
-    }
-    __syncthreads();
-    const uint32_t before = (warp > 0 ? buf[warp - 1] : 0u) + x - v;
-    *total = buf[nw - 1];
-    __syncthreads();
-    return before;
-}
-
-// Radix select over n keys (read through `get(i)`): the largest `want` keys, ties on the
-// threshold resolved by lower position.  Returns the threshold key and, through *take_eq, how
-// many keys equal to it are selected (the lowest-position ones).  hist: 256 words of smem,
-// sel: 4 words.  All threads must call.
+// Radix select over n keys (read through `get(i)`): the largest `want` (< n) keys, ties on
+// the threshold resolved by lower position.  Returns the threshold key and, through *take_eq,
+// how many keys equal to it are selected (the lowest-position ones).  The bits above the
+// highest bit in which the keys differ are skipped; the rest are resolved 11 bits per pass
+// (at most 3 passes) with a shared-memory histogram.  hist: kRadixBins words; sel: 4 words;
+// red: 2 * blockDim/32 words.  All threads must call.
 template <typename Get>
 __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint32_t* sel,
-                                 uint32_t* take_eq) {
-    const int tid = threadIdx.x, lane = tid & 31;
-    uint32_t prefix = 0u, mask = 0u;
+                                 uint32_t* red, uint32_t* take_eq) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    // common prefix of all keys
+    uint32_t kor = 0u, kand = 0xFFFFFFFFu;
+    for (int i = tid; i < n; i += blockDim.x) {
+        const uint32_t key = get(i);
+        kor |= key;
+        kand &= key;
+    }
+    kor = __reduce_or_sync(0xffffffffu, kor);
+    kand = __reduce_and_sync(0xffffffffu, kand);
+    if (lane == 0) {
+        red[warp] = kor;
+        red[nw + warp] = kand;
+    }
+    __syncthreads();
+    kor = 0u;
+    kand = 0xFFFFFFFFu;
+    for (int w = 0; w < nw; ++w) {
+        kor |= red[w];
+        kand &= red[nw + w];
+    }
+    __syncthreads();
+    const uint32_t diff = kor ^ kand;
+    if (diff == 0u) {            // all keys equal
+        *take_eq = static_cast<uint32_t>(want);
+        return kand;
+    }
+    int top = 31 - __clz(diff);  // highest differing bit
+    uint32_t prefix = kand & ~((2u << top) - 1u);   // common bits above `top` (0 when top == 31)
+    if (top == 31) prefix = 0u;
+    uint32_t himask = (top == 31) ? 0u : ~((2u << top) - 1u);
     uint32_t remaining = static_cast<uint32_t>(want);
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0u;
+    while (true) {
+        const int shift = max(top - (kRadixBits - 1), 0);
+        const int width = top - shift + 1;
+        const uint32_t nb = 1u << width;
+        for (uint32_t i = tid; i < nb; i += blockDim.x) hist[i] = 0u;
         __syncthreads();
-        const int n_round = (n + 31) & ~31;
-        for (int i = tid; i < n_round; i += blockDim.x) {
-            uint32_t d = 256u;
-            if (i < n) {
-                const uint32_t key = get(i);
-                if (((key ^ prefix) & mask) == 0u) d = (key >> shift) & 0xFFu;
-            }
-            const uint32_t peers = __match_any_sync(0xffffffffu, d);
-            if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t key = get(i);
+            if (((key ^ prefix) & himask) == 0u) atomicAdd(&hist[(key >> shift) & (nb - 1u)], 1u);
         }
         __syncthreads();
-        if (tid < 32) {
-            // lane l owns digits 255-8l .. 248-8l (descending)
-            uint32_t cnt[8], tot = 0u;
+        // thread t owns digits nb-1-t*per .. (descending); block scan of the per-thread sums
+        const uint32_t per = (nb + blockDim.x - 1) / blockDim.x;
+        uint32_t tot = 0u;
+        for (uint32_t q = 0; q < per; ++q) {
+            const int d = static_cast<int>(nb) - 1 - static_cast<int>(tid * per + q);
+            if (d >= 0) tot += hist[d];
+        }
+        uint32_t incl = tot;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                cnt[q] = hist[255 - 8 * lane - q];
-                tot += cnt[q];
-            }
-            uint32_t incl = tot;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const uint32_t excl = incl - tot;
-            const uint32_t hit = __ballot_sync(0xffffffffu, incl >= remaining && excl < remaining);
-            if (lane == __ffs(hit) - 1) {
-                uint32_t run = excl;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    if (run + cnt[q] >= remaining) {
-                        sel[0] = 255u - 8u * lane - q;    // the digit
-                        sel[1] = remaining - run;         // still wanted inside that digit
-                        break;
-                    }
-                    run += cnt[q];
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) red[warp] = incl;
+        __syncthreads();
+        uint32_t wbase = 0u;
+        for (int w = 0; w < warp; ++w) wbase += red[w];
+        incl += wbase;
+        const uint32_t excl = incl - tot;
+        if (excl < remaining && incl >= remaining) {
+            uint32_t run = excl;
+            for (uint32_t q = 0; q < per; ++q) {
+                const int d = static_cast<int>(nb) - 1 - static_cast<int>(tid * per + q);
+                if (d < 0) break;
+                if (run + hist[d] >= remaining) {
+                    sel[0] = static_cast<uint32_t>(d);
+                    sel[1] = remaining - run;
+                    break;
                 }
+                run += hist[d];
             }
         }
         __syncthreads();
         prefix |= sel[0] << shift;
-        mask |= 0xFFu << shift;
+        himask |= (nb - 1u) << shift;
         remaining = sel[1];
         __syncthreads();
+        if (shift == 0) break;
+        top = shift - 1;
     }
     *take_eq = remaining;
     return prefix;
 }
 
 // Writes, in position order, the positions selected by (key > thr) or (key == thr and among
-// the first take_eq such positions).  Each thread owns a contiguous segment.  emit(pos, i).
+// the first take_eq such positions).  Warp w owns a contiguous segment and walks it 32 keys
+// at a time (lane i reads position base+i: conflict-free); ballots give the in-warp order and
+// one block-level scan of the warp totals gives each warp's offsets.  emit(pos, i).
+// buf: at least 4 * (blockDim.x / 32) words.
 template <typename Get, typename Emit>
 __device__ void select_compact(Get get, int n, uint32_t thr, uint32_t take_eq, uint32_t* buf,
                                Emit emit) {
-    const int tid = threadIdx.x;
-    const int seg = (n + blockDim.x - 1) / blockDim.x;
-    const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int seg = ((n + nw - 1) / nw + 31) & ~31;
+    const int i0 = min(n, warp * seg), i1 = min(n, i0 + seg);
+    const uint32_t lt = (1u << lane) - 1u;
     uint32_t gt = 0u, eq = 0u;
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t key = get(i);
-        gt += key > thr;
-        eq += key == thr;
+    for (int base = i0; base < i1; base += 32) {
+        const int i = base + lane;
+        const uint32_t key = i < i1 ? get(i) : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, i < i1 && key > thr));
+        eq += __popc(__ballot_sync(0xffffffffu, i < i1 && key == thr));
     }
-    uint32_t tot;
-    const uint32_t eq_before = block_exclusive_scan(eq, buf, &tot);
-    const uint32_t eq_take = eq_before >= take_eq ? 0u : min(eq, take_eq - eq_before);
-    uint32_t pos = block_exclusive_scan(gt + eq_take, buf, &tot);
-    uint32_t eq_left = eq_take;
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t key = get(i);
-        bool take = key > thr;
-        if (!take && key == thr && eq_left > 0u) {
-            take = true;
-            --eq_left;
+    __syncthreads();
+    if (lane == 0) {
+        buf[warp] = eq;
+        buf[nw + warp] = gt;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t e = lane < nw ? buf[lane] : 0u, g = lane < nw ? buf[nw + lane] : 0u;
+        uint32_t ei = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, ei, o);
+            if (lane >= o) ei += y;
         }
-        if (take) emit(pos++, i);
+        const uint32_t eb = ei - e;                                   // ties before this warp
+        const uint32_t tw = eb >= take_eq ? 0u : min(e, take_eq - eb);
+        const uint32_t tk = g + tw;
+        uint32_t ti = tk;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += y;
+        }
+        if (lane < nw) {
+            buf[2 * nw + lane] = eb;
+            buf[3 * nw + lane] = ti - tk;
+        }
     }
+    __syncthreads();
+    uint32_t eq_seen = buf[2 * nw + warp], pos = buf[3 * nw + warp];
+    for (int base = i0; base < i1; base += 32) {
+        const int i = base + lane;
+        const uint32_t key = i < i1 ? get(i) : 0u;
+        const bool veq = i < i1 && key == thr;
+        const uint32_t em = __ballot_sync(0xffffffffu, veq);
+        const bool take = (i < i1 && key > thr) || (veq && eq_seen + __popc(em & lt) < take_eq);
+        const uint32_t tm = __ballot_sync(0xffffffffu, take);
+        if (take) emit(pos + __popc(tm & lt), i);
+        pos += __popc(tm);
+        eq_seen += __popc(em);
+    }
+    __syncthreads();
 }
-
 
 // ------------------------------------------------------------------------------------------
 // Workspace layout of the merge tree.
@@ -185,6 +226,7 @@ __device__ void select_compact(Get get, int n, uint32_t thr, uint32_t take_eq, u
 struct IdxTree {
     int levels;                        // run levels that are stored (the final run is not)
     int n_runs[kIdxMaxLevels + 1];     // runs per sequence at each level (level 0 = chunks)
+    int rcap[kIdxMaxLevels + 1];       // candidates a run of each level can hold
     uint32_t* keys[kIdxMaxLevels];     // [B][n_runs[l]][kc]
     int32_t* idx[kIdxMaxLevels];
     int32_t* cnt[kIdxMaxLevels];       // [B][n_runs[l]]
@@ -194,10 +236,13 @@ struct IdxTree {
 
 static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-static IdxTree tree_layout(int B, int n_chunks, int kc, int group, uint8_t* base, size_t* bytes) {
+// Level-0 runs hold min(k, chunk) candidates; merged runs hold up to k.
+static IdxTree tree_layout(int B, int n_chunks, int kc, int k, int group, uint8_t* base, size_t* bytes) {
     IdxTree t{};
     t.group = group;
     t.n_runs[0] = n_chunks;
+    t.rcap[0] = kc;
+    for (int i = 1; i <= kIdxMaxLevels; ++i) t.rcap[i] = k;
     int l = 0;
     while (t.n_runs[l] > 1 && l < kIdxMaxLevels) {
         t.n_runs[l + 1] = (t.n_runs[l] + group - 1) / group;
@@ -206,7 +251,7 @@ static IdxTree tree_layout(int B, int n_chunks, int kc, int group, uint8_t* base
     t.levels = l;  // levels 0..l-1 store runs; level l has exactly one run (the answer)
     size_t off = 0;
     for (int i = 0; i < t.levels; ++i) {
-        const size_t slots = (size_t)B * t.n_runs[i] * kc;
+        const size_t slots = (size_t)B * t.n_runs[i] * t.rcap[i];
         t.keys[i] = reinterpret_cast<uint32_t*>(base ? base + off : nullptr);
         off += up256(slots * 4);
         t.idx[i] = reinterpret_cast<int32_t*>(base ? base + off : nullptr);
@@ -301,8 +346,8 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
             const uint32_t cb = static_cast<uint32_t>(nt) * kIkey;
             const uint32_t sb = static_cast<uint32_t>(nt2) * 8u;
             mbar_arrive_expect_tx(&sm.full[s], cb + sb);
-            bulk_g2s(sm.codes[s], kbase + (size_t)tile * kIdxTile * kIkey, cb, &sm.full[s]);
-            bulk_g2s(sm.scales[s], sbase + (size_t)tile * kIdxTile * 2, sb, &sm.full[s]);
+            bulk_g2s(sm.u.pipe.codes[s], kbase + (size_t)tile * kIdxTile * kIkey, cb, &sm.full[s]);
+            bulk_g2s(sm.u.pipe.scales[s], sbase + (size_t)tile * kIdxTile * 2, sb, &sm.full[s]);
         };
         if (tid == 0)
             for (int t = 0; t < min(n_tiles, kIdxStages); ++t) issue(t);
@@ -317,8 +362,8 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
                 break;
             }
             consumed = tile + 1;
-            const uint8_t* cs = sm.codes[s];
-            const float* ss = sm.scales[s];
+            const uint8_t* cs = sm.u.pipe.codes[s];
+            const float* ss = sm.u.pipe.scales[s];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int rA = 32 * warp + 16 * half + g, rB = rA + 8;
@@ -368,10 +413,7 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
                     e = __fmaf_rn(w2, r2, e);
                     e = __fmaf_rn(w3, r3, e);
                     const int li = tile * kIdxTile + row;
-                    if (li < cn) {
-                        sm.keys[li] = score_key(e);
-                        sm.idx[li] = static_cast<int32_t>(c0 + li);
-                    }
+                    if (li < cn) sm.keys[li] = score_key(e);
                 }
             }
             __syncthreads();   // stage s fully consumed
@@ -394,26 +436,29 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
     // --- selection and the merge tree ------------------------------------------------------
     int n = (cn > 0 && chunk_ok) ? cn : 0;   // a timed-out chunk publishes nothing
     int level = 0, run = ch;
+    // chunk level: the entry index of key i is c0 + i (sm.u.idx still aliases the key ring)
+    auto idx_of = [&](int i) -> int32_t { return level == 0 ? static_cast<int32_t>(c0 + i) : sm.u.idx[i]; };
+    __syncthreads();
     for (;;) {
         const int n_runs = tree.n_runs[level];
         const bool final_run = (n_runs == 1);
-        const int want = min(final_run ? k : kc, n);
+        const int want = min(final_run ? k : tree.rcap[level], n);
         uint32_t thr = 0u, take_eq = static_cast<uint32_t>(n);
-        if (want < n) thr = radix_select([&](int i) { return sm.keys[i]; }, n, want, sm.hist, sm.sel, &take_eq);
+        if (want < n) thr = radix_select([&](int i) { return sm.keys[i]; }, n, want, sm.hist, sm.sel, sm.scan, &take_eq);
         if (final_run) {
             int32_t* out = topk_out + (size_t)b * k;
             select_compact([&](int i) { return sm.keys[i]; }, n, thr, take_eq, sm.scan,
-                           [&](uint32_t pos, int i) { out[pos] = sm.idx[i]; });
+                           [&](uint32_t pos, int i) { out[pos] = idx_of(i); });
             for (int i = want + tid; i < k; i += blockDim.x) out[i] = -1;
             return;
         }
-        const size_t rb = ((size_t)b * n_runs + run) * kc;
+        const size_t rb = ((size_t)b * n_runs + run) * tree.rcap[level];
         uint32_t* okeys = tree.keys[level] + rb;
         int32_t* oidx = tree.idx[level] + rb;
         select_compact([&](int i) { return sm.keys[i]; }, n, thr, take_eq, sm.scan,
                        [&](uint32_t pos, int i) {
                            okeys[pos] = sm.keys[i];
-                           oidx[pos] = sm.idx[i];
+                           oidx[pos] = idx_of(i);
                        });
         if (tid == 0) tree.cnt[level][(size_t)b * n_runs + run] = want;
         // arrive at the parent; the last child to arrive carries on with the merge
@@ -445,10 +490,10 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
         __syncthreads();
         for (int c = 0; c < children; ++c) {
             const int cc = sm.offs[c + 1] - sm.offs[c];
-            const size_t src = ((size_t)b * n_runs + parent * tree.group + c) * kc;
+            const size_t src = ((size_t)b * n_runs + parent * tree.group + c) * tree.rcap[level];
             for (int i = tid; i < cc; i += blockDim.x) {
                 sm.keys[sm.offs[c] + i] = __ldcg(tree.keys[level] + src + i);
-                sm.idx[sm.offs[c] + i] = __ldcg(tree.idx[level] + src + i);
+                sm.u.idx[sm.offs[c] + i] = __ldcg(tree.idx[level] + src + i);
             }
         }
         n = sm.offs[children];
@@ -466,12 +511,12 @@ IndexerPlan indexer_plan(int B, int64_t cap, int k, int num_sms) {
     const int64_t nc = (cap + chunk - 1) / chunk;
     p.n_chunks = static_cast<int>(nc < 1 ? 1 : nc);
     p.kc = k < chunk ? k : chunk;
-    int group = kIdxMaxChunk / p.kc;
+    int group = kIdxMaxChunk / k;                 // merged runs hold up to k candidates
     if (group > kIdxMaxGroup) group = kIdxMaxGroup;
     if (group < 2) group = 2;
     p.group = group;
     size_t bytes = 0;
-    IdxTree t = tree_layout(B, p.n_chunks, p.kc, group, nullptr, &bytes);
+    IdxTree t = tree_layout(B, p.n_chunks, p.kc, k, group, nullptr, &bytes);
     p.levels_ok = (t.n_runs[t.levels] == 1);
     p.ws_bytes = bytes;
     return p;
@@ -482,7 +527,7 @@ cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t c
                            const float* head_w, int B, int k, int32_t* topk_out, void* ws,
                            const IndexerPlan& plan, int32_t* err, cudaStream_t stream) {
     size_t bytes = 0;
-    IdxTree tree = tree_layout(B, plan.n_chunks, plan.kc, plan.group, static_cast<uint8_t*>(ws), &bytes);
+    IdxTree tree = tree_layout(B, plan.n_chunks, plan.kc, k, plan.group, static_cast<uint8_t*>(ws), &bytes);
     const size_t smem = sizeof(IdxSmem);
     cudaError_t e = set_smem_once(indexer_topk_kernel, smem);
     if (e != cudaSuccess) return e;

@@ -1,9 +1,13 @@
 """End-to-end parity of the tiny single-layer-pair decode workload: 4080 prefill tokens then 16
 decode steps (each: append to the CSA and HCA layers, indexer top-k 128 on the CSA layer,
 sparse CSA attention and dense HCA attention, both with a 128-token window), ending at 4096
-tokens = 1024 CSA and 32 HCA entries.  Each stage is also checked on identical input bytes:
-the GPU indexer on the oracle's keys must reproduce the oracle's selection bit for bit, and
-the GPU attention on the oracle's cache must match the oracle's output."""
+tokens = 1024 CSA and 32 HCA entries.  Each stage is checked on identical input bytes: the
+GPU indexer on the oracle's keys must reproduce the oracle's selection bit for bit, and the
+GPU attention on the oracle's cache and selection must match the oracle's output.  On each
+side's own state, the HCA output is compared at every step; the CSA output is compared
+whenever both sides selected the same entries -- GPU and oracle keys may differ by one FP4
+step (the key tolerance), which can legitimately move an entry across the top-k boundary,
+so there the selections are only required to overlap almost entirely."""
 import math
 
 import numpy as np
@@ -64,9 +68,10 @@ def test_tiny_decode_workload(csld, orc):
         ro_csa, rl_csa = orc.attention_batch(qb, ocsa.comp_kv, 4, osel, ocsa.win_kv, ocsa.seq_len, SCALE)
         ro_hca, rl_hca = orc.attention_batch(qb, ohca.comp_kv, 128, None, ohca.win_kv, ohca.seq_len, SCALE)
         H.assert_attention_close(o_hca.cpu().numpy(), l_hca.cpu().numpy(), ro_hca, rl_hca, f"HCA step {step}")
-        H.assert_attention_close(o_csa.cpu().numpy(), l_csa.cpu().numpy(), ro_csa, rl_csa, f"CSA step {step}")
         gsel = sel.cpu().numpy()
         overlap.append(len(set(gsel[0]) & set(osel[0])) / k)
+        if np.array_equal(gsel, osel):
+            H.assert_attention_close(o_csa.cpu().numpy(), l_csa.cpu().numpy(), ro_csa, rl_csa, f"CSA step {step}")
         # stage checks on identical bytes: the oracle's keys -> GPU indexer; the oracle's cache -> GPU attention
         sel_o = csld.indexer_topk(torch.from_numpy(ocsa.ikeys).cuda(), torch.from_numpy(ocsa.iscales).cuda(),
                                   torch.from_numpy(ocsa.seq_len).cuda(), 4, qs["q_idx"].cuda(),
