@@ -19,8 +19,9 @@
 //    entries 8w..8w+7 for all 16 heads.  The E4M3 dims are widened in registers with
 //    cvt.rn.f16x2.e4m3x2 (exact) and multiplied with the query in f16; the query of head h is
 //    pre-scaled by a power of two alpha_h so that max|alpha_h q_h| < 2^14 (exact in f16 for
-//    the bf16 inputs); the 64 RoPE dims stay bf16 and use the bf16 MMA on the same accumulator.
-//    The query rows are staged once per CTA by bulk copies.
+//    the bf16 inputs); the 64 RoPE dims stay bf16 and use the bf16 MMA on the same
+//    accumulators.  The query rows are staged once per CTA by bulk copies and converted once
+//    per CTA into shared memory.
 //  - Online softmax in the log2 domain; per-tile maxima and P go through double-buffered
 //    shared memory, so a tile needs two barriers.  P is kept as f16 (E4M3 dims) and bf16
 //    (RoPE dims).
@@ -40,11 +41,15 @@ constexpr int kAStages = 4;
 constexpr int kEStride = 592;                  // staged bytes per entry (576 + 16: conflict-free PV reads)
 constexpr int kPStride = kAT + 8;              // P row stride in 16-bit elements (144 bytes)
 constexpr int kQStride = kDim + 8;             // staged query row stride in bf16 elements (1040 bytes)
+constexpr int kQHStride = kNope + 8;           // f16 query row stride in elements (912 bytes)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnSmem {
     uint8_t stage[kAStages][kAT * kEStride];
     uint16_t qs[kHeads * kQStride];
+    uint16_t qf16[kHeads][kQHStride];          // alpha_h q_h of the 448 E4M3 dims, f16
+    uint16_t qrope[kHeads][kRope];             // alpha_h q_h of the RoPE dims, bf16
+    float c2[kHeads];                          // log2-domain logit factor per head
     uint16_t p16[2][kHeads * kPStride];        // P as f16 [head][entry], double-buffered
     uint16_t pbf[2][kHeads * kPStride];        // P as bf16
     float tmax[2][kWarps][kHeads];
@@ -112,31 +117,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
     }
 
     // ---- gather: warp w fills slots 8w..8w+7 of tile `it` (lanes 0..7, one entry each) -----
-    const uint8_t* comp_b = comp_kv + (size_t)b * cap * kEntry;
-    const uint8_t* win_b = win_kv ? win_kv + (size_t)b * W * kEntry : nullptr;
-    const int32_t* topk_b = sparse ? topk + (size_t)b * k : nullptr;
+    // Everything here is recomputed from the kernel parameters (constant bank) when needed, so
+    // the main loop does not hold the gather state in registers.
+    auto slot_of = [&](int it) -> int64_t {
+        const int64_t tiles = ((sparse ? (int64_t)k : min64(n / ratio, cap)) + (W > 0 ? min(W, n) : 0) + kAT - 1) / kAT;
+        return (tiles * blockIdx.x / splits + it) * kAT + 8 * warp + lane;
+    };
     // list slot -> source entry (nullptr: empty slot); `pre` is the prefetched top-k index
     auto source = [&](int64_t i, int32_t pre) -> const uint8_t* {
-        if (i >= L) return nullptr;
-        if (i < n_comp) {
+        const int64_t nv = min64(n / ratio, cap);
+        const int64_t nc = sparse ? (int64_t)k : nv;
+        const int nw = W > 0 ? min(W, n) : 0;
+        if (i >= nc + nw) return nullptr;
+        if (i < nc) {
             int64_t v = sparse ? (int64_t)pre : i;
-            if (sparse && v >= n_vis) {
+            if (sparse && v >= nv) {
                 dev_error(err, CSLD_DEVERR_BAD_INDEX);
                 v = -1;
             }
-            return v >= 0 ? comp_b + (size_t)v * kEntry : nullptr;
+            return v >= 0 ? comp_kv + ((size_t)blockIdx.y * cap + (size_t)v) * kEntry : nullptr;
         }
-        const int64_t t = (int64_t)n - n_win + (i - n_comp);
-        return win_b + (size_t)(t % W) * kEntry;
+        const int64_t t = (int64_t)n - nw + (i - nc);
+        return win_kv + ((size_t)blockIdx.y * W + (size_t)(t % W)) * kEntry;
     };
     auto prefetch_index = [&](int it) -> int32_t {
-        const int64_t i = (t_begin + it) * kAT + 8 * warp + lane;
-        return (sparse && lane < 8 && it < n_tiles && i < n_comp) ? topk_b[i] : -1;
+        const int64_t i = slot_of(it);
+        return (sparse && lane < 8 && it < n_tiles && i < k) ? topk[(size_t)blockIdx.y * k + i] : -1;
     };
     auto produce = [&](int it, int32_t pre) {
         const int st = it % kAStages;
-        const int64_t i = (t_begin + it) * kAT + 8 * warp + lane;
-        const uint8_t* src = lane < 8 ? source(i, pre) : nullptr;
+        const uint8_t* src = lane < 8 ? source(slot_of(it), pre) : nullptr;
         uint8_t* dst = sm.stage[st] + (8 * warp + lane) * kEStride;
         if (lane < 8 && src == nullptr) {
             uint4* d4 = reinterpret_cast<uint4*>(dst);
@@ -156,63 +166,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
         if (lane == 0) dev_error(err, CSLD_DEVERR_TIMEOUT);
         atomicExch(&sm.fail, 1);
     }
-    // query fragments (A operand, 32 k-steps x 4 registers):
-    // k-step s < 28 (E4M3 dims): a0/a1 = dims 112*cq + 4s + {0,1} of heads g / g+8,
-    // a2/a3 = dims 112*cq + 4s + {2,3}.  k-step 28+s' (RoPE): dims 448 + 16*cq + 4s' + ...
-    uint32_t qa[32][4];
-    float c2[2];   // log2-domain logit factor for heads g and g+8
+    // ---- the query, once per CTA: 16 threads per head, 32 consecutive dims each -----------
+    // alpha_h = 2^(14 - e) with max|q_h| < 2^e, so |alpha_h q_h| < 2^14: bf16 values scaled by a
+    // power of two are exact in f16 there (components below 2^-24 of that range flush).
     {
-        const uint16_t* qh[2] = {sm.qs + g * kQStride, sm.qs + (g + 8) * kQStride};
-        float amax[2] = {0.f, 0.f};
+        const int h = tid >> 4, d0 = (tid & 15) * 32;
+        const uint16_t* row = sm.qs + h * kQStride + d0;
+        float x[32];
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = *reinterpret_cast<const uint4*>(row + 8 * i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                x[8 * i + 2 * j] = bf16_bits_to_f32(w[j]);
+                x[8 * i + 2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        int e2 = 0;
+        if (amax > 0.f) frexpf(amax, &e2);          // amax < 2^e2
+        e2 = max(e2, -100);                         // keep alpha finite for tiny queries
+        const float alpha = ldexpf(1.f, 14 - e2);   // alpha * amax < 2^14
+        if ((tid & 15) == 0) sm.c2[h] = scale * kLog2e / alpha;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int d = d0 + 2 * i;
+            if (d < kNope)
+                *reinterpret_cast<uint32_t*>(&sm.qf16[h][d]) = pack_half2(alpha * x[2 * i], alpha * x[2 * i + 1]);
+            else
+                *reinterpret_cast<uint32_t*>(&sm.qrope[h][d - kNope]) = pack_bf162(alpha * x[2 * i], alpha * x[2 * i + 1]);
+        }
+    }
+    __syncthreads();
+    // fragments (A operand, 32 k-steps x 4 registers): k-step s < 28 (E4M3 dims): a0/a1 = dims
+    // 112*cq + 4s + {0,1} of heads g / g+8, a2/a3 = dims 112*cq + 4s + {2,3} (the key bytes a
+    // thread reads: its 112-byte slice).  k-step 28+s' (RoPE): dims 448 + 16*cq + 4s' + ...
+    uint32_t qa[32][4];
+    const float c2[2] = {sm.c2[g], sm.c2[g + 8]};
+#pragma unroll
+    for (int s = 0; s < 28; ++s) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-#pragma unroll
-            for (int i = 0; i < 14; ++i) {
-                const uint4 v = *reinterpret_cast<const uint4*>(qh[r] + 112 * cq + 8 * i);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    amax[r] = fmaxf(amax[r], fmaxf(fabsf(bf16_bits_to_f32(w[j])), fabsf(bf16_bits_to_f32(w[j] >> 16))));
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const uint4 v = *reinterpret_cast<const uint4*>(qh[r] + kNope + 16 * cq + 8 * i);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    amax[r] = fmaxf(amax[r], fmaxf(fabsf(bf16_bits_to_f32(w[j])), fabsf(bf16_bits_to_f32(w[j] >> 16))));
-            }
-            amax[r] = fmaxf(amax[r], __shfl_xor_sync(0xffffffffu, amax[r], 1));
-            amax[r] = fmaxf(amax[r], __shfl_xor_sync(0xffffffffu, amax[r], 2));
+            const uint2 v = *reinterpret_cast<const uint2*>(&sm.qf16[g + 8 * r][112 * cq + 4 * s]);
+            qa[s][r] = v.x;
+            qa[s][2 + r] = v.y;
         }
-        float alpha[2];
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-            int e2 = 0;
-            if (amax[r] > 0.f) frexpf(amax[r], &e2);      // amax < 2^e2
-            e2 = max(e2, -100);                           // keep alpha finite for tiny queries
-            alpha[r] = ldexpf(1.f, 14 - e2);              // alpha * amax < 2^14
-            c2[r] = scale * kLog2e / alpha[r];
-        }
-#pragma unroll
-        for (int s = 0; s < 28; ++s) {
-            const int d = 112 * cq + 4 * s;
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const uint2 v = *reinterpret_cast<const uint2*>(qh[r] + d);
-                qa[s][r] = pack_half2(alpha[r] * bf16_bits_to_f32(v.x), alpha[r] * bf16_bits_to_f32(v.x >> 16));
-                qa[s][2 + r] = pack_half2(alpha[r] * bf16_bits_to_f32(v.y), alpha[r] * bf16_bits_to_f32(v.y >> 16));
-            }
-        }
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int d = kNope + 16 * cq + 4 * s;
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const uint2 v = *reinterpret_cast<const uint2*>(qh[r] + d);
-                qa[28 + s][r] = pack_bf162(alpha[r] * bf16_bits_to_f32(v.x), alpha[r] * bf16_bits_to_f32(v.x >> 16));
-                qa[28 + s][2 + r] = pack_bf162(alpha[r] * bf16_bits_to_f32(v.y), alpha[r] * bf16_bits_to_f32(v.y >> 16));
-            }
+            const uint2 v = *reinterpret_cast<const uint2*>(&sm.qrope[g + 8 * r][16 * cq + 4 * s]);
+            qa[28 + s][r] = v.x;
+            qa[28 + s][2 + r] = v.y;
         }
     }
 
@@ -235,9 +246,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
         }
         const uint8_t* stg = sm.stage[st];
 
-        // -- QK: entries 8*warp + g --
+        // -- QK: entries 8*warp + g; two accumulators (even / odd k-steps) halve the MMA chain --
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
         {
+            float t4[4] = {0.f, 0.f, 0.f, 0.f};
             const uint8_t* ent = stg + (8 * warp + g) * kEStride;
 #pragma unroll
             for (int i = 0; i < 7; ++i) {
@@ -248,15 +260,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
                     const int s = 4 * i + j;
                     uint32_t b0, b1;
                     e4m3x4_to_f16x2x2(w[j], b0, b1);
-                    mma_f16(s4, qa[s][0], qa[s][1], qa[s][2], qa[s][3], b0, b1);
+                    if (j & 1) mma_f16(t4, qa[s][0], qa[s][1], qa[s][2], qa[s][3], b0, b1);
+                    else mma_f16(s4, qa[s][0], qa[s][1], qa[s][2], qa[s][3], b0, b1);
                 }
             }
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const uint4 v = *reinterpret_cast<const uint4*>(ent + kNope + 32 * cq + 16 * i);
                 mma_bf16(s4, qa[28 + 2 * i][0], qa[28 + 2 * i][1], qa[28 + 2 * i][2], qa[28 + 2 * i][3], v.x, v.y);
-                mma_bf16(s4, qa[29 + 2 * i][0], qa[29 + 2 * i][1], qa[29 + 2 * i][2], qa[29 + 2 * i][3], v.z, v.w);
+                mma_bf16(t4, qa[29 + 2 * i][0], qa[29 + 2 * i][1], qa[29 + 2 * i][2], qa[29 + 2 * i][3], v.z, v.w);
             }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) s4[r] += t4[r];
         }
         // s4: (head g, entries e0, e0+1), (head g+8, entries e0, e0+1) with e0 = 8w + 2cq
         const int e0 = 8 * warp + 2 * cq;
@@ -330,18 +345,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
                 const uint2 Bv = *reinterpret_cast<const uint2*>(stg + (ea + 1) * kEStride + off);
                 const uint2 C = *reinterpret_cast<const uint2*>(stg + (ea + 8) * kEStride + off);
                 const uint2 D = *reinterpret_cast<const uint2*>(stg + (ea + 9) * kEStride + off);
-                uint32_t bb0[8], bb1[8];
 #pragma unroll
-                for (int hw = 0; hw < 2; ++hw) {
+                for (int hw = 0; hw < 2; ++hw) {   // n-tiles 4hw .. 4hw+3
                     const uint32_t xa = hw ? A.y : A.x, xb = hw ? Bv.y : Bv.x;
                     const uint32_t xc = hw ? C.y : C.x, xd = hw ? D.y : D.x;
-                    e4m3x4_to_f16x2x2(prmt(xa, xb, 0x5140u), bb0[4 * hw + 0], bb0[4 * hw + 1]);
-                    e4m3x4_to_f16x2x2(prmt(xa, xb, 0x7362u), bb0[4 * hw + 2], bb0[4 * hw + 3]);
-                    e4m3x4_to_f16x2x2(prmt(xc, xd, 0x5140u), bb1[4 * hw + 0], bb1[4 * hw + 1]);
-                    e4m3x4_to_f16x2x2(prmt(xc, xd, 0x7362u), bb1[4 * hw + 2], bb1[4 * hw + 3]);
-                }
+                    uint32_t bb0[4], bb1[4];
+                    e4m3x4_to_f16x2x2(prmt(xa, xb, 0x5140u), bb0[0], bb0[1]);
+                    e4m3x4_to_f16x2x2(prmt(xa, xb, 0x7362u), bb0[2], bb0[3]);
+                    e4m3x4_to_f16x2x2(prmt(xc, xd, 0x5140u), bb1[0], bb1[1]);
+                    e4m3x4_to_f16x2x2(prmt(xc, xd, 0x7362u), bb1[2], bb1[3]);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) mma_f16(o[j], a0, a1, a2, a3, bb0[j], bb1[j]);
+                    for (int j = 0; j < 4; ++j) mma_f16(o[4 * hw + j], a0, a1, a2, a3, bb0[j], bb1[j]);
+                }
             } else {
                 const int off = kNope + 16 * g;   // bf16 elements 8g..8g+7 of the RoPE part
                 const uint4 A = *reinterpret_cast<const uint4*>(stg + (ea)*kEStride + off);
@@ -401,31 +416,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_partial_kernel(
 }
 
 // Merge the splits of one (sequence, head): out = sum_j 2^(m_j - M) O_j / L,
-// lse = ln 2 * (M + log2 L) with L = sum_j 2^(m_j - M) l_j.
+// lse = ln 2 * (M + log2 L) with L = sum_j 2^(m_j - M) l_j.  The split summaries go through
+// shared memory; the O rows are read 8 splits at a time so their loads overlap.
 __global__ void __launch_bounds__(128) attention_merge_kernel(const float* __restrict__ opart,
                                                               const float2* __restrict__ mlpart,
                                                               int splits, float* __restrict__ out,
                                                               float* __restrict__ lse_out) {
+    __shared__ float fsh[256];
+    __shared__ float lw[4];
     const int b = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-    float M = -INFINITY;
-    for (int j = 0; j < splits; ++j) {
-        const float2 ml = mlpart[((size_t)b * splits + j) * kHeads + h];
-        if (ml.y > 0.f) M = fmaxf(M, ml.x);
+    const int ns = min(splits, 256);
+    // 1) summaries: M = max over non-empty splits, f_j = 2^(m_j - M), L = sum f_j l_j
+    float mj[2], lj[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int j = tid + 128 * r;
+        const float2 ml = j < ns ? mlpart[((size_t)b * splits + j) * kHeads + h] : make_float2(-INFINITY, 0.f);
+        mj[r] = ml.y > 0.f ? ml.x : -INFINITY;
+        lj[r] = ml.y;
     }
+    float M = fmaxf(mj[0], mj[1]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if ((tid & 31) == 0) fsh[tid >> 5] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(fsh[0], fsh[1]), fmaxf(fsh[2], fsh[3]));
+    __syncthreads();
+    float Lp = 0.f;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int j = tid + 128 * r;
+        const float f = (M == -INFINITY || mj[r] == -INFINITY) ? 0.f : exp2f(mj[r] - M);
+        if (j < ns) fsh[j] = f;
+        Lp += f * lj[r];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
+    if ((tid & 31) == 0) lw[tid >> 5] = Lp;
+    __syncthreads();
+    const float Lsum = (lw[0] + lw[1]) + (lw[2] + lw[3]);
+    // 2) weighted sum of the O rows; this thread owns dims 4*tid .. 4*tid+3
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Lsum = 0.f;
-    if (M != -INFINITY) {
-        for (int j = 0; j < splits; ++j) {
-            const float2 ml = mlpart[((size_t)b * splits + j) * kHeads + h];
-            if (!(ml.y > 0.f)) continue;
-            const float f = exp2f(ml.x - M);
-            Lsum += f * ml.y;
-            const float4 v = reinterpret_cast<const float4*>(opart + (((size_t)b * splits + j) * kHeads + h) * kDim)[tid];
-            acc.x += f * v.x;
-            acc.y += f * v.y;
-            acc.z += f * v.z;
-            acc.w += f * v.w;
+    const float4* ob = reinterpret_cast<const float4*>(opart + ((size_t)b * splits * kHeads + h) * kDim) + tid;
+    const size_t jstride = (size_t)kHeads * kDim / 4;
+    for (int j0 = 0; j0 < ns; j0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            v[u] = (j0 + u < ns && fsh[j0 + u] > 0.f) ? ob[(size_t)(j0 + u) * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float f = (j0 + u < ns) ? fsh[j0 + u] : 0.f;
+            acc.x += f * v[u].x;
+            acc.y += f * v[u].y;
+            acc.z += f * v[u].z;
+            acc.w += f * v[u].w;
         }
+    }
+    if (Lsum > 0.f) {
         const float inv = 1.f / Lsum;
         acc.x *= inv;
         acc.y *= inv;
@@ -434,7 +482,7 @@ __global__ void __launch_bounds__(128) attention_merge_kernel(const float* __res
     }
     reinterpret_cast<float4*>(out + ((size_t)b * kHeads + h) * kDim)[tid] = acc;
     if (lse_out && tid == 0)
-        lse_out[(size_t)b * kHeads + h] = (M == -INFINITY) ? -INFINITY : (M + log2f(Lsum)) * 0.69314718055994531f;
+        lse_out[(size_t)b * kHeads + h] = (M == -INFINITY || !(Lsum > 0.f)) ? -INFINITY : (M + log2f(Lsum)) * 0.69314718055994531f;
 }
 
 AttentionPlan attention_plan(int B, int64_t cap, int k, bool sparse, int W, int num_sms) {
@@ -445,7 +493,7 @@ AttentionPlan attention_plan(int B, int64_t cap, int k, bool sparse, int W, int 
     if (s < 1) s = 1;
     if (s > tiles) s = tiles;
     if (s < 1) s = 1;
-    if (s > 256) s = 256;
+    if (s > 256) s = 256;   // the merge kernel handles up to 256 splits
     p.splits = static_cast<int>(s);
     p.ws_bytes = (size_t)B * p.splits * kHeads * (kDim * sizeof(float) + sizeof(float2));
     return p;

@@ -57,13 +57,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase.  Returns false if the phase did not complete within the
-// limit (about a second); callers then record CSLD_DEVERR_TIMEOUT and stop issuing work.
+// Bounded wait on an mbarrier phase: polls first (try_wait itself suspends briefly), then
+// backs off with short sleeps.  Returns false if the phase did not complete within about a
+// second; callers then record CSLD_DEVERR_TIMEOUT and stop issuing work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
     for (uint32_t i = 0; i < (1u << 22); ++i) {
-        __nanosleep(256);
         if (mbar_try_wait(bar, parity)) return true;
+        if (i >= 32) __nanosleep(128);
     }
     return false;
 }
@@ -76,6 +76,15 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// 16-byte shared-memory load kept in program order relative to other volatile asm (the MMAs),
+// so a software-pipelined loop keeps only the next load in flight.
+__device__ __forceinline__ uint4 lds128_ordered(const void* p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
 }
 
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
@@ -98,6 +107,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D += A * B with A, B E4M3 (m16n8k32; A row-major 16x32, B col-major 32x8), fp32 accumulate.
+__device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -149,6 +168,13 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// E4M3 byte -> fp32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+    uint32_t h2, dummy;
+    e4m3x4_to_f16x2x2(byte & 0xFFu, h2, dummy);
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
 }
 
 // fp32 -> E4M3 byte: round to nearest even, saturating to +-448.

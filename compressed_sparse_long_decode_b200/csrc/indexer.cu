@@ -33,7 +33,7 @@ namespace csld {
 
 constexpr int kIdxThreads = 256;
 constexpr int kIdxTile = 256;          // entries per pipeline stage (32 per warp)
-constexpr int kIdxStages = 3;
+constexpr int kIdxStages = 3;   // 256-entry stages of the key stream
 constexpr int kRadixBits = 11;
 constexpr int kRadixBins = 1 << kRadixBits;
 constexpr int kIdxMaxChunk = 8192;
@@ -488,13 +488,29 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
             sm.offs[children] = acc;
         }
         __syncthreads();
-        for (int c = 0; c < children; ++c) {
-            const int cc = sm.offs[c + 1] - sm.offs[c];
-            const size_t src = ((size_t)b * n_runs + parent * tree.group + c) * tree.rcap[level];
-            for (int i = tid; i < cc; i += blockDim.x) {
-                sm.keys[sm.offs[c] + i] = __ldcg(tree.keys[level] + src + i);
-                sm.u.idx[sm.offs[c] + i] = __ldcg(tree.idx[level] + src + i);
+        // all children's loads are issued before any is stored (8 per thread in flight)
+        for (int base = 0; base < children * tree.rcap[level]; base += 8 * blockDim.x) {
+            uint32_t kv[8];
+            int32_t iv[8];
+            int dst[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int flat = base + u * blockDim.x + tid;     // child c, position i
+                const int c = flat / tree.rcap[level], i = flat - c * tree.rcap[level];
+                dst[u] = -1;
+                if (c < children && i < sm.offs[c + 1] - sm.offs[c]) {
+                    const size_t src = ((size_t)b * n_runs + parent * tree.group + c) * tree.rcap[level] + i;
+                    kv[u] = __ldcg(tree.keys[level] + src);
+                    iv[u] = __ldcg(tree.idx[level] + src);
+                    dst[u] = sm.offs[c] + i;
+                }
             }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (dst[u] >= 0) {
+                    sm.keys[dst[u]] = kv[u];
+                    sm.u.idx[dst[u]] = iv[u];
+                }
         }
         n = sm.offs[children];
         __syncthreads();
