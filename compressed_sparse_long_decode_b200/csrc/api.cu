@@ -199,4 +199,35 @@ csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t*
     return CSLD_OK;
 }
 
+csld_status hybrid_decode_attention_static(const uint16_t* q, int heads, const uint8_t* comp_kv,
+                                           int64_t cap, int ratio, const int32_t* topk, int k,
+                                           const uint8_t* win_kv, int W, const int32_t* seq_len, int B,
+                                           float scale, float* out, float* lse_out, int32_t* err,
+                                           void* stream) {
+    if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; this build implements %d", heads, CSLD_HEADS);
+    if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
+    if (cap < 1 || cap > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^31-1", (long long)cap);
+    if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
+    if (W < 0 || W > CSLD_MAX_WINDOW) return fail(CSLD_ERR_ARG, "W %d outside 0..%d", W, CSLD_MAX_WINDOW);
+    if (topk && (k < 1 || k > CSLD_MAX_TOPK)) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
+    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return fail(CSLD_ERR_ARG, "scale is not finite");
+    if (!q || !comp_kv || !seq_len || !out) return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (W > 0 && !win_kv) return fail(CSLD_ERR_ARG, "win_kv is NULL with W > 0");
+    if (!aligned16(q) || !aligned16(comp_kv) || (win_kv && !aligned16(win_kv)) || !aligned16(out))
+        return fail(CSLD_ERR_ALIGN, "q, comp_kv, win_kv and out must be 16-byte aligned");
+    const csld::AttentionPlan plan = csld::attention_plan(B, cap, k, topk != nullptr, W, num_sms());
+    if (plan.ws_bytes > (size_t)CSLD_STATIC_SCRATCH_BYTES)
+        return fail(CSLD_ERR_CAPACITY,
+                    "this call needs %zu bytes of scratch; the library-owned scratch holds %zu bytes "
+                    "(use hybrid_decode_attention with a workspace, or a smaller batch)",
+                    plan.ws_bytes, (size_t)CSLD_STATIC_SCRATCH_BYTES);
+    void* ws = nullptr;
+    cudaError_t e = csld::attention_static_scratch(&ws);
+    if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention_static (scratch address)");
+    e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, seq_len, B, scale, out,
+                               lse_out, ws, plan, err, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention_static");
+    return CSLD_OK;
+}
+
 }  // extern "C"

@@ -29,6 +29,8 @@
 //    staged bytes (pairs of entries per dim), widened, and multiplied with P.
 //  - Each split writes unnormalised O, the running max m (log2 units) and the sum l; a second
 //    kernel merges the splits (log-sum-exp) into out and lse.
+#include <mutex>
+
 #include "csld_internal.cuh"
 #include "kernels.cuh"
 
@@ -517,6 +519,37 @@ cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t 
     if (e != cudaSuccess) return e;
     attention_merge_kernel<<<dim3(B, kHeads), 128, 0, stream>>>(opart, mlpart, plan.splits, out, lse_out);
     return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// Library-owned scratch for callers that cannot allocate device memory (see
+// hybrid_decode_attention_static in csld.h).  The array lives in the library's module: every
+// GPU that loads the library holds these bytes until the process exits.  Host code must not
+// hand the array's name to a kernel (on the host it only stands for the symbol); the device
+// address is looked up once per device with cudaGetSymbolAddress.
+// ------------------------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_attention_static_scratch[CSLD_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+}  // namespace
+
+cudaError_t attention_static_scratch(void** ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_attention_static_scratch);   // the current device's copy
+        if (e != cudaSuccess) return e;
+        g_static_ptr[dev] = p;
+    }
+    *ptr = g_static_ptr[dev];
+    return cudaSuccess;
 }
 
 }  // namespace csld

@@ -47,4 +47,8 @@ cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t 
                              float* lse_out, void* ws, const AttentionPlan& plan, int32_t* err,
                              cudaStream_t stream);
 
+// Device address of the library-owned attention scratch on the current device (looked up on
+// the first call per device).
+cudaError_t attention_static_scratch(void** ptr);
+
 }  // namespace csld

@@ -198,6 +198,36 @@ CSLD_API csld_status hybrid_decode_attention(const uint16_t* q, int heads, const
                                     float scale, float* out, float* lse_out, void* ws,
                                     size_t ws_bytes, int32_t* err, void* stream);
 
+/* ----------------------------------------------------------------------------------------
+ * hybrid_decode_attention_static -- the same computation as hybrid_decode_attention, for
+ * callers that cannot allocate device memory on their call path.  The pages have no
+ * counterpart to this entry point: it exists for integration only.  Examples are a plug-in
+ * whose host framework owns every device allocation and hands it only inputs and outputs,
+ * and a decode loop that must not call the CUDA allocator between steps (an allocation can
+ * synchronise the device or fail under memory pressure).
+ *
+ * Instead of a caller workspace it uses one fixed scratch array of CSLD_STATIC_SCRATCH_BYTES
+ * inside the library.  Every GPU that loads libcsld.so keeps that array until the process
+ * exits.  It allocates nothing:
+ *  - The first call on a device (with that device current) looks up the array's device
+ *    address once. Make that first call before any stream capture.
+ *  - A call that would need more scratch than the array holds returns CSLD_ERR_CAPACITY and
+ *    launches nothing (the need is about B * min(#SMs/B, tiles) * 16 * 2056 bytes; batches up
+ *    to ~250 sequences fit).
+ *  - All calls share the array, and it keeps the last call's contents. Nothing in it needs to
+ *    start at zero, but two calls that overlap on the GPU (different streams without ordering,
+ *    or different host threads) race on it and corrupt each other's results.
+ * Arguments, layouts, results and error handling are those of hybrid_decode_attention.
+ * -------------------------------------------------------------------------------------- */
+#define CSLD_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+CSLD_API csld_status hybrid_decode_attention_static(const uint16_t* q, int heads,
+                                                    const uint8_t* comp_kv, int64_t cap, int ratio,
+                                                    const int32_t* topk, int k,
+                                                    const uint8_t* win_kv, int W,
+                                                    const int32_t* seq_len, int B, float scale,
+                                                    float* out, float* lse_out, int32_t* err,
+                                                    void* stream);
+
 #ifdef __cplusplus
 }
 #endif
