@@ -17,10 +17,12 @@
 // The fp32 score then follows a fixed operation order (see the ABI header), so the selection
 // is reproducible bit for bit; order key = (score, -index).
 //
-// One kernel (indexer_topk_kernel), grid (chunk, sequence): each CTA streams `chunk` entries
-// of keys through shared memory with 1-D bulk copies (4-stage mbarrier ring), scores them into
-// 32-bit order keys held in shared memory, and radix-selects its chunk's top min(k, chunk),
-// written as a run in index order.  The runs are then merged by a tree inside the same kernel:
+// One kernel (indexer_topk_kernel), grid (chunk, sequence), 16 warps per CTA: each CTA streams
+// `chunk` entries of keys through shared memory with 1-D bulk copies (3-stage mbarrier ring of
+// 512-entry tiles), scores them into 32-bit order keys held in shared memory while building a
+// histogram of the keys' top 11 bits, and selects its chunk's top min(k, chunk) -- threshold
+// bin from the histogram, one pass to count and collect that bin's candidates, a radix
+// select among the candidates only, one pass to emit in index order -- written as a run.  The runs are then merged by a tree inside the same kernel:
 // the last CTA of a group of G runs to finish (an atomic arrival counter; nothing ever waits)
 // loads the group's runs, selects their top min(k, ...) and publishes one run for the next
 // level; the last run is the answer, written in ascending index order and -1 padded.
@@ -31,47 +33,52 @@
 
 namespace csld {
 
-constexpr int kIdxThreads = 256;
-constexpr int kIdxTile = 256;          // entries per pipeline stage (32 per warp)
-constexpr int kIdxStages = 3;   // 256-entry stages of the key stream
-constexpr int kRadixBits = 11;
-constexpr int kRadixBins = 1 << kRadixBits;
-constexpr int kIdxMaxChunk = 8192;
-
+constexpr int kIdxThreads = 512;
+constexpr int kIdxWarps = kIdxThreads / 32;
+constexpr int kIdxTile = 512;          // entries per pipeline stage (32 per warp)
+constexpr int kIdxStages = 3;
+constexpr int kIdxMaxChunk = 8192;     // keys a CTA holds (chunk, or runs being merged)
 constexpr int kIdxMaxGroup = 64;       // runs merged by one CTA
 constexpr int kIdxMaxLevels = 4;
+constexpr int kBinShift = 21;          // histogram bin = top 11 bits of the order key
+constexpr int kBins = 1 << (32 - kBinShift);
+constexpr int kRadixBits = 11;
+constexpr int kRadixBins = 1 << kRadixBits;
 
 struct IdxSmem {
     union {
         struct {
             uint8_t codes[kIdxStages][kIdxTile * kIkey];
             float scales[kIdxStages][kIdxTile * 2];
-        } pipe;                        // key stream ring (scoring phase)
-        int32_t idx[kIdxMaxChunk];     // entry indices of the runs being merged (merge phase)
+        } pipe;                        // key stream ring (scoring)
+        struct {
+            uint32_t key[kIdxMaxChunk];
+            uint16_t pos[kIdxMaxChunk];
+        } cand;                        // threshold-bin candidates (selection)
     } u;
     uint32_t keys[kIdxMaxChunk];       // order keys of the chunk, or of the runs being merged
-    uint32_t hist[kRadixBins];
-    uint32_t scan[4 * (kIdxThreads / 32)];
+    uint32_t hist[kBins];              // top-11-bit histogram of keys[]
+    uint32_t rhist[kRadixBins];        // radix passes over the candidates
+    uint32_t wgt[kIdxWarps], wsel[kIdxWarps], weq[kIdxWarps], wbase[kIdxWarps], weqb[kIdxWarps];
+    uint32_t red[2 * kIdxWarps];
     int32_t offs[kIdxMaxGroup + 1];
-    float qscale[8];                   // [group*4 + head]
+    float qscale[8];                   // [group*4 + head] * 0.25
     uint64_t full[kIdxStages];
-    uint32_t sel[4];
+    uint32_t sel[4];                   // bin / threshold results
+    uint32_t ncand;
     int32_t last;
 };
 
-// --- block-wide helpers (256 threads) ----------------------------------------------------
-
-// Radix select over n keys (read through `get(i)`): the largest `want` (< n) keys, ties on
-// the threshold resolved by lower position.  Returns the threshold key and, through *take_eq,
-// how many keys equal to it are selected (the lowest-position ones).  The bits above the
-// highest bit in which the keys differ are skipped; the rest are resolved 11 bits per pass
-// (at most 3 passes) with a shared-memory histogram.  hist: kRadixBins words; sel: 4 words;
-// red: 2 * blockDim/32 words.  All threads must call.
+// ------------------------------------------------------------------------------------------
+// Block-level helpers (512 threads).
+// ------------------------------------------------------------------------------------------
+// Radix select among n candidate keys (read through get): the largest `want` (< n), ties on the
+// threshold left to the caller (who takes the first take_eq equal keys by position).  The bits
+// shared by all candidates are skipped; the rest are resolved 11 bits per pass.
 template <typename Get>
 __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint32_t* sel,
                                  uint32_t* red, uint32_t* take_eq) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    // common prefix of all keys
     uint32_t kor = 0u, kand = 0xFFFFFFFFu;
     for (int i = tid; i < n; i += blockDim.x) {
         const uint32_t key = get(i);
@@ -93,19 +100,17 @@ __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint3
     }
     __syncthreads();
     const uint32_t diff = kor ^ kand;
-    if (diff == 0u) {            // all keys equal
+    if (diff == 0u) {
         *take_eq = static_cast<uint32_t>(want);
         return kand;
     }
-    int top = 31 - __clz(diff);  // highest differing bit
-    uint32_t prefix = kand & ~((2u << top) - 1u);   // common bits above `top` (0 when top == 31)
-    if (top == 31) prefix = 0u;
+    int top = 31 - __clz(diff);
     uint32_t himask = (top == 31) ? 0u : ~((2u << top) - 1u);
+    uint32_t prefix = kand & himask;
     uint32_t remaining = static_cast<uint32_t>(want);
     while (true) {
         const int shift = max(top - (kRadixBits - 1), 0);
-        const int width = top - shift + 1;
-        const uint32_t nb = 1u << width;
+        const uint32_t nb = 1u << (top - shift + 1);
         for (uint32_t i = tid; i < nb; i += blockDim.x) hist[i] = 0u;
         __syncthreads();
         for (int i = tid; i < n; i += blockDim.x) {
@@ -113,7 +118,6 @@ __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint3
             if (((key ^ prefix) & himask) == 0u) atomicAdd(&hist[(key >> shift) & (nb - 1u)], 1u);
         }
         __syncthreads();
-        // thread t owns digits nb-1-t*per .. (descending); block scan of the per-thread sums
         const uint32_t per = (nb + blockDim.x - 1) / blockDim.x;
         uint32_t tot = 0u;
         for (uint32_t q = 0; q < per; ++q) {
@@ -128,9 +132,9 @@ __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint3
         }
         if (lane == 31) red[warp] = incl;
         __syncthreads();
-        uint32_t wbase = 0u;
-        for (int w = 0; w < warp; ++w) wbase += red[w];
-        incl += wbase;
+        uint32_t wb = 0u;
+        for (int w = 0; w < warp; ++w) wb += red[w];
+        incl += wb;
         const uint32_t excl = incl - tot;
         if (excl < remaining && incl >= remaining) {
             uint32_t run = excl;
@@ -157,61 +161,129 @@ __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint3
     return prefix;
 }
 
-// Writes, in position order, the positions selected by (key > thr) or (key == thr and among
-// the first take_eq such positions).  Warp w owns a contiguous segment and walks it 32 keys
-// at a time (lane i reads position base+i: conflict-free); ballots give the in-warp order and
-// one block-level scan of the warp totals gives each warp's offsets.  emit(pos, i).
-// buf: at least 4 * (blockDim.x / 32) words.
-template <typename Get, typename Emit>
-__device__ void select_compact(Get get, int n, uint32_t thr, uint32_t take_eq, uint32_t* buf,
-                               Emit emit) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const int seg = ((n + nw - 1) / nw + 31) & ~31;
-    const int i0 = min(n, warp * seg), i1 = min(n, i0 + seg);
+// Selects the top `want` of sm.keys[0..n) under (key desc, position asc) and emits them in
+// position order: emit(out_pos, position).  Requires sm.hist = histogram of key >> kBinShift.
+template <typename Emit>
+__device__ void select_emit(IdxSmem& sm, int n, int want, Emit emit) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t lt = (1u << lane) - 1u;
-    uint32_t gt = 0u, eq = 0u;
+    const int seg = ((n + kIdxWarps - 1) / kIdxWarps + 31) & ~31;
+    const int i0 = min(n, warp * seg), i1 = min(n, i0 + seg);
+    if (want >= n) {                                   // everything is selected
+        for (int base = i0; base < i1; base += 32)
+            if (base + lane < i1) emit(base + lane, base + lane);
+        __syncthreads();
+        return;
+    }
+    // 1) the bin holding the want-th largest key (thread t owns bins 2047-4t .. 2044-4t)
+    {
+        uint32_t c[4], tot = 0u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            c[q] = sm.hist[kBins - 1 - 4 * tid - q];
+            tot += c[q];
+        }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) sm.red[warp] = incl;
+        if (tid == 0) sm.ncand = 0u;
+        __syncthreads();
+        uint32_t wb = 0u;
+        for (int w = 0; w < warp; ++w) wb += sm.red[w];
+        incl += wb;
+        const uint32_t excl = incl - tot;
+        const uint32_t W = static_cast<uint32_t>(want);
+        if (excl < W && incl >= W) {
+            uint32_t run = excl;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (run + c[q] >= W) {
+                    sm.sel[0] = static_cast<uint32_t>(kBins - 1 - 4 * tid - q);   // bin beta
+                    sm.sel[1] = W - run;                                          // wanted inside it
+                    break;
+                }
+                run += c[q];
+            }
+        }
+        if (tid < kIdxWarps) {
+            sm.wsel[tid] = 0u;
+            sm.weq[tid] = 0u;
+        }
+        __syncthreads();
+    }
+    const uint32_t beta = sm.sel[0], need = sm.sel[1];
+    // 2) pass 1: per-warp count above the bin; collect the bin's candidates with positions
+    uint32_t gt = 0u;
     for (int base = i0; base < i1; base += 32) {
         const int i = base + lane;
-        const uint32_t key = i < i1 ? get(i) : 0u;
-        gt += __popc(__ballot_sync(0xffffffffu, i < i1 && key > thr));
-        eq += __popc(__ballot_sync(0xffffffffu, i < i1 && key == thr));
+        const uint32_t key = i < i1 ? sm.keys[i] : 0u;
+        const uint32_t bin = key >> kBinShift;
+        gt += __popc(__ballot_sync(0xffffffffu, i < i1 && bin > beta));
+        const uint32_t cm = __ballot_sync(0xffffffffu, i < i1 && bin == beta);
+        if (cm) {
+            uint32_t slot = 0u;
+            if (lane == 0) slot = atomicAdd(&sm.ncand, static_cast<uint32_t>(__popc(cm)));
+            slot = __shfl_sync(0xffffffffu, slot, 0);
+            if (i < i1 && bin == beta) {
+                const uint32_t at = slot + __popc(cm & lt);
+                sm.u.cand.key[at] = key;
+                sm.u.cand.pos[at] = static_cast<uint16_t>(i);
+            }
+        }
     }
+    if (lane == 0) sm.wgt[warp] = gt;
     __syncthreads();
-    if (lane == 0) {
-        buf[warp] = eq;
-        buf[nw + warp] = gt;
+    // 3) exact threshold among the candidates
+    const int P = static_cast<int>(sm.ncand);
+    uint32_t thr = 0u, take_eq = static_cast<uint32_t>(P);
+    if (static_cast<int>(need) < P)
+        thr = radix_select([&](int c) { return sm.u.cand.key[c]; }, P, static_cast<int>(need), sm.rhist, sm.sel + 2,
+                           sm.red, &take_eq);
+    // 4) per-warp counts of selected candidates (above the threshold, equal to it)
+    for (int c = tid; c < P; c += blockDim.x) {
+        const uint32_t key = sm.u.cand.key[c];
+        const int w = sm.u.cand.pos[c] / seg;
+        if (key > thr) atomicAdd(&sm.wsel[w], 1u);
+        else if (key == thr) atomicAdd(&sm.weq[w], 1u);
     }
     __syncthreads();
     if (warp == 0) {
-        const uint32_t e = lane < nw ? buf[lane] : 0u, g = lane < nw ? buf[nw + lane] : 0u;
+        const uint32_t e = lane < kIdxWarps ? sm.weq[lane] : 0u;
         uint32_t ei = e;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, ei, o);
             if (lane >= o) ei += y;
         }
-        const uint32_t eb = ei - e;                                   // ties before this warp
+        const uint32_t eb = ei - e;
         const uint32_t tw = eb >= take_eq ? 0u : min(e, take_eq - eb);
-        const uint32_t tk = g + tw;
+        const uint32_t tk = (lane < kIdxWarps ? sm.wgt[lane] + sm.wsel[lane] : 0u) + tw;
         uint32_t ti = tk;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, ti, o);
             if (lane >= o) ti += y;
         }
-        if (lane < nw) {
-            buf[2 * nw + lane] = eb;
-            buf[3 * nw + lane] = ti - tk;
+        if (lane < kIdxWarps) {
+            sm.wbase[lane] = ti - tk;
+            sm.weqb[lane] = eb;
         }
     }
     __syncthreads();
-    uint32_t eq_seen = buf[2 * nw + warp], pos = buf[3 * nw + warp];
+    // 5) pass 2: emit in position order
+    uint32_t pos = sm.wbase[warp], eq_seen = sm.weqb[warp];
     for (int base = i0; base < i1; base += 32) {
         const int i = base + lane;
-        const uint32_t key = i < i1 ? get(i) : 0u;
-        const bool veq = i < i1 && key == thr;
+        const uint32_t key = i < i1 ? sm.keys[i] : 0u;
+        const uint32_t bin = key >> kBinShift;
+        const bool inb = i < i1 && bin == beta;
+        const bool veq = inb && key == thr;
         const uint32_t em = __ballot_sync(0xffffffffu, veq);
-        const bool take = (i < i1 && key > thr) || (veq && eq_seen + __popc(em & lt) < take_eq);
+        const bool take = (i < i1 && bin > beta) || (inb && key > thr) || (veq && eq_seen + __popc(em & lt) < take_eq);
         const uint32_t tm = __ballot_sync(0xffffffffu, take);
         if (take) emit(pos + __popc(tm & lt), i);
         pos += __popc(tm);
@@ -227,7 +299,7 @@ struct IdxTree {
     int levels;                        // run levels that are stored (the final run is not)
     int n_runs[kIdxMaxLevels + 1];     // runs per sequence at each level (level 0 = chunks)
     int rcap[kIdxMaxLevels + 1];       // candidates a run of each level can hold
-    uint32_t* keys[kIdxMaxLevels];     // [B][n_runs[l]][kc]
+    uint32_t* keys[kIdxMaxLevels];     // [B][n_runs[l]][rcap[l]]
     int32_t* idx[kIdxMaxLevels];
     int32_t* cnt[kIdxMaxLevels];       // [B][n_runs[l]]
     int32_t* ctr[kIdxMaxLevels + 1];   // arrival counters of level l runs, [B][n_runs[l]]
@@ -287,6 +359,7 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
     const int64_t c0 = (int64_t)ch * chunk;
     const int cn = static_cast<int>(max64(0, min64(chunk, n_b - c0)));
 
+    for (int i = tid; i < kBins; i += blockDim.x) sm.hist[i] = 0u;
     bool chunk_ok = true;
     if (cn > 0) {
         // --- query: FP4 codes doubled as int8, in the MMA's B layout ----------------------
@@ -300,7 +373,7 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
             for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[i]));
             const float sg = fp4_group_scale(amax);
             const float inv = 1.0f / sg;   // exact: a power of two
-            if (cq == 0) sm.qscale[grp * 4 + h] = sg;
+            if (warp == 0 && cq == 0) sm.qscale[grp * 4 + h] = sg;
             uint32_t w0 = 0u, w1 = 0u;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -335,6 +408,10 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
             fence_barrier_init();
         }
         __syncthreads();
+        // query group scales of the two heads this lane finishes
+        const int hp = (cq & 1) * 2;
+        const float qs0a = sm.qscale[hp], qs0b = sm.qscale[hp + 1];
+        const float qs1a = sm.qscale[4 + hp], qs1b = sm.qscale[4 + hp + 1];
 
         const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
         const uint8_t* kbase = ikeys + ((size_t)b * cap + (size_t)c0) * kIkey;
@@ -371,18 +448,18 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
                 const uint32_t kB0 = *reinterpret_cast<const uint32_t*>(cs + rB * kIkey + 4 * cq);
                 const uint32_t kA1 = *reinterpret_cast<const uint32_t*>(cs + rA * kIkey + 16 + 4 * cq);
                 const uint32_t kB1 = *reinterpret_cast<const uint32_t*>(cs + rB * kIkey + 16 + 4 * cq);
-                int acc[4] = {0, 0, 0, 0};
+                // positive and negative magnitude planes accumulate separately (two MMA chains)
+                int accp[4] = {0, 0, 0, 0}, accn[4] = {0, 0, 0, 0};
                 auto lut = [](uint32_t sel) { return prmt(kTwiceE2M1Lo, kTwiceE2M1Hi, sel); };
-                mma_s8(acc, lut(kA0), lut(kB0), lut(kA0 >> 16), lut(kB0 >> 16), b00, b01);
-                {
-                    const uint32_t nA = kA0 ^ 0x88888888u, nB = kB0 ^ 0x88888888u;
-                    mma_s8(acc, lut(nA), lut(nB), lut(nA >> 16), lut(nB >> 16), n00, n01);
-                }
-                mma_s8(acc, lut(kA1), lut(kB1), lut(kA1 >> 16), lut(kB1 >> 16), b10, b11);
-                {
-                    const uint32_t nA = kA1 ^ 0x88888888u, nB = kB1 ^ 0x88888888u;
-                    mma_s8(acc, lut(nA), lut(nB), lut(nA >> 16), lut(nB >> 16), n10, n11);
-                }
+                const uint32_t nA0 = kA0 ^ 0x88888888u, nB0 = kB0 ^ 0x88888888u;
+                const uint32_t nA1 = kA1 ^ 0x88888888u, nB1 = kB1 ^ 0x88888888u;
+                mma_s8(accp, lut(kA0), lut(kB0), lut(kA0 >> 16), lut(kB0 >> 16), b00, b01);
+                mma_s8(accn, lut(nA0), lut(nB0), lut(nA0 >> 16), lut(nB0 >> 16), n00, n01);
+                mma_s8(accp, lut(kA1), lut(kB1), lut(kA1 >> 16), lut(kB1 >> 16), b10, b11);
+                mma_s8(accn, lut(nA1), lut(nB1), lut(nA1 >> 16), lut(nB1 >> 16), n10, n11);
+                int acc[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc[r] = accp[r] + accn[r];
                 // acc: (row g, cols 2cq, 2cq+1), (row g+8, same).  cq < 2: group-0 dots of
                 // heads 2cq, 2cq+1; cq >= 2: group-1 dots of heads 2(cq-2), 2(cq-2)+1.
                 const bool lo = cq < 2;
@@ -390,30 +467,28 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
                 const int got0 = __shfl_xor_sync(0xffffffffu, send0, 2);
                 const int got1 = __shfl_xor_sync(0xffffffffu, send1, 2);
                 const int row = lo ? rA : rB;
-                const int hp = (cq & 1) * 2;
                 const int i0a = lo ? acc[0] : got0, i0b = lo ? acc[1] : got1;
                 const int i1a = lo ? got0 : acc[2], i1b = lo ? got1 : acc[3];
                 const float ks0 = ss[2 * row], ks1 = ss[2 * row + 1];
-                float r[2];
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int h = hp + q;
-                    const float s0 = __fmul_rn(__fmul_rn(sm.qscale[h], ks0), 0.25f);
-                    const float s1 = __fmul_rn(__fmul_rn(sm.qscale[4 + h], ks1), 0.25f);
-                    const int I0 = q ? i0b : i0a, I1 = q ? i1b : i1a;
-                    const float d = __fmaf_rn(static_cast<float>(I1), s1,
-                                              __fmul_rn(static_cast<float>(I0), s0));
-                    r[q] = d > 0.f ? d : 0.f;
-                }
-                const float r2 = __shfl_xor_sync(0xffffffffu, r[0], 1);
-                const float r3 = __shfl_xor_sync(0xffffffffu, r[1], 1);
+                // d = fma(I1, s1, I0*s0) with s_g = (qscale_g * kscale_g) * 0.25
+                const float s0a = __fmul_rn(__fmul_rn(qs0a, ks0), 0.25f), s1a = __fmul_rn(__fmul_rn(qs1a, ks1), 0.25f);
+                const float s0b = __fmul_rn(__fmul_rn(qs0b, ks0), 0.25f), s1b = __fmul_rn(__fmul_rn(qs1b, ks1), 0.25f);
+                const float da = __fmaf_rn(static_cast<float>(i1a), s1a, __fmul_rn(static_cast<float>(i0a), s0a));
+                const float db = __fmaf_rn(static_cast<float>(i1b), s1b, __fmul_rn(static_cast<float>(i0b), s0b));
+                const float r0 = da > 0.f ? da : 0.f, r1 = db > 0.f ? db : 0.f;
+                const float r2 = __shfl_xor_sync(0xffffffffu, r0, 1);
+                const float r3 = __shfl_xor_sync(0xffffffffu, r1, 1);
                 if ((cq & 1) == 0) {
-                    float e = __fmul_rn(w0, r[0]);
-                    e = __fmaf_rn(w1, r[1], e);
+                    float e = __fmul_rn(w0, r0);
+                    e = __fmaf_rn(w1, r1, e);
                     e = __fmaf_rn(w2, r2, e);
                     e = __fmaf_rn(w3, r3, e);
                     const int li = tile * kIdxTile + row;
-                    if (li < cn) sm.keys[li] = score_key(e);
+                    if (li < cn) {
+                        const uint32_t key = score_key(e);
+                        sm.keys[li] = key;
+                        atomicAdd(&sm.hist[key >> kBinShift], 1u);
+                    }
                 }
             }
             __syncthreads();   // stage s fully consumed
@@ -428,38 +503,60 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
                 for (int t = consumed; t < min(n_tiles, consumed + kIdxStages); ++t)
                     (void)mbar_wait(&sm.full[t % kIdxStages], (t / kIdxStages) & 1);
             }
-            __syncthreads();
         }
-        // (the stage barriers are not reused after this point)
     }
+    __syncthreads();
 
     // --- selection and the merge tree ------------------------------------------------------
     int n = (cn > 0 && chunk_ok) ? cn : 0;   // a timed-out chunk publishes nothing
     int level = 0, run = ch;
-    // chunk level: the entry index of key i is c0 + i (sm.u.idx still aliases the key ring)
-    auto idx_of = [&](int i) -> int32_t { return level == 0 ? static_cast<int32_t>(c0 + i) : sm.u.idx[i]; };
-    __syncthreads();
+    const uint32_t* child_idx = nullptr;     // merge levels: indices stay in the children runs
     for (;;) {
         const int n_runs = tree.n_runs[level];
         const bool final_run = (n_runs == 1);
         const int want = min(final_run ? k : tree.rcap[level], n);
-        uint32_t thr = 0u, take_eq = static_cast<uint32_t>(n);
-        if (want < n) thr = radix_select([&](int i) { return sm.keys[i]; }, n, want, sm.hist, sm.sel, sm.scan, &take_eq);
+        const size_t rb = final_run ? 0 : ((size_t)b * n_runs + run) * tree.rcap[level];
+        int32_t* out = topk_out + (size_t)b * k;
+        if (level == 0) {
+            // chunk level: the entry index of position i is c0 + i
+            if (final_run) {
+                select_emit(sm, n, want, [&](int p, int i) { out[p] = static_cast<int32_t>(c0 + i); });
+            } else {
+                uint32_t* okeys = tree.keys[0] + rb;
+                int32_t* oidx = tree.idx[0] + rb;
+                select_emit(sm, n, want, [&](int p, int i) {
+                    okeys[p] = sm.keys[i];
+                    oidx[p] = static_cast<int32_t>(c0 + i);
+                });
+            }
+        } else {
+            // merge levels: the entry indices stay in the children runs (L2).  The ordered pass
+            // records positions only; the indices are then fetched together, so their loads
+            // overlap instead of costing one round trip per 32 keys.
+            select_emit(sm, n, want, [&](int p, int i) { sm.rhist[p] = static_cast<uint32_t>(i); });
+            const int rcc = tree.rcap[level - 1];
+            for (int p = tid; p < want; p += blockDim.x) {
+                const int i = static_cast<int>(sm.rhist[p]);
+                int lo = 0, hi = kIdxMaxGroup - 1;           // child c with offs[c] <= i < offs[c+1]
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (sm.offs[mid] <= i) lo = mid;
+                    else hi = mid - 1;
+                }
+                const int32_t idx = __ldcg(reinterpret_cast<const int32_t*>(child_idx) + (size_t)lo * rcc + (i - sm.offs[lo]));
+                if (final_run) {
+                    out[p] = idx;
+                } else {
+                    tree.keys[level][rb + p] = sm.keys[i];
+                    tree.idx[level][rb + p] = idx;
+                }
+            }
+            __syncthreads();
+        }
         if (final_run) {
-            int32_t* out = topk_out + (size_t)b * k;
-            select_compact([&](int i) { return sm.keys[i]; }, n, thr, take_eq, sm.scan,
-                           [&](uint32_t pos, int i) { out[pos] = idx_of(i); });
             for (int i = want + tid; i < k; i += blockDim.x) out[i] = -1;
             return;
         }
-        const size_t rb = ((size_t)b * n_runs + run) * tree.rcap[level];
-        uint32_t* okeys = tree.keys[level] + rb;
-        int32_t* oidx = tree.idx[level] + rb;
-        select_compact([&](int i) { return sm.keys[i]; }, n, thr, take_eq, sm.scan,
-                       [&](uint32_t pos, int i) {
-                           okeys[pos] = sm.keys[i];
-                           oidx[pos] = idx_of(i);
-                       });
         if (tid == 0) tree.cnt[level][(size_t)b * n_runs + run] = want;
         // arrive at the parent; the last child to arrive carries on with the merge
         const int parent = run / tree.group;
@@ -478,7 +575,8 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
         }
         __syncthreads();
         if (!sm.last) return;
-        // load the children runs (published by other CTAs: read through L2)
+        // load the children runs' keys (published by other CTAs: read through L2) and rebuild
+        // the histogram; their indices are read from L2 when emitting
         if (tid == 0) {
             int acc = 0;
             for (int c = 0; c < children; ++c) {
@@ -486,22 +584,22 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
                 acc += __ldcg(tree.cnt[level] + (size_t)b * n_runs + parent * tree.group + c);
             }
             sm.offs[children] = acc;
+            for (int c = children + 1; c <= kIdxMaxGroup; ++c) sm.offs[c] = 1 << 30;   // > any position
         }
+        for (int i = tid; i < kBins; i += blockDim.x) sm.hist[i] = 0u;
         __syncthreads();
-        // all children's loads are issued before any is stored (8 per thread in flight)
-        for (int base = 0; base < children * tree.rcap[level]; base += 8 * blockDim.x) {
+        const size_t child0 = ((size_t)b * n_runs + (size_t)parent * tree.group) * tree.rcap[level];
+        const int rc = tree.rcap[level];
+        for (int base = 0; base < children * rc; base += 8 * blockDim.x) {
             uint32_t kv[8];
-            int32_t iv[8];
             int dst[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int flat = base + u * blockDim.x + tid;     // child c, position i
-                const int c = flat / tree.rcap[level], i = flat - c * tree.rcap[level];
+                const int c = flat / rc, i = flat - c * rc;
                 dst[u] = -1;
                 if (c < children && i < sm.offs[c + 1] - sm.offs[c]) {
-                    const size_t src = ((size_t)b * n_runs + parent * tree.group + c) * tree.rcap[level] + i;
-                    kv[u] = __ldcg(tree.keys[level] + src);
-                    iv[u] = __ldcg(tree.idx[level] + src);
+                    kv[u] = __ldcg(tree.keys[level] + child0 + flat);
                     dst[u] = sm.offs[c] + i;
                 }
             }
@@ -509,9 +607,10 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
             for (int u = 0; u < 8; ++u)
                 if (dst[u] >= 0) {
                     sm.keys[dst[u]] = kv[u];
-                    sm.u.idx[dst[u]] = iv[u];
+                    atomicAdd(&sm.hist[kv[u] >> kBinShift], 1u);
                 }
         }
+        child_idx = reinterpret_cast<const uint32_t*>(tree.idx[level] + child0);
         n = sm.offs[children];
         __syncthreads();
         ++level;
