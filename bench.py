@@ -119,6 +119,64 @@ def algorithmic_bytes(wl):
     }
 
 
+# ncu summaries under profiles/: DRAM read+write bytes per launch, valid only while the kernel's
+# sources hash to the value recorded with the capture (a changed kernel reports null).
+PROFILES = {
+    "indexer": ("indexer_topk_decode1m.md", "indexer.cu", ""),
+    "csa_attention": ("attention_partial_decode1m.md", "attention.cu", " (CSA)"),
+    "hca_attention": ("attention_partial_decode1m.md", "attention.cu", " (HCA)"),
+}
+
+
+def kernel_source_hash(cu):
+    import hashlib
+    h = hashlib.sha256()
+    for f in (cu, "csld_internal.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "compressed_sparse_long_decode_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary of this kernel on this workload,
+    or None when there is none or the kernel changed since it was taken."""
+    if kernel not in PROFILES or workload != "decode1m":
+        return None
+    md, cu, tag = PROFILES[kernel]
+    try:
+        with open(os.path.join(ROOT, "profiles", md)) as fh:
+            text = fh.read()
+    except OSError:
+        return None
+    want_hash, traffic = None, None
+    for line in text.splitlines():
+        if line.startswith("source_sha256[:16]"):
+            want_hash = line.rsplit(":", 1)[1].strip()
+        if line.startswith(f"traffic_bytes_per_launch{tag}:"):
+            traffic = int(line.rsplit(":", 1)[1].strip())
+    if want_hash is None or traffic is None or want_hash != kernel_source_hash(cu):
+        return None
+    return traffic
+
+
+def max_over_ranks(ms, device):
+    """The slowest rank's time: every rank contributes its device-timed milliseconds and all
+    of them get the maximum back (a no-op without a process group)."""
+    import torch
+    import torch.distributed as td
+    if not (td.is_available() and td.is_initialized()) or td.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    td.all_reduce(t, op=td.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, ms_max, world):
+    """Whole-job rate: the units all ranks processed (each rank processes the same number:
+    independent sequences, weak scaling) over the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import compressed_sparse_long_decode_b200 as csld
@@ -259,16 +317,11 @@ def run_ours(args, rank, world, local_rank):
     t3.record()
     torch.cuda.synchronize()
     ms_dev = t2.elapsed_time(t3)
-    ms = min(ms_total, ms_dev)
-    if dist:
-        import torch.distributed as td
-        tt = torch.tensor([ms], device=dev)
-        td.all_reduce(tt, op=td.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(min(ms_total, ms_dev), dev)
     assert err.item() == 0, f"device error word {err.item()}"
 
     # --- end to end: host (pinned) inputs -> device -> step -> host outputs -----------------
-    e2e = run_e2e(csld, torch, layers, wl, dev, k, W, scale, ws_idx, ws_att, err, rounds_t)
+    e2e = run_e2e(csld, torch, layers, wl, dev, k, W, scale, ws_idx, ws_att, err, rounds_t, world)
 
     peaks, peak_kind = measured_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
@@ -278,7 +331,7 @@ def run_ours(args, rank, world, local_rank):
     achieved = bytes_[dominant] / (avg[dominant] * 1e-3) / 1e9
     step_bytes = sum(bytes_.values())
     ms_step = ms / steps_timed
-    value = world * B * steps_timed / (ms * 1e-3)
+    value = job_throughput(B * steps_timed, ms, world)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps_timed,
         "warmup": rounds_w * REPLICAS, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
@@ -297,7 +350,8 @@ def run_ours(args, rank, world, local_rank):
         "kernels_ms_per_step": {n: round(v, 5) for n, v in avg.items()},
         "roofline": {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "traffic": None, "algorithmic_bytes_per_launch": bytes_[dominant]},
+                     "traffic": profiled_traffic(dominant, wl.name),
+                     "algorithmic_bytes_per_launch": bytes_[dominant]},
         "roofline_all": {n: {"achieved_gbs": round(bytes_[n] / (avg[n] * 1e-3) / 1e9, 1),
                              "frac": round(bytes_[n] / (avg[n] * 1e-3) / 1e9 / hbm_peak, 4)} for n in avg},
         "clocks": clk,
@@ -307,7 +361,7 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
-def run_e2e(csld, torch, layers, wl, dev, k, W, scale, ws_idx, ws_att, err, rounds):
+def run_e2e(csld, torch, layers, wl, dev, k, W, scale, ws_idx, ws_att, err, rounds, world):
     """Same step through the public API with the step's inputs copied from pinned host memory
     and both layers' outputs copied back, inside the timed region (graph-replayed)."""
     B = wl.batch
@@ -361,10 +415,10 @@ def run_e2e(csld, torch, layers, wl, dev, k, W, scale, ws_idx, ws_att, err, roun
         graph.replay()
     t1.record()
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
     n_steps = rounds * REPLICAS
     assert torch.isfinite(h_out).all()
-    return {"value": round(B * n_steps / (ms * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": round(job_throughput(B * n_steps, ms, world), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / n_steps, 5)}
 
 
