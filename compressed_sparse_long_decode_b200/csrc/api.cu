@@ -150,7 +150,7 @@ csld_status indexer_topk(const uint8_t* ikeys, const float* iscales, int64_t cap
                          void* stream) {
     if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
     if (k < 1 || k > CSLD_MAX_TOPK) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
-    if (cap < 1 || cap > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^31-1", (long long)cap);
+    if (cap < 1 || cap > ((int64_t)1 << 30)) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^30", (long long)cap);
     if (cap & 1) return fail(CSLD_ERR_ALIGN, "cap must be even");
     if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
     if (!ikeys || !iscales || !seq_len || !q_idx || !head_w || !topk_out)
@@ -163,6 +163,7 @@ csld_status indexer_topk(const uint8_t* ikeys, const float* iscales, int64_t cap
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CSLD_ERR_ALIGN, "workspace must be 256-byte aligned");
     cudaError_t e = csld::launch_indexer(ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, B, k,
                                          topk_out, ws, plan, err, as_stream(stream));
+    if (e == cudaErrorNotSupported) return fail(CSLD_ERR_UNSUPPORTED, "no tensor-map encoder in this driver");
     if (e != cudaSuccess) return cuda_fail(e, "indexer_topk");
     return CSLD_OK;
 }

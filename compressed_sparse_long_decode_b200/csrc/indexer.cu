@@ -7,20 +7,21 @@
 //
 // Score of entry s for one query (4 heads, 64 dims, one key per entry shared by the heads):
 //   e_s = sum_h w_h * ReLU(q_h . k_s), q and k both FP4 (E2M1 codes, power-of-two scale / 32).
-// The two 32-element group dots of every (entry, head) are exact integers (codes doubled are
-// the integers {0,1,2,3,4,6,8,12} with sign), computed on the tensor cores with
-// mma.sync.m16n8k32 s8 x s8 -> s32.  A key nibble is turned into its doubled magnitude by one
-// PRMT lookup: the code's sign bit is PRMT's sign-replicate flag, so negative codes yield 0;
-// the same lookup on the nibbles with flipped signs yields the negative codes' magnitudes, and
-// dot = pos . q - neg . q = pos . q + neg . (-q).  B columns 0..3 hold the query heads over
-// group 0 and columns 4..7 over group 1, so one accumulator holds both group dots.
-// The fp32 score then follows a fixed operation order (see the ABI header), so the selection
-// is reproducible bit for bit; order key = (score, -index).
+// The group dots run on the 5th-generation tensor cores as block-scaled FP4 MMAs
+// (tcgen05.mma kind::mxf4, M = 128 entries, N = 8, K = 64) with every block scale set to 1, so
+// each product of two E2M1 values (a multiple of 1/4, at most 36) and their 32-term sums are
+// exact in the fp32 accumulator: the MMA returns I_g / 4 exactly.  B row n holds head n & 3
+// over group n >> 2 with the other group's codes zero, so each output column is one group's
+// dot.  The fp32 score then follows a fixed operation order (see the ABI header) using the
+// true scales, so the selection is reproducible bit for bit; order key = (score, -index).
 //
-// One kernel (indexer_topk_kernel), grid (chunk, sequence), 16 warps per CTA: each CTA streams
-// `chunk` entries of keys through shared memory with 1-D bulk copies (3-stage mbarrier ring of
-// 512-entry tiles), scores them into 32-bit order keys held in shared memory while building a
-// histogram of the keys' top 11 bits, and selects its chunk's top min(k, chunk) -- threshold
+// One kernel (indexer_topk_kernel), grid (chunk, sequence), 16 warps per CTA.  Scoring is
+// warp-specialised: warp 12 streams 256-entry tiles of key codes with TMA tensor copies (32-byte
+// swizzle, the MMA's canonical K-major layout) and their scales with bulk copies into a 4-stage
+// mbarrier ring; warp 13 owns 128 columns of tensor memory and issues two MMAs per tile into
+// one of 4 accumulator slots; warpgroups 0..2 take turns reading a slot back (tcgen05.ld, one
+// thread per TMEM lane = two entries), forming the 32-bit order keys in shared memory and a
+// histogram of their top 11 bits.  The CTA then selects its chunk's top min(k, chunk) -- threshold
 // bin from the histogram, one pass to count and collect that bin's candidates, a radix
 // select among the candidates only, one pass to emit in index order -- written as a run.  The runs are then merged by a tree inside the same kernel:
 // the last CTA of a group of G runs to finish (an atomic arrival counter; nothing ever waits)
@@ -28,15 +29,26 @@
 // level; the last run is the answer, written in ascending index order and -1 padded.
 // Selecting the top k of a union of per-part top-k sets is exact under the total order
 // (score desc, index asc), because every global top-k entry is in its part's top k.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "csld_internal.cuh"
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 namespace csld {
 
 constexpr int kIdxThreads = 512;
 constexpr int kIdxWarps = kIdxThreads / 32;
-constexpr int kIdxTile = 512;          // entries per pipeline stage (32 per warp)
-constexpr int kIdxStages = 3;
+constexpr int kIdxTile = 256;          // entries per pipeline stage: two 128-row MMAs
+constexpr int kIdxStages = 4;
+constexpr int kIdxEpiGroups = 3;       // epilogue warpgroups: warps 0..11
+constexpr int kIdxProducerWarp = 12;   // issues the tensor / bulk copies
+constexpr int kIdxMmaWarp = 13;        // owns the tensor memory, issues the MMAs
+constexpr uint32_t kIdxTmemCols = 128; // accumulator slot s = columns 16s..16s+15; scale factors
+constexpr uint32_t kIdxSfCol = 64;     // columns 64..71 (A) and 72..79 (B)
+constexpr uint32_t kIdxIdesc = idesc_mxf4_m128(8);
 constexpr int kIdxMaxChunk = 8192;     // keys a CTA holds (chunk, or runs being merged)
 constexpr int kIdxMaxGroup = 64;       // runs merged by one CTA
 constexpr int kIdxMaxLevels = 4;
@@ -44,11 +56,12 @@ constexpr int kBinShift = 21;          // histogram bin = top 11 bits of the ord
 constexpr int kBins = 1 << (32 - kBinShift);
 constexpr int kRadixBits = 11;
 constexpr int kRadixBins = 1 << kRadixBits;
+constexpr int kIdxSmemAlign = 1024;    // swizzled operand tiles start on 1024-byte boundaries
 
 struct IdxSmem {
     union {
         struct {
-            uint8_t codes[kIdxStages][kIdxTile * kIkey];
+            uint8_t codes[kIdxStages][kIdxTile * kIkey];   // key codes, K-major 32-byte swizzle
             float scales[kIdxStages][kIdxTile * 2];
         } pipe;                        // key stream ring (scoring)
         struct {
@@ -56,18 +69,25 @@ struct IdxSmem {
             uint16_t pos[kIdxMaxChunk];
         } cand;                        // threshold-bin candidates (selection)
     } u;
+    alignas(256) uint8_t bq[8 * kIkey];   // query operand (B): 8 rows x 32 bytes, swizzled
     uint32_t keys[kIdxMaxChunk];       // order keys of the chunk, or of the runs being merged
     uint32_t hist[kBins];              // top-11-bit histogram of keys[]
     uint32_t rhist[kRadixBins];        // radix passes over the candidates
     uint32_t wgt[kIdxWarps], wsel[kIdxWarps], weq[kIdxWarps], wbase[kIdxWarps], weqb[kIdxWarps];
     uint32_t red[2 * kIdxWarps];
     int32_t offs[kIdxMaxGroup + 1];
-    float qscale[8];                   // [group*4 + head] * 0.25
-    uint64_t full[kIdxStages];
+    float qscale[8];                   // [group*4 + head]
+    uint64_t full[kIdxStages];         // stage landed (copies)
+    uint64_t empty[kIdxStages];        // stage and accumulator slot consumed (epilogue)
+    uint64_t accf[kIdxStages];         // accumulator slot written (MMA commit)
+    uint64_t drain;
+    uint32_t tmem_base;
+    int32_t n_issued, n_mma, fail;
     uint32_t sel[4];                   // bin / threshold results
     uint32_t ncand;
     int32_t last;
 };
+static_assert(sizeof(((IdxSmem*)0)->u.pipe) <= sizeof(((IdxSmem*)0)->u.cand), "pipe fits the candidate area");
 
 // ------------------------------------------------------------------------------------------
 // Block-level helpers (512 threads).
@@ -342,15 +362,15 @@ static IdxTree tree_layout(int B, int n_chunks, int kc, int k, int group, uint8_
 // ------------------------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
-    const uint8_t* __restrict__ ikeys, const float* __restrict__ iscales, int64_t cap,
+__global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
+    const __grid_constant__ CUtensorMap kmap, const float* __restrict__ iscales, int64_t cap,
     const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
     const float* __restrict__ head_w, int chunk, int kc, int k, IdxTree tree,
     int32_t* __restrict__ topk_out, int32_t* err) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    IdxSmem& sm = *reinterpret_cast<IdxSmem*>(smem_raw);
+    IdxSmem& sm = *reinterpret_cast<IdxSmem*>(
+        smem_raw + ((kIdxSmemAlign - (smem_u32(smem_raw) & (kIdxSmemAlign - 1))) & (kIdxSmemAlign - 1)));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, cq = lane & 3;
     const int b = blockIdx.y, ch = blockIdx.x;
 
     int64_t n_b = seq_len[b];
@@ -362,151 +382,172 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_topk_kernel(
     for (int i = tid; i < kBins; i += blockDim.x) sm.hist[i] = 0u;
     bool chunk_ok = true;
     if (cn > 0) {
-        // --- query: FP4 codes doubled as int8, in the MMA's B layout ----------------------
-        // B column n (= g): n < 4 -> head n over group 0; n >= 4 -> head n-4 over group 1.
-        // K order inside a group: MMA k = 4c+i <-> dim 8c+i, k = 16+4c+i <-> dim 8c+4+i.
-        uint32_t bq0, bq1;
-        {
-            const int h = g & 3, grp = g >> 2;
-            const float* qv = q_idx + ((size_t)b * kIdxHeads + h) * kIdxDim + 32 * grp;
-            float amax = 0.f;
-            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[i]));
-            const float sg = fp4_group_scale(amax);
-            const float inv = 1.0f / sg;   // exact: a power of two
-            if (warp == 0 && cq == 0) sm.qscale[grp * 4 + h] = sg;
-            uint32_t w0 = 0u, w1 = 0u;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t c_lo = e2m1_code(qv[8 * cq + i] * inv);
-                const uint32_t c_hi = e2m1_code(qv[8 * cq + 4 + i] * inv);
-                const int v_lo = static_cast<int>(prmt(kTwiceE2M1Lo, kTwiceE2M1Hi, c_lo & 7u) & 0xFFu) *
-                                 ((c_lo & 8u) ? -1 : 1);
-                const int v_hi = static_cast<int>(prmt(kTwiceE2M1Lo, kTwiceE2M1Hi, c_hi & 7u) & 0xFFu) *
-                                 ((c_hi & 8u) ? -1 : 1);
-                w0 |= (static_cast<uint32_t>(v_lo) & 0xFFu) << (8 * i);
-                w1 |= (static_cast<uint32_t>(v_hi) & 0xFFu) << (8 * i);
-            }
-            bq0 = w0;
-            bq1 = w1;
-        }
-        // group-0 MMAs see columns 0..3 only, group-1 MMAs columns 4..7 only
-        const bool col_grp1 = g >= 4;
-        const uint32_t b00 = col_grp1 ? 0u : bq0, b01 = col_grp1 ? 0u : bq1;
-        const uint32_t b10 = col_grp1 ? bq0 : 0u, b11 = col_grp1 ? bq1 : 0u;
-        auto neg4 = [](uint32_t v) -> uint32_t {   // bytewise negation (|values| <= 12)
-            uint32_t r = 0u;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) r |= ((0u - ((v >> (8 * i)) & 0xFFu)) & 0xFFu) << (8 * i);
-            return r;
-        };
-        const uint32_t n00 = neg4(b00), n01 = neg4(b01), n10 = neg4(b10), n11 = neg4(b11);
-        const float w0 = head_w[b * kIdxHeads + 0], w1 = head_w[b * kIdxHeads + 1];
-        const float w2 = head_w[b * kIdxHeads + 2], w3 = head_w[b * kIdxHeads + 3];
-
+        const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
+        volatile int32_t* fail = &sm.fail;
         if (tid == 0) {
-            for (int s = 0; s < kIdxStages; ++s) mbar_init(&sm.full[s], 1);
+            for (int s = 0; s < kIdxStages; ++s) {
+                mbar_init(&sm.full[s], 1);
+                mbar_init(&sm.empty[s], 4);          // the 4 warps of the epilogue warpgroup
+                mbar_init(&sm.accf[s], 1);
+            }
+            mbar_init(&sm.drain, 1);
+            sm.fail = 0;
+            sm.n_issued = 0;
+            sm.n_mma = 0;
             fence_barrier_init();
         }
-        __syncthreads();
-        // query group scales of the two heads this lane finishes
-        const int hp = (cq & 1) * 2;
-        const float qs0a = sm.qscale[hp], qs0b = sm.qscale[hp + 1];
-        const float qs1a = sm.qscale[4 + hp], qs1b = sm.qscale[4 + hp + 1];
-
-        const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
-        const uint8_t* kbase = ikeys + ((size_t)b * cap + (size_t)c0) * kIkey;
-        const float* sbase = iscales + ((size_t)b * cap + (size_t)c0) * 2;
-        auto issue = [&](int tile) {
-            const int s = tile % kIdxStages;
-            const int nt = min(kIdxTile, cn - tile * kIdxTile);
-            const int nt2 = (nt + 1) & ~1;   // scales copy: a multiple of 16 bytes (cap is even)
-            const uint32_t cb = static_cast<uint32_t>(nt) * kIkey;
-            const uint32_t sb = static_cast<uint32_t>(nt2) * 8u;
-            mbar_arrive_expect_tx(&sm.full[s], cb + sb);
-            bulk_g2s(sm.u.pipe.codes[s], kbase + (size_t)tile * kIdxTile * kIkey, cb, &sm.full[s]);
-            bulk_g2s(sm.u.pipe.scales[s], sbase + (size_t)tile * kIdxTile * 2, sb, &sm.full[s]);
-        };
-        if (tid == 0)
-            for (int t = 0; t < min(n_tiles, kIdxStages); ++t) issue(t);
-
-        int consumed = 0;
-        bool ok = true;
-        for (int tile = 0; tile < n_tiles; ++tile) {
-            const int s = tile % kIdxStages;
-            const bool landed = mbar_wait(&sm.full[s], (tile / kIdxStages) & 1);
-            if (__syncthreads_or(!landed)) {
-                ok = false;
-                break;
+        if (warp == kIdxMmaWarp) {
+            tmem_alloc(&sm.tmem_base, kIdxTmemCols);
+            tmem_relinquish();
+        }
+        if (warp == kIdxProducerWarp && lane == 0) tma_prefetch_map(&kmap);
+        // --- query operand: FP4 codes in the MMA's B layout (8 rows x 32 bytes, 32-byte swizzle)
+        // Row n is head n & 3 over group n >> 2; the row's other 32-element group is zero, so
+        // every output column is one exact group dot.  Thread t writes bytes 4j..4j+3 of row n.
+        if (tid < 64) {
+            const int n = tid >> 3, j = tid & 7, h = n & 3, grp = n >> 2;
+            const float* qv = q_idx + ((size_t)b * kIdxHeads + h) * kIdxDim;
+            float amax = 0.f;
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[32 * grp + i]));
+            const float sg = fp4_group_scale(amax);
+            const float inv = 1.0f / sg;   // exact: a power of two
+            uint32_t word = 0u;
+            if ((j >> 2) == grp) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) word |= e2m1_code(qv[8 * j + i] * inv) << (4 * i);
             }
-            consumed = tile + 1;
-            const uint8_t* cs = sm.u.pipe.codes[s];
-            const float* ss = sm.u.pipe.scales[s];
+            const int half = (j >> 2) ^ ((n >> 2) & 1);
+            *reinterpret_cast<uint32_t*>(sm.bq + n * kIkey + half * 16 + (j & 3) * 4) = word;
+            if (j == 0) sm.qscale[grp * 4 + h] = sg;
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        const uint32_t tmem = sm.tmem_base;
+        if (warp < 4) {   // unit block-scale factors (UE8M0 0x7F = 2^0) for A and B, every lane
+            tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kIdxSfCol, 0x7F7F7F7Fu);
+            tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kIdxSfCol + 8, 0x7F7F7F7Fu);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        const float* sbase = iscales + ((size_t)b * cap + (size_t)c0) * 2;
+        if (warp == kIdxProducerWarp) {
+            // --- producer: key tile (TMA, swizzled) + its scales (bulk copy) per stage -------
+            if (lane == 0) {
+                int t = 0;
+                for (; t < n_tiles; ++t) {
+                    const int s = t % kIdxStages;
+                    if (*fail) break;
+                    if (t >= kIdxStages && !mbar_wait(&sm.empty[s], ((t / kIdxStages) - 1) & 1)) break;
+                    const int nt = min(kIdxTile, cn - t * kIdxTile);
+                    const uint32_t sb = static_cast<uint32_t>((nt + 1) & ~1) * 8u;   // cap is even
+                    mbar_arrive_expect_tx(&sm.full[s], kIdxTile * kIkey + sb);
+                    tma_load_3d(sm.u.pipe.codes[s], &kmap, 0, static_cast<int>(c0) + t * kIdxTile, b, &sm.full[s]);
+                    bulk_g2s(sm.u.pipe.scales[s], sbase + (size_t)t * kIdxTile * 2, sb, &sm.full[s]);
+                }
+                sm.n_issued = t;
+                if (t < n_tiles) *fail = 1;
+            }
+        } else if (warp == kIdxMmaWarp) {
+            // --- MMA issuer: two 128-row block-scaled FP4 MMAs per tile into accumulator slot s
+            if (lane == 0) {
+                const uint64_t bdesc = smem_desc_kmajor_sw32(sm.bq);
+                const uint32_t sfa = tmem + kIdxSfCol, sfb = tmem + kIdxSfCol + 8;
+                int t = 0;
+                for (; t < n_tiles; ++t) {
+                    const int s = t % kIdxStages;
+                    if (*fail || !mbar_wait(&sm.full[s], (t / kIdxStages) & 1)) break;
+                    tc_fence_after();
+                    const uint32_t d = tmem + 16u * static_cast<uint32_t>(s);
+                    umma_mxf4(d, smem_desc_kmajor_sw32(sm.u.pipe.codes[s]), bdesc, kIdxIdesc, sfa, sfb, 0u);
+                    umma_mxf4(d + 8u, smem_desc_kmajor_sw32(sm.u.pipe.codes[s] + 128 * kIkey), bdesc, kIdxIdesc,
+                              sfa, sfb, 0u);
+                    umma_commit(&sm.accf[s]);
+                }
+                sm.n_mma = t;
+                if (t < n_tiles) *fail = 1;
+            }
+        } else if (warp < 4 * kIdxEpiGroups) {
+            // --- epilogue: warpgroup wg finishes tiles wg, wg + 3, ...; thread = TMEM lane m
+            // holds entries m and 128 + m of the tile: columns 0..3 / 4..7 their group-0 /
+            // group-1 dots of heads 0..3 (8..15 for entry 128 + m), each exactly I_g / 4.
+            const int wg = warp >> 2, quad = warp & 3;
+            const int m = 32 * quad + lane;
+            const uint32_t lane_addr = tmem + ((32u * quad) << 16);
+            float qsc[8];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int rA = 32 * warp + 16 * half + g, rB = rA + 8;
-                const uint32_t kA0 = *reinterpret_cast<const uint32_t*>(cs + rA * kIkey + 4 * cq);
-                const uint32_t kB0 = *reinterpret_cast<const uint32_t*>(cs + rB * kIkey + 4 * cq);
-                const uint32_t kA1 = *reinterpret_cast<const uint32_t*>(cs + rA * kIkey + 16 + 4 * cq);
-                const uint32_t kB1 = *reinterpret_cast<const uint32_t*>(cs + rB * kIkey + 16 + 4 * cq);
-                // positive and negative magnitude planes accumulate separately (two MMA chains)
-                int accp[4] = {0, 0, 0, 0}, accn[4] = {0, 0, 0, 0};
-                auto lut = [](uint32_t sel) { return prmt(kTwiceE2M1Lo, kTwiceE2M1Hi, sel); };
-                const uint32_t nA0 = kA0 ^ 0x88888888u, nB0 = kB0 ^ 0x88888888u;
-                const uint32_t nA1 = kA1 ^ 0x88888888u, nB1 = kB1 ^ 0x88888888u;
-                mma_s8(accp, lut(kA0), lut(kB0), lut(kA0 >> 16), lut(kB0 >> 16), b00, b01);
-                mma_s8(accn, lut(nA0), lut(nB0), lut(nA0 >> 16), lut(nB0 >> 16), n00, n01);
-                mma_s8(accp, lut(kA1), lut(kB1), lut(kA1 >> 16), lut(kB1 >> 16), b10, b11);
-                mma_s8(accn, lut(nA1), lut(nB1), lut(nA1 >> 16), lut(nB1 >> 16), n10, n11);
-                int acc[4];
+            for (int i = 0; i < 8; ++i) qsc[i] = sm.qscale[i];
+            const float w0 = head_w[b * kIdxHeads + 0], w1 = head_w[b * kIdxHeads + 1];
+            const float w2 = head_w[b * kIdxHeads + 2], w3 = head_w[b * kIdxHeads + 3];
+            for (int t = wg; t < n_tiles; t += kIdxEpiGroups) {
+                const int s = t % kIdxStages;
+                const bool landed = !*fail && mbar_wait(&sm.accf[s], (t / kIdxStages) & 1);
+                if (!__all_sync(0xffffffffu, landed)) {
+                    if (lane == 0) *fail = 1;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(lane_addr + 16u * static_cast<uint32_t>(s), r);
+                tmem_ld_wait();
+                const float2* ss = reinterpret_cast<const float2*>(sm.u.pipe.scales[s]);
 #pragma unroll
-                for (int r = 0; r < 4; ++r) acc[r] = accp[r] + accn[r];
-                // acc: (row g, cols 2cq, 2cq+1), (row g+8, same).  cq < 2: group-0 dots of
-                // heads 2cq, 2cq+1; cq >= 2: group-1 dots of heads 2(cq-2), 2(cq-2)+1.
-                const bool lo = cq < 2;
-                const int send0 = lo ? acc[2] : acc[0], send1 = lo ? acc[3] : acc[1];
-                const int got0 = __shfl_xor_sync(0xffffffffu, send0, 2);
-                const int got1 = __shfl_xor_sync(0xffffffffu, send1, 2);
-                const int row = lo ? rA : rB;
-                const int i0a = lo ? acc[0] : got0, i0b = lo ? acc[1] : got1;
-                const int i1a = lo ? got0 : acc[2], i1b = lo ? got1 : acc[3];
-                const float ks0 = ss[2 * row], ks1 = ss[2 * row + 1];
-                // d = fma(I1, s1, I0*s0) with s_g = (qscale_g * kscale_g) * 0.25
-                const float s0a = __fmul_rn(__fmul_rn(qs0a, ks0), 0.25f), s1a = __fmul_rn(__fmul_rn(qs1a, ks1), 0.25f);
-                const float s0b = __fmul_rn(__fmul_rn(qs0b, ks0), 0.25f), s1b = __fmul_rn(__fmul_rn(qs1b, ks1), 0.25f);
-                const float da = __fmaf_rn(static_cast<float>(i1a), s1a, __fmul_rn(static_cast<float>(i0a), s0a));
-                const float db = __fmaf_rn(static_cast<float>(i1b), s1b, __fmul_rn(static_cast<float>(i0b), s0b));
-                const float r0 = da > 0.f ? da : 0.f, r1 = db > 0.f ? db : 0.f;
-                const float r2 = __shfl_xor_sync(0xffffffffu, r0, 1);
-                const float r3 = __shfl_xor_sync(0xffffffffu, r1, 1);
-                if ((cq & 1) == 0) {
-                    float e = __fmul_rn(w0, r0);
-                    e = __fmaf_rn(w1, r1, e);
-                    e = __fmaf_rn(w2, r2, e);
-                    e = __fmaf_rn(w3, r3, e);
-                    const int li = tile * kIdxTile + row;
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int e = 128 * hf + m;
+                    const float2 ks = ss[e];
+                    float rr[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        // d = fma(I1, s1, I0*s0) with s_g = (qscale_g * kscale_g) * 0.25
+                        const float i0 = __fmul_rn(__uint_as_float(r[8 * hf + h]), 4.0f);
+                        const float i1 = __fmul_rn(__uint_as_float(r[8 * hf + 4 + h]), 4.0f);
+                        const float s0 = __fmul_rn(__fmul_rn(qsc[h], ks.x), 0.25f);
+                        const float s1 = __fmul_rn(__fmul_rn(qsc[4 + h], ks.y), 0.25f);
+                        const float d = __fmaf_rn(i1, s1, __fmul_rn(i0, s0));
+                        rr[h] = d > 0.f ? d : 0.f;
+                    }
+                    float sc = __fmul_rn(w0, rr[0]);
+                    sc = __fmaf_rn(w1, rr[1], sc);
+                    sc = __fmaf_rn(w2, rr[2], sc);
+                    sc = __fmaf_rn(w3, rr[3], sc);
+                    const int li = t * kIdxTile + e;
                     if (li < cn) {
-                        const uint32_t key = score_key(e);
+                        const uint32_t key = score_key(sc);
                         sm.keys[li] = key;
                         atomicAdd(&sm.hist[key >> kBinShift], 1u);
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.empty[s]);   // stage s and accumulator slot s free
             }
-            __syncthreads();   // stage s fully consumed
-            if (tid == 0 && tile + kIdxStages < n_tiles) issue(tile + kIdxStages);
         }
-        chunk_ok = ok;
-        if (!ok) {
-            // A copy did not land in time: record it, drain what is in flight (bounded), and
-            // publish this chunk as empty so the merge tree still completes.
-            if (tid == 0) {
+        tc_fence_before();
+        __syncthreads();
+        chunk_ok = (sm.fail == 0);
+        if (!chunk_ok) {
+            // A copy or an MMA did not complete in time: record it, let the copies in flight
+            // land and the MMAs in flight finish (bounded waits) before the shared and tensor
+            // memory are reused, and publish this chunk as empty so the merge tree completes.
+            if (warp == kIdxMmaWarp && lane == 0) {
                 dev_error(err, CSLD_DEVERR_TIMEOUT);
-                for (int t = consumed; t < min(n_tiles, consumed + kIdxStages); ++t)
+                for (int t = sm.n_mma; t < sm.n_issued; ++t)
                     (void)mbar_wait(&sm.full[t % kIdxStages], (t / kIdxStages) & 1);
+                umma_commit(&sm.drain);
+                (void)mbar_wait(&sm.drain, 0);
             }
+            __syncthreads();
+        }
+        if (warp == kIdxMmaWarp) {
+            tc_fence_after();
+            tmem_dealloc(tmem, kIdxTmemCols);
         }
     }
     __syncthreads();
-
     // --- selection and the merge tree ------------------------------------------------------
     int n = (cn > 0 && chunk_ok) ? cn : 0;   // a timed-out chunk publishes nothing
     int level = 0, run = ch;
@@ -637,17 +678,44 @@ IndexerPlan indexer_plan(int B, int64_t cap, int k, int num_sms) {
     return p;
 }
 
+// cuTensorMapEncodeTiled from the driver (through the runtime, so nothing links libcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
 cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t cap,
                            const int32_t* seq_len, int ratio, const float* q_idx,
                            const float* head_w, int B, int k, int32_t* topk_out, void* ws,
                            const IndexerPlan& plan, int32_t* err, cudaStream_t stream) {
     size_t bytes = 0;
     IdxTree tree = tree_layout(B, plan.n_chunks, plan.kc, k, plan.group, static_cast<uint8_t*>(ws), &bytes);
-    const size_t smem = sizeof(IdxSmem);
+    // Key codes as a 3-D byte tensor [B][cap][32]; one box = one stage of 256 entries.  Rows
+    // past cap read as zeros (their scores are never used).
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (encode == nullptr) return cudaErrorNotSupported;
+    CUtensorMap kmap;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kIkey), static_cast<cuuint64_t>(cap), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kIkey), static_cast<cuuint64_t>(cap) * kIkey};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kIkey), static_cast<cuuint32_t>(kIdxTile), 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    if (encode(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(ikeys), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(IdxSmem) + kIdxSmemAlign;
     cudaError_t e = set_smem_once(indexer_topk_kernel, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(plan.n_chunks, B);
-    indexer_topk_kernel<<<grid, kIdxThreads, smem, stream>>>(ikeys, iscales, cap, seq_len, ratio,
+    indexer_topk_kernel<<<grid, kIdxThreads, smem, stream>>>(kmap, iscales, cap, seq_len, ratio,
                                                              q_idx, head_w, plan.chunk, plan.kc, k,
                                                              tree, topk_out, err);
     return cudaGetLastError();

@@ -1,0 +1,121 @@
+// Blackwell (sm_100a) tensor-memory, 5th-generation tensor-core and tensor-copy helpers.
+// Internal to libcsld.
+//
+// Conventions used by the callers:
+//  * TMEM addresses are (lane << 16) | column.  A warp may only touch the 32 lanes of its
+//    sub-partition: lanes 32*(warp % 4) .. 32*(warp % 4) + 31.
+//  * tcgen05.mma / tcgen05.commit are issued by one thread; tcgen05.alloc / dealloc / ld / st
+//    are warp-collective (.sync.aligned).
+//  * Shared-memory operands use the K-major, 32-byte-swizzle canonical layout: rows of 32
+//    bytes, 8-row groups of 256 bytes, and inside every group the two 16-byte halves of rows
+//    4..7 exchanged (byte-address bit 4 XOR bit 7).  TMA writes that layout when its tensor
+//    map asks for CU_TENSOR_MAP_SWIZZLE_32B; hand-written operands apply the same XOR.
+#pragma once
+#include <cuda.h>
+#include <stdint.h>
+
+#include "csld_internal.cuh"
+
+namespace csld {
+
+// ---- tensor memory ------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(slot)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+}
+// Order tcgen05 operations around thread synchronisation (barriers, mbarrier waits).
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Make this thread's ordinary shared-memory writes visible to the tensor cores / TMA.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 lanes x 16 columns of 32 bits: thread i gets lane (base lane + i), columns col .. col+15.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Writes v to 8 consecutive columns of the warp's 32 lanes.
+__device__ __forceinline__ void tmem_st_32x32b_x8_fill(uint32_t taddr, uint32_t v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1};"
+                 :: "r"(taddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ---- shared-memory matrix descriptor --------------------------------------------------------
+// K-major operand in the 32-byte-swizzle layout starting at p (256-byte aligned): rows of 32
+// bytes, 8-row groups 256 bytes apart.  Fields: start address >> 4 (bits 0-13), leading byte
+// offset >> 4 (16-29; unused by swizzled K-major layouts whose K fits one row), stride byte
+// offset >> 4 (32-45), descriptor version 1 (46-47), base offset 0, swizzle mode 6 = 32 B
+// (61-63).
+__device__ __forceinline__ uint64_t smem_desc_kmajor_sw32(const void* p) {
+    const uint32_t a = smem_u32(p);
+    uint64_t d = static_cast<uint64_t>((a >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1u) << 16;
+    d |= static_cast<uint64_t>(256u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(6u) << 61;
+    return d;
+}
+
+// Instruction descriptor of the block-scaled FP4 MMA (kind::mxf4): A and B E2M1 (format 1),
+// K-major, UE8M0 scale factors (bit 23), N = n (bits 17-22 hold n / 8), M = 128 (bits 24-28
+// hold M / 16), scale-factor byte selectors 0, dense, K = 64 per instruction.
+__host__ __device__ constexpr uint32_t idesc_mxf4_m128(uint32_t n) {
+    return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
+}
+
+// D[tmem] (=|+=) A x B^T, A 128 x 64 E2M1 and B n x 64 E2M1 from shared memory, each 32-element
+// K block scaled by its UE8M0 factor from TMEM (sfa, sfb), fp32 accumulate.
+__device__ __forceinline__ void umma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// Arrive once on the mbarrier when every tcgen05.mma issued so far by this thread completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(smem_u32(bar)) : "memory");
+}
+
+// ---- tensor (TMA) copies ---------------------------------------------------------------------
+// 3-D tile of the tensor map at element coordinates (x, y, z) -> shared memory, completing the
+// box's bytes on the mbarrier.  x * element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+}  // namespace csld

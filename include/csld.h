@@ -166,7 +166,9 @@ CSLD_API csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint1
  * s_g = (qscale_g * kscale_g) * 0.25.  The min(k, n_b) entries with the largest (score,
  * -index) are written to topk_out[b] in ascending index order, followed by -1 padding.
  *   ikeys [B][cap][32] u8, iscales [B][cap][2] f32, seq_len [B] i32, q_idx [B][4][64] f32,
- *   head_w [B][4] f32, topk_out [B][k] i32.  cap even; ikeys 16-byte aligned; 1 <= k <= 2048.
+ *   head_w [B][4] f32, topk_out [B][k] i32.  cap even, 2 <= cap <= 2^30; ikeys 16-byte
+ *   aligned; 1 <= k <= 2048.  Returns CSLD_ERR_UNSUPPORTED if the driver offers no tensor-map
+ *   encoder (the keys are streamed by tensor copies).
  * Workspace: csld_indexer_workspace_size(B, cap, k) bytes, 256-byte aligned, zero-filled once
  * before its first use (it holds arrival counters that every call leaves at zero again); calls
  * that share one workspace must not overlap on the GPU.  err: device error word or NULL. */
