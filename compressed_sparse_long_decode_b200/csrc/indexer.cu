@@ -15,15 +15,26 @@
 // dot.  The fp32 score then follows a fixed operation order (see the ABI header) using the
 // true scales, so the selection is reproducible bit for bit; order key = (score, -index).
 //
-// One kernel (indexer_topk_kernel), grid (chunk, sequence), 16 warps per CTA.  Scoring is
-// warp-specialised: warp 12 streams 256-entry tiles of key codes with TMA tensor copies (32-byte
-// swizzle, the MMA's canonical K-major layout) and their scales with bulk copies into a 4-stage
-// mbarrier ring; warp 13 owns 128 columns of tensor memory and issues two MMAs per tile into
-// one of 4 accumulator slots; warpgroups 0..2 take turns reading a slot back (tcgen05.ld, one
-// thread per TMEM lane = two entries), forming the 32-bit order keys in shared memory and a
-// histogram of their top 11 bits.  The CTA then selects its chunk's top min(k, chunk) -- threshold
-// bin from the histogram, one pass to count and collect that bin's candidates, a radix
-// select among the candidates only, one pass to emit in index order -- written as a run.  The runs are then merged by a tree inside the same kernel:
+// Scoring (score_chunk, shared by both kernels below) is warp-specialised over 16 warps:
+// warp 12 streams 256-entry tiles of key codes with TMA tensor copies (32-byte swizzle, the
+// MMA's canonical K-major layout) and their scales with bulk copies into an mbarrier ring;
+// warp 13 owns 128 columns of tensor memory and issues two MMAs per tile into one of the
+// accumulator slots; warpgroups 0..2 take turns reading a slot back (tcgen05.ld, one thread
+// per TMEM lane = two entries), forming the 32-bit order keys in shared memory and a histogram
+// of their top 11 bits.
+//
+// Selection, when the whole grid can be resident (indexer_topk_coop_kernel, cooperative
+// launch): each sequence is split into `units` ranges, one CTA each, and the CTAs of a sequence
+// run an exact radix select together.  They add their histograms into the sequence's global
+// histogram, meet at a barrier (an arrival counter; every wait is bounded), and each derive the
+// same threshold bin; two more rounds over the next 11 and 10 key bits give the exact
+// threshold key and how many keys equal to it are taken (the lowest indices win).  After a
+// last barrier every CTA knows how many selected entries precede its range and writes its own
+// in ascending index order.
+//
+// Otherwise (indexer_topk_kernel): each CTA selects its chunk's top min(k, chunk) -- threshold
+// bin from the histogram, the bin's candidates collected, a radix select among them, an emit in
+// index order -- written as a run, and the runs are merged by a tree inside the same kernel:
 // the last CTA of a group of G runs to finish (an atomic arrival counter; nothing ever waits)
 // loads the group's runs, selects their top min(k, ...) and publishes one run for the next
 // level; the last run is the answer, written in ascending index order and -1 padded.
@@ -42,14 +53,17 @@ namespace csld {
 constexpr int kIdxThreads = 512;
 constexpr int kIdxWarps = kIdxThreads / 32;
 constexpr int kIdxTile = 256;          // entries per pipeline stage: two 128-row MMAs
-constexpr int kIdxStages = 4;
+constexpr int kIdxStages = 4;          // ring depth of the merge-tree kernel (shares the candidate area)
+constexpr int kCoopStages = 12;        // ring depth of the cooperative kernel (one CTA per SM)
+constexpr int kMaxStages = 12;
 constexpr int kIdxEpiGroups = 3;       // epilogue warpgroups: warps 0..11
 constexpr int kIdxProducerWarp = 12;   // issues the tensor / bulk copies
 constexpr int kIdxMmaWarp = 13;        // owns the tensor memory, issues the MMAs
-constexpr uint32_t kIdxTmemCols = 128; // accumulator slot s = columns 16s..16s+15; scale factors
-constexpr uint32_t kIdxSfCol = 64;     // columns 64..71 (A) and 72..79 (B)
+// Tensor memory: accumulator slot s = columns 16s..16s+15; the last 16 allocated columns hold
+// the unit scale factors (8 for A, 8 for B).  128 columns for the 4-slot ring, 256 for 12.
 constexpr uint32_t kIdxIdesc = idesc_mxf4_m128(8);
-constexpr int kIdxMaxChunk = 8192;     // keys a CTA holds (chunk, or runs being merged)
+constexpr int kIdxMaxChunk = 8192;     // keys a merge-tree CTA holds (chunk, or runs being merged)
+constexpr int kCoopMaxRange = 16384;   // keys a cooperative CTA holds
 constexpr int kIdxMaxGroup = 64;       // runs merged by one CTA
 constexpr int kIdxMaxLevels = 4;
 constexpr int kBinShift = 21;          // histogram bin = top 11 bits of the order key
@@ -57,6 +71,19 @@ constexpr int kBins = 1 << (32 - kBinShift);
 constexpr int kRadixBits = 11;
 constexpr int kRadixBins = 1 << kRadixBits;
 constexpr int kIdxSmemAlign = 1024;    // swizzled operand tiles start on 1024-byte boundaries
+constexpr int kCoopSeqWords = 2 * kBins + 1024;   // per sequence: three levels of histograms
+
+// Scoring control block: query operand, ring barriers, tensor-memory base, progress.
+struct ScoreCtl {
+    alignas(256) uint8_t bq[8 * kIkey];   // query operand (B): 8 rows x 32 bytes, swizzled
+    float qscale[8];                   // [group*4 + head]
+    uint64_t full[kMaxStages];         // stage landed (copies)
+    uint64_t empty[kMaxStages];        // stage and accumulator slot consumed (epilogue)
+    uint64_t accf[kMaxStages];         // accumulator slot written (MMA commit)
+    uint64_t drain;
+    uint32_t tmem_base;
+    int32_t n_issued, n_mma, fail;
+};
 
 struct IdxSmem {
     union {
@@ -69,25 +96,30 @@ struct IdxSmem {
             uint16_t pos[kIdxMaxChunk];
         } cand;                        // threshold-bin candidates (selection)
     } u;
-    alignas(256) uint8_t bq[8 * kIkey];   // query operand (B): 8 rows x 32 bytes, swizzled
+    ScoreCtl ctl;
     uint32_t keys[kIdxMaxChunk];       // order keys of the chunk, or of the runs being merged
     uint32_t hist[kBins];              // top-11-bit histogram of keys[]
     uint32_t rhist[kRadixBins];        // radix passes over the candidates
-    uint32_t wgt[kIdxWarps], wsel[kIdxWarps], weq[kIdxWarps], wbase[kIdxWarps], weqb[kIdxWarps];
-    uint32_t red[2 * kIdxWarps];
+    uint32_t red[3 * kIdxWarps];
     int32_t offs[kIdxMaxGroup + 1];
-    float qscale[8];                   // [group*4 + head]
-    uint64_t full[kIdxStages];         // stage landed (copies)
-    uint64_t empty[kIdxStages];        // stage and accumulator slot consumed (epilogue)
-    uint64_t accf[kIdxStages];         // accumulator slot written (MMA commit)
-    uint64_t drain;
-    uint32_t tmem_base;
-    int32_t n_issued, n_mma, fail;
     uint32_t sel[4];                   // bin / threshold results
-    uint32_t ncand;
     int32_t last;
 };
 static_assert(sizeof(((IdxSmem*)0)->u.pipe) <= sizeof(((IdxSmem*)0)->u.cand), "pipe fits the candidate area");
+
+struct CoopSmem {
+    uint8_t codes[kCoopStages][kIdxTile * kIkey];
+    float scales[kCoopStages][kIdxTile * 2];
+    ScoreCtl ctl;
+    uint32_t keys[kCoopMaxRange];      // order keys of this CTA's range
+    uint32_t hist[kBins];              // this CTA's histograms of radix levels 1, 2, 3
+    uint32_t hist2[kBins];
+    uint32_t hist3[1024];
+    uint32_t red[3 * kIdxWarps];
+    uint32_t sel[4];
+    int32_t fail, last;
+};
+static_assert(sizeof(((CoopSmem*)0)->codes) >= kCoopMaxRange * 4, "candidate regions fit the idle copy ring");
 
 // ------------------------------------------------------------------------------------------
 // Block-level helpers (512 threads).
@@ -181,17 +213,49 @@ __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint3
     return prefix;
 }
 
+// Warp-level exclusive prefix over the 16 warps of the block: v is the warp's value (uniform in
+// the warp); returns the sum over lower warps, *total the block's sum.  red: kIdxWarps words
+// not touched by anyone else until the next barrier.
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t* red, uint32_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    uint32_t before = 0u, all = 0u;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) {
+        const uint32_t r = red[w];
+        before += (w < warp) ? r : 0u;
+        all += r;
+    }
+    *total = all;
+    return before;
+}
+
+// Histogram increment with the lanes of a warp that hit the same bin combined into one atomic
+// (the keys being merged crowd into few bins).  Every lane of the warp must call it.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
+    const uint32_t same = __match_any_sync(0xffffffffu, valid ? bin : 0xFFFFFFFFu);
+    const int lane = threadIdx.x & 31;
+    if (valid && lane == __ffs(same) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(same)));
+}
+
 // Selects the top `want` of sm.keys[0..n) under (key desc, position asc) and emits them in
 // position order: emit(out_pos, position).  Requires sm.hist = histogram of key >> kBinShift.
+// Warp w owns positions 512w .. 512w+511, read 32 at a time (lane = position mod 32), so warp
+// order then step order then lane order is position order; every count comes from ballots and
+// two prefix sums over the 16 warps: no atomics and no dependent round trips per key.
 template <typename Emit>
 __device__ void select_emit(IdxSmem& sm, int n, int want, Emit emit) {
+    constexpr int kSeg = kIdxMaxChunk / kIdxWarps;     // 512 positions per warp
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t lt = (1u << lane) - 1u;
-    const int seg = ((n + kIdxWarps - 1) / kIdxWarps + 31) & ~31;
-    const int i0 = min(n, warp * seg), i1 = min(n, i0 + seg);
+    const int i0 = warp * kSeg;
+    const int steps = max(0, min(kSeg, n - i0) + 31) >> 5;
     if (want >= n) {                                   // everything is selected
-        for (int base = i0; base < i1; base += 32)
-            if (base + lane < i1) emit(base + lane, base + lane);
+        for (int s = 0; s < steps; ++s) {
+            const int i = i0 + 32 * s + lane;
+            if (i < n) emit(i, i);
+        }
         __syncthreads();
         return;
     }
@@ -209,15 +273,11 @@ __device__ void select_emit(IdxSmem& sm, int n, int want, Emit emit) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        if (lane == 31) sm.red[warp] = incl;
-        if (tid == 0) sm.ncand = 0u;
-        __syncthreads();
-        uint32_t wb = 0u;
-        for (int w = 0; w < warp; ++w) wb += sm.red[w];
-        incl += wb;
-        const uint32_t excl = incl - tot;
+        uint32_t all;
+        const uint32_t wb = warp_excl_scan(__shfl_sync(0xffffffffu, incl, 31), sm.red, &all);
+        const uint32_t excl = wb + incl - tot;
         const uint32_t W = static_cast<uint32_t>(want);
-        if (excl < W && incl >= W) {
+        if (excl < W && excl + tot >= W) {
             uint32_t run = excl;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -229,87 +289,254 @@ __device__ void select_emit(IdxSmem& sm, int n, int want, Emit emit) {
                 run += c[q];
             }
         }
-        if (tid < kIdxWarps) {
-            sm.wsel[tid] = 0u;
-            sm.weq[tid] = 0u;
-        }
         __syncthreads();
     }
     const uint32_t beta = sm.sel[0], need = sm.sel[1];
-    // 2) pass 1: per-warp count above the bin; collect the bin's candidates with positions
-    uint32_t gt = 0u;
-    for (int base = i0; base < i1; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = i < i1 ? sm.keys[i] : 0u;
+    // 2) per warp: keys above the bin and keys in it; the bin's candidates are then written
+    //    compactly in position order
+    uint32_t gt = 0u, nc = 0u;
+    for (int s = 0; s < steps; ++s) {
+        const int i = i0 + 32 * s + lane;
+        const uint32_t bin = i < n ? sm.keys[i] >> kBinShift : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, i < n && bin > beta));
+        nc += __popc(__ballot_sync(0xffffffffu, i < n && bin == beta));
+    }
+    uint32_t P;
+    uint32_t at = warp_excl_scan(nc, sm.red + kIdxWarps, &P);
+    for (int s = 0; s < steps && nc; ++s) {
+        const int i = i0 + 32 * s + lane;
+        const uint32_t key = i < n ? sm.keys[i] : 0u;
+        const bool in = i < n && (key >> kBinShift) == beta;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        if (in) {
+            const uint32_t slot = at + __popc(m & lt);
+            sm.u.cand.key[slot] = key;
+            sm.u.cand.pos[slot] = static_cast<uint16_t>(i);
+        }
+        at += __popc(m);
+    }
+    __syncthreads();
+    // 3) exact threshold among the candidates: all keys > thr and the first take_eq == thr
+    uint32_t thr = 0u, take_eq = P;
+    if (need < P)
+        thr = radix_select([&](int c) { return sm.u.cand.key[c]; }, static_cast<int>(P), static_cast<int>(need),
+                           sm.rhist, sm.sel + 2, sm.red, &take_eq);
+    // 4) selected keys before this warp: above-threshold ones plus the equal ones that fit
+    uint32_t ga = gt, eq = 0u;
+    for (int s = 0; s < steps && nc; ++s) {
+        const int i = i0 + 32 * s + lane;
+        const uint32_t key = i < n ? sm.keys[i] : 0u;
+        const bool in = i < n && (key >> kBinShift) == beta;
+        ga += __popc(__ballot_sync(0xffffffffu, in && key > thr));
+        eq += __popc(__ballot_sync(0xffffffffu, in && key == thr));
+    }
+    uint32_t tot2;
+    const uint32_t pre = warp_excl_scan((ga << 16) | eq, sm.red + 2 * kIdxWarps, &tot2);   // counts < 2^16
+    uint32_t eq_seen = pre & 0xFFFFu;
+    uint32_t pos = (pre >> 16) + min(eq_seen, take_eq);
+    // 5) emit in position order
+    for (int s = 0; s < steps; ++s) {
+        const int i = i0 + 32 * s + lane;
+        const uint32_t key = i < n ? sm.keys[i] : 0u;
         const uint32_t bin = key >> kBinShift;
-        gt += __popc(__ballot_sync(0xffffffffu, i < i1 && bin > beta));
-        const uint32_t cm = __ballot_sync(0xffffffffu, i < i1 && bin == beta);
-        if (cm) {
-            uint32_t slot = 0u;
-            if (lane == 0) slot = atomicAdd(&sm.ncand, static_cast<uint32_t>(__popc(cm)));
-            slot = __shfl_sync(0xffffffffu, slot, 0);
-            if (i < i1 && bin == beta) {
-                const uint32_t at = slot + __popc(cm & lt);
-                sm.u.cand.key[at] = key;
-                sm.u.cand.pos[at] = static_cast<uint16_t>(i);
-            }
-        }
-    }
-    if (lane == 0) sm.wgt[warp] = gt;
-    __syncthreads();
-    // 3) exact threshold among the candidates
-    const int P = static_cast<int>(sm.ncand);
-    uint32_t thr = 0u, take_eq = static_cast<uint32_t>(P);
-    if (static_cast<int>(need) < P)
-        thr = radix_select([&](int c) { return sm.u.cand.key[c]; }, P, static_cast<int>(need), sm.rhist, sm.sel + 2,
-                           sm.red, &take_eq);
-    // 4) per-warp counts of selected candidates (above the threshold, equal to it)
-    for (int c = tid; c < P; c += blockDim.x) {
-        const uint32_t key = sm.u.cand.key[c];
-        const int w = sm.u.cand.pos[c] / seg;
-        if (key > thr) atomicAdd(&sm.wsel[w], 1u);
-        else if (key == thr) atomicAdd(&sm.weq[w], 1u);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const uint32_t e = lane < kIdxWarps ? sm.weq[lane] : 0u;
-        uint32_t ei = e;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, ei, o);
-            if (lane >= o) ei += y;
-        }
-        const uint32_t eb = ei - e;
-        const uint32_t tw = eb >= take_eq ? 0u : min(e, take_eq - eb);
-        const uint32_t tk = (lane < kIdxWarps ? sm.wgt[lane] + sm.wsel[lane] : 0u) + tw;
-        uint32_t ti = tk;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, ti, o);
-            if (lane >= o) ti += y;
-        }
-        if (lane < kIdxWarps) {
-            sm.wbase[lane] = ti - tk;
-            sm.weqb[lane] = eb;
-        }
-    }
-    __syncthreads();
-    // 5) pass 2: emit in position order
-    uint32_t pos = sm.wbase[warp], eq_seen = sm.weqb[warp];
-    for (int base = i0; base < i1; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = i < i1 ? sm.keys[i] : 0u;
-        const uint32_t bin = key >> kBinShift;
-        const bool inb = i < i1 && bin == beta;
-        const bool veq = inb && key == thr;
+        const bool in = i < n && bin == beta;
+        const bool veq = in && key == thr;
         const uint32_t em = __ballot_sync(0xffffffffu, veq);
-        const bool take = (i < i1 && bin > beta) || (inb && key > thr) || (veq && eq_seen + __popc(em & lt) < take_eq);
+        const bool take = (i < n && bin > beta) || (in && key > thr) || (veq && eq_seen + __popc(em & lt) < take_eq);
         const uint32_t tm = __ballot_sync(0xffffffffu, take);
-        if (take) emit(pos + __popc(tm & lt), i);
+        if (take && pos + __popc(tm & lt) < static_cast<uint32_t>(want)) emit(pos + __popc(tm & lt), i);
         pos += __popc(tm);
         eq_seen += __popc(em);
     }
     __syncthreads();
+}
+
+// Scores entries c0 .. c0+cn-1 (cn >= 1) of sequence b through an S-stage ring: their order
+// keys into keys[0..cn) and their top-11-bit histogram added into hist (zeroed by the caller).
+// Returns false (and records CSLD_DEVERR_TIMEOUT) if a copy or an MMA did not complete in
+// time.  Called by all 512 threads; allocates and frees NCOLS columns of tensor memory.
+template <int S, uint32_t NCOLS>
+__device__ bool score_chunk(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], float (*scales)[kIdxTile * 2],
+                            uint32_t* keys, uint32_t* hist, const CUtensorMap& kmap, const float* iscales,
+                            int64_t cap, int b, int64_t c0, int cn, const float* q_idx, const float* head_w,
+                            int32_t* err) {
+    static_assert(S <= kMaxStages, "ring depth");
+    static_assert(16 * S + 16 <= static_cast<int>(NCOLS), "accumulator slots and scale factors fit");
+    constexpr uint32_t kIdxTmemCols = NCOLS, kIdxSfCol = NCOLS - 16;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
+    volatile int32_t* fail = &ctl.fail;
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&ctl.full[s], 1);
+            mbar_init(&ctl.empty[s], 4);          // the 4 warps of the epilogue warpgroup
+            mbar_init(&ctl.accf[s], 1);
+        }
+        mbar_init(&ctl.drain, 1);
+        ctl.fail = 0;
+        ctl.n_issued = 0;
+        ctl.n_mma = 0;
+        fence_barrier_init();
+    }
+    if (warp == kIdxMmaWarp) {
+        tmem_alloc(&ctl.tmem_base, kIdxTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == kIdxProducerWarp && lane == 0) tma_prefetch_map(&kmap);
+    tc_fence_before();
+    __syncthreads();   // barriers initialised, tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+    const float* sbase = iscales + ((size_t)b * cap + (size_t)c0) * 2;
+    if (warp == kIdxProducerWarp) {
+        // --- producer: key tile (TMA, swizzled) + its scales (bulk copy) per stage -------
+        if (lane == 0) {
+            int t = 0;
+            for (; t < n_tiles; ++t) {
+                const int s = t % S;
+                if (*fail) break;
+                if (t >= S && !mbar_wait(&ctl.empty[s], ((t / S) - 1) & 1)) break;
+                const int nt = min(kIdxTile, cn - t * kIdxTile);
+                const uint32_t sb = static_cast<uint32_t>((nt + 1) & ~1) * 8u;   // cap is even
+                mbar_arrive_expect_tx(&ctl.full[s], kIdxTile * kIkey + sb);
+                tma_load_3d(codes[s], &kmap, 0, static_cast<int>(c0) + t * kIdxTile, b, &ctl.full[s]);
+                bulk_g2s(scales[s], sbase + (size_t)t * kIdxTile * 2, sb, &ctl.full[s]);
+            }
+            ctl.n_issued = t;
+            if (t < n_tiles) *fail = 1;
+        }
+    } else {
+        // --- query operand: FP4 codes in the MMA's B layout (8 rows x 32 bytes, 32-byte
+        // swizzle), prepared while the producer already streams.  Row n is head n & 3 over
+        // group n >> 2; the row's other 32-element group is zero, so every output column is one
+        // exact group dot.  Thread t writes bytes 4j..4j+3 of row n.
+        if (tid < 64) {
+            const int n = tid >> 3, j = tid & 7, h = n & 3, grp = n >> 2;
+            const float4* qv = reinterpret_cast<const float4*>(q_idx + ((size_t)b * kIdxHeads + h) * kIdxDim + 32 * grp);
+            float amax = 0.f;
+            float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;   // dims 8(j&3)..8(j&3)+7 of the group
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 t = __ldg(qv + i);
+                amax = fmaxf(fmaxf(fmaxf(amax, fabsf(t.x)), fmaxf(fabsf(t.y), fabsf(t.z))), fabsf(t.w));
+                if (i == 2 * (j & 3)) lo = t;
+                if (i == 2 * (j & 3) + 1) hi = t;
+            }
+            const float sg = fp4_group_scale(amax);
+            const float inv = 1.0f / sg;   // exact: a power of two
+            uint32_t word = 0u;
+            if ((j >> 2) == grp) {         // dims 8j..8j+7 = group dims 8(j&3)..8(j&3)+7
+                const float x[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) word |= e2m1_code(x[i] * inv) << (4 * i);
+            }
+            const int half = (j >> 2) ^ ((n >> 2) & 1);
+            *reinterpret_cast<uint32_t*>(ctl.bq + n * kIkey + half * 16 + (j & 3) * 4) = word;
+            if (j == 0) ctl.qscale[grp * 4 + h] = sg;
+            fence_proxy_async_smem();
+        }
+        if (warp < 4) {   // unit block-scale factors (UE8M0 0x7F = 2^0) for A and B, every lane
+            tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kIdxSfCol, 0x7F7F7F7Fu);
+            tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kIdxSfCol + 8, 0x7F7F7F7Fu);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        named_barrier(1, kIdxThreads - 32);   // every warp but the producer
+        tc_fence_after();
+        if (warp == kIdxMmaWarp) {
+            // --- MMA issuer: two 128-row block-scaled FP4 MMAs per tile into accumulator slot s
+            if (lane == 0) {
+                const uint64_t bdesc = smem_desc_kmajor_sw32(ctl.bq);
+                const uint32_t sfa = tmem + kIdxSfCol, sfb = tmem + kIdxSfCol + 8;
+                int t = 0;
+                for (; t < n_tiles; ++t) {
+                    const int s = t % S;
+                    if (*fail || !mbar_wait(&ctl.full[s], (t / S) & 1)) break;
+                    tc_fence_after();
+                    const uint32_t d = tmem + 16u * static_cast<uint32_t>(s);
+                    umma_mxf4(d, smem_desc_kmajor_sw32(codes[s]), bdesc, kIdxIdesc, sfa, sfb, 0u);
+                    umma_mxf4(d + 8u, smem_desc_kmajor_sw32(codes[s] + 128 * kIkey), bdesc, kIdxIdesc,
+                              sfa, sfb, 0u);
+                    umma_commit(&ctl.accf[s]);
+                }
+                ctl.n_mma = t;
+                if (t < n_tiles) *fail = 1;
+            }
+        } else if (warp < 4 * kIdxEpiGroups) {
+            // --- epilogue: warpgroup wg finishes tiles wg, wg + 3, ...; thread = TMEM lane m
+            // holds entries m and 128 + m of the tile: columns 0..3 / 4..7 their group-0 /
+            // group-1 dots of heads 0..3 (8..15 for entry 128 + m), each exactly I_g / 4.
+            const int wg = warp >> 2, quad = warp & 3;
+            const int m = 32 * quad + lane;
+            const uint32_t lane_addr = tmem + ((32u * quad) << 16);
+            float qsc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qsc[i] = ctl.qscale[i];
+            const float w0 = head_w[b * kIdxHeads + 0], w1 = head_w[b * kIdxHeads + 1];
+            const float w2 = head_w[b * kIdxHeads + 2], w3 = head_w[b * kIdxHeads + 3];
+            for (int t = wg; t < n_tiles; t += kIdxEpiGroups) {
+                const int s = t % S;
+                const bool landed = !*fail && mbar_wait(&ctl.accf[s], (t / S) & 1);
+                if (!__all_sync(0xffffffffu, landed)) {
+                    if (lane == 0) *fail = 1;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(lane_addr + 16u * static_cast<uint32_t>(s), r);
+                tmem_ld_wait();
+                const float2* ss = reinterpret_cast<const float2*>(scales[s]);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int e = 128 * hf + m;
+                    const float2 ks = ss[e];
+                    float rr[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        // d = fma(I1, s1, I0*s0) with s_g = (qscale_g * kscale_g) * 0.25
+                        const float i0 = __fmul_rn(__uint_as_float(r[8 * hf + h]), 4.0f);
+                        const float i1 = __fmul_rn(__uint_as_float(r[8 * hf + 4 + h]), 4.0f);
+                        const float s0 = __fmul_rn(__fmul_rn(qsc[h], ks.x), 0.25f);
+                        const float s1 = __fmul_rn(__fmul_rn(qsc[4 + h], ks.y), 0.25f);
+                        const float d = __fmaf_rn(i1, s1, __fmul_rn(i0, s0));
+                        rr[h] = d > 0.f ? d : 0.f;
+                    }
+                    float sc = __fmul_rn(w0, rr[0]);
+                    sc = __fmaf_rn(w1, rr[1], sc);
+                    sc = __fmaf_rn(w2, rr[2], sc);
+                    sc = __fmaf_rn(w3, rr[3], sc);
+                    const int li = t * kIdxTile + e;
+                    const uint32_t key = score_key(sc);
+                    if (li < cn) keys[li] = key;
+                    hist_add(hist, key >> kBinShift, li < cn);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl.empty[s]);   // stage s and accumulator slot s free
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    const bool ok = (ctl.fail == 0);
+    if (!ok) {
+        // A copy or an MMA did not complete in time: record it, let the copies in flight
+        // land and the MMAs in flight finish (bounded waits) before the shared and tensor
+        // memory are reused.
+        if (warp == kIdxMmaWarp && lane == 0) {
+            dev_error(err, CSLD_DEVERR_TIMEOUT);
+            for (int t = ctl.n_mma; t < ctl.n_issued; ++t)
+                (void)mbar_wait(&ctl.full[t % S], (t / S) & 1);
+            umma_commit(&ctl.drain);
+            (void)mbar_wait(&ctl.drain, 0);
+        }
+        __syncthreads();
+    }
+    if (warp == kIdxMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kIdxTmemCols);
+    }
+    return ok;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -360,7 +587,7 @@ static IdxTree tree_layout(int B, int n_chunks, int kc, int k, int group, uint8_
 }
 
 // ------------------------------------------------------------------------------------------
-// The kernel.
+// The merge-tree kernel.
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
     const __grid_constant__ CUtensorMap kmap, const float* __restrict__ iscales, int64_t cap,
@@ -370,7 +597,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
     extern __shared__ __align__(128) uint8_t smem_raw[];
     IdxSmem& sm = *reinterpret_cast<IdxSmem*>(
         smem_raw + ((kIdxSmemAlign - (smem_u32(smem_raw) & (kIdxSmemAlign - 1))) & (kIdxSmemAlign - 1)));
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int b = blockIdx.y, ch = blockIdx.x;
 
     int64_t n_b = seq_len[b];
@@ -381,172 +608,9 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
 
     for (int i = tid; i < kBins; i += blockDim.x) sm.hist[i] = 0u;
     bool chunk_ok = true;
-    if (cn > 0) {
-        const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
-        volatile int32_t* fail = &sm.fail;
-        if (tid == 0) {
-            for (int s = 0; s < kIdxStages; ++s) {
-                mbar_init(&sm.full[s], 1);
-                mbar_init(&sm.empty[s], 4);          // the 4 warps of the epilogue warpgroup
-                mbar_init(&sm.accf[s], 1);
-            }
-            mbar_init(&sm.drain, 1);
-            sm.fail = 0;
-            sm.n_issued = 0;
-            sm.n_mma = 0;
-            fence_barrier_init();
-        }
-        if (warp == kIdxMmaWarp) {
-            tmem_alloc(&sm.tmem_base, kIdxTmemCols);
-            tmem_relinquish();
-        }
-        if (warp == kIdxProducerWarp && lane == 0) tma_prefetch_map(&kmap);
-        // --- query operand: FP4 codes in the MMA's B layout (8 rows x 32 bytes, 32-byte swizzle)
-        // Row n is head n & 3 over group n >> 2; the row's other 32-element group is zero, so
-        // every output column is one exact group dot.  Thread t writes bytes 4j..4j+3 of row n.
-        if (tid < 64) {
-            const int n = tid >> 3, j = tid & 7, h = n & 3, grp = n >> 2;
-            const float* qv = q_idx + ((size_t)b * kIdxHeads + h) * kIdxDim;
-            float amax = 0.f;
-            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[32 * grp + i]));
-            const float sg = fp4_group_scale(amax);
-            const float inv = 1.0f / sg;   // exact: a power of two
-            uint32_t word = 0u;
-            if ((j >> 2) == grp) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) word |= e2m1_code(qv[8 * j + i] * inv) << (4 * i);
-            }
-            const int half = (j >> 2) ^ ((n >> 2) & 1);
-            *reinterpret_cast<uint32_t*>(sm.bq + n * kIkey + half * 16 + (j & 3) * 4) = word;
-            if (j == 0) sm.qscale[grp * 4 + h] = sg;
-            fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        const uint32_t tmem = sm.tmem_base;
-        if (warp < 4) {   // unit block-scale factors (UE8M0 0x7F = 2^0) for A and B, every lane
-            tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kIdxSfCol, 0x7F7F7F7Fu);
-            tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kIdxSfCol + 8, 0x7F7F7F7Fu);
-            tmem_st_wait();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        const float* sbase = iscales + ((size_t)b * cap + (size_t)c0) * 2;
-        if (warp == kIdxProducerWarp) {
-            // --- producer: key tile (TMA, swizzled) + its scales (bulk copy) per stage -------
-            if (lane == 0) {
-                int t = 0;
-                for (; t < n_tiles; ++t) {
-                    const int s = t % kIdxStages;
-                    if (*fail) break;
-                    if (t >= kIdxStages && !mbar_wait(&sm.empty[s], ((t / kIdxStages) - 1) & 1)) break;
-                    const int nt = min(kIdxTile, cn - t * kIdxTile);
-                    const uint32_t sb = static_cast<uint32_t>((nt + 1) & ~1) * 8u;   // cap is even
-                    mbar_arrive_expect_tx(&sm.full[s], kIdxTile * kIkey + sb);
-                    tma_load_3d(sm.u.pipe.codes[s], &kmap, 0, static_cast<int>(c0) + t * kIdxTile, b, &sm.full[s]);
-                    bulk_g2s(sm.u.pipe.scales[s], sbase + (size_t)t * kIdxTile * 2, sb, &sm.full[s]);
-                }
-                sm.n_issued = t;
-                if (t < n_tiles) *fail = 1;
-            }
-        } else if (warp == kIdxMmaWarp) {
-            // --- MMA issuer: two 128-row block-scaled FP4 MMAs per tile into accumulator slot s
-            if (lane == 0) {
-                const uint64_t bdesc = smem_desc_kmajor_sw32(sm.bq);
-                const uint32_t sfa = tmem + kIdxSfCol, sfb = tmem + kIdxSfCol + 8;
-                int t = 0;
-                for (; t < n_tiles; ++t) {
-                    const int s = t % kIdxStages;
-                    if (*fail || !mbar_wait(&sm.full[s], (t / kIdxStages) & 1)) break;
-                    tc_fence_after();
-                    const uint32_t d = tmem + 16u * static_cast<uint32_t>(s);
-                    umma_mxf4(d, smem_desc_kmajor_sw32(sm.u.pipe.codes[s]), bdesc, kIdxIdesc, sfa, sfb, 0u);
-                    umma_mxf4(d + 8u, smem_desc_kmajor_sw32(sm.u.pipe.codes[s] + 128 * kIkey), bdesc, kIdxIdesc,
-                              sfa, sfb, 0u);
-                    umma_commit(&sm.accf[s]);
-                }
-                sm.n_mma = t;
-                if (t < n_tiles) *fail = 1;
-            }
-        } else if (warp < 4 * kIdxEpiGroups) {
-            // --- epilogue: warpgroup wg finishes tiles wg, wg + 3, ...; thread = TMEM lane m
-            // holds entries m and 128 + m of the tile: columns 0..3 / 4..7 their group-0 /
-            // group-1 dots of heads 0..3 (8..15 for entry 128 + m), each exactly I_g / 4.
-            const int wg = warp >> 2, quad = warp & 3;
-            const int m = 32 * quad + lane;
-            const uint32_t lane_addr = tmem + ((32u * quad) << 16);
-            float qsc[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) qsc[i] = sm.qscale[i];
-            const float w0 = head_w[b * kIdxHeads + 0], w1 = head_w[b * kIdxHeads + 1];
-            const float w2 = head_w[b * kIdxHeads + 2], w3 = head_w[b * kIdxHeads + 3];
-            for (int t = wg; t < n_tiles; t += kIdxEpiGroups) {
-                const int s = t % kIdxStages;
-                const bool landed = !*fail && mbar_wait(&sm.accf[s], (t / kIdxStages) & 1);
-                if (!__all_sync(0xffffffffu, landed)) {
-                    if (lane == 0) *fail = 1;
-                    break;
-                }
-                tc_fence_after();
-                uint32_t r[16];
-                tmem_ld_32x32b_x16(lane_addr + 16u * static_cast<uint32_t>(s), r);
-                tmem_ld_wait();
-                const float2* ss = reinterpret_cast<const float2*>(sm.u.pipe.scales[s]);
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int e = 128 * hf + m;
-                    const float2 ks = ss[e];
-                    float rr[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        // d = fma(I1, s1, I0*s0) with s_g = (qscale_g * kscale_g) * 0.25
-                        const float i0 = __fmul_rn(__uint_as_float(r[8 * hf + h]), 4.0f);
-                        const float i1 = __fmul_rn(__uint_as_float(r[8 * hf + 4 + h]), 4.0f);
-                        const float s0 = __fmul_rn(__fmul_rn(qsc[h], ks.x), 0.25f);
-                        const float s1 = __fmul_rn(__fmul_rn(qsc[4 + h], ks.y), 0.25f);
-                        const float d = __fmaf_rn(i1, s1, __fmul_rn(i0, s0));
-                        rr[h] = d > 0.f ? d : 0.f;
-                    }
-                    float sc = __fmul_rn(w0, rr[0]);
-                    sc = __fmaf_rn(w1, rr[1], sc);
-                    sc = __fmaf_rn(w2, rr[2], sc);
-                    sc = __fmaf_rn(w3, rr[3], sc);
-                    const int li = t * kIdxTile + e;
-                    if (li < cn) {
-                        const uint32_t key = score_key(sc);
-                        sm.keys[li] = key;
-                        atomicAdd(&sm.hist[key >> kBinShift], 1u);
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.empty[s]);   // stage s and accumulator slot s free
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-        chunk_ok = (sm.fail == 0);
-        if (!chunk_ok) {
-            // A copy or an MMA did not complete in time: record it, let the copies in flight
-            // land and the MMAs in flight finish (bounded waits) before the shared and tensor
-            // memory are reused, and publish this chunk as empty so the merge tree completes.
-            if (warp == kIdxMmaWarp && lane == 0) {
-                dev_error(err, CSLD_DEVERR_TIMEOUT);
-                for (int t = sm.n_mma; t < sm.n_issued; ++t)
-                    (void)mbar_wait(&sm.full[t % kIdxStages], (t / kIdxStages) & 1);
-                umma_commit(&sm.drain);
-                (void)mbar_wait(&sm.drain, 0);
-            }
-            __syncthreads();
-        }
-        if (warp == kIdxMmaWarp) {
-            tc_fence_after();
-            tmem_dealloc(tmem, kIdxTmemCols);
-        }
-    }
+    if (cn > 0)
+        chunk_ok = score_chunk<kIdxStages, 128>(sm.ctl, sm.u.pipe.codes, sm.u.pipe.scales, sm.keys, sm.hist, kmap, iscales,
+                                           cap, b, c0, cn, q_idx, head_w, err);
     __syncthreads();
     // --- selection and the merge tree ------------------------------------------------------
     int n = (cn > 0 && chunk_ok) ? cn : 0;   // a timed-out chunk publishes nothing
@@ -639,17 +703,17 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
                 const int flat = base + u * blockDim.x + tid;     // child c, position i
                 const int c = flat / rc, i = flat - c * rc;
                 dst[u] = -1;
+                kv[u] = 0u;
                 if (c < children && i < sm.offs[c + 1] - sm.offs[c]) {
                     kv[u] = __ldcg(tree.keys[level] + child0 + flat);
                     dst[u] = sm.offs[c] + i;
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (dst[u] >= 0) {
-                    sm.keys[dst[u]] = kv[u];
-                    atomicAdd(&sm.hist[kv[u] >> kBinShift], 1u);
-                }
+            for (int u = 0; u < 8; ++u) {
+                if (dst[u] >= 0) sm.keys[dst[u]] = kv[u];
+                hist_add(sm.hist, kv[u] >> kBinShift, dst[u] >= 0);
+            }
         }
         child_idx = reinterpret_cast<const uint32_t*>(tree.idx[level] + child0);
         n = sm.offs[children];
@@ -659,14 +723,335 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
     }
 }
 
+// ------------------------------------------------------------------------------------------
+// The cooperative kernel: one exact radix select per sequence across its CTAs.
+// ------------------------------------------------------------------------------------------
+struct CoopWs {
+    uint32_t* hist;    // [B][kCoopSeqWords]: level 1 (2048 bins), level 2 (2048), level 3 (1024)
+    uint32_t* sync;    // [B][64]: word 0 barrier arrivals, word 1 finished CTAs
+    uint32_t* counts;  // [B][units][2]: keys above the threshold, keys equal to it
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Barrier of the CTAs of one sequence: arrival counter *ctr reaches `target`.  The spin is
+// bounded (about half a second); on time-out the device error word gets CSLD_DEVERR_TIMEOUT
+// and false is returned to every thread of the CTA.
+__device__ bool seq_barrier(uint32_t* ctr, uint32_t target, int32_t* fail_flag, int32_t* err) {
+    __threadfence();   // this thread's histogram / count updates before the arrival
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        bool ok = false;
+        for (uint32_t i = 0; i < (1u << 22); ++i) {
+            if (ld_acquire_u32(ctr) >= target) {
+                ok = true;
+                break;
+            }
+            if (i >= 16) __nanosleep(64);
+        }
+        if (!ok) {
+            dev_error(err, CSLD_DEVERR_TIMEOUT);
+            *fail_flag = 1;
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    return *reinterpret_cast<volatile int32_t*>(fail_flag) == 0;
+}
+
+// From a global histogram g of nbins bins (2048 or 1024), the bin holding the want-th largest
+// key and how many keys are wanted inside it (*need).  Block-wide; g read through L2.
+__device__ void find_bin_global(const uint32_t* g, int nbins, uint32_t want, uint32_t* red, uint32_t* sel,
+                                uint32_t* bin, uint32_t* need) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int per = nbins / kIdxThreads;     // 4 or 2 bins per thread, from the top
+    uint32_t c[4] = {0u, 0u, 0u, 0u}, tot = 0u;
+    for (int q = 0; q < per; ++q) {
+        c[q] = __ldcg(g + nbins - 1 - per * tid - q);
+        tot += c[q];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (tid == 0) {
+        sel[0] = 0u;
+        sel[1] = 0u;
+    }
+    uint32_t all;
+    const uint32_t wb = warp_excl_scan(__shfl_sync(0xffffffffu, incl, 31), red, &all);
+    const uint32_t excl = wb + incl - tot;
+    if (excl < want && excl + tot >= want) {
+        uint32_t run = excl;
+        for (int q = 0; q < per; ++q) {
+            if (run + c[q] >= want) {
+                sel[0] = static_cast<uint32_t>(nbins - 1 - per * tid - q);
+                sel[1] = want - run;
+                break;
+            }
+            run += c[q];
+        }
+    }
+    __syncthreads();
+    *bin = sel[0];
+    *need = sel[1];
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
+    const __grid_constant__ CUtensorMap kmap, const float* __restrict__ iscales, int64_t cap,
+    const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
+    const float* __restrict__ head_w, int chunk, int units, int k, CoopWs ws,
+    int32_t* __restrict__ topk_out, int32_t* err) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    CoopSmem& sm = *reinterpret_cast<CoopSmem*>(
+        smem_raw + ((kIdxSmemAlign - (smem_u32(smem_raw) & (kIdxSmemAlign - 1))) & (kIdxSmemAlign - 1)));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int b = blockIdx.y, u = blockIdx.x;
+
+    int64_t n_b = seq_len[b];
+    n_b = n_b < 0 ? 0 : n_b / ratio;
+    if (n_b > cap) n_b = cap;
+    const int64_t c0 = (int64_t)u * chunk;
+    const int cn = static_cast<int>(max64(0, min64(chunk, n_b - c0)));
+    int32_t* out = topk_out + (size_t)b * k;
+
+    if (n_b <= k) {
+        // every visible entry is selected: no scores needed, and no barrier (the whole
+        // sequence takes this branch); entry i goes to position i, the rest is -1
+        for (int i = tid; i < cn; i += blockDim.x) out[c0 + i] = static_cast<int32_t>(c0 + i);
+        if (u == 0)
+            for (int64_t i = n_b + tid; i < k; i += blockDim.x) out[i] = -1;
+        return;
+    }
+    const uint32_t want = static_cast<uint32_t>(k);
+    uint32_t* g1 = ws.hist + (size_t)b * kCoopSeqWords;
+    uint32_t* g2 = g1 + kBins;
+    uint32_t* g3 = g2 + kBins;
+    uint32_t* bar = ws.sync + (size_t)b * 64;
+    uint32_t* done = bar + 1;
+    uint32_t* cnt = ws.counts + (size_t)b * units * 2;
+    const uint32_t nu = static_cast<uint32_t>(units);
+
+    for (int i = tid; i < kBins; i += blockDim.x) {
+        sm.hist[i] = 0u;
+        sm.hist2[i] = 0u;
+    }
+    for (int i = tid; i < 1024; i += blockDim.x) sm.hist3[i] = 0u;
+    if (tid == 0) sm.fail = 0;
+    __syncthreads();
+    bool ok = true;
+    if (cn > 0)
+        ok = score_chunk<kCoopStages, 256>(sm.ctl, sm.codes, sm.scales, sm.keys, sm.hist, kmap, iscales, cap, b, c0, cn,
+                                      q_idx, head_w, err);
+    __syncthreads();
+    // --- level 1: bits 31..21 ------------------------------------------------------------------
+    if (ok)
+        for (int i = tid; i < kBins; i += blockDim.x) {
+            const uint32_t c = sm.hist[i];
+            if (c) atomicAdd(g1 + i, c);
+        }
+    if (!seq_barrier(bar, 1 * nu, &sm.fail, err)) return;
+    uint32_t beta1, need1;
+    find_bin_global(g1, kBins, want, sm.red, sm.sel, &beta1, &need1);
+    // --- level 2: bits 20..10.  One pass over the range: each warp counts its keys above bin
+    //     beta1 and copies the keys inside it to its own candidate region (the copy ring is
+    //     idle now); later levels only look at the candidates ---------------------------------
+    constexpr int kSeg = kCoopMaxRange / kIdxWarps;    // warp w owns positions 1024w .. 1024w+1023
+    uint32_t* cand = reinterpret_cast<uint32_t*>(&sm.codes[0][0]) + warp * kSeg;
+    const int i0 = warp * kSeg;
+    const int steps = max(0, min(kSeg, cn - i0) + 31) >> 5;
+    uint32_t gt = 0u, nc = 0u;
+    for (int s = 0; s < steps; ++s) {
+        const int i = i0 + 32 * s + lane;
+        const uint32_t key = i < cn ? sm.keys[i] : 0u;
+        const uint32_t bin = key >> kBinShift;
+        gt += __popc(__ballot_sync(0xffffffffu, i < cn && bin > beta1));
+        const bool in = i < cn && bin == beta1;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        if (in) {
+            cand[nc + __popc(m & lt)] = key;
+            const uint32_t sub = (key >> 10) & (kBins - 1);
+            const uint32_t same = __match_any_sync(m, sub);   // lanes sharing a bin: one atomic
+            if (lane == __ffs(same) - 1) atomicAdd(&sm.hist2[sub], static_cast<uint32_t>(__popc(same)));
+        }
+        nc += __popc(m);
+    }
+    __syncthreads();
+    for (int i = tid; i < kBins; i += blockDim.x) {
+        const uint32_t c = sm.hist2[i];
+        if (c) atomicAdd(g2 + i, c);
+    }
+    if (!seq_barrier(bar, 2 * nu, &sm.fail, err)) return;
+    uint32_t beta2, need2;
+    find_bin_global(g2, kBins, need1, sm.red, sm.sel, &beta2, &need2);
+    const uint32_t top22 = (beta1 << 11) | beta2;
+    // --- level 3: bits 9..0 of the candidates whose top 22 bits are (beta1, beta2) -------------
+    const int csteps = static_cast<int>((nc + 31) >> 5);
+    for (int s = 0; s < csteps; ++s) {
+        const int j = 32 * s + lane;
+        const uint32_t key = j < static_cast<int>(nc) ? cand[j] : 0u;
+        const bool in = j < static_cast<int>(nc) && (key >> 10) == top22;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        if (in) {
+            const uint32_t low = key & 1023u;
+            const uint32_t same = __match_any_sync(m, low);
+            if (lane == __ffs(same) - 1) atomicAdd(&sm.hist3[low], static_cast<uint32_t>(__popc(same)));
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < 1024; i += blockDim.x) {
+        const uint32_t c = sm.hist3[i];
+        if (c) atomicAdd(g3 + i, c);
+    }
+    if (!seq_barrier(bar, 3 * nu, &sm.fail, err)) return;
+    uint32_t beta3, take_eq;
+    find_bin_global(g3, 1024, need2, sm.red, sm.sel, &beta3, &take_eq);
+    const uint32_t thr = (top22 << 10) | beta3;   // keys > thr are in; of keys == thr the first take_eq
+    // --- this range's counts (keys above bin beta1 plus candidates above thr; candidates equal
+    //     to thr); then the counts of the ranges before it ------------------------------------
+    uint32_t above = 0u, equal = 0u;
+    for (int s = 0; s < csteps; ++s) {
+        const int j = 32 * s + lane;
+        const uint32_t key = j < static_cast<int>(nc) ? cand[j] : 0u;
+        above += j < static_cast<int>(nc) && key > thr;
+        equal += j < static_cast<int>(nc) && key == thr;
+    }
+    above = gt + __reduce_add_sync(0xffffffffu, above);
+    equal = __reduce_add_sync(0xffffffffu, equal);
+    uint32_t tot;
+    const uint32_t pre = warp_excl_scan((above << 16) | equal, sm.red + kIdxWarps, &tot);   // counts <= 2^14
+    if (tid == 0) {
+        cnt[2 * u] = tot >> 16;
+        cnt[2 * u + 1] = tot & 0xFFFFu;
+    }
+    if (!seq_barrier(bar, 4 * nu, &sm.fail, err)) return;
+    uint32_t a_before = 0u, e_before = 0u;
+    for (int v = tid; v < u; v += blockDim.x) {
+        a_before += __ldcg(cnt + 2 * v);
+        e_before += __ldcg(cnt + 2 * v + 1);
+    }
+    a_before = __reduce_add_sync(0xffffffffu, a_before);
+    e_before = __reduce_add_sync(0xffffffffu, e_before);
+    if (lane == 0) {
+        sm.red[2 * kIdxWarps + warp] = a_before;   // red[32..47]: free after the scan above
+    }
+    __syncthreads();
+    uint32_t A = 0u;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) A += sm.red[2 * kIdxWarps + w];
+    __syncthreads();
+    if (lane == 0) sm.red[2 * kIdxWarps + warp] = e_before;
+    __syncthreads();
+    uint32_t E = 0u;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) E += sm.red[2 * kIdxWarps + w];
+    // --- emit this range's selected entries in index order ------------------------------------
+    uint32_t eq_seen = E + (pre & 0xFFFFu);
+    uint32_t pos = A + (pre >> 16) + min(eq_seen, take_eq);
+    for (int s = 0; s < steps; ++s) {
+        const int i = i0 + 32 * s + lane;
+        const uint32_t key = i < cn ? sm.keys[i] : 0u;
+        const bool veq = i < cn && key == thr;
+        const uint32_t em = __ballot_sync(0xffffffffu, veq);
+        const bool take = (i < cn && key > thr) || (veq && eq_seen + __popc(em & lt) < take_eq);
+        const uint32_t tm = __ballot_sync(0xffffffffu, take);
+        const uint32_t at = pos + __popc(tm & lt);
+        // the counts add up to exactly k when every range scored; after a timed-out range the
+        // positions are not trusted
+        if (take && at < want) out[at] = static_cast<int32_t>(c0 + i);
+        pos += __popc(tm);
+        eq_seen += __popc(em);
+    }
+    // --- the last CTA of the sequence leaves its histograms and counters at zero --------------
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        sm.last = (atomicAdd(done, 1u) == nu - 1u);
+    }
+    __syncthreads();
+    if (sm.last) {
+        for (int i = tid; i < kCoopSeqWords; i += blockDim.x) g1[i] = 0u;
+        if (tid == 0) {
+            *bar = 0u;
+            *done = 0u;
+        }
+        __threadfence();
+    }
+}
+
+// Resident CTAs of the cooperative kernel on this device (0 if it cannot run).
+static int coop_slots(int num_sms) {
+    static int per_sm = -1;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const size_t smem = sizeof(CoopSmem) + kIdxSmemAlign;
+        int n = 0;
+        if (set_smem_once(indexer_topk_coop_kernel, smem) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, indexer_topk_coop_kernel, kIdxThreads, smem) ==
+                cudaSuccess)
+            per_sm = n;
+        else
+            per_sm = 0;
+        (void)cudaGetLastError();
+    });
+    return per_sm * num_sms;
+}
+
+static size_t coop_layout(int B, int units, uint8_t* base, CoopWs* ws) {
+    size_t off = 0;
+    const size_t h = up256((size_t)B * kCoopSeqWords * 4), s = up256((size_t)B * 64 * 4),
+                 c = up256((size_t)B * units * 2 * 4);
+    if (ws) {
+        ws->hist = reinterpret_cast<uint32_t*>(base + off);
+        ws->sync = reinterpret_cast<uint32_t*>(base + off + h);
+        ws->counts = reinterpret_cast<uint32_t*>(base + off + h + s);
+    }
+    off += h + s + c;
+    return off;
+}
+
 IndexerPlan indexer_plan(int B, int64_t cap, int k, int num_sms) {
-    IndexerPlan p;
-    int chunk = kIdxMaxChunk;
-    while (chunk > 1024 && (int64_t)B * ((cap + chunk - 1) / chunk) < num_sms) chunk >>= 1;
-    p.chunk = chunk;
+    IndexerPlan p{};
+    // Cooperative path: every sequence split into `units` ranges of at most kCoopMaxRange
+    // entries (a multiple of the tile), all B * units CTAs resident at once (one per SM: the
+    // occupancy the runtime grants a kernel that allocates tensor memory).
+    const int slots = coop_slots(num_sms);
+    if (slots > 0) {
+        const int64_t per_seq = max64(1, slots / B);
+        int64_t chunk = (cap + per_seq - 1) / per_seq;
+        chunk = max64(kIdxTile, (chunk + kIdxTile - 1) / kIdxTile * kIdxTile);
+        const int64_t units = (cap + chunk - 1) / chunk;
+        if (chunk <= kCoopMaxRange && (int64_t)B * units <= slots) {
+            p.coop = true;
+            p.chunk = static_cast<int>(chunk);
+            p.n_chunks = static_cast<int>(units);
+            p.kc = k < chunk ? k : static_cast<int>(chunk);
+            p.group = 0;
+            p.levels_ok = true;
+            p.ws_bytes = coop_layout(B, p.n_chunks, nullptr, nullptr);
+            return p;
+        }
+    }
+    // Merge-tree path: chunks of all sequences spread over the SMs (2 CTAs each) as evenly as
+    // possible, a multiple of the tile between 1024 and kIdxMaxChunk entries.
+    const int64_t per_seq = max64(1, (2LL * num_sms) / B);
+    int64_t chunk = (cap + per_seq - 1) / per_seq;
+    chunk = (chunk + kIdxTile - 1) / kIdxTile * kIdxTile;
+    chunk = max64(1024, min64(kIdxMaxChunk, chunk));
+    p.chunk = static_cast<int>(chunk);
     const int64_t nc = (cap + chunk - 1) / chunk;
     p.n_chunks = static_cast<int>(nc < 1 ? 1 : nc);
-    p.kc = k < chunk ? k : chunk;
+    p.kc = k < chunk ? k : static_cast<int>(chunk);
     int group = kIdxMaxChunk / k;                 // merged runs hold up to k candidates
     if (group > kIdxMaxGroup) group = kIdxMaxGroup;
     if (group < 2) group = 2;
@@ -696,8 +1081,6 @@ cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t c
                            const int32_t* seq_len, int ratio, const float* q_idx,
                            const float* head_w, int B, int k, int32_t* topk_out, void* ws,
                            const IndexerPlan& plan, int32_t* err, cudaStream_t stream) {
-    size_t bytes = 0;
-    IdxTree tree = tree_layout(B, plan.n_chunks, plan.kc, k, plan.group, static_cast<uint8_t*>(ws), &bytes);
     // Key codes as a 3-D byte tensor [B][cap][32]; one box = one stage of 256 entries.  Rows
     // past cap read as zeros (their scores are never used).
     PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
@@ -711,6 +1094,29 @@ cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t c
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    if (plan.coop) {
+        CoopWs cws;
+        coop_layout(B, plan.n_chunks, static_cast<uint8_t*>(ws), &cws);
+        const size_t smem = sizeof(CoopSmem) + kIdxSmemAlign;
+        cudaError_t e = set_smem_once(indexer_topk_coop_kernel, smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(plan.n_chunks, B);
+        cfg.blockDim = dim3(kIdxThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs resident: the barriers can complete
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, indexer_topk_coop_kernel, kmap, iscales, cap, seq_len, ratio, q_idx, head_w,
+                               plan.chunk, plan.n_chunks, k, cws, topk_out, err);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+    size_t bytes = 0;
+    IdxTree tree = tree_layout(B, plan.n_chunks, plan.kc, k, plan.group, static_cast<uint8_t*>(ws), &bytes);
     const size_t smem = sizeof(IdxSmem) + kIdxSmemAlign;
     cudaError_t e = set_smem_once(indexer_topk_kernel, smem);
     if (e != cudaSuccess) return e;

@@ -22,8 +22,9 @@ cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
 
 // Lightning indexer + top-k.
 struct IndexerPlan {
+    bool coop;          // one cooperative pass (all CTAs resident) instead of the merge tree
     int chunk;          // entries per scoring CTA (multiple of 256)
-    int n_chunks;       // chunks per sequence (over the capacity)
+    int n_chunks;       // chunks (ranges) per sequence (over the capacity)
     int kc;             // candidates kept per chunk = min(k, chunk)
     int group;          // runs merged by one CTA in the merge tree
     bool levels_ok;     // the merge tree reaches one run within its level limit

@@ -93,3 +93,31 @@ def test_indexer_full_workloads(csld, orc, name):
     s32, s64 = orc.indexer_scores(ik[0, :wl.csa_entries].numpy(), isc[0, :wl.csa_entries].numpy(),
                                   q[0].numpy(), w[0].numpy())
     assert H.near_tie_only(ref[0], orc.topk64(s64, wl.topk), s64)
+
+
+@pytest.mark.parametrize("B,cap,k", [(300, 2048, 64), (40, 65536, 512)])
+def test_indexer_many_sequences_merge_tree_path(csld, orc, B, cap, k):
+    """Shapes whose CTAs cannot all be resident at once (more than 2 x 148 CTAs, or ranges
+    longer than 8192 entries) take the merge-tree kernel instead of the cooperative one."""
+    ik, isc, q, w = _inputs(B, cap, cap, seed=B + k)
+    g = synth.gen(77)
+    seq = (torch.randint(0, 4 * cap + 8, (B,), generator=g)).to(torch.int32)
+    seq[0] = 4 * cap
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, k)
+    H.assert_topk_equal(got, ref)
+
+
+def test_indexer_workspace_reused_across_calls(csld, orc):
+    """The workspace's counters and histograms are left at zero by every call, so one
+    zero-filled workspace serves any number of calls (here with different inputs)."""
+    B, cap, k = 4, 40000, 256
+    ws = csld.indexer_workspace(B, cap, k)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for it in range(3):
+        ik, isc, q, w = _inputs(B, cap, cap, seed=300 + it)
+        seq = torch.tensor([4 * cap, 4 * (cap // 2) + 1, 4 * 1000, 4 * cap - 5], dtype=torch.int32)
+        out = csld.indexer_topk(ik.cuda(), isc.cuda(), seq.cuda(), 4, q.cuda(), w.cuda(), k, ws=ws, err=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        ref = orc.indexer_topk_batch(ik.numpy(), isc.numpy(), seq.numpy(), 4, q.numpy(), w.numpy(), k)
+        H.assert_topk_equal(out.cpu().numpy(), ref)
