@@ -335,7 +335,7 @@ def run_ours(args, rank, world, local_rank):
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps_timed,
         "warmup": rounds_w * REPLICAS, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16 KV, e2m1 indexer; f16/bf16/s8 MMA, fp32 acc",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16 KV, e2m1 indexer keys; tcgen05 e2m1, e4m3 and bf16 MMA, fp32 accumulate",
         "data": "synthetic (seeded)",
         "config": {"workload": wl.name, "batch_per_gpu": B, "context": wl.context, "csa_entries": wl.csa_entries,
                    "hca_entries": wl.hca_entries, "topk": k, "window": W, "heads": 16, "dim": 512,

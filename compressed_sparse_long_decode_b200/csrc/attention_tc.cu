@@ -1,0 +1,585 @@
+// Hybrid decode attention on the 5th-generation tensor cores (tcgen05).
+//
+// Source: "DeepSeek-V4: a million-token context that agents can actually use" -- CSA paragraph
+// and Figure 3 caption (each query attends to its top-k compressed blocks; a sliding-window
+// branch covers the most recent uncompressed tokens), HCA paragraph and Figure 4 caption
+// (every query attends densely to all compressed blocks; the same window branch), storage
+// paragraph (entries FP8 except the RoPE dims in bf16); velog.io paper review, core
+// techniques 1-2.  Keys and values are the same 576-byte entry (448 E4M3 dims + 64 bf16 RoPE
+// dims); 16 query heads share it; one softmax runs over {selected or all visible entries} +
+// {window tokens}.
+//
+// One CTA = one split of one sequence's key list, walked in tiles of 128 entries; 16 warps.
+//  - Warps 0-3 bring a tile in with TMA: five 128-byte column blocks of every entry (bytes 0,
+//    128, 256, 384 and 448 -- the last one is the RoPE part), each block [128 entries][128 B]
+//    with the 128-byte swizzle.  Contiguous tiles take one box copy per block; otherwise rows
+//    come four at a time by index (tile::gather4).  The same image is the K-major operand of
+//    QK (rows = entries) and the MN-major operand of PV (rows = dims).
+//  - Warp 4 issues the MMAs (one thread):
+//      S[entry][hi|lo head] = K_nope . [Qhi;Qlo]^T    kind::f8f6f4, E4M3 x E4M3, N = 32
+//                           + K_rope . Qrope^T         kind::f16, bf16 (into the hi columns)
+//      O^T[dim][hi|lo head] += V_nope^T . [Phi;Plo]^T  kind::mxf8f6f4, P scaled per 32 entries
+//      O^T_rope[dim][head]  += V_rope^T . Pbf^T        kind::f16, bf16 x bf16
+//    The bf16 query of each head is scaled by a power of two and split into two E4M3 terms
+//    (hi = E4M3(q), lo = E4M3(q - hi)); P is split the same way after a power-of-two scale
+//    per 32-entry block (the MMA's UE8M0 block scale), so each product keeps about as many
+//    significant bits as a bf16 operand.  The hi and lo rows are stacked into one N = 32
+//    operand and their results added when read back.  Block 3 holds bytes 384..511, whose
+//    upper half is the bf16 RoPE part: QK reads only its first 64 bytes, and the PV rows of
+//    dims 448..511 it yields are discarded.  S and O accumulate in fp32 in tensor memory.
+//  - Warps 8-15 run the online softmax: thread = entry (TMEM lane); warps 8-11 own heads 0-7,
+//    warps 12-15 heads 8-15.  The running max is raised lazily: O is rescaled in tensor memory
+//    only when a tile's max exceeds it by more than 8 (log2 units), so P <= 256 always.
+//  - Warps 4-15 prepare the query operands while the first copies are in flight.
+//  Two tile buffers, two S slots and two P buffers overlap the copy of tile t+1, QK of t+1,
+//  softmax of t and PV of t-1.  Every wait is bounded.  Each split writes its unnormalised O,
+//  the running max m (log2 units) and the sum l; attention_merge_kernel combines the splits.
+#include <stdint.h>
+
+#include "csld_internal.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace csld {
+
+namespace {
+
+constexpr int kTcThreads = 512;
+constexpr int kTcTile = 128;                  // entries per tile
+constexpr int kBlk = 5;                       // 128-byte column blocks per entry
+constexpr int kBlkBytes = kTcTile * 128;      // 16 KB: one column block of a tile
+constexpr int kTileBytes = kBlk * kBlkBytes;  // 80 KB
+constexpr int kRopeBlk = 4;                   // block 4 = entry bytes 448..575 (bf16 RoPE)
+constexpr uint32_t kTmemCols = 256;
+// tensor-memory columns
+constexpr uint32_t kColS = 0;                 // S slots at 0 and 32: hi heads +0..15, lo heads +16..31
+constexpr uint32_t kColO = 64;                // O^T nope blocks at 64, 96, 128, 160 (hi +0..15, lo +16..31)
+constexpr uint32_t kColOR = 192;              // O^T RoPE block 192..207
+constexpr uint32_t kColSFA = 208;             // 208..211: unit scale factors of V
+constexpr uint32_t kColSFB = 212;             // 212 and 216: P block scales of the two P buffers
+constexpr float kRescaleLog2 = 8.f;           // lazy rescale threshold (P <= 2^8)
+constexpr uint32_t kIdQK = idesc_e4m3_m128(32, false, false);
+constexpr uint32_t kIdQKr = idesc_bf16_m128(16, false, false);
+constexpr uint32_t kIdPVr = idesc_bf16_m128(16, true, false);
+constexpr int kSmBar = 1;                     // named barrier of the 8 softmax warps (256 threads)
+constexpr int kReadyBar = 2;                  // warps 4-15: query and tensor memory ready (384 threads)
+constexpr int kScaleBar = 3;                  // warps 4-15: query scales ready (384 threads)
+constexpr int kCopyBar = 4;                   // warps 0-3: the copy warps (128 threads)
+
+struct TcAttnSmem {
+    uint8_t tile[2][kTileBytes];              // [block][entry][128 B], 128-byte swizzle
+    uint8_t qk[4][32 * 128];                  // QK B operand per nope block: rows 0..15 Qhi, 16..31 Qlo
+    uint8_t qr[16 * 128];                     // RoPE query, bf16, 16 rows
+    uint8_t p8[2][32 * 128];                  // PV B operand: rows 0..15 Phi, 16..31 Plo, K = 128 entries
+    uint8_t pbf[2][2][16 * 128];              // bf16 P: two 64-entry K blocks of 16 rows
+    float c2[kHeads];                         // log2-domain logit factor per head
+    float sq[kHeads];                         // power-of-two query scale per head
+    float tmax[4][kHeads];                    // tile maxima per lane quarter
+    uint32_t sfb[2][4][kHeads];               // P block-scale bytes [buffer][32-entry block][head]
+    float lred[4][kHeads];
+    uint64_t full[2], empty[2], sfull[2], sfree[2], pfull[2], pdone[2], drain;
+    uint32_t tmem_base;
+    int32_t fail, n_issued, n_landed;
+};
+
+// Offset of byte c of row r in a [rows][128 B] block with the 128-byte swizzle (the 16-byte
+// chunk index XOR the row index within each 8-row, 1024-byte atom).
+__device__ __forceinline__ int sw128(int r, int c) {
+    return (r >> 3) * 1024 + (r & 7) * 128 + ((((c >> 4) ^ r) & 7) << 4) + (c & 15);
+}
+__device__ __forceinline__ float order_key_to_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+// 2^e as a float, -126 <= e <= 127.
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float(static_cast<uint32_t>(e + 127) << 23); }
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int y0, int y1, int y2, int y3,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+           "r"(smem_u32(bar))
+        : "memory");
+}
+// Operand with the 128-byte swizzle (1024-byte aligned atoms): 8-row groups 1024 bytes apart
+// (SBO); LBO = stride between 128-byte column blocks of an MN-major operand wider than 128 B.
+__device__ __forceinline__ uint64_t desc_sw128(const void* p, uint32_t lbo) {
+    const uint32_t a = smem_u32(p);
+    uint64_t d = static_cast<uint64_t>((a >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+// Scales 8 consecutive TMEM columns of this warp's lanes by f[0..7].
+__device__ __forceinline__ void tmem_scale8(uint32_t taddr, const float (&f)[8]) {
+    uint32_t o[8];
+    tmem_ld_32x32b_x8(taddr, o);
+    tmem_ld_wait();
+#pragma unroll
+    for (int h = 0; h < 8; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * f[h]);
+    tmem_st_32x32b_x8(taddr, o);
+}
+
+// Query scales (256 threads, t = 0..255): head t / 16, dims 32*(t % 16) .. +31.  The query of
+// head h is scaled by sq = 2^(7 - floor(log2 max|q_h|)), so it stays below 256 (E4M3 max 448).
+__device__ __forceinline__ void qprep_scale(TcAttnSmem& sm, const uint16_t* q, int b, int t, float scale) {
+    const int h = t >> 4, part = t & 15;
+    const uint4* src = reinterpret_cast<const uint4*>(q + ((size_t)b * kHeads + h) * kDim + 32 * part);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 v = __ldg(src + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(w[c] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[c] >> 16))));
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (part == 0) {
+        const int sh = amax > 0.f ? max(-100, min(100, 7 - ilogbf(amax))) : 0;
+        const float sq = ldexpf(1.f, sh);
+        sm.sq[h] = sq;
+        sm.c2[h] = scale * 1.4426950408889634f / sq;
+    }
+}
+// Query operands (384 threads, t = 0..383): pairs of dims.  Nope dims -> E4M3 hi and lo terms
+// in the swizzled QK operand, RoPE dims -> bf16.
+__device__ __forceinline__ void qprep_convert(TcAttnSmem& sm, const uint16_t* q, int b, int t) {
+    for (int p = t; p < kHeads * kDim / 2; p += 384) {
+        const int h = p >> 8, d = 2 * (p & 255);
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(q + ((size_t)b * kHeads + h) * kDim + d));
+        const float sq = sm.sq[h];
+        const float x0 = bf16_bits_to_f32(w & 0xFFFFu) * sq, x1 = bf16_bits_to_f32(w >> 16) * sq;
+        if (d < kNope) {
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t back = e4m3x2_to_f16x2(hi);   // exact
+            const float r0 = x0 - __half2float(__ushort_as_half(static_cast<unsigned short>(back & 0xFFFFu)));
+            const float r1 = x1 - __half2float(__ushort_as_half(static_cast<unsigned short>(back >> 16)));
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
+            *reinterpret_cast<uint16_t*>(&sm.qk[d >> 7][sw128(h, d & 127)]) = static_cast<uint16_t>(hi);
+            *reinterpret_cast<uint16_t*>(&sm.qk[d >> 7][sw128(16 + h, d & 127)]) = static_cast<uint16_t>(lo);
+        } else {
+            const int r = d - kNope;
+            *reinterpret_cast<uint32_t*>(sm.qr + sw128(h, 2 * r)) = f32_to_bf16_bits(x0) | (f32_to_bf16_bits(x1) << 16);
+        }
+    }
+    fence_proxy_async_smem();
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
+    const __grid_constant__ CUtensorMap kv_tile, const __grid_constant__ CUtensorMap kv_rows,
+    const __grid_constant__ CUtensorMap win_rows, const uint16_t* __restrict__ q, int64_t cap, int ratio,
+    const int32_t* __restrict__ topk, int k, int W, const int32_t* __restrict__ seq_len, float scale, int splits,
+    float* __restrict__ opart, float2* __restrict__ mlpart, int32_t* err) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    TcAttnSmem& sm = *reinterpret_cast<TcAttnSmem*>(smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.y, split = blockIdx.x;
+    const int B = gridDim.y;
+
+    // ---- the key list of sequence b and this split's tile range ----------------------------
+    // list = [compressed slots padded to a multiple of 4 with empty slots][window tokens], so a
+    // group of 4 slots never mixes the two sources
+    int32_t n = seq_len[b];
+    if (n < 0) {
+        if (tid == 0 && split == 0) dev_error(err, CSLD_DEVERR_SEQ_LEN);
+        n = 0;
+    }
+    const int64_t n_vis = min64(n / ratio, cap);
+    const bool sparse = topk != nullptr;
+    const int64_t n_comp = sparse ? (int64_t)k : n_vis;
+    const int64_t n_comp4 = (n_comp + 3) & ~int64_t(3);
+    const int n_win = W > 0 ? min(W, n) : 0;
+    const int64_t L = n_comp4 + n_win;
+    const int64_t n_tiles_all = (L + kTcTile - 1) / kTcTile;
+    const int64_t t_begin = n_tiles_all * split / splits;
+    const int n_tiles = static_cast<int>(n_tiles_all * (split + 1) / splits - t_begin);
+    const size_t part = (size_t)b * splits + split;
+    if (n_tiles <= 0) {
+        if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
+        return;
+    }
+    // rows past the end of each map read as zeros
+    const int32_t oob_kv = static_cast<int32_t>(min64((int64_t)B * cap, 0x7FFFFFFF));
+    const int32_t oob_win = static_cast<int32_t>(min64((int64_t)B * max(W, 1), 0x7FFFFFFF));
+    // compressed slot i -> row of the compressed map, or -1 for an empty slot
+    auto comp_row = [&](int64_t i, bool report) -> int32_t {
+        if (i >= n_comp) return -1;
+        int64_t v = i;
+        if (sparse) {
+            v = topk[(size_t)b * k + i];
+            if (v >= n_vis) {
+                if (report) dev_error(err, CSLD_DEVERR_BAD_INDEX);
+                return -1;
+            }
+            if (v < 0) return -1;
+        }
+        return static_cast<int32_t>((int64_t)b * cap + v);
+    };
+
+    // ---- setup --------------------------------------------------------------------------------
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.sfull[s], 1);
+            mbar_init(&sm.sfree[s], 8);
+            mbar_init(&sm.pfull[s], 8);
+            mbar_init(&sm.pdone[s], 1);
+        }
+        mbar_init(&sm.drain, 1);
+        sm.fail = 0;
+        sm.n_issued = 0;
+        sm.n_landed = 0;
+        fence_barrier_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&kv_tile);
+        tma_prefetch_map(&kv_rows);
+        tma_prefetch_map(&win_rows);
+    }
+    tc_fence_before();
+    __syncthreads();   // barriers initialised, tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int32_t* fail = &sm.fail;
+
+    if (warp < 4) {
+        // ===== copies (warps 0-3): tile t into buffer t & 1, started before the query is ready =====
+        int t = 0;
+        for (; t < n_tiles; ++t) {
+            const int s = t & 1;
+            const bool ok = !*fail && (t < 2 || mbar_wait(&sm.empty[s], ((t >> 1) - 1) & 1));
+            if (ok && tid == 0) mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+            if (named_barrier_or(kCopyBar, 128, !ok)) {   // the four copy warps leave together
+                if (tid == 0) *fail = 1;
+                break;
+            }
+            const int64_t i0 = (t_begin + t) * kTcTile;
+            uint8_t* tl = sm.tile[s];
+            if (!sparse && i0 + kTcTile <= n_comp) {
+                // contiguous, all valid: one box per column block
+                if (tid < kBlk)
+                    tma_load_2d(tl + tid * kBlkBytes, &kv_tile, tid < 4 ? 128 * tid : kNope,
+                                static_cast<int>((int64_t)b * cap + i0), &sm.full[s]);
+            } else {
+                // thread t: slots 4g .. 4g+3 (g = t / 4) of column block t % 4 (and block 4 when
+                // t % 4 == 0), from one of the two maps
+                const int g = tid >> 2, j = tid & 3;
+                const int64_t ib = i0 + 4 * g;
+                const bool win = ib >= n_comp4 && ib < L;
+                int32_t y[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int64_t i = ib + r;
+                    if (!win) {
+                        const int32_t row = comp_row(i, j == 0);
+                        y[r] = row >= 0 ? row : oob_kv;
+                    } else if (i < L) {
+                        const int64_t tok = (int64_t)n - n_win + (i - n_comp4);
+                        y[r] = static_cast<int32_t>((int64_t)b * W + tok % W);
+                    } else {
+                        y[r] = oob_win;
+                    }
+                }
+                const CUtensorMap* map = win ? &win_rows : &kv_rows;
+                tma_gather4(tl + j * kBlkBytes + 4 * g * 128, map, 128 * j, y[0], y[1], y[2], y[3], &sm.full[s]);
+                if (j == 0)
+                    tma_gather4(tl + kRopeBlk * kBlkBytes + 4 * g * 128, map, kNope, y[0], y[1], y[2], y[3], &sm.full[s]);
+            }
+        }
+        if (tid == 0) sm.n_issued = t;
+    } else if (warp >= 4 && warp < 8) {
+        // ===== the query operands (warps 4-15; the scales come from warps 8-15 first) ============
+        named_barrier(kScaleBar, 384);
+        qprep_convert(sm, q, b, tid - 128);
+        tc_fence_before();
+        named_barrier(kReadyBar, 384);   // query operands written; tensor memory initialised
+        tc_fence_after();
+        if (warp == 4 && lane == 0) {
+            // ===== MMA issue (one thread) =========================================================
+            const uint64_t dq = desc_sw128(sm.qk[0], 0), dqr = desc_sw128(sm.qr, 0);
+            int landed = 0;
+            for (int t = 0; t <= n_tiles; ++t) {
+                if (t < n_tiles) {
+                    const int s = t & 1;
+                    bool ok = !*fail && mbar_wait(&sm.full[s], (t >> 1) & 1);
+                    if (ok) landed = t + 1;
+                    if (ok && t >= 2) ok = mbar_wait(&sm.sfree[s], ((t >> 1) - 1) & 1);
+                    if (!ok) {
+                        *fail = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t dS = tmem + kColS + 32u * s;
+                    const uint64_t da = desc_sw128(sm.tile[s], 0);
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                        for (int ks = 0; ks < (kb < 3 ? 4 : 2); ++ks)   // 32 bytes of K per MMA; block 3
+                            // stops at byte 448 (the RoPE half is bf16: as E4M3 it may hold NaNs)
+                            umma_f8f6f4(dS, da + (kb * kBlkBytes + 32 * ks) / 16, dq + (kb * 4096 + 32 * ks) / 16, kIdQK,
+                                        (kb | ks) != 0 ? 1u : 0u);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_f16(dS, da + (kRopeBlk * kBlkBytes + 32 * ks) / 16, dqr + (32 * ks) / 16, kIdQKr, 1u);
+                    umma_commit(&sm.sfull[s]);
+                }
+                if (t >= 1) {   // PV of the previous tile
+                    const int u = t - 1, su = u & 1;
+                    if (*fail || !mbar_wait(&sm.pfull[su], (u >> 1) & 1)) {
+                        *fail = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = desc_sw128(sm.tile[su], 0);
+                    const uint64_t dp = desc_sw128(sm.p8[su], 0);
+                    const uint32_t sfb0 = tmem + kColSFB + 4u * su;
+#pragma unroll
+                    for (int mb = 0; mb < 4; ++mb)
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb)   // 32 entries (4 row groups) per MMA
+                            umma_mxf8f6f4(tmem + kColO + 32u * mb, da + (mb * kBlkBytes + kb * 4096) / 16,
+                                          dp + (32 * kb) / 16, idesc_mxe4m3_m128(32, true, false, kb), tmem + kColSFA,
+                                          sfb0 | (static_cast<uint32_t>(kb) << 30), 1u);
+                    // RoPE: M = 128 with LBO 16 KB (rows 64..127 read the next 16 KB: unused)
+                    const uint64_t dar = desc_sw128(sm.tile[su] + kRopeBlk * kBlkBytes, kBlkBytes);
+                    const uint64_t dpb = desc_sw128(sm.pbf[su][0], 0);
+#pragma unroll
+                    for (int ks = 0; ks < kTcTile / 16; ++ks)
+                        umma_f16(tmem + kColOR, dar + (ks * 2048) / 16, dpb + ((ks >> 2) * 2048 + 32 * (ks & 3)) / 16,
+                                 kIdPVr, 1u);
+                    umma_commit(&sm.empty[su]);
+                    umma_commit(&sm.pdone[su]);
+                }
+            }
+            sm.n_landed = landed;
+        }
+    } else if (warp >= 8) {
+        // ===== online softmax: thread = entry e = TMEM lane; head group hg = 8 heads =============
+        const int sub = warp & 3, hg = (warp - 8) >> 2, e = 32 * sub + lane;
+        const uint32_t lb = tmem + ((32u * sub) << 16);
+        qprep_scale(sm, q, b, tid - 256, scale);
+        if (hg == 0) {   // O = 0 and unit scale factors of V for this lane quarter
+            for (uint32_t c = kColO; c < kColSFA; c += 8) tmem_st_32x32b_x8_fill(lb + c, 0u);
+            tmem_st_32x32b_x8_fill(lb + kColSFA, 0x7F7F7F7Fu);
+            tmem_st_wait();
+        }
+        named_barrier(kScaleBar, 384);
+        qprep_convert(sm, q, b, tid - 128);
+        tc_fence_before();
+        named_barrier(kReadyBar, 384);
+        tc_fence_after();
+        float c2[8], mref[8], lsum[8];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            c2[h] = sm.c2[8 * hg + h];
+            mref[h] = -INFINITY;
+            lsum[h] = 0.f;
+        }
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int s = t & 1;
+            const int64_t i = (t_begin + t) * kTcTile + e;
+            const bool valid = i < n_comp4 ? comp_row(i, false) >= 0 : i < L;
+            ok = !*fail && mbar_wait(&sm.sfull[s], (t >> 1) & 1);
+            if (named_barrier_or(kSmBar, 256, !ok)) {   // the softmax warps leave together
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t shi[8], slo[8];
+            tmem_ld_32x32b_x8(lb + kColS + 32u * s + 8u * hg, shi);
+            tmem_ld_32x32b_x8(lb + kColS + 32u * s + 16u + 8u * hg, slo);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sfree[s]);
+            float x[8];
+#pragma unroll
+            for (int h = 0; h < 8; ++h)
+                x[h] = valid ? (__uint_as_float(shi[h]) + __uint_as_float(slo[h])) * c2[h] : -INFINITY;
+            // tile max per head: warp max of order keys, then across the four lane quarters
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                const uint32_t km = __reduce_max_sync(0xffffffffu, score_key(x[h]));
+                if (lane == h) sm.tmax[sub][8 * hg + h] = order_key_to_float(km);
+            }
+            named_barrier(kSmBar, 256);
+            bool rescale = false;
+            float mnew[8];
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                const int hh = 8 * hg + h;
+                const float tm = fmaxf(fmaxf(sm.tmax[0][hh], sm.tmax[1][hh]), fmaxf(sm.tmax[2][hh], sm.tmax[3][hh]));
+                mnew[h] = (tm > mref[h] + kRescaleLog2 || mref[h] == -INFINITY) ? fmaxf(tm, mref[h]) : mref[h];
+                rescale |= (mnew[h] != mref[h]) && (mref[h] != -INFINITY);
+            }
+            // P buffer s is free once PV(t-2) completed; a rescale also needs PV(t-1) done.  The
+            // barriers also tell every warp that all of them have read sm.tmax.
+            if (t >= 2) ok = mbar_wait(&sm.pdone[s], ((t >> 1) - 1) & 1);
+            const bool any_rescale = named_barrier_or(kSmBar, 256, rescale);
+            if (ok && any_rescale && t >= 1) ok = mbar_wait(&sm.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1);
+            if (named_barrier_or(kSmBar, 256, !ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (rescale) {   // this warp's 8 heads in every O block of its lane quarter
+                float f[8];
+#pragma unroll
+                for (int h = 0; h < 8; ++h) f[h] = (mref[h] == -INFINITY) ? 1.f : exp2f(mref[h] - mnew[h]);
+#pragma unroll 1
+                for (int blk = 0; blk < 4; ++blk) {
+                    tmem_scale8(lb + kColO + 32u * blk + 8u * hg, f);
+                    tmem_scale8(lb + kColO + 32u * blk + 16u + 8u * hg, f);
+                }
+                tmem_scale8(lb + kColOR + 8u * hg, f);
+                tmem_st_wait();
+            }
+            // P: two E4M3 terms after a power-of-two scale per (32-entry block = this lane
+            // quarter, head), and bf16 for the RoPE dims
+            uint8_t* p8 = sm.p8[s];
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                const int hh = 8 * hg + h;
+                if (mref[h] != -INFINITY) lsum[h] *= exp2f(mref[h] - mnew[h]);
+                mref[h] = mnew[h];
+                const float p = (x[h] == -INFINITY) ? 0.f : exp2f(x[h] - mref[h]);
+                lsum[h] += p;
+                const uint32_t pm = __reduce_max_sync(0xffffffffu, __float_as_uint(p));   // p >= 0
+                // ks = 7 - floor(log2 max p): the scaled block stays below 256
+                const int ks = pm >= 0x00800000u ? max(-126, min(127, 134 - static_cast<int>(pm >> 23))) : 0;
+                const float xs = p * pow2f(ks);
+                const uint32_t hi = f32_to_e4m3(xs);
+                const uint32_t lo = f32_to_e4m3(xs - e4m3_to_f32(hi));
+                p8[sw128(hh, e)] = static_cast<uint8_t>(hi);
+                p8[sw128(16 + hh, e)] = static_cast<uint8_t>(lo);
+                *reinterpret_cast<uint16_t*>(sm.pbf[s][e >> 6] + sw128(hh, 2 * (e & 63))) =
+                    static_cast<uint16_t>(f32_to_bf16_bits(p));
+                if (lane == h) sm.sfb[s][sub][hh] = static_cast<uint32_t>(127 - ks);
+            }
+            fence_proxy_async_smem();
+            named_barrier(kSmBar, 256);
+            if (hg == 0) {   // block-scale word of row `lane` (rows h and 16 + h: head lane & 15)
+                const int hh = lane & 15;
+                const uint32_t wsf = sm.sfb[s][0][hh] | (sm.sfb[s][1][hh] << 8) | (sm.sfb[s][2][hh] << 16) |
+                                     (sm.sfb[s][3][hh] << 24);
+                tmem_st_32x32b_x1(lb + kColSFB + 4u * s, wsf);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.pfull[s]);
+        }
+        // ---- the split's results ---------------------------------------------------------
+        if (ok) {
+            const int tl = n_tiles - 1;
+            ok = !named_barrier_or(kSmBar, 256, !mbar_wait(&sm.pdone[tl & 1], (tl >> 1) & 1));
+        }
+        if (ok) {
+            tc_fence_after();
+            float* ob = opart + part * kHeads * kDim;
+#pragma unroll 1
+            for (int blk = 0; blk < 4; ++blk) {
+                uint32_t oh[8], ol[8];
+                tmem_ld_32x32b_x8(lb + kColO + 32u * blk + 8u * hg, oh);
+                tmem_ld_32x32b_x8(lb + kColO + 32u * blk + 16u + 8u * hg, ol);
+                tmem_ld_wait();
+                const int d = 128 * blk + e;
+                if (d < kNope) {
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) ob[(8 * hg + h) * kDim + d] = __uint_as_float(oh[h]) + __uint_as_float(ol[h]);
+                }
+            }
+            {
+                uint32_t o[8];
+                tmem_ld_32x32b_x8(lb + kColOR + 8u * hg, o);
+                tmem_ld_wait();
+                if (e < kRope) {
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) ob[(8 * hg + h) * kDim + kNope + e] = __uint_as_float(o[h]);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                float v = lsum[h];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == h) sm.lred[sub][8 * hg + h] = v;
+            }
+            named_barrier(kSmBar, 256);
+            if (sub == 0 && lane < 8) {
+                float mine = -INFINITY;
+#pragma unroll
+                for (int h = 0; h < 8; ++h) mine = (lane == h) ? mref[h] : mine;
+                const int hh = 8 * hg + lane;
+                mlpart[part * kHeads + hh] =
+                    make_float2(mine, (sm.lred[0][hh] + sm.lred[1][hh]) + (sm.lred[2][hh] + sm.lred[3][hh]));
+            }
+        } else {
+            *fail = 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (sm.fail) {
+        // a bounded wait gave up: record it, let the copies and MMAs in flight finish (bounded),
+        // publish nothing
+        if (warp == 4 && lane == 0) {
+            dev_error(err, CSLD_DEVERR_TIMEOUT);
+            for (int t = sm.n_landed; t < sm.n_issued; ++t) (void)mbar_wait(&sm.full[t & 1], (t >> 1) & 1);
+            umma_commit(&sm.drain);
+            (void)mbar_wait(&sm.drain, 0);
+        }
+        if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
+        __syncthreads();
+    }
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+size_t attention_tc_smem_bytes() { return sizeof(TcAttnSmem) + 1024; }
+int attention_tc_tile() { return kTcTile; }
+
+cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
+                                        const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                                        const int32_t* seq_len, int B, float scale, int splits, float* opart,
+                                        float2* mlpart, int32_t* err, cudaStream_t stream) {
+    // the caches as 2-D byte tensors [rows][576]: 128-byte boxes with the 128-byte swizzle, 128
+    // rows tall (box copies of contiguous tiles) or one row (the gather4 form)
+    CUtensorMap kv_tile, kv_rows, win_rows;
+    const uint64_t rows = (uint64_t)B * (uint64_t)cap;
+    if (!make_tensor_map_2d_u8(&kv_tile, comp_kv, kEntry, rows, 128, kTcTile) ||
+        !make_tensor_map_2d_u8(&kv_rows, comp_kv, kEntry, rows, 128, 1))
+        return cudaErrorInvalidValue;
+    // a window-less call still passes a valid map (the compressed cache; never read)
+    const bool has_win = W > 0 && win_kv != nullptr;
+    if (!make_tensor_map_2d_u8(&win_rows, has_win ? win_kv : comp_kv, kEntry, has_win ? (uint64_t)B * W : rows, 128, 1))
+        return cudaErrorInvalidValue;
+    const size_t smem = attention_tc_smem_bytes();
+    cudaError_t e = set_smem_once(attention_tc_partial_kernel, smem);
+    if (e != cudaSuccess) return e;
+    attention_tc_partial_kernel<<<dim3(splits, B), kTcThreads, smem, stream>>>(
+        kv_tile, kv_rows, win_rows, q, cap, ratio, topk, k, W, seq_len, scale, splits, opart, mlpart, err);
+    return cudaGetLastError();
+}
+
+}  // namespace csld

@@ -90,6 +90,17 @@ __device__ __forceinline__ uint4 lds128_ordered(const void* p) {
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Named barrier that also ORs a predicate over its threads: every thread gets the same answer,
+// so a group can leave a loop together when any of its threads saw a failed wait.
+__device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
 
 // ------------------------------------------------------------------------------------------
 // Warp-level tensor-core MMAs (legacy mma.sync path; fragments in registers).

@@ -51,5 +51,12 @@ cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t 
 // Device address of the library-owned attention scratch on the current device (looked up on
 // the first call per device).
 cudaError_t attention_static_scratch(void** ptr);
+// The tensor-core (tcgen05) partial kernel of the hybrid decode attention (attention_tc.cu).
+int attention_tc_tile();
+size_t attention_tc_smem_bytes();
+cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
+                                        const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                                        const int32_t* seq_len, int B, float scale, int splits, float* opart,
+                                        float2* mlpart, int32_t* err, cudaStream_t stream);
 
 }  // namespace csld

@@ -41,7 +41,7 @@ def _run(csld, orc, q, comp, ratio, sel, win, W, seq, scale=SCALE):
 
 @pytest.mark.parametrize("B,n,W,ratio", [(1, 4096, 128, 128), (2, 128 * 64 + 5, 128, 128), (3, 1000, 64, 4),
                                          (1, 70, 128, 128), (2, 0, 16, 4), (1, 9, 0, 4), (2, 640, 1, 128),
-                                         (1, 50000, 128, 4)])
+                                         (1, 50000, 128, 4), (32, 128 * 600 + 7, 128, 128), (20, 4 * 3000, 64, 4)])
 def test_dense_matches_oracle(csld, orc, B, n, W, ratio):
     cap = max(2, n // ratio + 8)
     comp, win = _caches(B, cap, W, seed=n + B)
@@ -54,7 +54,8 @@ def test_dense_matches_oracle(csld, orc, B, n, W, ratio):
         assert np.all(out == 0) and np.all(np.isneginf(lse))
 
 
-@pytest.mark.parametrize("B,n_c,k,W", [(1, 1024, 128, 128), (4, 32768, 512, 128), (2, 300, 512, 64), (3, 5000, 1, 8)])
+@pytest.mark.parametrize("B,n_c,k,W", [(1, 1024, 128, 128), (4, 32768, 512, 128), (2, 300, 512, 64), (3, 5000, 1, 8),
+                                       (40, 5000, 1024, 128)])
 def test_sparse_matches_oracle(csld, orc, B, n_c, k, W):
     cap = n_c + 16
     comp, win = _caches(B, cap, W, seed=k + n_c)
