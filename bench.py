@@ -123,16 +123,18 @@ def algorithmic_bytes(wl):
 # sources hash to the value recorded with the capture (a changed kernel reports null).
 PROFILES = {
     "indexer": ("indexer_topk_decode1m.md", "indexer.cu", ""),
-    "csa_attention": ("attention_partial_decode1m.md", "attention.cu", " (CSA)"),
-    "hca_attention": ("attention_partial_decode1m.md", "attention.cu", " (HCA)"),
+    "csa_attention": ("attention_tc_partial_decode1m.md", "attention_tc.cu", " (CSA)"),
+    "hca_attention": ("attention_tc_partial_decode1m.md", "attention_tc.cu", " (HCA)"),
 }
 
 
 def kernel_source_hash(cu):
+    """sha256[:16] of the kernel's source file followed by every shared header (sorted)."""
     import hashlib
+    d = os.path.join(ROOT, "compressed_sparse_long_decode_b200", "csrc")
     h = hashlib.sha256()
-    for f in (cu, "csld_internal.cuh", "kernels.cuh"):
-        with open(os.path.join(ROOT, "compressed_sparse_long_decode_b200", "csrc", f), "rb") as fh:
+    for f in [cu] + sorted(x for x in os.listdir(d) if x.endswith(".cuh")):
+        with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
