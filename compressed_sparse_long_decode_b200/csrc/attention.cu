@@ -30,6 +30,8 @@ __global__ void __launch_bounds__(128) attention_merge_kernel(const float* __res
     __shared__ float fsh[256];
     __shared__ float lw[4];
     const int b = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    pdl_wait();      // the partials come from the partial kernel
+    pdl_trigger();
     const int ns = min(splits, 256);
     // 1) summaries: M = max over non-empty splits, f_j = 2^(m_j - M), L = sum f_j l_j
     float mj[2], lj[2];
@@ -114,7 +116,9 @@ cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t 
     cudaError_t e = launch_attention_tc_partial(q, comp_kv, cap, ratio, topk, k, win_kv, W, seq_len, B, scale,
                                                 plan.splits, opart, mlpart, err, stream);
     if (e != cudaSuccess) return e;
-    attention_merge_kernel<<<dim3(B, kHeads), 128, 0, stream>>>(opart, mlpart, plan.splits, out, lse_out);
+    e = launch_pdl(attention_merge_kernel, dim3(B, kHeads), dim3(128), 0, stream, static_cast<const float*>(opart),
+                   static_cast<const float2*>(mlpart), plan.splits, out, lse_out);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

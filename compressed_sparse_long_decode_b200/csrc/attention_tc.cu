@@ -188,46 +188,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     const int b = blockIdx.y, split = blockIdx.x;
     const int B = gridDim.y;
 
-    // ---- the key list of sequence b and this split's tile range ----------------------------
-    // list = [compressed slots padded to a multiple of 4 with empty slots][window tokens], so a
-    // group of 4 slots never mixes the two sources
-    int32_t n = seq_len[b];
-    if (n < 0) {
-        if (tid == 0 && split == 0) dev_error(err, CSLD_DEVERR_SEQ_LEN);
-        n = 0;
-    }
-    const int64_t n_vis = min64(n / ratio, cap);
-    const bool sparse = topk != nullptr;
-    const int64_t n_comp = sparse ? (int64_t)k : n_vis;
-    const int64_t n_comp4 = (n_comp + 3) & ~int64_t(3);
-    const int n_win = W > 0 ? min(W, n) : 0;
-    const int64_t L = n_comp4 + n_win;
-    const int64_t n_tiles_all = (L + kTcTile - 1) / kTcTile;
-    const int64_t t_begin = n_tiles_all * split / splits;
-    const int n_tiles = static_cast<int>(n_tiles_all * (split + 1) / splits - t_begin);
-    const size_t part = (size_t)b * splits + split;
-    if (n_tiles <= 0) {
-        if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
-        return;
-    }
-    // rows past the end of each map read as zeros
-    const int32_t oob_kv = static_cast<int32_t>(min64((int64_t)B * cap, 0x7FFFFFFF));
-    const int32_t oob_win = static_cast<int32_t>(min64((int64_t)B * max(W, 1), 0x7FFFFFFF));
-    // compressed slot i -> row of the compressed map, or -1 for an empty slot
-    auto comp_row = [&](int64_t i, bool report) -> int32_t {
-        if (i >= n_comp) return -1;
-        int64_t v = i;
-        if (sparse) {
-            v = topk[(size_t)b * k + i];
-            if (v >= n_vis) {
-                if (report) dev_error(err, CSLD_DEVERR_BAD_INDEX);
-                return -1;
-            }
-            if (v < 0) return -1;
-        }
-        return static_cast<int32_t>((int64_t)b * cap + v);
-    };
-
     // ---- setup --------------------------------------------------------------------------------
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -256,10 +216,51 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     tc_fence_before();
     __syncthreads();   // barriers initialised, tensor memory allocated
     tc_fence_after();
+    pdl_wait();      // lengths, top-k indices and the caches come from upstream
+    pdl_trigger();
+
+    // ---- the key list of sequence b and this split's tile range ----------------------------
+    // list = [compressed slots padded to a multiple of 4 with empty slots][window tokens], so a
+    // group of 4 slots never mixes the two sources
+    int32_t n = seq_len[b];
+    if (n < 0) {
+        if (tid == 0 && split == 0) dev_error(err, CSLD_DEVERR_SEQ_LEN);
+        n = 0;
+    }
+    const int64_t n_vis = min64(n / ratio, cap);
+    const bool sparse = topk != nullptr;
+    const int64_t n_comp = sparse ? (int64_t)k : n_vis;
+    const int64_t n_comp4 = (n_comp + 3) & ~int64_t(3);
+    const int n_win = W > 0 ? min(W, n) : 0;
+    const int64_t L = n_comp4 + n_win;
+    const int64_t n_tiles_all = (L + kTcTile - 1) / kTcTile;
+    const int64_t t_begin = n_tiles_all * split / splits;
+    const int n_tiles = static_cast<int>(n_tiles_all * (split + 1) / splits - t_begin);
+    const size_t part = (size_t)b * splits + split;
+    // rows past the end of each map read as zeros
+    const int32_t oob_kv = static_cast<int32_t>(min64((int64_t)B * cap, 0x7FFFFFFF));
+    const int32_t oob_win = static_cast<int32_t>(min64((int64_t)B * max(W, 1), 0x7FFFFFFF));
+    // compressed slot i -> row of the compressed map, or -1 for an empty slot
+    auto comp_row = [&](int64_t i, bool report) -> int32_t {
+        if (i >= n_comp) return -1;
+        int64_t v = i;
+        if (sparse) {
+            v = topk[(size_t)b * k + i];
+            if (v >= n_vis) {
+                if (report) dev_error(err, CSLD_DEVERR_BAD_INDEX);
+                return -1;
+            }
+            if (v < 0) return -1;
+        }
+        return static_cast<int32_t>((int64_t)b * cap + v);
+    };
+
     const uint32_t tmem = sm.tmem_base;
     volatile int32_t* fail = &sm.fail;
 
-    if (warp < 4) {
+    if (n_tiles <= 0) {
+        if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
+    } else if (warp < 4) {
         // ===== copies (warps 0-3): tile t into buffer t & 1, started before the query is ready =====
         int t = 0;
         for (; t < n_tiles; ++t) {
@@ -314,38 +315,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         if (warp == 4 && lane == 0) {
             // ===== MMA issue (one thread) =========================================================
             const uint64_t dq = desc_sw128(sm.qk[0], 0), dqr = desc_sw128(sm.qr, 0);
-            int landed = 0;
-            for (int t = 0; t <= n_tiles; ++t) {
-                if (t < n_tiles) {
-                    const int s = t & 1;
-                    bool ok = !*fail && mbar_wait(&sm.full[s], (t >> 1) & 1);
-                    if (ok) landed = t + 1;
-                    if (ok && t >= 2) ok = mbar_wait(&sm.sfree[s], ((t >> 1) - 1) & 1);
-                    if (!ok) {
-                        *fail = 1;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t dS = tmem + kColS + 32u * s;
-                    const uint64_t da = desc_sw128(sm.tile[s], 0);
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb)
-#pragma unroll
-                        for (int ks = 0; ks < (kb < 3 ? 4 : 2); ++ks)   // 32 bytes of K per MMA; block 3
-                            // stops at byte 448 (the RoPE half is bf16: as E4M3 it may hold NaNs)
-                            umma_f8f6f4(dS, da + (kb * kBlkBytes + 32 * ks) / 16, dq + (kb * 4096 + 32 * ks) / 16, kIdQK,
-                                        (kb | ks) != 0 ? 1u : 0u);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_f16(dS, da + (kRopeBlk * kBlkBytes + 32 * ks) / 16, dqr + (32 * ks) / 16, kIdQKr, 1u);
-                    umma_commit(&sm.sfull[s]);
-                }
-                if (t >= 1) {   // PV of the previous tile
-                    const int u = t - 1, su = u & 1;
-                    if (*fail || !mbar_wait(&sm.pfull[su], (u >> 1) & 1)) {
-                        *fail = 1;
-                        break;
-                    }
+            // Issue whatever is ready, PV first (it frees a tile buffer for the next copy):
+            // PV(np) once P(np) is published; QK(nq) once tile nq landed and its S slot is free.
+            int nq = 0, np = 0, landed = 0;
+            uint32_t idle = 0;
+            while (np < n_tiles) {
+                if (*fail) break;
+                if (np < nq && mbar_try_wait(&sm.pfull[np & 1], (np >> 1) & 1)) {
+                    const int su = np & 1;
                     tc_fence_after();
                     const uint64_t da = desc_sw128(sm.tile[su], 0);
                     const uint64_t dp = desc_sw128(sm.p8[su], 0);
@@ -366,7 +343,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                                  kIdPVr, 1u);
                     umma_commit(&sm.empty[su]);
                     umma_commit(&sm.pdone[su]);
+                    ++np;
+                    idle = 0;
+                    continue;
                 }
+                if (nq < n_tiles && nq < np + 2 && mbar_try_wait(&sm.full[nq & 1], (nq >> 1) & 1) &&
+                    (nq < 2 || mbar_try_wait(&sm.sfree[nq & 1], ((nq >> 1) - 1) & 1))) {
+                    const int s = nq & 1;
+                    landed = nq + 1;
+                    tc_fence_after();
+                    const uint32_t dS = tmem + kColS + 32u * s;
+                    const uint64_t da = desc_sw128(sm.tile[s], 0);
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                        for (int ks = 0; ks < (kb < 3 ? 4 : 2); ++ks)   // 32 bytes of K per MMA; block 3
+                            // stops at byte 448 (the RoPE half is bf16: as E4M3 it may hold NaNs)
+                            umma_f8f6f4(dS, da + (kb * kBlkBytes + 32 * ks) / 16, dq + (kb * 4096 + 32 * ks) / 16, kIdQK,
+                                        (kb | ks) != 0 ? 1u : 0u);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_f16(dS, da + (kRopeBlk * kBlkBytes + 32 * ks) / 16, dqr + (32 * ks) / 16, kIdQKr, 1u);
+                    umma_commit(&sm.sfull[s]);
+                    ++nq;
+                    idle = 0;
+                    continue;
+                }
+                if (++idle > (1u << 22)) {   // nothing became ready for about a second
+                    *fail = 1;
+                    break;
+                }
+                if (idle > 64) __nanosleep(64);
             }
             sm.n_landed = landed;
         }
@@ -577,8 +584,9 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
     const size_t smem = attention_tc_smem_bytes();
     cudaError_t e = set_smem_once(attention_tc_partial_kernel, smem);
     if (e != cudaSuccess) return e;
-    attention_tc_partial_kernel<<<dim3(splits, B), kTcThreads, smem, stream>>>(
-        kv_tile, kv_rows, win_rows, q, cap, ratio, topk, k, W, seq_len, scale, splits, opart, mlpart, err);
+    e = launch_pdl(attention_tc_partial_kernel, dim3(splits, B), dim3(kTcThreads), smem, stream, kv_tile, kv_rows,
+                   win_rows, q, cap, ratio, topk, k, W, seq_len, scale, splits, opart, mlpart, err);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

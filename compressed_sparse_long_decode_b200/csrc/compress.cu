@@ -325,13 +325,17 @@ namespace csld {
 // block, the m tail rows are pooled with the same warp routine as the prefill (so the entry
 // bytes match csld_compress bit for bit) and, for CSA, projected and FP4-quantised.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) append_kernel(csld_layer_cache cache,
-                                                     const uint16_t* __restrict__ kv_new,
-                                                     const float* __restrict__ gate_new,
-                                                     int32_t* err) {
+constexpr int kAppendThreads = 256;
+
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache cache,
+                                                                const uint16_t* __restrict__ kv_new,
+                                                                const float* __restrict__ gate_new,
+                                                                int32_t* err) {
     __shared__ float cbuf[kDim];
-    __shared__ float upart[2][kIdxDim];
+    __shared__ float upart[kAppendThreads / 32][kIdxDim];
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();      // the token and the cache come from upstream
+    pdl_trigger();
     const int m = cache.ratio, W = cache.window;
     const int64_t cap = cache.capacity;
     const int32_t t = cache.seq_len[b];
@@ -345,8 +349,10 @@ __global__ void __launch_bounds__(128) append_kernel(csld_layer_cache cache,
         if (tid == 0) dev_error(err, CSLD_DEVERR_CAPACITY);
         return;
     }
-    const uint2 x = *reinterpret_cast<const uint2*>(kv_new + (size_t)b * kDim + 4 * tid);
-    if (W > 0) {
+    // threads 0..127 move the token (4 dims each); all 256 share the block's projection
+    const bool mover = tid < kDim / 4;
+    const uint2 x = mover ? *reinterpret_cast<const uint2*>(kv_new + (size_t)b * kDim + 4 * tid) : make_uint2(0u, 0u);
+    if (W > 0 && mover) {
         uint8_t* e = cache.win_kv + ((size_t)b * W + (size_t)(t % W)) * kEntry;
         if (tid < kNope / 4) {
             const uint32_t v = f32_to_e4m3(bf16_bits_to_f32(x.x)) |
@@ -360,7 +366,7 @@ __global__ void __launch_bounds__(128) append_kernel(csld_layer_cache cache,
     }
     uint16_t* tail = cache.tail_kv + (size_t)b * m * kDim;
     float* tgate = cache.tail_gate + (size_t)b * m;
-    *reinterpret_cast<uint2*>(tail + (size_t)(t % m) * kDim + 4 * tid) = x;
+    if (mover) *reinterpret_cast<uint2*>(tail + (size_t)(t % m) * kDim + 4 * tid) = x;
     if (tid == 0) tgate[t % m] = gate_new[b];
     if (complete) {
         __syncthreads();  // the new tail row and gate are visible to the whole block
@@ -374,19 +380,26 @@ __global__ void __launch_bounds__(128) append_kernel(csld_layer_cache cache,
         if (cache.has_indexer) {
             __syncthreads();
             // u_j = sum_d bf16(c_d) * bf16(W_I[d][j]) in fp32 (the operands the prefill
-            // projection feeds its tensor cores); two threads per output, 256 dims each.
-            const int j = tid & (kIdxDim - 1), half = tid >> 6;
-            float acc = 0.f;
-            const float* wcol = cache.w_idx + (size_t)(half * (kDim / 2)) * kIdxDim + j;
-#pragma unroll 8
-            for (int d = 0; d < kDim / 2; ++d)
-                acc = fmaf(cbuf[half * (kDim / 2) + d],
-                           bf16_bits_to_f32(f32_to_bf16_bits(wcol[(size_t)d * kIdxDim])), acc);
-            upart[half][j] = acc;
+            // projection feeds its tensor cores).  Warp w takes dims 64w..64w+63, lane outputs
+            // lane and lane + 32: every W_I load is independent and warp-coalesced.
+            float a0 = 0.f, a1 = 0.f;
+            const float* wrow = cache.w_idx + (size_t)(64 * warp) * kIdxDim;
+#pragma unroll 16
+            for (int d = 0; d < 64; ++d) {
+                const float cd = cbuf[64 * warp + d];
+                a0 = fmaf(cd, bf16_bits_to_f32(f32_to_bf16_bits(__ldg(wrow + (size_t)d * kIdxDim + lane))), a0);
+                a1 = fmaf(cd, bf16_bits_to_f32(f32_to_bf16_bits(__ldg(wrow + (size_t)d * kIdxDim + 32 + lane))), a1);
+            }
+            upart[warp][lane] = a0;
+            upart[warp][32 + lane] = a1;
             __syncthreads();
             if (warp == 0) {
-                const float u0 = upart[0][2 * lane] + upart[1][2 * lane];
-                const float u1 = upart[0][2 * lane + 1] + upart[1][2 * lane + 1];
+                float u0 = 0.f, u1 = 0.f;
+#pragma unroll
+                for (int w = 0; w < kAppendThreads / 32; ++w) {
+                    u0 += upart[w][2 * lane];
+                    u1 += upart[w][2 * lane + 1];
+                }
                 warp_store_fp4(cache.ikeys + ((size_t)b * cap + (size_t)s) * kIkey,
                                cache.iscales + ((size_t)b * cap + (size_t)s) * 2, lane, u0, u1);
             }
@@ -397,7 +410,8 @@ __global__ void __launch_bounds__(128) append_kernel(csld_layer_cache cache,
 
 cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
                           const float* gate_new, int32_t* err, cudaStream_t stream) {
-    append_kernel<<<cache.batch, 128, 0, stream>>>(cache, kv_new, gate_new, err);
+    cudaError_t e = launch_pdl(append_kernel, dim3(cache.batch), dim3(kAppendThreads), 0, stream, cache, kv_new, gate_new, err);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
