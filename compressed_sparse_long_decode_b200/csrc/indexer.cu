@@ -72,6 +72,7 @@ constexpr int kRadixBits = 11;
 constexpr int kRadixBins = 1 << kRadixBits;
 constexpr int kIdxSmemAlign = 1024;    // swizzled operand tiles start on 1024-byte boundaries
 constexpr int kCoopSeqWords = 2 * kBins + 1024;   // per sequence: three levels of histograms
+constexpr int kListMax = 8192;       // candidates a sequence's list holds (cooperative fast path)
 
 // Scoring control block: query operand, ring barriers, tensor-memory base, progress.
 struct ScoreCtl {
@@ -229,6 +230,28 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t* red, ui
     }
     *total = all;
     return before;
+}
+
+// Sums a and e over the 512 threads of the block (every thread gets both sums).  red: 32 words
+// no one else uses until the trailing barrier.
+__device__ __forceinline__ void block_sum2(uint32_t a, uint32_t e, uint32_t* red, uint32_t* A, uint32_t* E) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    a = __reduce_add_sync(0xffffffffu, a);
+    e = __reduce_add_sync(0xffffffffu, e);
+    if (lane == 0) {
+        red[warp] = a;
+        red[kIdxWarps + warp] = e;
+    }
+    __syncthreads();
+    uint32_t sa = 0u, se = 0u;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) {
+        sa += red[w];
+        se += red[kIdxWarps + w];
+    }
+    *A = sa;
+    *E = se;
+    __syncthreads();
 }
 
 // Histogram increment with the lanes of a warp that hit the same bin combined into one atomic
@@ -728,8 +751,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
 // ------------------------------------------------------------------------------------------
 struct CoopWs {
     uint32_t* hist;    // [B][kCoopSeqWords]: level 1 (2048 bins), level 2 (2048), level 3 (1024)
-    uint32_t* sync;    // [B][64]: word 0 barrier arrivals, word 1 finished CTAs
+    uint32_t* sync;    // [B][64]: word 0 barrier arrivals, word 1 finished CTAs, word 2 list length
     uint32_t* counts;  // [B][units][2]: keys above the threshold, keys equal to it
+    uint32_t* lkeys;   // [B][kListMax]: candidate list (keys of the threshold bin)
+    uint8_t* lunit;    // [B][kListMax]: the range each listed key comes from
 };
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
@@ -840,6 +865,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     uint32_t* bar = ws.sync + (size_t)b * 64;
     uint32_t* done = bar + 1;
     uint32_t* cnt = ws.counts + (size_t)b * units * 2;
+    uint32_t* lcount = bar + 2;
+    uint32_t* lkeys = ws.lkeys + (size_t)b * kListMax;
+    uint8_t* lunit = ws.lunit + (size_t)b * kListMax;
     const uint32_t nu = static_cast<uint32_t>(units);
 
     for (int i = tid; i < kBins; i += blockDim.x) {
@@ -863,9 +891,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     if (!seq_barrier(bar, 1 * nu, &sm.fail, err)) return;
     uint32_t beta1, need1;
     find_bin_global(g1, kBins, want, sm.red, sm.sel, &beta1, &need1);
-    // --- level 2: bits 20..10.  One pass over the range: each warp counts its keys above bin
-    //     beta1 and copies the keys inside it to its own candidate region (the copy ring is
-    //     idle now); later levels only look at the candidates ---------------------------------
+    // --- candidates: one pass over the range.  Each warp counts its keys above bin beta1 and
+    //     copies the keys inside it to its own candidate region (the copy ring is idle now).
+    //     When the sequence's bin beta1 is small, the candidates of all its ranges go to one
+    //     global list that every CTA then resolves on its own (two barriers in all); otherwise
+    //     two more histogram levels run (bits 20..10, then 9..0) and the ranges exchange their
+    //     counts (four barriers).  The choice is the same in every CTA of the sequence. --------
+    const uint32_t cnt1 = __ldcg(g1 + beta1);
+    const bool fast = cnt1 <= static_cast<uint32_t>(kListMax) && units <= 255;
     constexpr int kSeg = kCoopMaxRange / kIdxWarps;    // warp w owns positions 1024w .. 1024w+1023
     uint32_t* cand = reinterpret_cast<uint32_t*>(&sm.codes[0][0]) + warp * kSeg;
     const int i0 = warp * kSeg;
@@ -880,45 +913,116 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         const uint32_t m = __ballot_sync(0xffffffffu, in);
         if (in) {
             cand[nc + __popc(m & lt)] = key;
-            const uint32_t sub = (key >> 10) & (kBins - 1);
-            const uint32_t same = __match_any_sync(m, sub);   // lanes sharing a bin: one atomic
-            if (lane == __ffs(same) - 1) atomicAdd(&sm.hist2[sub], static_cast<uint32_t>(__popc(same)));
+            if (!fast) {   // level-2 histogram: bits 20..10
+                const uint32_t sub = (key >> 10) & (kBins - 1);
+                const uint32_t same = __match_any_sync(m, sub);   // lanes sharing a bin: one atomic
+                if (lane == __ffs(same) - 1) atomicAdd(&sm.hist2[sub], static_cast<uint32_t>(__popc(same)));
+            }
         }
         nc += __popc(m);
     }
-    __syncthreads();
-    for (int i = tid; i < kBins; i += blockDim.x) {
-        const uint32_t c = sm.hist2[i];
-        if (c) atomicAdd(g2 + i, c);
-    }
-    if (!seq_barrier(bar, 2 * nu, &sm.fail, err)) return;
-    uint32_t beta2, need2;
-    find_bin_global(g2, kBins, need1, sm.red, sm.sel, &beta2, &need2);
-    const uint32_t top22 = (beta1 << 11) | beta2;
-    // --- level 3: bits 9..0 of the candidates whose top 22 bits are (beta1, beta2) -------------
     const int csteps = static_cast<int>((nc + 31) >> 5);
-    for (int s = 0; s < csteps; ++s) {
-        const int j = 32 * s + lane;
-        const uint32_t key = j < static_cast<int>(nc) ? cand[j] : 0u;
-        const bool in = j < static_cast<int>(nc) && (key >> 10) == top22;
-        const uint32_t m = __ballot_sync(0xffffffffu, in);
-        if (in) {
-            const uint32_t low = key & 1023u;
-            const uint32_t same = __match_any_sync(m, low);
-            if (lane == __ffs(same) - 1) atomicAdd(&sm.hist3[low], static_cast<uint32_t>(__popc(same)));
+    uint32_t thr, take_eq, A, E;
+    if (fast) {
+        // this range's candidates -> the sequence's list; its keys above bin beta1 -> counts
+        uint32_t nc_all, gt_all;
+        const uint32_t woff = warp_excl_scan(nc, sm.red + kIdxWarps, &nc_all);
+        (void)warp_excl_scan(gt, sm.red + 2 * kIdxWarps, &gt_all);
+        if (tid == 0) {
+            sm.sel[2] = atomicAdd(lcount, nc_all);
+            cnt[2 * u] = gt_all;
         }
+        __syncthreads();
+        const uint32_t lbase = sm.sel[2] + woff;
+        for (int j = lane; j < static_cast<int>(nc); j += 32) {
+            const uint32_t at = lbase + static_cast<uint32_t>(j);
+            if (at < static_cast<uint32_t>(kListMax)) {
+                lkeys[at] = cand[j];
+                lunit[at] = static_cast<uint8_t>(u);
+            }
+        }
+        if (!seq_barrier(bar, 2 * nu, &sm.fail, err)) return;
+        // every CTA loads the list into the ring's last 32 KB (keys) and hist2 (range ids) and
+        // finds the exact threshold among its keys
+        const int P = static_cast<int>(min(cnt1, static_cast<uint32_t>(kListMax)));
+        uint32_t* lk = reinterpret_cast<uint32_t*>(&sm.codes[0][0]) + kCoopMaxRange;
+        uint8_t* lu = reinterpret_cast<uint8_t*>(sm.hist2);
+        for (int i = tid; i < P; i += blockDim.x) {
+            lk[i] = __ldcg(lkeys + i);
+            lu[i] = __ldcg(lunit + i);
+        }
+        __syncthreads();
+        thr = 0u;
+        take_eq = static_cast<uint32_t>(P);
+        if (static_cast<int>(need1) < P)
+            thr = radix_select([&](int c) { return lk[c]; }, P, static_cast<int>(need1), sm.hist, sm.sel + 2, sm.red,
+                               &take_eq);
+        // selected before this range: the earlier ranges' keys above bin beta1, and their
+        // candidates above / equal to the threshold
+        uint32_t a_loc = 0u, e_loc = 0u;
+        for (int v = tid; v < u; v += blockDim.x) a_loc += __ldcg(cnt + 2 * v);
+        for (int i = tid; i < P; i += blockDim.x)
+            if (lu[i] < u) {
+                a_loc += lk[i] > thr;
+                e_loc += lk[i] == thr;
+            }
+        block_sum2(a_loc, e_loc, sm.red + kIdxWarps, &A, &E);
+    } else {
+        __syncthreads();
+        for (int i = tid; i < kBins; i += blockDim.x) {
+            const uint32_t c = sm.hist2[i];
+            if (c) atomicAdd(g2 + i, c);
+        }
+        if (!seq_barrier(bar, 2 * nu, &sm.fail, err)) return;
+        uint32_t beta2, need2;
+        find_bin_global(g2, kBins, need1, sm.red, sm.sel, &beta2, &need2);
+        const uint32_t top22 = (beta1 << 11) | beta2;
+        // level 3: bits 9..0 of the candidates whose top 22 bits are (beta1, beta2)
+        for (int s = 0; s < csteps; ++s) {
+            const int j = 32 * s + lane;
+            const uint32_t key = j < static_cast<int>(nc) ? cand[j] : 0u;
+            const bool in = j < static_cast<int>(nc) && (key >> 10) == top22;
+            const uint32_t m = __ballot_sync(0xffffffffu, in);
+            if (in) {
+                const uint32_t low = key & 1023u;
+                const uint32_t same = __match_any_sync(m, low);
+                if (lane == __ffs(same) - 1) atomicAdd(&sm.hist3[low], static_cast<uint32_t>(__popc(same)));
+            }
+        }
+        __syncthreads();
+        for (int i = tid; i < 1024; i += blockDim.x) {
+            const uint32_t c = sm.hist3[i];
+            if (c) atomicAdd(g3 + i, c);
+        }
+        if (!seq_barrier(bar, 3 * nu, &sm.fail, err)) return;
+        uint32_t beta3;
+        find_bin_global(g3, 1024, need2, sm.red, sm.sel, &beta3, &take_eq);
+        thr = (top22 << 10) | beta3;
+        // this range's counts, then the counts of the ranges before it
+        uint32_t above = 0u, equal = 0u;
+        for (int s = 0; s < csteps; ++s) {
+            const int j = 32 * s + lane;
+            const uint32_t key = j < static_cast<int>(nc) ? cand[j] : 0u;
+            above += j < static_cast<int>(nc) && key > thr;
+            equal += j < static_cast<int>(nc) && key == thr;
+        }
+        above = gt + __reduce_add_sync(0xffffffffu, above);
+        equal = __reduce_add_sync(0xffffffffu, equal);
+        uint32_t tot;
+        (void)warp_excl_scan((above << 16) | equal, sm.red + kIdxWarps, &tot);   // counts <= 2^14
+        if (tid == 0) {
+            cnt[2 * u] = tot >> 16;
+            cnt[2 * u + 1] = tot & 0xFFFFu;
+        }
+        if (!seq_barrier(bar, 4 * nu, &sm.fail, err)) return;
+        uint32_t a_loc = 0u, e_loc = 0u;
+        for (int v = tid; v < u; v += blockDim.x) {
+            a_loc += __ldcg(cnt + 2 * v);
+            e_loc += __ldcg(cnt + 2 * v + 1);
+        }
+        block_sum2(a_loc, e_loc, sm.red + kIdxWarps, &A, &E);
     }
-    __syncthreads();
-    for (int i = tid; i < 1024; i += blockDim.x) {
-        const uint32_t c = sm.hist3[i];
-        if (c) atomicAdd(g3 + i, c);
-    }
-    if (!seq_barrier(bar, 3 * nu, &sm.fail, err)) return;
-    uint32_t beta3, take_eq;
-    find_bin_global(g3, 1024, need2, sm.red, sm.sel, &beta3, &take_eq);
-    const uint32_t thr = (top22 << 10) | beta3;   // keys > thr are in; of keys == thr the first take_eq
-    // --- this range's counts (keys above bin beta1 plus candidates above thr; candidates equal
-    //     to thr); then the counts of the ranges before it ------------------------------------
+    // this warp's selected keys: above bin beta1, and candidates above / equal to thr
     uint32_t above = 0u, equal = 0u;
     for (int s = 0; s < csteps; ++s) {
         const int j = 32 * s + lane;
@@ -930,31 +1034,6 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     equal = __reduce_add_sync(0xffffffffu, equal);
     uint32_t tot;
     const uint32_t pre = warp_excl_scan((above << 16) | equal, sm.red + kIdxWarps, &tot);   // counts <= 2^14
-    if (tid == 0) {
-        cnt[2 * u] = tot >> 16;
-        cnt[2 * u + 1] = tot & 0xFFFFu;
-    }
-    if (!seq_barrier(bar, 4 * nu, &sm.fail, err)) return;
-    uint32_t a_before = 0u, e_before = 0u;
-    for (int v = tid; v < u; v += blockDim.x) {
-        a_before += __ldcg(cnt + 2 * v);
-        e_before += __ldcg(cnt + 2 * v + 1);
-    }
-    a_before = __reduce_add_sync(0xffffffffu, a_before);
-    e_before = __reduce_add_sync(0xffffffffu, e_before);
-    if (lane == 0) {
-        sm.red[2 * kIdxWarps + warp] = a_before;   // red[32..47]: free after the scan above
-    }
-    __syncthreads();
-    uint32_t A = 0u;
-#pragma unroll
-    for (int w = 0; w < kIdxWarps; ++w) A += sm.red[2 * kIdxWarps + w];
-    __syncthreads();
-    if (lane == 0) sm.red[2 * kIdxWarps + warp] = e_before;
-    __syncthreads();
-    uint32_t E = 0u;
-#pragma unroll
-    for (int w = 0; w < kIdxWarps; ++w) E += sm.red[2 * kIdxWarps + w];
     // --- emit this range's selected entries in index order ------------------------------------
     uint32_t eq_seen = E + (pre & 0xFFFFu);
     uint32_t pos = A + (pre >> 16) + min(eq_seen, take_eq);
@@ -984,6 +1063,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         if (tid == 0) {
             *bar = 0u;
             *done = 0u;
+            *lcount = 0u;
         }
         __threadfence();
     }
@@ -1008,16 +1088,17 @@ static int coop_slots(int num_sms) {
 }
 
 static size_t coop_layout(int B, int units, uint8_t* base, CoopWs* ws) {
-    size_t off = 0;
     const size_t h = up256((size_t)B * kCoopSeqWords * 4), s = up256((size_t)B * 64 * 4),
-                 c = up256((size_t)B * units * 2 * 4);
+                 c = up256((size_t)B * units * 2 * 4), lk = up256((size_t)B * kListMax * 4),
+                 lu = up256((size_t)B * kListMax);
     if (ws) {
-        ws->hist = reinterpret_cast<uint32_t*>(base + off);
-        ws->sync = reinterpret_cast<uint32_t*>(base + off + h);
-        ws->counts = reinterpret_cast<uint32_t*>(base + off + h + s);
+        ws->hist = reinterpret_cast<uint32_t*>(base);
+        ws->sync = reinterpret_cast<uint32_t*>(base + h);
+        ws->counts = reinterpret_cast<uint32_t*>(base + h + s);
+        ws->lkeys = reinterpret_cast<uint32_t*>(base + h + s + c);
+        ws->lunit = base + h + s + c + lk;
     }
-    off += h + s + c;
-    return off;
+    return h + s + c + lk + lu;
 }
 
 IndexerPlan indexer_plan(int B, int64_t cap, int k, int num_sms) {

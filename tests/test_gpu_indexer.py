@@ -121,3 +121,20 @@ def test_indexer_workspace_reused_across_calls(csld, orc):
         assert err.item() == 0
         ref = orc.indexer_topk_batch(ik.numpy(), isc.numpy(), seq.numpy(), 4, q.numpy(), w.numpy(), k)
         H.assert_topk_equal(out.cpu().numpy(), ref)
+
+
+def test_indexer_large_ties_take_the_slow_selection(csld, orc):
+    """More than 8192 keys share the threshold's histogram bin (here: 40,000 identical keys
+    with 300 larger ones planted), so the cooperative kernel resolves the threshold with two
+    more histogram levels instead of its candidate list; ties still go to the lower indices."""
+    B, cap, k = 2, 40000, 512
+    ik = torch.full((B, cap, 32), 0x22, dtype=torch.uint8)     # every code +1.0: identical keys
+    ik[0, 20000:20300, :] = 0x44                                # 300 keys with code +2.0 on seq 0
+    isc = torch.ones((B, cap, 2), dtype=torch.float32)
+    q = torch.ones((B, 4, 64))
+    w = torch.ones((B, 4))
+    seq = torch.full((B,), 4 * cap, dtype=torch.int32)
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, k)
+    H.assert_topk_equal(got, ref)
+    assert np.array_equal(got[1], np.arange(k))
+    assert np.array_equal(got[0], np.concatenate([np.arange(k - 300), np.arange(20000, 20300)]))
