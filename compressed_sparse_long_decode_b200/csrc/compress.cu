@@ -320,7 +320,7 @@ cudaError_t launch_prefill_state(const uint16_t* raw, const float* gate, int64_t
 namespace csld {
 
 // ------------------------------------------------------------------------------------------
-// Decode-time append of one token per sequence (one CTA of 128 threads per sequence).
+// Decode-time append of one token per sequence (one CTA of 256 threads per sequence).
 // Token t = seq_len[b] goes to window slot t mod W and tail slot t mod m; when it completes a
 // block, the m tail rows are pooled with the same warp routine as the prefill (so the entry
 // bytes match csld_compress bit for bit) and, for CSA, projected and FP4-quantised.

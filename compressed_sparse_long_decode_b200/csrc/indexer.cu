@@ -765,9 +765,10 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 
 // Barrier of the CTAs of one sequence: arrival counter *ctr reaches `target`.  The spin is
 // bounded (about half a second); on time-out the device error word gets CSLD_DEVERR_TIMEOUT
-// and false is returned to every thread of the CTA.
+// and false is returned to every thread of the CTA.  The CTA barrier orders every thread's
+// global writes before thread 0's fence and arrival (the fence is cumulative), so only
+// thread 0 fences, as in a grid-wide sync.
 __device__ bool seq_barrier(uint32_t* ctr, uint32_t target, int32_t* fail_flag, int32_t* err) {
-    __threadfence();   // this thread's histogram / count updates before the arrival
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -778,7 +779,7 @@ __device__ bool seq_barrier(uint32_t* ctr, uint32_t target, int32_t* fail_flag, 
                 ok = true;
                 break;
             }
-            if (i >= 16) __nanosleep(64);
+            if (i >= 64) __nanosleep(32);
         }
         if (!ok) {
             dev_error(err, CSLD_DEVERR_TIMEOUT);

@@ -41,7 +41,8 @@ def _run(csld, orc, q, comp, ratio, sel, win, W, seq, scale=SCALE):
 
 @pytest.mark.parametrize("B,n,W,ratio", [(1, 4096, 128, 128), (2, 128 * 64 + 5, 128, 128), (3, 1000, 64, 4),
                                          (1, 70, 128, 128), (2, 0, 16, 4), (1, 9, 0, 4), (2, 640, 1, 128),
-                                         (1, 50000, 128, 4), (32, 128 * 600 + 7, 128, 128), (20, 4 * 3000, 64, 4)])
+                                         (1, 50000, 128, 4), (32, 128 * 600 + 7, 128, 128), (20, 4 * 3000, 64, 4),
+                                         (100, 128 * 20 + 3, 32, 128), (200, 640, 16, 4)])
 def test_dense_matches_oracle(csld, orc, B, n, W, ratio):
     cap = max(2, n // ratio + 8)
     comp, win = _caches(B, cap, W, seed=n + B)
@@ -122,3 +123,4 @@ def test_full_workload_dense_and_sparse(csld, orc, name):
                                  wl.window, seq[:Bs].contiguous())
     assert err == 0
     H.assert_attention_close(out, lse, ro, rl, f"{name} CSA")
+
