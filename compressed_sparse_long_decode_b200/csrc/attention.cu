@@ -21,75 +21,98 @@
 namespace csld {
 
 // Merge the splits of one (sequence, head): out = sum_j 2^(m_j - M) O_j / L,
-// lse = ln 2 * (M + log2 L) with L = sum_j 2^(m_j - M) l_j.  The split summaries go through
-// shared memory; the O rows are read 8 splits at a time so their loads overlap.
-__global__ void __launch_bounds__(128) attention_merge_kernel(const float* __restrict__ opart,
-                                                              const float2* __restrict__ mlpart,
-                                                              int splits, float* __restrict__ out,
-                                                              float* __restrict__ lse_out) {
-    __shared__ float fsh[256];
-    __shared__ float lw[4];
-    const int b = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+// lse = ln 2 * (M + log2 L) with L = sum_j 2^(m_j - M) l_j over the non-empty splits (M = their
+// largest m).  512 threads: thread t owns dims 4 (t % 128) .. +3 and adds every fourth split
+// starting at t / 128; the four partial sums are then added in a fixed order.  Every thread
+// issues its O loads before warp 0 forms the split weights, so the merge costs about one round
+// trip to L2.
+constexpr int kMergeThreads = 512;
+constexpr int kMergeGroups = kMergeThreads / (kDim / 4);   // 4
+constexpr int kMergeU = 8;                                 // O loads a thread keeps in flight
+__global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const float* __restrict__ opart,
+                                                                        const float2* __restrict__ mlpart,
+                                                                        int splits, float* __restrict__ out,
+                                                                        float* __restrict__ lse_out) {
+    __shared__ float fw[256];
+    __shared__ float4 red[kMergeGroups - 1][kDim / 4];
+    __shared__ float mlw[2];
+    const int b = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+    const int d4 = tid % (kDim / 4), g = tid / (kDim / 4);
     pdl_wait();      // the partials come from the partial kernel
     pdl_trigger();
     const int ns = min(splits, 256);
-    // 1) summaries: M = max over non-empty splits, f_j = 2^(m_j - M), L = sum f_j l_j
-    float mj[2], lj[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int j = tid + 128 * r;
-        const float2 ml = j < ns ? mlpart[((size_t)b * splits + j) * kHeads + h] : make_float2(-INFINITY, 0.f);
-        mj[r] = ml.y > 0.f ? ml.x : -INFINITY;
-        lj[r] = ml.y;
-    }
-    float M = fmaxf(mj[0], mj[1]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if ((tid & 31) == 0) fsh[tid >> 5] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(fsh[0], fsh[1]), fmaxf(fsh[2], fsh[3]));
-    __syncthreads();
-    float Lp = 0.f;
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int j = tid + 128 * r;
-        const float f = (M == -INFINITY || mj[r] == -INFINITY) ? 0.f : exp2f(mj[r] - M);
-        if (j < ns) fsh[j] = f;
-        Lp += f * lj[r];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
-    if ((tid & 31) == 0) lw[tid >> 5] = Lp;
-    __syncthreads();
-    const float Lsum = (lw[0] + lw[1]) + (lw[2] + lw[3]);
-    // 2) weighted sum of the O rows; this thread owns dims 4*tid .. 4*tid+3
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4* ob = reinterpret_cast<const float4*>(opart + ((size_t)b * splits * kHeads + h) * kDim) + tid;
+    const float4* ob = reinterpret_cast<const float4*>(opart + ((size_t)b * splits * kHeads + h) * kDim) + d4;
     const size_t jstride = (size_t)kHeads * kDim / 4;
-    for (int j0 = 0; j0 < ns; j0 += 8) {
-        float4 v[8];
+    float4 v[kMergeU];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            v[u] = (j0 + u < ns && fsh[j0 + u] > 0.f) ? ob[(size_t)(j0 + u) * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kMergeU; ++u) {
+        const int j = g + kMergeGroups * u;
+        v[u] = j < ns ? __ldcg(ob + (size_t)j * jstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (tid < 32) {
+        float2 ml[8];
+        float M = -INFINITY;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const float f = (j0 + u < ns) ? fsh[j0 + u] : 0.f;
-            acc.x += f * v[u].x;
-            acc.y += f * v[u].y;
-            acc.z += f * v[u].z;
-            acc.w += f * v[u].w;
+        for (int i = 0; i < 8; ++i) {
+            const int j = lane + 32 * i;
+            ml[i] = j < ns ? __ldcg(&mlpart[((size_t)b * splits + j) * kHeads + h]) : make_float2(-INFINITY, 0.f);
+            if (ml[i].y > 0.f) M = fmaxf(M, ml[i].x);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float Lp = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int j = lane + 32 * i;
+            const float f = (ml[i].y > 0.f && M != -INFINITY) ? exp2f(ml[i].x - M) : 0.f;
+            if (j < ns) fw[j] = f;
+            Lp += f * ml[i].y;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
+        if (lane == 0) {
+            mlw[0] = M;
+            mlw[1] = Lp;
         }
     }
-    if (Lsum > 0.f) {
-        const float inv = 1.f / Lsum;
-        acc.x *= inv;
-        acc.y *= inv;
-        acc.z *= inv;
-        acc.w *= inv;
+    __syncthreads();
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto add = [&](float f, const float4& x) {
+        acc.x = fmaf(f, x.x, acc.x);
+        acc.y = fmaf(f, x.y, acc.y);
+        acc.z = fmaf(f, x.z, acc.z);
+        acc.w = fmaf(f, x.w, acc.w);
+    };
+#pragma unroll
+    for (int u = 0; u < kMergeU; ++u) {
+        const int j = g + kMergeGroups * u;
+        if (j < ns && fw[j] > 0.f) add(fw[j], v[u]);   // empty splits may hold stale rows
     }
-    reinterpret_cast<float4*>(out + ((size_t)b * kHeads + h) * kDim)[tid] = acc;
-    if (lse_out && tid == 0)
-        lse_out[(size_t)b * kHeads + h] = (M == -INFINITY || !(Lsum > 0.f)) ? -INFINITY : (M + log2f(Lsum)) * 0.69314718055994531f;
+    for (int j = g + kMergeGroups * kMergeU; j < ns; j += kMergeGroups)
+        if (fw[j] > 0.f) add(fw[j], __ldcg(ob + (size_t)j * jstride));
+    if (g > 0) red[g - 1][d4] = acc;
+    __syncthreads();
+    if (g == 0) {
+#pragma unroll
+        for (int gg = 0; gg < kMergeGroups - 1; ++gg) {
+            acc.x += red[gg][d4].x;
+            acc.y += red[gg][d4].y;
+            acc.z += red[gg][d4].z;
+            acc.w += red[gg][d4].w;
+        }
+        const float M = mlw[0], Lsum = mlw[1];
+        if (Lsum > 0.f) {
+            const float inv = 1.f / Lsum;
+            acc.x *= inv;
+            acc.y *= inv;
+            acc.z *= inv;
+            acc.w *= inv;
+        }
+        reinterpret_cast<float4*>(out + ((size_t)b * kHeads + h) * kDim)[d4] = acc;
+        if (lse_out && tid == 0)
+            lse_out[(size_t)b * kHeads + h] =
+                (M == -INFINITY || !(Lsum > 0.f)) ? -INFINITY : (M + log2f(Lsum)) * 0.69314718055994531f;
+    }
 }
 
 AttentionPlan attention_plan(int B, int64_t cap, int k, bool sparse, int W, int num_sms) {
@@ -116,7 +139,7 @@ cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t 
     cudaError_t e = launch_attention_tc_partial(q, comp_kv, cap, ratio, topk, k, win_kv, W, seq_len, B, scale,
                                                 plan.splits, opart, mlpart, err, stream);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attention_merge_kernel, dim3(B, kHeads), dim3(128), 0, stream, static_cast<const float*>(opart),
+    e = launch_pdl(attention_merge_kernel, dim3(B, kHeads), dim3(kMergeThreads), 0, stream, static_cast<const float*>(opart),
                    static_cast<const float2*>(mlpart), plan.splits, out, lse_out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -378,17 +378,11 @@ __device__ void select_emit(IdxSmem& sm, int n, int want, Emit emit) {
 // keys into keys[0..cn) and their top-11-bit histogram added into hist (zeroed by the caller).
 // Returns false (and records CSLD_DEVERR_TIMEOUT) if a copy or an MMA did not complete in
 // time.  Called by all 512 threads; allocates and frees NCOLS columns of tensor memory.
+// Scoring setup, which reads nothing produced upstream: the ring's barriers, the tensor memory
+// (NCOLS columns) and the tensor-map prefetch.  Block-wide; ends with a CTA barrier.
 template <int S, uint32_t NCOLS>
-__device__ bool score_chunk(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], float (*scales)[kIdxTile * 2],
-                            uint32_t* keys, uint32_t* hist, const CUtensorMap& kmap, const float* iscales,
-                            int64_t cap, int b, int64_t c0, int cn, const float* q_idx, const float* head_w,
-                            int32_t* err) {
-    static_assert(S <= kMaxStages, "ring depth");
-    static_assert(16 * S + 16 <= static_cast<int>(NCOLS), "accumulator slots and scale factors fit");
-    constexpr uint32_t kIdxTmemCols = NCOLS, kIdxSfCol = NCOLS - 16;
+__device__ void score_setup(ScoreCtl& ctl, const CUtensorMap& kmap) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
-    volatile int32_t* fail = &ctl.fail;
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&ctl.full[s], 1);
@@ -402,13 +396,37 @@ __device__ bool score_chunk(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], f
         fence_barrier_init();
     }
     if (warp == kIdxMmaWarp) {
-        tmem_alloc(&ctl.tmem_base, kIdxTmemCols);
+        tmem_alloc(&ctl.tmem_base, NCOLS);
         tmem_relinquish();
     }
     if (warp == kIdxProducerWarp && lane == 0) tma_prefetch_map(&kmap);
     tc_fence_before();
     __syncthreads();   // barriers initialised, tensor memory allocated
     tc_fence_after();
+}
+
+// Gives back the tensor memory of score_setup when no chunk is scored.
+template <uint32_t NCOLS>
+__device__ void score_release(ScoreCtl& ctl) {
+    if ((threadIdx.x >> 5) == kIdxMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(ctl.tmem_base, NCOLS);
+    }
+}
+
+// Scores entries c0 .. c0 + cn - 1 of sequence b after score_setup (and gives the tensor
+// memory back).
+template <int S, uint32_t NCOLS>
+__device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], float (*scales)[kIdxTile * 2],
+                          uint32_t* keys, uint32_t* hist, const CUtensorMap& kmap, const float* iscales,
+                          int64_t cap, int b, int64_t c0, int cn, const float* q_idx, const float* head_w,
+                          int32_t* err) {
+    static_assert(S <= kMaxStages, "ring depth");
+    static_assert(16 * S + 16 <= static_cast<int>(NCOLS), "accumulator slots and scale factors fit");
+    constexpr uint32_t kIdxTmemCols = NCOLS, kIdxSfCol = NCOLS - 16;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
+    volatile int32_t* fail = &ctl.fail;
     const uint32_t tmem = ctl.tmem_base;
     const float* sbase = iscales + ((size_t)b * cap + (size_t)c0) * 2;
     if (warp == kIdxProducerWarp) {
@@ -560,6 +578,15 @@ __device__ bool score_chunk(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], f
         tmem_dealloc(tmem, kIdxTmemCols);
     }
     return ok;
+}
+
+template <int S, uint32_t NCOLS>
+__device__ bool score_chunk(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], float (*scales)[kIdxTile * 2],
+                            uint32_t* keys, uint32_t* hist, const CUtensorMap& kmap, const float* iscales,
+                            int64_t cap, int b, int64_t c0, int cn, const float* q_idx, const float* head_w,
+                            int32_t* err) {
+    score_setup<S, NCOLS>(ctl, kmap);
+    return score_run<S, NCOLS>(ctl, codes, scales, keys, hist, kmap, iscales, cap, b, c0, cn, q_idx, head_w, err);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -844,6 +871,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     const uint32_t lt = (1u << lane) - 1u;
     const int b = blockIdx.y, u = blockIdx.x;
 
+    for (int i = tid; i < kBins; i += blockDim.x) {
+        sm.hist[i] = 0u;
+        sm.hist2[i] = 0u;
+    }
+    for (int i = tid; i < 1024; i += blockDim.x) sm.hist3[i] = 0u;
+    if (tid == 0) sm.fail = 0;
+    score_setup<kCoopStages, 256>(sm.ctl, kmap);
+
     int64_t n_b = seq_len[b];
     n_b = n_b < 0 ? 0 : n_b / ratio;
     if (n_b > cap) n_b = cap;
@@ -854,6 +889,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     if (n_b <= k) {
         // every visible entry is selected: no scores needed, and no barrier (the whole
         // sequence takes this branch); entry i goes to position i, the rest is -1
+        score_release<256>(sm.ctl);
         for (int i = tid; i < cn; i += blockDim.x) out[c0 + i] = static_cast<int32_t>(c0 + i);
         if (u == 0)
             for (int64_t i = n_b + tid; i < k; i += blockDim.x) out[i] = -1;
@@ -871,17 +907,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     uint8_t* lunit = ws.lunit + (size_t)b * kListMax;
     const uint32_t nu = static_cast<uint32_t>(units);
 
-    for (int i = tid; i < kBins; i += blockDim.x) {
-        sm.hist[i] = 0u;
-        sm.hist2[i] = 0u;
-    }
-    for (int i = tid; i < 1024; i += blockDim.x) sm.hist3[i] = 0u;
-    if (tid == 0) sm.fail = 0;
-    __syncthreads();
     bool ok = true;
     if (cn > 0)
-        ok = score_chunk<kCoopStages, 256>(sm.ctl, sm.codes, sm.scales, sm.keys, sm.hist, kmap, iscales, cap, b, c0, cn,
-                                      q_idx, head_w, err);
+        ok = score_run<kCoopStages, 256>(sm.ctl, sm.codes, sm.scales, sm.keys, sm.hist, kmap, iscales, cap, b, c0, cn,
+                                         q_idx, head_w, err);
+    else
+        score_release<256>(sm.ctl);
     __syncthreads();
     // --- level 1: bits 31..21 ------------------------------------------------------------------
     if (ok)
