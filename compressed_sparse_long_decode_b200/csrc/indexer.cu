@@ -821,7 +821,7 @@ __device__ bool seq_barrier(uint32_t* ctr, uint32_t target, int32_t* fail_flag, 
 // From a global histogram g of nbins bins (2048 or 1024), the bin holding the want-th largest
 // key and how many keys are wanted inside it (*need).  Block-wide; g read through L2.
 __device__ void find_bin_global(const uint32_t* g, int nbins, uint32_t want, uint32_t* red, uint32_t* sel,
-                                uint32_t* bin, uint32_t* need) {
+                                uint32_t* bin, uint32_t* need, uint32_t* count = nullptr) {
     const int tid = threadIdx.x, lane = tid & 31;
     const int per = nbins / kIdxThreads;     // 4 or 2 bins per thread, from the top
     uint32_t c[4] = {0u, 0u, 0u, 0u}, tot = 0u;
@@ -838,6 +838,7 @@ __device__ void find_bin_global(const uint32_t* g, int nbins, uint32_t want, uin
     if (tid == 0) {
         sel[0] = 0u;
         sel[1] = 0u;
+        sel[2] = 0u;
     }
     uint32_t all;
     const uint32_t wb = warp_excl_scan(__shfl_sync(0xffffffffu, incl, 31), red, &all);
@@ -848,6 +849,7 @@ __device__ void find_bin_global(const uint32_t* g, int nbins, uint32_t want, uin
             if (run + c[q] >= want) {
                 sel[0] = static_cast<uint32_t>(nbins - 1 - per * tid - q);
                 sel[1] = want - run;
+                sel[2] = c[q];
                 break;
             }
             run += c[q];
@@ -856,6 +858,7 @@ __device__ void find_bin_global(const uint32_t* g, int nbins, uint32_t want, uin
     __syncthreads();
     *bin = sel[0];
     *need = sel[1];
+    if (count != nullptr) *count = sel[2];
     __syncthreads();
 }
 
@@ -921,28 +924,30 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             if (c) atomicAdd(g1 + i, c);
         }
     if (!seq_barrier(bar, 1 * nu, &sm.fail, err)) return;
-    uint32_t beta1, need1;
-    find_bin_global(g1, kBins, want, sm.red, sm.sel, &beta1, &need1);
+    uint32_t beta1, need1, cnt1;
+    find_bin_global(g1, kBins, want, sm.red, sm.sel, &beta1, &need1, &cnt1);
     // --- candidates: one pass over the range.  Each warp counts its keys above bin beta1 and
     //     copies the keys inside it to its own candidate region (the copy ring is idle now).
     //     When the sequence's bin beta1 is small, the candidates of all its ranges go to one
     //     global list that every CTA then resolves on its own (two barriers in all); otherwise
     //     two more histogram levels run (bits 20..10, then 9..0) and the ranges exchange their
     //     counts (four barriers).  The choice is the same in every CTA of the sequence. --------
-    const uint32_t cnt1 = __ldcg(g1 + beta1);
     const bool fast = cnt1 <= static_cast<uint32_t>(kListMax) && units <= 255;
     constexpr int kSeg = kCoopMaxRange / kIdxWarps;    // warp w owns positions 1024w .. 1024w+1023
     uint32_t* cand = reinterpret_cast<uint32_t*>(&sm.codes[0][0]) + warp * kSeg;
     const int i0 = warp * kSeg;
     const int steps = max(0, min(kSeg, cn - i0) + 31) >> 5;
     uint32_t gt = 0u, nc = 0u;
+    uint32_t cmask = 0u;   // 32-key steps of this warp's segment holding a key of bin >= beta1
     for (int s = 0; s < steps; ++s) {
         const int i = i0 + 32 * s + lane;
         const uint32_t key = i < cn ? sm.keys[i] : 0u;
         const uint32_t bin = key >> kBinShift;
-        gt += __popc(__ballot_sync(0xffffffffu, i < cn && bin > beta1));
+        const uint32_t ma = __ballot_sync(0xffffffffu, i < cn && bin > beta1);
+        gt += __popc(ma);
         const bool in = i < cn && bin == beta1;
         const uint32_t m = __ballot_sync(0xffffffffu, in);
+        if ((ma | m) != 0u) cmask |= 1u << s;
         if (in) {
             cand[nc + __popc(m & lt)] = key;
             if (!fast) {   // level-2 histogram: bits 20..10
@@ -979,6 +984,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         const int P = static_cast<int>(min(cnt1, static_cast<uint32_t>(kListMax)));
         uint32_t* lk = reinterpret_cast<uint32_t*>(&sm.codes[0][0]) + kCoopMaxRange;
         uint8_t* lu = reinterpret_cast<uint8_t*>(sm.hist2);
+        uint32_t a_loc = 0u, e_loc = 0u;
+        for (int v = tid; v < u; v += blockDim.x) a_loc += __ldcg(cnt + 2 * v);   // with the list loads
         for (int i = tid; i < P; i += blockDim.x) {
             lk[i] = __ldcg(lkeys + i);
             lu[i] = __ldcg(lunit + i);
@@ -989,10 +996,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         if (static_cast<int>(need1) < P)
             thr = radix_select([&](int c) { return lk[c]; }, P, static_cast<int>(need1), sm.hist, sm.sel + 2, sm.red,
                                &take_eq);
-        // selected before this range: the earlier ranges' keys above bin beta1, and their
-        // candidates above / equal to the threshold
-        uint32_t a_loc = 0u, e_loc = 0u;
-        for (int v = tid; v < u; v += blockDim.x) a_loc += __ldcg(cnt + 2 * v);
+        // selected before this range: the earlier ranges' keys above bin beta1 (a_loc, loaded
+        // above), and their candidates above / equal to the threshold
         for (int i = tid; i < P; i += blockDim.x)
             if (lu[i] < u) {
                 a_loc += lk[i] > thr;
@@ -1069,7 +1074,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     // --- emit this range's selected entries in index order ------------------------------------
     uint32_t eq_seen = E + (pre & 0xFFFFu);
     uint32_t pos = A + (pre >> 16) + min(eq_seen, take_eq);
-    for (int s = 0; s < steps; ++s) {
+    // only steps with a key of bin >= beta1 can hold a selected key (the threshold lies in bin
+    // beta1), so the others are skipped
+    for (uint32_t mk = cmask; mk != 0u; mk &= mk - 1u) {
+        const int s = __ffs(mk) - 1;
         const int i = i0 + 32 * s + lane;
         const uint32_t key = i < cn ? sm.keys[i] : 0u;
         const bool veq = i < cn && key == thr;
