@@ -211,7 +211,7 @@ def run_ours(args, rank, world, local_rank):
             c.tail_kv.normal_(generator=g)
             c.seq_len.fill_(wl.context)
         ik, isc = synth.random_ikeys(B, csa.capacity, g, dev, heavy_frac=wl.heavy_frac, n_valid=wl.csa_entries)
-        csa.ikeys.copy_(ik)
+        csa.ikeys.copy_(synth.ikeys_swap_halves(ik))   # the cache's stored layout
         csa.iscales.copy_(isc)
         del ik, isc
         layers.append((csa, hca))

@@ -163,7 +163,6 @@ csld_status indexer_topk(const uint8_t* ikeys, const float* iscales, int64_t cap
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CSLD_ERR_ALIGN, "workspace must be 256-byte aligned");
     cudaError_t e = csld::launch_indexer(ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, B, k,
                                          topk_out, ws, plan, err, as_stream(stream));
-    if (e == cudaErrorNotSupported) return fail(CSLD_ERR_UNSUPPORTED, "no tensor-map encoder in this driver");
     if (e != cudaSuccess) return cuda_fail(e, "indexer_topk");
     return CSLD_OK;
 }

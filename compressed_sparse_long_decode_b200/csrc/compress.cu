@@ -118,15 +118,17 @@ __device__ __forceinline__ void warp_store_entry(uint8_t* __restrict__ entry, in
 }
 
 // FP4-quantises the 64-vector u (lane l holds u[2l], u[2l+1]) into 32 code bytes + 2 scales.
+// Entry s's code bytes go to their stored positions: the two 16-byte halves (the two
+// 32-element groups) are swapped when bit 2 of s is set (the key cache layout of csld.h).
 __device__ __forceinline__ void warp_store_fp4(uint8_t* __restrict__ codes, float* __restrict__ scales,
-                                               int lane, float u0, float u1) {
+                                               int64_t s, int lane, float u0, float u1) {
     float amax = fmaxf(fabsf(u0), fabsf(u1));
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sg = fp4_group_scale(amax);    // lanes 0..15: group 0, lanes 16..31: group 1
     const float inv = 1.0f / sg;               // exact: sg is a power of two
     const uint32_t byte = e2m1_code(u0 * inv) | (e2m1_code(u1 * inv) << 4);
-    codes[lane] = static_cast<uint8_t>(byte);
+    codes[lane ^ (static_cast<int>((s >> 2) & 1) << 4)] = static_cast<uint8_t>(byte);
     if ((lane & 15) == 0) scales[lane >> 4] = sg;
 }
 
@@ -243,7 +245,7 @@ __global__ void __launch_bounds__(256) pool_index_kernel(
             const float u0 = sm.u[r * kUStride + 2 * lane];
             const float u1 = sm.u[r * kUStride + 2 * lane + 1];
             warp_store_fp4(ikey_out + ((size_t)b * out_seq_stride + (size_t)s) * kIkey,
-                           iscale_out + ((size_t)b * out_seq_stride + (size_t)s) * 2, lane, u0, u1);
+                           iscale_out + ((size_t)b * out_seq_stride + (size_t)s) * 2, s, lane, u0, u1);
         }
     }
 }
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
                     u1 += upart[w][2 * lane + 1];
                 }
                 warp_store_fp4(cache.ikeys + ((size_t)b * cap + (size_t)s) * kIkey,
-                               cache.iscales + ((size_t)b * cap + (size_t)s) * 2, lane, u0, u1);
+                               cache.iscales + ((size_t)b * cap + (size_t)s) * 2, s, lane, u0, u1);
             }
         }
     }

@@ -55,6 +55,7 @@ constexpr int kIdxWarps = kIdxThreads / 32;
 constexpr int kIdxTile = 256;          // entries per pipeline stage: two 128-row MMAs
 constexpr int kIdxStages = 4;          // ring depth of the merge-tree kernel (shares the candidate area)
 constexpr int kCoopStages = 12;        // ring depth of the cooperative kernel (one CTA per SM)
+constexpr int kCoopGroup = 4;          // tiles per key copy in the cooperative kernel (32 KB of codes)
 constexpr int kMaxStages = 12;
 constexpr int kIdxEpiGroups = 3;       // epilogue warpgroups: warps 0..11
 constexpr int kIdxProducerWarp = 12;   // issues the tensor / bulk copies
@@ -381,8 +382,8 @@ __device__ void select_emit(IdxSmem& sm, int n, int want, Emit emit) {
 // Scoring setup, which reads nothing produced upstream: the ring's barriers, the tensor memory
 // (NCOLS columns) and the tensor-map prefetch.  Block-wide; ends with a CTA barrier.
 template <int S, uint32_t NCOLS>
-__device__ void score_setup(ScoreCtl& ctl, const CUtensorMap& kmap) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ void score_setup(ScoreCtl& ctl) {
+    const int tid = threadIdx.x, warp = tid >> 5;
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&ctl.full[s], 1);
@@ -399,7 +400,6 @@ __device__ void score_setup(ScoreCtl& ctl, const CUtensorMap& kmap) {
         tmem_alloc(&ctl.tmem_base, NCOLS);
         tmem_relinquish();
     }
-    if (warp == kIdxProducerWarp && lane == 0) tma_prefetch_map(&kmap);
     tc_fence_before();
     __syncthreads();   // barriers initialised, tensor memory allocated
     tc_fence_after();
@@ -415,33 +415,45 @@ __device__ void score_release(ScoreCtl& ctl) {
 }
 
 // Scores entries c0 .. c0 + cn - 1 of sequence b after score_setup (and gives the tensor
-// memory back).
-template <int S, uint32_t NCOLS>
+// memory back).  The ring has S tile stages, filled GT tiles at a time: one 1-D bulk copy of
+// the GT tiles' key codes (stored pre-swizzled, so the bytes land in the MMA's operand layout)
+// and one of their scales, completing on the group's first stage barrier.  Larger copies keep
+// the DRAM stream denser than one 8 KB tile per request.
+template <int S, int GT, uint32_t NCOLS>
 __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], float (*scales)[kIdxTile * 2],
-                          uint32_t* keys, uint32_t* hist, const CUtensorMap& kmap, const float* iscales,
+                          uint32_t* keys, uint32_t* hist, const uint8_t* ikeys, const float* iscales,
                           int64_t cap, int b, int64_t c0, int cn, const float* q_idx, const float* head_w,
                           int32_t* err) {
     static_assert(S <= kMaxStages, "ring depth");
+    static_assert(S % GT == 0 && S / GT >= 2, "the ring holds at least two copy groups");
     static_assert(16 * S + 16 <= static_cast<int>(NCOLS), "accumulator slots and scale factors fit");
+    constexpr int kGroups = S / GT;
     constexpr uint32_t kIdxTmemCols = NCOLS, kIdxSfCol = NCOLS - 16;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n_tiles = (cn + kIdxTile - 1) / kIdxTile;
     volatile int32_t* fail = &ctl.fail;
     const uint32_t tmem = ctl.tmem_base;
+    const uint8_t* cbase = ikeys + ((size_t)b * cap + (size_t)c0) * kIkey;
     const float* sbase = iscales + ((size_t)b * cap + (size_t)c0) * 2;
     if (warp == kIdxProducerWarp) {
-        // --- producer: key tile (TMA, swizzled) + its scales (bulk copy) per stage -------
+        // --- producer: GT tiles of key codes + their scales per copy group ----------------
         if (lane == 0) {
             int t = 0;
-            for (; t < n_tiles; ++t) {
-                const int s = t % S;
+            for (int g = 0; t < n_tiles; ++g) {
+                const int s0 = (g % kGroups) * GT;
                 if (*fail) break;
-                if (t >= S && !mbar_wait(&ctl.empty[s], ((t / S) - 1) & 1)) break;
-                const int nt = min(kIdxTile, cn - t * kIdxTile);
-                const uint32_t sb = static_cast<uint32_t>((nt + 1) & ~1) * 8u;   // cap is even
-                mbar_arrive_expect_tx(&ctl.full[s], kIdxTile * kIkey + sb);
-                tma_load_3d(codes[s], &kmap, 0, static_cast<int>(c0) + t * kIdxTile, b, &ctl.full[s]);
-                bulk_g2s(scales[s], sbase + (size_t)t * kIdxTile * 2, sb, &ctl.full[s]);
+                bool free = true;   // the group's stages held tiles t - S .. t - S + GT - 1
+                if (g >= kGroups)
+                    for (int i = 0; i < GT && free; ++i)
+                        free = mbar_wait(&ctl.empty[s0 + i], ((g / kGroups) - 1) & 1);
+                if (!free) break;
+                const int ne = min(GT * kIdxTile, cn - t * kIdxTile);          // entries in the group
+                const uint32_t cb = static_cast<uint32_t>(ne) * kIkey;
+                const uint32_t sb = static_cast<uint32_t>((ne + 1) & ~1) * 8u;   // cap is even
+                mbar_arrive_expect_tx(&ctl.full[s0], cb + sb);
+                bulk_g2s(codes[s0], cbase + (size_t)t * kIdxTile * kIkey, cb, &ctl.full[s0]);
+                bulk_g2s(scales[s0], sbase + (size_t)t * kIdxTile * 2, sb, &ctl.full[s0]);
+                t = min(n_tiles, t + GT);
             }
             ctl.n_issued = t;
             if (t < n_tiles) *fail = 1;
@@ -492,7 +504,8 @@ __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], flo
                 int t = 0;
                 for (; t < n_tiles; ++t) {
                     const int s = t % S;
-                    if (*fail || !mbar_wait(&ctl.full[s], (t / S) & 1)) break;
+                    // a copy group lands as a whole on the barrier of its first stage
+                    if (*fail || (t % GT == 0 && !mbar_wait(&ctl.full[s], ((t / GT) / kGroups) & 1))) break;
                     tc_fence_after();
                     const uint32_t d = tmem + 16u * static_cast<uint32_t>(s);
                     umma_mxf4(d, smem_desc_kmajor_sw32(codes[s]), bdesc, kIdxIdesc, sfa, sfb, 0u);
@@ -566,8 +579,8 @@ __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], flo
         // memory are reused.
         if (warp == kIdxMmaWarp && lane == 0) {
             dev_error(err, CSLD_DEVERR_TIMEOUT);
-            for (int t = ctl.n_mma; t < ctl.n_issued; ++t)
-                (void)mbar_wait(&ctl.full[t % S], (t / S) & 1);
+            for (int t = (ctl.n_mma + GT - 1) / GT * GT; t < ctl.n_issued; t += GT)
+                (void)mbar_wait(&ctl.full[t % S], ((t / GT) / kGroups) & 1);
             umma_commit(&ctl.drain);
             (void)mbar_wait(&ctl.drain, 0);
         }
@@ -580,13 +593,14 @@ __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], flo
     return ok;
 }
 
-template <int S, uint32_t NCOLS>
+template <int S, int GT, uint32_t NCOLS>
 __device__ bool score_chunk(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], float (*scales)[kIdxTile * 2],
-                            uint32_t* keys, uint32_t* hist, const CUtensorMap& kmap, const float* iscales,
+                            uint32_t* keys, uint32_t* hist, const uint8_t* ikeys, const float* iscales,
                             int64_t cap, int b, int64_t c0, int cn, const float* q_idx, const float* head_w,
                             int32_t* err) {
-    score_setup<S, NCOLS>(ctl, kmap);
-    return score_run<S, NCOLS>(ctl, codes, scales, keys, hist, kmap, iscales, cap, b, c0, cn, q_idx, head_w, err);
+    score_setup<S, NCOLS>(ctl);
+    return score_run<S, GT, NCOLS>(ctl, codes, scales, keys, hist, ikeys, iscales, cap, b, c0, cn, q_idx, head_w,
+                                   err);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -640,7 +654,7 @@ static IdxTree tree_layout(int B, int n_chunks, int kc, int k, int group, uint8_
 // The merge-tree kernel.
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
-    const __grid_constant__ CUtensorMap kmap, const float* __restrict__ iscales, int64_t cap,
+    const uint8_t* __restrict__ ikeys, const float* __restrict__ iscales, int64_t cap,
     const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
     const float* __restrict__ head_w, int chunk, int kc, int k, IdxTree tree,
     int32_t* __restrict__ topk_out, int32_t* err) {
@@ -659,7 +673,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
     for (int i = tid; i < kBins; i += blockDim.x) sm.hist[i] = 0u;
     bool chunk_ok = true;
     if (cn > 0)
-        chunk_ok = score_chunk<kIdxStages, 128>(sm.ctl, sm.u.pipe.codes, sm.u.pipe.scales, sm.keys, sm.hist, kmap, iscales,
+        chunk_ok = score_chunk<kIdxStages, 1, 128>(sm.ctl, sm.u.pipe.codes, sm.u.pipe.scales, sm.keys, sm.hist, ikeys, iscales,
                                            cap, b, c0, cn, q_idx, head_w, err);
     __syncthreads();
     // --- selection and the merge tree ------------------------------------------------------
@@ -863,7 +877,7 @@ __device__ void find_bin_global(const uint32_t* g, int nbins, uint32_t want, uin
 }
 
 __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
-    const __grid_constant__ CUtensorMap kmap, const float* __restrict__ iscales, int64_t cap,
+    const uint8_t* __restrict__ ikeys, const float* __restrict__ iscales, int64_t cap,
     const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
     const float* __restrict__ head_w, int chunk, int units, int k, CoopWs ws,
     int32_t* __restrict__ topk_out, int32_t* err) {
@@ -880,7 +894,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     }
     for (int i = tid; i < 1024; i += blockDim.x) sm.hist3[i] = 0u;
     if (tid == 0) sm.fail = 0;
-    score_setup<kCoopStages, 256>(sm.ctl, kmap);
+    score_setup<kCoopStages, 256>(sm.ctl);
 
     int64_t n_b = seq_len[b];
     n_b = n_b < 0 ? 0 : n_b / ratio;
@@ -912,7 +926,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
 
     bool ok = true;
     if (cn > 0)
-        ok = score_run<kCoopStages, 256>(sm.ctl, sm.codes, sm.scales, sm.keys, sm.hist, kmap, iscales, cap, b, c0, cn,
+        ok = score_run<kCoopStages, kCoopGroup, 256>(sm.ctl, sm.codes, sm.scales, sm.keys, sm.hist, ikeys, iscales, cap, b,
+                                                     c0, cn,
                                          q_idx, head_w, err);
     else
         score_release<256>(sm.ctl);
@@ -1215,19 +1230,6 @@ cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t c
                            const int32_t* seq_len, int ratio, const float* q_idx,
                            const float* head_w, int B, int k, int32_t* topk_out, void* ws,
                            const IndexerPlan& plan, int32_t* err, cudaStream_t stream) {
-    // Key codes as a 3-D byte tensor [B][cap][32]; one box = one stage of 256 entries.  Rows
-    // past cap read as zeros (their scores are never used).
-    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-    if (encode == nullptr) return cudaErrorNotSupported;
-    CUtensorMap kmap;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kIkey), static_cast<cuuint64_t>(cap), static_cast<cuuint64_t>(B)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kIkey), static_cast<cuuint64_t>(cap) * kIkey};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kIkey), static_cast<cuuint32_t>(kIdxTile), 1u};
-    const cuuint32_t estr[3] = {1u, 1u, 1u};
-    if (encode(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(ikeys), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
     if (plan.coop) {
         CoopWs cws;
         coop_layout(B, plan.n_chunks, static_cast<uint8_t*>(ws), &cws);
@@ -1244,7 +1246,7 @@ cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t c
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, indexer_topk_coop_kernel, kmap, iscales, cap, seq_len, ratio, q_idx, head_w,
+        e = cudaLaunchKernelEx(&cfg, indexer_topk_coop_kernel, ikeys, iscales, cap, seq_len, ratio, q_idx, head_w,
                                plan.chunk, plan.n_chunks, k, cws, topk_out, err);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
@@ -1255,7 +1257,7 @@ cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t c
     cudaError_t e = set_smem_once(indexer_topk_kernel, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(plan.n_chunks, B);
-    indexer_topk_kernel<<<grid, kIdxThreads, smem, stream>>>(kmap, iscales, cap, seq_len, ratio,
+    indexer_topk_kernel<<<grid, kIdxThreads, smem, stream>>>(ikeys, iscales, cap, seq_len, ratio,
                                                              q_idx, head_w, plan.chunk, plan.kc, k,
                                                              tree, topk_out, err);
     return cudaGetLastError();

@@ -54,7 +54,9 @@ extern "C" {
 #define CSLD_HEADS 16           /* query heads sharing the KV head (decode kernel) */
 #define CSLD_IDX_HEADS 4        /* lightning-indexer heads */
 #define CSLD_IDX_DIM 64         /* lightning-indexer dims per head (one key shared by the heads) */
-#define CSLD_IKEY_BYTES 32      /* 64 E2M1 codes, element 2i in the low nibble of byte i */
+#define CSLD_IKEY_BYTES 32      /* 64 E2M1 codes, element 2i in the low nibble of byte i,
+                                   stored with halves swapped when bit 2 of the entry index
+                                   is set (see "Indexer key storage" below) */
 #define CSLD_IKEY_SCALES 2      /* fp32 power-of-two scale per group of 32 codes */
 #define CSLD_MAX_RATIO 128      /* tokens per compressed entry: 1..128 (CSA 4, HCA 128) */
 #define CSLD_MAX_WINDOW 1024    /* sliding-window length in raw tokens: 0..1024 */
@@ -82,12 +84,23 @@ CSLD_API const char* csld_last_error(void);
 CSLD_API const char* csld_status_string(csld_status s);
 
 /* ----------------------------------------------------------------------------------------
+ * Indexer key storage.  Entry s of a key array ([..][cap][32] u8) holds the 64 E2M1 codes of
+ * its key: logical byte c (elements 2c and 2c+1; bytes 0..15 are group 0, 16..31 group 1)
+ * is stored at byte  s*32 + (c XOR 16*((s >> 2) & 1)),  i.e. the two 16-byte halves trade
+ * places in entries 4..7 of every 8.  That is the 32-byte-swizzled K-major operand layout of
+ * the tensor cores, so a run of entries that starts at a multiple of 8 is copied into shared
+ * memory byte for byte and used as an MMA operand as it lands.  csld_compress and
+ * kv_cache_append write this layout and indexer_topk reads it; the swap is its own inverse.
+ * The scales ([..][cap][2] f32, group 0 then group 1) are not permuted.
+ * ---------------------------------------------------------------------------------------- */
+/* ----------------------------------------------------------------------------------------
  * Prefill compression ([HF] CSA paragraph, Figure 3; HCA paragraph, Figure 4).
  * For one sequence of T raw tokens, block s = tokens s*m .. s*m+m-1 becomes entry s:
  *   a_j = gate[s*m+j] + pos_bias[j];  w = softmax(a);  c = sum_j w_j * raw[s*m+j]   (fp32)
  *   kv_out[s]  = E4M3(c[0:448]) || bf16(c[448:512])                                 (RNE)
  * and, when w_idx != NULL (CSA layers), the lightning-indexer key
- *   u = c . W_I  (bf16 operands, fp32 accumulation),  ikey_out[s] = E2M1 codes of u / sigma_g,
+ *   u = c . W_I  (bf16 operands, fp32 accumulation),  ikey_out[s] = E2M1 codes of u / sigma_g
+ *   (stored as "Indexer key storage" describes),
  *   iscale_out[s][g] = sigma_g = smallest power of two with max|u in group g| <= 6 sigma_g.
  * The trailing T mod m tokens form no entry.
  *   raw        [T][512] bf16     gate [T] f32     pos_bias [m] f32     w_idx [512][64] f32
@@ -166,9 +179,8 @@ CSLD_API csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint1
  * s_g = (qscale_g * kscale_g) * 0.25.  The min(k, n_b) entries with the largest (score,
  * -index) are written to topk_out[b] in ascending index order, followed by -1 padding.
  *   ikeys [B][cap][32] u8, iscales [B][cap][2] f32, seq_len [B] i32, q_idx [B][4][64] f32,
- *   head_w [B][4] f32, topk_out [B][k] i32.  cap even, 2 <= cap <= 2^30; ikeys 16-byte
- *   aligned; 1 <= k <= 2048.  Returns CSLD_ERR_UNSUPPORTED if the driver offers no tensor-map
- *   encoder (the keys are streamed by tensor copies).
+ *   head_w [B][4] f32, topk_out [B][k] i32.  ikeys in the stored layout of "Indexer key
+ *   storage".  cap even, 2 <= cap <= 2^30; ikeys and iscales 16-byte aligned; 1 <= k <= 2048.
  * Workspace: csld_indexer_workspace_size(B, cap, k) bytes, 256-byte aligned, zero-filled once
  * before its first use (it holds arrival counters that every call leaves at zero again); calls
  * that share one workspace must not overlap on the GPU.  err: device error word or NULL. */

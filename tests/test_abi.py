@@ -102,3 +102,16 @@ def test_cache_validation(lib):
     c.ikeys = None
     assert f(C.byref(c), 16, 16, None, None) == 1          # indexer arrays missing
     assert f(None, 16, 16, None, None) == 1
+
+
+def test_indexer_key_storage_swap_is_an_involution_on_entries_4_to_7_of_8():
+    """The key cache stores logical byte c of entry s at s*32 + (c ^ 16*((s >> 2) & 1))."""
+    import numpy as np
+    import synth
+    rng = np.random.default_rng(5)
+    a = rng.integers(0, 256, (3, 21, 32), dtype=np.uint8)
+    b = synth.ikeys_swap_halves(a)
+    assert np.array_equal(synth.ikeys_swap_halves(b), a)
+    for s in range(21):
+        for c in range(32):
+            assert np.array_equal(b[:, s, c ^ (16 * ((s >> 2) & 1))], a[:, s, c])

@@ -57,7 +57,7 @@ def _compare(cache, st, with_idx, ramax_fn=None, slack=0.0):
         for b in range(cache.batch):
             gs = cache.iscales[b, :n].cpu().numpy()
             ramax = ramax_fn(b, n) if not np.array_equal(gs, st.iscales[b, :n]) else None
-            H.assert_fp4_keys_close(cache.ikeys[b, :n].cpu().numpy(), gs, st.ikeys[b, :n],
+            H.assert_fp4_keys_close(synth.ikeys_swap_halves(cache.ikeys[b, :n].cpu().numpy()), gs, st.ikeys[b, :n],
                                     st.iscales[b, :n], ramax=ramax)
 
 
@@ -101,8 +101,8 @@ def test_append_equals_prefill_on_gpu(csld):
     assert torch.equal(a.seq_len, b.seq_len)
     _compare_ring_and_tail(a, b.win_kv.cpu().numpy(), b.tail_kv.view(torch.int16).cpu().numpy().view(np.uint16),
                            b.tail_gate.cpu().numpy(), b.seq_len.cpu().numpy())
-    H.assert_fp4_keys_close(a.ikeys[0].cpu().numpy(), a.iscales[0].cpu().numpy(),
-                            b.ikeys[0].cpu().numpy(), b.iscales[0].cpu().numpy(),
+    H.assert_fp4_keys_close(synth.ikeys_swap_halves(a.ikeys[0].cpu().numpy()), a.iscales[0].cpu().numpy(),
+                            synth.ikeys_swap_halves(b.ikeys[0].cpu().numpy()), b.iscales[0].cpu().numpy(),
                             ramax=np.full((a.capacity, 2), 6.0))
 
 

@@ -73,7 +73,8 @@ def test_tiny_decode_workload(csld, orc):
         if np.array_equal(gsel, osel):
             H.assert_attention_close(o_csa.cpu().numpy(), l_csa.cpu().numpy(), ro_csa, rl_csa, f"CSA step {step}")
         # stage checks on identical bytes: the oracle's keys -> GPU indexer; the oracle's cache -> GPU attention
-        sel_o = csld.indexer_topk(torch.from_numpy(ocsa.ikeys).cuda(), torch.from_numpy(ocsa.iscales).cuda(),
+        sel_o = csld.indexer_topk(torch.from_numpy(synth.ikeys_swap_halves(ocsa.ikeys)).cuda(),
+                                  torch.from_numpy(ocsa.iscales).cuda(),
                                   torch.from_numpy(ocsa.seq_len).cuda(), 4, qs["q_idx"].cuda(),
                                   qs["head_w"].cuda(), k)
         H.assert_topk_equal(sel_o.cpu().numpy(), osel)

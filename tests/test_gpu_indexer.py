@@ -19,7 +19,8 @@ def csld():
 
 
 def _run(csld, orc, ikeys, iscales, seq_len, q_idx, head_w, k, ratio=4):
-    dev = [t.cuda() for t in (ikeys, iscales, seq_len, q_idx, head_w)]
+    # the GPU reads the key cache's stored layout; the oracle the logical one
+    dev = [t.cuda() for t in (synth.ikeys_swap_halves(ikeys), iscales, seq_len, q_idx, head_w)]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = csld.indexer_topk(*dev[:3], ratio, dev[3], dev[4], k, err=err)
     torch.cuda.synchronize()
@@ -116,7 +117,8 @@ def test_indexer_workspace_reused_across_calls(csld, orc):
     for it in range(3):
         ik, isc, q, w = _inputs(B, cap, cap, seed=300 + it)
         seq = torch.tensor([4 * cap, 4 * (cap // 2) + 1, 4 * 1000, 4 * cap - 5], dtype=torch.int32)
-        out = csld.indexer_topk(ik.cuda(), isc.cuda(), seq.cuda(), 4, q.cuda(), w.cuda(), k, ws=ws, err=err)
+        out = csld.indexer_topk(synth.ikeys_swap_halves(ik).cuda(), isc.cuda(), seq.cuda(), 4, q.cuda(), w.cuda(), k,
+                                ws=ws, err=err)
         torch.cuda.synchronize()
         assert err.item() == 0
         ref = orc.indexer_topk_batch(ik.numpy(), isc.numpy(), seq.numpy(), 4, q.numpy(), w.numpy(), k)
