@@ -119,7 +119,7 @@ struct CoopSmem {
     uint32_t hist3[1024];
     uint32_t red[3 * kIdxWarps];
     uint32_t sel[4];
-    int32_t fail, last;
+    int32_t fail;
 };
 static_assert(sizeof(((CoopSmem*)0)->codes) >= kCoopMaxRange * 4, "candidate regions fit the idle copy ring");
 
@@ -129,6 +129,14 @@ static_assert(sizeof(((CoopSmem*)0)->codes) >= kCoopMaxRange * 4, "candidate reg
 // Radix select among n candidate keys (read through get): the largest `want` (< n), ties on the
 // threshold left to the caller (who takes the first take_eq equal keys by position).  The bits
 // shared by all candidates are skipped; the rest are resolved 11 bits per pass.
+// Histogram increment with the lanes of a warp that hit the same bin combined into one atomic
+// (the keys being merged crowd into few bins).  Every lane of the warp must call it.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
+    const uint32_t same = __match_any_sync(0xffffffffu, valid ? bin : 0xFFFFFFFFu);
+    const int lane = threadIdx.x & 31;
+    if (valid && lane == __ffs(same) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(same)));
+}
+
 template <typename Get>
 __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint32_t* sel,
                                  uint32_t* red, uint32_t* take_eq) {
@@ -167,9 +175,10 @@ __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint3
         const uint32_t nb = 1u << (top - shift + 1);
         for (uint32_t i = tid; i < nb; i += blockDim.x) hist[i] = 0u;
         __syncthreads();
-        for (int i = tid; i < n; i += blockDim.x) {
-            const uint32_t key = get(i);
-            if (((key ^ prefix) & himask) == 0u) atomicAdd(&hist[(key >> shift) & (nb - 1u)], 1u);
+        for (int i0 = 0; i0 < n; i0 += blockDim.x) {   // uniform trip count: warp-aggregated adds
+            const int i = i0 + tid;
+            const uint32_t key = i < n ? get(i) : 0u;
+            hist_add(hist, (key >> shift) & (nb - 1u), i < n && ((key ^ prefix) & himask) == 0u);
         }
         __syncthreads();
         const uint32_t per = (nb + blockDim.x - 1) / blockDim.x;
@@ -255,13 +264,6 @@ __device__ __forceinline__ void block_sum2(uint32_t a, uint32_t e, uint32_t* red
     __syncthreads();
 }
 
-// Histogram increment with the lanes of a warp that hit the same bin combined into one atomic
-// (the keys being merged crowd into few bins).  Every lane of the warp must call it.
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
-    const uint32_t same = __match_any_sync(0xffffffffu, valid ? bin : 0xFFFFFFFFu);
-    const int lane = threadIdx.x & 31;
-    if (valid && lane == __ffs(same) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(same)));
-}
 
 // Selects the top `want` of sm.keys[0..n) under (key desc, position asc) and emits them in
 // position order: emit(out_pos, position).  Requires sm.hist = histogram of key >> kBinShift.
@@ -791,8 +793,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
 // The cooperative kernel: one exact radix select per sequence across its CTAs.
 // ------------------------------------------------------------------------------------------
 struct CoopWs {
-    uint32_t* hist;    // [B][kCoopSeqWords]: level 1 (2048 bins), level 2 (2048), level 3 (1024)
-    uint32_t* sync;    // [B][64]: word 0 barrier arrivals, word 1 finished CTAs, word 2 list length
+    uint32_t* hist;    // [B][2][kCoopSeqWords]: level 1 (2048 bins), level 2 (2048), level 3 (1024)
+    uint32_t* sync;    // [B][64]: words 0-1 barrier arrivals, 2-3 list length (one per set), 4 epoch
     uint32_t* counts;  // [B][units][2]: keys above the threshold, keys equal to it
     uint32_t* lkeys;   // [B][kListMax]: candidate list (keys of the threshold bin)
     uint8_t* lunit;    // [B][kListMax]: the range each listed key comes from
@@ -913,13 +915,28 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         return;
     }
     const uint32_t want = static_cast<uint32_t>(k);
-    uint32_t* g1 = ws.hist + (size_t)b * kCoopSeqWords;
+    // Two sets of selection state (histograms, barrier counter, list length) per sequence; the
+    // epoch (calls completed on this sequence) picks this call's set.  The other set belonged to
+    // the previous call, which has finished: every CTA clears its share of it here for the next
+    // call, so nothing has to be reset at the end of this one.  The epoch is read before the
+    // first barrier and advanced only after it, by range 0 at its end.
+    uint32_t* sq = ws.sync + (size_t)b * 64;
+    const uint32_t par = __ldcg(sq + 4) & 1u;
+    uint32_t* g1 = ws.hist + ((size_t)b * 2 + par) * kCoopSeqWords;
     uint32_t* g2 = g1 + kBins;
     uint32_t* g3 = g2 + kBins;
-    uint32_t* bar = ws.sync + (size_t)b * 64;
-    uint32_t* done = bar + 1;
+    uint32_t* bar = sq + par;
     uint32_t* cnt = ws.counts + (size_t)b * units * 2;
-    uint32_t* lcount = bar + 2;
+    uint32_t* lcount = sq + 2 + par;
+    {
+        uint32_t* other = ws.hist + ((size_t)b * 2 + (par ^ 1u)) * kCoopSeqWords;
+        const int lo = kCoopSeqWords * u / units, hi = kCoopSeqWords * (u + 1) / units;
+        for (int i = lo + tid; i < hi; i += blockDim.x) other[i] = 0u;
+        if (u == 0 && tid == 0) {
+            sq[par ^ 1u] = 0u;
+            sq[2 + (par ^ 1u)] = 0u;
+        }
+    }
     uint32_t* lkeys = ws.lkeys + (size_t)b * kListMax;
     uint8_t* lunit = ws.lunit + (size_t)b * kListMax;
     const uint32_t nu = static_cast<uint32_t>(units);
@@ -1106,22 +1123,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         pos += __popc(tm);
         eq_seen += __popc(em);
     }
-    // --- the last CTA of the sequence leaves its histograms and counters at zero --------------
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        sm.last = (atomicAdd(done, 1u) == nu - 1u);
-    }
-    __syncthreads();
-    if (sm.last) {
-        for (int i = tid; i < kCoopSeqWords; i += blockDim.x) g1[i] = 0u;
-        if (tid == 0) {
-            *bar = 0u;
-            *done = 0u;
-            *lcount = 0u;
-        }
-        __threadfence();
-    }
+    // --- this call is over for the sequence: the next one takes the other state set ------------
+    if (u == 0 && tid == 0) atomicAdd(sq + 4, 1u);
 }
 
 // Resident CTAs of the cooperative kernel on this device (0 if it cannot run).
@@ -1143,7 +1146,7 @@ static int coop_slots(int num_sms) {
 }
 
 static size_t coop_layout(int B, int units, uint8_t* base, CoopWs* ws) {
-    const size_t h = up256((size_t)B * kCoopSeqWords * 4), s = up256((size_t)B * 64 * 4),
+    const size_t h = up256((size_t)B * 2 * kCoopSeqWords * 4), s = up256((size_t)B * 64 * 4),
                  c = up256((size_t)B * units * 2 * 4), lk = up256((size_t)B * kListMax * 4),
                  lu = up256((size_t)B * kListMax);
     if (ws) {

@@ -182,8 +182,10 @@ CSLD_API csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint1
  *   head_w [B][4] f32, topk_out [B][k] i32.  ikeys in the stored layout of "Indexer key
  *   storage".  cap even, 2 <= cap <= 2^30; ikeys and iscales 16-byte aligned; 1 <= k <= 2048.
  * Workspace: csld_indexer_workspace_size(B, cap, k) bytes, 256-byte aligned, zero-filled once
- * before its first use (it holds arrival counters that every call leaves at zero again); calls
- * that share one workspace must not overlap on the GPU.  err: device error word or NULL. */
+ * before its first use (it holds per-sequence selection state, in two sets that alternate
+ * between calls: each call clears the set the next call will use); calls that share one
+ * workspace must not overlap on the GPU.  After a call that reported CSLD_DEVERR_TIMEOUT,
+ * zero it again.  err: device error word or NULL. */
 CSLD_API size_t csld_indexer_workspace_size(int B, int64_t cap, int k);
 CSLD_API csld_status indexer_topk(const uint8_t* ikeys, const float* iscales, int64_t cap,
                          const int32_t* seq_len, int ratio, const float* q_idx,

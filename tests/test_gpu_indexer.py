@@ -109,14 +109,16 @@ def test_indexer_many_sequences_merge_tree_path(csld, orc, B, cap, k):
 
 
 def test_indexer_workspace_reused_across_calls(csld, orc):
-    """The workspace's counters and histograms are left at zero by every call, so one
-    zero-filled workspace serves any number of calls (here with different inputs)."""
+    """Each call clears the selection state the next call uses, so one zero-filled workspace
+    serves any number of calls (here with different inputs; sequence 2 is short enough to skip
+    the selection on calls 1 and 2, so its state sets alternate out of step with the others)."""
     B, cap, k = 4, 40000, 256
     ws = csld.indexer_workspace(B, cap, k)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for it in range(3):
+    for it in range(5):
         ik, isc, q, w = _inputs(B, cap, cap, seed=300 + it)
-        seq = torch.tensor([4 * cap, 4 * (cap // 2) + 1, 4 * 1000, 4 * cap - 5], dtype=torch.int32)
+        short = 4 * 100 if it in (1, 2) else 4 * 1000
+        seq = torch.tensor([4 * cap, 4 * (cap // 2) + 1, short, 4 * cap - 5], dtype=torch.int32)
         out = csld.indexer_topk(synth.ikeys_swap_halves(ik).cuda(), isc.cuda(), seq.cuda(), 4, q.cuda(), w.cuda(), k,
                                 ws=ws, err=err)
         torch.cuda.synchronize()
