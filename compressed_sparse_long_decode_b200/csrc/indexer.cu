@@ -126,9 +126,6 @@ static_assert(sizeof(((CoopSmem*)0)->codes) >= kCoopMaxRange * 4, "candidate reg
 // ------------------------------------------------------------------------------------------
 // Block-level helpers (512 threads).
 // ------------------------------------------------------------------------------------------
-// Radix select among n candidate keys (read through get): the largest `want` (< n), ties on the
-// threshold left to the caller (who takes the first take_eq equal keys by position).  The bits
-// shared by all candidates are skipped; the rest are resolved 11 bits per pass.
 // Histogram increment with the lanes of a warp that hit the same bin combined into one atomic
 // (the keys being merged crowd into few bins).  Every lane of the warp must call it.
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
@@ -137,6 +134,70 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool vali
     if (valid && lane == __ffs(same) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(same)));
 }
 
+// Exact threshold among n keys that share their top 11 bits (prefix): the want-th largest key,
+// and in *take_eq how many keys equal to it are taken.  Three radix levels of 8, 8 and 5 bits
+// over bits 20..0.  A level is one histogram pass by the whole block (plain shared atomics:
+// warp-level match_any aggregation measured slower on keys this spread) and a scan of the
+// 256 bins by warp 0, which also clears the other histogram buffer for the next level: two CTA
+// barriers a level.
+// hist holds 512 words; hist[0..255] must be zero on entry.  sel: 2 words of shared scratch.
+__device__ uint32_t list_select(const uint32_t* keys, int n, uint32_t want, uint32_t prefix, uint32_t* hist,
+                                uint32_t* sel, uint32_t* take_eq) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t himask = 0xFFFFFFFFu << kBinShift;
+    uint32_t remaining = want;
+#pragma unroll 1
+    for (int lv = 0; lv < 3; ++lv) {
+        const int shift = lv == 0 ? 13 : (lv == 1 ? 5 : 0);
+        const uint32_t dmask = lv == 2 ? 31u : 255u;
+        uint32_t* h = hist + 256 * (lv & 1);
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t key = keys[i];
+            if ((key & himask) == prefix) atomicAdd(&h[(key >> shift) & dmask], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t c[8], tot = 0u;   // lane l: digits 255 - 8l down to 248 - 8l
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                c[q] = h[255 - 8 * lane - q];
+                tot += c[q];
+            }
+            uint32_t incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const uint32_t excl = incl - tot;
+            if (excl < remaining && incl >= remaining) {
+                uint32_t run = excl;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    if (run + c[q] >= remaining) {
+                        sel[0] = static_cast<uint32_t>(255 - 8 * lane - q);
+                        sel[1] = remaining - run;
+                        break;
+                    }
+                    run += c[q];
+                }
+            }
+            uint32_t* o = hist + 256 * ((lv + 1) & 1);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) o[8 * lane + q] = 0u;
+        }
+        __syncthreads();
+        prefix |= sel[0] << shift;
+        remaining = sel[1];
+        himask |= dmask << shift;
+    }
+    *take_eq = remaining;
+    return prefix;
+}
+
+// Radix select among n candidate keys (read through get): the largest `want` (< n), ties on the
+// threshold left to the caller (who takes the first take_eq equal keys by position).  The bits
+// shared by all candidates are skipped; the rest are resolved 11 bits per pass.
 template <typename Get>
 __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint32_t* sel,
                                  uint32_t* red, uint32_t* take_eq) {
@@ -175,10 +236,9 @@ __device__ uint32_t radix_select(Get get, int n, int want, uint32_t* hist, uint3
         const uint32_t nb = 1u << (top - shift + 1);
         for (uint32_t i = tid; i < nb; i += blockDim.x) hist[i] = 0u;
         __syncthreads();
-        for (int i0 = 0; i0 < n; i0 += blockDim.x) {   // uniform trip count: warp-aggregated adds
-            const int i = i0 + tid;
-            const uint32_t key = i < n ? get(i) : 0u;
-            hist_add(hist, (key >> shift) & (nb - 1u), i < n && ((key ^ prefix) & himask) == 0u);
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t key = get(i);
+            if (((key ^ prefix) & himask) == 0u) atomicAdd(&hist[(key >> shift) & (nb - 1u)], 1u);
         }
         __syncthreads();
         const uint32_t per = (nb + blockDim.x - 1) / blockDim.x;
@@ -564,7 +624,7 @@ __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], flo
                     const int li = t * kIdxTile + e;
                     const uint32_t key = score_key(sc);
                     if (li < cn) keys[li] = key;
-                    hist_add(hist, key >> kBinShift, li < cn);
+                    if (li < cn) atomicAdd(&hist[key >> kBinShift], 1u);   // plain: scores spread over bins
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -1022,12 +1082,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             lk[i] = __ldcg(lkeys + i);
             lu[i] = __ldcg(lunit + i);
         }
+        if (tid < 256) sm.hist[tid] = 0u;
         __syncthreads();
         thr = 0u;
         take_eq = static_cast<uint32_t>(P);
         if (static_cast<int>(need1) < P)
-            thr = radix_select([&](int c) { return lk[c]; }, P, static_cast<int>(need1), sm.hist, sm.sel + 2, sm.red,
-                               &take_eq);
+            thr = list_select(lk, P, need1, beta1 << kBinShift, sm.hist, sm.sel + 2, &take_eq);
         // selected before this range: the earlier ranges' keys above bin beta1 (a_loc, loaded
         // above), and their candidates above / equal to the threshold
         for (int i = tid; i < P; i += blockDim.x)
