@@ -855,9 +855,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_topk_kernel(
 struct CoopWs {
     uint32_t* hist;    // [B][2][kCoopSeqWords]: level 1 (2048 bins), level 2 (2048), level 3 (1024)
     uint32_t* sync;    // [B][64]: words 0-1 barrier arrivals, 2-3 list length (one per set), 4 epoch
-    uint32_t* counts;  // [B][units][2]: keys above the threshold, keys equal to it
-    uint32_t* lkeys;   // [B][kListMax]: candidate list (keys of the threshold bin)
-    uint8_t* lunit;    // [B][kListMax]: the range each listed key comes from
+    uint32_t* counts;  // [B][2][units][2]: keys above the threshold, keys equal to it
+    uint64_t* lslot;   // [B][2][kListMax]: candidate list, (range + 1) << 32 | key; 0 = not written
 };
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
@@ -892,6 +891,33 @@ __device__ bool seq_barrier(uint32_t* ctr, uint32_t target, int32_t* fail_flag, 
     }
     __syncthreads();
     return *reinterpret_cast<volatile int32_t*>(fail_flag) == 0;
+}
+
+__device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
+}
+// A word another CTA of the sequence writes once (from zero) during this call: polled until it
+// is non-zero, about a second at most; 0 if it never was.
+__device__ __forceinline__ uint32_t poll_nonzero_u32(const uint32_t* p) {
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        uint32_t v;
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        if (v != 0u) return v;
+        if (i >= 64) __nanosleep(32);
+    }
+    return 0u;
+}
+__device__ __forceinline__ uint64_t poll_nonzero_u64(const uint64_t* p) {
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        uint64_t v;
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+        if (v != 0ull) return v;
+        if (i >= 64) __nanosleep(32);
+    }
+    return 0ull;
 }
 
 // From a global histogram g of nbins bins (2048 or 1024), the bin holding the want-th largest
@@ -975,30 +1001,38 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         return;
     }
     const uint32_t want = static_cast<uint32_t>(k);
-    // Two sets of selection state (histograms, barrier counter, list length) per sequence; the
-    // epoch (calls completed on this sequence) picks this call's set.  The other set belonged to
-    // the previous call, which has finished: every CTA clears its share of it here for the next
-    // call, so nothing has to be reset at the end of this one.  The epoch is read before the
-    // first barrier and advanced only after it, by range 0 at its end.
+    // Two sets of selection state (histograms, barrier counter, list length, candidate list,
+    // per-range counts) per sequence; the epoch (calls completed on this sequence) picks this
+    // call's set.  The other set belonged to the previous call, which has finished: every CTA
+    // clears its share of it here for the next call, so nothing has to be reset at the end of
+    // this one.  The epoch is read before the first barrier and advanced only after it, by
+    // range 0 at its end.
     uint32_t* sq = ws.sync + (size_t)b * 64;
     const uint32_t par = __ldcg(sq + 4) & 1u;
     uint32_t* g1 = ws.hist + ((size_t)b * 2 + par) * kCoopSeqWords;
     uint32_t* g2 = g1 + kBins;
     uint32_t* g3 = g2 + kBins;
     uint32_t* bar = sq + par;
-    uint32_t* cnt = ws.counts + (size_t)b * units * 2;
+    uint32_t* cnt = ws.counts + ((size_t)b * 2 + par) * units * 2;
     uint32_t* lcount = sq + 2 + par;
+    uint64_t* lslot = ws.lslot + ((size_t)b * 2 + par) * kListMax;
     {
         uint32_t* other = ws.hist + ((size_t)b * 2 + (par ^ 1u)) * kCoopSeqWords;
-        const int lo = kCoopSeqWords * u / units, hi = kCoopSeqWords * (u + 1) / units;
+        int lo = kCoopSeqWords * u / units, hi = kCoopSeqWords * (u + 1) / units;
         for (int i = lo + tid; i < hi; i += blockDim.x) other[i] = 0u;
-        if (u == 0 && tid == 0) {
-            sq[par ^ 1u] = 0u;
-            sq[2 + (par ^ 1u)] = 0u;
+        uint64_t* olist = ws.lslot + ((size_t)b * 2 + (par ^ 1u)) * kListMax;
+        lo = kListMax * u / units;
+        hi = kListMax * (u + 1) / units;
+        for (int i = lo + tid; i < hi; i += blockDim.x) olist[i] = 0ull;
+        if (u == 0) {
+            uint32_t* ocnt = ws.counts + ((size_t)b * 2 + (par ^ 1u)) * units * 2;
+            for (int i = tid; i < 2 * units; i += blockDim.x) ocnt[i] = 0u;
+            if (tid == 0) {
+                sq[par ^ 1u] = 0u;
+                sq[2 + (par ^ 1u)] = 0u;
+            }
         }
     }
-    uint32_t* lkeys = ws.lkeys + (size_t)b * kListMax;
-    uint8_t* lunit = ws.lunit + (size_t)b * kListMax;
     const uint32_t nu = static_cast<uint32_t>(units);
 
     bool ok = true;
@@ -1059,31 +1093,53 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         (void)warp_excl_scan(gt, sm.red + 2 * kIdxWarps, &gt_all);
         if (tid == 0) {
             sm.sel[2] = atomicAdd(lcount, nc_all);
-            cnt[2 * u] = gt_all;
+            st_relaxed_u32(cnt + 2 * u, gt_all + 1u);   // + 1: zero means not written yet
         }
         __syncthreads();
         const uint32_t lbase = sm.sel[2] + woff;
         for (int j = lane; j < static_cast<int>(nc); j += 32) {
             const uint32_t at = lbase + static_cast<uint32_t>(j);
-            if (at < static_cast<uint32_t>(kListMax)) {
-                lkeys[at] = cand[j];
-                lunit[at] = static_cast<uint8_t>(u);
-            }
+            if (at < static_cast<uint32_t>(kListMax))
+                st_relaxed_u64(lslot + at, (static_cast<uint64_t>(u + 1) << 32) | cand[j]);
         }
-        if (!seq_barrier(bar, 2 * nu, &sm.fail, err)) return;
-        // every CTA loads the list into the ring's last 32 KB (keys) and hist2 (range ids) and
-        // finds the exact threshold among its keys
+        // No second barrier: the list holds exactly cnt1 entries (the global histogram's count
+        // of bin beta1), so every CTA reads slots 0 .. cnt1 - 1, each as soon as it is written,
+        // into the ring's last 32 KB (keys) and hist2 (range ids), and finds the exact
+        // threshold among them.  Every wait is bounded.
         const int P = static_cast<int>(min(cnt1, static_cast<uint32_t>(kListMax)));
         uint32_t* lk = reinterpret_cast<uint32_t*>(&sm.codes[0][0]) + kCoopMaxRange;
         uint8_t* lu = reinterpret_cast<uint8_t*>(sm.hist2);
         uint32_t a_loc = 0u, e_loc = 0u;
-        for (int v = tid; v < u; v += blockDim.x) a_loc += __ldcg(cnt + 2 * v);   // with the list loads
-        for (int i = tid; i < P; i += blockDim.x) {
-            lk[i] = __ldcg(lkeys + i);
-            lu[i] = __ldcg(lunit + i);
+        bool waited = true;
+        for (int v = tid; v < u && waited; v += blockDim.x) {
+            const uint32_t c = poll_nonzero_u32(cnt + 2 * v);
+            waited = c != 0u;
+            a_loc += c - 1u;
+        }
+        for (int i0 = tid; i0 < P && waited; i0 += 4 * kIdxThreads) {
+            uint64_t w[4];   // four slots in flight; re-read only those not written yet
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = i0 + q * kIdxThreads;
+                w[q] = 1ull;
+                if (i < P) asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w[q]) : "l"(lslot + i) : "memory");
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = i0 + q * kIdxThreads;
+                if (i < P) {
+                    if (w[q] == 0ull) w[q] = poll_nonzero_u64(lslot + i);
+                    waited = waited && w[q] != 0ull;
+                    lk[i] = static_cast<uint32_t>(w[q]);
+                    lu[i] = static_cast<uint8_t>((w[q] >> 32) - 1u);
+                }
+            }
         }
         if (tid < 256) sm.hist[tid] = 0u;
-        __syncthreads();
+        if (__syncthreads_or(!waited)) {
+            if (tid == 0) dev_error(err, CSLD_DEVERR_TIMEOUT);
+            return;
+        }
         thr = 0u;
         take_eq = static_cast<uint32_t>(P);
         if (static_cast<int>(need1) < P)
@@ -1207,16 +1263,14 @@ static int coop_slots(int num_sms) {
 
 static size_t coop_layout(int B, int units, uint8_t* base, CoopWs* ws) {
     const size_t h = up256((size_t)B * 2 * kCoopSeqWords * 4), s = up256((size_t)B * 64 * 4),
-                 c = up256((size_t)B * units * 2 * 4), lk = up256((size_t)B * kListMax * 4),
-                 lu = up256((size_t)B * kListMax);
+                 c = up256((size_t)B * 2 * units * 2 * 4), lk = up256((size_t)B * 2 * kListMax * 8);
     if (ws) {
         ws->hist = reinterpret_cast<uint32_t*>(base);
         ws->sync = reinterpret_cast<uint32_t*>(base + h);
         ws->counts = reinterpret_cast<uint32_t*>(base + h + s);
-        ws->lkeys = reinterpret_cast<uint32_t*>(base + h + s + c);
-        ws->lunit = base + h + s + c + lk;
+        ws->lslot = reinterpret_cast<uint64_t*>(base + h + s + c);
     }
-    return h + s + c + lk + lu;
+    return h + s + c + lk;
 }
 
 IndexerPlan indexer_plan(int B, int64_t cap, int k, int num_sms) {
