@@ -82,6 +82,19 @@ struct TcAttnSmem {
     int32_t fail, n_issued, n_landed;
 };
 
+// Non-blocking test of an mbarrier phase (the MMA issuer polls several barriers in turn; a
+// try_wait could suspend it on one that is not ready while another is).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Offset of byte c of row r in a [rows][128 B] block with the 128-byte swizzle (the 16-byte
 // chunk index XOR the row index within each 8-row, 1024-byte atom).
 __device__ __forceinline__ int sw128(int r, int c) {
@@ -179,7 +192,8 @@ __device__ __forceinline__ void qprep_convert(TcAttnSmem& sm, const uint16_t* q,
 
 __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     const __grid_constant__ CUtensorMap kv_tile, const __grid_constant__ CUtensorMap kv_rows,
-    const __grid_constant__ CUtensorMap win_rows, const uint16_t* __restrict__ q, int64_t cap, int ratio,
+    const __grid_constant__ CUtensorMap win_rows, const __grid_constant__ CUtensorMap win_tile,
+    const uint16_t* __restrict__ q, int64_t cap, int ratio,
     const int32_t* __restrict__ topk, int k, int W, const int32_t* __restrict__ seq_len, float scale, int splits,
     float* __restrict__ opart, float2* __restrict__ mlpart, int32_t* err) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -212,6 +226,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         tma_prefetch_map(&kv_tile);
         tma_prefetch_map(&kv_rows);
         tma_prefetch_map(&win_rows);
+        tma_prefetch_map(&win_tile);
     }
     tc_fence_before();
     __syncthreads();   // barriers initialised, tensor memory allocated
@@ -278,6 +293,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                 if (tid < kBlk)
                     tma_load_2d(tl + tid * kBlkBytes, &kv_tile, tid < 4 ? 128 * tid : kNope,
                                 static_cast<int>((int64_t)b * cap + i0), &sm.full[s]);
+            } else if (W == kTcTile && n_win == W && i0 == n_comp4) {
+                // the tile is the whole window and the ring is full: its W slots hold exactly
+                // those tokens (in ring order, which the softmax does not care about), so the
+                // ring itself comes in one box per column block
+                if (tid < kBlk)
+                    tma_load_2d(tl + tid * kBlkBytes, &win_tile, tid < 4 ? 128 * tid : kNope, b * W, &sm.full[s]);
             } else {
                 // thread t: slots 4g .. 4g+3 (g = t / 4) of column block t % 4 (and block 4 when
                 // t % 4 == 0), from one of the two maps
@@ -317,11 +338,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
             const uint64_t dq = desc_sw128(sm.qk[0], 0), dqr = desc_sw128(sm.qr, 0);
             // Issue whatever is ready, PV first (it frees a tile buffer for the next copy):
             // PV(np) once P(np) is published; QK(nq) once tile nq landed and its S slot is free.
+            // The polls do not block (test_wait), so a barrier that is not ready never holds up
+            // another that is.
             int nq = 0, np = 0, landed = 0;
             uint32_t idle = 0;
             while (np < n_tiles) {
                 if (*fail) break;
-                if (np < nq && mbar_try_wait(&sm.pfull[np & 1], (np >> 1) & 1)) {
+                if (np < nq && mbar_test_wait(&sm.pfull[np & 1], (np >> 1) & 1)) {
                     const int su = np & 1;
                     tc_fence_after();
                     const uint64_t da = desc_sw128(sm.tile[su], 0);
@@ -347,8 +370,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                     idle = 0;
                     continue;
                 }
-                if (nq < n_tiles && nq < np + 2 && mbar_try_wait(&sm.full[nq & 1], (nq >> 1) & 1) &&
-                    (nq < 2 || mbar_try_wait(&sm.sfree[nq & 1], ((nq >> 1) - 1) & 1))) {
+                if (nq < n_tiles && nq < np + 2 && mbar_test_wait(&sm.full[nq & 1], (nq >> 1) & 1) &&
+                    (nq < 2 || mbar_test_wait(&sm.sfree[nq & 1], ((nq >> 1) - 1) & 1))) {
                     const int s = nq & 1;
                     landed = nq + 1;
                     tc_fence_after();
@@ -373,7 +396,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                     *fail = 1;
                     break;
                 }
-                if (idle > 64) __nanosleep(64);
+                if (idle > 64) __nanosleep(32);
             }
             sm.n_landed = landed;
         }
@@ -572,7 +595,7 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
                                         float2* mlpart, int32_t* err, cudaStream_t stream) {
     // the caches as 2-D byte tensors [rows][576]: 128-byte boxes with the 128-byte swizzle, 128
     // rows tall (box copies of contiguous tiles) or one row (the gather4 form)
-    CUtensorMap kv_tile, kv_rows, win_rows;
+    CUtensorMap kv_tile, kv_rows, win_rows, win_tile;
     const uint64_t rows = (uint64_t)B * (uint64_t)cap;
     if (!make_tensor_map_2d_u8(&kv_tile, comp_kv, kEntry, rows, 128, kTcTile) ||
         !make_tensor_map_2d_u8(&kv_rows, comp_kv, kEntry, rows, 128, 1))
@@ -581,11 +604,16 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
     const bool has_win = W > 0 && win_kv != nullptr;
     if (!make_tensor_map_2d_u8(&win_rows, has_win ? win_kv : comp_kv, kEntry, has_win ? (uint64_t)B * W : rows, 128, 1))
         return cudaErrorInvalidValue;
+    // a full ring of kTcTile slots as one tile (only used when W == kTcTile)
+    const bool win_box = has_win && W == kTcTile;
+    if (!make_tensor_map_2d_u8(&win_tile, win_box ? win_kv : comp_kv, kEntry, win_box ? (uint64_t)B * W : rows, 128,
+                               win_box ? kTcTile : 1))
+        return cudaErrorInvalidValue;
     const size_t smem = attention_tc_smem_bytes();
     cudaError_t e = set_smem_once(attention_tc_partial_kernel, smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(attention_tc_partial_kernel, dim3(splits, B), dim3(kTcThreads), smem, stream, kv_tile, kv_rows,
-                   win_rows, q, cap, ratio, topk, k, W, seq_len, scale, splits, opart, mlpart, err);
+                   win_rows, win_tile, q, cap, ratio, topk, k, W, seq_len, scale, splits, opart, mlpart, err);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
