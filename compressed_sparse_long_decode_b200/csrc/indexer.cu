@@ -15,22 +15,25 @@
 // dot.  The fp32 score then follows a fixed operation order (see the ABI header) using the
 // true scales, so the selection is reproducible bit for bit; order key = (score, -index).
 //
-// Scoring (score_chunk, shared by both kernels below) is warp-specialised over 16 warps:
-// warp 12 streams 256-entry tiles of key codes with TMA tensor copies (32-byte swizzle, the
-// MMA's canonical K-major layout) and their scales with bulk copies into an mbarrier ring;
-// warp 13 owns 128 columns of tensor memory and issues two MMAs per tile into one of the
+// Scoring (score_setup + score_run, shared by both kernels below) is warp-specialised over 16
+// warps: warp 12 streams 256-entry tiles of key codes into an mbarrier ring with 1-D bulk
+// copies -- the cache stores the codes pre-swizzled (32-byte swizzle, the MMA's canonical
+// K-major layout), so they land ready to use -- together with their scales, several tiles per
+// copy; warp 13 owns the tensor memory and issues two MMAs per tile into one of the
 // accumulator slots; warpgroups 0..2 take turns reading a slot back (tcgen05.ld, one thread
 // per TMEM lane = two entries), forming the 32-bit order keys in shared memory and a histogram
 // of their top 11 bits.
 //
 // Selection, when the whole grid can be resident (indexer_topk_coop_kernel, cooperative
 // launch): each sequence is split into `units` ranges, one CTA each, and the CTAs of a sequence
-// run an exact radix select together.  They add their histograms into the sequence's global
+// run an exact select together.  They add their histograms into the sequence's global
 // histogram, meet at a barrier (an arrival counter; every wait is bounded), and each derive the
-// same threshold bin; two more rounds over the next 11 and 10 key bits give the exact
-// threshold key and how many keys equal to it are taken (the lowest indices win).  After a
-// last barrier every CTA knows how many selected entries precede its range and writes its own
-// in ascending index order.
+// same threshold bin.  When that bin holds at most kListMax keys, every CTA appends its keys in
+// the bin to a list of self-announcing slots, then reads the whole list as it fills and finds
+// the exact threshold key with three radix levels; otherwise two more histogram rounds over
+// the next 11 and 10 key bits (and barriers) give it.  Either way every CTA learns how many
+// selected entries precede its range (ties go to the lowest indices) and writes its own in
+// ascending index order.
 //
 // Otherwise (indexer_topk_kernel): each CTA selects its chunk's top min(k, chunk) -- threshold
 // bin from the histogram, the bin's candidates collected, a radix select among them, an emit in
@@ -441,8 +444,8 @@ __device__ void select_emit(IdxSmem& sm, int n, int want, Emit emit) {
 // keys into keys[0..cn) and their top-11-bit histogram added into hist (zeroed by the caller).
 // Returns false (and records CSLD_DEVERR_TIMEOUT) if a copy or an MMA did not complete in
 // time.  Called by all 512 threads; allocates and frees NCOLS columns of tensor memory.
-// Scoring setup, which reads nothing produced upstream: the ring's barriers, the tensor memory
-// (NCOLS columns) and the tensor-map prefetch.  Block-wide; ends with a CTA barrier.
+// Scoring setup, which reads nothing produced upstream: the ring's barriers and the tensor
+// memory (NCOLS columns).  Block-wide; ends with a CTA barrier.
 template <int S, uint32_t NCOLS>
 __device__ void score_setup(ScoreCtl& ctl) {
     const int tid = threadIdx.x, warp = tid >> 5;
