@@ -178,7 +178,7 @@ csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t*
                                     int ratio, const int32_t* topk, int k, const uint8_t* win_kv, int W,
                                     const int32_t* seq_len, int B, float scale, float* out, float* lse_out,
                                     void* ws, size_t ws_bytes, int32_t* err, void* stream) {
-    if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; this build implements %d", heads, CSLD_HEADS);
+    if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; the library implements %d", heads, CSLD_HEADS);
     if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
     if (cap < 1 || cap > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^31-1", (long long)cap);
     if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
@@ -204,7 +204,7 @@ csld_status hybrid_decode_attention_static(const uint16_t* q, int heads, const u
                                            const uint8_t* win_kv, int W, const int32_t* seq_len, int B,
                                            float scale, float* out, float* lse_out, int32_t* err,
                                            void* stream) {
-    if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; this build implements %d", heads, CSLD_HEADS);
+    if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; the library implements %d", heads, CSLD_HEADS);
     if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
     if (cap < 1 || cap > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^31-1", (long long)cap);
     if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);

@@ -69,7 +69,7 @@ typedef enum csld_status {
     CSLD_ERR_ALIGN = 3,        /* a pointer or stride is not 16-byte aligned */
     CSLD_ERR_CAPACITY = 4,     /* a size exceeds a stated maximum or the cache capacity */
     CSLD_ERR_CUDA = 5,         /* a CUDA runtime error (launch failure, no device, ...) */
-    CSLD_ERR_UNSUPPORTED = 6,  /* a shape this build does not implement (e.g. heads != 16) */
+    CSLD_ERR_UNSUPPORTED = 6,  /* a shape the library does not implement (e.g. heads != 16) */
     CSLD_ERR_WORKSPACE = 7     /* workspace pointer NULL or smaller than required */
 } csld_status;
 

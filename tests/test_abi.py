@@ -57,7 +57,7 @@ def test_host_validation_without_launch(lib):
     f = lib.hybrid_decode_attention
     f.restype = I
     f.argtypes = [P, I, P, I64, I, P, I, P, I, P, I, F, P, P, P, S, P, P]
-    # 8 heads: not implemented by this build -> CSLD_ERR_UNSUPPORTED, nothing launched
+    # 8 heads: not implemented by the library -> CSLD_ERR_UNSUPPORTED, nothing launched
     assert f(1, 8, 16, 64, 4, None, 0, 16, 4, 16, 1, 0.05, 16, None, 16, 1 << 20, None, None) == 6
     assert b"heads" in lib.csld_last_error()
     # NULL q -> CSLD_ERR_ARG
