@@ -990,8 +990,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     int64_t n_b = seq_len[b];
     n_b = n_b < 0 ? 0 : n_b / ratio;
     if (n_b > cap) n_b = cap;
-    const int64_t c0 = (int64_t)u * chunk;
-    const int cn = static_cast<int>(max64(0, min64(chunk, n_b - c0)));
+    // this CTA's range: an even share of the sequence's visible tiles (the plan's chunk, sized
+    // from cap, bounds it), so the last range is not left short
+    const int64_t tiles_b = (n_b + kIdxTile - 1) / kIdxTile;
+    const int64_t c0 = tiles_b * u / units * kIdxTile;
+    const int cn = static_cast<int>(max64(0, min64(min64(tiles_b * (u + 1) / units * kIdxTile, n_b) - c0, chunk)));
     int32_t* out = topk_out + (size_t)b * k;
 
     if (n_b <= k) {
