@@ -68,8 +68,9 @@ def _load():
     L.csld_attention_workspace_size.restype = S
     L.csld_attention_workspace_size.argtypes = [I, I, I64, I, I]
     L.hybrid_decode_attention.argtypes = [P, I, P, I64, I, P, I, P, I, P, I, F, P, P, P, S, P, P]
+    L.csld_stage.argtypes = [P, P, S, P]
     for fn in ("csld_compress", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
-               "indexer_topk", "hybrid_decode_attention"):
+               "indexer_topk", "hybrid_decode_attention", "csld_stage"):
         getattr(L, fn).restype = I
     return L
 
@@ -91,12 +92,17 @@ def _stream():
     return torch.cuda.current_stream().cuda_stream
 
 
-def _need(t, dtype, name):
+def _need(t, dtype, name, host_ok=False):
+    """t must be a contiguous tensor of dtype on the GPU, or (host_ok) in pinned host memory,
+    which the kernels reach through unified addressing."""
     if t is None:
         raise CsldError(f"{name} is required")
-    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
-        raise CsldError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {t.dtype} "
-                        f"{'cuda' if t.is_cuda else 'cpu'} contiguous={t.is_contiguous()}")
+    where_ok = t.is_cuda or (host_ok and t.is_pinned())
+    if t.dtype != dtype or not where_ok or not t.is_contiguous():
+        want = "CUDA or pinned host" if host_ok else "CUDA"
+        raise CsldError(f"{name}: expected a contiguous {want} {dtype} tensor, got {t.dtype} "
+                        f"{'cuda' if t.is_cuda else ('pinned cpu' if t.is_pinned() else 'cpu')} "
+                        f"contiguous={t.is_contiguous()}")
     return t
 
 
@@ -230,8 +236,14 @@ def hybrid_decode_attention(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, 
         _need(win_kv, torch.uint8, "win_kv")
     if out is None:
         out = torch.empty((B, H, DIM), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, "out", host_ok=True)   # a pinned host buffer receives the result directly
+    if out.shape != (B, H, DIM):
+        raise CsldError(f"out: expected shape {(B, H, DIM)}, got {tuple(out.shape)}")
     if lse is None:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    _need(lse, torch.float32, "lse", host_ok=True)
+    if lse.shape != (B, H):
+        raise CsldError(f"lse: expected shape {(B, H)}, got {tuple(lse.shape)}")
     if ws is None:
         ws = attention_workspace(B, cap, max(k, 1), W, q.device)
     _check(lib.hybrid_decode_attention(_ptr(q), H, _ptr(comp_kv), cap, ratio, _ptr(topk), k,
@@ -239,3 +251,17 @@ def hybrid_decode_attention(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, 
                                        float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                        _ptr(err), _stream()), "hybrid_decode_attention")
     return out, lse
+
+
+# ---- staging copies -----------------------------------------------------------------------
+def stage(dst, src):
+    """dst <- src (same byte size, both contiguous; each a CUDA tensor or pinned host memory)
+    by a kernel on the current stream: csld_stage.  Returns dst."""
+    for t, name in ((dst, "dst"), (src, "src")):
+        if t is None or not t.is_contiguous() or not (t.is_cuda or t.is_pinned()):
+            raise CsldError(f"{name}: expected a contiguous CUDA or pinned host tensor")
+    nb = dst.numel() * dst.element_size()
+    if src.numel() * src.element_size() != nb:
+        raise CsldError("dst and src differ in size")
+    _check(lib.csld_stage(_ptr(dst), _ptr(src), nb, _stream()), "csld_stage")
+    return dst

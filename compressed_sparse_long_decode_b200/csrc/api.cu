@@ -7,6 +7,11 @@
 #include "csld_internal.cuh"
 #include "kernels.cuh"
 
+namespace csld {
+// stage.cu
+cudaError_t launch_stage(void* dst, const void* src, size_t bytes, int num_sms, cudaStream_t stream);
+}  // namespace csld
+
 namespace {
 
 thread_local char g_msg[512] = "";
@@ -196,6 +201,16 @@ csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t*
     cudaError_t e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, seq_len, B,
                                            scale, out, lse_out, ws, plan, err, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention");
+    return CSLD_OK;
+}
+
+csld_status csld_stage(void* dst, const void* src, size_t bytes, void* stream) {
+    if (bytes == 0) return CSLD_OK;
+    if (!dst || !src) return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (!aligned16(dst) || !aligned16(src) || (bytes & 15u))
+        return fail(CSLD_ERR_ALIGN, "dst and src must be 16-byte aligned and bytes a multiple of 16");
+    cudaError_t e = csld::launch_stage(dst, src, bytes, num_sms(), as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "csld_stage");
     return CSLD_OK;
 }
 

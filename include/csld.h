@@ -205,6 +205,8 @@ CSLD_API csld_status indexer_topk(const uint8_t* ikeys, const float* iscales, in
  * units.  An empty key set gives out = 0 and lse = -inf.
  *   q [B][heads][512] bf16 (heads == 16), comp_kv [B][cap][576], topk [B][k] i32 or NULL,
  *   win_kv [B][W][576], seq_len [B] i32, out [B][heads][512] f32, lse_out [B][heads] f32 or NULL.
+ * out and lse_out are written with plain stores, so they may also be pinned host memory mapped
+ * into the device's address space (the result then lands on the host without a separate copy).
  * comp_kv, win_kv must be 16-byte aligned.  Workspace: csld_attention_workspace_size(...).
  * -------------------------------------------------------------------------------------- */
 CSLD_API size_t csld_attention_workspace_size(int B, int heads, int64_t cap, int k, int W);
@@ -243,6 +245,18 @@ CSLD_API csld_status hybrid_decode_attention_static(const uint16_t* q, int heads
                                                     const int32_t* seq_len, int B, float scale,
                                                     float* out, float* lse_out, int32_t* err,
                                                     void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * csld_stage -- copies `bytes` from src to dst with a kernel on `stream`.  The pages have no
+ * counterpart to this entry point: it serves callers that bring a decode step's inputs from
+ * the host.  dst and src may each be device memory or pinned host memory mapped into the
+ * device's address space (with unified addressing, any cudaHostAlloc / cudaMallocHost
+ * allocation).  As a kernel it chains directly to the decode kernel after it and may start
+ * while the kernel before it finishes (dst is written only after that kernel has completed),
+ * where a copy-engine transfer between two kernels costs a round trip through the copy engine.
+ * dst and src 16-byte aligned, bytes a multiple of 16; the two ranges must not overlap.
+ * ---------------------------------------------------------------------------------------- */
+CSLD_API csld_status csld_stage(void* dst, const void* src, size_t bytes, void* stream);
 
 #ifdef __cplusplus
 }
