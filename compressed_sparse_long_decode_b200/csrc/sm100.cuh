@@ -6,10 +6,11 @@
 //    sub-partition: lanes 32*(warp % 4) .. 32*(warp % 4) + 31.
 //  * tcgen05.mma / tcgen05.commit are issued by one thread; tcgen05.alloc / dealloc / ld / st
 //    are warp-collective (.sync.aligned).
-//  * Shared-memory operands use the K-major, 32-byte-swizzle canonical layout: rows of 32
-//    bytes, 8-row groups of 256 bytes, and inside every group the two 16-byte halves of rows
-//    4..7 exchanged (byte-address bit 4 XOR bit 7).  TMA writes that layout when its tensor
-//    map asks for CU_TENSOR_MAP_SWIZZLE_32B; hand-written operands apply the same XOR.
+//  * The indexer's shared-memory operands use the K-major, 32-byte-swizzle canonical layout:
+//    rows of 32 bytes, 8-row groups of 256 bytes, and inside every group the two 16-byte
+//    halves of rows 4..7 exchanged (byte-address bit 4 XOR bit 7).  The key cache is stored
+//    that way, so bulk copies reproduce it; hand-written operands apply the same XOR.  The
+//    attention's operands use the 128-byte swizzle that its tensor maps write.
 #pragma once
 #include <cuda.h>
 #include <stdint.h>
