@@ -1146,7 +1146,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             if (tid == 0) dev_error(err, CSLD_DEVERR_TIMEOUT);
             return;
         }
-        thr = 0u;
+        // when the whole of bin beta1 is wanted, its lowest key is the threshold (every key
+        // equal to it taken): keys of lower bins, which the emit pass also visits, stay below it
+        thr = beta1 << kBinShift;
         take_eq = static_cast<uint32_t>(P);
         if (static_cast<int>(need1) < P)
             thr = list_select(lk, P, need1, beta1 << kBinShift, sm.hist, sm.sel + 2, &take_eq);

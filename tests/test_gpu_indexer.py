@@ -142,3 +142,26 @@ def test_indexer_large_ties_take_the_slow_selection(csld, orc):
     H.assert_topk_equal(got, ref)
     assert np.array_equal(got[1], np.arange(k))
     assert np.array_equal(got[0], np.concatenate([np.arange(k - 300), np.arange(20000, 20300)]))
+
+
+def test_indexer_threshold_bin_taken_whole(csld, orc):
+    """The k-th largest key is the lowest key of its histogram bin, so the whole bin is taken
+    and no key below it may be: on sequence 0 exactly k planted keys share the top bin, on
+    sequence 1 the k planted keys have scales 2, 2, 4, 4, 8, ... (two per binade), and the
+    other keys of the steps they sit in score lower; sequence 2 is random."""
+    B, cap, k = 3, 6000, 100
+    ik = torch.full((B, cap, 32), 0x22, dtype=torch.uint8)     # every code +1.0
+    isc = torch.ones((B, cap, 2), dtype=torch.float32)
+    ik[0, 4000:4000 + k, :] = 0x44                              # k keys with code +2.0
+    planted = np.sort(np.random.default_rng(17).choice(cap, size=k, replace=False))
+    for j, i in enumerate(planted):
+        isc[1, int(i), :] = 2.0 ** (1 + j // 2)
+    rk, rs, _, _ = _inputs(1, cap, cap, seed=23)
+    ik[2], isc[2] = rk[0], rs[0]
+    q = torch.ones((B, 4, 64))
+    w = torch.ones((B, 4))
+    seq = torch.full((B,), 4 * cap, dtype=torch.int32)
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, k)
+    H.assert_topk_equal(got, ref)
+    assert np.array_equal(got[0], np.arange(4000, 4000 + k))
+    assert np.array_equal(got[1], planted)
