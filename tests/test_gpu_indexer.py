@@ -165,3 +165,23 @@ def test_indexer_threshold_bin_taken_whole(csld, orc):
     H.assert_topk_equal(got, ref)
     assert np.array_equal(got[0], np.arange(4000, 4000 + k))
     assert np.array_equal(got[1], planted)
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_indexer_one_long_sequence(csld, orc, ties):
+    """One sequence of 262,144 entries split over 147 ranges (one CTA each): with random keys
+    (1 % heavy) the threshold bin goes through the candidate list; with identical keys (300
+    planted larger) it holds more than 8,192 keys and takes two more histogram levels."""
+    B, n_c, k = 1, 262144, 1024
+    if ties:
+        ik = torch.full((B, n_c, 32), 0x22, dtype=torch.uint8)
+        ik[0, 100000:100300, :] = 0x44
+        isc = torch.ones((B, n_c, 2), dtype=torch.float32)
+        q, w = torch.ones((B, 4, 64)), torch.ones((B, 4))
+    else:
+        ik, isc, q, w = _inputs(B, n_c, n_c, seed=41, heavy=0.01)
+    seq = torch.full((B,), 4 * n_c, dtype=torch.int32)
+    got, ref = _run(csld, orc, ik, isc, seq, q, w, k)
+    H.assert_topk_equal(got, ref)
+    if ties:
+        assert np.array_equal(got[0], np.concatenate([np.arange(k - 300), np.arange(100000, 100300)]))
