@@ -3,6 +3,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
 
 #include "csld_internal.cuh"
 #include "kernels.cuh"
@@ -10,6 +13,19 @@
 namespace csld {
 // stage.cu
 cudaError_t launch_stage(void* dst, const void* src, size_t bytes, int num_sms, cudaStream_t stream);
+
+cudaError_t set_smem_attr_once(const void* kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<const void*, int>> done;   // (kernel, device) pairs already set
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kernel, dev})) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e == cudaSuccess) done.insert({kernel, dev});
+    return e;
+}
 }  // namespace csld
 
 namespace {

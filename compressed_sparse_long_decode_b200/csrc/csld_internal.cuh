@@ -214,16 +214,14 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 
-// Opt a kernel into its dynamic shared-memory size once per process (a function attribute,
-// not a stream operation, so later calls may be captured into CUDA graphs).
+// Opt a kernel into its dynamic shared-memory size, once per (kernel, device): a function
+// attribute, not a stream operation, so later calls may be captured into CUDA graphs.  The
+// record is keyed by the kernel's address and the current device, so every GPU a process drives
+// gets the attribute set before its first launch there.
+cudaError_t set_smem_attr_once(const void* kernel, size_t bytes);
 template <typename K>
 inline cudaError_t set_smem_once(K kernel, size_t bytes) {
-    static int done = 0;
-    if (done) return cudaSuccess;
-    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(bytes));
-    if (e == cudaSuccess) done = 1;
-    return e;
+    return set_smem_attr_once(reinterpret_cast<const void*>(kernel), bytes);
 }
 
 __device__ __forceinline__ void dev_error(int32_t* err, uint32_t flag) {

@@ -1251,22 +1251,32 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     if (u == 0 && tid == 0) atomicAdd(sq + 4, 1u);
 }
 
-// Resident CTAs of the cooperative kernel on this device (0 if it cannot run).
+// Resident CTAs of the cooperative kernel on the current device (0 if it cannot run), found
+// once per device.
 static int coop_slots(int num_sms) {
-    static int per_sm = -1;
-    static std::once_flag once;
-    std::call_once(once, [] {
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static int per_sm[kMaxDev];
+    static bool known[kMaxDev] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!known[dev]) {
         const size_t smem = sizeof(CoopSmem) + kIdxSmemAlign;
         int n = 0;
         if (set_smem_once(indexer_topk_coop_kernel, smem) == cudaSuccess &&
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, indexer_topk_coop_kernel, kIdxThreads, smem) ==
                 cudaSuccess)
-            per_sm = n;
+            per_sm[dev] = n;
         else
-            per_sm = 0;
+            per_sm[dev] = 0;
         (void)cudaGetLastError();
-    });
-    return per_sm * num_sms;
+        known[dev] = true;
+    }
+    return per_sm[dev] * num_sms;
 }
 
 static size_t coop_layout(int B, int units, uint8_t* base, CoopWs* ws) {

@@ -228,7 +228,9 @@ CSLD_API csld_status hybrid_decode_attention(const uint16_t* q, int heads, const
  * inside the library.  Every GPU that loads libcsld.so keeps that array until the process
  * exits.  It allocates nothing:
  *  - The first call on a device (with that device current) looks up the array's device
- *    address once. Make that first call before any stream capture.
+ *    address once and keeps it for the life of the process. Make that first call before any
+ *    stream capture.  A cudaDeviceReset on that device invalidates the kept address: do not
+ *    call this entry point on a device after resetting it.
  *  - A call that would need more scratch than the array holds returns CSLD_ERR_CAPACITY and
  *    launches nothing (the need is about B * min(#SMs/B, tiles) * 16 * 2056 bytes; batches up
  *    to ~250 sequences fit).

@@ -46,6 +46,7 @@ def test_tiny_decode_workload(csld, orc):
         orc.append_batch(ocsa, inp["bias4"].numpy(), inp["w_idx"].numpy(), bits[:, t].copy(), gates[:, t].copy())
         orc.append_batch(ohca, inp["bias128"].numpy(), None, bits[:, t].copy(), gates[:, t].copy())
     overlap = []
+    csa_compared = 0
     for step in range(steps):
         t = T0 + step
         qs = synth.decode_queries(1, seed=100 + step)
@@ -72,12 +73,21 @@ def test_tiny_decode_workload(csld, orc):
         overlap.append(len(set(gsel[0]) & set(osel[0])) / k)
         if np.array_equal(gsel, osel):
             H.assert_attention_close(o_csa.cpu().numpy(), l_csa.cpu().numpy(), ro_csa, rl_csa, f"CSA step {step}")
+            csa_compared += 1
+        # the stated top-k rule on each side's own keys: the float64 selection up to near-ties
+        H.assert_topk_matches_f64(orc, gsel, synth.ikeys_swap_halves(csa.ikeys.cpu().numpy()),
+                                  csa.iscales.cpu().numpy(), csa.seq_len.cpu().numpy(), 4, qs["q_idx"].numpy(),
+                                  qs["head_w"].numpy(), k)
+        H.assert_topk_matches_f64(orc, osel, ocsa.ikeys, ocsa.iscales, ocsa.seq_len, 4, qs["q_idx"].numpy(),
+                                  qs["head_w"].numpy(), k)
         # stage checks on identical bytes: the oracle's keys -> GPU indexer; the oracle's cache -> GPU attention
         sel_o = csld.indexer_topk(torch.from_numpy(synth.ikeys_swap_halves(ocsa.ikeys)).cuda(),
                                   torch.from_numpy(ocsa.iscales).cuda(),
                                   torch.from_numpy(ocsa.seq_len).cuda(), 4, qs["q_idx"].cuda(),
                                   qs["head_w"].cuda(), k)
         H.assert_topk_equal(sel_o.cpu().numpy(), osel)
+        H.assert_topk_matches_f64(orc, sel_o.cpu().numpy(), ocsa.ikeys, ocsa.iscales, ocsa.seq_len, 4,
+                                  qs["q_idx"].numpy(), qs["head_w"].numpy(), k)
         o2, l2 = csld.hybrid_decode_attention(qs["q"].cuda(), torch.from_numpy(ocsa.comp_kv).cuda(), 4,
                                               torch.from_numpy(osel).cuda(), torch.from_numpy(ocsa.win_kv).cuda(),
                                               W, torch.from_numpy(ocsa.seq_len).cuda(), SCALE)
@@ -90,3 +100,6 @@ def test_tiny_decode_workload(csld, orc):
                             H.pool_slack(raw, 128))
     # GPU and oracle keys differ by at most one FP4 step; their selections nearly coincide
     assert min(overlap) >= 0.95, overlap
+    # the CSA output on each side's own state was compared on at least one step
+    print(f"CSA outputs compared on {csa_compared} of {steps} steps")
+    assert csa_compared >= 1, f"CSA outputs compared on none of the {steps} steps"
