@@ -18,7 +18,8 @@ import torch
 __all__ = [
     "csa_compress", "hca_compress", "compress", "indexer_topk", "hybrid_decode_attention",
     "kv_cache_append", "kv_cache_prefill", "LayerCache", "CsldError", "lib", "ENTRY_BYTES",
-    "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace",
+    "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace", "DecodeStack",
+    "layer_pattern", "stage",
 ]
 
 DIM = 512
@@ -265,3 +266,62 @@ def stage(dst, src):
         raise CsldError("dst and src differ in size")
     _check(lib.csld_stage(_ptr(dst), _ptr(src), nb, _stream()), "csld_stage")
     return dst
+
+
+# ---- a stack of layers --------------------------------------------------------------------
+def layer_pattern(n_layers=61):
+    """Layer kinds of the hybrid stack: layers 0 and 1 HCA, then CSA and HCA alternating from
+    layer 2 (CSA) on -- for 61 layers, 30 CSA and 31 HCA ("DeepSeek-V4: a million-token context
+    that agents can actually use", layer-pattern paragraph)."""
+    return ["hca" if i < 2 or (i - 2) % 2 else "csa" for i in range(n_layers)]
+
+
+class DecodeStack:
+    """The attention layers of a hybrid stack for B sequences, each with its own cache (a
+    LayerCache per layer), and one decode step through all of them: per layer kv_cache_append,
+    then on CSA layers indexer_topk followed by sparse hybrid_decode_attention, on HCA layers
+    dense hybrid_decode_attention.  The layers run in order on the current stream; every
+    call is one of the C-ABI entry points above (this class only holds tensors).
+
+    kinds: list of "csa" / "hca"; csa_cap / hca_cap: compressed-entry capacity per sequence;
+    pos_bias4 [4], pos_bias128 [128], w_idx [512,64]: the pooling biases and the indexer
+    projection (shared by the layers of a kind here; per-layer weights only change bytes)."""
+
+    def __init__(self, batch, kinds, csa_cap, hca_cap, window, topk, pos_bias4, pos_bias128, w_idx,
+                 device="cuda"):
+        self.batch, self.kinds, self.window, self.topk = batch, list(kinds), window, topk
+        dev = torch.device(device)
+        self.layers = [LayerCache(batch, csa_cap, 4, window, pos_bias4, w_idx, device=dev) if k == "csa"
+                       else LayerCache(batch, hca_cap, 128, window, pos_bias128, device=dev) for k in self.kinds]
+        csa = [c for c in self.layers if c.ratio == 4]
+        caps = [c.capacity for c in self.layers]
+        self.ws_idx = indexer_workspace(batch, csa[0].capacity, topk, dev) if csa else None
+        self.ws_att = attention_workspace(batch, max(caps), topk, window, dev)
+        self.sel = torch.empty((batch, topk), dtype=torch.int32, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def kv_bytes_per_sequence(self, context):
+        """Bytes one sequence's cache holds at `context` raw tokens: compressed entries (576 B),
+        indexer keys (32 B codes + 8 B scales) on CSA layers, the window ring and the tail."""
+        total = 0
+        for c in self.layers:
+            n = context // c.ratio
+            total += n * ENTRY_BYTES + (n * (IKEY_BYTES + 8) if c.has_indexer else 0)
+            total += min(self.window, context) * ENTRY_BYTES + (context % c.ratio) * (2 * DIM + 4)
+        return total
+
+    def step(self, kv_new, gate_new, q, q_idx, head_w, scale, out, lse=None):
+        """One decode token per sequence through every layer.  kv_new [L,B,512] bf16, gate_new
+        [L,B] f32, q [L,B,16,512] bf16, q_idx [L,B,4,64] f32, head_w [L,B,4] f32; out
+        [L,B,16,512] f32, lse [L,B,16] f32 or None (device tensors)."""
+        for i, c in enumerate(self.layers):
+            kv_cache_append(c, kv_new[i], gate_new[i], self.err)
+            l_i = None if lse is None else lse[i]
+            if c.has_indexer:
+                indexer_topk(c.ikeys, c.iscales, c.seq_len, 4, q_idx[i], head_w[i], self.topk, out=self.sel,
+                             ws=self.ws_idx, err=self.err)
+                hybrid_decode_attention(q[i], c.comp_kv, 4, self.sel, c.win_kv, self.window, c.seq_len, scale,
+                                        out=out[i], lse=l_i, ws=self.ws_att, err=self.err)
+            else:
+                hybrid_decode_attention(q[i], c.comp_kv, 128, None, c.win_kv, self.window, c.seq_len, scale,
+                                        out=out[i], lse=l_i, ws=self.ws_att, err=self.err)
