@@ -25,6 +25,7 @@ roofline of the dominant kernel.  `--impl reference` times the float64 CPU oracl
 rank 0 only), on a bounded sample of the same workload.
 """
 import argparse
+import gc
 import json
 import math
 import os
@@ -158,6 +159,7 @@ PROFILES = {
     ("indexer", "decode1m"): ("indexer_topk_decode1m.md", "indexer.cu", ""),
     ("csa_attention", "decode1m"): ("attention_tc_partial_decode1m.md", "attention_tc.cu", " (CSA)"),
     ("hca_attention", "decode1m"): ("attention_tc_partial_decode1m.md", "attention_tc.cu", " (HCA)"),
+    ("attention", "decode1m"): ("attention_tc_partial_decode1m.md", "attention_tc.cu", " (CSA+HCA)"),
     ("csa_compress", "prefill128k"): ("compress_prefill128k.md", "compress.cu", " (CSA)"),
     ("hca_compress", "prefill128k"): ("compress_prefill128k.md", "compress.cu", " (HCA)"),
 }
@@ -385,18 +387,55 @@ def run_decode(args, wl, rank, world, local_rank, steps=None, with_e2e=True):
             per[n] += sum(evs[2 * r].elapsed_time(evs[2 * r + 1]) for r in range(n_rep))
     avg = {n: per[n] / (n_instr * n_rep) for n in per}             # ms per launch (one call per step)
 
+    # Each operation alone, graph-replayed with its early-launch edges kept: the attention calls
+    # (CSA on the selections of the last step, HCA) rotating over 8 HCA cache copies so a round
+    # touches ~350 MB before any data comes round again, and the indexer calls over the 3
+    # replicas (252 MB per round).  These give the per-launch durations of the roofline.
+    n_hca = 8
+    hca_copies = [layers[r % n_rep][1].comp_kv if r < n_rep else layers[r % n_rep][1].comp_kv.clone()
+                  for r in range(n_hca)]
+
+    def att_round():
+        for r in range(n_hca):
+            csa, hca = layers[r % n_rep]
+            csld.hybrid_decode_attention(q_all[r % n_rep], csa.comp_kv, 4, sel[r % n_rep], csa.win_kv, W, csa.seq_len,
+                                         scale, out=out_csa[r % n_rep], lse=lse_csa[r % n_rep], ws=ws_att, err=err)
+            csld.hybrid_decode_attention(q_all[r % n_rep], hca_copies[r], 128, None, hca.win_kv, W, hca.seq_len,
+                                         scale, out=out_hca[r % n_rep], lse=lse_hca[r % n_rep], ws=ws_att, err=err)
+
+    def idx_round():
+        for r in range(n_rep):
+            csa = layers[r][0]
+            csld.indexer_topk(csa.ikeys, csa.iscales, csa.seq_len, 4, qi_all[r], hw_all[r], k, out=sel[r],
+                              ws=ws_idx[r], err=err)
+
+    op_ms = {}
+    for name, fn, per_round in (("attention", att_round, n_hca), ("indexer", idx_round, n_rep)):
+        g_op = capture(torch, dev, fn)
+        g_op.replay()
+        n_op = max(20, int(0.3 / max(1e-6, avg["csa_attention" if name == "attention" else "indexer"] * 1e-3 *
+                                       per_round)))
+        ms_op, _ = time_steps(torch, dev, world, g_op, [g_op], n_op)
+        op_ms[name] = ms_op / (n_op * per_round)                    # ms per step (one call of each layer)
+        del g_op
+    del hca_copies
+    assert err.item() == 0, f"device error word {err.item()}"
+
     e2e = run_decode_e2e(csld, torch, layers, wl, dev, k, W, scale, ws_idx, ws_att, err, steps, world) \
         if with_e2e else None
 
     peaks, peak_kind = measured_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
     bytes_ = algorithmic_bytes(wl)
-    dominant = max(avg, key=avg.get)
-    achieved = bytes_[dominant] / (avg[dominant] * 1e-3) / 1e9
     step_bytes = sum(bytes_.values())
     ms_step = ms / steps
     att_bytes = bytes_["csa_attention"] + bytes_["hca_attention"]
-    att_ms = avg["csa_attention"] + avg["hca_attention"]
+    att_ms = op_ms["attention"]
+    # the dominant kernel of the step, and its per-launch duration from its own graph
+    dom_ms = {"indexer": op_ms["indexer"], "attention": att_ms}
+    dom_bytes = {"indexer": bytes_["indexer"], "attention": att_bytes}
+    dominant = max(dom_ms, key=dom_ms.get)
+    achieved = dom_bytes[dominant] / (dom_ms[dominant] * 1e-3) / 1e9
     return {
         "value": round(job_throughput(B * steps, ms, world), 1), "steps": steps, "ms_per_step": round(ms_step, 5),
         "config": {"workload": wl.name, "batch_per_gpu": B, "context": wl.context, "csa_entries": wl.csa_entries,
@@ -410,15 +449,23 @@ def run_decode(args, wl, rank, world, local_rank, steps=None, with_e2e=True):
                 "frac_of_peak": round(step_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak, 4),
                 "frac_of_8tbs": round(step_bytes / (ms_step * 1e-3) / 1e9 / 8000.0, 4)},
         "kernels_ms_per_step": {n: round(v, 5) for n, v in avg.items()},
-        "roofline": {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+        "roofline": {"kernel": "indexer_topk" if dominant == "indexer" else
+                     "hybrid_decode_attention (CSA + HCA calls)", "bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "traffic": profiled_traffic(dominant, wl.name),
-                     "algorithmic_bytes_per_launch": bytes_[dominant]},
-        "roofline_all": {n: {"achieved_gbs": round(bytes_[n] / (avg[n] * 1e-3) / 1e9, 1),
-                             "frac": round(bytes_[n] / (avg[n] * 1e-3) / 1e9 / hbm_peak, 4)} for n in avg},
+                     "algorithmic_bytes_per_launch": dom_bytes[dominant],
+                     "ms_per_launch": round(dom_ms[dominant], 5),
+                     "timing": "the operation's calls alone, graph-replayed with early-launch edges, CUDA events"},
+        "roofline_in_step": {n: {"achieved_gbs": round(bytes_[n] / (avg[n] * 1e-3) / 1e9, 1),
+                                 "frac": round(bytes_[n] / (avg[n] * 1e-3) / 1e9 / hbm_peak, 4)} for n in avg},
         "attention": {"bytes_per_step": att_bytes, "ms_per_step": round(att_ms, 5),
                       "gbs": round(att_bytes / (att_ms * 1e-3) / 1e9, 1),
-                      "frac": round(att_bytes / (att_ms * 1e-3) / 1e9 / hbm_peak, 4)},
+                      "frac": round(att_bytes / (att_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                      "timing": "CSA + HCA hybrid_decode_attention calls alone, graph-replayed over 8 HCA cache "
+                                "copies (early-launch edges kept)"},
+        "indexer": {"bytes_per_step": bytes_["indexer"], "ms_per_step": round(op_ms["indexer"], 5),
+                    "gbs": round(bytes_["indexer"] / (op_ms["indexer"] * 1e-3) / 1e9, 1),
+                    "frac": round(bytes_["indexer"] / (op_ms["indexer"] * 1e-3) / 1e9 / hbm_peak, 4)},
         "clocks": clk,
         "gpu_launches": LAUNCHES_PER_STEP * steps,
         "e2e": e2e,
@@ -733,6 +780,7 @@ def run_sweep(args, rank, world, local_rank):
             q_idx = qs["q_idx"].view(n_rep, L, B, 4, 64)
             head_w = qs["head_w"].view(n_rep, L, B, 4)
             out = torch.empty((n_rep, L, B, 16, 512), dtype=torch.float32, device=dev)
+            sel_all = torch.full((n_rep, L, B, k), -1, dtype=torch.int32, device=dev)
             ev_idx = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * L)] for _ in range(n_rep)]
             ev_att = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * L)] for _ in range(n_rep)]
 
@@ -744,12 +792,12 @@ def run_sweep(args, rank, world, local_rank):
                         if timed:
                             ev_idx[r][2 * i].record()
                         csld.indexer_topk(lay.ikeys, lay.iscales, lay.seq_len, 4, q_idx[r, i], head_w[r, i], k,
-                                          out=st.sel, ws=st.ws_idx, err=st.err)
+                                          out=sel_all[r, i], ws=st.ws_idx, err=st.err)
                         if timed:
                             ev_idx[r][2 * i + 1].record()
                             ev_att[r][2 * i].record()
-                        csld.hybrid_decode_attention(q[r, i], lay.comp_kv, 4, st.sel, lay.win_kv, W, lay.seq_len,
-                                                     scale, out=out[r, i], ws=st.ws_att, err=st.err)
+                        csld.hybrid_decode_attention(q[r, i], lay.comp_kv, 4, sel_all[r, i], lay.win_kv, W,
+                                                     lay.seq_len, scale, out=out[r, i], ws=st.ws_att, err=st.err)
                     else:
                         if timed:
                             ev_att[r][2 * i].record()
@@ -785,6 +833,32 @@ def run_sweep(args, rank, world, local_rank):
                             t_idx += ev_idx[r][2 * i].elapsed_time(ev_idx[r][2 * i + 1])
             t_att /= n_instr * n_rep
             t_idx /= n_instr * n_rep
+            # each operation alone over all layers (early-launch edges kept): attention calls on
+            # the selections of the last step, and the indexer calls
+            def att_only():
+                for r in range(n_rep):
+                    st = stacks[r]
+                    for i, lay in enumerate(st.layers):
+                        csld.hybrid_decode_attention(q[r, i], lay.comp_kv, lay.ratio,
+                                                     sel_all[r, i] if lay.has_indexer else None, lay.win_kv, W,
+                                                     lay.seq_len, scale, out=out[r, i], ws=st.ws_att, err=st.err)
+
+            def idx_only():
+                for r in range(n_rep):
+                    st = stacks[r]
+                    for i, lay in enumerate(st.layers):
+                        if lay.has_indexer:
+                            csld.indexer_topk(lay.ikeys, lay.iscales, lay.seq_len, 4, q_idx[r, i], head_w[r, i], k,
+                                              out=sel_all[r, i], ws=st.ws_idx, err=st.err)
+
+            op_ms = {}
+            for name, fn, guess in (("attention", att_only, t_att), ("indexer", idx_only, t_idx)):
+                g_op = capture(torch, dev, fn)
+                g_op.replay()
+                n_op = max(5, int(0.3 / max(1e-6, guess * 1e-3 * n_rep)))
+                ms_op, _ = time_steps(torch, dev, world, g_op, [g_op], n_op)
+                op_ms[name] = ms_op / (n_op * n_rep)
+                del g_op
             errs = [int(st.err.item()) for st in stacks]
             assert not any(errs), f"device error words {errs}"
             ms_step = ms / steps
@@ -795,13 +869,15 @@ def run_sweep(args, rank, world, local_rank):
                 "us_per_token": round(ms_step * 1e3 / B, 3),
                 "value": round(job_throughput(B * steps, ms, world), 1),
                 "bytes_per_step": step_bytes, "hbm_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
-                "attention": {"bytes_per_step": b_att, "ms_per_step": round(t_att, 4),
-                              "gbs": round(b_att / (t_att * 1e-3) / 1e9, 1),
-                              "frac": round(b_att / (t_att * 1e-3) / 1e9 / hbm_peak, 4),
-                              "us_per_layer_call": round(t_att * 1e3 / L, 2)},
-                "indexer": {"bytes_per_step": b_idx, "ms_per_step": round(t_idx, 4),
-                            "gbs": round(b_idx / (t_idx * 1e-3) / 1e9, 1),
-                            "frac": round(b_idx / (t_idx * 1e-3) / 1e9 / hbm_peak, 4)},
+                "attention": {"bytes_per_step": b_att, "ms_per_step": round(op_ms["attention"], 4),
+                              "gbs": round(b_att / (op_ms["attention"] * 1e-3) / 1e9, 1),
+                              "frac": round(b_att / (op_ms["attention"] * 1e-3) / 1e9 / hbm_peak, 4),
+                              "us_per_layer_call": round(op_ms["attention"] * 1e3 / L, 2),
+                              "in_step_ms": round(t_att, 4)},
+                "indexer": {"bytes_per_step": b_idx, "ms_per_step": round(op_ms["indexer"], 4),
+                            "gbs": round(b_idx / (op_ms["indexer"] * 1e-3) / 1e9, 1),
+                            "frac": round(b_idx / (op_ms["indexer"] * 1e-3) / 1e9 / hbm_peak, 4),
+                            "in_step_ms": round(t_idx, 4)},
                 "kv_bytes_per_sequence": kv_seq, "gqa8_bf16_bytes_per_sequence": gqa8,
                 "kv_frac_of_gqa8": round(kv_seq / gqa8, 5), "clocks": clk,
             })
@@ -809,8 +885,9 @@ def run_sweep(args, rank, world, local_rank):
                 pt["e2e"] = sweep_e2e(torch, dev, world, csld, stacks[0], kinds, kv_new[0], gate_new[0], q[0],
                                       q_idx[0], head_w[0], out[0], scale, B, min(steps, 200))
             points.append(pt)
-            del stacks, singles, rounds, instr, out, toks, qs
+            del stacks, singles, rounds, instr, out, toks, qs, sel_all, step, att_only, idx_only, src, lay, st, s_
             torch.cuda.synchronize()
+            gc.collect()
             torch.cuda.empty_cache()
     measured = [p for p in points if "skipped" not in p]
     assert measured, "no sweep point fits"
@@ -1003,8 +1080,8 @@ def decode_line(args, rank, world, local_rank):
             torch.cuda.empty_cache()
             e = run_decode(args, synth.WORKLOADS[name], rank, world, local_rank, steps=None)
             res["extra"][name] = {k: e[k] for k in ("value", "steps", "ms_per_step", "config", "hbm",
-                                                    "kernels_ms_per_step", "roofline", "roofline_all", "attention",
-                                                    "clocks", "e2e")}
+                                                    "kernels_ms_per_step", "roofline", "roofline_in_step",
+                                                    "attention", "indexer", "clocks", "e2e")}
             res["gpu_launches"] += e["gpu_launches"]
     return res
 

@@ -19,7 +19,8 @@ __all__ = [
     "csa_compress", "hca_compress", "compress", "indexer_topk", "hybrid_decode_attention",
     "kv_cache_append", "kv_cache_prefill", "LayerCache", "CsldError", "lib", "ENTRY_BYTES",
     "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace", "DecodeStack",
-    "layer_pattern", "stage",
+    "layer_pattern", "stage", "indexer_rescore", "topk_merge", "lse_merge", "ContextParallelLayer",
+    "partition_entries", "all_gather_stacked", "indexer_topk_multi", "indexer_multi_workspace",
 ]
 
 DIM = 512
@@ -70,8 +71,15 @@ def _load():
     L.csld_attention_workspace_size.argtypes = [I, I, I64, I, I]
     L.hybrid_decode_attention.argtypes = [P, I, P, I64, I, P, I, P, I, P, I, F, P, P, P, S, P, P]
     L.csld_stage.argtypes = [P, P, S, P]
+    L.indexer_rescore.argtypes = [P, P, I64, P, P, P, I, I, P, P]
+    L.csld_indexer_multi_workspace_size.restype = S
+    L.csld_indexer_multi_workspace_size.argtypes = [I, I, I64]
+    L.indexer_topk_multi.argtypes = [P, P, I64, P, I, P, P, I, I, I, P, P, S, P, P]
+    L.csld_topk_merge.argtypes = [P, P, P, I, I, I, I64, I64, P, P]
+    L.csld_lse_merge.argtypes = [P, P, I, I, I, P, P, P]
     for fn in ("csld_compress", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
-               "indexer_topk", "hybrid_decode_attention", "csld_stage"):
+               "indexer_topk", "hybrid_decode_attention", "csld_stage", "indexer_rescore", "csld_topk_merge",
+               "csld_lse_merge", "indexer_topk_multi"):
         getattr(L, fn).restype = I
     return L
 
@@ -214,6 +222,31 @@ def indexer_topk(ikeys, iscales, seq_len, ratio, q_idx, head_w, k, out=None, ws=
     return out
 
 
+def indexer_multi_workspace(B, Q, cap, device="cuda"):
+    n = lib.csld_indexer_multi_workspace_size(B, Q, cap)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def indexer_topk_multi(ikeys, iscales, seq_len, ratio, q_idx, head_w, k, out=None, ws=None, err=None):
+    """Q query tokens per sequence in one pass over the keys: q_idx [B,Q,4,64] f32, head_w
+    [B,Q,4] f32 -> top-k [B,Q,k] i32 (query j at raw position seq_len - Q + j)."""
+    _need(ikeys, torch.uint8, "ikeys")
+    _need(iscales, torch.float32, "iscales")
+    _need(seq_len, torch.int32, "seq_len")
+    _need(q_idx, torch.float32, "q_idx")
+    _need(head_w, torch.float32, "head_w")
+    B, cap = ikeys.shape[0], ikeys.shape[1]
+    Q = q_idx.shape[1]
+    if out is None:
+        out = torch.empty((B, Q, k), dtype=torch.int32, device=ikeys.device)
+    if ws is None:
+        ws = indexer_multi_workspace(B, Q, cap, ikeys.device)
+    _check(lib.indexer_topk_multi(_ptr(ikeys), _ptr(iscales), cap, _ptr(seq_len), ratio, _ptr(q_idx), _ptr(head_w),
+                                  B, Q, k, _ptr(out), _ptr(ws), ws.numel(), _ptr(err), _stream()),
+           "indexer_topk_multi")
+    return out
+
+
 # ---- attention ----------------------------------------------------------------------------
 def attention_workspace(B, cap, k, W, device="cuda"):
     n = lib.csld_attention_workspace_size(B, HEADS, cap, k, W)
@@ -325,3 +358,122 @@ class DecodeStack:
             else:
                 hybrid_decode_attention(q[i], c.comp_kv, 128, None, c.win_kv, self.window, c.seq_len, scale,
                                         out=out[i], lse=l_i, ws=self.ws_att, err=self.err)
+
+
+# ---- context-parallel split of a sequence over ranks -----------------------------------------
+def indexer_rescore(ikeys, iscales, q_idx, head_w, sel, out=None):
+    """fp32 scores [B,k] of the selected entries sel [B,k] (-inf where sel < 0): indexer_rescore."""
+    for t, dt, n in ((ikeys, torch.uint8, "ikeys"), (iscales, torch.float32, "iscales"), (q_idx, torch.float32, "q_idx"),
+                     (head_w, torch.float32, "head_w"), (sel, torch.int32, "sel")):
+        _need(t, dt, n)
+    B, k = sel.shape
+    if out is None:
+        out = torch.empty((B, k), dtype=torch.float32, device=sel.device)
+    _need(out, torch.float32, "out")
+    _check(lib.indexer_rescore(_ptr(ikeys), _ptr(iscales), ikeys.shape[1], _ptr(q_idx), _ptr(head_w), _ptr(sel), B, k,
+                               _ptr(out), _stream()), "indexer_rescore")
+    return out
+
+
+def topk_merge(cand_scores, cand_idx, rank_lo, lo, n_local, out=None):
+    """Global top-k over the gathered candidates cand_scores / cand_idx [R,B,k] (indices local to
+    rank r's range starting at rank_lo[r], i64 [R] on the device), written as indices local to
+    [lo, lo + n_local) (-1 elsewhere): csld_topk_merge."""
+    _need(cand_scores, torch.float32, "cand_scores")
+    _need(cand_idx, torch.int32, "cand_idx")
+    _need(rank_lo, torch.int64, "rank_lo")
+    R, B, k = cand_idx.shape
+    if out is None:
+        out = torch.empty((B, k), dtype=torch.int32, device=cand_idx.device)
+    _need(out, torch.int32, "out")
+    _check(lib.csld_topk_merge(_ptr(cand_scores), _ptr(cand_idx), _ptr(rank_lo), R, B, k, int(lo), int(n_local),
+                               _ptr(out), _stream()), "csld_topk_merge")
+    return out
+
+
+def lse_merge(outs, lses, out=None, lse=None):
+    """Combine partial attention results outs [R,B,16,512], lses [R,B,16]: csld_lse_merge."""
+    _need(outs, torch.float32, "outs")
+    _need(lses, torch.float32, "lses")
+    R, B, H = lses.shape
+    if out is None:
+        out = torch.empty((B, H, DIM), dtype=torch.float32, device=outs.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=outs.device)
+    _check(lib.csld_lse_merge(_ptr(outs), _ptr(lses), R, B, H, _ptr(out), _ptr(lse), _stream()), "csld_lse_merge")
+    return out, lse
+
+
+def all_gather_stacked(t, group=None):
+    """[world, *t.shape]: every rank's t, in rank order (torch.distributed all-gather into one
+    flat tensor: NCCL over NVLink between GPUs, gloo on CPU)."""
+    import torch.distributed as td
+    world = td.get_world_size(group)
+    t = t.contiguous()
+    flat = torch.empty((world * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+    td.all_gather_into_tensor(flat, t, group=group)
+    return flat.view((world,) + tuple(t.shape))
+
+
+def partition_entries(n_entries, world):
+    """Contiguous, near-equal ranges [lo_r, lo_r + n_r) of n_entries compressed entries over
+    `world` ranks, each start a multiple of 8 (the key layout's 8-entry groups stay whole)."""
+    per = -(-n_entries // world)
+    per = -(-per // 8) * 8
+    out = []
+    for r in range(world):
+        lo = min(n_entries, r * per)
+        out.append((lo, min(n_entries, lo + per) - lo))
+    return out
+
+
+class ContextParallelLayer:
+    """One layer's share of a context-parallel split on this rank: a LayerCache holding the
+    compressed entries [lo, lo + n_local) of every sequence (indices local to the range), and, on
+    the rank that owns the newest tokens, the window ring.  Lengths:
+      cache.seq_len   ratio x the visible local entries (what indexer_topk and the local
+                      attention see);
+      seq_len_total   the sequence's raw tokens (the window branch; window rank only).
+    step() runs one decode query through the layer on every rank of `group` (all ranks call it
+    together): local indexer top-k and rescoring, an all-gather of the candidates, the exact
+    global top-k, local attention, an all-gather of (out, lse), and their log-sum-exp merge.
+    `all_gather(t)` returns the [R, ...] stack of every rank's t; the default uses
+    torch.distributed (NCCL between GPUs)."""
+
+    def __init__(self, cache: LayerCache, lo, n_local, rank_lo, window_rank, seq_len_total=None, group=None,
+                 all_gather=None):
+        self.cache, self.lo, self.n_local = cache, int(lo), int(n_local)
+        self.rank_lo = rank_lo                      # i64 [R] on the device
+        self.window_rank = bool(window_rank)
+        self.seq_len_total = seq_len_total
+        self.group = group
+        self.all_gather = all_gather or self._dist_all_gather
+        B = cache.batch
+        dev = cache.comp_kv.device
+        self._no_sel = torch.full((B, 1), -1, dtype=torch.int32, device=dev)
+
+    def _dist_all_gather(self, t):
+        import torch.distributed as td
+        return all_gather_stacked(t, self.group)
+
+    def step(self, q, scale, k=None, q_idx=None, head_w=None, ws_idx=None, ws_att=None, err=None):
+        c = self.cache
+        B = c.batch
+        W = c.window if self.window_rank else 0
+        parts_o, parts_l = [], []
+        if c.has_indexer:
+            sel = indexer_topk(c.ikeys, c.iscales, c.seq_len, c.ratio, q_idx, head_w, k, ws=ws_idx, err=err)
+            sc = indexer_rescore(c.ikeys, c.iscales, q_idx, head_w, sel)
+            g_sc, g_idx = self.all_gather(sc), self.all_gather(sel)
+            mine = topk_merge(g_sc, g_idx, self.rank_lo, self.lo, self.n_local)
+            seq = self.seq_len_total if self.window_rank else c.seq_len
+            o, l = hybrid_decode_attention(q, c.comp_kv, c.ratio, mine, c.win_kv, W, seq, scale, ws=ws_att, err=err)
+        else:
+            o, l = hybrid_decode_attention(q, c.comp_kv, c.ratio, None, c.win_kv, 0, c.seq_len, scale, ws=ws_att,
+                                           err=err)
+            if self.window_rank and c.window > 0:
+                # the window alone: a sparse call whose one selected slot is empty
+                ow, lw = hybrid_decode_attention(q, c.comp_kv, c.ratio, self._no_sel, c.win_kv, c.window,
+                                                 self.seq_len_total, scale, err=err)
+                o, l = lse_merge(torch.stack([o, ow]), torch.stack([l, lw]))
+        return lse_merge(self.all_gather(o), self.all_gather(l))

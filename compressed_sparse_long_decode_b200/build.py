@@ -10,7 +10,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcsld.so")
-SOURCES = ["api.cu", "compress.cu", "indexer.cu", "attention.cu", "attention_tc.cu", "stage.cu"]
+SOURCES = ["api.cu", "compress.cu", "indexer.cu", "attention.cu", "attention_tc.cu", "stage.cu", "cp.cu", "indexer_multi.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-gencode", "arch=compute_100a,code=sm_100a",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",

@@ -13,6 +13,20 @@
 namespace csld {
 // stage.cu
 cudaError_t launch_stage(void* dst, const void* src, size_t bytes, int num_sms, cudaStream_t stream);
+// indexer_multi.cu
+size_t indexer_multi_ws_bytes(int B, int Q, int64_t cap);
+cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
+                                 int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
+                                 int32_t* topk_out, void* ws, int num_sms, int32_t* err, cudaStream_t stream);
+// cp.cu
+cudaError_t launch_indexer_rescore(const uint8_t* ikeys, const float* iscales, int64_t cap, const float* q_idx,
+                                   const float* head_w, const int32_t* sel, int B, int k, float* scores,
+                                   cudaStream_t stream);
+int topk_merge_max_candidates();
+cudaError_t launch_topk_merge(const float* cand_score, const int32_t* cand_idx, const int64_t* rank_lo, int R, int B,
+                              int k, int64_t lo, int64_t n_local, int32_t* out, cudaStream_t stream);
+cudaError_t launch_lse_merge(const float* outs, const float* lses, int R, int BH, float* out, float* lse,
+                             cudaStream_t stream);
 
 cudaError_t set_smem_attr_once(const void* kernel, size_t bytes) {
     static std::mutex mu;
@@ -258,6 +272,75 @@ csld_status hybrid_decode_attention_static(const uint16_t* q, int heads, const u
     e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, seq_len, B, scale, out,
                                lse_out, ws, plan, err, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention_static");
+    return CSLD_OK;
+}
+
+csld_status indexer_rescore(const uint8_t* ikeys, const float* iscales, int64_t cap, const float* q_idx,
+                            const float* head_w, const int32_t* sel, int B, int k, float* scores_out,
+                            void* stream) {
+    if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
+    if (k < 1 || k > CSLD_MAX_TOPK) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
+    if (cap < 1 || cap > ((int64_t)1 << 30)) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^30", (long long)cap);
+    if (cap & 1) return fail(CSLD_ERR_ALIGN, "cap must be even");
+    if (!ikeys || !iscales || !q_idx || !head_w || !sel || !scores_out)
+        return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (!aligned16(iscales)) return fail(CSLD_ERR_ALIGN, "iscales must be 16-byte aligned");
+    cudaError_t e = csld::launch_indexer_rescore(ikeys, iscales, cap, q_idx, head_w, sel, B, k, scores_out,
+                                                 as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "indexer_rescore");
+    return CSLD_OK;
+}
+
+csld_status csld_topk_merge(const float* cand_scores, const int32_t* cand_idx, const int64_t* rank_lo, int R, int B,
+                            int k, int64_t lo, int64_t n_local, int32_t* topk_out, void* stream) {
+    if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
+    if (k < 1 || k > CSLD_MAX_TOPK) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
+    if (R < 1 || (int64_t)R * k > csld::topk_merge_max_candidates())
+        return fail(CSLD_ERR_CAPACITY, "R * k = %lld candidates; at most %d", (long long)R * k,
+                    csld::topk_merge_max_candidates());
+    if (lo < 0 || n_local < 0 || lo + n_local > ((int64_t)1 << 30))
+        return fail(CSLD_ERR_ARG, "local range [%lld, %lld) outside 0..2^30", (long long)lo, (long long)(lo + n_local));
+    if (!cand_scores || !cand_idx || !rank_lo || !topk_out) return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    cudaError_t e = csld::launch_topk_merge(cand_scores, cand_idx, rank_lo, R, B, k, lo, n_local, topk_out,
+                                            as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "csld_topk_merge");
+    return CSLD_OK;
+}
+
+csld_status csld_lse_merge(const float* outs, const float* lses, int R, int B, int heads, float* out,
+                           float* lse_out, void* stream) {
+    if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; the library implements %d", heads, CSLD_HEADS);
+    if (B < 1 || B > 65535 || R < 1) return fail(CSLD_ERR_ARG, "B %d or R %d out of range", B, R);
+    if (!outs || !lses || !out) return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (!aligned16(outs) || !aligned16(out)) return fail(CSLD_ERR_ALIGN, "outs and out must be 16-byte aligned");
+    cudaError_t e = csld::launch_lse_merge(outs, lses, R, B * heads, out, lse_out, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "csld_lse_merge");
+    return CSLD_OK;
+}
+
+size_t csld_indexer_multi_workspace_size(int B, int Q, int64_t cap) {
+    if (B < 1 || Q < 1 || Q > CSLD_MULTI_MAX_Q || cap < 1) return 0;
+    return csld::indexer_multi_ws_bytes(B, Q, cap);
+}
+
+csld_status indexer_topk_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
+                               int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
+                               int32_t* topk_out, void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+    if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
+    if (Q < 1 || Q > CSLD_MULTI_MAX_Q) return fail(CSLD_ERR_ARG, "Q %d outside 1..%d", Q, CSLD_MULTI_MAX_Q);
+    if (k < 1 || k > CSLD_MAX_TOPK) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
+    if (cap < 2 || cap > ((int64_t)1 << 30)) return fail(CSLD_ERR_ARG, "cap %lld outside 2..2^30", (long long)cap);
+    if (cap & 1) return fail(CSLD_ERR_ALIGN, "cap must be even");
+    if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
+    if (!ikeys || !iscales || !seq_len || !q_idx || !head_w || !topk_out)
+        return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (!aligned16(ikeys) || !aligned16(iscales)) return fail(CSLD_ERR_ALIGN, "ikeys / iscales must be 16-byte aligned");
+    const size_t need = csld::indexer_multi_ws_bytes(B, Q, cap);
+    if (!ws || ws_bytes < need) return fail(CSLD_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CSLD_ERR_ALIGN, "workspace must be 256-byte aligned");
+    cudaError_t e = csld::launch_indexer_multi(ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, B, Q, k, topk_out,
+                                               ws, num_sms(), err, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_multi");
     return CSLD_OK;
 }
 

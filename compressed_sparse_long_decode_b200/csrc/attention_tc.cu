@@ -65,6 +65,7 @@ constexpr int kSmBar = 1;                     // named barrier of the 8 softmax 
 constexpr int kReadyBar = 2;                  // warps 4-15: query and tensor memory ready (384 threads)
 constexpr int kScaleBar = 3;                  // warps 4-15: query scales ready (384 threads)
 constexpr int kCopyBar = 4;                   // warps 0-3: the copy warps (128 threads)
+constexpr int kPrefetchTiles = 4;             // contiguous tiles requested into L2 ahead of their copy
 
 struct TcAttnSmem {
     uint8_t tile[2][kTileBytes];              // [block][entry][128 B], 128-byte swizzle
@@ -95,11 +96,6 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Offset of byte c of row r in a [rows][128 B] block with the 128-byte swizzle (the 16-byte
-// chunk index XOR the row index within each 8-row, 1024-byte atom).
-__device__ __forceinline__ int sw128(int r, int c) {
-    return (r >> 3) * 1024 + (r & 7) * 128 + ((((c >> 4) ^ r) & 7) << 4) + (c & 15);
-}
 __device__ __forceinline__ float order_key_to_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
@@ -119,17 +115,6 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
         :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
            "r"(smem_u32(bar))
         : "memory");
-}
-// Operand with the 128-byte swizzle (1024-byte aligned atoms): 8-row groups 1024 bytes apart
-// (SBO); LBO = stride between 128-byte column blocks of an MN-major operand wider than 128 B.
-__device__ __forceinline__ uint64_t desc_sw128(const void* p, uint32_t lbo) {
-    const uint32_t a = smem_u32(p);
-    uint64_t d = static_cast<uint64_t>((a >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-    d |= static_cast<uint64_t>(1024u >> 4) << 32;
-    d |= static_cast<uint64_t>(1u) << 46;
-    d |= static_cast<uint64_t>(2u) << 61;
-    return d;
 }
 // Scales 8 consecutive TMEM columns of this warp's lanes by f[0..7].
 __device__ __forceinline__ void tmem_scale8(uint32_t taddr, const float (&f)[8]) {
@@ -193,6 +178,7 @@ __device__ __forceinline__ void qprep_convert(TcAttnSmem& sm, const uint16_t* q,
 __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     const __grid_constant__ CUtensorMap kv_tile, const __grid_constant__ CUtensorMap kv_rows,
     const __grid_constant__ CUtensorMap win_rows, const __grid_constant__ CUtensorMap win_tile,
+    const uint8_t* __restrict__ comp_kv, const uint8_t* __restrict__ win_kv,
     const uint16_t* __restrict__ q, int64_t cap, int ratio,
     const int32_t* __restrict__ topk, int k, int W, const int32_t* __restrict__ seq_len, float scale, int splits,
     float* __restrict__ opart, float2* __restrict__ mlpart, int32_t* err) {
@@ -277,8 +263,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
     } else if (warp < 4) {
         // ===== copies (warps 0-3): tile t into buffer t & 1, started before the query is ready =====
+        // Contiguous tiles (dense mode) are also requested into L2 kPrefetchTiles ahead of their
+        // copy, so HBM keeps streaming while both tile buffers are busy; the copy of a tile then
+        // reads L2.  The window ring of the sequence is requested once.
+        auto prefetch_tile = [&](int tt) {
+            if (sparse || tt >= n_tiles) return;
+            const int64_t i0 = (t_begin + tt) * kTcTile;
+            if (i0 >= n_comp) return;
+            const int64_t rows = min64(kTcTile, n_comp - i0);
+            bulk_prefetch_l2(comp_kv + ((size_t)b * cap + (size_t)i0) * kEntry, static_cast<uint32_t>(rows * kEntry));
+        };
+        if (tid == 0) {
+            for (int tt = 0; tt < kPrefetchTiles; ++tt) prefetch_tile(tt);
+            if (n_win > 0 && (t_begin + n_tiles) * kTcTile > n_comp4)
+                bulk_prefetch_l2(win_kv + (size_t)b * W * kEntry, static_cast<uint32_t>(W * kEntry));
+        }
         int t = 0;
         for (; t < n_tiles; ++t) {
+            if (tid == 0) prefetch_tile(t + kPrefetchTiles);
             const int s = t & 1;
             const bool ok = !*fail && (t < 2 || mbar_wait(&sm.empty[s], ((t >> 1) - 1) & 1));
             if (ok && tid == 0) mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
@@ -613,7 +615,8 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
     cudaError_t e = set_smem_once(attention_tc_partial_kernel, smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(attention_tc_partial_kernel, dim3(splits, B), dim3(kTcThreads), smem, stream, kv_tile, kv_rows,
-                   win_rows, win_tile, q, cap, ratio, topk, k, W, seq_len, scale, splits, opart, mlpart, err);
+                   win_rows, win_tile, comp_kv, has_win ? win_kv : comp_kv, q, cap, ratio, topk, k, W, seq_len, scale,
+                   splits, opart, mlpart, err);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -7,12 +7,13 @@
 // tokens -> one entry), storage paragraph (FP8 entries, bf16 RoPE dims, FP4 indexer).
 //
 // Layout: one warp pools one entry; lane l owns dims [16l, 16l+16).  The raw stream is read
-// once with 16-byte loads (HBM-bound).  For CSA the pooled vectors of a 32-entry tile are
+// once with 16-byte loads (HBM-bound).  For CSA the pooled vectors of a 128-entry tile are
 // staged as bf16 in shared memory and projected by W_I (512x64, bf16 copy resident in shared
-// memory for the whole persistent CTA) on the tensor cores (mma.sync m16n8k16, fp32
-// accumulation); the FP4 quantisation runs on the fp32 result.
+// memory for the whole persistent CTA) on the 5th-generation tensor cores (tcgen05.mma
+// kind::f16, fp32 accumulation in tensor memory); the FP4 quantisation runs on the fp32 result.
 #include "csld_internal.cuh"
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 namespace csld {
 
@@ -27,10 +28,10 @@ __device__ __forceinline__ uint4 load_row16(const uint4* p) {
 // Pools the m rows of one block.  rows: [m][512] bf16; gate, bias: [m].  Lane l returns the
 // fp32 pooled values of dims [16l, 16l+16) in c[].  Deterministic order: weights are
 // normalised by a warp-tree sum, the weighted sum runs over j = 0..m-1 with fmaf.
-template <bool kReadOnly>
-__device__ __forceinline__ void warp_pool(const uint16_t* rows, const float* gate,
-                                          const float* __restrict__ bias, int m, int lane,
-                                          float (&c)[16]) {
+// Softmax weights of the m <= 128 slots of a block: lane l returns the weights of slots
+// l, l+32, l+64, l+96 in w[] (0 past m).
+__device__ __forceinline__ void warp_pool_weights(const float* gate, const float* __restrict__ bias, int m,
+                                                  int lane, float (&w)[4]) {
     float a[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -48,10 +49,16 @@ __device__ __forceinline__ void warp_pool(const uint16_t* rows, const float* gat
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    float w[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] = e[i] / s;
+}
 
+template <bool kReadOnly>
+__device__ __forceinline__ void warp_pool(const uint16_t* rows, const float* gate,
+                                          const float* __restrict__ bias, int m, int lane,
+                                          float (&c)[16]) {
+    float w[4];
+    warp_pool_weights(gate, bias, m, lane, w);
 #pragma unroll
     for (int d = 0; d < 16; ++d) c[d] = 0.f;
     const uint4* base = reinterpret_cast<const uint4*>(rows) + 2 * lane;
@@ -59,39 +66,29 @@ __device__ __forceinline__ void warp_pool(const uint16_t* rows, const float* gat
     for (int i = 0; i < 4; ++i) {
         if (32 * i >= m) break;
         const int jn = min(32, m - 32 * i);
-        int jj = 0;
-        // two rows per iteration keep four 16-byte loads in flight per lane
-        for (; jj + 1 < jn; jj += 2) {
-            const int j = 32 * i + jj;
-            const uint4 x0 = load_row16<kReadOnly>(base + (size_t)j * (kDim / 8));
-            const uint4 x1 = load_row16<kReadOnly>(base + (size_t)j * (kDim / 8) + 1);
-            const uint4 y0 = load_row16<kReadOnly>(base + (size_t)(j + 1) * (kDim / 8));
-            const uint4 y1 = load_row16<kReadOnly>(base + (size_t)(j + 1) * (kDim / 8) + 1);
-            const float wj = __shfl_sync(0xffffffffu, w[i], jj);
-            const float wk = __shfl_sync(0xffffffffu, w[i], jj + 1);
-            const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            const uint32_t yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+        // eight rows per batch: all sixteen 16-byte loads of a lane are issued before the
+        // first is used, then the rows are added in order (one fmaf per row and dim)
+        for (int j0 = 0; j0 < jn; j0 += 8) {
+            uint4 x[8][2];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                c[2 * q] = fmaf(wj, bf16_bits_to_f32(xv[q]), c[2 * q]);
-                c[2 * q + 1] = fmaf(wj, bf16_bits_to_f32(xv[q] >> 16), c[2 * q + 1]);
+            for (int r = 0; r < 8; ++r) {
+                const int j = 32 * i + j0 + r;
+                if (j0 + r < jn) {
+                    x[r][0] = load_row16<kReadOnly>(base + (size_t)j * (kDim / 8));
+                    x[r][1] = load_row16<kReadOnly>(base + (size_t)j * (kDim / 8) + 1);
+                }
             }
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                c[2 * q] = fmaf(wk, bf16_bits_to_f32(yv[q]), c[2 * q]);
-                c[2 * q + 1] = fmaf(wk, bf16_bits_to_f32(yv[q] >> 16), c[2 * q + 1]);
-            }
-        }
-        for (; jj < jn; ++jj) {
-            const int j = 32 * i + jj;
-            const uint4 x0 = load_row16<kReadOnly>(base + (size_t)j * (kDim / 8));
-            const uint4 x1 = load_row16<kReadOnly>(base + (size_t)j * (kDim / 8) + 1);
-            const float wj = __shfl_sync(0xffffffffu, w[i], jj);
-            const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            for (int r = 0; r < 8; ++r) {
+                if (j0 + r >= jn) break;
+                const float wj = __shfl_sync(0xffffffffu, w[i], j0 + r);
+                const uint32_t xv[8] = {x[r][0].x, x[r][0].y, x[r][0].z, x[r][0].w,
+                                        x[r][1].x, x[r][1].y, x[r][1].z, x[r][1].w};
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                c[2 * q] = fmaf(wj, bf16_bits_to_f32(xv[q]), c[2 * q]);
-                c[2 * q + 1] = fmaf(wj, bf16_bits_to_f32(xv[q] >> 16), c[2 * q + 1]);
+                for (int q = 0; q < 8; ++q) {
+                    c[2 * q] = fmaf(wj, bf16_bits_to_f32(xv[q]), c[2 * q]);
+                    c[2 * q + 1] = fmaf(wj, bf16_bits_to_f32(xv[q] >> 16), c[2 * q + 1]);
+                }
             }
         }
     }
@@ -152,105 +149,241 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
 }
 
 // ------------------------------------------------------------------------------------------
-// Pooling + indexer key (CSA).  Persistent CTAs of 8 warps over 32-entry tiles.
+// Pooling + indexer key (CSA) on the 5th-generation tensor cores.  Persistent CTAs (one per
+// SM) of 16 warps over 128-entry tiles:
+//  1. every warp pools 8 entries of the tile (one warp per entry, as above; for m = 4 two
+//     entries' raw rows are loaded at once, 256 bytes per lane in flight) and writes each
+//     entry to the cache and its bf16 copy into shared memory as row r of the A operand
+//     ([128 entries][512 dims], K-major, 128-byte swizzle: 8 column blocks of 64 dims);
+//  2. one thread issues the projection U = A . W_I (tcgen05.mma kind::f16, M = 128 entries,
+//     N = 64, K = 512 in 32 steps of 16; W_I^T resident in shared memory in the same layout)
+//     into 64 fp32 columns of tensor memory;
+//  3. warps 0-3 read U back (thread = entry = TMEM lane) and FP4-quantise its two 32-value
+//     groups in registers, writing the 32 code bytes (stored layout of csld.h) and 2 scales.
+// Each warp's first write of the next tile's A rows waits for the MMA that read the previous
+// tile, so the pooling loads of the next tile are already in flight meanwhile.
 // ------------------------------------------------------------------------------------------
-constexpr int kCTile = 32;                 // entries per tile
-constexpr int kAStride = kDim + 8;         // bf16 elements per staged row (16-byte pad)
-constexpr int kWStride = kDim + 8;         // bf16 elements per W^T row
-constexpr int kUStride = kIdxDim + 4;      // floats per projected row
+constexpr int kCTile = 128;                // entries per tile = the MMA's M
+constexpr int kCThreads = 512;
+constexpr uint32_t kCTmemCols = 64;        // U: 128 lanes x 64 fp32 columns
+constexpr uint32_t kIdProj = idesc_bf16_m128(kIdxDim, false, false);
 
 struct CompressSmem {
-    uint16_t wt[kIdxDim * kWStride];       // W_I^T in bf16: wt[n][k] = bf16(W_I[k][n])
-    uint16_t a[kCTile * kAStride];         // pooled rows of the tile, bf16
-    float u[kCTile * kUStride];            // projected rows, fp32
+    uint8_t a[kDim / 64][kCTile * 128];    // pooled rows, bf16: column block kb holds dims 64kb..64kb+63
+    uint8_t w[kDim / 64][kIdxDim * 128];   // W_I^T, bf16: row n of block kb holds W_I[64kb..64kb+63][n]
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int32_t fail;
 };
 
-__global__ void __launch_bounds__(256) pool_index_kernel(
-    const uint16_t* __restrict__ raw, const float* __restrict__ gate, const float* __restrict__ bias,
-    int m, const float* __restrict__ w_idx, int64_t T, int64_t E, int B, int64_t out_seq_stride,
-    uint8_t* __restrict__ kv_out, uint8_t* __restrict__ ikey_out, float* __restrict__ iscale_out) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    CompressSmem& sm = *reinterpret_cast<CompressSmem*>(smem_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-    // W_I^T (bf16) resident for the CTA's lifetime.
-    for (int i = tid; i < kDim * kIdxDim; i += blockDim.x) {
-        const int k = i / kIdxDim, n = i % kIdxDim;
-        sm.wt[n * kWStride + k] = static_cast<uint16_t>(f32_to_bf16_bits(w_idx[i]));
+// The 4 raw rows of an m = 4 block, this lane's 16 dims: x[2j], x[2j+1] = token j.
+__device__ __forceinline__ void load_block4(const uint16_t* rows, int lane, uint4 (&x)[8]) {
+    const uint4* base = reinterpret_cast<const uint4*>(rows) + 2 * lane;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        x[2 * j] = __ldg(base + (size_t)j * (kDim / 8));
+        x[2 * j + 1] = __ldg(base + (size_t)j * (kDim / 8) + 1);
     }
-
-    const int64_t tiles_per_seq = (E + kCTile - 1) / kCTile;
-    const int64_t n_tiles = tiles_per_seq * B;
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t b = tile / tiles_per_seq;
-        const int64_t s0 = (tile % tiles_per_seq) * kCTile;
-        const int n_here = static_cast<int>(min64(kCTile, E - s0));
-        __syncthreads();  // previous tile's smem fully consumed (and W^T written on the first pass)
-
-        // 1) pool 4 entries per warp; store entries; stage bf16 rows
-        for (int r = warp; r < kCTile; r += 8) {
-            uint32_t packed[8];
-            if (r < n_here) {
-                const int64_t s = s0 + r;
-                float c[16];
-                warp_pool<true>(raw + ((size_t)b * T + (size_t)s * m) * kDim,
-                          gate + (size_t)b * T + (size_t)s * m, bias, m, lane, c);
-                warp_store_entry(kv_out + ((size_t)b * out_seq_stride + (size_t)s) * kEntry, lane, c);
+}
+// Weighted sum of preloaded m = 4 rows, in the order warp_pool uses (slot 0, 1, 2, 3, one fmaf
+// per slot and dim), so the pooled values are bit-identical to it.
+__device__ __forceinline__ void pool4_preloaded(const uint4 (&x)[8], const float (&w)[4], float (&c)[16]) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    packed[q] = f32_to_bf16_bits(c[2 * q]) | (f32_to_bf16_bits(c[2 * q + 1]) << 16);
-            } else {
+    for (int d = 0; d < 16; ++d) c[d] = 0.f;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) packed[q] = 0u;
-            }
-            uint4* dst = reinterpret_cast<uint4*>(&sm.a[r * kAStride + 16 * lane]);
-            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-        }
-        __syncthreads();
-
-        // 2) u[32][64] = A[32][512] . W[512][64]; warp w: m-tile (w&1), n-tiles 2*(w>>1)+{0,1}
-        {
-            const int mt = warp & 1, nt0 = 2 * (warp >> 1);
-            const int g = lane >> 2, cq = lane & 3;
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            // ldmatrix addresses: lanes 0-15 rows 0-15 (k 0..7), lanes 16-31 rows 0-15 (k 8..15)
-            const uint16_t* arow = &sm.a[(mt * 16 + (lane & 15)) * kAStride + ((lane >> 4) << 3)];
-#pragma unroll 4
-            for (int ks = 0; ks < kDim / 16; ++ks) {
-                uint32_t a0, a1, a2, a3;
-                ldmatrix_x4(a0, a1, a2, a3, arow + ks * 16);
+    for (int j = 0; j < 4; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w[0], j);
+        const uint32_t xv[8] = {x[2 * j].x, x[2 * j].y, x[2 * j].z, x[2 * j].w,
+                                x[2 * j + 1].x, x[2 * j + 1].y, x[2 * j + 1].z, x[2 * j + 1].w};
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const uint16_t* wr = &sm.wt[((nt0 + j) * 8 + g) * kWStride + ks * 16 + 2 * cq];
-                    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wr);
-                    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wr + 8);
-                    mma_bf16(acc[j], a0, a1, a2, a3, b0, b1);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int col = (nt0 + j) * 8 + 2 * cq;
-                sm.u[(mt * 16 + g) * kUStride + col] = acc[j][0];
-                sm.u[(mt * 16 + g) * kUStride + col + 1] = acc[j][1];
-                sm.u[(mt * 16 + g + 8) * kUStride + col] = acc[j][2];
-                sm.u[(mt * 16 + g + 8) * kUStride + col + 1] = acc[j][3];
-            }
-        }
-        __syncthreads();
-
-        // 3) FP4 keys
-        for (int r = warp; r < n_here; r += 8) {
-            const int64_t s = s0 + r;
-            const float u0 = sm.u[r * kUStride + 2 * lane];
-            const float u1 = sm.u[r * kUStride + 2 * lane + 1];
-            warp_store_fp4(ikey_out + ((size_t)b * out_seq_stride + (size_t)s) * kIkey,
-                           iscale_out + ((size_t)b * out_seq_stride + (size_t)s) * 2, s, lane, u0, u1);
+        for (int q = 0; q < 8; ++q) {
+            c[2 * q] = fmaf(wj, bf16_bits_to_f32(xv[q]), c[2 * q]);
+            c[2 * q + 1] = fmaf(wj, bf16_bits_to_f32(xv[q] >> 16), c[2 * q + 1]);
         }
     }
 }
 
-size_t compress_index_smem_bytes() { return sizeof(CompressSmem); }
+// kM4: the block ratio is 4 (two blocks' raw rows are loaded at once); otherwise any ratio.
+template <bool kM4>
+__global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
+    const uint16_t* __restrict__ raw, const float* __restrict__ gate, const float* __restrict__ bias,
+    int m, const float* __restrict__ w_idx, int64_t T, int64_t E, int B, int64_t out_seq_stride,
+    uint8_t* __restrict__ kv_out, uint8_t* __restrict__ ikey_out, float* __restrict__ iscale_out) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    CompressSmem& sm = *reinterpret_cast<CompressSmem*>(smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kWarps = kCThreads / 32;
+
+    if (tid == 0) {
+        mbar_init(&sm.mma_done, 1);
+        sm.fail = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, kCTmemCols);
+        tmem_relinquish();
+    }
+    // W_I^T in bf16, resident for the CTA's lifetime
+    for (int i = tid; i < kDim * kIdxDim; i += kCThreads) {
+        const int k = i / kIdxDim, n = i % kIdxDim;
+        *reinterpret_cast<uint16_t*>(&sm.w[k >> 6][sw128(n, 2 * (k & 63))]) =
+            static_cast<uint16_t>(f32_to_bf16_bits(__ldg(w_idx + i)));
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int32_t* fail = &sm.fail;
+
+    const int64_t tiles_per_seq = (E + kCTile - 1) / kCTile;
+    const int64_t n_tiles = tiles_per_seq * B;
+    uint32_t phase = 0;
+    bool mma_pending = false;   // an MMA reading sm.a was issued and this warp has not seen it end
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int64_t b = tile / tiles_per_seq;
+        const int64_t s0 = (tile % tiles_per_seq) * kCTile;
+        const int n_here = static_cast<int>(min64(kCTile, E - s0));
+        const uint16_t* rb = raw + (size_t)b * T * kDim;
+        const float* gb = gate + (size_t)b * T;
+        uint8_t* kvb = kv_out + (size_t)b * out_seq_stride * kEntry;
+
+        // ---- 1) pooling: rows warp, warp + 16, ...; two rows at a time -------------------
+        for (int r0 = warp; r0 < kCTile; r0 += 2 * kWarps) {
+            // entries go to the cache as soon as they are pooled; their bf16 copies wait in
+            // registers for the shared-memory operand to be free
+            uint32_t packed[2][8];
+            if constexpr (kM4) {
+                uint4 x[2][8];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = r0 + h * kWarps;
+                    if (r < n_here) load_block4(rb + (size_t)(s0 + r) * 4 * kDim, lane, x[h]);
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = r0 + h * kWarps;
+                    float c[16];
+                    if (r < n_here) {
+                        float w[4];
+                        warp_pool_weights(gb + (s0 + r) * 4, bias, 4, lane, w);
+                        pool4_preloaded(x[h], w, c);
+                        warp_store_entry(kvb + (size_t)(s0 + r) * kEntry, lane, c);
+                    } else {
+#pragma unroll
+                        for (int d = 0; d < 16; ++d) c[d] = 0.f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        packed[h][q] = f32_to_bf16_bits(c[2 * q]) | (f32_to_bf16_bits(c[2 * q + 1]) << 16);
+                }
+            } else {
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    const int r = r0 + h * kWarps;
+                    float c[16];
+                    if (r < n_here) {
+                        warp_pool<true>(rb + (size_t)(s0 + r) * m * kDim, gb + (s0 + r) * m, bias, m, lane, c);
+                        warp_store_entry(kvb + (size_t)(s0 + r) * kEntry, lane, c);
+                    } else {
+#pragma unroll
+                        for (int d = 0; d < 16; ++d) c[d] = 0.f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        packed[h][q] = f32_to_bf16_bits(c[2 * q]) | (f32_to_bf16_bits(c[2 * q + 1]) << 16);
+                }
+            }
+            // the previous tile's MMA must be done reading sm.a before the first write
+            if (mma_pending) {
+                if (!mbar_wait(&sm.mma_done, phase ^ 1u)) *fail = 1;
+                mma_pending = false;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = r0 + h * kWarps;
+                // lane l holds dims 16l..16l+15: column block l / 4, bytes 32 (l % 4) .. +31
+                uint8_t* blk = sm.a[lane >> 2];
+                const int cb = 32 * (lane & 3);
+                *reinterpret_cast<uint4*>(blk + sw128(r, cb)) =
+                    make_uint4(packed[h][0], packed[h][1], packed[h][2], packed[h][3]);
+                *reinterpret_cast<uint4*>(blk + sw128(r, cb + 16)) =
+                    make_uint4(packed[h][4], packed[h][5], packed[h][6], packed[h][7]);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (*fail) break;
+        // ---- 2) projection on the tensor cores ---------------------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kb = 0; kb < kDim / 64; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // 16 bf16 = 32 bytes of K per MMA
+                    umma_f16(tmem, desc_sw128(sm.a[kb], 0) + (32 * ks) / 16, desc_sw128(sm.w[kb], 0) + (32 * ks) / 16,
+                             kIdProj, (kb | ks) != 0 ? 1u : 0u);
+            umma_commit(&sm.mma_done);
+        }
+        mma_pending = true;
+        // ---- 3) FP4 keys: warps 0-3, thread = entry ------------------------------------------
+        if (warp < 4) {
+            const bool ok = mbar_wait(&sm.mma_done, phase);
+            mma_pending = false;
+            if (!ok) *fail = 1;
+            tc_fence_after();
+            const int r = 32 * warp + lane;
+            const int64_t s = s0 + r;
+            const int sw = static_cast<int>((s >> 2) & 1);
+            const bool store = ok && r < n_here;
+            uint4* kdst = reinterpret_cast<uint4*>(ikey_out + ((size_t)b * out_seq_stride + (size_t)s) * kIkey);
+            float sc[2];
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {   // group g = columns 32g .. 32g+31
+                uint32_t u[2][16];
+                tmem_ld_32x32b_x16(tmem + ((32u * warp) << 16) + 32u * g, u[0]);
+                tmem_ld_32x32b_x16(tmem + ((32u * warp) << 16) + 32u * g + 16u, u[1]);
+                tmem_ld_wait();
+                float amax = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(u[i >> 4][i & 15])));
+                sc[g] = fp4_group_scale(amax);
+                const float inv = 1.0f / sc[g];   // exact: a power of two
+                uint32_t words[4];
+#pragma unroll
+                for (int wq = 0; wq < 4; ++wq) {
+                    uint32_t word = 0u;
+#pragma unroll
+                    for (int bq = 0; bq < 4; ++bq) {
+                        const int i = 8 * wq + 2 * bq;   // elements i, i+1 of the group
+                        const uint32_t byte = e2m1_code(__uint_as_float(u[i >> 4][i & 15]) * inv) |
+                                              (e2m1_code(__uint_as_float(u[(i + 1) >> 4][(i + 1) & 15]) * inv) << 4);
+                        word |= byte << (8 * bq);
+                    }
+                    words[wq] = word;
+                }
+                // group g's 16 bytes go to half g XOR (bit 2 of s) of the stored key
+                if (store) kdst[g ^ sw] = make_uint4(words[0], words[1], words[2], words[3]);
+            }
+            tc_fence_before();
+            if (store)
+                *reinterpret_cast<float2*>(iscale_out + ((size_t)b * out_seq_stride + (size_t)s) * 2) =
+                    make_float2(sc[0], sc[1]);
+        }
+        phase ^= 1u;
+    }
+    // the last MMA (if any) must end before tensor memory is released
+    if (mma_pending && tid == 0) (void)mbar_wait(&sm.mma_done, phase ^ 1u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kCTmemCols);
+    }
+}
+
+size_t compress_index_smem_bytes() { return sizeof(CompressSmem) + 1024; }
 
 cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float* bias, int m,
                             const float* w_idx, int64_t T, int B, int64_t out_seq_stride,
@@ -265,13 +398,14 @@ cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float*
                                                                        out_seq_stride, kv_out);
         return cudaGetLastError();
     }
-    const size_t smem = sizeof(CompressSmem);
-    cudaError_t e = set_smem_once(pool_index_kernel, smem);
-    if (e != cudaSuccess) return e;
+    const size_t smem = compress_index_smem_bytes();
     const int64_t tiles = ((E + kCTile - 1) / kCTile) * B;
-    const int64_t grid = min64(tiles, 2LL * num_sms);
-    pool_index_kernel<<<static_cast<unsigned>(grid), 256, smem, stream>>>(
-        raw, gate, bias, m, w_idx, T, E, B, out_seq_stride, kv_out, ikey_out, iscale_out);
+    const int64_t grid = min64(tiles, num_sms);
+    auto kernel = (m == 4) ? pool_index_kernel<true> : pool_index_kernel<false>;
+    cudaError_t e = set_smem_once(kernel, smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<static_cast<unsigned>(grid), kCThreads, smem, stream>>>(raw, gate, bias, m, w_idx, T, E, B, out_seq_stride,
+                                                                     kv_out, ikey_out, iscale_out);
     return cudaGetLastError();
 }
 

@@ -59,6 +59,7 @@ constexpr int kIdxTile = 256;          // entries per pipeline stage: two 128-ro
 constexpr int kIdxStages = 4;          // ring depth of the merge-tree kernel (shares the candidate area)
 constexpr int kCoopStages = 12;        // ring depth of the cooperative kernel (one CTA per SM)
 constexpr int kCoopGroup = 4;          // tiles per key copy in the cooperative kernel (32 KB of codes)
+constexpr int kIdxPrefetchGroups = 4;  // copy groups requested into L2 beyond the ring
 constexpr int kMaxStages = 12;
 constexpr int kIdxEpiGroups = 3;       // epilogue warpgroups: warps 0..11
 constexpr int kIdxProducerWarp = 12;   // issues the tensor / bulk copies
@@ -503,10 +504,21 @@ __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], flo
     if (warp == kIdxProducerWarp) {
         // --- producer: GT tiles of key codes + their scales per copy group ----------------
         if (lane == 0) {
+            // copy groups beyond the ring's reach are requested into L2 kIdxPrefetchGroups ahead,
+            // so the key stream keeps more bytes in flight than the ring holds
+            auto prefetch_group = [&](int gg) {
+                const int tg = gg * GT;
+                if (tg >= n_tiles) return;
+                const int ne = min(GT * kIdxTile, cn - tg * kIdxTile);
+                bulk_prefetch_l2(cbase + (size_t)tg * kIdxTile * kIkey, static_cast<uint32_t>(ne) * kIkey);
+                bulk_prefetch_l2(sbase + (size_t)tg * kIdxTile * 2, static_cast<uint32_t>((ne + 1) & ~1) * 8u);
+            };
+            for (int gg = kGroups; gg < kGroups + kIdxPrefetchGroups; ++gg) prefetch_group(gg);
             int t = 0;
             for (int g = 0; t < n_tiles; ++g) {
                 const int s0 = (g % kGroups) * GT;
                 if (*fail) break;
+                prefetch_group(g + kGroups + kIdxPrefetchGroups);
                 bool free = true;   // the group's stages held tiles t - S .. t - S + GT - 1
                 if (g >= kGroups)
                     for (int i = 0; i < GT && free; ++i)

@@ -1,0 +1,446 @@
+// Multi-query lightning indexer: Q query tokens of one sequence (a speculative or multi-token
+// prediction draft, or a prefill chunk) scored against the FP4 key cache in ONE pass over the
+// keys, then an exact top-k per query.
+//
+// Source: "DeepSeek-V4: a million-token context that agents can actually use" -- CSA paragraph
+// (FP4, ReLU-scored multi-head dot product of each query against the 4x-compressed entries; the
+// top-k compressed blocks per query), layer-pattern paragraph (the multi-token-prediction block
+// runs several query tokens per step).  Query j of sequence b stands at raw position
+// p = seq_len[b] - Q + j and sees the entries s < min((p + 1) / ratio, cap) (an entry is visible
+// once its last token is in).  Every query's score and selection are those indexer_topk forms
+// for it alone (same FP4 quantisation, exact integer group dots, same fp32 operation order, ties
+// to the lower index), so the result equals Q separate indexer_topk calls.
+//
+// 1. indexer_multi_score_kernel -- persistent CTAs over 128-entry tiles of every sequence.  A
+//    copy warp streams the key codes and scales with 1-D bulk copies, eight tiles (32 KB + 8 KB)
+//    per copy, three copies in flight; one thread issues one tcgen05.mma kind::mxf4 per tile
+//    (M = 128 entries, N = 8 Q rows of the query operand: row 8q + 4g + h holds group g of head
+//    h of query q, the other group zero, so each output column is one exact group dot); warps
+//    0-3 read the dots back (thread = entry), form every query's fp32 score and write its
+//    order key to the workspace, and add the keys' top 11 bits to per-query histograms, which
+//    the CTA adds into global ones at the end.
+// 2. indexer_multi_select_kernel -- one CTA per (sequence, query): the threshold bin from the
+//    global histogram, two more radix levels (11 + 10 bits) over that query's keys, then the
+//    entries in index order: every key above the threshold and the first ones equal to it.
+//    It zeroes the histogram it used, so the workspace stays ready for the next call.
+#include "csld_internal.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace csld {
+
+namespace {
+
+constexpr int kMqThreads = 256;          // warps 0-3 epilogue, warp 4 copies, warp 5 MMA
+constexpr int kMqTile = 128;             // entries per MMA (M)
+constexpr int kMqGroupTiles = 8;         // tiles per bulk copy
+constexpr int kMqGroup = kMqTile * kMqGroupTiles;   // 1024 entries per copy group
+constexpr int kMqStages = 3;             // copy groups in flight
+constexpr int kMqBins = 2048;            // histogram of the keys' top 11 bits
+constexpr uint32_t kMqTmemCols = 256;    // two accumulator slots of 8 Q <= 64 columns, scale factors at 128
+constexpr uint32_t kMqSfCol = 128;
+constexpr int kMqCopyWarp = 4, kMqMmaWarp = 5;
+
+struct MqSmem {
+    uint8_t codes[kMqStages][kMqGroup * kIkey];     // 32 KB per group, stored (pre-swizzled) layout
+    float scales[kMqStages][kMqGroup * 2];          // 8 KB per group
+    alignas(256) uint8_t bq[8 * CSLD_MULTI_MAX_Q * kIkey];   // query operand, 32-byte swizzle
+    float qscale[CSLD_MULTI_MAX_Q][8];              // [q][group * 4 + head]
+    uint32_t hist[CSLD_MULTI_MAX_Q][kMqBins];
+    uint64_t full[kMqStages], gfree[kMqStages], accf[2], sfree[2], drain;
+    uint32_t tmem_base;
+    int32_t fail, n_mma;
+};
+
+}  // namespace
+
+// Grid (chunks, B): CTA (c, b) scores tiles c, c + chunks, ... of sequence b's visible range.
+__global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
+    const uint8_t* __restrict__ ikeys, const float* __restrict__ iscales, int64_t cap,
+    const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
+    const float* __restrict__ head_w, int Q, uint32_t* __restrict__ keys_out, uint32_t* __restrict__ ghist,
+    int32_t* err) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    MqSmem& sm = *reinterpret_cast<MqSmem*>(smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.y, chunks = gridDim.x, c = blockIdx.x;
+    if (tid == 0) {
+        for (int s = 0; s < kMqStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.gfree[s], 4);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.accf[s], 1);
+            mbar_init(&sm.sfree[s], 4);
+        }
+        mbar_init(&sm.drain, 1);
+        sm.fail = 0;
+        sm.n_mma = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMqMmaWarp) {
+        tmem_alloc(&sm.tmem_base, kMqTmemCols);
+        tmem_relinquish();
+    }
+    for (int i = tid; i < Q * kMqBins; i += kMqThreads) (&sm.hist[0][0])[i] = 0u;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_wait();      // lengths, keys and queries come from upstream
+    pdl_trigger();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int32_t* fail = &sm.fail;
+
+    int32_t n = seq_len[b];
+    if (n < 0) {
+        if (tid == 0 && c == 0) dev_error(err, CSLD_DEVERR_SEQ_LEN);
+        n = 0;
+    }
+    // the newest query sees the most entries; query q sees n_q of them
+    const int64_t n_max = min64(n / ratio, cap);
+    const int n_tiles_all = static_cast<int>((n_max + kMqTile - 1) / kMqTile);
+    // this CTA's tiles: whole copy groups g = c, c + chunks, ...
+    const int n_groups_all = (n_tiles_all + kMqGroupTiles - 1) / kMqGroupTiles;
+    const int my_groups = n_groups_all > c ? (n_groups_all - c + chunks - 1) / chunks : 0;
+    const uint8_t* cbase = ikeys + (size_t)b * cap * kIkey;
+    const float* sbase = iscales + (size_t)b * cap * 2;
+
+    // ---- query operand (warps 0-3, then handed to the MMA warp; the copy warp starts at once) --
+    if (warp < 4) {
+        // thread t < 8 Q writes row n = t / 8 ... one row per 8 threads: thread (n, j) writes
+        // bytes 4j .. 4j+3 of row n
+        for (int t = tid; t < 64 * Q; t += 128) {
+            const int n_row = t >> 3, j = t & 7;
+            const int q = n_row >> 3, r8 = n_row & 7, h = r8 & 3, grp = r8 >> 2;
+            const float* qv = q_idx + (((size_t)b * Q + q) * kIdxHeads + h) * kIdxDim + 32 * grp;
+            float amax = 0.f;
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(__ldg(qv + i)));
+            const float sg = fp4_group_scale(amax);
+            const float inv = 1.0f / sg;   // exact: a power of two
+            uint32_t word = 0u;
+            if ((j >> 2) == grp) {   // bytes 4j..4j+3 hold elements 8(j&3) .. 8(j&3)+7 of group grp
+#pragma unroll
+                for (int i = 0; i < 8; ++i) word |= e2m1_code(__ldg(qv + 8 * (j & 3) + i) * inv) << (4 * i);
+            }
+            const int half = (j >> 2) ^ ((n_row >> 2) & 1);
+            *reinterpret_cast<uint32_t*>(sm.bq + n_row * kIkey + half * 16 + (j & 3) * 4) = word;
+            if (j == 0) sm.qscale[q][grp * 4 + h] = sg;
+        }
+        fence_proxy_async_smem();
+        // unit block-scale factors (UE8M0 0x7F = 2^0) for A and B, every lane
+        tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kMqSfCol, 0x7F7F7F7Fu);
+        tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kMqSfCol + 8, 0x7F7F7F7Fu);
+        tmem_st_wait();
+    }
+    if (warp < 4 || warp == kMqMmaWarp) {   // query operand and scale factors ready (warps 0-3, 5)
+        tc_fence_before();
+        named_barrier(1, 5 * 32);
+        tc_fence_after();
+    }
+
+    if (warp == kMqCopyWarp) {
+        if (lane == 0) {
+            for (int i = 0; i < my_groups; ++i) {
+                const int s = i % kMqStages;
+                if (*fail) break;
+                if (i >= kMqStages && !mbar_wait(&sm.gfree[s], ((i / kMqStages) - 1) & 1)) {
+                    *fail = 1;
+                    break;
+                }
+                const int64_t e0 = (int64_t)(c + i * chunks) * kMqGroup;
+                const int ne = static_cast<int>(min64(kMqGroup, n_max - e0));
+                const uint32_t cb = static_cast<uint32_t>(ne) * kIkey;
+                const uint32_t sb = static_cast<uint32_t>((ne + 1) & ~1) * 8u;   // cap is even
+                mbar_arrive_expect_tx(&sm.full[s], cb + sb);
+                bulk_g2s(sm.codes[s], cbase + (size_t)e0 * kIkey, cb, &sm.full[s]);
+                bulk_g2s(sm.scales[s], sbase + (size_t)e0 * 2, sb, &sm.full[s]);
+            }
+        }
+    } else if (warp == kMqMmaWarp) {
+        if (lane == 0) {
+            const uint64_t bdesc = smem_desc_kmajor_sw32(sm.bq);
+            const uint32_t idesc = idesc_mxf4_m128(static_cast<uint32_t>(8 * Q));
+            int t = 0;
+            for (int i = 0; i < my_groups && !*fail; ++i) {
+                const int s = i % kMqStages;
+                if (!mbar_wait(&sm.full[s], (i / kMqStages) & 1)) {
+                    *fail = 1;
+                    break;
+                }
+                tc_fence_after();
+                const int g = c + i * chunks;
+                const int nt = min(kMqGroupTiles, n_tiles_all - g * kMqGroupTiles);
+                for (int tt = 0; tt < nt; ++tt, ++t) {
+                    const int slot = t & 1;
+                    if (t >= 2 && !mbar_wait(&sm.sfree[slot], ((t >> 1) - 1) & 1)) {
+                        *fail = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    umma_mxf4(tmem + 64u * slot, smem_desc_kmajor_sw32(sm.codes[s] + tt * kMqTile * kIkey), bdesc, idesc,
+                              tmem + kMqSfCol, tmem + kMqSfCol + 8, 0u);
+                    umma_commit(&sm.accf[slot]);
+                }
+                if (*fail) break;
+            }
+            sm.n_mma = t;
+        }
+    } else if (warp < 4) {
+        // ---- epilogue: thread = entry m of the tile -------------------------------------------
+        const int m = 32 * warp + lane;
+        const uint32_t lane_addr = tmem + ((32u * warp) << 16);
+        const float* hw = head_w + (size_t)b * Q * kIdxHeads;
+        int t = 0;
+        for (int i = 0; i < my_groups; ++i) {
+            const int s = i % kMqStages;
+            const int g = c + i * chunks;
+            const int nt = min(kMqGroupTiles, n_tiles_all - g * kMqGroupTiles);
+            bool ok = true;
+            for (int tt = 0; tt < nt; ++tt, ++t) {
+                const int slot = t & 1;
+                ok = !*fail && mbar_wait(&sm.accf[slot], (t >> 1) & 1);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) *fail = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int64_t e = (int64_t)g * kMqGroup + tt * kMqTile + m;
+                const float2 ks = reinterpret_cast<const float2*>(sm.scales[s])[tt * kMqTile + m];
+                for (int q0 = 0; q0 < Q; q0 += 2) {   // two queries (16 columns) per load
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(lane_addr + 64u * slot + 8u * q0, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq) {
+                        const int q = q0 + qq;
+                        if (q >= Q) break;
+                        const int64_t n_q = min64((int64_t)(n - Q + q + 1) / ratio, cap);
+                        float rr[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            // d = fma(I1, s1, I0*s0) with s_g = (qscale_g * kscale_g) * 0.25
+                            const float i0 = __fmul_rn(__uint_as_float(r[8 * qq + h]), 4.0f);
+                            const float i1 = __fmul_rn(__uint_as_float(r[8 * qq + 4 + h]), 4.0f);
+                            const float s0 = __fmul_rn(__fmul_rn(sm.qscale[q][h], ks.x), 0.25f);
+                            const float s1 = __fmul_rn(__fmul_rn(sm.qscale[q][4 + h], ks.y), 0.25f);
+                            const float d = __fmaf_rn(i1, s1, __fmul_rn(i0, s0));
+                            rr[h] = d > 0.f ? d : 0.f;
+                        }
+                        const float* w = hw + q * kIdxHeads;
+                        float sc = __fmul_rn(__ldg(w + 0), rr[0]);
+                        sc = __fmaf_rn(__ldg(w + 1), rr[1], sc);
+                        sc = __fmaf_rn(__ldg(w + 2), rr[2], sc);
+                        sc = __fmaf_rn(__ldg(w + 3), rr[3], sc);
+                        const uint32_t key = score_key(sc);
+                        if (e < n_q) {
+                            keys_out[((size_t)b * Q + q) * cap + (size_t)e] = key;
+                            atomicAdd(&sm.hist[q][key >> 21], 1u);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sfree[slot]);
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.gfree[s]);   // the group's codes and scales are consumed
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (sm.fail) {
+        // a bounded wait gave up: record it and let the MMAs in flight finish before the tensor
+        // memory is released (the histograms of this call are then incomplete; zero the
+        // workspace again, as for indexer_topk)
+        if (warp == kMqMmaWarp && lane == 0) {
+            dev_error(err, CSLD_DEVERR_TIMEOUT);
+            umma_commit(&sm.drain);
+            (void)mbar_wait(&sm.drain, 0);
+        }
+        __syncthreads();
+    }
+    // this CTA's histograms into the global ones
+    for (int i = tid; i < Q * kMqBins; i += kMqThreads) {
+        const uint32_t v = (&sm.hist[0][0])[i];
+        if (v) atomicAdd(ghist + (size_t)b * Q * kMqBins + i, v);
+    }
+    if (warp == kMqMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kMqTmemCols);
+    }
+}
+
+namespace {
+
+// The bin of nb bins (counts in smem h) holding the want-th largest key and how many keys are
+// wanted inside it.  Warp 0 computes; results in sel[0..1].  Block-wide (ends with a barrier).
+__device__ void mq_find_bin(const uint32_t* h, int nb, uint32_t want, uint32_t* sel) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    if (tid < 32) {
+        if (lane == 0) {   // defaults if the counts fall short (an incomplete histogram)
+            sel[0] = 0u;
+            sel[1] = want;
+        }
+        __syncwarp();
+        const int per = nb / 32;                   // bins per lane, from the top
+        uint32_t tot = 0u;
+        for (int i = 0; i < per; ++i) tot += h[nb - 1 - per * lane - i];
+        uint32_t incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - tot;
+        if (excl < want && incl >= want) {
+            uint32_t run = excl;
+            for (int i = 0; i < per; ++i) {
+                const uint32_t cnt = h[nb - 1 - per * lane - i];
+                if (run + cnt >= want) {
+                    sel[0] = static_cast<uint32_t>(nb - 1 - per * lane - i);
+                    sel[1] = want - run;
+                    break;
+                }
+                run += cnt;
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// Block-wide exclusive scan of v (1024 threads); *total = the sum.
+__device__ __forceinline__ uint32_t mq_block_scan(uint32_t v, uint32_t* red, uint32_t* total) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t w = red[lane];
+        uint32_t wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        red[32 + lane] = wi - w;
+        if (lane == 31) red[64] = wi;
+    }
+    __syncthreads();
+    const uint32_t r = red[32 + warp] + incl - v;
+    *total = red[64];
+    __syncthreads();
+    return r;
+}
+
+}  // namespace
+
+// Grid (Q, B), 1024 threads: the exact top-k of query q of sequence b.
+__global__ void __launch_bounds__(1024) indexer_multi_select_kernel(const uint32_t* __restrict__ keys, int64_t cap,
+                                                                    const int32_t* __restrict__ seq_len, int ratio,
+                                                                    int Q, int k, uint32_t* __restrict__ ghist,
+                                                                    int32_t* __restrict__ topk_out) {
+    __shared__ uint32_t h[kMqBins];
+    __shared__ uint32_t sel[4];
+    __shared__ uint32_t red[96];
+    const int q = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    int32_t n = seq_len[b];
+    if (n < 0) n = 0;
+    const int64_t pos1 = (int64_t)n - Q + q + 1;                      // tokens this query sees
+    const int64_t n_q = pos1 > 0 ? min64(pos1 / ratio, cap) : 0;
+    const uint32_t* kq = keys + ((size_t)b * Q + q) * cap;
+    uint32_t* gh = ghist + ((size_t)b * Q + q) * kMqBins;
+    int32_t* out = topk_out + ((size_t)b * Q + q) * k;
+    for (int i = tid; i < kMqBins; i += blockDim.x) {
+        h[i] = gh[i];
+        gh[i] = 0u;    // ready for the next call
+    }
+    if (tid < 4) sel[tid] = 0u;
+    __syncthreads();
+    if (n_q <= k) {
+        for (int64_t i = tid; i < k; i += blockDim.x) out[i] = i < n_q ? static_cast<int32_t>(i) : -1;
+        return;
+    }
+    // level 1 (bits 31..21) from the scoring histogram
+    mq_find_bin(h, kMqBins, static_cast<uint32_t>(k), sel);
+    const uint32_t b1 = sel[0], need1 = sel[1];
+    __syncthreads();
+    // level 2 (bits 20..10) among the keys of bin b1
+    for (int i = tid; i < kMqBins; i += blockDim.x) h[i] = 0u;
+    __syncthreads();
+    for (int64_t i = tid; i < n_q; i += blockDim.x) {
+        const uint32_t key = kq[i];
+        if ((key >> 21) == b1) atomicAdd(&h[(key >> 10) & 2047u], 1u);
+    }
+    __syncthreads();
+    mq_find_bin(h, kMqBins, need1, sel);
+    const uint32_t b2 = sel[0], need2 = sel[1];
+    __syncthreads();
+    // level 3 (bits 9..0) among the keys with those top 22 bits
+    for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
+    __syncthreads();
+    const uint32_t top22 = (b1 << 11) | b2;
+    for (int64_t i = tid; i < n_q; i += blockDim.x) {
+        const uint32_t key = kq[i];
+        if ((key >> 10) == top22) atomicAdd(&h[key & 1023u], 1u);
+    }
+    __syncthreads();
+    mq_find_bin(h, 1024, need2, sel);
+    const uint32_t thr = (top22 << 10) | sel[0], take_eq = sel[1];
+    __syncthreads();
+    // emit in index order: keys above the threshold, and the first take_eq keys equal to it
+    uint32_t base_sel = 0u, base_eq = 0u;
+    for (int64_t i0 = 0; i0 < n_q; i0 += blockDim.x) {
+        const int64_t i = i0 + tid;
+        const uint32_t key = i < n_q ? kq[i] : 0u;
+        const uint32_t eq = (i < n_q && key == thr) ? 1u : 0u;
+        uint32_t eq_tot;
+        const uint32_t eq_before = base_eq + mq_block_scan(eq, red, &eq_tot);
+        const uint32_t take = (i < n_q && key > thr) || (eq && eq_before < take_eq) ? 1u : 0u;
+        uint32_t take_tot;
+        const uint32_t at = base_sel + mq_block_scan(take, red, &take_tot);
+        if (take && at < static_cast<uint32_t>(k)) out[at] = static_cast<int32_t>(i);
+        base_sel += take_tot;
+        base_eq += eq_tot;
+        if (base_sel >= static_cast<uint32_t>(k)) break;   // uniform: every thread sees the same totals
+    }
+}
+
+size_t indexer_multi_smem_bytes() { return sizeof(MqSmem) + 1024; }
+
+size_t indexer_multi_ws_bytes(int B, int Q, int64_t cap) {
+    const size_t keys = (size_t)B * Q * (size_t)cap * 4;
+    return (keys + 255) / 256 * 256 + (size_t)B * Q * kMqBins * 4;
+}
+
+cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
+                                 int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
+                                 int32_t* topk_out, void* ws, int num_sms, int32_t* err, cudaStream_t stream) {
+    uint32_t* keys = static_cast<uint32_t*>(ws);
+    uint32_t* ghist = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ((size_t)B * Q * (size_t)cap * 4 + 255) /
+                                                                                   256 * 256);
+    const size_t smem = indexer_multi_smem_bytes();
+    cudaError_t e = set_smem_once(indexer_multi_score_kernel, smem);
+    if (e != cudaSuccess) return e;
+    // copy groups of every sequence spread over about one CTA per SM
+    const int64_t groups = (cap + kMqGroup - 1) / kMqGroup;
+    int64_t chunks = max64(1, num_sms / max(B, 1));
+    chunks = min64(chunks, groups);
+    e = launch_pdl(indexer_multi_score_kernel, dim3(static_cast<unsigned>(chunks), B), dim3(kMqThreads), smem, stream,
+                   ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, Q, keys, ghist, err);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(indexer_multi_select_kernel, dim3(Q, B), dim3(1024), 0, stream, static_cast<const uint32_t*>(keys),
+                   cap, seq_len, ratio, Q, k, ghist, topk_out);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace csld

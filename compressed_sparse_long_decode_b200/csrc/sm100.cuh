@@ -104,6 +104,12 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                  :: "r"(smem_u32(bar)) : "memory");
 }
 
+// Hint: bring `bytes` (a multiple of 16) of global memory at p (16-byte aligned) into L2.  The
+// request is fire-and-forget; no smem, barrier or completion is involved.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
+}
+
 // ---- tensor maps -------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -167,6 +173,25 @@ __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
                  :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                  : "memory");
+}
+
+// Offset of byte c of row r in a [rows][128 B] block with the 128-byte swizzle (the 16-byte
+// chunk index XOR the row index within each 8-row, 1024-byte atom).
+__device__ __forceinline__ int sw128(int r, int c) {
+    return (r >> 3) * 1024 + (r & 7) * 128 + ((((c >> 4) ^ r) & 7) << 4) + (c & 15);
+}
+// Operand with the 128-byte swizzle (1024-byte aligned atoms): 8-row groups 1024 bytes apart
+// (SBO); LBO = stride between 128-byte column blocks of an MN-major operand wider than 128 B.
+// Advancing the start address by 32 bytes inside the row selects the next K slice of a K-major
+// operand.
+__device__ __forceinline__ uint64_t desc_sw128(const void* p, uint32_t lbo) {
+    const uint32_t a = smem_u32(p);
+    uint64_t d = static_cast<uint64_t>((a >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
 }
 
 // 2-D tensor map over a byte array of `rows` rows of `row_bytes` bytes (row_bytes a multiple of

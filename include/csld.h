@@ -193,6 +193,28 @@ CSLD_API csld_status indexer_topk(const uint8_t* ikeys, const float* iscales, in
                          size_t ws_bytes, int32_t* err, void* stream);
 
 /* ----------------------------------------------------------------------------------------
+ * Multi-query lightning indexer ([HF] CSA paragraph; layer-pattern paragraph: the
+ * multi-token-prediction block runs several query tokens per step).  Q query tokens per
+ * sequence -- the Q newest tokens: query j of sequence b stands at raw position
+ * p = seq_len[b] - Q + j and sees the entries s < min((p + 1) / ratio, cap) -- are scored in
+ * one pass over the key cache (the tensor cores take all Q queries as one operand), and each
+ * gets its own exact top-k.  Scores, ties and output order are those of indexer_topk for that
+ * query alone, so topk_out[b][j] equals indexer_topk with seq_len = p + 1 and query j.
+ *   ikeys / iscales as for indexer_topk, q_idx [B][Q][4][64] f32, head_w [B][Q][4] f32,
+ *   topk_out [B][Q][k] i32 (ascending, -1 padded).  1 <= Q <= CSLD_MULTI_MAX_Q, 1 <= k <= 2048.
+ * Workspace: csld_indexer_multi_workspace_size(B, Q, cap) bytes (the Q score arrays and their
+ * histograms), 256-byte aligned, zero-filled once before its first use; each call leaves it
+ * ready for the next.  Calls that share one workspace must not overlap on the GPU; after a call
+ * that reported CSLD_DEVERR_TIMEOUT, zero it again.
+ * ---------------------------------------------------------------------------------------- */
+#define CSLD_MULTI_MAX_Q 8
+CSLD_API size_t csld_indexer_multi_workspace_size(int B, int Q, int64_t cap);
+CSLD_API csld_status indexer_topk_multi(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                                        const int32_t* seq_len, int ratio, const float* q_idx,
+                                        const float* head_w, int B, int Q, int k, int32_t* topk_out,
+                                        void* ws, size_t ws_bytes, int32_t* err, void* stream);
+
+/* ----------------------------------------------------------------------------------------
  * Hybrid decode attention ([HF] CSA paragraph + Figure 3: attention over the selected entries
  * plus a sliding-window branch; HCA paragraph + Figure 4: dense attention over every
  * compressed entry plus the same window branch).
@@ -247,6 +269,47 @@ CSLD_API csld_status hybrid_decode_attention_static(const uint16_t* q, int heads
                                                     const int32_t* seq_len, int B, float scale,
                                                     float* out, float* lse_out, int32_t* err,
                                                     void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Context-parallel decode: one sequence's compressed cache split over R GPUs, rank r holding
+ * the contiguous entries [lo_r, lo_r + n_r) of every sequence (the window ring and the tail on
+ * one rank).  ([HF] CSA paragraph: the indexer picks the top-k compressed blocks per query; HCA
+ * paragraph: dense attention over the compressed stream.  The split is this library's; the
+ * pages run everything on one device.)  A decode step on rank r:
+ *   1. indexer_topk on the local keys -> local selection;  indexer_rescore -> their scores;
+ *      the caller all-gathers (score, local index) over the ranks into [R][B][k];
+ *   2. csld_topk_merge -> the global top-k, written as this rank's local indices;
+ *   3. hybrid_decode_attention on the local cache with that selection (sparse mode; dense mode
+ *      for HCA layers) -> (out_r, lse_r); the caller all-gathers them into [R][B][16][512] and
+ *      [R][B][16];
+ *   4. csld_lse_merge -> the step's output.
+ * Because the top-k of a union is the top-k of the union of the parts' top-k, and a softmax over
+ * a union of key sets is the log-sum-exp combination of the parts, the result is the single-GPU
+ * one: the same selection, and the same output up to fp32 rounding.
+ *
+ * indexer_rescore: scores_out[b][j] = the fp32 score (same quantisation and operation order as
+ * indexer_topk) of entry sel[b][j] of sequence b, or -inf where sel[b][j] < 0 or >= cap.
+ *   ikeys / iscales as for indexer_topk (stored layout, cap even, iscales 16-byte aligned),
+ *   q_idx [B][4][64] f32, head_w [B][4] f32, sel [B][k] i32, scores_out [B][k] f32.
+ * csld_topk_merge: cand_scores [R][B][k] f32 and cand_idx [R][B][k] i32 (indices local to rank
+ *   r's range, -1 = none), rank_lo [R] i64 (device: where rank r's range starts) -> topk_out[b] =
+ *   the min(k, #candidates) best candidates of sequence b by (score desc, global index asc), in
+ *   ascending index order, each written as global - lo when lo <= global < lo + n_local and as
+ *   -1 otherwise; -1 padded.  R * k <= 16384; global indices below 2^31 - 1.
+ * csld_lse_merge: outs [R][B][heads][512] f32, lses [R][B][heads] f32 (natural log; -inf =
+ *   empty part) -> out [B][heads][512] = sum_r exp(lses_r - L) outs_r, lse_out [B][heads] = L
+ *   = log sum_r exp(lses_r) (may be NULL).  heads == 16; outs and out 16-byte aligned.
+ * All three only enqueue kernels on `stream`; the all-gathers between them are the caller's
+ * (NCCL over NVLink in the Python binding).
+ * ---------------------------------------------------------------------------------------- */
+CSLD_API csld_status indexer_rescore(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                                     const float* q_idx, const float* head_w, const int32_t* sel, int B,
+                                     int k, float* scores_out, void* stream);
+CSLD_API csld_status csld_topk_merge(const float* cand_scores, const int32_t* cand_idx,
+                                     const int64_t* rank_lo, int R, int B, int k, int64_t lo,
+                                     int64_t n_local, int32_t* topk_out, void* stream);
+CSLD_API csld_status csld_lse_merge(const float* outs, const float* lses, int R, int B, int heads,
+                                    float* out, float* lse_out, void* stream);
 
 /* ----------------------------------------------------------------------------------------
  * csld_stage -- copies `bytes` from src to dst with a kernel on `stream`.  The pages have no
