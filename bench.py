@@ -14,6 +14,10 @@ Workloads (seeded synthetic data resident in HBM; see synth/__init__.py):
   sweep61                one step = one decode token per sequence through a 61-layer stack (layers
                          0-1 HCA, then CSA / HCA alternating), swept over context x batch; the
                          line's value is the 1M-token, batch-8 point, every point is under "sweep".
+  mtp1m                  one step = Q = 4 query tokens per sequence (a multi-token-prediction or
+                         speculative draft) at the decode1m shape: the multi-query indexer (one
+                         pass over the FP4 keys for all 4), multi-query sparse CSA attention and
+                         multi-query dense HCA attention.
 
 Timing: exactly K steps are replayed from CUDA graphs (graphs of one step per cache replica, the
 replicas rotating so that no step finds its data in L2 from the step before), between a
@@ -52,7 +56,8 @@ def parse(argv=None):
     p.add_argument("--steps", type=int, default=None,
                    help="timed steps (default: as many as fill about 1.2 s; 10 for the reference arm)")
     p.add_argument("--warmup", type=int, default=6)
-    p.add_argument("--workload", default="decode1m", choices=["decode1m", "decode128k", "prefill128k", "sweep61"])
+    p.add_argument("--workload", default="decode1m",
+                   choices=["decode1m", "decode128k", "prefill128k", "sweep61", "mtp1m"])
     p.add_argument("--extra", default="decode128k", help="decode workloads reported under 'extra' ('none')")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -661,6 +666,112 @@ def run_prefill(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------------------------------
+# Multi-query decode (mtp1m): Q draft tokens per sequence at the decode1m shape.
+# ------------------------------------------------------------------------------------------
+MTP_Q = 4
+
+
+def run_mtp(args, rank, world, local_rank):
+    import torch
+    import compressed_sparse_long_decode_b200 as csld
+    import synth
+    wl = synth.WORKLOADS["decode1m"]
+    Q = MTP_Q
+    B, W, k = wl.batch, wl.window, wl.topk
+    n_rep = REPLICAS
+    dev = torch.device("cuda", local_rank)
+    scale = 1.0 / math.sqrt(512.0)
+    g = synth.gen(4242 + rank, dev)
+    W_ring = W + Q - 1
+    reps = []
+    for r in range(n_rep):
+        csa_kv = synth.random_entries((B, wl.csa_cap), g, dev)
+        hca_kv = synth.random_entries((B, wl.hca_cap), g, dev)
+        ring_c = synth.random_entries((B, W_ring), g, dev)
+        ring_h = synth.random_entries((B, W_ring), g, dev)
+        ik, isc = synth.random_ikeys(B, wl.csa_cap, g, dev, heavy_frac=wl.heavy_frac, n_valid=wl.csa_entries)
+        reps.append(dict(csa=csa_kv, hca=hca_kv, ring_c=ring_c, ring_h=ring_h, ik=synth.ikeys_swap_halves(ik), isc=isc,
+                         ws=csld.indexer_multi_workspace(B, Q, wl.csa_cap, dev)))
+        del ik
+    seq = torch.full((B,), wl.context, dtype=torch.int32, device=dev)
+    qd = synth.decode_queries(B * Q * n_rep, seed=300 + rank, device=dev)
+    q_all = qd["q"].view(n_rep, B, Q, 16, 512)
+    qgen = synth.gen(301 + rank, dev)
+    qi_all = torch.randn((n_rep, B, Q, 4, 64), generator=qgen, device=dev)
+    hw_all = torch.randn((n_rep, B, Q, 4), generator=qgen, device=dev).abs()
+    sel = torch.empty((n_rep, B, Q, k), dtype=torch.int32, device=dev)
+    out_c = torch.empty((n_rep, B, Q, 16, 512), dtype=torch.float32, device=dev)
+    out_h = torch.empty_like(out_c)
+    ws_att = csld.attention_workspace(B * Q, max(wl.csa_cap, wl.hca_cap), k, W, dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ev = {n: [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n_rep)]
+          for n in ("indexer", "csa_attention", "hca_attention")}
+
+    def step(r, timed):
+        x = reps[r]
+        if timed:
+            ev["indexer"][2 * r].record()
+        csld.indexer_topk_multi(x["ik"], x["isc"], seq, 4, qi_all[r], hw_all[r], k, out=sel[r], ws=x["ws"], err=err)
+        if timed:
+            ev["indexer"][2 * r + 1].record()
+            ev["csa_attention"][2 * r].record()
+        csld.hybrid_decode_attention_multi(q_all[r], x["csa"], 4, sel[r], x["ring_c"], W, seq, scale, out=out_c[r],
+                                           ws=ws_att, err=err)
+        if timed:
+            ev["csa_attention"][2 * r + 1].record()
+            ev["hca_attention"][2 * r].record()
+        csld.hybrid_decode_attention_multi(q_all[r], x["hca"], 128, None, x["ring_h"], W, seq, scale, out=out_h[r],
+                                           ws=ws_att, err=err)
+        if timed:
+            ev["hca_attention"][2 * r + 1].record()
+
+    for r in range(n_rep):
+        step(r, False)
+    torch.cuda.synchronize()
+    singles = [capture(torch, dev, lambda r=r: step(r, False)) for r in range(n_rep)]
+    rounds = capture(torch, dev, lambda: [step(r, False) for r in range(n_rep)])
+    instr = capture(torch, dev, lambda: [step(r, True) for r in range(n_rep)])
+    replay_steps(rounds, singles, max(3, args.warmup))
+    steps = args.steps or auto_steps(torch, rounds, singles, n_rep)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ms, (h0, h1) = time_steps(torch, dev, world, rounds, singles, steps)
+    clk = clocks.stop(h0, h1)
+    per = {n: 0.0 for n in ev}
+    for _ in range(10):
+        instr.replay()
+        torch.cuda.synchronize()
+        for n, evs in ev.items():
+            per[n] += sum(evs[2 * r].elapsed_time(evs[2 * r + 1]) for r in range(n_rep))
+    avg = {n: per[n] / (10 * n_rep) for n in per}
+    assert err.item() == 0, f"device error word {err.item()}"
+    peaks, peak_kind = measured_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    bytes_ = {"indexer": B * wl.csa_entries * 40 + 2 * B * Q * wl.csa_entries * 4,   # keys once; score keys out and in
+              "csa_attention": B * Q * (k + W) * 576,
+              "hca_attention": B * (wl.hca_entries + W + Q - 1) * 576}              # the cache once per step
+    dominant = max(avg, key=avg.get)
+    achieved = bytes_[dominant] / (avg[dominant] * 1e-3) / 1e9
+    ms_step = ms / steps
+    return {
+        "metric": METRIC, "value": round(job_throughput(B * Q * steps, ms, world), 1), "unit": UNIT,
+        "n_gpus": world, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3+bf16 KV, e2m1 indexer keys; tcgen05 e2m1, e4m3 and bf16 MMA, fp32 accumulate",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "mtp1m", "batch_per_gpu": B, "queries_per_sequence": Q, "context": wl.context,
+                   "topk": k, "window": W,
+                   "l2": f"{n_rep} rotating cache replicas", "parallelism": f"replicas x{world}"},
+        "kernels_ms_per_step": {n: round(v, 5) for n, v in avg.items()},
+        "indexer_keys_gbs": round(B * wl.csa_entries * 40 / (avg["indexer"] * 1e-3) / 1e9, 1),
+        "roofline": {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                     "algorithmic_bytes_per_launch": bytes_[dominant]},
+        "clocks": clk, "gpu_launches": steps * 6,
+    }
+
+
+# ------------------------------------------------------------------------------------------
 # The 61-layer stack (sweep61).
 # ------------------------------------------------------------------------------------------
 def stack_bytes_per_step(kinds, B, context, topk, window):
@@ -1039,7 +1150,7 @@ def run_reference(args):
         sample = f"{T} of the 131072 tokens per step, compressed at ratios 4 and 128, float64 C"
         config = {"workload": "prefill128k", "tokens": T}
     else:
-        wl = synth.WORKLOADS["decode1m" if args.workload == "sweep61" else args.workload]
+        wl = synth.WORKLOADS["decode1m" if args.workload in ("sweep61", "mtp1m") else args.workload]
         smp = oracle_sample(wl, 1)
         for _ in range(args.warmup):
             oracle_step(oracle, wl, smp)
@@ -1111,6 +1222,9 @@ def main():
         elif args.workload == "sweep61":
             res = run_sweep(args, rank, world, local_rank)
             baseline = cpu_baseline_sweep
+        elif args.workload == "mtp1m":
+            res = run_mtp(args, rank, world, local_rank)
+            baseline = lambda: None   # noqa: E731
         else:
             import synth
             res = decode_line(args, rank, world, local_rank)
@@ -1118,7 +1232,9 @@ def main():
         if res is None:
             return
         if rank == 0 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = baseline()
+            cb = baseline()
+            if cb is not None:
+                res["cpu_baseline"] = cb
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

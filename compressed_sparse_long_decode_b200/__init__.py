@@ -21,6 +21,7 @@ __all__ = [
     "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace", "DecodeStack",
     "layer_pattern", "stage", "indexer_rescore", "topk_merge", "lse_merge", "ContextParallelLayer",
     "partition_entries", "all_gather_stacked", "indexer_topk_multi", "indexer_multi_workspace",
+    "hybrid_decode_attention_multi",
 ]
 
 DIM = 512
@@ -75,11 +76,12 @@ def _load():
     L.csld_indexer_multi_workspace_size.restype = S
     L.csld_indexer_multi_workspace_size.argtypes = [I, I, I64]
     L.indexer_topk_multi.argtypes = [P, P, I64, P, I, P, P, I, I, I, P, P, S, P, P]
+    L.hybrid_decode_attention_multi.argtypes = [P, I, P, I64, I, P, I, P, I, I, P, I, I, F, P, P, P, S, P, P]
     L.csld_topk_merge.argtypes = [P, P, P, I, I, I, I64, I64, P, P]
     L.csld_lse_merge.argtypes = [P, P, I, I, I, P, P, P]
     for fn in ("csld_compress", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
                "indexer_topk", "hybrid_decode_attention", "csld_stage", "indexer_rescore", "csld_topk_merge",
-               "csld_lse_merge", "indexer_topk_multi"):
+               "csld_lse_merge", "indexer_topk_multi", "hybrid_decode_attention_multi"):
         getattr(L, fn).restype = I
     return L
 
@@ -284,6 +286,35 @@ def hybrid_decode_attention(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, 
                                        _ptr(win_kv) if W > 0 else None, W, _ptr(seq_len), B,
                                        float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                        _ptr(err), _stream()), "hybrid_decode_attention")
+    return out, lse
+
+
+def hybrid_decode_attention_multi(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, out=None, lse=None, ws=None,
+                                  err=None):
+    """Q query tokens per sequence: q [B,Q,16,512] bf16; topk [B,Q,k] i32 or None; win_kv
+    [B,W_ring,576] (W_ring >= W + Q - 1) -> (out [B,Q,16,512] f32, lse [B,Q,16] f32)."""
+    _bits(q, "q")
+    _need(comp_kv, torch.uint8, "comp_kv")
+    _need(seq_len, torch.int32, "seq_len")
+    B, Q, H = q.shape[0], q.shape[1], q.shape[2]
+    cap = comp_kv.shape[1]
+    k = 0
+    if topk is not None:
+        _need(topk, torch.int32, "topk")
+        k = topk.shape[2]
+    W_ring = win_kv.shape[1] if W > 0 else 0
+    if W > 0:
+        _need(win_kv, torch.uint8, "win_kv")
+    if out is None:
+        out = torch.empty((B, Q, H, DIM), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Q, H), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = attention_workspace(B * Q, cap, max(k, 1), W, q.device)
+    _check(lib.hybrid_decode_attention_multi(_ptr(q), H, _ptr(comp_kv), cap, ratio, _ptr(topk), k,
+                                             _ptr(win_kv) if W > 0 else None, W_ring, W, _ptr(seq_len), B, Q,
+                                             float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(err),
+                                             _stream()), "hybrid_decode_attention_multi")
     return out, lse
 
 

@@ -228,7 +228,7 @@ csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t*
     if (!ws || ws_bytes < plan.ws_bytes)
         return fail(CSLD_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, plan.ws_bytes);
     if (!aligned16(ws)) return fail(CSLD_ERR_ALIGN, "workspace must be 16-byte aligned");
-    cudaError_t e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, seq_len, B,
+    cudaError_t e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, W, 1, seq_len, B,
                                            scale, out, lse_out, ws, plan, err, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention");
     return CSLD_OK;
@@ -269,7 +269,7 @@ csld_status hybrid_decode_attention_static(const uint16_t* q, int heads, const u
     void* ws = nullptr;
     cudaError_t e = csld::attention_static_scratch(&ws);
     if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention_static (scratch address)");
-    e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, seq_len, B, scale, out,
+    e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, W, 1, seq_len, B, scale, out,
                                lse_out, ws, plan, err, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention_static");
     return CSLD_OK;
@@ -343,5 +343,36 @@ csld_status indexer_topk_multi(const uint8_t* ikeys, const float* iscales, int64
     if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_multi");
     return CSLD_OK;
 }
+
+csld_status hybrid_decode_attention_multi(const uint16_t* q, int heads, const uint8_t* comp_kv, int64_t cap,
+                                          int ratio, const int32_t* topk, int k, const uint8_t* win_kv, int W_ring,
+                                          int W, const int32_t* seq_len, int B, int Q, float scale, float* out,
+                                          float* lse_out, void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+    if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; the library implements %d", heads, CSLD_HEADS);
+    if (B < 1 || Q < 1 || Q > CSLD_MULTI_MAX_Q || (int64_t)B * Q > 65535)
+        return fail(CSLD_ERR_ARG, "B %d, Q %d: need 1 <= Q <= %d and B * Q <= 65535", B, Q, CSLD_MULTI_MAX_Q);
+    if (cap < 1 || cap > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^31-1", (long long)cap);
+    if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
+    if (W < 0 || W > CSLD_MAX_WINDOW) return fail(CSLD_ERR_ARG, "W %d outside 0..%d", W, CSLD_MAX_WINDOW);
+    if (W > 0 && (W_ring < W + Q - 1 || W_ring > CSLD_MAX_WINDOW + CSLD_MULTI_MAX_Q))
+        return fail(CSLD_ERR_ARG, "W_ring %d: need W + Q - 1 = %d <= W_ring <= %d", W_ring, W + Q - 1,
+                    CSLD_MAX_WINDOW + CSLD_MULTI_MAX_Q);
+    if (topk && (k < 1 || k > CSLD_MAX_TOPK)) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
+    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return fail(CSLD_ERR_ARG, "scale is not finite");
+    if (!q || !comp_kv || !seq_len || !out) return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (W > 0 && !win_kv) return fail(CSLD_ERR_ARG, "win_kv is NULL with W > 0");
+    if (!aligned16(q) || !aligned16(comp_kv) || (win_kv && !aligned16(win_kv)) || !aligned16(out))
+        return fail(CSLD_ERR_ALIGN, "q, comp_kv, win_kv and out must be 16-byte aligned");
+    const csld::AttentionPlan plan = csld::attention_plan(B * Q, cap, k, topk != nullptr, W, num_sms());
+    if (!ws || ws_bytes < plan.ws_bytes)
+        return fail(CSLD_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, plan.ws_bytes);
+    if (!aligned16(ws)) return fail(CSLD_ERR_ALIGN, "workspace must be 16-byte aligned");
+    cudaError_t e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, W > 0 ? W_ring : 0,
+                                           Q, seq_len, B, scale, out, lse_out, ws, plan, err, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention_multi");
+    return CSLD_OK;
+}
+
+void csld_test_set_barrier_extra(int extra) { csld::g_test_barrier_extra.store(extra < 0 ? 0 : extra); }
 
 }  // extern "C"

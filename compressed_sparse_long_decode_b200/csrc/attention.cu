@@ -130,17 +130,18 @@ AttentionPlan attention_plan(int B, int64_t cap, int k, bool sparse, int W, int 
 }
 
 cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
-                             const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                             const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                              const int32_t* seq_len, int B, float scale, float* out,
                              float* lse_out, void* ws, const AttentionPlan& plan, int32_t* err,
                              cudaStream_t stream) {
+    // B cache rows, Q query rows each: the plan and the partials count B * Q query rows
     float* opart = static_cast<float*>(ws);
-    float2* mlpart = reinterpret_cast<float2*>(opart + (size_t)B * plan.splits * kHeads * kDim);
-    cudaError_t e = launch_attention_tc_partial(q, comp_kv, cap, ratio, topk, k, win_kv, W, seq_len, B, scale,
+    float2* mlpart = reinterpret_cast<float2*>(opart + (size_t)B * Q * plan.splits * kHeads * kDim);
+    cudaError_t e = launch_attention_tc_partial(q, comp_kv, cap, ratio, topk, k, win_kv, W, Wr, Q, seq_len, B, scale,
                                                 plan.splits, opart, mlpart, err, stream);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attention_merge_kernel, dim3(B, kHeads), dim3(kMergeThreads), 0, stream, static_cast<const float*>(opart),
-                   static_cast<const float2*>(mlpart), plan.splits, out, lse_out);
+    e = launch_pdl(attention_merge_kernel, dim3(B * Q, kHeads), dim3(kMergeThreads), 0, stream,
+                   static_cast<const float*>(opart), static_cast<const float2*>(mlpart), plan.splits, out, lse_out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

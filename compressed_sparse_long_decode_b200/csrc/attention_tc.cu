@@ -9,10 +9,12 @@
 // dims); 16 query heads share it; one softmax runs over {selected or all visible entries} +
 // {window tokens}.
 //
-// One CTA = one split of one sequence's key list, walked in tiles of 128 entries; 16 warps.
+// One CTA = one split of one sequence's key list, walked in tiles of 96 entries; 16 warps.
 //  - Warps 0-3 bring a tile in with TMA: five 128-byte column blocks of every entry (bytes 0,
-//    128, 256, 384 and 448 -- the last one is the RoPE part), each block [128 entries][128 B]
-//    with the 128-byte swizzle.  Contiguous tiles take one box copy per block; otherwise rows
+//    128, 256, 384 and 448 -- the last one is the RoPE part), each block [96 entries][128 B]
+//    with the 128-byte swizzle, into one of three tile buffers, so copies run up to two tiles
+//    ahead of the PV that frees a buffer.  (The QK MMA has 128 rows: it also reads the 32 rows
+//    after a block, whose scores are never used.)  Contiguous tiles take one box copy per block; otherwise rows
 //    come four at a time by index (tile::gather4).  The same image is the K-major operand of
 //    QK (rows = entries) and the MN-major operand of PV (rows = dims).
 //  - Warp 4 issues the MMAs (one thread):
@@ -31,8 +33,8 @@
 //    warps 12-15 heads 8-15.  The running max is raised lazily: O is rescaled in tensor memory
 //    only when a tile's max exceeds it by more than 8 (log2 units), so P <= 256 always.
 //  - Warps 4-15 prepare the query operands while the first copies are in flight.
-//  Two tile buffers, two S slots and two P buffers overlap the copy of tile t+1, QK of t+1,
-//  softmax of t and PV of t-1.  Every wait is bounded.  Each split writes its unnormalised O,
+//  Three tile buffers, two S slots and two P buffers overlap the copies of tiles t+1 and t+2,
+//  QK of t+1, softmax of t and PV of t-1.  Every wait is bounded.  Each split writes its unnormalised O,
 //  the running max m (log2 units) and the sum l; attention_merge_kernel combines the splits.
 #include <stdint.h>
 
@@ -45,10 +47,13 @@ namespace csld {
 namespace {
 
 constexpr int kTcThreads = 512;
-constexpr int kTcTile = 128;                  // entries per tile
+constexpr int kTcTile = 96;                   // entries per tile: K of PV, valid rows of QK (a multiple of 32)
+constexpr int kTcRows = 128;                  // rows of the QK MMA (M); rows past kTcTile are read, never used
+constexpr int kBufs = 3;                      // tile buffers: copies run up to two tiles ahead of PV
+constexpr int kKBlocks = kTcTile / 32;        // 32-entry K blocks of PV per tile (one P block scale each)
 constexpr int kBlk = 5;                       // 128-byte column blocks per entry
-constexpr int kBlkBytes = kTcTile * 128;      // 16 KB: one column block of a tile
-constexpr int kTileBytes = kBlk * kBlkBytes;  // 80 KB
+constexpr int kBlkBytes = kTcTile * 128;      // 12 KB: one column block of a tile
+constexpr int kTileBytes = kBlk * kBlkBytes;  // 60 KB
 constexpr int kRopeBlk = 4;                   // block 4 = entry bytes 448..575 (bf16 RoPE)
 constexpr uint32_t kTmemCols = 256;
 // tensor-memory columns
@@ -65,10 +70,10 @@ constexpr int kSmBar = 1;                     // named barrier of the 8 softmax 
 constexpr int kReadyBar = 2;                  // warps 4-15: query and tensor memory ready (384 threads)
 constexpr int kScaleBar = 3;                  // warps 4-15: query scales ready (384 threads)
 constexpr int kCopyBar = 4;                   // warps 0-3: the copy warps (128 threads)
-constexpr int kPrefetchTiles = 4;             // contiguous tiles requested into L2 ahead of their copy
 
 struct TcAttnSmem {
-    uint8_t tile[2][kTileBytes];              // [block][entry][128 B], 128-byte swizzle
+    uint8_t tile[kBufs][kTileBytes];          // [block][entry][128 B], 128-byte swizzle
+    uint8_t tile_pad[(kTcRows - kTcTile) * 128];   // the QK rows read past the last block
     uint8_t qk[4][32 * 128];                  // QK B operand per nope block: rows 0..15 Qhi, 16..31 Qlo
     uint8_t qr[16 * 128];                     // RoPE query, bf16, 16 rows
     uint8_t p8[2][32 * 128];                  // PV B operand: rows 0..15 Phi, 16..31 Plo, K = 128 entries
@@ -78,7 +83,7 @@ struct TcAttnSmem {
     float tmax[4][kHeads];                    // tile maxima per lane quarter
     uint32_t sfb[2][4][kHeads];               // P block-scale bytes [buffer][32-entry block][head]
     float lred[4][kHeads];
-    uint64_t full[2], empty[2], sfull[2], sfree[2], pfull[2], pdone[2], drain;
+    uint64_t full[kBufs], empty[kBufs], sfull[2], sfree[2], pfull[2], pdone[2], drain;
     uint32_t tmem_base;
     int32_t fail, n_issued, n_landed;
 };
@@ -178,21 +183,24 @@ __device__ __forceinline__ void qprep_convert(TcAttnSmem& sm, const uint16_t* q,
 __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     const __grid_constant__ CUtensorMap kv_tile, const __grid_constant__ CUtensorMap kv_rows,
     const __grid_constant__ CUtensorMap win_rows, const __grid_constant__ CUtensorMap win_tile,
-    const uint8_t* __restrict__ comp_kv, const uint8_t* __restrict__ win_kv,
     const uint16_t* __restrict__ q, int64_t cap, int ratio,
-    const int32_t* __restrict__ topk, int k, int W, const int32_t* __restrict__ seq_len, float scale, int splits,
-    float* __restrict__ opart, float2* __restrict__ mlpart, int32_t* err) {
+    const int32_t* __restrict__ topk, int k, int W, int Wr, int Q, const int32_t* __restrict__ seq_len, float scale,
+    int splits, float* __restrict__ opart, float2* __restrict__ mlpart, int32_t* err) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     TcAttnSmem& sm = *reinterpret_cast<TcAttnSmem*>(smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.y, split = blockIdx.x;
-    const int B = gridDim.y;
+    // query row vq = cache row b times Q + the query's place jq among the Q newest tokens
+    const int vq = blockIdx.y, split = blockIdx.x;
+    const int b = vq / Q, jq = vq % Q;
+    const int B = gridDim.y / Q;
 
     // ---- setup --------------------------------------------------------------------------------
     if (tid == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kBufs; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.sfull[s], 1);
             mbar_init(&sm.sfree[s], 8);
             mbar_init(&sm.pfull[s], 8);
@@ -228,6 +236,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         if (tid == 0 && split == 0) dev_error(err, CSLD_DEVERR_SEQ_LEN);
         n = 0;
     }
+    n = max(0, n - (Q - 1 - jq));   // the tokens this query sees (itself included)
     const int64_t n_vis = min64(n / ratio, cap);
     const bool sparse = topk != nullptr;
     const int64_t n_comp = sparse ? (int64_t)k : n_vis;
@@ -237,16 +246,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     const int64_t n_tiles_all = (L + kTcTile - 1) / kTcTile;
     const int64_t t_begin = n_tiles_all * split / splits;
     const int n_tiles = static_cast<int>(n_tiles_all * (split + 1) / splits - t_begin);
-    const size_t part = (size_t)b * splits + split;
+    const size_t part = (size_t)vq * splits + split;
     // rows past the end of each map read as zeros
     const int32_t oob_kv = static_cast<int32_t>(min64((int64_t)B * cap, 0x7FFFFFFF));
-    const int32_t oob_win = static_cast<int32_t>(min64((int64_t)B * max(W, 1), 0x7FFFFFFF));
+    const int32_t oob_win = static_cast<int32_t>(min64((int64_t)B * max(Wr, 1), 0x7FFFFFFF));
     // compressed slot i -> row of the compressed map, or -1 for an empty slot
     auto comp_row = [&](int64_t i, bool report) -> int32_t {
         if (i >= n_comp) return -1;
         int64_t v = i;
         if (sparse) {
-            v = topk[(size_t)b * k + i];
+            v = topk[(size_t)vq * k + i];
             if (v >= n_vis) {
                 if (report) dev_error(err, CSLD_DEVERR_BAD_INDEX);
                 return -1;
@@ -262,27 +271,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     if (n_tiles <= 0) {
         if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
     } else if (warp < 4) {
-        // ===== copies (warps 0-3): tile t into buffer t & 1, started before the query is ready =====
-        // Contiguous tiles (dense mode) are also requested into L2 kPrefetchTiles ahead of their
-        // copy, so HBM keeps streaming while both tile buffers are busy; the copy of a tile then
-        // reads L2.  The window ring of the sequence is requested once.
-        auto prefetch_tile = [&](int tt) {
-            if (sparse || tt >= n_tiles) return;
-            const int64_t i0 = (t_begin + tt) * kTcTile;
-            if (i0 >= n_comp) return;
-            const int64_t rows = min64(kTcTile, n_comp - i0);
-            bulk_prefetch_l2(comp_kv + ((size_t)b * cap + (size_t)i0) * kEntry, static_cast<uint32_t>(rows * kEntry));
-        };
-        if (tid == 0) {
-            for (int tt = 0; tt < kPrefetchTiles; ++tt) prefetch_tile(tt);
-            if (n_win > 0 && (t_begin + n_tiles) * kTcTile > n_comp4)
-                bulk_prefetch_l2(win_kv + (size_t)b * W * kEntry, static_cast<uint32_t>(W * kEntry));
-        }
+        // ===== copies (warps 0-3): tile t into buffer t % kBufs, started before the query is ready =====
         int t = 0;
         for (; t < n_tiles; ++t) {
-            if (tid == 0) prefetch_tile(t + kPrefetchTiles);
-            const int s = t & 1;
-            const bool ok = !*fail && (t < 2 || mbar_wait(&sm.empty[s], ((t >> 1) - 1) & 1));
+            const int s = t % kBufs;
+            const bool ok = !*fail && (t < kBufs || mbar_wait(&sm.empty[s], ((t / kBufs) - 1) & 1));
             if (ok && tid == 0) mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
             if (named_barrier_or(kCopyBar, 128, !ok)) {   // the four copy warps leave together
                 if (tid == 0) *fail = 1;
@@ -295,17 +288,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                 if (tid < kBlk)
                     tma_load_2d(tl + tid * kBlkBytes, &kv_tile, tid < 4 ? 128 * tid : kNope,
                                 static_cast<int>((int64_t)b * cap + i0), &sm.full[s]);
-            } else if (W == kTcTile && n_win == W && i0 == n_comp4) {
+            } else if (W == kTcTile && Wr == W && n_win == W && i0 == n_comp4) {
                 // the tile is the whole window and the ring is full: its W slots hold exactly
                 // those tokens (in ring order, which the softmax does not care about), so the
                 // ring itself comes in one box per column block
                 if (tid < kBlk)
                     tma_load_2d(tl + tid * kBlkBytes, &win_tile, tid < 4 ? 128 * tid : kNope, b * W, &sm.full[s]);
             } else {
-                // thread t: slots 4g .. 4g+3 (g = t / 4) of column block t % 4 (and block 4 when
-                // t % 4 == 0), from one of the two maps
+                // thread t: slots 4g .. 4g+3 (g = t / 4 < kTcTile / 4) of column block t % 4 (and
+                // block 4 when t % 4 == 0), from one of the two maps
                 const int g = tid >> 2, j = tid & 3;
                 const int64_t ib = i0 + 4 * g;
+                if (4 * g < kTcTile) {
                 const bool win = ib >= n_comp4 && ib < L;
                 int32_t y[4];
 #pragma unroll
@@ -316,7 +310,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                         y[r] = row >= 0 ? row : oob_kv;
                     } else if (i < L) {
                         const int64_t tok = (int64_t)n - n_win + (i - n_comp4);
-                        y[r] = static_cast<int32_t>((int64_t)b * W + tok % W);
+                        y[r] = static_cast<int32_t>((int64_t)b * Wr + tok % Wr);
                     } else {
                         y[r] = oob_win;
                     }
@@ -325,13 +319,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                 tma_gather4(tl + j * kBlkBytes + 4 * g * 128, map, 128 * j, y[0], y[1], y[2], y[3], &sm.full[s]);
                 if (j == 0)
                     tma_gather4(tl + kRopeBlk * kBlkBytes + 4 * g * 128, map, kNope, y[0], y[1], y[2], y[3], &sm.full[s]);
+                }
             }
         }
         if (tid == 0) sm.n_issued = t;
     } else if (warp >= 4 && warp < 8) {
         // ===== the query operands (warps 4-15; the scales come from warps 8-15 first) ============
         named_barrier(kScaleBar, 384);
-        qprep_convert(sm, q, b, tid - 128);
+        qprep_convert(sm, q, vq, tid - 128);
         tc_fence_before();
         named_barrier(kReadyBar, 384);   // query operands written; tensor memory initialised
         tc_fence_after();
@@ -347,38 +342,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
             while (np < n_tiles) {
                 if (*fail) break;
                 if (np < nq && mbar_test_wait(&sm.pfull[np & 1], (np >> 1) & 1)) {
-                    const int su = np & 1;
+                    const int su = np & 1, sb = np % kBufs;   // P buffer, tile buffer
                     tc_fence_after();
-                    const uint64_t da = desc_sw128(sm.tile[su], 0);
+                    const uint64_t da = desc_sw128(sm.tile[sb], 0);
                     const uint64_t dp = desc_sw128(sm.p8[su], 0);
                     const uint32_t sfb0 = tmem + kColSFB + 4u * su;
 #pragma unroll
                     for (int mb = 0; mb < 4; ++mb)
 #pragma unroll
-                        for (int kb = 0; kb < 4; ++kb)   // 32 entries (4 row groups) per MMA
+                        for (int kb = 0; kb < kKBlocks; ++kb)   // 32 entries (4 row groups) per MMA
                             umma_mxf8f6f4(tmem + kColO + 32u * mb, da + (mb * kBlkBytes + kb * 4096) / 16,
                                           dp + (32 * kb) / 16, idesc_mxe4m3_m128(32, true, false, kb), tmem + kColSFA,
                                           sfb0 | (static_cast<uint32_t>(kb) << 30), 1u);
-                    // RoPE: M = 128 with LBO 16 KB (rows 64..127 read the next 16 KB: unused)
-                    const uint64_t dar = desc_sw128(sm.tile[su] + kRopeBlk * kBlkBytes, kBlkBytes);
+                    // RoPE: M = 128 with LBO one block (rows 64..127 read the next block: unused)
+                    const uint64_t dar = desc_sw128(sm.tile[sb] + kRopeBlk * kBlkBytes, kBlkBytes);
                     const uint64_t dpb = desc_sw128(sm.pbf[su][0], 0);
 #pragma unroll
                     for (int ks = 0; ks < kTcTile / 16; ++ks)
                         umma_f16(tmem + kColOR, dar + (ks * 2048) / 16, dpb + ((ks >> 2) * 2048 + 32 * (ks & 3)) / 16,
                                  kIdPVr, 1u);
-                    umma_commit(&sm.empty[su]);
+                    umma_commit(&sm.empty[sb]);
                     umma_commit(&sm.pdone[su]);
                     ++np;
                     idle = 0;
                     continue;
                 }
-                if (nq < n_tiles && nq < np + 2 && mbar_test_wait(&sm.full[nq & 1], (nq >> 1) & 1) &&
+                if (nq < n_tiles && nq < np + 2 && mbar_test_wait(&sm.full[nq % kBufs], (nq / kBufs) & 1) &&
                     (nq < 2 || mbar_test_wait(&sm.sfree[nq & 1], ((nq >> 1) - 1) & 1))) {
-                    const int s = nq & 1;
+                    const int s = nq & 1;   // S slot
                     landed = nq + 1;
                     tc_fence_after();
                     const uint32_t dS = tmem + kColS + 32u * s;
-                    const uint64_t da = desc_sw128(sm.tile[s], 0);
+                    const uint64_t da = desc_sw128(sm.tile[nq % kBufs], 0);
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
@@ -406,14 +401,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         // ===== online softmax: thread = entry e = TMEM lane; head group hg = 8 heads =============
         const int sub = warp & 3, hg = (warp - 8) >> 2, e = 32 * sub + lane;
         const uint32_t lb = tmem + ((32u * sub) << 16);
-        qprep_scale(sm, q, b, tid - 256, scale);
+        qprep_scale(sm, q, vq, tid - 256, scale);
         if (hg == 0) {   // O = 0 and unit scale factors of V for this lane quarter
             for (uint32_t c = kColO; c < kColSFA; c += 8) tmem_st_32x32b_x8_fill(lb + c, 0u);
             tmem_st_32x32b_x8_fill(lb + kColSFA, 0x7F7F7F7Fu);
             tmem_st_wait();
         }
         named_barrier(kScaleBar, 384);
-        qprep_convert(sm, q, b, tid - 128);
+        qprep_convert(sm, q, vq, tid - 128);
         tc_fence_before();
         named_barrier(kReadyBar, 384);
         tc_fence_after();
@@ -428,7 +423,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         for (int t = 0; t < n_tiles; ++t) {
             const int s = t & 1;
             const int64_t i = (t_begin + t) * kTcTile + e;
-            const bool valid = i < n_comp4 ? comp_row(i, false) >= 0 : i < L;
+            const bool valid = e < kTcTile && (i < n_comp4 ? comp_row(i, false) >= 0 : i < L);
             ok = !*fail && mbar_wait(&sm.sfull[s], (t >> 1) & 1);
             if (named_barrier_or(kSmBar, 256, !ok)) {   // the softmax warps leave together
                 ok = false;
@@ -575,7 +570,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         // publish nothing
         if (warp == 4 && lane == 0) {
             dev_error(err, CSLD_DEVERR_TIMEOUT);
-            for (int t = sm.n_landed; t < sm.n_issued; ++t) (void)mbar_wait(&sm.full[t & 1], (t >> 1) & 1);
+            for (int t = sm.n_landed; t < sm.n_issued; ++t) (void)mbar_wait(&sm.full[t % kBufs], (t / kBufs) & 1);
             umma_commit(&sm.drain);
             (void)mbar_wait(&sm.drain, 0);
         }
@@ -592,11 +587,12 @@ size_t attention_tc_smem_bytes() { return sizeof(TcAttnSmem) + 1024; }
 int attention_tc_tile() { return kTcTile; }
 
 cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
-                                        const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                                        const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                                         const int32_t* seq_len, int B, float scale, int splits, float* opart,
                                         float2* mlpart, int32_t* err, cudaStream_t stream) {
     // the caches as 2-D byte tensors [rows][576]: 128-byte boxes with the 128-byte swizzle, 128
-    // rows tall (box copies of contiguous tiles) or one row (the gather4 form)
+    // rows tall (box copies of contiguous tiles) or one row (the gather4 form).  B cache rows,
+    // each serving Q query rows; the window ring has Wr >= W slots per cache row.
     CUtensorMap kv_tile, kv_rows, win_rows, win_tile;
     const uint64_t rows = (uint64_t)B * (uint64_t)cap;
     if (!make_tensor_map_2d_u8(&kv_tile, comp_kv, kEntry, rows, 128, kTcTile) ||
@@ -604,19 +600,19 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
         return cudaErrorInvalidValue;
     // a window-less call still passes a valid map (the compressed cache; never read)
     const bool has_win = W > 0 && win_kv != nullptr;
-    if (!make_tensor_map_2d_u8(&win_rows, has_win ? win_kv : comp_kv, kEntry, has_win ? (uint64_t)B * W : rows, 128, 1))
+    if (!make_tensor_map_2d_u8(&win_rows, has_win ? win_kv : comp_kv, kEntry, has_win ? (uint64_t)B * Wr : rows, 128, 1))
         return cudaErrorInvalidValue;
-    // a full ring of kTcTile slots as one tile (only used when W == kTcTile)
-    const bool win_box = has_win && W == kTcTile;
+    // a full ring of kTcTile slots as one tile (only used when W == Wr == kTcTile)
+    const bool win_box = has_win && W == kTcTile && Wr == W;
     if (!make_tensor_map_2d_u8(&win_tile, win_box ? win_kv : comp_kv, kEntry, win_box ? (uint64_t)B * W : rows, 128,
                                win_box ? kTcTile : 1))
         return cudaErrorInvalidValue;
     const size_t smem = attention_tc_smem_bytes();
     cudaError_t e = set_smem_once(attention_tc_partial_kernel, smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attention_tc_partial_kernel, dim3(splits, B), dim3(kTcThreads), smem, stream, kv_tile, kv_rows,
-                   win_rows, win_tile, comp_kv, has_win ? win_kv : comp_kv, q, cap, ratio, topk, k, W, seq_len, scale,
-                   splits, opart, mlpart, err);
+    e = launch_pdl(attention_tc_partial_kernel, dim3(splits, B * Q), dim3(kTcThreads), smem, stream, kv_tile, kv_rows,
+                   win_rows, win_tile, q, cap, ratio, topk, k, W, Wr, Q, seq_len,
+                   scale, splits, opart, mlpart, err);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

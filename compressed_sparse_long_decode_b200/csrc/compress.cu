@@ -165,6 +165,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
 // ------------------------------------------------------------------------------------------
 constexpr int kCTile = 128;                // entries per tile = the MMA's M
 constexpr int kCThreads = 512;
+constexpr int kRif = 2;                    // rows (entries) a warp has loaded at once
 constexpr uint32_t kCTmemCols = 64;        // U: 128 lanes x 64 fp32 columns
 constexpr uint32_t kIdProj = idesc_bf16_m128(kIdxDim, false, false);
 
@@ -248,20 +249,20 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
         const float* gb = gate + (size_t)b * T;
         uint8_t* kvb = kv_out + (size_t)b * out_seq_stride * kEntry;
 
-        // ---- 1) pooling: rows warp, warp + 16, ...; two rows at a time -------------------
-        for (int r0 = warp; r0 < kCTile; r0 += 2 * kWarps) {
+        // ---- 1) pooling: rows warp, warp + 16, ...; kRif rows at a time ------------------
+        for (int r0 = warp; r0 < kCTile; r0 += kRif * kWarps) {
             // entries go to the cache as soon as they are pooled; their bf16 copies wait in
             // registers for the shared-memory operand to be free
-            uint32_t packed[2][8];
+            uint32_t packed[kRif][8];
             if constexpr (kM4) {
-                uint4 x[2][8];
+                uint4 x[kRif][8];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < kRif; ++h) {
                     const int r = r0 + h * kWarps;
                     if (r < n_here) load_block4(rb + (size_t)(s0 + r) * 4 * kDim, lane, x[h]);
                 }
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < kRif; ++h) {
                     const int r = r0 + h * kWarps;
                     float c[16];
                     if (r < n_here) {
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                 }
             } else {
 #pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < kRif; ++h) {
                     const int r = r0 + h * kWarps;
                     float c[16];
                     if (r < n_here) {
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                 mma_pending = false;
             }
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < kRif; ++h) {
                 const int r = r0 + h * kWarps;
                 // lane l holds dims 16l..16l+15: column block l / 4, bytes 32 (l % 4) .. +31
                 uint8_t* blk = sm.a[lane >> 2];

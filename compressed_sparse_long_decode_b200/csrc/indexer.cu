@@ -45,6 +45,7 @@
 // (score desc, index asc), because every global top-k entry is in its part's top k.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "csld_internal.cuh"
@@ -59,7 +60,6 @@ constexpr int kIdxTile = 256;          // entries per pipeline stage: two 128-ro
 constexpr int kIdxStages = 4;          // ring depth of the merge-tree kernel (shares the candidate area)
 constexpr int kCoopStages = 12;        // ring depth of the cooperative kernel (one CTA per SM)
 constexpr int kCoopGroup = 4;          // tiles per key copy in the cooperative kernel (32 KB of codes)
-constexpr int kIdxPrefetchGroups = 4;  // copy groups requested into L2 beyond the ring
 constexpr int kMaxStages = 12;
 constexpr int kIdxEpiGroups = 3;       // epilogue warpgroups: warps 0..11
 constexpr int kIdxProducerWarp = 12;   // issues the tensor / bulk copies
@@ -504,21 +504,10 @@ __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], flo
     if (warp == kIdxProducerWarp) {
         // --- producer: GT tiles of key codes + their scales per copy group ----------------
         if (lane == 0) {
-            // copy groups beyond the ring's reach are requested into L2 kIdxPrefetchGroups ahead,
-            // so the key stream keeps more bytes in flight than the ring holds
-            auto prefetch_group = [&](int gg) {
-                const int tg = gg * GT;
-                if (tg >= n_tiles) return;
-                const int ne = min(GT * kIdxTile, cn - tg * kIdxTile);
-                bulk_prefetch_l2(cbase + (size_t)tg * kIdxTile * kIkey, static_cast<uint32_t>(ne) * kIkey);
-                bulk_prefetch_l2(sbase + (size_t)tg * kIdxTile * 2, static_cast<uint32_t>((ne + 1) & ~1) * 8u);
-            };
-            for (int gg = kGroups; gg < kGroups + kIdxPrefetchGroups; ++gg) prefetch_group(gg);
             int t = 0;
             for (int g = 0; t < n_tiles; ++g) {
                 const int s0 = (g % kGroups) * GT;
                 if (*fail) break;
-                prefetch_group(g + kGroups + kIdxPrefetchGroups);
                 bool free = true;   // the group's stages held tiles t - S .. t - S + GT - 1
                 if (g >= kGroups)
                     for (int i = 0; i < GT && free; ++i)
@@ -983,7 +972,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     const uint8_t* __restrict__ ikeys, const float* __restrict__ iscales, int64_t cap,
     const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
     const float* __restrict__ head_w, int chunk, int units, int k, CoopWs ws,
-    int32_t* __restrict__ topk_out, int32_t* err) {
+    int32_t* __restrict__ topk_out, int32_t* err, uint32_t barrier_extra) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     CoopSmem& sm = *reinterpret_cast<CoopSmem*>(
         smem_raw + ((kIdxSmemAlign - (smem_u32(smem_raw) & (kIdxSmemAlign - 1))) & (kIdxSmemAlign - 1)));
@@ -1067,7 +1056,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             const uint32_t c = sm.hist[i];
             if (c) atomicAdd(g1 + i, c);
         }
-    if (!seq_barrier(bar, 1 * nu, &sm.fail, err)) return;
+    if (!seq_barrier(bar, 1 * nu + barrier_extra, &sm.fail, err)) return;
     uint32_t beta1, need1, cnt1;
     find_bin_global(g1, kBins, want, sm.red, sm.sel, &beta1, &need1, &cnt1);
     // --- candidates: one pass over the range.  Each warp counts its keys above bin beta1 and
@@ -1178,7 +1167,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             const uint32_t c = sm.hist2[i];
             if (c) atomicAdd(g2 + i, c);
         }
-        if (!seq_barrier(bar, 2 * nu, &sm.fail, err)) return;
+        if (!seq_barrier(bar, 2 * nu + barrier_extra, &sm.fail, err)) return;
         uint32_t beta2, need2;
         find_bin_global(g2, kBins, need1, sm.red, sm.sel, &beta2, &need2);
         const uint32_t top22 = (beta1 << 11) | beta2;
@@ -1199,7 +1188,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             const uint32_t c = sm.hist3[i];
             if (c) atomicAdd(g3 + i, c);
         }
-        if (!seq_barrier(bar, 3 * nu, &sm.fail, err)) return;
+        if (!seq_barrier(bar, 3 * nu + barrier_extra, &sm.fail, err)) return;
         uint32_t beta3;
         find_bin_global(g3, 1024, need2, sm.red, sm.sel, &beta3, &take_eq);
         thr = (top22 << 10) | beta3;
@@ -1219,7 +1208,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             cnt[2 * u] = tot >> 16;
             cnt[2 * u + 1] = tot & 0xFFFFu;
         }
-        if (!seq_barrier(bar, 4 * nu, &sm.fail, err)) return;
+        if (!seq_barrier(bar, 4 * nu + barrier_extra, &sm.fail, err)) return;
         uint32_t a_loc = 0u, e_loc = 0u;
         for (int v = tid; v < u; v += blockDim.x) {
             a_loc += __ldcg(cnt + 2 * v);
@@ -1262,6 +1251,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     // --- this call is over for the sequence: the next one takes the other state set ------------
     if (u == 0 && tid == 0) atomicAdd(sq + 4, 1u);
 }
+
+// Test hook (csld_test_set_barrier_extra): arrivals added to every cross-CTA barrier target of
+// the cooperative kernel, so that a test can make its bounded waits run out.  0 in normal use.
+std::atomic<int> g_test_barrier_extra{0};
 
 // Resident CTAs of the cooperative kernel on the current device (0 if it cannot run), found
 // once per device.
@@ -1394,7 +1387,8 @@ cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t c
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, indexer_topk_coop_kernel, ikeys, iscales, cap, seq_len, ratio, q_idx, head_w,
-                               plan.chunk, plan.n_chunks, k, cws, topk_out, err);
+                               plan.chunk, plan.n_chunks, k, cws, topk_out, err,
+                               static_cast<uint32_t>(g_test_barrier_extra.load()));
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }

@@ -15,14 +15,16 @@
 //    copy warp streams the key codes and scales with 1-D bulk copies, eight tiles (32 KB + 8 KB)
 //    per copy, three copies in flight; one thread issues one tcgen05.mma kind::mxf4 per tile
 //    (M = 128 entries, N = 8 Q rows of the query operand: row 8q + 4g + h holds group g of head
-//    h of query q, the other group zero, so each output column is one exact group dot); warps
-//    0-3 read the dots back (thread = entry), form every query's fp32 score and write its
-//    order key to the workspace, and add the keys' top 11 bits to per-query histograms, which
-//    the CTA adds into global ones at the end.
+//    h of query q, the other group zero, so each output column is one exact group dot) into one
+//    of six accumulator slots; three warpgroups take the tiles in turn, read the dots back
+//    (thread = entry), form every query's fp32 score and write its order key to the workspace,
+//    and add the keys' top 11 bits to per-query histograms, which the CTA adds into global ones
+//    at the end.
 // 2. indexer_multi_select_kernel -- one CTA per (sequence, query): the threshold bin from the
-//    global histogram, two more radix levels (11 + 10 bits) over that query's keys, then the
-//    entries in index order: every key above the threshold and the first ones equal to it.
-//    It zeroes the histogram it used, so the workspace stays ready for the next call.
+//    global histogram, the keys of that bin and above gathered into shared memory in index
+//    order by one pass, two more radix levels (11 + 10 bits) there, then the entries in index
+//    order: every key above the threshold and the first ones equal to it.  It zeroes the
+//    histogram it used, so the workspace stays ready for the next call.
 #include "csld_internal.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -31,15 +33,17 @@ namespace csld {
 
 namespace {
 
-constexpr int kMqThreads = 256;          // warps 0-3 epilogue, warp 4 copies, warp 5 MMA
+constexpr int kMqThreads = 512;          // warps 0-11 epilogue (3 warpgroups), warp 12 copies, warp 13 MMA
 constexpr int kMqTile = 128;             // entries per MMA (M)
 constexpr int kMqGroupTiles = 8;         // tiles per bulk copy
 constexpr int kMqGroup = kMqTile * kMqGroupTiles;   // 1024 entries per copy group
 constexpr int kMqStages = 3;             // copy groups in flight
 constexpr int kMqBins = 2048;            // histogram of the keys' top 11 bits
-constexpr uint32_t kMqTmemCols = 256;    // two accumulator slots of 8 Q <= 64 columns, scale factors at 128
-constexpr uint32_t kMqSfCol = 128;
-constexpr int kMqCopyWarp = 4, kMqMmaWarp = 5;
+constexpr int kMqEpi = 3;                // epilogue warpgroups: tile t goes to warpgroup t % 3
+constexpr int kMqSlots = 6;              // accumulator slots (tile t uses slot t % 6), 64 columns each
+constexpr uint32_t kMqTmemCols = 512;    // 6 x 64 columns (8 Q <= 64), scale factors at 384
+constexpr uint32_t kMqSfCol = 384;
+constexpr int kMqCopyWarp = 12, kMqMmaWarp = 13;
 
 struct MqSmem {
     uint8_t codes[kMqStages][kMqGroup * kIkey];     // 32 KB per group, stored (pre-swizzled) layout
@@ -47,7 +51,7 @@ struct MqSmem {
     alignas(256) uint8_t bq[8 * CSLD_MULTI_MAX_Q * kIkey];   // query operand, 32-byte swizzle
     float qscale[CSLD_MULTI_MAX_Q][8];              // [q][group * 4 + head]
     uint32_t hist[CSLD_MULTI_MAX_Q][kMqBins];
-    uint64_t full[kMqStages], gfree[kMqStages], accf[2], sfree[2], drain;
+    uint64_t full[kMqStages], gfree[kMqStages], accf[kMqSlots], sfree[kMqSlots], drain;
     uint32_t tmem_base;
     int32_t fail, n_mma;
 };
@@ -67,11 +71,11 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
     if (tid == 0) {
         for (int s = 0; s < kMqStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.gfree[s], 4);
+            mbar_init(&sm.gfree[s], 4 * kMqEpi);   // every epilogue warp, once per copy group
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kMqSlots; ++s) {
             mbar_init(&sm.accf[s], 1);
-            mbar_init(&sm.sfree[s], 4);
+            mbar_init(&sm.sfree[s], 4);            // the 4 warps of the slot's warpgroup
         }
         mbar_init(&sm.drain, 1);
         sm.fail = 0;
@@ -132,7 +136,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
         tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kMqSfCol + 8, 0x7F7F7F7Fu);
         tmem_st_wait();
     }
-    if (warp < 4 || warp == kMqMmaWarp) {   // query operand and scale factors ready (warps 0-3, 5)
+    if (warp < 4 || warp == kMqMmaWarp) {   // query operand and scale factors ready (warps 0-3 and the MMA warp)
         tc_fence_before();
         named_barrier(1, 5 * 32);
         tc_fence_after();
@@ -171,8 +175,8 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
                 const int g = c + i * chunks;
                 const int nt = min(kMqGroupTiles, n_tiles_all - g * kMqGroupTiles);
                 for (int tt = 0; tt < nt; ++tt, ++t) {
-                    const int slot = t & 1;
-                    if (t >= 2 && !mbar_wait(&sm.sfree[slot], ((t >> 1) - 1) & 1)) {
+                    const int slot = t % kMqSlots;
+                    if (t >= kMqSlots && !mbar_wait(&sm.sfree[slot], ((t / kMqSlots) - 1) & 1)) {
                         *fail = 1;
                         break;
                     }
@@ -185,10 +189,11 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
             }
             sm.n_mma = t;
         }
-    } else if (warp < 4) {
-        // ---- epilogue: thread = entry m of the tile -------------------------------------------
-        const int m = 32 * warp + lane;
-        const uint32_t lane_addr = tmem + ((32u * warp) << 16);
+    } else if (warp < 4 * kMqEpi) {
+        // ---- epilogue: warpgroup wg takes tiles wg, wg + 3, ...; thread = entry m of the tile ---
+        const int wg = warp >> 2, quad = warp & 3;
+        const int m = 32 * quad + lane;
+        const uint32_t lane_addr = tmem + ((32u * quad) << 16);
         const float* hw = head_w + (size_t)b * Q * kIdxHeads;
         int t = 0;
         for (int i = 0; i < my_groups; ++i) {
@@ -197,8 +202,9 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
             const int nt = min(kMqGroupTiles, n_tiles_all - g * kMqGroupTiles);
             bool ok = true;
             for (int tt = 0; tt < nt; ++tt, ++t) {
-                const int slot = t & 1;
-                ok = !*fail && mbar_wait(&sm.accf[slot], (t >> 1) & 1);
+                if (t % kMqEpi != wg) continue;
+                const int slot = t % kMqSlots;
+                ok = !*fail && mbar_wait(&sm.accf[slot], (t / kMqSlots) & 1);
                 if (!__all_sync(0xffffffffu, ok)) {
                     if (lane == 0) *fail = 1;
                     ok = false;
@@ -341,14 +347,34 @@ __device__ __forceinline__ uint32_t mq_block_scan(uint32_t v, uint32_t* red, uin
 
 }  // namespace
 
-// Grid (Q, B), 1024 threads: the exact top-k of query q of sequence b.
-__global__ void __launch_bounds__(1024) indexer_multi_select_kernel(const uint32_t* __restrict__ keys, int64_t cap,
-                                                                    const int32_t* __restrict__ seq_len, int ratio,
-                                                                    int Q, int k, uint32_t* __restrict__ ghist,
-                                                                    int32_t* __restrict__ topk_out) {
-    __shared__ uint32_t h[kMqBins];
-    __shared__ uint32_t sel[4];
-    __shared__ uint32_t red[96];
+// Grid (Q, B), 1024 threads: the exact top-k of query q of sequence b.  The keys of the
+// threshold bin (found from the scoring histogram) and above are gathered into shared memory
+// in index order by one pass over the query's keys (sixteen per thread at a time, 16-byte
+// loads); the last two radix levels and the emission then run in shared memory.  When they do
+// not fit (more than kMqCand keys: heavy ties), the levels and the emission read the keys from
+// global memory instead.
+constexpr int kMqSelThreads = 1024;
+constexpr int kMqPer = 16;                       // keys per thread per pass step
+constexpr int kMqCand = 20480;                   // candidates kept in shared memory
+struct MqSelSmem {
+    uint32_t ckey[kMqCand];
+    uint32_t cidx[kMqCand];
+    uint32_t h[kMqBins];
+    uint32_t sel[4];
+    uint32_t red[96];
+};
+
+__global__ void __launch_bounds__(kMqSelThreads) indexer_multi_select_kernel(const uint32_t* __restrict__ keys,
+                                                                             int64_t cap,
+                                                                             const int32_t* __restrict__ seq_len,
+                                                                             int ratio, int Q, int k,
+                                                                             uint32_t* __restrict__ ghist,
+                                                                             int32_t* __restrict__ topk_out) {
+    extern __shared__ __align__(16) uint8_t sel_raw[];
+    MqSelSmem& sm = *reinterpret_cast<MqSelSmem*>(sel_raw);
+    uint32_t* h = sm.h;
+    uint32_t* sel = sm.sel;
+    uint32_t* red = sm.red;
     const int q = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     pdl_wait();
     pdl_trigger();
@@ -363,7 +389,6 @@ __global__ void __launch_bounds__(1024) indexer_multi_select_kernel(const uint32
         h[i] = gh[i];
         gh[i] = 0u;    // ready for the next call
     }
-    if (tid < 4) sel[tid] = 0u;
     __syncthreads();
     if (n_q <= k) {
         for (int64_t i = tid; i < k; i += blockDim.x) out[i] = i < n_q ? static_cast<int32_t>(i) : -1;
@@ -372,42 +397,101 @@ __global__ void __launch_bounds__(1024) indexer_multi_select_kernel(const uint32
     // level 1 (bits 31..21) from the scoring histogram
     mq_find_bin(h, kMqBins, static_cast<uint32_t>(k), sel);
     const uint32_t b1 = sel[0], need1 = sel[1];
+    const uint32_t above1 = static_cast<uint32_t>(k) - need1;   // keys above bin b1
+    const uint32_t in1 = h[b1];                                  // keys in it
     __syncthreads();
-    // level 2 (bits 20..10) among the keys of bin b1
+    const bool in_smem = above1 + in1 <= static_cast<uint32_t>(kMqCand);
+    // ---- gather the keys of bin >= b1 in index order (when they fit) ------------------------
+    const uint32_t lo1 = b1 << 21;
+    uint32_t n_c = 0u;
+    if (in_smem) {
+        // n_q keys: thread t reads keys base + 16 t .. base + 16 t + 15 (four 16-byte loads when
+        // the row start allows it)
+        const bool vec = ((reinterpret_cast<uintptr_t>(kq) & 15u) == 0);
+        for (int64_t base = 0; base < n_q; base += (int64_t)kMqSelThreads * kMqPer) {
+            const int64_t i0 = base + (int64_t)tid * kMqPer;
+            uint32_t v[kMqPer];
+            if (vec && i0 + kMqPer <= n_q) {
+#pragma unroll
+                for (int j = 0; j < kMqPer / 4; ++j) {
+                    const uint4 x = __ldcg(reinterpret_cast<const uint4*>(kq + i0) + j);
+                    v[4 * j] = x.x;
+                    v[4 * j + 1] = x.y;
+                    v[4 * j + 2] = x.z;
+                    v[4 * j + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < kMqPer; ++j) v[j] = i0 + j < n_q ? __ldcg(kq + i0 + j) : 0u;
+            }
+            uint32_t cnt = 0u;
+#pragma unroll
+            for (int j = 0; j < kMqPer; ++j) cnt += (i0 + j < n_q && v[j] >= lo1) ? 1u : 0u;
+            uint32_t tot;
+            uint32_t at = n_c + mq_block_scan(cnt, red, &tot);
+#pragma unroll
+            for (int j = 0; j < kMqPer; ++j)
+                if (i0 + j < n_q && v[j] >= lo1) {
+                    if (at < static_cast<uint32_t>(kMqCand)) {   // holds whenever the histogram is exact
+                        sm.ckey[at] = v[j];
+                        sm.cidx[at] = static_cast<uint32_t>(i0 + j);
+                    }
+                    ++at;
+                }
+            n_c += tot;
+        }
+        n_c = min(n_c, static_cast<uint32_t>(kMqCand));
+        __syncthreads();
+    }
+    // ---- levels 2 (bits 20..10) and 3 (bits 9..0) inside bin b1 --------------------------------
     for (int i = tid; i < kMqBins; i += blockDim.x) h[i] = 0u;
     __syncthreads();
-    for (int64_t i = tid; i < n_q; i += blockDim.x) {
-        const uint32_t key = kq[i];
-        if ((key >> 21) == b1) atomicAdd(&h[(key >> 10) & 2047u], 1u);
+    if (in_smem) {
+        for (uint32_t i = tid; i < n_c; i += blockDim.x)
+            if ((sm.ckey[i] >> 21) == b1) atomicAdd(&h[(sm.ckey[i] >> 10) & 2047u], 1u);
+    } else {
+        for (int64_t i = tid; i < n_q; i += blockDim.x) {
+            const uint32_t key = __ldcg(kq + i);
+            if ((key >> 21) == b1) atomicAdd(&h[(key >> 10) & 2047u], 1u);
+        }
     }
     __syncthreads();
     mq_find_bin(h, kMqBins, need1, sel);
     const uint32_t b2 = sel[0], need2 = sel[1];
     __syncthreads();
-    // level 3 (bits 9..0) among the keys with those top 22 bits
     for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
     __syncthreads();
     const uint32_t top22 = (b1 << 11) | b2;
-    for (int64_t i = tid; i < n_q; i += blockDim.x) {
-        const uint32_t key = kq[i];
-        if ((key >> 10) == top22) atomicAdd(&h[key & 1023u], 1u);
+    if (in_smem) {
+        for (uint32_t i = tid; i < n_c; i += blockDim.x)
+            if ((sm.ckey[i] >> 10) == top22) atomicAdd(&h[sm.ckey[i] & 1023u], 1u);
+    } else {
+        for (int64_t i = tid; i < n_q; i += blockDim.x) {
+            const uint32_t key = __ldcg(kq + i);
+            if ((key >> 10) == top22) atomicAdd(&h[key & 1023u], 1u);
+        }
     }
     __syncthreads();
     mq_find_bin(h, 1024, need2, sel);
     const uint32_t thr = (top22 << 10) | sel[0], take_eq = sel[1];
     __syncthreads();
-    // emit in index order: keys above the threshold, and the first take_eq keys equal to it
+    // ---- emit in index order: keys above the threshold, and the first take_eq equal to it -----
+    const int64_t n_e = in_smem ? (int64_t)n_c : n_q;
     uint32_t base_sel = 0u, base_eq = 0u;
-    for (int64_t i0 = 0; i0 < n_q; i0 += blockDim.x) {
+    for (int64_t i0 = 0; i0 < n_e; i0 += blockDim.x) {
         const int64_t i = i0 + tid;
-        const uint32_t key = i < n_q ? kq[i] : 0u;
-        const uint32_t eq = (i < n_q && key == thr) ? 1u : 0u;
+        uint32_t key = 0u, idx = 0u;
+        if (i < n_e) {
+            key = in_smem ? sm.ckey[i] : __ldcg(kq + i);
+            idx = in_smem ? sm.cidx[i] : static_cast<uint32_t>(i);
+        }
+        const uint32_t eq = (i < n_e && key == thr) ? 1u : 0u;
         uint32_t eq_tot;
         const uint32_t eq_before = base_eq + mq_block_scan(eq, red, &eq_tot);
-        const uint32_t take = (i < n_q && key > thr) || (eq && eq_before < take_eq) ? 1u : 0u;
+        const uint32_t take = (i < n_e && key > thr) || (eq && eq_before < take_eq) ? 1u : 0u;
         uint32_t take_tot;
         const uint32_t at = base_sel + mq_block_scan(take, red, &take_tot);
-        if (take && at < static_cast<uint32_t>(k)) out[at] = static_cast<int32_t>(i);
+        if (take && at < static_cast<uint32_t>(k)) out[at] = static_cast<int32_t>(idx);
         base_sel += take_tot;
         base_eq += eq_tot;
         if (base_sel >= static_cast<uint32_t>(k)) break;   // uniform: every thread sees the same totals
@@ -437,8 +521,10 @@ cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int
     e = launch_pdl(indexer_multi_score_kernel, dim3(static_cast<unsigned>(chunks), B), dim3(kMqThreads), smem, stream,
                    ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, Q, keys, ghist, err);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(indexer_multi_select_kernel, dim3(Q, B), dim3(1024), 0, stream, static_cast<const uint32_t*>(keys),
-                   cap, seq_len, ratio, Q, k, ghist, topk_out);
+    e = set_smem_once(indexer_multi_select_kernel, sizeof(MqSelSmem));
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(indexer_multi_select_kernel, dim3(Q, B), dim3(kMqSelThreads), sizeof(MqSelSmem), stream,
+                   static_cast<const uint32_t*>(keys), cap, seq_len, ratio, Q, k, ghist, topk_out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -1,6 +1,8 @@
 // Launchers of the libcsld kernels (host side, internal).
 #pragma once
 #include <cuda_runtime.h>
+
+#include <atomic>
 #include <stdint.h>
 
 #include "csld.h"
@@ -36,14 +38,19 @@ cudaError_t launch_indexer(const uint8_t* ikeys, const float* iscales, int64_t c
                            const float* head_w, int B, int k, int32_t* topk_out, void* ws,
                            const IndexerPlan& plan, int32_t* err, cudaStream_t stream);
 
+// Test hook of the cooperative indexer (see csld_test_set_barrier_extra).
+extern std::atomic<int> g_test_barrier_extra;
+
 // Hybrid decode attention.
 struct AttentionPlan {
     int splits;         // CTAs per sequence
     size_t ws_bytes;
 };
 AttentionPlan attention_plan(int B, int64_t cap, int k, bool sparse, int W, int num_sms);
+// B cache rows with Q query rows each (query j of row b sees the first seq_len[b] - Q + 1 + j
+// tokens); the window ring has Wr >= W slots per cache row.  The plan counts B * Q rows.
 cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
-                             const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                             const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                              const int32_t* seq_len, int B, float scale, float* out,
                              float* lse_out, void* ws, const AttentionPlan& plan, int32_t* err,
                              cudaStream_t stream);
@@ -55,7 +62,7 @@ cudaError_t attention_static_scratch(void** ptr);
 int attention_tc_tile();
 size_t attention_tc_smem_bytes();
 cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
-                                        const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                                        const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                                         const int32_t* seq_len, int B, float scale, int splits, float* opart,
                                         float2* mlpart, int32_t* err, cudaStream_t stream);
 

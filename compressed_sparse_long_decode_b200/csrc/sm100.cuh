@@ -104,12 +104,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                  :: "r"(smem_u32(bar)) : "memory");
 }
 
-// Hint: bring `bytes` (a multiple of 16) of global memory at p (16-byte aligned) into L2.  The
-// request is fire-and-forget; no smem, barrier or completion is involved.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
-}
-
 // ---- tensor maps -------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");

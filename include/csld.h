@@ -239,6 +239,29 @@ CSLD_API csld_status hybrid_decode_attention(const uint16_t* q, int heads, const
                                     size_t ws_bytes, int32_t* err, void* stream);
 
 /* ----------------------------------------------------------------------------------------
+ * Multi-query decode attention ([HF] layer-pattern paragraph: the multi-token-prediction block
+ * runs several query tokens per step; CSA / HCA paragraphs as above).  Q query tokens per
+ * sequence -- the Q newest: query j of sequence b stands at raw position seq_len[b] - Q + j --
+ * share one launch over the cache; query j sees the first seq_len[b] - Q + 1 + j tokens: the
+ * compressed entries they complete (dense mode) or its own top-k row (sparse mode), and the W
+ * newest of them through the window ring.  Each (b, j) gets exactly what hybrid_decode_attention
+ * gives that query alone.
+ *   q [B][Q][heads][512] bf16, topk [B][Q][k] i32 or NULL, out [B][Q][heads][512] f32,
+ *   lse_out [B][Q][heads] f32 or NULL; the window ring win_kv [B][W_ring][576] holds token t at
+ *   slot t mod W_ring, W_ring >= W + Q - 1 (so the oldest query's window is still in it: a
+ *   layer cache whose window is W_ring, fed by kv_cache_append, keeps it that way).
+ *   1 <= Q <= CSLD_MULTI_MAX_Q, B * Q <= 65535.
+ * Workspace: csld_attention_workspace_size(B * Q, heads, cap, k, W).  Other rules as for
+ * hybrid_decode_attention.
+ * -------------------------------------------------------------------------------------- */
+CSLD_API csld_status hybrid_decode_attention_multi(const uint16_t* q, int heads, const uint8_t* comp_kv,
+                                                   int64_t cap, int ratio, const int32_t* topk, int k,
+                                                   const uint8_t* win_kv, int W_ring, int W,
+                                                   const int32_t* seq_len, int B, int Q, float scale,
+                                                   float* out, float* lse_out, void* ws,
+                                                   size_t ws_bytes, int32_t* err, void* stream);
+
+/* ----------------------------------------------------------------------------------------
  * hybrid_decode_attention_static -- the same computation as hybrid_decode_attention, for
  * callers that cannot allocate device memory on their call path.  The pages have no
  * counterpart to this entry point: it exists for integration only.  Examples are a plug-in
@@ -322,6 +345,16 @@ CSLD_API csld_status csld_lse_merge(const float* outs, const float* lses, int R,
  * dst and src 16-byte aligned, bytes a multiple of 16; the two ranges must not overlap.
  * ---------------------------------------------------------------------------------------- */
 CSLD_API csld_status csld_stage(void* dst, const void* src, size_t bytes, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Test hook (no counterpart on the pages): the indexer's cooperative kernel waits, with a bound
+ * of about half a second, for the CTAs of a sequence at four cross-CTA barriers.  This call adds
+ * `extra` arrivals to every barrier target of the calls that follow (0 restores normal use), so
+ * that a test can make those waits run out and check the recovery: the kernel returns,
+ * CSLD_DEVERR_TIMEOUT is set in the error word, and the workspace must be zero-filled again
+ * before the next call.  Process-wide; not for production use.
+ * ---------------------------------------------------------------------------------------- */
+CSLD_API void csld_test_set_barrier_extra(int extra);
 
 #ifdef __cplusplus
 }
