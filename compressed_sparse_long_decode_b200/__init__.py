@@ -16,7 +16,7 @@ import os
 import torch
 
 __all__ = [
-    "csa_compress", "hca_compress", "compress", "indexer_topk", "hybrid_decode_attention",
+    "csa_compress", "hca_compress", "compress", "compress_channel", "indexer_topk", "hybrid_decode_attention",
     "kv_cache_append", "kv_cache_prefill", "LayerCache", "CsldError", "lib", "ENTRY_BYTES",
     "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace", "DecodeStack",
     "layer_pattern", "stage", "indexer_rescore", "topk_merge", "lse_merge", "ContextParallelLayer",
@@ -61,6 +61,7 @@ def _load():
     L.csld_status_string.restype = C.c_char_p
     L.csld_status_string.argtypes = [I]
     L.csld_compress.argtypes = [P, P, P, I, P, I64, P, P, P, P]
+    L.csld_compress_channel.argtypes = [P, P, P, I, P, I64, P, P, P, P]
     L.csa_compress.argtypes = [P, P, P, P, I64, P, P, P, P]
     L.hca_compress.argtypes = [P, P, P, I64, P, P]
     L.kv_cache_append.argtypes = [C.POINTER(_Cache), P, P, P, P]
@@ -79,7 +80,7 @@ def _load():
     L.hybrid_decode_attention_multi.argtypes = [P, I, P, I64, I, P, I, P, I, I, P, I, I, F, P, P, P, S, P, P]
     L.csld_topk_merge.argtypes = [P, P, P, I, I, I, I64, I64, P, P]
     L.csld_lse_merge.argtypes = [P, P, I, I, I, P, P, P]
-    for fn in ("csld_compress", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
+    for fn in ("csld_compress", "csld_compress_channel", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
                "indexer_topk", "hybrid_decode_attention", "csld_stage", "indexer_rescore", "csld_topk_merge",
                "csld_lse_merge", "indexer_topk_multi", "hybrid_decode_attention_multi"):
         getattr(L, fn).restype = I
@@ -142,6 +143,28 @@ def compress(raw, gate, pos_bias, ratio, w_idx=None, kv_out=None, ikey_out=None,
             iscale_out = torch.empty((E, 2), dtype=torch.float32, device=dev)
     _check(lib.csld_compress(_ptr(raw), _ptr(gate), _ptr(pos_bias), ratio, _ptr(w_idx), T,
                              _ptr(kv_out), _ptr(ikey_out), _ptr(iscale_out), _stream()), "csld_compress")
+    return (kv_out, ikey_out, iscale_out) if w_idx is not None else kv_out
+
+
+def compress_channel(raw, gate, pos_bias, ratio, w_idx=None, kv_out=None, ikey_out=None, iscale_out=None):
+    """Per-channel gated compression of one sequence: raw [T,512] bf16, gate [T,512] f32,
+    pos_bias [ratio,512] f32 (csld_compress_channel)."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    _need(pos_bias, torch.float32, "pos_bias")
+    T = raw.shape[0]
+    E = T // ratio
+    dev = raw.device
+    if kv_out is None:
+        kv_out = torch.empty((E, ENTRY_BYTES), dtype=torch.uint8, device=dev)
+    if w_idx is not None:
+        _need(w_idx, torch.float32, "w_idx")
+        if ikey_out is None:
+            ikey_out = torch.empty((E, IKEY_BYTES), dtype=torch.uint8, device=dev)
+        if iscale_out is None:
+            iscale_out = torch.empty((E, 2), dtype=torch.float32, device=dev)
+    _check(lib.csld_compress_channel(_ptr(raw), _ptr(gate), _ptr(pos_bias), ratio, _ptr(w_idx), T, _ptr(kv_out),
+                                     _ptr(ikey_out), _ptr(iscale_out), _stream()), "csld_compress_channel")
     return (kv_out, ikey_out, iscale_out) if w_idx is not None else kv_out
 
 

@@ -375,4 +375,21 @@ csld_status hybrid_decode_attention_multi(const uint16_t* q, int heads, const ui
 
 void csld_test_set_barrier_extra(int extra) { csld::g_test_barrier_extra.store(extra < 0 ? 0 : extra); }
 
+csld_status csld_compress_channel(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
+                                  const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
+                                  float* iscale_out, void* stream) {
+    if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
+    if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
+    if (T / ratio == 0) return CSLD_OK;
+    if (!raw || !gate || !pos_bias || !kv_out) return fail(CSLD_ERR_ARG, "a required pointer is NULL");
+    if (w_idx && (!ikey_out || !iscale_out)) return fail(CSLD_ERR_ARG, "ikey_out / iscale_out NULL with w_idx");
+    if (!aligned16(raw) || !aligned16(gate) || !aligned16(pos_bias) || !aligned16(kv_out) ||
+        (ikey_out && !aligned16(ikey_out)))
+        return fail(CSLD_ERR_ALIGN, "raw, gate, pos_bias, kv_out and ikey_out must be 16-byte aligned");
+    cudaError_t e = csld::launch_compress_channel(raw, gate, pos_bias, ratio, w_idx, T, kv_out, ikey_out, iscale_out,
+                                                  num_sms(), as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "csld_compress_channel");
+    return CSLD_OK;
+}
+
 }  // extern "C"

@@ -31,7 +31,9 @@
 //    dims 448..511 it yields are discarded.  S and O accumulate in fp32 in tensor memory.
 //  - Warps 8-15 run the online softmax: thread = entry (TMEM lane); warps 8-11 own heads 0-7,
 //    warps 12-15 heads 8-15.  The running max is raised lazily: O is rescaled in tensor memory
-//    only when a tile's max exceeds it by more than 8 (log2 units), so P <= 256 always.
+//    only when a tile's max exceeds it by more than 8 (log2 units), so P <= 256 always.  Per
+//    tile the softmax warps meet at three barriers in the common case (the tile maxima, the
+//    rescale check, the P block scales), two more only when O must be rescaled.
 //  - Warps 4-15 prepare the query operands while the first copies are in flight.
 //  Three tile buffers, two S slots and two P buffers overlap the copies of tiles t+1 and t+2,
 //  QK of t+1, softmax of t and PV of t-1.  Every wait is bounded.  Each split writes its unnormalised O,
@@ -80,7 +82,7 @@ struct TcAttnSmem {
     uint8_t pbf[2][2][16 * 128];              // bf16 P: two 64-entry K blocks of 16 rows
     float c2[kHeads];                         // log2-domain logit factor per head
     float sq[kHeads];                         // power-of-two query scale per head
-    float tmax[4][kHeads];                    // tile maxima per lane quarter
+    float tmax[2][4][kHeads];                 // tile maxima per lane quarter, two sets by tile parity
     uint32_t sfb[2][4][kHeads];               // P block-scale bytes [buffer][32-entry block][head]
     float lred[4][kHeads];
     uint64_t full[kBufs], empty[kBufs], sfull[2], sfree[2], pfull[2], pdone[2], drain;
@@ -424,47 +426,58 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
             const int s = t & 1;
             const int64_t i = (t_begin + t) * kTcTile + e;
             const bool valid = e < kTcTile && (i < n_comp4 ? comp_row(i, false) >= 0 : i < L);
-            ok = !*fail && mbar_wait(&sm.sfull[s], (t >> 1) & 1);
-            if (named_barrier_or(kSmBar, 256, !ok)) {   // the softmax warps leave together
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t shi[8], slo[8];
-            tmem_ld_32x32b_x8(lb + kColS + 32u * s + 8u * hg, shi);
-            tmem_ld_32x32b_x8(lb + kColS + 32u * s + 16u + 8u * hg, slo);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.sfree[s]);
+            ok = __all_sync(0xffffffffu, !*fail && mbar_wait(&sm.sfull[s], (t >> 1) & 1));
             float x[8];
+            if (ok) {
+                tc_fence_after();
+                uint32_t shi[8], slo[8];
+                tmem_ld_32x32b_x8(lb + kColS + 32u * s + 8u * hg, shi);
+                tmem_ld_32x32b_x8(lb + kColS + 32u * s + 16u + 8u * hg, slo);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sfree[s]);
 #pragma unroll
-            for (int h = 0; h < 8; ++h)
-                x[h] = valid ? (__uint_as_float(shi[h]) + __uint_as_float(slo[h])) * c2[h] : -INFINITY;
-            // tile max per head: warp max of order keys, then across the four lane quarters
+                for (int h = 0; h < 8; ++h)
+                    x[h] = valid ? (__uint_as_float(shi[h]) + __uint_as_float(slo[h])) * c2[h] : -INFINITY;
+            } else {
+#pragma unroll
+                for (int h = 0; h < 8; ++h) x[h] = -INFINITY;
+            }
+            // tile max per head: warp max of order keys, published per lane quarter (two sets,
+            // alternating by tile, so the next tile's maxima never overwrite ones still read)
 #pragma unroll
             for (int h = 0; h < 8; ++h) {
                 const uint32_t km = __reduce_max_sync(0xffffffffu, score_key(x[h]));
-                if (lane == h) sm.tmax[sub][8 * hg + h] = order_key_to_float(km);
+                if (lane == h) sm.tmax[s][sub][8 * hg + h] = order_key_to_float(km);
             }
-            named_barrier(kSmBar, 256);
+            if (named_barrier_or(kSmBar, 256, !ok)) {   // maxima published; the warps leave together
+                ok = false;
+                break;
+            }
             bool rescale = false;
             float mnew[8];
 #pragma unroll
             for (int h = 0; h < 8; ++h) {
                 const int hh = 8 * hg + h;
-                const float tm = fmaxf(fmaxf(sm.tmax[0][hh], sm.tmax[1][hh]), fmaxf(sm.tmax[2][hh], sm.tmax[3][hh]));
+                const float tm =
+                    fmaxf(fmaxf(sm.tmax[s][0][hh], sm.tmax[s][1][hh]), fmaxf(sm.tmax[s][2][hh], sm.tmax[s][3][hh]));
                 mnew[h] = (tm > mref[h] + kRescaleLog2 || mref[h] == -INFINITY) ? fmaxf(tm, mref[h]) : mref[h];
                 rescale |= (mnew[h] != mref[h]) && (mref[h] != -INFINITY);
             }
-            // P buffer s is free once PV(t-2) completed; a rescale also needs PV(t-1) done.  The
-            // barriers also tell every warp that all of them have read sm.tmax.
+            // P buffer s is free once PV(t-2) completed; a rescale of O also needs PV(t-1) done.
+            // One barrier in the common case; a rescale or a failed wait anywhere takes two more.
             if (t >= 2) ok = mbar_wait(&sm.pdone[s], ((t >> 1) - 1) & 1);
-            const bool any_rescale = named_barrier_or(kSmBar, 256, rescale);
-            if (ok && any_rescale && t >= 1) ok = mbar_wait(&sm.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1);
-            if (named_barrier_or(kSmBar, 256, !ok)) {
-                ok = false;
-                break;
+            if (named_barrier_or(kSmBar, 256, rescale || !ok)) {
+                if (named_barrier_or(kSmBar, 256, !ok)) {
+                    ok = false;
+                    break;
+                }
+                if (t >= 1) ok = mbar_wait(&sm.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1);
+                if (named_barrier_or(kSmBar, 256, !ok)) {
+                    ok = false;
+                    break;
+                }
             }
             tc_fence_after();
             if (rescale) {   // this warp's 8 heads in every O block of its lane quarter

@@ -411,6 +411,126 @@ cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float*
 }
 
 // ------------------------------------------------------------------------------------------
+// Per-channel gating (a layout / gating variant): one gate logit per token and dimension and one
+// bias per block slot and dimension; every dimension d of entry s pools its own softmax,
+//   a_j = gate[s m + j][d] + bias[j][d],  w = softmax_j(a),  c_d = sum_j w_j x[s m + j][d].
+// One warp per entry (lane l: dims 16l..16l+15), an online softmax over the slots in order, four
+// slots' loads in flight.  With w_idx the indexer key is projected on the CUDA cores from bf16
+// operands (W_I^T staged in shared memory) and FP4-quantised as for csld_compress.
+// ------------------------------------------------------------------------------------------
+constexpr int kChThreads = 256;
+struct ChannelSmem {
+    uint16_t wt[kIdxDim][kDim];       // W_I^T, bf16
+    float c[kChThreads / 32][kDim];   // each warp's pooled entry
+};
+
+__global__ void __launch_bounds__(kChThreads) pool_channel_kernel(
+    const uint16_t* __restrict__ raw, const float* __restrict__ gate, const float* __restrict__ bias, int m,
+    const float* __restrict__ w_idx, int64_t T, int64_t E, uint8_t* __restrict__ kv_out, uint8_t* __restrict__ ikey_out,
+    float* __restrict__ iscale_out) {
+    extern __shared__ __align__(16) uint8_t ch_raw[];
+    ChannelSmem& sm = *reinterpret_cast<ChannelSmem*>(ch_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (w_idx) {
+        for (int i = tid; i < kDim * kIdxDim; i += kChThreads) {
+            const int k = i / kIdxDim, n = i % kIdxDim;
+            sm.wt[n][k] = static_cast<uint16_t>(f32_to_bf16_bits(__ldg(w_idx + i)));
+        }
+        __syncthreads();
+    }
+    const int64_t n_warps = (int64_t)gridDim.x * (kChThreads / 32);
+    for (int64_t s = (int64_t)blockIdx.x * (kChThreads / 32) + warp; s < E; s += n_warps) {
+        float mx[16], sum[16], acc[16];
+#pragma unroll
+        for (int d = 0; d < 16; ++d) {
+            mx[d] = -INFINITY;
+            sum[d] = 0.f;
+            acc[d] = 0.f;
+        }
+        const size_t t0 = (size_t)s * m;
+        for (int j0 = 0; j0 < m; j0 += 4) {
+            uint4 x[4][2];
+            float4 g[4][4], bb[4][4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (j0 + r < m) {
+                    const size_t t = t0 + j0 + r;
+                    const uint4* xr = reinterpret_cast<const uint4*>(raw + t * kDim) + 2 * lane;
+                    const float4* gr = reinterpret_cast<const float4*>(gate + t * kDim) + 4 * lane;
+                    const float4* br = reinterpret_cast<const float4*>(bias + (size_t)(j0 + r) * kDim) + 4 * lane;
+                    x[r][0] = __ldg(xr);
+                    x[r][1] = __ldg(xr + 1);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        g[r][q] = __ldg(gr + q);
+                        bb[r][q] = __ldg(br + q);
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (j0 + r >= m) break;
+                const uint32_t xv[8] = {x[r][0].x, x[r][0].y, x[r][0].z, x[r][0].w,
+                                        x[r][1].x, x[r][1].y, x[r][1].z, x[r][1].w};
+                const float gv[16] = {g[r][0].x, g[r][0].y, g[r][0].z, g[r][0].w, g[r][1].x, g[r][1].y, g[r][1].z,
+                                      g[r][1].w, g[r][2].x, g[r][2].y, g[r][2].z, g[r][2].w, g[r][3].x, g[r][3].y,
+                                      g[r][3].z, g[r][3].w};
+                const float bv[16] = {bb[r][0].x, bb[r][0].y, bb[r][0].z, bb[r][0].w, bb[r][1].x, bb[r][1].y,
+                                      bb[r][1].z, bb[r][1].w, bb[r][2].x, bb[r][2].y, bb[r][2].z, bb[r][2].w,
+                                      bb[r][3].x, bb[r][3].y, bb[r][3].z, bb[r][3].w};
+#pragma unroll
+                for (int d = 0; d < 16; ++d) {
+                    const float a = gv[d] + bv[d];
+                    const float xd = bf16_bits_to_f32(d & 1 ? xv[d >> 1] >> 16 : xv[d >> 1]);
+                    if (a > mx[d]) {   // a new maximum: rescale what was accumulated
+                        const float f = expf(mx[d] - a);
+                        sum[d] = fmaf(sum[d], f, 1.f);
+                        acc[d] = fmaf(acc[d], f, xd);
+                        mx[d] = a;
+                    } else {
+                        const float e = expf(a - mx[d]);
+                        sum[d] += e;
+                        acc[d] = fmaf(e, xd, acc[d]);
+                    }
+                }
+            }
+        }
+        float c[16];
+#pragma unroll
+        for (int d = 0; d < 16; ++d) c[d] = acc[d] / sum[d];
+        warp_store_entry(kv_out + (size_t)s * kEntry, lane, c);
+        if (w_idx) {
+            // u_j = sum_d bf16(c_d) * bf16(W_I[d][j]) in fp32; lane l forms u_{2l}, u_{2l+1}
+#pragma unroll
+            for (int d = 0; d < 16; ++d) sm.c[warp][16 * lane + d] = bf16_bits_to_f32(f32_to_bf16_bits(c[d]));
+            __syncwarp();
+            float u0 = 0.f, u1 = 0.f;
+            for (int d = 0; d < kDim; ++d) {
+                const float cd = sm.c[warp][d];
+                u0 = fmaf(cd, bf16_bits_to_f32(sm.wt[2 * lane][d]), u0);
+                u1 = fmaf(cd, bf16_bits_to_f32(sm.wt[2 * lane + 1][d]), u1);
+            }
+            __syncwarp();
+            warp_store_fp4(ikey_out + (size_t)s * kIkey, iscale_out + (size_t)s * 2, s, lane, u0, u1);
+        }
+    }
+}
+
+cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, const float* bias, int m,
+                                    const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
+                                    float* iscale_out, int num_sms, cudaStream_t stream) {
+    const int64_t E = T / m;
+    if (E <= 0) return cudaSuccess;
+    const size_t smem = w_idx ? sizeof(ChannelSmem) : 0;
+    cudaError_t e = set_smem_once(pool_channel_kernel, sizeof(ChannelSmem));
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = min64((E + kChThreads / 32 - 1) / (kChThreads / 32), 4LL * num_sms);
+    pool_channel_kernel<<<static_cast<unsigned>(blocks), kChThreads, smem, stream>>>(raw, gate, bias, m, w_idx, T, E,
+                                                                                    kv_out, ikey_out, iscale_out);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
 // Window ring + tail after a prefill of T tokens (one CTA per sequence).
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) prefill_state_kernel(const uint16_t* __restrict__ raw,

@@ -14,6 +14,9 @@ cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float*
                             uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, int num_sms,
                             cudaStream_t stream);
 size_t compress_index_smem_bytes();
+cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, const float* bias, int m,
+                                    const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
+                                    float* iscale_out, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_prefill_state(const uint16_t* raw, const float* gate, int64_t T, int m, int W,
                                  int B, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,

@@ -119,6 +119,22 @@ CSLD_API csld_status hca_compress(const uint16_t* raw, const float* gate, const 
                          int64_t T, uint8_t* kv_out, void* stream);
 
 /* ----------------------------------------------------------------------------------------
+ * Per-channel gated compression -- the other plain reading of "softmax-gated pooling with a
+ * learned positional bias" ([HF] CSA paragraph; Figure 3 caption; HCA paragraph): a gate
+ * logit for every token AND dimension and a bias for every block slot and dimension.  Each
+ * dimension d of entry s pools its own softmax:
+ *   a_j = gate[s*m+j][d] + pos_bias[j][d],  w = softmax_j(a),  c_d = sum_j w_j raw[s*m+j][d],
+ * then the entry and (w_idx != NULL) the FP4 indexer key exactly as csld_compress writes them
+ * (the key projected from bf16 operands with fp32 accumulation).  With gate and bias equal
+ * across dimensions this is csld_compress.
+ *   gate [T][512] f32, pos_bias [ratio][512] f32; others as for csld_compress; raw, gate,
+ *   pos_bias, kv_out, ikey_out 16-byte aligned.
+ * -------------------------------------------------------------------------------------- */
+CSLD_API csld_status csld_compress_channel(const uint16_t* raw, const float* gate, const float* pos_bias,
+                                           int ratio, const float* w_idx, int64_t T, uint8_t* kv_out,
+                                           uint8_t* ikey_out, float* iscale_out, void* stream);
+
+/* ----------------------------------------------------------------------------------------
  * One layer's KV-cache state for B sequences ([VEL] KV-cache-layout section: compressed
  * cache, separate sliding-window state, separately kept uncompressed tail).  A host struct of
  * device pointers; the caller owns all of it.

@@ -68,6 +68,10 @@ def _declare(L):
     L.orc_pool_block.argtypes = [_P, _P, _P, C.c_int, _P]
     L.orc_compress.restype = None
     L.orc_compress.argtypes = [_P, _P, _P, _P, C.c_int64, C.c_int, _P, _P, _P]
+    L.orc_pool_block_channel.restype = None
+    L.orc_pool_block_channel.argtypes = [_P, _P, _P, C.c_int, _P]
+    L.orc_compress_channel.restype = None
+    L.orc_compress_channel.argtypes = [_P, _P, _P, _P, C.c_int64, C.c_int, _P, _P, _P]
     L.orc_indexer_scores.restype = None
     L.orc_indexer_scores.argtypes = [_P, _P, C.c_int64, _P, _P, _P, _P]
     L.orc_topk.restype = None
@@ -201,6 +205,32 @@ def compress(raw_bits, gate, bias, m, w_idx=None):
     w = _c(w_idx, np.float32) if w_idx is not None else None
     lib().orc_compress(_ptr(raw_bits), _ptr(gate), _ptr(bias), _ptr(w), T, m, _ptr(kv), _ptr(ik),
                        _ptr(isc))
+    return kv, ik, isc
+
+
+def pool_block_channel(raw_bits, gate, bias):
+    """Per-channel gating: raw_bits uint16 [m,512]; gate, bias float32 [m,512] -> float64 [512]."""
+    raw_bits = _c(raw_bits, np.uint16)
+    gate = _c(gate, np.float32)
+    bias = _c(bias, np.float32)
+    m = raw_bits.shape[0]
+    out = np.zeros(D, np.float64)
+    lib().orc_pool_block_channel(_ptr(raw_bits), _ptr(gate), _ptr(bias), m, _ptr(out))
+    return out
+
+
+def compress_channel(raw_bits, gate, bias, m, w_idx=None):
+    """Per-channel prefill compression: gate [T,512], bias [m,512].  Returns (kv, ikeys, iscales)."""
+    raw_bits = _c(raw_bits, np.uint16)
+    gate = _c(gate, np.float32)
+    bias = _c(bias, np.float32)
+    T = raw_bits.shape[0]
+    E = T // m
+    kv = np.zeros((E, ENTRY_BYTES), np.uint8)
+    ik = np.zeros((E, IKEY_BYTES), np.uint8) if w_idx is not None else None
+    isc = np.zeros((E, 2), np.float32) if w_idx is not None else None
+    w = _c(w_idx, np.float32) if w_idx is not None else None
+    lib().orc_compress_channel(_ptr(raw_bits), _ptr(gate), _ptr(bias), _ptr(w), T, m, _ptr(kv), _ptr(ik), _ptr(isc))
     return kv, ik, isc
 
 

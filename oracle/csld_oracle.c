@@ -232,6 +232,31 @@ void orc_pool_block(const uint16_t* raw, const float* gate, const float* bias, i
     free(w);
 }
 
+/* O1, per-channel variant (the other plain reading of "softmax-gated pooling with a learned
+ * positional bias", [HF] CSA paragraph): one gate logit per token AND dimension, one bias per
+ * block slot and dimension.  For every dimension d separately:
+ *   a_j = z[j][d] + b[j][d],  w = softmax_j(a),  c_d = sum_j w_j x[j][d].
+ * gate [m][512] and bias [m][512] f32; with z[j][d] = z_j and b[j][d] = b_j for every d it is
+ * orc_pool_block. */
+void orc_pool_block_channel(const uint16_t* raw, const float* gate, const float* bias, int m, double* c) {
+    for (int d = 0; d < ORC_D; ++d) {
+        double amax = -INFINITY;
+        for (int j = 0; j < m; ++j) {
+            double a = (double)gate[(size_t)j * ORC_D + d] + (double)bias[(size_t)j * ORC_D + d];
+            if (a > amax) amax = a;
+        }
+        double wsum = 0.0;
+        for (int j = 0; j < m; ++j)
+            wsum += exp((double)gate[(size_t)j * ORC_D + d] + (double)bias[(size_t)j * ORC_D + d] - amax);
+        double acc = 0.0;
+        for (int j = 0; j < m; ++j) {
+            double wj = exp((double)gate[(size_t)j * ORC_D + d] + (double)bias[(size_t)j * ORC_D + d] - amax) / wsum;
+            acc += wj * orc_bf16_decode(raw[(size_t)j * ORC_D + d]);
+        }
+        c[d] = acc;
+    }
+}
+
 /* O2 -- indexer key before quantisation: u = c . W_I with W_I [512][64] row-major. */
 void orc_indexer_key_raw(const double* c, const float* w_idx, double* u) {
     for (int j = 0; j < ORC_IDX_DIM; ++j) {
@@ -251,6 +276,22 @@ void orc_compress(const uint16_t* raw, const float* gate, const float* bias, con
     for (int64_t s = 0; s < E; ++s) {
         double c[ORC_D], u[ORC_IDX_DIM];
         orc_pool_block(raw + (size_t)s * m * ORC_D, gate + (size_t)s * m, bias, m, c);
+        orc_entry_encode(c, kv_out + (size_t)s * ORC_ENTRY_BYTES);
+        if (w_idx) {
+            orc_indexer_key_raw(c, w_idx, u);
+            orc_fp4_quantize64(u, ikey_out + (size_t)s * ORC_IKEY_BYTES, iscale_out + (size_t)s * 2);
+        }
+    }
+}
+
+/* O1 (per-channel) + O2 over a whole prefill: gate [T][512], bias [m][512]. */
+void orc_compress_channel(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
+                          int64_t T, int m, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
+    int64_t E = T / m;
+#pragma omp parallel for schedule(static)
+    for (int64_t s = 0; s < E; ++s) {
+        double c[ORC_D], u[ORC_IDX_DIM];
+        orc_pool_block_channel(raw + (size_t)s * m * ORC_D, gate + (size_t)s * m * ORC_D, bias, m, c);
         orc_entry_encode(c, kv_out + (size_t)s * ORC_ENTRY_BYTES);
         if (w_idx) {
             orc_indexer_key_raw(c, w_idx, u);

@@ -83,3 +83,49 @@ def test_window_entries_are_bit_exact_on_codec_edge_cases(csld, orc):
     for i in range(n_tok):
         want = orc.entry_encode(tt[i].to(torch.float64).numpy())
         assert np.array_equal(got[i % W], want), f"token {i}"
+
+
+def _channel_inputs(T, m, seed):
+    g = synth.gen(seed)
+    raw = synth.bf16_normal((T, 512), g)
+    gate = torch.randn((T, 512), generator=g)
+    bias = torch.randn((m, 512), generator=g) * 0.1
+    return raw, gate, bias
+
+
+@pytest.mark.parametrize("T,m,with_key", [(4096 + 3, 4, True), (128 * 9 + 5, 128, False), (700, 7, True)])
+def test_compress_channel_matches_oracle(csld, orc, T, m, with_key):
+    """Per-channel gating (a gate logit per token and dimension, a bias per slot and dimension),
+    against the oracle's per-dimension softmax pooling.  The GPU runs an online softmax over the
+    slots in fp32, so the bf16 RoPE values get four times the fp32 slack of the two-pass sum."""
+    raw, gate, bias = _channel_inputs(T, m, seed=T + m)
+    w = synth.prefill_inputs(8, seed=5)["w_idx"] if with_key else None
+    out = csld.compress_channel(raw.cuda(), gate.cuda(), bias.cuda(), m, None if w is None else w.cuda())
+    torch.cuda.synchronize()
+    bits = synth.bits16(raw)
+    rkv, rik, risc = orc.compress_channel(bits, gate.numpy(), bias.numpy(), m, None if w is None else w.numpy())
+    kv = out[0] if with_key else out
+    H.assert_entries_close(kv.cpu().numpy(), rkv, f"per-channel ratio-{m} entries", 4 * H.pool_slack(raw, m))
+    if with_key:
+        gsc = out[2].cpu().numpy()
+        ramax = None
+        if not np.array_equal(gsc, risc):
+            E = T // m
+            ramax = np.zeros((E, 2))
+            for s in range(E):
+                c = orc.pool_block_channel(bits[s * m:(s + 1) * m], gate.numpy()[s * m:(s + 1) * m], bias.numpy())
+                u = orc.indexer_key_raw(c, w.numpy())
+                ramax[s] = [np.abs(u[:32]).max(), np.abs(u[32:]).max()]
+        H.assert_fp4_keys_close(synth.ikeys_swap_halves(out[1].cpu().numpy()), gsc, rik, risc, ramax)
+
+
+def test_compress_channel_with_scalar_gates_is_csld_compress(csld, orc):
+    """Gates and biases equal across dimensions reduce per-channel gating to csld_compress."""
+    T, m = 1024, 4
+    inp = synth.prefill_inputs(T, seed=44)
+    gate = inp["gate"][:, None].expand(T, 512).contiguous()
+    bias = inp["bias4"][:, None].expand(m, 512).contiguous()
+    kv = csld.compress_channel(inp["raw"].cuda(), gate.cuda(), bias.cuda(), m)
+    torch.cuda.synchronize()
+    rkv, _, _ = orc.compress(synth.bits16(inp["raw"]), inp["gate"].numpy(), inp["bias4"].numpy(), m)
+    H.assert_entries_close(kv.cpu().numpy(), rkv, "per-channel with scalar gates", 4 * H.pool_slack(inp["raw"], m))

@@ -482,3 +482,53 @@ def test_kv_byte_accounting_reproduces_page_figure(orc):
     assert abs(frac - fig["kv_fraction_vs_gqa8_bf16"]["value"]) < 0.005, frac
     # entry counts of the 4096-token case
     assert 4096 // r_csa == 1024 and 4096 // r_hca == 32
+
+
+# ---- per-channel gating (layout / gating variant) ---------------------------------------------
+def test_pool_channel_reduces_to_scalar_gating(orc):
+    """Gates and biases equal across dimensions: per-channel pooling is the scalar pooling."""
+    rng = np.random.default_rng(5)
+    for m in (1, 4, 7, 128):
+        raw = rng.standard_normal((m, 512)).astype(np.float32)
+        bits = (raw.view(np.uint32) >> 16).astype(np.uint16)
+        z = rng.standard_normal(m).astype(np.float32)
+        b = (0.1 * rng.standard_normal(m)).astype(np.float32)
+        ref = orc.pool_block(bits, z, b)
+        got = orc.pool_block_channel(bits, np.repeat(z[:, None], 512, 1), np.repeat(b[:, None], 512, 1))
+        assert np.allclose(got, ref, rtol=0, atol=1e-12 * max(1.0, np.abs(ref).max()))
+
+
+def test_pool_channel_dims_are_independent(orc):
+    """A dominant logit on one dimension picks that slot's value there; a dimension with equal
+    logits is the mean; the other dimensions do not see either."""
+    m = 4
+    rng = np.random.default_rng(6)
+    raw = rng.standard_normal((m, 512)).astype(np.float32)
+    bits = (raw.view(np.uint32) >> 16).astype(np.uint16)
+    x = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    gate = np.zeros((m, 512), np.float32)
+    bias = np.zeros((m, 512), np.float32)
+    gate[2, 10] = 80.0                      # dim 10: slot 2 dominates
+    gate[:, 11] = rng.standard_normal(m)     # dim 11: a softmax of its own
+    c = orc.pool_block_channel(bits, gate, bias)
+    assert abs(c[10] - x[2, 10]) < 1e-12
+    w = np.exp(gate[:, 11].astype(np.float64) - gate[:, 11].max())
+    w /= w.sum()
+    assert abs(c[11] - (w * x[:, 11]).sum()) < 1e-12
+    others = [d for d in range(512) if d not in (10, 11)]
+    assert np.allclose(c[others], x[:, others].mean(0), rtol=0, atol=1e-12)
+
+
+def test_compress_channel_shift_invariance(orc):
+    """Adding a constant to one dimension's logits of a block leaves the entry unchanged."""
+    m, T = 4, 64
+    rng = np.random.default_rng(7)
+    raw = rng.standard_normal((T, 512)).astype(np.float32)
+    bits = (raw.view(np.uint32) >> 16).astype(np.uint16)
+    gate = rng.standard_normal((T, 512)).astype(np.float32)
+    bias = (0.1 * rng.standard_normal((m, 512))).astype(np.float32)
+    kv0, _, _ = orc.compress_channel(bits, gate, bias, m)
+    g2 = gate.copy()
+    g2[4:8, 100] += 3.0                     # block 1, dimension 100
+    kv1, _, _ = orc.compress_channel(bits, g2, bias, m)
+    assert np.array_equal(kv0, kv1)
