@@ -10,13 +10,14 @@
 // {window tokens}.
 //
 // One CTA = one split of one sequence's key list, walked in tiles of 96 entries; 16 warps.
-//  - Warps 0-3 bring a tile in with TMA: five 128-byte column blocks of every entry (bytes 0,
-//    128, 256, 384 and 448 -- the last one is the RoPE part), each block [96 entries][128 B]
-//    with the 128-byte swizzle, into one of three tile buffers, so copies run up to two tiles
-//    ahead of the PV that frees a buffer.  (The QK MMA has 128 rows: it also reads the 32 rows
-//    after a block, whose scores are never used.)  Contiguous tiles take one box copy per block; otherwise rows
-//    come four at a time by index (tile::gather4).  The same image is the K-major operand of
-//    QK (rows = entries) and the MN-major operand of PV (rows = dims).
+//  - Warps 0-3 bring a tile in: five 128-byte column blocks of every entry (bytes 0, 128, 256,
+//    384 and 448 -- the last one is the RoPE part), each block [96 entries][128 B] with the
+//    128-byte swizzle, into one of three tile buffers, so copies run up to two tiles ahead of
+//    the PV that frees a buffer.  (The QK MMA has 128 rows: it also reads the 32 rows after a
+//    block, whose scores are never used.)  Contiguous tiles take one TMA box copy per block;
+//    other tiles are gathered entry by entry with 16-byte cp.async copies (one TMA request per
+//    four rows measured about 40 cycles each, ~2.4 us for a 96-entry tile).  The same image is
+//    the K-major operand of QK (rows = entries) and the MN-major operand of PV (rows = dims).
 //  - Warp 4 issues the MMAs (one thread):
 //      S[entry][hi|lo head] = K_nope . [Qhi;Qlo]^T    kind::f8f6f4, E4M3 x E4M3, N = 32
 //                           + K_rope . Qrope^T         kind::f16, bf16 (into the hi columns)
@@ -26,15 +27,16 @@
 //    (hi = E4M3(q), lo = E4M3(q - hi)); P is split the same way after a power-of-two scale
 //    per 32-entry block (the MMA's UE8M0 block scale), so each product keeps about as many
 //    significant bits as a bf16 operand.  The hi and lo rows are stacked into one N = 32
-//    operand and their results added when read back.  Block 3 holds bytes 384..511, whose
-//    upper half is the bf16 RoPE part: QK reads only its first 64 bytes, and the PV rows of
-//    dims 448..511 it yields are discarded.  S and O accumulate in fp32 in tensor memory.
+//    operand and their results added when read back.  Block 3 holds bytes 384..511 (box copies;
+//    a gathered tile fills only 384..447), whose upper half is the bf16 RoPE part: QK reads
+//    only its first 64 bytes, and the PV rows of dims 448..511 it yields are discarded.  S and O accumulate in fp32 in tensor memory.
 //  - Warps 8-15 run the online softmax: thread = entry (TMEM lane); warps 8-11 own heads 0-7,
 //    warps 12-15 heads 8-15.  The running max is raised lazily: O is rescaled in tensor memory
 //    only when a tile's max exceeds it by more than 8 (log2 units), so P <= 256 always.  Per
 //    tile the softmax warps meet at three barriers in the common case (the tile maxima, the
 //    rescale check, the P block scales), two more only when O must be rescaled.
-//  - Warps 4-15 prepare the query operands while the first copies are in flight.
+//  - Warps 8-15 prepare the query operands (one load per thread, issued right after the
+//    upstream wait) while the first copies are in flight.
 //  Three tile buffers, two S slots and two P buffers overlap the copies of tiles t+1 and t+2,
 //  QK of t+1, softmax of t and PV of t-1.  Every wait is bounded.  Each split writes its unnormalised O,
 //  the running max m (log2 units) and the sum l; attention_merge_kernel combines the splits.
@@ -70,7 +72,6 @@ constexpr uint32_t kIdQKr = idesc_bf16_m128(16, false, false);
 constexpr uint32_t kIdPVr = idesc_bf16_m128(16, true, false);
 constexpr int kSmBar = 1;                     // named barrier of the 8 softmax warps (256 threads)
 constexpr int kReadyBar = 2;                  // warps 4-15: query and tensor memory ready (384 threads)
-constexpr int kScaleBar = 3;                  // warps 4-15: query scales ready (384 threads)
 constexpr int kCopyBar = 4;                   // warps 0-3: the copy warps (128 threads)
 
 struct TcAttnSmem {
@@ -82,9 +83,10 @@ struct TcAttnSmem {
     uint8_t pbf[2][2][16 * 128];              // bf16 P: two 64-entry K blocks of 16 rows
     float c2[kHeads];                         // log2-domain logit factor per head
     float sq[kHeads];                         // power-of-two query scale per head
-    float tmax[2][4][kHeads];                 // tile maxima per lane quarter, two sets by tile parity
+    alignas(16) float tmax[2][4][kHeads];     // tile maxima per lane quarter, two sets by tile parity
     uint32_t sfb[2][4][kHeads];               // P block-scale bytes [buffer][32-entry block][head]
     float lred[4][kHeads];
+    const uint8_t* src[kTcTile];              // per-entry source of the tile being gathered (null: zeros)
     uint64_t full[kBufs], empty[kBufs], sfull[2], sfree[2], pfull[2], pdone[2], drain;
     uint32_t tmem_base;
     int32_t fail, n_issued, n_landed;
@@ -114,15 +116,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int y0, int y1, int y2, int y3,
-                                            uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
-        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
-           "r"(smem_u32(bar))
-        : "memory");
+// 16-byte copy global -> shared through L2 (cp.async.cg); src_bytes = 0 writes 16 zero bytes and
+// reads nothing.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 // Scales 8 consecutive TMEM columns of this warp's lanes by f[0..7].
 __device__ __forceinline__ void tmem_scale8(uint32_t taddr, const float (&f)[8]) {
     uint32_t o[8];
@@ -133,48 +135,75 @@ __device__ __forceinline__ void tmem_scale8(uint32_t taddr, const float (&f)[8])
     tmem_st_32x32b_x8(taddr, o);
 }
 
-// Query scales (256 threads, t = 0..255): head t / 16, dims 32*(t % 16) .. +31.  The query of
-// head h is scaled by sq = 2^(7 - floor(log2 max|q_h|)), so it stays below 256 (E4M3 max 448).
-__device__ __forceinline__ void qprep_scale(TcAttnSmem& sm, const uint16_t* q, int b, int t, float scale) {
-    const int h = t >> 4, part = t & 15;
-    const uint4* src = reinterpret_cast<const uint4*>(q + ((size_t)b * kHeads + h) * kDim + 32 * part);
-    float amax = 0.f;
+// The query of head h, t = 0..255 (head t / 16, dims 32 (t % 16) .. +31), loaded once into
+// registers.
+__device__ __forceinline__ void qprep_load(uint4 (&v)[4], const uint16_t* q, int b, int t) {
+    const uint4* src = reinterpret_cast<const uint4*>(q + ((size_t)b * kHeads + (t >> 4)) * kDim + 32 * (t & 15));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __ldg(src + i);
+}
+// Query operands from those registers.  Head h is scaled by sq = 2^(7 - floor(log2 max|q_h|)),
+// so it stays below 256 (E4M3 max 448); the 16 threads of a head find max|q_h| by shuffles.
+// Nope dims -> E4M3 hi and lo terms (rows h and 16 + h of the swizzled QK operand), RoPE dims
+// -> bf16; each thread writes whole 16-byte chunks.
+__device__ __forceinline__ void qprep_store(TcAttnSmem& sm, const uint4 (&v)[4], int t, float scale) {
+    const int h = t >> 4, part = t & 15, d0 = 32 * part;
+    uint32_t w[16];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint4 v = __ldg(src + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(w[c] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[c] >> 16))));
+        w[4 * i] = v[i].x;
+        w[4 * i + 1] = v[i].y;
+        w[4 * i + 2] = v[i].z;
+        w[4 * i + 3] = v[i].w;
     }
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(w[c] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[c] >> 16))));
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const int sh = amax > 0.f ? max(-100, min(100, 7 - ilogbf(amax))) : 0;
+    const float sq = ldexpf(1.f, sh);
     if (part == 0) {
-        const int sh = amax > 0.f ? max(-100, min(100, 7 - ilogbf(amax))) : 0;
-        const float sq = ldexpf(1.f, sh);
         sm.sq[h] = sq;
         sm.c2[h] = scale * 1.4426950408889634f / sq;
     }
-}
-// Query operands (384 threads, t = 0..383): pairs of dims.  Nope dims -> E4M3 hi and lo terms
-// in the swizzled QK operand, RoPE dims -> bf16.
-__device__ __forceinline__ void qprep_convert(TcAttnSmem& sm, const uint16_t* q, int b, int t) {
-    for (int p = t; p < kHeads * kDim / 2; p += 384) {
-        const int h = p >> 8, d = 2 * (p & 255);
-        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(q + ((size_t)b * kHeads + h) * kDim + d));
-        const float sq = sm.sq[h];
-        const float x0 = bf16_bits_to_f32(w & 0xFFFFu) * sq, x1 = bf16_bits_to_f32(w >> 16) * sq;
-        if (d < kNope) {
-            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
-            const uint32_t back = e4m3x2_to_f16x2(hi);   // exact
-            const float r0 = x0 - __half2float(__ushort_as_half(static_cast<unsigned short>(back & 0xFFFFu)));
-            const float r1 = x1 - __half2float(__ushort_as_half(static_cast<unsigned short>(back >> 16)));
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
-            *reinterpret_cast<uint16_t*>(&sm.qk[d >> 7][sw128(h, d & 127)]) = static_cast<uint16_t>(hi);
-            *reinterpret_cast<uint16_t*>(&sm.qk[d >> 7][sw128(16 + h, d & 127)]) = static_cast<uint16_t>(lo);
-        } else {
-            const int r = d - kNope;
-            *reinterpret_cast<uint32_t*>(sm.qr + sw128(h, 2 * r)) = f32_to_bf16_bits(x0) | (f32_to_bf16_bits(x1) << 16);
+    if (d0 < kNope) {
+        uint32_t hw[8], lw[8];   // bytes of dims d0 + 4c .. +3
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t hi2[2], lo2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t x = w[2 * c + u];
+                const float x0 = bf16_bits_to_f32(x & 0xFFFFu) * sq, x1 = bf16_bits_to_f32(x >> 16) * sq;
+                hi2[u] = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+                const uint32_t back = e4m3x2_to_f16x2(hi2[u]);   // exact
+                const float r0 = x0 - __half2float(__ushort_as_half(static_cast<unsigned short>(back & 0xFFFFu)));
+                const float r1 = x1 - __half2float(__ushort_as_half(static_cast<unsigned short>(back >> 16)));
+                lo2[u] = __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
+            }
+            hw[c] = (hi2[0] & 0xFFFFu) | (hi2[1] << 16);
+            lw[c] = (lo2[0] & 0xFFFFu) | (lo2[1] << 16);
+        }
+        uint8_t* blk = sm.qk[d0 >> 7];
+        const int c0 = d0 & 127;
+        *reinterpret_cast<uint4*>(blk + sw128(h, c0)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(blk + sw128(h, c0 + 16)) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+        *reinterpret_cast<uint4*>(blk + sw128(16 + h, c0)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        *reinterpret_cast<uint4*>(blk + sw128(16 + h, c0 + 16)) = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    } else {
+        const int r0 = d0 - kNope;   // RoPE dims r0 .. r0 + 31: 64 bytes of row h
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t o[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t x = w[4 * j + c];
+                o[c] = f32_to_bf16_bits(bf16_bits_to_f32(x & 0xFFFFu) * sq) |
+                       (f32_to_bf16_bits(bf16_bits_to_f32(x >> 16) * sq) << 16);
+            }
+            *reinterpret_cast<uint4*>(sm.qr + sw128(h, 2 * r0 + 16 * j)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
     }
     fence_proxy_async_smem();
@@ -183,8 +212,8 @@ __device__ __forceinline__ void qprep_convert(TcAttnSmem& sm, const uint16_t* q,
 }  // namespace
 
 __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
-    const __grid_constant__ CUtensorMap kv_tile, const __grid_constant__ CUtensorMap kv_rows,
-    const __grid_constant__ CUtensorMap win_rows, const __grid_constant__ CUtensorMap win_tile,
+    const __grid_constant__ CUtensorMap kv_tile, const __grid_constant__ CUtensorMap win_tile,
+    const uint8_t* __restrict__ comp_kv, const uint8_t* __restrict__ win_kv,
     const uint16_t* __restrict__ q, int64_t cap, int ratio,
     const int32_t* __restrict__ topk, int k, int W, int Wr, int Q, const int32_t* __restrict__ seq_len, float scale,
     int splits, float* __restrict__ opart, float2* __restrict__ mlpart, int32_t* err) {
@@ -199,7 +228,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     // ---- setup --------------------------------------------------------------------------------
     if (tid == 0) {
         for (int s = 0; s < kBufs; ++s) {
-            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.full[s], 128);   // one arrival per copy thread
             mbar_init(&sm.empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -220,8 +249,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_map(&kv_tile);
-        tma_prefetch_map(&kv_rows);
-        tma_prefetch_map(&win_rows);
         tma_prefetch_map(&win_tile);
     }
     tc_fence_before();
@@ -229,6 +256,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     tc_fence_after();
     pdl_wait();      // lengths, top-k indices and the caches come from upstream
     pdl_trigger();
+    uint4 qv[4];     // the softmax warps' query values, in flight while the length loads
+    if (warp >= 8) qprep_load(qv, q, vq, tid - 256);
 
     // ---- the key list of sequence b and this split's tile range ----------------------------
     // list = [compressed slots padded to a multiple of 4 with empty slots][window tokens], so a
@@ -249,15 +278,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     const int64_t t_begin = n_tiles_all * split / splits;
     const int n_tiles = static_cast<int>(n_tiles_all * (split + 1) / splits - t_begin);
     const size_t part = (size_t)vq * splits + split;
-    // rows past the end of each map read as zeros
-    const int32_t oob_kv = static_cast<int32_t>(min64((int64_t)B * cap, 0x7FFFFFFF));
-    const int32_t oob_win = static_cast<int32_t>(min64((int64_t)B * max(Wr, 1), 0x7FFFFFFF));
-    // compressed slot i -> row of the compressed map, or -1 for an empty slot
-    auto comp_row = [&](int64_t i, bool report) -> int32_t {
+    // compressed slot i -> row of the compressed map, or -1 for an empty slot; sel = the slot's
+    // top-k entry (sparse lists; loaded by sel_of, so several loads can be in flight at once)
+    auto sel_of = [&](int64_t i) -> int32_t { return (sparse && i < n_comp) ? __ldg(topk + (size_t)vq * k + i) : 0; };
+    auto comp_row = [&](int64_t i, int32_t sel, bool report) -> int32_t {
         if (i >= n_comp) return -1;
         int64_t v = i;
         if (sparse) {
-            v = topk[(size_t)vq * k + i];
+            v = sel;
             if (v >= n_vis) {
                 if (report) dev_error(err, CSLD_DEVERR_BAD_INDEX);
                 return -1;
@@ -274,63 +302,77 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
     } else if (warp < 4) {
         // ===== copies (warps 0-3): tile t into buffer t % kBufs, started before the query is ready =====
-        int t = 0;
+        // Whole tiles of consecutive compressed entries (or the full window ring) come as TMA
+        // boxes, one per column block.  Every other tile (selected entries, the tail, the window)
+        // is gathered with 16-byte cp.async copies: entry e's 36 chunks go to row e of the five
+        // column blocks (bytes 0..447 to blocks 0-3, bytes 448..575 to block 4), so a copy
+        // thread moves 27 chunks and the four warps fetch whole entries in order.  A gathered
+        // tile is published (fence to the async proxy, arrival on its full barrier) once the
+        // thread's copies of it have landed, checked after the next tile's copies are issued.
+        int t = 0, pend = -1;   // pend: the gathered tile whose arrivals are still owed
+        auto publish = [&](int wait_all) {
+            if (pend < 0) return;
+            if (wait_all) cp_async_wait<0>();
+            else cp_async_wait<1>();
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.full[pend % kBufs]);
+            pend = -1;
+        };
         for (; t < n_tiles; ++t) {
             const int s = t % kBufs;
+            const int64_t i0 = (t_begin + t) * kTcTile;
+            uint8_t* tl = sm.tile[s];
+            const bool box_comp = !sparse && i0 + kTcTile <= n_comp;
+            // the tile is the whole window and the ring is full: its W slots hold exactly those
+            // tokens (in ring order, which the softmax does not care about)
+            const bool box_win = W == kTcTile && Wr == W && n_win == W && i0 == n_comp4;
             const bool ok = !*fail && (t < kBufs || mbar_wait(&sm.empty[s], ((t / kBufs) - 1) & 1));
-            if (ok && tid == 0) mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
             if (named_barrier_or(kCopyBar, 128, !ok)) {   // the four copy warps leave together
+                publish(1);
                 if (tid == 0) *fail = 1;
                 break;
             }
-            const int64_t i0 = (t_begin + t) * kTcTile;
-            uint8_t* tl = sm.tile[s];
-            if (!sparse && i0 + kTcTile <= n_comp) {
-                // contiguous, all valid: one box per column block
-                if (tid < kBlk)
-                    tma_load_2d(tl + tid * kBlkBytes, &kv_tile, tid < 4 ? 128 * tid : kNope,
-                                static_cast<int>((int64_t)b * cap + i0), &sm.full[s]);
-            } else if (W == kTcTile && Wr == W && n_win == W && i0 == n_comp4) {
-                // the tile is the whole window and the ring is full: its W slots hold exactly
-                // those tokens (in ring order, which the softmax does not care about), so the
-                // ring itself comes in one box per column block
-                if (tid < kBlk)
-                    tma_load_2d(tl + tid * kBlkBytes, &win_tile, tid < 4 ? 128 * tid : kNope, b * W, &sm.full[s]);
-            } else {
-                // thread t: slots 4g .. 4g+3 (g = t / 4 < kTcTile / 4) of column block t % 4 (and
-                // block 4 when t % 4 == 0), from one of the two maps
-                const int g = tid >> 2, j = tid & 3;
-                const int64_t ib = i0 + 4 * g;
-                if (4 * g < kTcTile) {
-                const bool win = ib >= n_comp4 && ib < L;
-                int32_t y[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int64_t i = ib + r;
-                    if (!win) {
-                        const int32_t row = comp_row(i, j == 0);
-                        y[r] = row >= 0 ? row : oob_kv;
-                    } else if (i < L) {
-                        const int64_t tok = (int64_t)n - n_win + (i - n_comp4);
-                        y[r] = static_cast<int32_t>((int64_t)b * Wr + tok % Wr);
-                    } else {
-                        y[r] = oob_win;
-                    }
+            if (box_comp || box_win) {
+                publish(1);
+                if (tid == 0) mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+                else mbar_arrive(&sm.full[s]);
+                if (tid < kBlk) {
+                    const int x = tid < 4 ? 128 * tid : kNope;
+                    if (box_comp) tma_load_2d(tl + tid * kBlkBytes, &kv_tile, x, static_cast<int>((int64_t)b * cap + i0), &sm.full[s]);
+                    else tma_load_2d(tl + tid * kBlkBytes, &win_tile, x, b * W, &sm.full[s]);
                 }
-                const CUtensorMap* map = win ? &win_rows : &kv_rows;
-                tma_gather4(tl + j * kBlkBytes + 4 * g * 128, map, 128 * j, y[0], y[1], y[2], y[3], &sm.full[s]);
-                if (j == 0)
-                    tma_gather4(tl + kRopeBlk * kBlkBytes + 4 * g * 128, map, kNope, y[0], y[1], y[2], y[3], &sm.full[s]);
-                }
+                continue;
             }
+            if (tid < kTcTile) {   // entry tid's source row
+                const int64_t i = i0 + tid;
+                const uint8_t* src = nullptr;
+                if (i < n_comp4) {
+                    const int32_t row = comp_row(i, sel_of(i), true);
+                    if (row >= 0) src = comp_kv + (size_t)row * kEntry;
+                } else if (i < L && win_kv != nullptr) {
+                    const int64_t tok = (int64_t)n - n_win + (i - n_comp4);
+                    src = win_kv + ((size_t)b * Wr + (size_t)(tok % Wr)) * kEntry;
+                }
+                sm.src[tid] = src;
+            }
+            named_barrier(kCopyBar, 128);
+#pragma unroll 3
+            for (int g = tid; g < kTcTile * (kEntry / 16); g += 128) {
+                const int e = g / (kEntry / 16), c = g - e * (kEntry / 16);
+                const uint8_t* src = sm.src[e];
+                uint8_t* dst = c < 28 ? tl + (c >> 3) * kBlkBytes + sw128(e, 16 * (c & 7))
+                                      : tl + kRopeBlk * kBlkBytes + sw128(e, 16 * (c - 28));
+                cp_async16(dst, src ? src + 16 * c : comp_kv, src ? 16u : 0u);
+            }
+            cp_async_commit();
+            publish(0);   // the tile before, if it was gathered
+            pend = t;
         }
+        publish(1);
         if (tid == 0) sm.n_issued = t;
     } else if (warp >= 4 && warp < 8) {
-        // ===== the query operands (warps 4-15; the scales come from warps 8-15 first) ============
-        named_barrier(kScaleBar, 384);
-        qprep_convert(sm, q, vq, tid - 128);
-        tc_fence_before();
-        named_barrier(kReadyBar, 384);   // query operands written; tensor memory initialised
+        // ===== warps 4-7 wait for the query operands and tensor memory (written by warps 8-15) ====
+        named_barrier(kReadyBar, 384);
         tc_fence_after();
         if (warp == 4 && lane == 0) {
             // ===== MMA issue (one thread) =========================================================
@@ -403,14 +445,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         // ===== online softmax: thread = entry e = TMEM lane; head group hg = 8 heads =============
         const int sub = warp & 3, hg = (warp - 8) >> 2, e = 32 * sub + lane;
         const uint32_t lb = tmem + ((32u * sub) << 16);
-        qprep_scale(sm, q, vq, tid - 256, scale);
         if (hg == 0) {   // O = 0 and unit scale factors of V for this lane quarter
             for (uint32_t c = kColO; c < kColSFA; c += 8) tmem_st_32x32b_x8_fill(lb + c, 0u);
             tmem_st_32x32b_x8_fill(lb + kColSFA, 0x7F7F7F7Fu);
             tmem_st_wait();
         }
-        named_barrier(kScaleBar, 384);
-        qprep_convert(sm, q, vq, tid - 128);
+        qprep_store(sm, qv, tid - 256, scale);
         tc_fence_before();
         named_barrier(kReadyBar, 384);
         tc_fence_after();
@@ -425,7 +465,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         for (int t = 0; t < n_tiles; ++t) {
             const int s = t & 1;
             const int64_t i = (t_begin + t) * kTcTile + e;
-            const bool valid = e < kTcTile && (i < n_comp4 ? comp_row(i, false) >= 0 : i < L);
+            const bool valid = e < kTcTile && (i < n_comp4 ? comp_row(i, sel_of(i), false) >= 0 : i < L);
             ok = __all_sync(0xffffffffu, !*fail && mbar_wait(&sm.sfull[s], (t >> 1) & 1));
             float x[8];
             if (ok) {
@@ -457,13 +497,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
             }
             bool rescale = false;
             float mnew[8];
+            {
+                float tm[8];
 #pragma unroll
-            for (int h = 0; h < 8; ++h) {
-                const int hh = 8 * hg + h;
-                const float tm =
-                    fmaxf(fmaxf(sm.tmax[s][0][hh], sm.tmax[s][1][hh]), fmaxf(sm.tmax[s][2][hh], sm.tmax[s][3][hh]));
-                mnew[h] = (tm > mref[h] + kRescaleLog2 || mref[h] == -INFINITY) ? fmaxf(tm, mref[h]) : mref[h];
-                rescale |= (mnew[h] != mref[h]) && (mref[h] != -INFINITY);
+                for (int q4 = 0; q4 < 4; ++q4) {   // the four quarters' maxima of this warp's 8 heads
+                    const float4 a = *reinterpret_cast<const float4*>(&sm.tmax[s][q4][8 * hg]);
+                    const float4 c = *reinterpret_cast<const float4*>(&sm.tmax[s][q4][8 * hg + 4]);
+                    const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) tm[h] = q4 == 0 ? v[h] : fmaxf(tm[h], v[h]);
+                }
+#pragma unroll
+                for (int h = 0; h < 8; ++h) {
+                    mnew[h] = (tm[h] > mref[h] + kRescaleLog2 || mref[h] == -INFINITY) ? fmaxf(tm[h], mref[h]) : mref[h];
+                    rescale |= (mnew[h] != mref[h]) && (mref[h] != -INFINITY);
+                }
             }
             // P buffer s is free once PV(t-2) completed; a rescale of O also needs PV(t-1) done.
             // One barrier in the common case; a rescale or a failed wait anywhere takes two more.
@@ -480,10 +528,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                 }
             }
             tc_fence_after();
-            if (rescale) {   // this warp's 8 heads in every O block of its lane quarter
+            if (rescale) {   // l, and this warp's 8 heads in every O block of its lane quarter
                 float f[8];
 #pragma unroll
-                for (int h = 0; h < 8; ++h) f[h] = (mref[h] == -INFINITY) ? 1.f : exp2f(mref[h] - mnew[h]);
+                for (int h = 0; h < 8; ++h) {
+                    f[h] = (mref[h] == -INFINITY || mref[h] == mnew[h]) ? 1.f : exp2_ftz(mref[h] - mnew[h]);
+                    lsum[h] *= f[h];
+                }
 #pragma unroll 1
                 for (int blk = 0; blk < 4; ++blk) {
                     tmem_scale8(lb + kColO + 32u * blk + 8u * hg, f);
@@ -493,26 +544,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                 tmem_st_wait();
             }
             // P: two E4M3 terms after a power-of-two scale per (32-entry block = this lane
-            // quarter, head), and bf16 for the RoPE dims
+            // quarter, head), and bf16 for the RoPE dims.  Heads go in pairs through the paired
+            // converts.  A head that has seen no visible entry yet (m = -inf) has p = 0.
             uint8_t* p8 = sm.p8[s];
+            uint8_t* pb = sm.pbf[s][e >> 6];
 #pragma unroll
-            for (int h = 0; h < 8; ++h) {
+            for (int h = 0; h < 8; h += 2) {
                 const int hh = 8 * hg + h;
-                if (mref[h] != -INFINITY) lsum[h] *= exp2f(mref[h] - mnew[h]);
                 mref[h] = mnew[h];
-                const float p = (x[h] == -INFINITY) ? 0.f : exp2f(x[h] - mref[h]);
-                lsum[h] += p;
-                const uint32_t pm = __reduce_max_sync(0xffffffffu, __float_as_uint(p));   // p >= 0
+                mref[h + 1] = mnew[h + 1];
+                const float p0 = mref[h] == -INFINITY ? 0.f : exp2_ftz(x[h] - mref[h]);
+                const float p1 = mref[h + 1] == -INFINITY ? 0.f : exp2_ftz(x[h + 1] - mref[h + 1]);
+                lsum[h] += p0;
+                lsum[h + 1] += p1;
+                const uint32_t pm0 = __reduce_max_sync(0xffffffffu, __float_as_uint(p0));   // p >= 0
+                const uint32_t pm1 = __reduce_max_sync(0xffffffffu, __float_as_uint(p1));
                 // ks = 7 - floor(log2 max p): the scaled block stays below 256
-                const int ks = pm >= 0x00800000u ? max(-126, min(127, 134 - static_cast<int>(pm >> 23))) : 0;
-                const float xs = p * pow2f(ks);
-                const uint32_t hi = f32_to_e4m3(xs);
-                const uint32_t lo = f32_to_e4m3(xs - e4m3_to_f32(hi));
+                const int ks0 = pm0 >= 0x00800000u ? max(-126, min(127, 134 - static_cast<int>(pm0 >> 23))) : 0;
+                const int ks1 = pm1 >= 0x00800000u ? max(-126, min(127, 134 - static_cast<int>(pm1 >> 23))) : 0;
+                const float xs0 = p0 * pow2f(ks0), xs1 = p1 * pow2f(ks1);
+                const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(xs0, xs1), __NV_SATFINITE, __NV_E4M3);
+                const uint32_t back = e4m3x2_to_f16x2(hi);   // exact
+                const float r0 = xs0 - __half2float(__ushort_as_half(static_cast<unsigned short>(back & 0xFFFFu)));
+                const float r1 = xs1 - __half2float(__ushort_as_half(static_cast<unsigned short>(back >> 16)));
+                const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
+                const uint32_t pbf2 = f32x2_to_bf16x2_bits(p0, p1);
                 p8[sw128(hh, e)] = static_cast<uint8_t>(hi);
+                p8[sw128(hh + 1, e)] = static_cast<uint8_t>(hi >> 8);
                 p8[sw128(16 + hh, e)] = static_cast<uint8_t>(lo);
-                *reinterpret_cast<uint16_t*>(sm.pbf[s][e >> 6] + sw128(hh, 2 * (e & 63))) =
-                    static_cast<uint16_t>(f32_to_bf16_bits(p));
-                if (lane == h) sm.sfb[s][sub][hh] = static_cast<uint32_t>(127 - ks);
+                p8[sw128(17 + hh, e)] = static_cast<uint8_t>(lo >> 8);
+                *reinterpret_cast<uint16_t*>(pb + sw128(hh, 2 * (e & 63))) = static_cast<uint16_t>(pbf2);
+                *reinterpret_cast<uint16_t*>(pb + sw128(hh + 1, 2 * (e & 63))) = static_cast<uint16_t>(pbf2 >> 16);
+                if (lane == h) sm.sfb[s][sub][hh] = static_cast<uint32_t>(127 - ks0);
+                if (lane == h + 1) sm.sfb[s][sub][hh + 1] = static_cast<uint32_t>(127 - ks1);
             }
             fence_proxy_async_smem();
             named_barrier(kSmBar, 256);
@@ -603,17 +667,16 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
                                         const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                                         const int32_t* seq_len, int B, float scale, int splits, float* opart,
                                         float2* mlpart, int32_t* err, cudaStream_t stream) {
-    // the caches as 2-D byte tensors [rows][576]: 128-byte boxes with the 128-byte swizzle, 128
-    // rows tall (box copies of contiguous tiles) or one row (the gather4 form).  B cache rows,
-    // each serving Q query rows; the window ring has Wr >= W slots per cache row.
-    CUtensorMap kv_tile, kv_rows, win_rows, win_tile;
+    // the caches as 2-D byte tensors [rows][576] for the box copies of whole tiles: 128-byte
+    // boxes with the 128-byte swizzle, kTcTile rows tall.  B cache rows, each serving Q query
+    // rows; the window ring has Wr >= W slots per cache row.  Gathered tiles read the caches
+    // through the plain pointers.
+    CUtensorMap kv_tile, win_tile;
     const uint64_t rows = (uint64_t)B * (uint64_t)cap;
-    if (!make_tensor_map_2d_u8(&kv_tile, comp_kv, kEntry, rows, 128, kTcTile) ||
-        !make_tensor_map_2d_u8(&kv_rows, comp_kv, kEntry, rows, 128, 1))
-        return cudaErrorInvalidValue;
-    // a window-less call still passes a valid map (the compressed cache; never read)
+    if (!make_tensor_map_2d_u8(&kv_tile, comp_kv, kEntry, rows, 128, kTcTile)) return cudaErrorInvalidValue;
     const bool has_win = W > 0 && win_kv != nullptr;
-    if (!make_tensor_map_2d_u8(&win_rows, has_win ? win_kv : comp_kv, kEntry, has_win ? (uint64_t)B * Wr : rows, 128, 1))
+    // the gathers copy 16-byte chunks of 576-byte entries
+    if ((reinterpret_cast<uintptr_t>(comp_kv) & 15) != 0 || (has_win && (reinterpret_cast<uintptr_t>(win_kv) & 15) != 0))
         return cudaErrorInvalidValue;
     // a full ring of kTcTile slots as one tile (only used when W == Wr == kTcTile)
     const bool win_box = has_win && W == kTcTile && Wr == W;
@@ -623,8 +686,8 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
     const size_t smem = attention_tc_smem_bytes();
     cudaError_t e = set_smem_once(attention_tc_partial_kernel, smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attention_tc_partial_kernel, dim3(splits, B * Q), dim3(kTcThreads), smem, stream, kv_tile, kv_rows,
-                   win_rows, win_tile, q, cap, ratio, topk, k, W, Wr, Q, seq_len,
+    e = launch_pdl(attention_tc_partial_kernel, dim3(splits, B * Q), dim3(kTcThreads), smem, stream, kv_tile, win_tile,
+                   comp_kv, has_win ? win_kv : nullptr, q, cap, ratio, topk, k, W, Wr, Q, seq_len,
                    scale, splits, opart, mlpart, err);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -151,6 +151,21 @@ __device__ __forceinline__ uint32_t f32_to_bf16_bits(float x) {
     return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(x)));
 }
 
+// (a, b) -> bf16 bits (low half = a), round to nearest even.
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2_bits(float a, float b) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 2^x by the hardware approximation with subnormal results flushed to zero (ex2.approx.ftz).
+// Used for softmax weights relative to a running maximum, where anything below 2^-126 is
+// negligible; 2^-inf = +0.
+__device__ __forceinline__ float exp2_ftz(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
     return __uint_as_float((h & 0xFFFFu) << 16);
 }
