@@ -223,7 +223,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     // query row vq = cache row b times Q + the query's place jq among the Q newest tokens
     const int vq = blockIdx.y, split = blockIdx.x;
     const int b = vq / Q, jq = vq % Q;
-    const int B = gridDim.y / Q;
 
     // ---- setup --------------------------------------------------------------------------------
     if (tid == 0) {

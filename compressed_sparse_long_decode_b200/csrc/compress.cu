@@ -53,6 +53,27 @@ __device__ __forceinline__ void warp_pool_weights(const float* gate, const float
     for (int i = 0; i < 4; ++i) w[i] = e[i] / s;
 }
 
+// The same weights for m <= 32 from values the caller loaded ahead: lane l < m passes
+// gate[l] + bias[l] in a0.  The operations and their order are those of warp_pool_weights (its
+// slots past lane 31 contribute -inf to the maximum and 0 to the sum), so the weights are
+// bit-identical to it.
+__device__ __forceinline__ void warp_pool_weights_pre(float a0, int m, int lane, float (&w)[4]) {
+    float a[4] = {lane < m ? a0 : -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    float mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float e[4], s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        e[i] = (lane + 32 * i < m) ? expf(a[i] - mx) : 0.f;
+        s += e[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = e[i] / s;
+}
+
 template <bool kReadOnly>
 __device__ __forceinline__ void warp_pool(const uint16_t* rows, const float* gate,
                                           const float* __restrict__ bias, int m, int lane,
@@ -224,11 +245,19 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
         tmem_alloc(&sm.tmem_base, kCTmemCols);
         tmem_relinquish();
     }
-    // W_I^T in bf16, resident for the CTA's lifetime
-    for (int i = tid; i < kDim * kIdxDim; i += kCThreads) {
-        const int k = i / kIdxDim, n = i % kIdxDim;
-        *reinterpret_cast<uint16_t*>(&sm.w[k >> 6][sw128(n, 2 * (k & 63))]) =
-            static_cast<uint16_t>(f32_to_bf16_bits(__ldg(w_idx + i)));
+    // W_I^T in bf16, resident for the CTA's lifetime; 32 loads per thread in flight at a time
+    constexpr int kWBatch = 32;
+    for (int i0 = 0; i0 < kDim * kIdxDim; i0 += kWBatch * kCThreads) {
+        float v[kWBatch];
+#pragma unroll
+        for (int u = 0; u < kWBatch; ++u) v[u] = __ldg(w_idx + i0 + u * kCThreads + tid);
+#pragma unroll
+        for (int u = 0; u < kWBatch; ++u) {
+            const int i = i0 + u * kCThreads + tid;
+            const int k = i / kIdxDim, n = i % kIdxDim;
+            *reinterpret_cast<uint16_t*>(&sm.w[k >> 6][sw128(n, 2 * (k & 63))]) =
+                static_cast<uint16_t>(f32_to_bf16_bits(v[u]));
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -239,6 +268,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
 
     const int64_t tiles_per_seq = (E + kCTile - 1) / kCTile;
     const int64_t n_tiles = tiles_per_seq * B;
+    const float bias_l = (kM4 && lane < 4) ? __ldg(bias + lane) : 0.f;   // slot l's positional bias
     uint32_t phase = 0;
     bool mma_pending = false;   // an MMA reading sm.a was issued and this warp has not seen it end
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
@@ -255,11 +285,17 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
             // registers for the shared-memory operand to be free
             uint32_t packed[kRif][8];
             if constexpr (kM4) {
+                // the rows and their gates of kRif entries in flight together
                 uint4 x[kRif][8];
+                float ga[kRif];
 #pragma unroll
                 for (int h = 0; h < kRif; ++h) {
                     const int r = r0 + h * kWarps;
-                    if (r < n_here) load_block4(rb + (size_t)(s0 + r) * 4 * kDim, lane, x[h]);
+                    ga[h] = 0.f;
+                    if (r < n_here) {
+                        load_block4(rb + (size_t)(s0 + r) * 4 * kDim, lane, x[h]);
+                        if (lane < 4) ga[h] = __ldg(gb + (s0 + r) * 4 + lane);
+                    }
                 }
 #pragma unroll
                 for (int h = 0; h < kRif; ++h) {
@@ -267,7 +303,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                     float c[16];
                     if (r < n_here) {
                         float w[4];
-                        warp_pool_weights(gb + (s0 + r) * 4, bias, 4, lane, w);
+                        warp_pool_weights_pre(ga[h] + bias_l, 4, lane, w);
                         pool4_preloaded(x[h], w, c);
                         warp_store_entry(kvb + (size_t)(s0 + r) * kEntry, lane, c);
                     } else {
