@@ -14,7 +14,7 @@ namespace csld {
 // stage.cu
 cudaError_t launch_stage(void* dst, const void* src, size_t bytes, int num_sms, cudaStream_t stream);
 // indexer_multi.cu
-size_t indexer_multi_ws_bytes(int B, int Q, int64_t cap);
+size_t indexer_multi_ws_bytes(int B, int Q, int64_t cap, int num_sms);
 cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
                                  int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
                                  int32_t* topk_out, void* ws, int num_sms, int32_t* err, cudaStream_t stream);
@@ -320,7 +320,7 @@ csld_status csld_lse_merge(const float* outs, const float* lses, int R, int B, i
 
 size_t csld_indexer_multi_workspace_size(int B, int Q, int64_t cap) {
     if (B < 1 || Q < 1 || Q > CSLD_MULTI_MAX_Q || cap < 1) return 0;
-    return csld::indexer_multi_ws_bytes(B, Q, cap);
+    return csld::indexer_multi_ws_bytes(B, Q, cap, num_sms());
 }
 
 csld_status indexer_topk_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
@@ -335,7 +335,7 @@ csld_status indexer_topk_multi(const uint8_t* ikeys, const float* iscales, int64
     if (!ikeys || !iscales || !seq_len || !q_idx || !head_w || !topk_out)
         return fail(CSLD_ERR_ARG, "a required pointer is NULL");
     if (!aligned16(ikeys) || !aligned16(iscales)) return fail(CSLD_ERR_ALIGN, "ikeys / iscales must be 16-byte aligned");
-    const size_t need = csld::indexer_multi_ws_bytes(B, Q, cap);
+    const size_t need = csld::indexer_multi_ws_bytes(B, Q, cap, num_sms());
     if (!ws || ws_bytes < need) return fail(CSLD_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CSLD_ERR_ALIGN, "workspace must be 256-byte aligned");
     cudaError_t e = csld::launch_indexer_multi(ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, B, Q, k, topk_out,

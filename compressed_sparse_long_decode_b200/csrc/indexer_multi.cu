@@ -20,11 +20,14 @@
 //    (thread = entry), form every query's fp32 score and write its order key to the workspace,
 //    and add the keys' top 11 bits to per-query histograms, which the CTA adds into global ones
 //    at the end.
-// 2. indexer_multi_select_kernel -- one CTA per (sequence, query): the threshold bin from the
-//    global histogram, the keys of that bin and above gathered into shared memory in index
-//    order by one pass, two more radix levels (11 + 10 bits) there, then the entries in index
-//    order: every key above the threshold and the first ones equal to it.  It zeroes the
-//    histogram it used, so the workspace stays ready for the next call.
+// 2. indexer_multi_gather_kernel -- P CTAs per (sequence, query), each over one contiguous part
+//    of the query's keys: the threshold bin from the global histogram, then the keys of that bin
+//    and above, with their indices, compacted in index order into the part's candidate list.
+// 3. indexer_multi_select_kernel -- one CTA per (sequence, query): the P lists, concatenated in
+//    part order (so still in index order), go to shared memory; two more radix levels
+//    (11 + 10 bits) there, then the entries in index order: every key above the threshold and
+//    the first ones equal to it.  It zeroes the histogram it used, so the workspace stays ready
+//    for the next call.
 #include "csld_internal.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -364,11 +367,87 @@ struct MqSelSmem {
     uint32_t red[96];
 };
 
+// Grid (P, Q, B), 1024 threads: part p of query q of sequence b.  The query's keys are walked in
+// steps of kMqSelThreads * kMqPer; part p takes steps [S p / P, S (p + 1) / P).  Keys of the
+// threshold bin and above go to the part's list as (key, index) in index order; the count goes
+// to counts.  When the candidates of the whole query would not fit in the select kernel's shared
+// memory (heavy ties) nothing is gathered: the select kernel then reads the keys itself.
+struct MqGatherSmem {
+    uint32_t h[kMqBins];
+    uint32_t sel[4];
+    uint32_t red[96];
+};
+__global__ void __launch_bounds__(kMqSelThreads) indexer_multi_gather_kernel(const uint32_t* __restrict__ keys,
+                                                                             int64_t cap,
+                                                                             const int32_t* __restrict__ seq_len,
+                                                                             int ratio, int Q, int k, int P,
+                                                                             const uint32_t* __restrict__ ghist,
+                                                                             uint2* __restrict__ lists,
+                                                                             uint32_t* __restrict__ counts) {
+    __shared__ MqGatherSmem sm;
+    const int p = blockIdx.x, q = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    int32_t n = seq_len[b];
+    if (n < 0) n = 0;
+    const int64_t pos1 = (int64_t)n - Q + q + 1;
+    const int64_t n_q = pos1 > 0 ? min64(pos1 / ratio, cap) : 0;
+    const size_t row = (size_t)b * Q + q;
+    if (n_q <= k) return;   // the select kernel lists every visible entry
+    const uint32_t* gh = ghist + row * kMqBins;
+    for (int i = tid; i < kMqBins; i += blockDim.x) sm.h[i] = __ldcg(gh + i);
+    __syncthreads();
+    mq_find_bin(sm.h, kMqBins, static_cast<uint32_t>(k), sm.sel);
+    const uint32_t b1 = sm.sel[0], need1 = sm.sel[1];
+    if (static_cast<uint32_t>(k) - need1 + sm.h[b1] > static_cast<uint32_t>(kMqCand)) return;
+    const uint32_t lo1 = b1 << 21;
+    const uint32_t* kq = keys + row * cap;
+    const int64_t pcap = min64(kMqCand, cap);   // a part's list holds at most this many
+    uint2* list = lists + (row * P + p) * pcap;
+    constexpr int64_t kStep = (int64_t)kMqSelThreads * kMqPer;
+    const int64_t steps = (n_q + kStep - 1) / kStep;
+    const int64_t i_lo = steps * p / P * kStep, i_hi = min64(steps * (p + 1) / P * kStep, n_q);
+    const bool vec = ((reinterpret_cast<uintptr_t>(kq) & 15u) == 0);
+    uint32_t n_c = 0u;
+    for (int64_t base = i_lo; base < i_hi; base += kStep) {
+        const int64_t i0 = base + (int64_t)tid * kMqPer;
+        uint32_t v[kMqPer];
+        if (vec && i0 + kMqPer <= i_hi) {
+#pragma unroll
+            for (int j = 0; j < kMqPer / 4; ++j) {
+                const uint4 x = __ldcg(reinterpret_cast<const uint4*>(kq + i0) + j);
+                v[4 * j] = x.x;
+                v[4 * j + 1] = x.y;
+                v[4 * j + 2] = x.z;
+                v[4 * j + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < kMqPer; ++j) v[j] = i0 + j < i_hi ? __ldcg(kq + i0 + j) : 0u;
+        }
+        uint32_t cnt = 0u;
+#pragma unroll
+        for (int j = 0; j < kMqPer; ++j) cnt += (i0 + j < i_hi && v[j] >= lo1) ? 1u : 0u;
+        uint32_t tot;
+        uint32_t at = n_c + mq_block_scan(cnt, sm.red, &tot);
+#pragma unroll
+        for (int j = 0; j < kMqPer; ++j)
+            if (i0 + j < i_hi && v[j] >= lo1) {
+                if (at < static_cast<uint32_t>(pcap)) list[at] = make_uint2(v[j], static_cast<uint32_t>(i0 + j));
+                ++at;
+            }
+        n_c += tot;
+    }
+    if (tid == 0) counts[row * P + p] = min(n_c, static_cast<uint32_t>(pcap));
+}
+
 __global__ void __launch_bounds__(kMqSelThreads) indexer_multi_select_kernel(const uint32_t* __restrict__ keys,
                                                                              int64_t cap,
                                                                              const int32_t* __restrict__ seq_len,
-                                                                             int ratio, int Q, int k,
+                                                                             int ratio, int Q, int k, int P,
                                                                              uint32_t* __restrict__ ghist,
+                                                                             const uint2* __restrict__ lists,
+                                                                             const uint32_t* __restrict__ counts,
                                                                              int32_t* __restrict__ topk_out) {
     extern __shared__ __align__(16) uint8_t sel_raw[];
     MqSelSmem& sm = *reinterpret_cast<MqSelSmem*>(sel_raw);
@@ -401,46 +480,43 @@ __global__ void __launch_bounds__(kMqSelThreads) indexer_multi_select_kernel(con
     const uint32_t in1 = h[b1];                                  // keys in it
     __syncthreads();
     const bool in_smem = above1 + in1 <= static_cast<uint32_t>(kMqCand);
-    // ---- gather the keys of bin >= b1 in index order (when they fit) ------------------------
-    const uint32_t lo1 = b1 << 21;
+    // ---- the keys of bin >= b1 in index order (when they fit): the parts' lists, in order ------
     uint32_t n_c = 0u;
     if (in_smem) {
-        // n_q keys: thread t reads keys base + 16 t .. base + 16 t + 15 (four 16-byte loads when
-        // the row start allows it)
-        const bool vec = ((reinterpret_cast<uintptr_t>(kq) & 15u) == 0);
-        for (int64_t base = 0; base < n_q; base += (int64_t)kMqSelThreads * kMqPer) {
-            const int64_t i0 = base + (int64_t)tid * kMqPer;
-            uint32_t v[kMqPer];
-            if (vec && i0 + kMqPer <= n_q) {
-#pragma unroll
-                for (int j = 0; j < kMqPer / 4; ++j) {
-                    const uint4 x = __ldcg(reinterpret_cast<const uint4*>(kq + i0) + j);
-                    v[4 * j] = x.x;
-                    v[4 * j + 1] = x.y;
-                    v[4 * j + 2] = x.z;
-                    v[4 * j + 3] = x.w;
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < kMqPer; ++j) v[j] = i0 + j < n_q ? __ldcg(kq + i0 + j) : 0u;
+        const size_t row = (size_t)b * Q + q;
+        if (tid < P) red[32 + tid] = __ldcg(counts + row * P + tid);
+        __syncthreads();
+        if (tid == 0) {   // red[pp] = where part pp's keys start; red[P] = all
+            uint32_t acc = 0u;
+            for (int pp = 0; pp < P; ++pp) {
+                red[pp] = acc;
+                acc += red[32 + pp];
             }
-            uint32_t cnt = 0u;
-#pragma unroll
-            for (int j = 0; j < kMqPer; ++j) cnt += (i0 + j < n_q && v[j] >= lo1) ? 1u : 0u;
-            uint32_t tot;
-            uint32_t at = n_c + mq_block_scan(cnt, red, &tot);
-#pragma unroll
-            for (int j = 0; j < kMqPer; ++j)
-                if (i0 + j < n_q && v[j] >= lo1) {
-                    if (at < static_cast<uint32_t>(kMqCand)) {   // holds whenever the histogram is exact
-                        sm.ckey[at] = v[j];
-                        sm.cidx[at] = static_cast<uint32_t>(i0 + j);
-                    }
-                    ++at;
-                }
-            n_c += tot;
+            red[P] = acc;
         }
-        n_c = min(n_c, static_cast<uint32_t>(kMqCand));
+        __syncthreads();
+        n_c = min(red[P], static_cast<uint32_t>(kMqCand));   // equal whenever the histogram is exact
+        for (uint32_t j0 = 0; j0 < n_c; j0 += 4u * kMqSelThreads) {
+            uint2 e[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t j = j0 + u * kMqSelThreads + tid;
+                e[u] = make_uint2(0u, 0u);
+                if (j < n_c) {
+                    int pp = 0;
+                    while (pp + 1 < P && red[pp + 1] <= j) ++pp;
+                    e[u] = __ldcg(lists + (row * P + pp) * min64(kMqCand, cap) + (j - red[pp]));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t j = j0 + u * kMqSelThreads + tid;
+                if (j < n_c) {
+                    sm.ckey[j] = e[u].x;
+                    sm.cidx[j] = e[u].y;
+                }
+            }
+        }
         __syncthreads();
     }
     // ---- levels 2 (bits 20..10) and 3 (bits 9..0) inside bin b1 --------------------------------
@@ -500,17 +576,32 @@ __global__ void __launch_bounds__(kMqSelThreads) indexer_multi_select_kernel(con
 
 size_t indexer_multi_smem_bytes() { return sizeof(MqSmem) + 1024; }
 
-size_t indexer_multi_ws_bytes(int B, int Q, int64_t cap) {
-    const size_t keys = (size_t)B * Q * (size_t)cap * 4;
-    return (keys + 255) / 256 * 256 + (size_t)B * Q * kMqBins * 4;
+// Parts per (sequence, query) of the gather: about one CTA per SM in all, at most 16.
+int indexer_multi_parts(int B, int Q, int num_sms) {
+    const int rows = max(B * Q, 1);
+    return max(1, min(16, num_sms / rows));
+}
+
+// Workspace: the order keys [B][Q][cap], the histograms [B][Q][2048], the parts' candidate
+// counts [B][Q][P] and lists [B][Q][P][min(kMqCand, cap)] of (key, index).
+size_t indexer_multi_ws_bytes(int B, int Q, int64_t cap, int num_sms) {
+    const size_t rows = (size_t)B * Q, P = (size_t)indexer_multi_parts(B, Q, num_sms);
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    return up(rows * (size_t)cap * 4) + up(rows * kMqBins * 4) + up(rows * P * 4) +
+           rows * P * (size_t)min64(kMqCand, cap) * sizeof(uint2);
 }
 
 cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
                                  int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
                                  int32_t* topk_out, void* ws, int num_sms, int32_t* err, cudaStream_t stream) {
-    uint32_t* keys = static_cast<uint32_t*>(ws);
-    uint32_t* ghist = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ((size_t)B * Q * (size_t)cap * 4 + 255) /
-                                                                                   256 * 256);
+    const int P = indexer_multi_parts(B, Q, num_sms);
+    const size_t rows = (size_t)B * Q;
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(w8);
+    uint32_t* ghist = reinterpret_cast<uint32_t*>(w8 + up(rows * (size_t)cap * 4));
+    uint32_t* counts = reinterpret_cast<uint32_t*>(w8 + up(rows * (size_t)cap * 4) + up(rows * kMqBins * 4));
+    uint2* lists = reinterpret_cast<uint2*>(w8 + up(rows * (size_t)cap * 4) + up(rows * kMqBins * 4) + up(rows * P * 4));
     const size_t smem = indexer_multi_smem_bytes();
     cudaError_t e = set_smem_once(indexer_multi_score_kernel, smem);
     if (e != cudaSuccess) return e;
@@ -521,10 +612,15 @@ cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int
     e = launch_pdl(indexer_multi_score_kernel, dim3(static_cast<unsigned>(chunks), B), dim3(kMqThreads), smem, stream,
                    ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, Q, keys, ghist, err);
     if (e != cudaSuccess) return e;
+    e = launch_pdl(indexer_multi_gather_kernel, dim3(P, Q, B), dim3(kMqSelThreads), 0, stream,
+                   static_cast<const uint32_t*>(keys), cap, seq_len, ratio, Q, k, P,
+                   static_cast<const uint32_t*>(ghist), lists, counts);
+    if (e != cudaSuccess) return e;
     e = set_smem_once(indexer_multi_select_kernel, sizeof(MqSelSmem));
     if (e != cudaSuccess) return e;
     e = launch_pdl(indexer_multi_select_kernel, dim3(Q, B), dim3(kMqSelThreads), sizeof(MqSelSmem), stream,
-                   static_cast<const uint32_t*>(keys), cap, seq_len, ratio, Q, k, ghist, topk_out);
+                   static_cast<const uint32_t*>(keys), cap, seq_len, ratio, Q, k, P, ghist,
+                   static_cast<const uint2*>(lists), static_cast<const uint32_t*>(counts), topk_out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
