@@ -53,6 +53,8 @@ struct MqSmem {
     float scales[kMqStages][kMqGroup * 2];          // 8 KB per group
     alignas(256) uint8_t bq[8 * CSLD_MULTI_MAX_Q * kIkey];   // query operand, 32-byte swizzle
     float qscale[CSLD_MULTI_MAX_Q][8];              // [q][group * 4 + head]
+    float hw[CSLD_MULTI_MAX_Q][kIdxHeads];          // head weights of each query
+    int64_t nq[CSLD_MULTI_MAX_Q];                   // entries query q sees
     uint32_t hist[CSLD_MULTI_MAX_Q][kMqBins];
     uint64_t full[kMqStages], gfree[kMqStages], accf[kMqSlots], sfree[kMqSlots], drain;
     uint32_t tmem_base;
@@ -105,6 +107,12 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
     }
     // the newest query sees the most entries; query q sees n_q of them
     const int64_t n_max = min64(n / ratio, cap);
+    if (tid < Q) {
+        sm.nq[tid] = min64((int64_t)(n - Q + tid + 1) / ratio, cap);
+#pragma unroll
+        for (int h = 0; h < kIdxHeads; ++h) sm.hw[tid][h] = __ldg(head_w + ((size_t)b * Q + tid) * kIdxHeads + h);
+    }
+    __syncthreads();
     const int n_tiles_all = static_cast<int>((n_max + kMqTile - 1) / kMqTile);
     // this CTA's tiles: whole copy groups g = c, c + chunks, ...
     const int n_groups_all = (n_tiles_all + kMqGroupTiles - 1) / kMqGroupTiles;
@@ -197,7 +205,6 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
         const int wg = warp >> 2, quad = warp & 3;
         const int m = 32 * quad + lane;
         const uint32_t lane_addr = tmem + ((32u * quad) << 16);
-        const float* hw = head_w + (size_t)b * Q * kIdxHeads;
         int t = 0;
         for (int i = 0; i < my_groups; ++i) {
             const int s = i % kMqStages;
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
                     for (int qq = 0; qq < 2; ++qq) {
                         const int q = q0 + qq;
                         if (q >= Q) break;
-                        const int64_t n_q = min64((int64_t)(n - Q + q + 1) / ratio, cap);
+                        const int64_t n_q = sm.nq[q];
                         float rr[4];
 #pragma unroll
                         for (int h = 0; h < 4; ++h) {
@@ -236,11 +243,11 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
                             const float d = __fmaf_rn(i1, s1, __fmul_rn(i0, s0));
                             rr[h] = d > 0.f ? d : 0.f;
                         }
-                        const float* w = hw + q * kIdxHeads;
-                        float sc = __fmul_rn(__ldg(w + 0), rr[0]);
-                        sc = __fmaf_rn(__ldg(w + 1), rr[1], sc);
-                        sc = __fmaf_rn(__ldg(w + 2), rr[2], sc);
-                        sc = __fmaf_rn(__ldg(w + 3), rr[3], sc);
+                        const float* w = sm.hw[q];
+                        float sc = __fmul_rn(w[0], rr[0]);
+                        sc = __fmaf_rn(w[1], rr[1], sc);
+                        sc = __fmaf_rn(w[2], rr[2], sc);
+                        sc = __fmaf_rn(w[3], rr[3], sc);
                         const uint32_t key = score_key(sc);
                         if (e < n_q) {
                             keys_out[((size_t)b * Q + q) * cap + (size_t)e] = key;
@@ -283,41 +290,6 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
 
 namespace {
 
-// The bin of nb bins (counts in smem h) holding the want-th largest key and how many keys are
-// wanted inside it.  Warp 0 computes; results in sel[0..1].  Block-wide (ends with a barrier).
-__device__ void mq_find_bin(const uint32_t* h, int nb, uint32_t want, uint32_t* sel) {
-    const int tid = threadIdx.x, lane = tid & 31;
-    if (tid < 32) {
-        if (lane == 0) {   // defaults if the counts fall short (an incomplete histogram)
-            sel[0] = 0u;
-            sel[1] = want;
-        }
-        __syncwarp();
-        const int per = nb / 32;                   // bins per lane, from the top
-        uint32_t tot = 0u;
-        for (int i = 0; i < per; ++i) tot += h[nb - 1 - per * lane - i];
-        uint32_t incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        const uint32_t excl = incl - tot;
-        if (excl < want && incl >= want) {
-            uint32_t run = excl;
-            for (int i = 0; i < per; ++i) {
-                const uint32_t cnt = h[nb - 1 - per * lane - i];
-                if (run + cnt >= want) {
-                    sel[0] = static_cast<uint32_t>(nb - 1 - per * lane - i);
-                    sel[1] = want - run;
-                    break;
-                }
-                run += cnt;
-            }
-        }
-    }
-    __syncthreads();
-}
 
 // Block-wide exclusive scan of v (1024 threads); *total = the sum.
 __device__ __forceinline__ uint32_t mq_block_scan(uint32_t v, uint32_t* red, uint32_t* total) {
@@ -346,6 +318,39 @@ __device__ __forceinline__ uint32_t mq_block_scan(uint32_t v, uint32_t* red, uin
     *total = red[64];
     __syncthreads();
     return r;
+}
+
+// The bin of nb bins (counts in smem h) holding the want-th largest key and how many keys are
+// wanted inside it, in sel[0..1] (bin 0 and want when the counts fall short: an incomplete
+// histogram).  The whole block (1024 threads; nb a multiple of it, at most 2 bins per thread):
+// thread t holds the bins at places per t .. per t + per - 1 from the top, and a block scan of
+// their counts finds the thread whose bins hold the want-th key.  Ends with a barrier.
+__device__ void mq_find_bin_block(const uint32_t* h, int nb, uint32_t want, uint32_t* red, uint32_t* sel) {
+    const int tid = threadIdx.x;
+    const int per = nb / static_cast<int>(blockDim.x);
+    uint32_t c[2] = {0u, 0u}, tot = 0u;
+    for (int j = 0; j < per; ++j) {
+        c[j] = h[nb - 1 - (per * tid + j)];
+        tot += c[j];
+    }
+    if (tid == 0) {   // defaults if the counts fall short (an incomplete histogram)
+        sel[0] = 0u;
+        sel[1] = want;
+    }
+    uint32_t total;
+    const uint32_t excl = mq_block_scan(tot, red, &total);
+    if (excl < want && excl + tot >= want) {
+        uint32_t run = excl;
+        for (int j = 0; j < per; ++j) {
+            if (run + c[j] >= want) {
+                sel[0] = static_cast<uint32_t>(nb - 1 - (per * tid + j));
+                sel[1] = want - run;
+                break;
+            }
+            run += c[j];
+        }
+    }
+    __syncthreads();
 }
 
 }  // namespace
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__(kMqSelThreads) indexer_multi_gather_kernel(con
     const uint32_t* gh = ghist + row * kMqBins;
     for (int i = tid; i < kMqBins; i += blockDim.x) sm.h[i] = __ldcg(gh + i);
     __syncthreads();
-    mq_find_bin(sm.h, kMqBins, static_cast<uint32_t>(k), sm.sel);
+    mq_find_bin_block(sm.h, kMqBins, static_cast<uint32_t>(k), sm.red, sm.sel);
     const uint32_t b1 = sm.sel[0], need1 = sm.sel[1];
     if (static_cast<uint32_t>(k) - need1 + sm.h[b1] > static_cast<uint32_t>(kMqCand)) return;
     const uint32_t lo1 = b1 << 21;
@@ -474,7 +479,7 @@ __global__ void __launch_bounds__(kMqSelThreads) indexer_multi_select_kernel(con
         return;
     }
     // level 1 (bits 31..21) from the scoring histogram
-    mq_find_bin(h, kMqBins, static_cast<uint32_t>(k), sel);
+    mq_find_bin_block(h, kMqBins, static_cast<uint32_t>(k), red, sel);
     const uint32_t b1 = sel[0], need1 = sel[1];
     const uint32_t above1 = static_cast<uint32_t>(k) - need1;   // keys above bin b1
     const uint32_t in1 = h[b1];                                  // keys in it
@@ -532,7 +537,7 @@ __global__ void __launch_bounds__(kMqSelThreads) indexer_multi_select_kernel(con
         }
     }
     __syncthreads();
-    mq_find_bin(h, kMqBins, need1, sel);
+    mq_find_bin_block(h, kMqBins, need1, red, sel);
     const uint32_t b2 = sel[0], need2 = sel[1];
     __syncthreads();
     for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
@@ -548,7 +553,7 @@ __global__ void __launch_bounds__(kMqSelThreads) indexer_multi_select_kernel(con
         }
     }
     __syncthreads();
-    mq_find_bin(h, 1024, need2, sel);
+    mq_find_bin_block(h, 1024, need2, red, sel);
     const uint32_t thr = (top22 << 10) | sel[0], take_eq = sel[1];
     __syncthreads();
     // ---- emit in index order: keys above the threshold, and the first take_eq equal to it -----
