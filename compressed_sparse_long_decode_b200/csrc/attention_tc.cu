@@ -50,9 +50,14 @@ namespace csld {
 
 namespace {
 
+// 16 warps: copies 0-3, MMA issue 4 (warps 5-7 only take part in the start-up barrier),
+// softmax 8-15
 constexpr int kTcThreads = 512;
+constexpr int kCopyThreads = 128;
+constexpr int kMmaWarp = 4;
 constexpr int kTcTile = 96;                   // entries per tile: K of PV, valid rows of QK (a multiple of 32)
 constexpr int kTcRows = 128;                  // rows of the QK MMA (M); rows past kTcTile are read, never used
+static_assert(kCopyThreads >= kTcTile, "each copy thread resolves at most one entry's source row");
 constexpr int kBufs = 3;                      // tile buffers: copies run up to two tiles ahead of PV
 constexpr int kKBlocks = kTcTile / 32;        // 32-entry K blocks of PV per tile (one P block scale each)
 constexpr int kBlk = 5;                       // 128-byte column blocks per entry
@@ -209,8 +214,50 @@ __device__ __forceinline__ void qprep_store(TcAttnSmem& sm, const uint4 (&v)[4],
     fence_proxy_async_smem();
 }
 
+// P of one tile for this thread's entry e and its head group's 8 heads against the maxima m
+// (log2 units): p = 2^(x - m), 0 for a head that has seen no visible entry yet (m = -inf).  P is
+// stored as two E4M3 terms after a power-of-two scale per (32-entry block = this lane quarter,
+// head) in the PV operand rows h and 16 + h, and as bf16 for the RoPE dims; the block scales go
+// to sfb[head].  Heads go in pairs through the paired converts.  The p of each head goes to
+// l: added (kAdd) or stored.
+template <bool kAdd>
+__device__ __forceinline__ void write_p(uint8_t* p8, uint8_t* pb, uint32_t* sfb, const float (&m)[8],
+                                       const float (&x)[8], float (&l)[8], int hg, int e, int lane) {
+#pragma unroll
+    for (int h = 0; h < 8; h += 2) {
+        const int hh = 8 * hg + h;
+        const float p0 = m[h] == -INFINITY ? 0.f : exp2_ftz(x[h] - m[h]);
+        const float p1 = m[h + 1] == -INFINITY ? 0.f : exp2_ftz(x[h + 1] - m[h + 1]);
+        l[h] = kAdd ? l[h] + p0 : p0;
+        l[h + 1] = kAdd ? l[h + 1] + p1 : p1;
+        const uint32_t pm0 = __reduce_max_sync(0xffffffffu, __float_as_uint(p0));   // p >= 0
+        const uint32_t pm1 = __reduce_max_sync(0xffffffffu, __float_as_uint(p1));
+        // ks = 7 - floor(log2 max p): the scaled block stays below 256
+        const int ks0 = pm0 >= 0x00800000u ? max(-126, min(127, 134 - static_cast<int>(pm0 >> 23))) : 0;
+        const int ks1 = pm1 >= 0x00800000u ? max(-126, min(127, 134 - static_cast<int>(pm1 >> 23))) : 0;
+        const float xs0 = p0 * pow2f(ks0), xs1 = p1 * pow2f(ks1);
+        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(xs0, xs1), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t back = e4m3x2_to_f16x2(hi);   // exact
+        const float r0 = xs0 - __half2float(__ushort_as_half(static_cast<unsigned short>(back & 0xFFFFu)));
+        const float r1 = xs1 - __half2float(__ushort_as_half(static_cast<unsigned short>(back >> 16)));
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t pbf2 = f32x2_to_bf16x2_bits(p0, p1);
+        p8[sw128(hh, e)] = static_cast<uint8_t>(hi);
+        p8[sw128(hh + 1, e)] = static_cast<uint8_t>(hi >> 8);
+        p8[sw128(16 + hh, e)] = static_cast<uint8_t>(lo);
+        p8[sw128(17 + hh, e)] = static_cast<uint8_t>(lo >> 8);
+        *reinterpret_cast<uint16_t*>(pb + sw128(hh, 2 * (e & 63))) = static_cast<uint16_t>(pbf2);
+        *reinterpret_cast<uint16_t*>(pb + sw128(hh + 1, 2 * (e & 63))) = static_cast<uint16_t>(pbf2 >> 16);
+        if (lane == h) sfb[hh] = static_cast<uint32_t>(127 - ks0);
+        if (lane == h + 1) sfb[hh + 1] = static_cast<uint32_t>(127 - ks1);
+    }
+}
+
 }  // namespace
 
+// kFast: tiles after a split's first try P against the running max first (worth it when splits
+// hold several tiles; a one-tile split runs the plain path).
+template <bool kFast>
 __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     const __grid_constant__ CUtensorMap kv_tile, const __grid_constant__ CUtensorMap win_tile,
     const uint8_t* __restrict__ comp_kv, const uint8_t* __restrict__ win_kv,
@@ -227,7 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     // ---- setup --------------------------------------------------------------------------------
     if (tid == 0) {
         for (int s = 0; s < kBufs; ++s) {
-            mbar_init(&sm.full[s], 128);   // one arrival per copy thread
+            mbar_init(&sm.full[s], kCopyThreads);   // one arrival per copy thread
             mbar_init(&sm.empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -242,7 +289,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         sm.n_landed = 0;
         fence_barrier_init();
     }
-    if (warp == 4) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -326,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
             // tokens (in ring order, which the softmax does not care about)
             const bool box_win = W == kTcTile && Wr == W && n_win == W && i0 == n_comp4;
             const bool ok = !*fail && (t < kBufs || mbar_wait(&sm.empty[s], ((t / kBufs) - 1) & 1));
-            if (named_barrier_or(kCopyBar, 128, !ok)) {   // the four copy warps leave together
+            if (named_barrier_or(kCopyBar, kCopyThreads, !ok)) {   // the copy warps leave together
                 publish(1);
                 if (tid == 0) *fail = 1;
                 break;
@@ -354,9 +401,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
                 }
                 sm.src[tid] = src;
             }
-            named_barrier(kCopyBar, 128);
+            named_barrier(kCopyBar, kCopyThreads);
 #pragma unroll 3
-            for (int g = tid; g < kTcTile * (kEntry / 16); g += 128) {
+            for (int g = tid; g < kTcTile * (kEntry / 16); g += kCopyThreads) {
                 const int e = g / (kEntry / 16), c = g - e * (kEntry / 16);
                 const uint8_t* src = sm.src[e];
                 uint8_t* dst = c < 28 ? tl + (c >> 3) * kBlkBytes + sw128(e, 16 * (c & 7))
@@ -373,7 +420,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         // ===== warps 4-7 wait for the query operands and tensor memory (written by warps 8-15) ====
         named_barrier(kReadyBar, 384);
         tc_fence_after();
-        if (warp == 4 && lane == 0) {
+        if (warp == kMmaWarp && lane == 0) {
             // ===== MMA issue (one thread) =========================================================
             const uint64_t dq = desc_sw128(sm.qk[0], 0), dqr = desc_sw128(sm.qr, 0);
             // Issue whatever is ready, PV first (it frees a tile buffer for the next copy):
@@ -483,102 +530,110 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
 #pragma unroll
                 for (int h = 0; h < 8; ++h) x[h] = -INFINITY;
             }
-            // tile max per head: warp max of order keys, published per lane quarter (two sets,
-            // alternating by tile, so the next tile's maxima never overwrite ones still read)
+            // Fast path: no entry of this tile lies more than 2^8 above the running max (the common
+            // case after a split's first tile), so P is formed against m as it stands and the
+            // softmax warps meet once, where they publish P.  Otherwise (a new maximum, the first
+            // tile, or a failed wait) the tile takes the full path: tile maxima, new m, O
+            // rescaled, P formed again.
+            bool over = true;
+            if constexpr (kFast) {
+                over = !ok;
 #pragma unroll
-            for (int h = 0; h < 8; ++h) {
-                const uint32_t km = __reduce_max_sync(0xffffffffu, score_key(x[h]));
-                if (lane == h) sm.tmax[s][sub][8 * hg + h] = order_key_to_float(km);
+                for (int h = 0; h < 8; ++h) over |= x[h] > mref[h] + kRescaleLog2;
+                // P buffer s is free once PV(t-2) completed
+                if (t >= 2 && !over) over = !mbar_wait(&sm.pdone[s], ((t >> 1) - 1) & 1);
             }
-            if (named_barrier_or(kSmBar, 256, !ok)) {   // maxima published; the warps leave together
+            // pass 0 (not on a split's first tile): P against the running max, kept when no warp
+            // saw a new maximum; pass 1: the full path
+            float ladd[8];
+            bool quit = false, kept = false;   // kept: the P of pass 0 stands
+            for (int pass = (kFast && t > 0) ? 0 : 1; pass < 2; ++pass) {
+                if (pass == 1) {
+                    // tile max per head: warp max of order keys, published per lane quarter (two sets,
+                    // alternating by tile, so the next tile's maxima never overwrite ones still read)
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        const uint32_t km = __reduce_max_sync(0xffffffffu, score_key(x[h]));
+                        if (lane == h) sm.tmax[s][sub][8 * hg + h] = order_key_to_float(km);
+                    }
+                    if (named_barrier_or(kSmBar, 256, !ok)) {   // maxima published; the warps leave together
+                        quit = true;
+                        break;
+                    }
+                    bool rescale = false;
+                    float mnew[8];
+                    {
+                        float tm[8];
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {   // the four quarters' maxima of this warp's 8 heads
+                            const float4 a = *reinterpret_cast<const float4*>(&sm.tmax[s][q4][8 * hg]);
+                            const float4 c = *reinterpret_cast<const float4*>(&sm.tmax[s][q4][8 * hg + 4]);
+                            const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+                            for (int h = 0; h < 8; ++h) tm[h] = q4 == 0 ? v[h] : fmaxf(tm[h], v[h]);
+                        }
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            mnew[h] = (tm[h] > mref[h] + kRescaleLog2 || mref[h] == -INFINITY) ? fmaxf(tm[h], mref[h]) : mref[h];
+                            rescale |= (mnew[h] != mref[h]) && (mref[h] != -INFINITY);
+                        }
+                    }
+                    // P buffer s is free once PV(t-2) completed; a rescale of O also needs PV(t-1) done
+                    // (two more barriers, taken only when some head must be rescaled or a wait failed).
+                    if (t >= 2) ok = mbar_wait(&sm.pdone[s], ((t >> 1) - 1) & 1);
+                    if (named_barrier_or(kSmBar, 256, rescale || !ok)) {
+                        if (named_barrier_or(kSmBar, 256, !ok)) {
+                            quit = true;
+                            break;
+                        }
+                        if (t >= 1) ok = mbar_wait(&sm.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1);
+                        if (named_barrier_or(kSmBar, 256, !ok)) {
+                            quit = true;
+                            break;
+                        }
+                    }
+                    tc_fence_after();
+                    if (rescale) {   // l, and this warp's 8 heads in every O block of its lane quarter
+                        float f[8];
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            f[h] = (mref[h] == -INFINITY || mref[h] == mnew[h]) ? 1.f : exp2_ftz(mref[h] - mnew[h]);
+                            lsum[h] *= f[h];
+                        }
+#pragma unroll 1
+                        for (int blk = 0; blk < 4; ++blk) {
+                            tmem_scale8(lb + kColO + 32u * blk + 8u * hg, f);
+                            tmem_scale8(lb + kColO + 32u * blk + 16u + 8u * hg, f);
+                        }
+                        tmem_scale8(lb + kColOR + 8u * hg, f);
+                        tmem_st_wait();
+                    }
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) mref[h] = mnew[h];
+                }
+                if (pass == 1)
+                    write_p<true>(sm.p8[s], sm.pbf[s][e >> 6], sm.sfb[s][sub], mref, x, lsum, hg, e, lane);
+                else if (kFast && !__any_sync(0xffffffffu, over))
+                    write_p<false>(sm.p8[s], sm.pbf[s][e >> 6], sm.sfb[s][sub], mref, x, ladd, hg, e, lane);
+                fence_proxy_async_smem();
+                // P published; after pass 0 the warps also learn whether any saw a new maximum
+                if (!kFast) {
+                    named_barrier(kSmBar, 256);
+                    break;
+                }
+                if (!named_barrier_or(kSmBar, 256, pass == 0 && over)) {
+                    kept = pass == 0;
+                    break;
+                }
+            }
+            if (quit) {
                 ok = false;
                 break;
             }
-            bool rescale = false;
-            float mnew[8];
-            {
-                float tm[8];
+            if (kFast && kept) {
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {   // the four quarters' maxima of this warp's 8 heads
-                    const float4 a = *reinterpret_cast<const float4*>(&sm.tmax[s][q4][8 * hg]);
-                    const float4 c = *reinterpret_cast<const float4*>(&sm.tmax[s][q4][8 * hg + 4]);
-                    const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) tm[h] = q4 == 0 ? v[h] : fmaxf(tm[h], v[h]);
-                }
-#pragma unroll
-                for (int h = 0; h < 8; ++h) {
-                    mnew[h] = (tm[h] > mref[h] + kRescaleLog2 || mref[h] == -INFINITY) ? fmaxf(tm[h], mref[h]) : mref[h];
-                    rescale |= (mnew[h] != mref[h]) && (mref[h] != -INFINITY);
-                }
+                for (int h = 0; h < 8; ++h) lsum[h] += ladd[h];
             }
-            // P buffer s is free once PV(t-2) completed; a rescale of O also needs PV(t-1) done.
-            // One barrier in the common case; a rescale or a failed wait anywhere takes two more.
-            if (t >= 2) ok = mbar_wait(&sm.pdone[s], ((t >> 1) - 1) & 1);
-            if (named_barrier_or(kSmBar, 256, rescale || !ok)) {
-                if (named_barrier_or(kSmBar, 256, !ok)) {
-                    ok = false;
-                    break;
-                }
-                if (t >= 1) ok = mbar_wait(&sm.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1);
-                if (named_barrier_or(kSmBar, 256, !ok)) {
-                    ok = false;
-                    break;
-                }
-            }
-            tc_fence_after();
-            if (rescale) {   // l, and this warp's 8 heads in every O block of its lane quarter
-                float f[8];
-#pragma unroll
-                for (int h = 0; h < 8; ++h) {
-                    f[h] = (mref[h] == -INFINITY || mref[h] == mnew[h]) ? 1.f : exp2_ftz(mref[h] - mnew[h]);
-                    lsum[h] *= f[h];
-                }
-#pragma unroll 1
-                for (int blk = 0; blk < 4; ++blk) {
-                    tmem_scale8(lb + kColO + 32u * blk + 8u * hg, f);
-                    tmem_scale8(lb + kColO + 32u * blk + 16u + 8u * hg, f);
-                }
-                tmem_scale8(lb + kColOR + 8u * hg, f);
-                tmem_st_wait();
-            }
-            // P: two E4M3 terms after a power-of-two scale per (32-entry block = this lane
-            // quarter, head), and bf16 for the RoPE dims.  Heads go in pairs through the paired
-            // converts.  A head that has seen no visible entry yet (m = -inf) has p = 0.
-            uint8_t* p8 = sm.p8[s];
-            uint8_t* pb = sm.pbf[s][e >> 6];
-#pragma unroll
-            for (int h = 0; h < 8; h += 2) {
-                const int hh = 8 * hg + h;
-                mref[h] = mnew[h];
-                mref[h + 1] = mnew[h + 1];
-                const float p0 = mref[h] == -INFINITY ? 0.f : exp2_ftz(x[h] - mref[h]);
-                const float p1 = mref[h + 1] == -INFINITY ? 0.f : exp2_ftz(x[h + 1] - mref[h + 1]);
-                lsum[h] += p0;
-                lsum[h + 1] += p1;
-                const uint32_t pm0 = __reduce_max_sync(0xffffffffu, __float_as_uint(p0));   // p >= 0
-                const uint32_t pm1 = __reduce_max_sync(0xffffffffu, __float_as_uint(p1));
-                // ks = 7 - floor(log2 max p): the scaled block stays below 256
-                const int ks0 = pm0 >= 0x00800000u ? max(-126, min(127, 134 - static_cast<int>(pm0 >> 23))) : 0;
-                const int ks1 = pm1 >= 0x00800000u ? max(-126, min(127, 134 - static_cast<int>(pm1 >> 23))) : 0;
-                const float xs0 = p0 * pow2f(ks0), xs1 = p1 * pow2f(ks1);
-                const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(xs0, xs1), __NV_SATFINITE, __NV_E4M3);
-                const uint32_t back = e4m3x2_to_f16x2(hi);   // exact
-                const float r0 = xs0 - __half2float(__ushort_as_half(static_cast<unsigned short>(back & 0xFFFFu)));
-                const float r1 = xs1 - __half2float(__ushort_as_half(static_cast<unsigned short>(back >> 16)));
-                const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
-                const uint32_t pbf2 = f32x2_to_bf16x2_bits(p0, p1);
-                p8[sw128(hh, e)] = static_cast<uint8_t>(hi);
-                p8[sw128(hh + 1, e)] = static_cast<uint8_t>(hi >> 8);
-                p8[sw128(16 + hh, e)] = static_cast<uint8_t>(lo);
-                p8[sw128(17 + hh, e)] = static_cast<uint8_t>(lo >> 8);
-                *reinterpret_cast<uint16_t*>(pb + sw128(hh, 2 * (e & 63))) = static_cast<uint16_t>(pbf2);
-                *reinterpret_cast<uint16_t*>(pb + sw128(hh + 1, 2 * (e & 63))) = static_cast<uint16_t>(pbf2 >> 16);
-                if (lane == h) sm.sfb[s][sub][hh] = static_cast<uint32_t>(127 - ks0);
-                if (lane == h + 1) sm.sfb[s][sub][hh + 1] = static_cast<uint32_t>(127 - ks1);
-            }
-            fence_proxy_async_smem();
-            named_barrier(kSmBar, 256);
             if (hg == 0) {   // block-scale word of row `lane` (rows h and 16 + h: head lane & 15)
                 const int hh = lane & 15;
                 const uint32_t wsf = sm.sfb[s][0][hh] | (sm.sfb[s][1][hh] << 8) | (sm.sfb[s][2][hh] << 16) |
@@ -644,7 +699,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     if (sm.fail) {
         // a bounded wait gave up: record it, let the copies and MMAs in flight finish (bounded),
         // publish nothing
-        if (warp == 4 && lane == 0) {
+        if (warp == kMmaWarp && lane == 0) {
             dev_error(err, CSLD_DEVERR_TIMEOUT);
             for (int t = sm.n_landed; t < sm.n_issued; ++t) (void)mbar_wait(&sm.full[t % kBufs], (t / kBufs) & 1);
             umma_commit(&sm.drain);
@@ -653,7 +708,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
         if (tid < kHeads) mlpart[part * kHeads + tid] = make_float2(-INFINITY, 0.f);
         __syncthreads();
     }
-    if (warp == 4) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -683,9 +738,14 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
                                win_box ? kTcTile : 1))
         return cudaErrorInvalidValue;
     const size_t smem = attention_tc_smem_bytes();
-    cudaError_t e = set_smem_once(attention_tc_partial_kernel, smem);
+    // splits of more than one tile take the first-try path (the longest list: k or cap entries,
+    // padded to a multiple of 4, plus the window)
+    const int64_t l_max = (((topk ? (int64_t)k : cap) + 3) & ~int64_t(3)) + W;
+    const int64_t tiles_per_split = ((l_max + kTcTile - 1) / kTcTile + splits - 1) / splits;
+    auto kernel = tiles_per_split > 1 ? attention_tc_partial_kernel<true> : attention_tc_partial_kernel<false>;
+    cudaError_t e = set_smem_once(kernel, smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attention_tc_partial_kernel, dim3(splits, B * Q), dim3(kTcThreads), smem, stream, kv_tile, win_tile,
+    e = launch_pdl(kernel, dim3(splits, B * Q), dim3(kTcThreads), smem, stream, kv_tile, win_tile,
                    comp_kv, has_win ? win_kv : nullptr, q, cap, ratio, topk, k, W, Wr, Q, seq_len,
                    scale, splits, opart, mlpart, err);
     if (e != cudaSuccess) return e;
