@@ -32,9 +32,12 @@
 //    only its first 64 bytes, and the PV rows of dims 448..511 it yields are discarded.  S and O accumulate in fp32 in tensor memory.
 //  - Warps 8-15 run the online softmax: thread = entry (TMEM lane); warps 8-11 own heads 0-7,
 //    warps 12-15 heads 8-15.  The running max is raised lazily: O is rescaled in tensor memory
-//    only when a tile's max exceeds it by more than 8 (log2 units), so P <= 256 always.  Per
-//    tile the softmax warps meet at three barriers in the common case (the tile maxima, the
-//    rescale check, the P block scales), two more only when O must be rescaled.
+//    only when a tile's max exceeds it by more than 8 (log2 units), so P <= 256 always.  After a
+//    split's first tile, P is first formed against the running max and the softmax warps meet
+//    once (P published, and whether any entry lay more than 8 above the max); only then does a
+//    tile take the full path: the tile maxima, the new max, O rescaled where needed, P formed
+//    again (three barriers, two more when O is rescaled).  A split of one tile runs the full
+//    path directly (the kernel is compiled both ways).
 //  - Warps 8-15 prepare the query operands (one load per thread, issued right after the
 //    upstream wait) while the first copies are in flight.
 //  Three tile buffers, two S slots and two P buffers overlap the copies of tiles t+1 and t+2,
