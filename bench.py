@@ -167,6 +167,7 @@ PROFILES = {
     ("attention", "decode1m"): ("attention_tc_partial_decode1m.md", "attention_tc.cu", " (CSA+HCA)"),
     ("csa_compress", "prefill128k"): ("compress_prefill128k.md", "compress.cu", " (CSA)"),
     ("hca_compress", "prefill128k"): ("compress_prefill128k.md", "compress.cu", " (HCA)"),
+    ("indexer", "mtp1m"): ("indexer_multi_mtp1m.md", "indexer_multi.cu", ""),
 }
 
 
@@ -765,9 +766,9 @@ def run_mtp(args, rank, world, local_rank):
         "kernels_ms_per_step": {n: round(v, 5) for n, v in avg.items()},
         "indexer_keys_gbs": round(B * wl.csa_entries * 40 / (avg["indexer"] * 1e-3) / 1e9, 1),
         "roofline": {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                     "algorithmic_bytes_per_launch": bytes_[dominant]},
-        "clocks": clk, "gpu_launches": steps * 6,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "traffic": profiled_traffic(dominant, "mtp1m"), "algorithmic_bytes_per_launch": bytes_[dominant]},
+        "clocks": clk, "gpu_launches": steps * 7,   # indexer: score, gather, select; 2 x attention: partial, merge
     }
 
 
