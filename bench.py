@@ -679,7 +679,7 @@ def run_mtp(args, rank, world, local_rank):
     wl = synth.WORKLOADS["decode1m"]
     Q = MTP_Q
     B, W, k = wl.batch, wl.window, wl.topk
-    n_rep = REPLICAS
+    n_rep = 1 if args.profile else REPLICAS
     dev = torch.device("cuda", local_rank)
     scale = 1.0 / math.sqrt(512.0)
     g = synth.gen(4242 + rank, dev)
@@ -729,6 +729,13 @@ def run_mtp(args, rank, world, local_rank):
     for r in range(n_rep):
         step(r, False)
     torch.cuda.synchronize()
+    if args.profile:
+        for _ in range(args.steps or 3):
+            step(0, False)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        print(f"profile run ok: {args.steps or 3} eager steps of mtp1m on one replica", flush=True)
+        return None
     singles = [capture(torch, dev, lambda r=r: step(r, False)) for r in range(n_rep)]
     rounds = capture(torch, dev, lambda: [step(r, False) for r in range(n_rep)])
     instr = capture(torch, dev, lambda: [step(r, True) for r in range(n_rep)])
