@@ -557,14 +557,38 @@ __global__ void __launch_bounds__(kMqSelThreads) indexer_multi_select_kernel(con
     const uint32_t thr = (top22 << 10) | sel[0], take_eq = sel[1];
     __syncthreads();
     // ---- emit in index order: keys above the threshold, and the first take_eq equal to it -----
-    const int64_t n_e = in_smem ? (int64_t)n_c : n_q;
+    if (in_smem) {
+        // thread t takes candidates [per t, per (t + 1)); one block scan of its (above, equal)
+        // counts, packed into one word (each below 2^16), gives where its entries go
+        const uint32_t per = (n_c + kMqSelThreads - 1) / kMqSelThreads;
+        const uint32_t c0 = min(n_c, per * static_cast<uint32_t>(tid)), c1 = min(n_c, c0 + per);
+        uint32_t gt = 0u, eq = 0u;
+        for (uint32_t i = c0; i < c1; ++i) {
+            gt += sm.ckey[i] > thr ? 1u : 0u;
+            eq += sm.ckey[i] == thr ? 1u : 0u;
+        }
+        uint32_t tot;
+        const uint32_t pre = mq_block_scan((gt << 16) | eq, red, &tot);
+        uint32_t at = (pre >> 16) + min(pre & 0xFFFFu, take_eq), e_seen = pre & 0xFFFFu;
+        for (uint32_t i = c0; i < c1; ++i) {
+            const uint32_t key = sm.ckey[i];
+            bool take = key > thr;
+            if (key == thr) take = e_seen++ < take_eq;
+            if (take) {
+                if (at < static_cast<uint32_t>(k)) out[at] = static_cast<int32_t>(sm.cidx[i]);
+                ++at;
+            }
+        }
+        return;
+    }
+    const int64_t n_e = n_q;
     uint32_t base_sel = 0u, base_eq = 0u;
     for (int64_t i0 = 0; i0 < n_e; i0 += blockDim.x) {
         const int64_t i = i0 + tid;
         uint32_t key = 0u, idx = 0u;
         if (i < n_e) {
-            key = in_smem ? sm.ckey[i] : __ldcg(kq + i);
-            idx = in_smem ? sm.cidx[i] : static_cast<uint32_t>(i);
+            key = __ldcg(kq + i);
+            idx = static_cast<uint32_t>(i);
         }
         const uint32_t eq = (i < n_e && key == thr) ? 1u : 0u;
         uint32_t eq_tot;
