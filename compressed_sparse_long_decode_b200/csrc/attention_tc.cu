@@ -29,7 +29,8 @@
 //    significant bits as a bf16 operand.  The hi and lo rows are stacked into one N = 32
 //    operand and their results added when read back.  Block 3 holds bytes 384..511 (box copies;
 //    a gathered tile fills only 384..447), whose upper half is the bf16 RoPE part: QK reads
-//    only its first 64 bytes, and the PV rows of dims 448..511 it yields are discarded.  S and O accumulate in fp32 in tensor memory.
+//    only its first 64 bytes, and the PV rows of dims 448..511 it yields are discarded.  S and O
+//    accumulate in fp32 in tensor memory.
 //  - Warps 8-15 run the online softmax: thread = entry (TMEM lane); warps 8-11 own heads 0-7,
 //    warps 12-15 heads 8-15.  The running max is raised lazily: O is rescaled in tensor memory
 //    only when a tile's max exceeds it by more than 8 (log2 units), so P <= 256 always.  After a
@@ -41,8 +42,9 @@
 //  - Warps 8-15 prepare the query operands (one load per thread, issued right after the
 //    upstream wait) while the first copies are in flight.
 //  Three tile buffers, two S slots and two P buffers overlap the copies of tiles t+1 and t+2,
-//  QK of t+1, softmax of t and PV of t-1.  Every wait is bounded.  Each split writes its unnormalised O,
-//  the running max m (log2 units) and the sum l; attention_merge_kernel combines the splits.
+//  QK of t+1, softmax of t and PV of t-1.  Every wait is bounded.  Each split writes its
+//  unnormalised O, the running max m (log2 units) and the sum l; attention_merge_kernel combines
+//  the splits.
 #include <stdint.h>
 
 #include "csld_internal.cuh"
