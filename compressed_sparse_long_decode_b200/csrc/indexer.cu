@@ -118,6 +118,7 @@ struct CoopSmem {
     float scales[kCoopStages][kIdxTile * 2];
     ScoreCtl ctl;
     uint32_t keys[kCoopMaxRange];      // order keys of this CTA's range
+    uint32_t stepmax[kCoopMaxRange / 32 + 8];   // largest key of each aligned 32-key step
     uint32_t hist[kBins];              // this CTA's histograms of radix levels 1, 2, 3
     uint32_t hist2[kBins];
     uint32_t hist3[1024];
@@ -487,9 +488,9 @@ __device__ void score_release(ScoreCtl& ctl) {
 // the DRAM stream denser than one 8 KB tile per request.
 template <int S, int GT, uint32_t NCOLS>
 __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], float (*scales)[kIdxTile * 2],
-                          uint32_t* keys, uint32_t* hist, const uint8_t* ikeys, const float* iscales,
-                          int64_t cap, int b, int64_t c0, int cn, const float* q_idx, const float* head_w,
-                          int32_t* err) {
+                          uint32_t* keys, uint32_t* hist, uint32_t* stepmax, const uint8_t* ikeys,
+                          const float* iscales, int64_t cap, int b, int64_t c0, int cn, const float* q_idx,
+                          const float* head_w, int32_t* err) {
     static_assert(S <= kMaxStages, "ring depth");
     static_assert(S % GT == 0 && S / GT >= 2, "the ring holds at least two copy groups");
     static_assert(16 * S + 16 <= static_cast<int>(NCOLS), "accumulator slots and scale factors fit");
@@ -629,6 +630,10 @@ __device__ bool score_run(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], flo
                     const uint32_t key = score_key(sc);
                     if (li < cn) keys[li] = key;
                     if (li < cn) atomicAdd(&hist[key >> kBinShift], 1u);   // plain: scores spread over bins
+                    if (stepmax != nullptr) {   // the warp's 32 entries are one aligned step
+                        const uint32_t mx = __reduce_max_sync(0xffffffffu, li < cn ? key : 0u);
+                        if (lane == 0) stepmax[li >> 5] = mx;
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -665,7 +670,7 @@ __device__ bool score_chunk(ScoreCtl& ctl, uint8_t (*codes)[kIdxTile * kIkey], f
                             int64_t cap, int b, int64_t c0, int cn, const float* q_idx, const float* head_w,
                             int32_t* err) {
     score_setup<S, NCOLS>(ctl);
-    return score_run<S, GT, NCOLS>(ctl, codes, scales, keys, hist, ikeys, iscales, cap, b, c0, cn, q_idx, head_w,
+    return score_run<S, GT, NCOLS>(ctl, codes, scales, keys, hist, nullptr, ikeys, iscales, cap, b, c0, cn, q_idx, head_w,
                                    err);
 }
 
@@ -1044,7 +1049,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
 
     bool ok = true;
     if (cn > 0)
-        ok = score_run<kCoopStages, kCoopGroup, 256>(sm.ctl, sm.codes, sm.scales, sm.keys, sm.hist, ikeys, iscales, cap, b,
+        ok = score_run<kCoopStages, kCoopGroup, 256>(sm.ctl, sm.codes, sm.scales, sm.keys, sm.hist, sm.stepmax, ikeys,
+                                                     iscales, cap, b,
                                                      c0, cn,
                                          q_idx, head_w, err);
     else
@@ -1071,8 +1077,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     const int i0 = warp * kSeg;
     const int steps = max(0, min(kSeg, cn - i0) + 31) >> 5;
     uint32_t gt = 0u, nc = 0u;
-    uint32_t cmask = 0u;   // 32-key steps of this warp's segment holding a key of bin >= beta1
-    for (int s = 0; s < steps; ++s) {
+    // 32-key steps of this warp's segment holding a key of bin >= beta1, from the step maxima
+    // kept while scoring (steps <= 32); only they can hold a key above or inside bin beta1
+    const uint32_t cmask = __ballot_sync(0xffffffffu, lane < steps && sm.stepmax[(i0 >> 5) + lane] >= (beta1 << kBinShift));
+    for (uint32_t mk = cmask; mk != 0u; mk &= mk - 1u) {
+        const int s = __ffs(mk) - 1;
         const int i = i0 + 32 * s + lane;
         const uint32_t key = i < cn ? sm.keys[i] : 0u;
         const uint32_t bin = key >> kBinShift;
@@ -1080,7 +1089,6 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
         gt += __popc(ma);
         const bool in = i < cn && bin == beta1;
         const uint32_t m = __ballot_sync(0xffffffffu, in);
-        if ((ma | m) != 0u) cmask |= 1u << s;
         if (in) {
             cand[nc + __popc(m & lt)] = key;
             if (!fast) {   // level-2 histogram: bits 20..10
