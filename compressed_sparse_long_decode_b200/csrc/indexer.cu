@@ -877,13 +877,15 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 // Barrier of the CTAs of one sequence: arrival counter *ctr reaches `target`.  The spin is
 // bounded (about half a second); on time-out the device error word gets CSLD_DEVERR_TIMEOUT
 // and false is returned to every thread of the CTA.  The CTA barrier orders every thread's
-// global writes before thread 0's fence and arrival (the fence is cumulative), so only
-// thread 0 fences, as in a grid-wide sync.
+// global writes before thread 0's arrival, a release add (release is cumulative), and thread
+// 0's acquire load of the count orders the other CTAs' writes before everything the CTA does
+// after the closing barrier, as in a grid-wide sync.
 __device__ bool seq_barrier(uint32_t* ctr, uint32_t target, int32_t* fail_flag, int32_t* err) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(ctr, 1u);
+        // a release add: the CTA's writes before the barrier above are visible to whoever
+        // acquires the count (no separate fence, and no wait for the add's return value)
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
         bool ok = false;
         for (uint32_t i = 0; i < (1u << 22); ++i) {
             if (ld_acquire_u32(ctr) >= target) {
@@ -896,7 +898,6 @@ __device__ bool seq_barrier(uint32_t* ctr, uint32_t target, int32_t* fail_flag, 
             dev_error(err, CSLD_DEVERR_TIMEOUT);
             *fail_flag = 1;
         }
-        __threadfence();
     }
     __syncthreads();
     return *reinterpret_cast<volatile int32_t*>(fail_flag) == 0;
