@@ -27,11 +27,11 @@
 // Selection, when the whole grid can be resident (indexer_topk_coop_kernel, cooperative
 // launch): each sequence is split into `units` ranges, one CTA each, and the CTAs of a sequence
 // run an exact select together.  They add their histograms into the sequence's global
-// histogram, meet at a barrier (an arrival counter; every wait is bounded), and each derive the
-// same threshold bin.  When that bin holds at most kListMax keys, every CTA appends its keys in
+// histogram, each re-read it until its bins account for every key of the sequence (every wait
+// is bounded), and each derive the same threshold bin.  When that bin holds at most kListMax keys, every CTA appends its keys in
 // the bin to a list of self-announcing slots, then reads the whole list as it fills and finds
 // the exact threshold key with three radix levels; otherwise two more histogram rounds over
-// the next 11 and 10 key bits (and barriers) give it.  Either way every CTA learns how many
+// the next 11 and 10 key bits (and arrival-counter barriers) give it.  Either way every CTA learns how many
 // selected entries precede its range (ties go to the lowest indices) and writes its own in
 // ascending index order.
 //
@@ -974,6 +974,69 @@ __device__ void find_bin_global(const uint32_t* g, int nbins, uint32_t want, uin
     __syncthreads();
 }
 
+// Level 1 without a barrier: the sequence's global histogram g (kBins bins) is complete once its
+// bins add up to `total`, the number of keys its ranges scored (bins only grow, so a read whose
+// sum is the total holds every bin's final count).  Re-read until it is (bounded: about half a
+// second, then CSLD_DEVERR_TIMEOUT and false in every thread); then, as find_bin_global, the bin
+// holding the want-th largest key, the keys wanted inside it and the bin's count.
+__device__ bool find_bin_complete(const uint32_t* g, uint32_t total, uint32_t want, uint32_t* red, uint32_t* sel,
+                                  uint32_t* bin, uint32_t* need, uint32_t* count, int32_t* err) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    constexpr int per = kBins / kIdxThreads;
+    uint32_t c[per], tot = 0u, incl = 0u, wb = 0u, all = 0u;
+    bool ok = false;
+    for (uint32_t it = 0; it < (1u << 20); ++it) {
+        tot = 0u;
+#pragma unroll
+        for (int q = 0; q < per; ++q) {
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(c[q]) : "l"(g + kBins - 1 - per * tid - q) : "memory");
+            tot += c[q];
+        }
+        incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        wb = warp_excl_scan(__shfl_sync(0xffffffffu, incl, 31), red, &all);
+        __syncthreads();   // red is written again by the next read
+        if (all == total) {
+            ok = true;
+            break;
+        }
+        if (it >= 16) __nanosleep(64);
+    }
+    if (!ok) {
+        if (tid == 0) dev_error(err, CSLD_DEVERR_TIMEOUT);
+        return false;
+    }
+    if (tid == 0) {
+        sel[0] = 0u;
+        sel[1] = 0u;
+        sel[2] = 0u;
+    }
+    __syncthreads();
+    const uint32_t excl = wb + incl - tot;
+    if (excl < want && excl + tot >= want) {
+        uint32_t run = excl;
+        for (int q = 0; q < per; ++q) {
+            if (run + c[q] >= want) {
+                sel[0] = static_cast<uint32_t>(kBins - 1 - per * tid - q);
+                sel[1] = want - run;
+                sel[2] = c[q];
+                break;
+            }
+            run += c[q];
+        }
+    }
+    __syncthreads();
+    *bin = sel[0];
+    *need = sel[1];
+    *count = sel[2];
+    __syncthreads();
+    return true;
+}
+
 __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     const uint8_t* __restrict__ ikeys, const float* __restrict__ iscales, int64_t cap,
     const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
@@ -1018,8 +1081,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     // per-range counts) per sequence; the epoch (calls completed on this sequence) picks this
     // call's set.  The other set belonged to the previous call, which has finished: every CTA
     // clears its share of it here for the next call, so nothing has to be reset at the end of
-    // this one.  The epoch is read before the first barrier and advanced only after it, by
-    // range 0 at its end.
+    // this one.  Every CTA reads the epoch before it adds to the level-1 histogram, and range 0
+    // advances it at its end, after it has seen the complete histogram.
     uint32_t* sq = ws.sync + (size_t)b * 64;
     const uint32_t par = __ldcg(sq + 4) & 1u;
     uint32_t* g1 = ws.hist + ((size_t)b * 2 + par) * kCoopSeqWords;
@@ -1057,21 +1120,28 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     else
         score_release<256>(sm.ctl);
     __syncthreads();
-    // --- level 1: bits 31..21 ------------------------------------------------------------------
-    if (ok)
+    // --- level 1: bits 31..21.  No barrier: every CTA re-reads the sequence's histogram until it
+    //     holds all n_b keys (the ranges partition the visible entries).  A range whose scoring
+    //     timed out adds its key count to bin 0, so the others still get past this point (the
+    //     error word already says the selection is not to be trusted). ---------------------------
+    if (ok) {
         for (int i = tid; i < kBins; i += blockDim.x) {
             const uint32_t c = sm.hist[i];
             if (c) atomicAdd(g1 + i, c);
         }
-    if (!seq_barrier(bar, 1 * nu + barrier_extra, &sm.fail, err)) return;
+    } else if (tid == 0 && cn > 0) {
+        atomicAdd(g1, static_cast<uint32_t>(cn));
+    }
     uint32_t beta1, need1, cnt1;
-    find_bin_global(g1, kBins, want, sm.red, sm.sel, &beta1, &need1, &cnt1);
+    if (!find_bin_complete(g1, static_cast<uint32_t>(n_b) + barrier_extra, want, sm.red, sm.sel, &beta1, &need1,
+                           &cnt1, err))
+        return;
     // --- candidates: one pass over the range.  Each warp counts its keys above bin beta1 and
     //     copies the keys inside it to its own candidate region (the copy ring is idle now).
     //     When the sequence's bin beta1 is small, the candidates of all its ranges go to one
-    //     global list that every CTA then resolves on its own (two barriers in all); otherwise
-    //     two more histogram levels run (bits 20..10, then 9..0) and the ranges exchange their
-    //     counts (four barriers).  The choice is the same in every CTA of the sequence. --------
+    //     global list that every CTA then resolves on its own (no barrier); otherwise two more
+    //     histogram levels run (bits 20..10, then 9..0) and the ranges exchange their counts
+    //     (three barriers).  The choice is the same in every CTA of the sequence. --------
     const bool fast = cnt1 <= static_cast<uint32_t>(kListMax) && units <= 255;
     constexpr int kSeg = kCoopMaxRange / kIdxWarps;    // warp w owns positions 1024w .. 1024w+1023
     uint32_t* cand = reinterpret_cast<uint32_t*>(&sm.codes[0][0]) + warp * kSeg;
@@ -1176,7 +1246,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             const uint32_t c = sm.hist2[i];
             if (c) atomicAdd(g2 + i, c);
         }
-        if (!seq_barrier(bar, 2 * nu + barrier_extra, &sm.fail, err)) return;
+        if (!seq_barrier(bar, 1 * nu + barrier_extra, &sm.fail, err)) return;
         uint32_t beta2, need2;
         find_bin_global(g2, kBins, need1, sm.red, sm.sel, &beta2, &need2);
         const uint32_t top22 = (beta1 << 11) | beta2;
@@ -1197,7 +1267,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             const uint32_t c = sm.hist3[i];
             if (c) atomicAdd(g3 + i, c);
         }
-        if (!seq_barrier(bar, 3 * nu + barrier_extra, &sm.fail, err)) return;
+        if (!seq_barrier(bar, 2 * nu + barrier_extra, &sm.fail, err)) return;
         uint32_t beta3;
         find_bin_global(g3, 1024, need2, sm.red, sm.sel, &beta3, &take_eq);
         thr = (top22 << 10) | beta3;
@@ -1217,7 +1287,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
             cnt[2 * u] = tot >> 16;
             cnt[2 * u + 1] = tot & 0xFFFFu;
         }
-        if (!seq_barrier(bar, 4 * nu + barrier_extra, &sm.fail, err)) return;
+        if (!seq_barrier(bar, 3 * nu + barrier_extra, &sm.fail, err)) return;
         uint32_t a_loc = 0u, e_loc = 0u;
         for (int v = tid; v < u; v += blockDim.x) {
             a_loc += __ldcg(cnt + 2 * v);
@@ -1261,8 +1331,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1) indexer_topk_coop_kernel(
     if (u == 0 && tid == 0) atomicAdd(sq + 4, 1u);
 }
 
-// Test hook (csld_test_set_barrier_extra): arrivals added to every cross-CTA barrier target of
-// the cooperative kernel, so that a test can make its bounded waits run out.  0 in normal use.
+// Test hook (csld_test_set_barrier_extra): added to the key total the level-1 histogram must
+// reach and to every cross-CTA barrier target of the cooperative kernel, so that a test can make
+// its bounded waits run out.  0 in normal use.
 std::atomic<int> g_test_barrier_extra{0};
 
 // Resident CTAs of the cooperative kernel on the current device (0 if it cannot run), found

@@ -364,9 +364,10 @@ CSLD_API csld_status csld_stage(void* dst, const void* src, size_t bytes, void* 
 
 /* ----------------------------------------------------------------------------------------
  * Test hook (no counterpart on the pages): the indexer's cooperative kernel waits, with a bound
- * of about half a second, for the CTAs of a sequence at four cross-CTA barriers.  This call adds
- * `extra` arrivals to every barrier target of the calls that follow (0 restores normal use), so
- * that a test can make those waits run out and check the recovery: the kernel returns,
+ * of about half a second each, for the CTAs of a sequence: until their level-1 histogram holds
+ * every key, and at up to three cross-CTA barriers.  This call adds `extra` to that key total and
+ * to every barrier target of the calls that follow (0 restores normal use), so that a test can
+ * make those waits run out and check the recovery: the kernel returns,
  * CSLD_DEVERR_TIMEOUT is set in the error word, and the workspace must be zero-filled again
  * before the next call.  Process-wide; not for production use.
  * ---------------------------------------------------------------------------------------- */
