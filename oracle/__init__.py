@@ -68,6 +68,10 @@ def _declare(L):
     L.orc_pool_block.argtypes = [_P, _P, _P, C.c_int, _P]
     L.orc_compress.restype = None
     L.orc_compress.argtypes = [_P, _P, _P, _P, C.c_int64, C.c_int, _P, _P, _P]
+    L.orc_rope_rotate.restype = None
+    L.orc_rope_rotate.argtypes = [_P, C.c_double, C.c_double]
+    L.orc_compress_rope.restype = None
+    L.orc_compress_rope.argtypes = [_P, _P, _P, _P, C.c_int64, C.c_int, C.c_int64, C.c_double, _P, _P, _P]
     L.orc_pool_block_channel.restype = None
     L.orc_pool_block_channel.argtypes = [_P, _P, _P, C.c_int, _P]
     L.orc_compress_channel.restype = None
@@ -92,6 +96,9 @@ def _declare(L):
     L.orc_append_batch.restype = C.c_int
     L.orc_append_batch.argtypes = [C.c_int, C.c_int, C.c_int64, C.c_int, _P, _P, _P, _P, _P, _P,
                                    _P, _P, _P, _P, _P]
+    L.orc_append_batch_rope.restype = C.c_int
+    L.orc_append_batch_rope.argtypes = [C.c_int, C.c_int, C.c_int64, C.c_int, _P, _P, _P, _P, _P, _P,
+                                        _P, _P, _P, _P, _P, C.c_double]
     L.orc_num_threads.restype = C.c_int
     L.orc_num_threads.argtypes = []
 
@@ -208,6 +215,31 @@ def compress(raw_bits, gate, bias, m, w_idx=None):
     return kv, ik, isc
 
 
+def rope_rotate(x, pos, base):
+    """O1r: a copy of x (float64 [512]) with its RoPE dims 448..511 rotated at position pos."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    assert x.shape == (D,)
+    lib().orc_rope_rotate(_ptr(x), float(pos), float(base))
+    return x
+
+
+def compress_rope(raw_bits, gate, bias, m, pos0, base, w_idx=None):
+    """Prefill compression with RoPE at compressed positions (raw token 0 at position pos0):
+    entry s rotated at pos0 + (s+1) m - 1.  Returns (kv [E,576], ikeys [E,32], iscales [E,2])."""
+    raw_bits = _c(raw_bits, np.uint16)
+    gate = _c(gate, np.float32)
+    bias = _c(bias, np.float32)
+    T = raw_bits.shape[0]
+    E = T // m
+    kv = np.zeros((E, ENTRY_BYTES), np.uint8)
+    ik = np.zeros((E, IKEY_BYTES), np.uint8) if w_idx is not None else None
+    isc = np.zeros((E, 2), np.float32) if w_idx is not None else None
+    w = _c(w_idx, np.float32) if w_idx is not None else None
+    lib().orc_compress_rope(_ptr(raw_bits), _ptr(gate), _ptr(bias), _ptr(w), T, m, int(pos0), float(base),
+                            _ptr(kv), _ptr(ik), _ptr(isc))
+    return kv, ik, isc
+
+
 def pool_block_channel(raw_bits, gate, bias):
     """Per-channel gating: raw_bits uint16 [m,512]; gate, bias float32 [m,512] -> float64 [512]."""
     raw_bits = _c(raw_bits, np.uint16)
@@ -317,16 +349,18 @@ class LayerState:
         self.seq_len = np.zeros(B, np.int32)
 
 
-def append_batch(st: LayerState, bias, w_idx, x_bits, gate):
-    """Append one token per sequence (x_bits [B,512] u16, gate [B] f32).  Raises on overflow."""
+def append_batch(st: LayerState, bias, w_idx, x_bits, gate, rope_base=0.0):
+    """Append one token per sequence (x_bits [B,512] u16, gate [B] f32).  Raises on overflow.
+    rope_base > 0: RoPE at compressed positions (window entry at its token, a completed entry
+    at its block's last token)."""
     bias = _c(bias, np.float32)
     w = _c(w_idx, np.float32) if w_idx is not None else None
     x_bits = _c(x_bits, np.uint16)
     gate = _c(gate, np.float32)
-    rc = lib().orc_append_batch(st.m, st.W, st.cap, st.B, _ptr(st.comp_kv), _ptr(st.ikeys),
-                                _ptr(st.iscales), _ptr(st.win_kv), _ptr(st.tail_kv),
-                                _ptr(st.tail_gate), _ptr(st.seq_len), _ptr(bias), _ptr(w),
-                                _ptr(x_bits), _ptr(gate))
+    rc = lib().orc_append_batch_rope(st.m, st.W, st.cap, st.B, _ptr(st.comp_kv), _ptr(st.ikeys),
+                                     _ptr(st.iscales), _ptr(st.win_kv), _ptr(st.tail_kv),
+                                     _ptr(st.tail_gate), _ptr(st.seq_len), _ptr(bias), _ptr(w),
+                                     _ptr(x_bits), _ptr(gate), float(rope_base))
     if rc != 0:
         raise OverflowError("oracle append: compressed cache capacity exceeded")
 

@@ -26,7 +26,10 @@
  *  - the indexer score is computed in fp32 in a fixed operation order (see
  *    orc_indexer_scores); selection is by (score desc, index asc);
  *  - attention is one joint softmax over {selected or all visible compressed entries} and
- *    {the last W raw tokens}; a compressed entry is visible once its last token arrived.
+ *    {the last W raw tokens}; a compressed entry is visible once its last token arrived;
+ *  - layout variants: per-channel gating (orc_pool_block_channel) and RoPE applied at
+ *    compressed positions (orc_rope_rotate: RoFormer pairs (448+2i, 449+2i), angle
+ *    pos * base^(-i/32); an entry at its block's last token, a window entry at its token).
  *
  * parity unpinned: the real model's gate form, indexer projection and FP4 scale rule are not
  * given by the pages (no weights); what is pinned is listed in the tests.
@@ -266,22 +269,58 @@ void orc_indexer_key_raw(const double* c, const float* w_idx, double* u) {
     }
 }
 
+/* ------------------------------------------------------------------------------------------
+ * O1r -- RoPE at compressed positions (a layout variant.  [HF] storage paragraph: each entry
+ * keeps its RoPE dims in bf16; in the base reading those dims are stored as given.  In this
+ * variant the raw tokens' dims 448..511 arrive before rotary position encoding and the
+ * compressor rotates them itself, at the entry's own position).  Readings: the rotation is
+ * RoFormer's -- consecutive pairs, pair i = dims (448 + 2i, 449 + 2i) for i = 0..31, turned by
+ * the angle pos * base^(-i/32); a compressed entry s of ratio m stands at its block's last
+ * token, pos0 + (s+1) m - 1 (where it becomes visible), a window entry at its own token; the
+ * indexer key is projected from the rotated pooled vector.
+ * ---------------------------------------------------------------------------------------- */
+void orc_rope_rotate(double* x, double pos, double base) {
+    for (int i = 0; i < ORC_D_ROPE / 2; ++i) {
+        double theta = pow(base, -(double)i / (double)(ORC_D_ROPE / 2));
+        double a = pos * theta;
+        double c = cos(a), s = sin(a);
+        double x0 = x[ORC_D_NOPE + 2 * i], x1 = x[ORC_D_NOPE + 2 * i + 1];
+        x[ORC_D_NOPE + 2 * i] = x0 * c - x1 * s;
+        x[ORC_D_NOPE + 2 * i + 1] = x0 * s + x1 * c;
+    }
+}
+
 /* O1 + O2 over a whole prefill: T tokens of one sequence -> floor(T/m) entries; the trailing
  * T mod m tokens form no entry.  ikey_out / iscale_out are written only when w_idx != NULL
- * (CSA; [HF] CSA paragraph: the lightning indexer runs over the 4x-compressed entries). */
-void orc_compress(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
-                  int64_t T, int m, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
+ * (CSA; [HF] CSA paragraph: the lightning indexer runs over the 4x-compressed entries).
+ * rope_base > 0: O1r, entry s rotated at position pos0 + (s+1) m - 1 after pooling. */
+static void orc_compress_impl(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
+                              int64_t T, int m, int64_t pos0, double rope_base, uint8_t* kv_out,
+                              uint8_t* ikey_out, float* iscale_out) {
     int64_t E = T / m;
 #pragma omp parallel for schedule(static)
     for (int64_t s = 0; s < E; ++s) {
         double c[ORC_D], u[ORC_IDX_DIM];
         orc_pool_block(raw + (size_t)s * m * ORC_D, gate + (size_t)s * m, bias, m, c);
+        if (rope_base > 0.0) orc_rope_rotate(c, (double)(pos0 + (s + 1) * (int64_t)m - 1), rope_base);
         orc_entry_encode(c, kv_out + (size_t)s * ORC_ENTRY_BYTES);
         if (w_idx) {
             orc_indexer_key_raw(c, w_idx, u);
             orc_fp4_quantize64(u, ikey_out + (size_t)s * ORC_IKEY_BYTES, iscale_out + (size_t)s * 2);
         }
     }
+}
+
+void orc_compress(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
+                  int64_t T, int m, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, kv_out, ikey_out, iscale_out);
+}
+
+/* O1r + O1 + O2: raw token 0 at position pos0, rotation base rope_base > 0. */
+void orc_compress_rope(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
+                       int64_t T, int m, int64_t pos0, double rope_base, uint8_t* kv_out,
+                       uint8_t* ikey_out, float* iscale_out) {
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, pos0, rope_base, kv_out, ikey_out, iscale_out);
 }
 
 /* O1 (per-channel) + O2 over a whole prefill: gate [T][512], bias [m][512]. */
@@ -519,9 +558,12 @@ int orc_attention_batch(const uint16_t* q, int H, const uint8_t* comp_kv, int64_
  * (plus its indexer key when w_idx != NULL).  Returns -1 and changes nothing when entry s
  * would not fit in cap.
  * ---------------------------------------------------------------------------------------- */
-int orc_append(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, float* iscales,
-               uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate, int32_t* seq_len,
-               const float* bias, const float* w_idx, const uint16_t* x, float gate) {
+/* rope_base > 0: O1r -- the window entry of token t rotated at position t, the completed
+ * entry s at position t = (s+1) m - 1, its block's last token. */
+static int orc_append_impl(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, float* iscales,
+                           uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate, int32_t* seq_len,
+                           const float* bias, const float* w_idx, const uint16_t* x, float gate,
+                           double rope_base) {
     int32_t t = *seq_len;
     int complete = ((t + 1) % m) == 0;
     int64_t s = t / m;
@@ -529,6 +571,7 @@ int orc_append(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, floa
     if (W > 0) {
         double xd[ORC_D];
         for (int d = 0; d < ORC_D; ++d) xd[d] = orc_bf16_decode(x[d]);
+        if (rope_base > 0.0) orc_rope_rotate(xd, (double)t, rope_base);
         orc_entry_encode(xd, win_kv + (size_t)(t % W) * ORC_ENTRY_BYTES);
     }
     memcpy(tail_kv + (size_t)(t % m) * ORC_D, x, sizeof(uint16_t) * ORC_D);
@@ -536,6 +579,7 @@ int orc_append(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, floa
     if (complete) {
         double c[ORC_D], u[ORC_IDX_DIM];
         orc_pool_block(tail_kv, tail_gate, bias, m, c);
+        if (rope_base > 0.0) orc_rope_rotate(c, (double)t, rope_base);
         orc_entry_encode(c, comp_kv + (size_t)s * ORC_ENTRY_BYTES);
         if (w_idx) {
             orc_indexer_key_raw(c, w_idx, u);
@@ -546,21 +590,36 @@ int orc_append(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, floa
     return 0;
 }
 
-/* The same for B sequences, one token each: x [B][512], gate [B]. */
+int orc_append(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, float* iscales,
+               uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate, int32_t* seq_len,
+               const float* bias, const float* w_idx, const uint16_t* x, float gate) {
+    return orc_append_impl(m, W, cap, comp_kv, ikeys, iscales, win_kv, tail_kv, tail_gate, seq_len, bias,
+                           w_idx, x, gate, 0.0);
+}
+
+/* The same for B sequences, one token each: x [B][512], gate [B]; rope_base as above (0: none). */
+int orc_append_batch_rope(int m, int W, int64_t cap, int B, uint8_t* comp_kv, uint8_t* ikeys,
+                          float* iscales, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
+                          int32_t* seq_len, const float* bias, const float* w_idx, const uint16_t* x,
+                          const float* gate, double rope_base) {
+    int rc = 0;
+    for (int b = 0; b < B; ++b) {
+        rc |= orc_append_impl(m, W, cap, comp_kv + (size_t)b * cap * ORC_ENTRY_BYTES,
+                              ikeys ? ikeys + (size_t)b * cap * ORC_IKEY_BYTES : NULL,
+                              iscales ? iscales + (size_t)b * cap * 2 : NULL,
+                              win_kv + (size_t)b * (W > 0 ? W : 0) * ORC_ENTRY_BYTES,
+                              tail_kv + (size_t)b * m * ORC_D, tail_gate + (size_t)b * m, seq_len + b,
+                              bias, w_idx, x + (size_t)b * ORC_D, gate[b], rope_base);
+    }
+    return rc;
+}
+
 int orc_append_batch(int m, int W, int64_t cap, int B, uint8_t* comp_kv, uint8_t* ikeys,
                      float* iscales, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
                      int32_t* seq_len, const float* bias, const float* w_idx, const uint16_t* x,
                      const float* gate) {
-    int rc = 0;
-    for (int b = 0; b < B; ++b) {
-        rc |= orc_append(m, W, cap, comp_kv + (size_t)b * cap * ORC_ENTRY_BYTES,
-                         ikeys ? ikeys + (size_t)b * cap * ORC_IKEY_BYTES : NULL,
-                         iscales ? iscales + (size_t)b * cap * 2 : NULL,
-                         win_kv + (size_t)b * (W > 0 ? W : 0) * ORC_ENTRY_BYTES,
-                         tail_kv + (size_t)b * m * ORC_D, tail_gate + (size_t)b * m, seq_len + b,
-                         bias, w_idx, x + (size_t)b * ORC_D, gate[b]);
-    }
-    return rc;
+    return orc_append_batch_rope(m, W, cap, B, comp_kv, ikeys, iscales, win_kv, tail_kv, tail_gate, seq_len,
+                                 bias, w_idx, x, gate, 0.0);
 }
 
 int orc_num_threads(void) {
