@@ -16,7 +16,8 @@ import os
 import torch
 
 __all__ = [
-    "csa_compress", "hca_compress", "compress", "compress_channel", "indexer_topk", "hybrid_decode_attention",
+    "csa_compress", "hca_compress", "compress", "compress_channel", "compress_rope", "kv_cache_append_rope",
+    "kv_cache_prefill_rope", "indexer_topk", "hybrid_decode_attention",
     "kv_cache_append", "kv_cache_prefill", "LayerCache", "CsldError", "lib", "ENTRY_BYTES",
     "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace", "DecodeStack",
     "layer_pattern", "stage", "indexer_rescore", "topk_merge", "lse_merge", "ContextParallelLayer",
@@ -62,6 +63,9 @@ def _load():
     L.csld_status_string.argtypes = [I]
     L.csld_compress.argtypes = [P, P, P, I, P, I64, P, P, P, P]
     L.csld_compress_channel.argtypes = [P, P, P, I, P, I64, P, P, P, P]
+    L.csld_compress_rope.argtypes = [P, P, P, I, P, I64, I64, C.c_double, P, P, P, P]
+    L.kv_cache_append_rope.argtypes = [C.POINTER(_Cache), P, P, C.c_double, P, P]
+    L.kv_cache_prefill_rope.argtypes = [C.POINTER(_Cache), P, P, I64, C.c_double, P]
     L.csa_compress.argtypes = [P, P, P, P, I64, P, P, P, P]
     L.hca_compress.argtypes = [P, P, P, I64, P, P]
     L.kv_cache_append.argtypes = [C.POINTER(_Cache), P, P, P, P]
@@ -80,7 +84,8 @@ def _load():
     L.hybrid_decode_attention_multi.argtypes = [P, I, P, I64, I, P, I, P, I, I, P, I, I, F, P, P, P, S, P, P]
     L.csld_topk_merge.argtypes = [P, P, P, I, I, I, I64, I64, P, P]
     L.csld_lse_merge.argtypes = [P, P, I, I, I, P, P, P]
-    for fn in ("csld_compress", "csld_compress_channel", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
+    for fn in ("csld_compress", "csld_compress_channel", "csld_compress_rope", "kv_cache_append_rope",
+               "kv_cache_prefill_rope", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
                "indexer_topk", "hybrid_decode_attention", "csld_stage", "indexer_rescore", "csld_topk_merge",
                "csld_lse_merge", "indexer_topk_multi", "hybrid_decode_attention_multi"):
         getattr(L, fn).restype = I
@@ -168,6 +173,30 @@ def compress_channel(raw, gate, pos_bias, ratio, w_idx=None, kv_out=None, ikey_o
     return (kv_out, ikey_out, iscale_out) if w_idx is not None else kv_out
 
 
+def compress_rope(raw, gate, pos_bias, ratio, pos0, rope_base, w_idx=None, kv_out=None, ikey_out=None,
+                  iscale_out=None):
+    """Compression with RoPE at compressed positions (csld_compress_rope): raw [T,512] bf16 with
+    its dims 448..511 before rotary encoding, raw[0] at position pos0."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    _need(pos_bias, torch.float32, "pos_bias")
+    T = raw.shape[0]
+    E = T // ratio
+    dev = raw.device
+    if kv_out is None:
+        kv_out = torch.empty((E, ENTRY_BYTES), dtype=torch.uint8, device=dev)
+    if w_idx is not None:
+        _need(w_idx, torch.float32, "w_idx")
+        if ikey_out is None:
+            ikey_out = torch.empty((E, IKEY_BYTES), dtype=torch.uint8, device=dev)
+        if iscale_out is None:
+            iscale_out = torch.empty((E, 2), dtype=torch.float32, device=dev)
+    _check(lib.csld_compress_rope(_ptr(raw), _ptr(gate), _ptr(pos_bias), ratio, _ptr(w_idx), T, int(pos0),
+                                  float(rope_base), _ptr(kv_out), _ptr(ikey_out), _ptr(iscale_out), _stream()),
+           "csld_compress_rope")
+    return (kv_out, ikey_out, iscale_out) if w_idx is not None else kv_out
+
+
 def csa_compress(raw, gate, pos_bias, w_idx, kv_out=None, ikey_out=None, iscale_out=None):
     return compress(raw, gate, pos_bias, 4, w_idx, kv_out, ikey_out, iscale_out)
 
@@ -211,6 +240,24 @@ def kv_cache_append(cache: LayerCache, kv_new, gate_new, err=None):
     s = cache.struct()
     _check(lib.kv_cache_append(C.byref(s), _ptr(kv_new), _ptr(gate_new),
                                _ptr(cache.err if err is None else err), _stream()), "kv_cache_append")
+
+
+def kv_cache_append_rope(cache: LayerCache, kv_new, gate_new, rope_base, err=None):
+    """kv_cache_append with RoPE at compressed positions (kv_cache_append_rope)."""
+    _bits(kv_new, "kv_new")
+    _need(gate_new, torch.float32, "gate_new")
+    s = cache.struct()
+    _check(lib.kv_cache_append_rope(C.byref(s), _ptr(kv_new), _ptr(gate_new), float(rope_base),
+                                    _ptr(cache.err if err is None else err), _stream()), "kv_cache_append_rope")
+
+
+def kv_cache_prefill_rope(cache: LayerCache, raw, gate, rope_base):
+    """kv_cache_prefill with RoPE at compressed positions (kv_cache_prefill_rope)."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    s = cache.struct()
+    _check(lib.kv_cache_prefill_rope(C.byref(s), _ptr(raw), _ptr(gate), raw.shape[1], float(rope_base), _stream()),
+           "kv_cache_prefill_rope")
 
 
 def kv_cache_prefill(cache: LayerCache, raw, gate):

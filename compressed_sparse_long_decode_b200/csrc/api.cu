@@ -113,9 +113,10 @@ const char* csld_status_string(csld_status s) {
     return "unknown status";
 }
 
-csld_status csld_compress(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
-                          const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
-                          float* iscale_out, void* stream) {
+namespace {
+csld_status compress_impl(const char* name, const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
+                          const float* w_idx, int64_t T, int64_t pos0, double rope_base, uint8_t* kv_out,
+                          uint8_t* ikey_out, float* iscale_out, void* stream) {
     if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
     if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
     if (T / ratio == 0) return CSLD_OK;
@@ -124,9 +125,26 @@ csld_status csld_compress(const uint16_t* raw, const float* gate, const float* p
     if (!aligned16(raw) || !aligned16(kv_out) || (ikey_out && !aligned16(ikey_out)))
         return fail(CSLD_ERR_ALIGN, "raw, kv_out and ikey_out must be 16-byte aligned");
     cudaError_t e = csld::launch_compress(raw, gate, pos_bias, ratio, w_idx, T, 1, T / ratio, kv_out,
-                                          ikey_out, iscale_out, num_sms(), as_stream(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "csld_compress");
+                                          ikey_out, iscale_out, num_sms(), as_stream(stream), pos0, rope_base);
+    if (e != cudaSuccess) return cuda_fail(e, name);
     return CSLD_OK;
+}
+}  // namespace
+
+csld_status csld_compress(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
+                          const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
+                          float* iscale_out, void* stream) {
+    return compress_impl("csld_compress", raw, gate, pos_bias, ratio, w_idx, T, 0, 0.0, kv_out, ikey_out, iscale_out,
+                         stream);
+}
+
+csld_status csld_compress_rope(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
+                               const float* w_idx, int64_t T, int64_t pos0, double rope_base, uint8_t* kv_out,
+                               uint8_t* ikey_out, float* iscale_out, void* stream) {
+    if (!(rope_base > 1.0) || rope_base == INFINITY) return fail(CSLD_ERR_ARG, "rope_base must be finite and > 1");
+    if (pos0 < 0 || pos0 > ((int64_t)1 << 40)) return fail(CSLD_ERR_ARG, "pos0 %lld outside 0..2^40", (long long)pos0);
+    return compress_impl("csld_compress_rope", raw, gate, pos_bias, ratio, w_idx, T, pos0, rope_base, kv_out,
+                         ikey_out, iscale_out, stream);
 }
 
 csld_status csa_compress(const uint16_t* raw, const float* gate, const float* pos_bias,
@@ -141,19 +159,33 @@ csld_status hca_compress(const uint16_t* raw, const float* gate, const float* po
     return csld_compress(raw, gate, pos_bias, 128, nullptr, T, kv_out, nullptr, nullptr, stream);
 }
 
-csld_status kv_cache_append(const csld_layer_cache* cache, const uint16_t* kv_new,
-                            const float* gate_new, int32_t* err, void* stream) {
+namespace {
+csld_status append_impl(const char* name, const csld_layer_cache* cache, const uint16_t* kv_new,
+                        const float* gate_new, int32_t* err, double rope_base, void* stream) {
     csld_status s = check_cache(cache);
     if (s != CSLD_OK) return s;
     if (!kv_new || !gate_new) return fail(CSLD_ERR_ARG, "kv_new / gate_new is NULL");
     if (!aligned16(kv_new)) return fail(CSLD_ERR_ALIGN, "kv_new must be 16-byte aligned");
-    cudaError_t e = csld::launch_append(*cache, kv_new, gate_new, err, as_stream(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "kv_cache_append");
+    cudaError_t e = csld::launch_append(*cache, kv_new, gate_new, err, as_stream(stream), rope_base);
+    if (e != cudaSuccess) return cuda_fail(e, name);
     return CSLD_OK;
 }
+}  // namespace
 
-csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
-                             int64_t T, void* stream) {
+csld_status kv_cache_append(const csld_layer_cache* cache, const uint16_t* kv_new,
+                            const float* gate_new, int32_t* err, void* stream) {
+    return append_impl("kv_cache_append", cache, kv_new, gate_new, err, 0.0, stream);
+}
+
+csld_status kv_cache_append_rope(const csld_layer_cache* cache, const uint16_t* kv_new,
+                                 const float* gate_new, double rope_base, int32_t* err, void* stream) {
+    if (!(rope_base > 1.0) || rope_base == INFINITY) return fail(CSLD_ERR_ARG, "rope_base must be finite and > 1");
+    return append_impl("kv_cache_append_rope", cache, kv_new, gate_new, err, rope_base, stream);
+}
+
+namespace {
+csld_status prefill_impl(const csld_layer_cache* cache, const uint16_t* raw, const float* gate, int64_t T,
+                         double rope_base, void* stream) {
     csld_status s = check_cache(cache);
     if (s != CSLD_OK) return s;
     if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
@@ -166,12 +198,24 @@ csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint16_t* raw,
     cudaError_t e = csld::launch_compress(raw, gate, cache->pos_bias, cache->ratio,
                                           cache->has_indexer ? cache->w_idx : nullptr, T, cache->batch,
                                           cache->capacity, cache->comp_kv, cache->ikeys,
-                                          cache->iscales, num_sms(), st);
+                                          cache->iscales, num_sms(), st, 0, rope_base);
     if (e != cudaSuccess) return cuda_fail(e, "kv_cache_prefill (compress)");
     e = csld::launch_prefill_state(raw, gate, T, cache->ratio, cache->window, cache->batch,
-                                   cache->win_kv, cache->tail_kv, cache->tail_gate, cache->seq_len, st);
+                                   cache->win_kv, cache->tail_kv, cache->tail_gate, cache->seq_len, st, rope_base);
     if (e != cudaSuccess) return cuda_fail(e, "kv_cache_prefill (state)");
     return CSLD_OK;
+}
+}  // namespace
+
+csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
+                             int64_t T, void* stream) {
+    return prefill_impl(cache, raw, gate, T, 0.0, stream);
+}
+
+csld_status kv_cache_prefill_rope(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
+                                  int64_t T, double rope_base, void* stream) {
+    if (!(rope_base > 1.0) || rope_base == INFINITY) return fail(CSLD_ERR_ARG, "rope_base must be finite and > 1");
+    return prefill_impl(cache, raw, gate, T, rope_base, stream);
 }
 
 size_t csld_indexer_workspace_size(int B, int64_t cap, int k) {

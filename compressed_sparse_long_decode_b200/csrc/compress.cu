@@ -11,6 +11,11 @@
 // staged as bf16 in shared memory and projected by W_I (512x64, bf16 copy resident in shared
 // memory for the whole persistent CTA) on the 5th-generation tensor cores (tcgen05.mma
 // kind::f16, fp32 accumulation in tensor memory); the FP4 quantisation runs on the fp32 result.
+//
+// RoPE at compressed positions (a layout variant of the storage paragraph's bf16 RoPE dims):
+// the kernels below are also compiled with kRope, where the raw tokens' dims 448..511 are taken
+// before rotary encoding and rotated here -- a pooled entry at its block's last token, a window
+// entry at its own token (RoFormer pairs, see rope_lane).
 #include "csld_internal.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -115,6 +120,39 @@ __device__ __forceinline__ void warp_pool(const uint16_t* rows, const float* gat
     }
 }
 
+// RoPE of a pooled vector held by a warp (lane l: dims 16l..16l+15; lanes 28..31 hold the RoPE
+// dims 448..511): pair i = dims (448 + 2i, 449 + 2i) turned by the angle pos * base^(-i/32)
+// (RoFormer).  The angle, its sine and cosine and the products in double (the position may be
+// in the millions), the result rounded to fp32.
+__device__ __forceinline__ void rope_lane(float (&c)[16], int lane, int64_t pos, double base) {
+    if (lane < kNope / 16) return;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        const int i = 8 * (lane - kNope / 16) + p;
+        double sn, cs;
+        sincos(static_cast<double>(pos) * pow(base, -static_cast<double>(i) / 32.0), &sn, &cs);
+        const double x0 = c[2 * p], x1 = c[2 * p + 1];
+        c[2 * p] = static_cast<float>(x0 * cs - x1 * sn);
+        c[2 * p + 1] = static_cast<float>(x0 * sn + x1 * cs);
+    }
+}
+// The same rotation for four consecutive RoPE dims 448 + 4j .. 448 + 4j + 3 held as bf16 (two
+// pairs), rounded back to bf16: a window entry's RoPE part.
+__device__ __forceinline__ uint2 rope_bf16x4(uint2 x, int j, int64_t pos, double base) {
+    const float v[4] = {bf16_bits_to_f32(x.x), bf16_bits_to_f32(x.x >> 16), bf16_bits_to_f32(x.y),
+                        bf16_bits_to_f32(x.y >> 16)};
+    uint32_t w[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        double sn, cs;
+        sincos(static_cast<double>(pos) * pow(base, -static_cast<double>(2 * j + p) / 32.0), &sn, &cs);
+        const double x0 = v[2 * p], x1 = v[2 * p + 1];
+        w[p] = f32_to_bf16_bits(static_cast<float>(x0 * cs - x1 * sn)) |
+               (f32_to_bf16_bits(static_cast<float>(x0 * sn + x1 * cs)) << 16);
+    }
+    return make_uint2(w[0], w[1]);
+}
+
 // Writes the 576-byte entry of the pooled vector held by the warp (lane l: dims 16l..16l+15).
 __device__ __forceinline__ void warp_store_entry(uint8_t* __restrict__ entry, int lane,
                                                  const float (&c)[16]) {
@@ -153,12 +191,13 @@ __device__ __forceinline__ void warp_store_fp4(uint8_t* __restrict__ codes, floa
 // ------------------------------------------------------------------------------------------
 // Pooling without an indexer key (HCA, or any ratio).  One warp per entry.
 // ------------------------------------------------------------------------------------------
+template <bool kRope>
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ raw,
                                                    const float* __restrict__ gate,
                                                    const float* __restrict__ bias, int m,
                                                    int64_t T, int64_t E, int B,
                                                    int64_t out_seq_stride,
-                                                   uint8_t* __restrict__ kv_out) {
+                                                   uint8_t* __restrict__ kv_out, int64_t pos0, double rope_base) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (gw >= E * B) return;
@@ -166,6 +205,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
     float c[16];
     warp_pool<true>(raw + ((size_t)b * T + (size_t)s * m) * kDim, gate + (size_t)b * T + (size_t)s * m,
               bias, m, lane, c);
+    if constexpr (kRope) rope_lane(c, lane, pos0 + (s + 1) * m - 1, rope_base);
     warp_store_entry(kv_out + ((size_t)b * out_seq_stride + (size_t)s) * kEntry, lane, c);
 }
 
@@ -226,11 +266,12 @@ __device__ __forceinline__ void pool4_preloaded(const uint4 (&x)[8], const float
 }
 
 // kM4: the block ratio is 4 (two blocks' raw rows are loaded at once); otherwise any ratio.
-template <bool kM4>
+template <bool kM4, bool kRope>
 __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
     const uint16_t* __restrict__ raw, const float* __restrict__ gate, const float* __restrict__ bias,
     int m, const float* __restrict__ w_idx, int64_t T, int64_t E, int B, int64_t out_seq_stride,
-    uint8_t* __restrict__ kv_out, uint8_t* __restrict__ ikey_out, float* __restrict__ iscale_out) {
+    uint8_t* __restrict__ kv_out, uint8_t* __restrict__ ikey_out, float* __restrict__ iscale_out, int64_t pos0,
+    double rope_base) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     CompressSmem& sm = *reinterpret_cast<CompressSmem*>(smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -305,6 +346,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                         float w[4];
                         warp_pool_weights_pre(ga[h] + bias_l, 4, lane, w);
                         pool4_preloaded(x[h], w, c);
+                        if constexpr (kRope) rope_lane(c, lane, pos0 + (s0 + r + 1) * 4 - 1, rope_base);
                         warp_store_entry(kvb + (size_t)(s0 + r) * kEntry, lane, c);
                     } else {
 #pragma unroll
@@ -321,6 +363,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                     float c[16];
                     if (r < n_here) {
                         warp_pool<true>(rb + (size_t)(s0 + r) * m * kDim, gb + (s0 + r) * m, bias, m, lane, c);
+                        if constexpr (kRope) rope_lane(c, lane, pos0 + (s0 + r + 1) * m - 1, rope_base);
                         warp_store_entry(kvb + (size_t)(s0 + r) * kEntry, lane, c);
                     } else {
 #pragma unroll
@@ -425,24 +468,27 @@ size_t compress_index_smem_bytes() { return sizeof(CompressSmem) + 1024; }
 cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float* bias, int m,
                             const float* w_idx, int64_t T, int B, int64_t out_seq_stride,
                             uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, int num_sms,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, int64_t pos0, double rope_base) {
     const int64_t E = T / m;
     if (E <= 0 || B <= 0) return cudaSuccess;
+    const bool rope = rope_base > 0.0;
     if (w_idx == nullptr) {
         const int64_t warps = E * B;
         const int64_t blocks = (warps + 7) / 8;
-        pool_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(raw, gate, bias, m, T, E, B,
-                                                                       out_seq_stride, kv_out);
+        auto kernel = rope ? pool_kernel<true> : pool_kernel<false>;
+        kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(raw, gate, bias, m, T, E, B, out_seq_stride, kv_out,
+                                                                  pos0, rope_base);
         return cudaGetLastError();
     }
     const size_t smem = compress_index_smem_bytes();
     const int64_t tiles = ((E + kCTile - 1) / kCTile) * B;
     const int64_t grid = min64(tiles, num_sms);
-    auto kernel = (m == 4) ? pool_index_kernel<true> : pool_index_kernel<false>;
+    auto kernel = (m == 4) ? (rope ? pool_index_kernel<true, true> : pool_index_kernel<true, false>)
+                           : (rope ? pool_index_kernel<false, true> : pool_index_kernel<false, false>);
     cudaError_t e = set_smem_once(kernel, smem);
     if (e != cudaSuccess) return e;
     kernel<<<static_cast<unsigned>(grid), kCThreads, smem, stream>>>(raw, gate, bias, m, w_idx, T, E, B, out_seq_stride,
-                                                                     kv_out, ikey_out, iscale_out);
+                                                                     kv_out, ikey_out, iscale_out, pos0, rope_base);
     return cudaGetLastError();
 }
 
@@ -569,13 +615,14 @@ cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, cons
 // ------------------------------------------------------------------------------------------
 // Window ring + tail after a prefill of T tokens (one CTA per sequence).
 // ------------------------------------------------------------------------------------------
+template <bool kRope>
 __global__ void __launch_bounds__(128) prefill_state_kernel(const uint16_t* __restrict__ raw,
                                                             const float* __restrict__ gate,
                                                             int64_t T, int m, int W,
                                                             uint8_t* __restrict__ win_kv,
                                                             uint16_t* __restrict__ tail_kv,
                                                             float* __restrict__ tail_gate,
-                                                            int32_t* __restrict__ seq_len) {
+                                                            int32_t* __restrict__ seq_len, double rope_base) {
     const int b = blockIdx.x, tid = threadIdx.x;
     const uint16_t* rb = raw + (size_t)b * T * kDim;
     // window: tokens max(0, T-W) .. T-1; thread handles 4 dims (8 bytes of bf16)
@@ -589,7 +636,9 @@ __global__ void __launch_bounds__(128) prefill_state_kernel(const uint16_t* __re
                                (f32_to_e4m3(bf16_bits_to_f32(x.y >> 16)) << 24);
             *reinterpret_cast<uint32_t*>(e + 4 * tid) = v;
         } else {
-            *reinterpret_cast<uint2*>(e + kNope + 8 * (tid - kNope / 4)) = x;
+            uint2 y = x;
+            if constexpr (kRope) y = rope_bf16x4(x, tid - kNope / 4, t, rope_base);   // at token t
+            *reinterpret_cast<uint2*>(e + kNope + 8 * (tid - kNope / 4)) = y;
         }
     }
     const int64_t t0 = T - (T % m);
@@ -603,8 +652,9 @@ __global__ void __launch_bounds__(128) prefill_state_kernel(const uint16_t* __re
 
 cudaError_t launch_prefill_state(const uint16_t* raw, const float* gate, int64_t T, int m, int W,
                                  int B, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
-                                 int32_t* seq_len, cudaStream_t stream) {
-    prefill_state_kernel<<<B, 128, 0, stream>>>(raw, gate, T, m, W, win_kv, tail_kv, tail_gate, seq_len);
+                                 int32_t* seq_len, cudaStream_t stream, double rope_base) {
+    auto kernel = rope_base > 0.0 ? prefill_state_kernel<true> : prefill_state_kernel<false>;
+    kernel<<<B, 128, 0, stream>>>(raw, gate, T, m, W, win_kv, tail_kv, tail_gate, seq_len, rope_base);
     return cudaGetLastError();
 }
 
@@ -620,10 +670,11 @@ namespace csld {
 // ------------------------------------------------------------------------------------------
 constexpr int kAppendThreads = 256;
 
+template <bool kRope>
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache cache,
                                                                 const uint16_t* __restrict__ kv_new,
                                                                 const float* __restrict__ gate_new,
-                                                                int32_t* err) {
+                                                                int32_t* err, double rope_base) {
     __shared__ float cbuf[kDim];
     __shared__ float upart[kAppendThreads / 32][kIdxDim];
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -654,7 +705,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
                                (f32_to_e4m3(bf16_bits_to_f32(x.y >> 16)) << 24);
             *reinterpret_cast<uint32_t*>(e + 4 * tid) = v;
         } else {
-            *reinterpret_cast<uint2*>(e + kNope + 8 * (tid - kNope / 4)) = x;
+            uint2 y = x;
+            if constexpr (kRope) y = rope_bf16x4(x, tid - kNope / 4, t, rope_base);   // at token t
+            *reinterpret_cast<uint2*>(e + kNope + 8 * (tid - kNope / 4)) = y;
         }
     }
     uint16_t* tail = cache.tail_kv + (size_t)b * m * kDim;
@@ -666,6 +719,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
         if (warp == 0) {
             float c[16];
             warp_pool<false>(tail, tgate, cache.pos_bias, m, lane, c);
+            if constexpr (kRope) rope_lane(c, lane, t, rope_base);   // token t ends the block
             warp_store_entry(cache.comp_kv + ((size_t)b * cap + (size_t)s) * kEntry, lane, c);
 #pragma unroll
             for (int d = 0; d < 16; ++d) cbuf[16 * lane + d] = bf16_bits_to_f32(f32_to_bf16_bits(c[d]));
@@ -702,8 +756,12 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
 }
 
 cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
-                          const float* gate_new, int32_t* err, cudaStream_t stream) {
-    cudaError_t e = launch_pdl(append_kernel, dim3(cache.batch), dim3(kAppendThreads), 0, stream, cache, kv_new, gate_new, err);
+                          const float* gate_new, int32_t* err, cudaStream_t stream, double rope_base) {
+    cudaError_t e = rope_base > 0.0
+                        ? launch_pdl(append_kernel<true>, dim3(cache.batch), dim3(kAppendThreads), 0, stream, cache,
+                                     kv_new, gate_new, err, rope_base)
+                        : launch_pdl(append_kernel<false>, dim3(cache.batch), dim3(kAppendThreads), 0, stream, cache,
+                                     kv_new, gate_new, err, rope_base);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -9,10 +9,12 @@
 
 namespace csld {
 
+// rope_base > 0: RoPE at compressed positions, raw token 0 at position pos0 (entry s rotated at
+// pos0 + (s+1) m - 1); 0: the entries' RoPE dims are pooled as given.
 cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float* bias, int m,
                             const float* w_idx, int64_t T, int B, int64_t out_seq_stride,
                             uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, int64_t pos0 = 0, double rope_base = 0.0);
 size_t compress_index_smem_bytes();
 cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, const float* bias, int m,
                                     const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
@@ -20,10 +22,10 @@ cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, cons
 
 cudaError_t launch_prefill_state(const uint16_t* raw, const float* gate, int64_t T, int m, int W,
                                  int B, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
-                                 int32_t* seq_len, cudaStream_t stream);
+                                 int32_t* seq_len, cudaStream_t stream, double rope_base = 0.0);
 
 cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
-                          const float* gate_new, int32_t* err, cudaStream_t stream);
+                          const float* gate_new, int32_t* err, cudaStream_t stream, double rope_base = 0.0);
 
 // Lightning indexer + top-k.
 struct IndexerPlan {

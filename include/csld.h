@@ -135,6 +135,26 @@ CSLD_API csld_status csld_compress_channel(const uint16_t* raw, const float* gat
                                            uint8_t* ikey_out, float* iscale_out, void* stream);
 
 /* ----------------------------------------------------------------------------------------
+ * RoPE at compressed positions -- a layout variant of the storage paragraph ([HF]: each
+ * entry keeps its RoPE dims in bf16), where the library applies the rotary position encoding
+ * itself instead of storing the RoPE dims as given.  raw's dims 448..511 are taken BEFORE
+ * rotary encoding.  Entry s (tokens s*m .. s*m+m-1 of raw) is pooled exactly as by
+ * csld_compress; then its dims 448..511 are rotated at the position of its block's last token,
+ *   p_s = pos0 + (s+1)*ratio - 1,
+ * pair i = dims (448 + 2i, 449 + 2i), i = 0..31, turned by the angle p_s * rope_base^(-i/32)
+ * (RoFormer), before the bf16 rounding of the entry and before the indexer key is projected
+ * (the key is the FP4 code of the rotated vector times W_I).  pos0 = position of raw[0],
+ * 0 <= pos0 <= 2^40; rope_base finite and > 1 (10000 in the usual setting).  The query's RoPE
+ * dims are the caller's to rotate, at the query's own position.  Arguments, layouts, alignment
+ * and errors otherwise as csld_compress; rotations are computed in double and rounded to fp32,
+ * so the stored bf16 values agree with an exact rotation to within one bf16 step.
+ * -------------------------------------------------------------------------------------- */
+CSLD_API csld_status csld_compress_rope(const uint16_t* raw, const float* gate, const float* pos_bias,
+                                        int ratio, const float* w_idx, int64_t T, int64_t pos0,
+                                        double rope_base, uint8_t* kv_out, uint8_t* ikey_out,
+                                        float* iscale_out, void* stream);
+
+/* ----------------------------------------------------------------------------------------
  * One layer's KV-cache state for B sequences ([VEL] KV-cache-layout section: compressed
  * cache, separate sliding-window state, separately kept uncompressed tail).  A host struct of
  * device pointers; the caller owns all of it.
@@ -182,6 +202,18 @@ CSLD_API csld_status kv_cache_append(const csld_layer_cache* cache, const uint16
  * an empty cache.  Requires T/m <= capacity. */
 CSLD_API csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint16_t* raw,
                              const float* gate, int64_t T, void* stream);
+
+/* kv_cache_append / kv_cache_prefill with RoPE at compressed positions (see csld_compress_rope):
+ * the tokens' dims 448..511 arrive before rotary encoding; token t's window entry holds them
+ * rotated at position t, and a completed entry s is rotated at position (s+1)*ratio - 1, the
+ * token that completes it (the tail keeps the tokens as given).  Positions count from 0 at the
+ * first token of each sequence.  rope_base finite and > 1; a cache must be filled by one kind
+ * of call throughout.  Otherwise as kv_cache_append / kv_cache_prefill. */
+CSLD_API csld_status kv_cache_append_rope(const csld_layer_cache* cache, const uint16_t* kv_new,
+                                          const float* gate_new, double rope_base, int32_t* err,
+                                          void* stream);
+CSLD_API csld_status kv_cache_prefill_rope(const csld_layer_cache* cache, const uint16_t* raw,
+                                           const float* gate, int64_t T, double rope_base, void* stream);
 
 /* ----------------------------------------------------------------------------------------
  * Lightning indexer + top-k ([HF] CSA paragraph: "FP4, ReLU-scored multi-head dot product"
