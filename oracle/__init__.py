@@ -96,9 +96,18 @@ def _declare(L):
     L.orc_append_batch.restype = C.c_int
     L.orc_append_batch.argtypes = [C.c_int, C.c_int, C.c_int64, C.c_int, _P, _P, _P, _P, _P, _P,
                                    _P, _P, _P, _P, _P]
-    L.orc_append_batch_rope.restype = C.c_int
-    L.orc_append_batch_rope.argtypes = [C.c_int, C.c_int, C.c_int64, C.c_int, _P, _P, _P, _P, _P, _P,
-                                        _P, _P, _P, _P, _P, C.c_double]
+    L.orc_append_batch_variant.restype = C.c_int
+    L.orc_append_batch_variant.argtypes = [C.c_int, C.c_int, C.c_int64, C.c_int, _P, _P, _P, _P, _P, _P,
+                                           _P, _P, _P, _P, _P, C.c_double, C.c_double]
+    L.orc_entry_encode_scaled.restype = None
+    L.orc_entry_encode_scaled.argtypes = [_P, C.c_double, _P]
+    L.orc_entry_decode_scaled.restype = None
+    L.orc_entry_decode_scaled.argtypes = [_P, C.c_double, _P]
+    L.orc_compress_scaled.restype = None
+    L.orc_compress_scaled.argtypes = [_P, _P, _P, _P, C.c_int64, C.c_int, C.c_double, _P, _P, _P]
+    L.orc_attention_batch_scaled.restype = C.c_int
+    L.orc_attention_batch_scaled.argtypes = [_P, C.c_int, _P, C.c_int64, C.c_int, _P, C.c_int, _P, C.c_int,
+                                             _P, C.c_int, C.c_double, C.c_double, _P, _P]
     L.orc_num_threads.restype = C.c_int
     L.orc_num_threads.argtypes = []
 
@@ -240,6 +249,37 @@ def compress_rope(raw_bits, gate, bias, m, pos0, base, w_idx=None):
     return kv, ik, isc
 
 
+def entry_encode_scaled(x, kv_scale):
+    """Scaled FP8 entry: E4M3(x / kv_scale) for dims 0..447, bf16 for the RoPE dims."""
+    x = _c(x, np.float64)
+    e = np.zeros(ENTRY_BYTES, np.uint8)
+    lib().orc_entry_encode_scaled(_ptr(x), float(kv_scale), _ptr(e))
+    return e
+
+
+def entry_decode_scaled(entry, kv_scale):
+    entry = _c(entry, np.uint8)
+    x = np.zeros(D, np.float64)
+    lib().orc_entry_decode_scaled(_ptr(entry), float(kv_scale), _ptr(x))
+    return x
+
+
+def compress_scaled(raw_bits, gate, bias, m, kv_scale, w_idx=None):
+    """Prefill compression into scaled FP8 entries.  Returns (kv [E,576], ikeys, iscales)."""
+    raw_bits = _c(raw_bits, np.uint16)
+    gate = _c(gate, np.float32)
+    bias = _c(bias, np.float32)
+    T = raw_bits.shape[0]
+    E = T // m
+    kv = np.zeros((E, ENTRY_BYTES), np.uint8)
+    ik = np.zeros((E, IKEY_BYTES), np.uint8) if w_idx is not None else None
+    isc = np.zeros((E, 2), np.float32) if w_idx is not None else None
+    w = _c(w_idx, np.float32) if w_idx is not None else None
+    lib().orc_compress_scaled(_ptr(raw_bits), _ptr(gate), _ptr(bias), _ptr(w), T, m, float(kv_scale), _ptr(kv),
+                              _ptr(ik), _ptr(isc))
+    return kv, ik, isc
+
+
 def pool_block_channel(raw_bits, gate, bias):
     """Per-channel gating: raw_bits uint16 [m,512]; gate, bias float32 [m,512] -> float64 [512]."""
     raw_bits = _c(raw_bits, np.uint16)
@@ -310,9 +350,10 @@ def indexer_topk_batch(ikeys, iscales, seq_len, ratio, q_idx, head_w, k):
 
 
 # ---- O5 ----------------------------------------------------------------------------------
-def attention_batch(q_bits, comp_kv, ratio, sel, win_kv, seq_len, scale):
+def attention_batch(q_bits, comp_kv, ratio, sel, win_kv, seq_len, scale, kv_scale=1.0):
     """q_bits [B,H,512] u16; comp_kv [B,cap,576]; sel [B,k] i32 or None; win_kv [B,W,576];
-    seq_len [B] i32.  Returns (out [B,H,512] f64, lse [B,H] f64)."""
+    seq_len [B] i32; kv_scale: scaled FP8 entries (1: the base layout).  Returns (out [B,H,512]
+    f64, lse [B,H] f64)."""
     q_bits = _c(q_bits, np.uint16)
     comp_kv = _c(comp_kv, np.uint8)
     win_kv = _c(win_kv, np.uint8)
@@ -326,9 +367,9 @@ def attention_batch(q_bits, comp_kv, ratio, sel, win_kv, seq_len, scale):
         k = sel.shape[1]
     out = np.zeros((B, H, D), np.float64)
     lse = np.zeros((B, H), np.float64)
-    rc = lib().orc_attention_batch(_ptr(q_bits), H, _ptr(comp_kv), cap, ratio, _ptr(sel), k,
-                                   _ptr(win_kv), W, _ptr(seq_len), B, float(scale), _ptr(out),
-                                   _ptr(lse))
+    rc = lib().orc_attention_batch_scaled(_ptr(q_bits), H, _ptr(comp_kv), cap, ratio, _ptr(sel), k,
+                                          _ptr(win_kv), W, _ptr(seq_len), B, float(scale), float(kv_scale),
+                                          _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle attention: a selected index is not a visible entry")
     return out, lse
@@ -349,18 +390,18 @@ class LayerState:
         self.seq_len = np.zeros(B, np.int32)
 
 
-def append_batch(st: LayerState, bias, w_idx, x_bits, gate, rope_base=0.0):
+def append_batch(st: LayerState, bias, w_idx, x_bits, gate, rope_base=0.0, kv_scale=1.0):
     """Append one token per sequence (x_bits [B,512] u16, gate [B] f32).  Raises on overflow.
     rope_base > 0: RoPE at compressed positions (window entry at its token, a completed entry
-    at its block's last token)."""
+    at its block's last token); kv_scale: scaled FP8 entries (1: the base layout)."""
     bias = _c(bias, np.float32)
     w = _c(w_idx, np.float32) if w_idx is not None else None
     x_bits = _c(x_bits, np.uint16)
     gate = _c(gate, np.float32)
-    rc = lib().orc_append_batch_rope(st.m, st.W, st.cap, st.B, _ptr(st.comp_kv), _ptr(st.ikeys),
-                                     _ptr(st.iscales), _ptr(st.win_kv), _ptr(st.tail_kv),
-                                     _ptr(st.tail_gate), _ptr(st.seq_len), _ptr(bias), _ptr(w),
-                                     _ptr(x_bits), _ptr(gate), float(rope_base))
+    rc = lib().orc_append_batch_variant(st.m, st.W, st.cap, st.B, _ptr(st.comp_kv), _ptr(st.ikeys),
+                                        _ptr(st.iscales), _ptr(st.win_kv), _ptr(st.tail_kv),
+                                        _ptr(st.tail_gate), _ptr(st.seq_len), _ptr(bias), _ptr(w),
+                                        _ptr(x_bits), _ptr(gate), float(rope_base), float(kv_scale))
     if rc != 0:
         raise OverflowError("oracle append: compressed cache capacity exceeded")
 

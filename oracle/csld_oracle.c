@@ -27,9 +27,10 @@
  *    orc_indexer_scores); selection is by (score desc, index asc);
  *  - attention is one joint softmax over {selected or all visible compressed entries} and
  *    {the last W raw tokens}; a compressed entry is visible once its last token arrived;
- *  - layout variants: per-channel gating (orc_pool_block_channel) and RoPE applied at
+ *  - layout variants: per-channel gating (orc_pool_block_channel), RoPE applied at
  *    compressed positions (orc_rope_rotate: RoFormer pairs (448+2i, 449+2i), angle
- *    pos * base^(-i/32); an entry at its block's last token, a window entry at its token).
+ *    pos * base^(-i/32); an entry at its block's last token, a window entry at its token) and
+ *    scaled FP8 entries (one scale per layer cache: E4M3(x / sigma), RoPE dims unscaled).
  *
  * parity unpinned: the real model's gate form, indexer projection and FP4 scale rule are not
  * given by the pages (no weights); what is pinned is listed in the tests.
@@ -209,6 +210,20 @@ void orc_entry_decode(const uint8_t* entry, double* x) {
     }
 }
 
+/* Scaled FP8 entries (a layout variant of the storage paragraph's FP8 entries): one positive
+ * scale sigma per layer cache; the E4M3 dims hold E4M3(x / sigma) and stand for sigma times
+ * their code value, the bf16 RoPE dims are unscaled.  sigma = 1 is the base layout. */
+void orc_entry_encode_scaled(const double* x, double kv_scale, uint8_t* entry) {
+    double y[ORC_D];
+    for (int d = 0; d < ORC_D; ++d) y[d] = d < ORC_D_NOPE ? x[d] / kv_scale : x[d];
+    orc_entry_encode(y, entry);
+}
+
+void orc_entry_decode_scaled(const uint8_t* entry, double kv_scale, double* x) {
+    orc_entry_decode(entry, x);
+    for (int d = 0; d < ORC_D_NOPE; ++d) x[d] *= kv_scale;
+}
+
 /* ------------------------------------------------------------------------------------------
  * O1 -- softmax-gated pooling with a learned positional bias ([HF] CSA paragraph: "compresses
  * KV entries 4x along the sequence with softmax-gated pooling and a learned positional bias";
@@ -295,7 +310,7 @@ void orc_rope_rotate(double* x, double pos, double base) {
  * (CSA; [HF] CSA paragraph: the lightning indexer runs over the 4x-compressed entries).
  * rope_base > 0: O1r, entry s rotated at position pos0 + (s+1) m - 1 after pooling. */
 static void orc_compress_impl(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
-                              int64_t T, int m, int64_t pos0, double rope_base, uint8_t* kv_out,
+                              int64_t T, int m, int64_t pos0, double rope_base, double kv_scale, uint8_t* kv_out,
                               uint8_t* ikey_out, float* iscale_out) {
     int64_t E = T / m;
 #pragma omp parallel for schedule(static)
@@ -303,7 +318,10 @@ static void orc_compress_impl(const uint16_t* raw, const float* gate, const floa
         double c[ORC_D], u[ORC_IDX_DIM];
         orc_pool_block(raw + (size_t)s * m * ORC_D, gate + (size_t)s * m, bias, m, c);
         if (rope_base > 0.0) orc_rope_rotate(c, (double)(pos0 + (s + 1) * (int64_t)m - 1), rope_base);
-        orc_entry_encode(c, kv_out + (size_t)s * ORC_ENTRY_BYTES);
+        if (kv_scale != 1.0)
+            orc_entry_encode_scaled(c, kv_scale, kv_out + (size_t)s * ORC_ENTRY_BYTES);
+        else
+            orc_entry_encode(c, kv_out + (size_t)s * ORC_ENTRY_BYTES);
         if (w_idx) {
             orc_indexer_key_raw(c, w_idx, u);
             orc_fp4_quantize64(u, ikey_out + (size_t)s * ORC_IKEY_BYTES, iscale_out + (size_t)s * 2);
@@ -313,14 +331,21 @@ static void orc_compress_impl(const uint16_t* raw, const float* gate, const floa
 
 void orc_compress(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
                   int64_t T, int m, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
-    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, kv_out, ikey_out, iscale_out);
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, 1.0, kv_out, ikey_out, iscale_out);
 }
 
 /* O1r + O1 + O2: raw token 0 at position pos0, rotation base rope_base > 0. */
 void orc_compress_rope(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
                        int64_t T, int m, int64_t pos0, double rope_base, uint8_t* kv_out,
                        uint8_t* ikey_out, float* iscale_out) {
-    orc_compress_impl(raw, gate, bias, w_idx, T, m, pos0, rope_base, kv_out, ikey_out, iscale_out);
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, pos0, rope_base, 1.0, kv_out, ikey_out, iscale_out);
+}
+
+/* Scaled FP8 entries: as orc_compress with entries encoded by orc_entry_encode_scaled (the
+ * indexer key is projected from the unscaled pooled vector). */
+void orc_compress_scaled(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
+                         int64_t T, int m, double kv_scale, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, kv_scale, kv_out, ikey_out, iscale_out);
 }
 
 /* O1 (per-channel) + O2 over a whole prefill: gate [T][512], bias [m][512]. */
@@ -472,9 +497,9 @@ void orc_indexer_topk_batch(const uint8_t* ikeys, const float* iscales, int64_t 
  * Returns 0, or -1 when a selected index is not a visible entry.
  * An empty key set gives out = 0 and lse = -inf.
  * ---------------------------------------------------------------------------------------- */
-int orc_attention(const uint16_t* q, int H, const uint8_t* comp_kv, int64_t cap, int ratio,
-                  const int32_t* sel, int k, const uint8_t* win_kv, int W, int32_t seq_len,
-                  double scale, double* out, double* lse) {
+static int orc_attention_impl(const uint16_t* q, int H, const uint8_t* comp_kv, int64_t cap, int ratio,
+                              const int32_t* sel, int k, const uint8_t* win_kv, int W, int32_t seq_len,
+                              double scale, double kv_scale, double* out, double* lse) {
     int64_t n_vis = seq_len / ratio;
     if (n_vis > cap) n_vis = cap;
     int64_t n_comp = 0;
@@ -494,13 +519,14 @@ int orc_attention(const uint16_t* q, int H, const uint8_t* comp_kv, int64_t cap,
     int64_t j = 0;
     if (sel) {
         for (int i = 0; i < k; ++i)
-            if (sel[i] >= 0) orc_entry_decode(comp_kv + (size_t)sel[i] * ORC_ENTRY_BYTES, kv + (size_t)(j++) * ORC_D);
+            if (sel[i] >= 0)
+                orc_entry_decode_scaled(comp_kv + (size_t)sel[i] * ORC_ENTRY_BYTES, kv_scale, kv + (size_t)(j++) * ORC_D);
     } else {
         for (int64_t s = 0; s < n_vis; ++s)
-            orc_entry_decode(comp_kv + (size_t)s * ORC_ENTRY_BYTES, kv + (size_t)(j++) * ORC_D);
+            orc_entry_decode_scaled(comp_kv + (size_t)s * ORC_ENTRY_BYTES, kv_scale, kv + (size_t)(j++) * ORC_D);
     }
     for (int64_t t = w0; t < seq_len && W > 0; ++t)
-        orc_entry_decode(win_kv + (size_t)(t % W) * ORC_ENTRY_BYTES, kv + (size_t)(j++) * ORC_D);
+        orc_entry_decode_scaled(win_kv + (size_t)(t % W) * ORC_ENTRY_BYTES, kv_scale, kv + (size_t)(j++) * ORC_D);
 
     double* logit = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
     for (int h = 0; h < H; ++h) {
@@ -532,19 +558,33 @@ int orc_attention(const uint16_t* q, int H, const uint8_t* comp_kv, int64_t cap,
     return 0;
 }
 
-/* Batched attention: q [B][H][512]; caches [B][cap] and [B][W]; sel [B][k] or NULL. */
-int orc_attention_batch(const uint16_t* q, int H, const uint8_t* comp_kv, int64_t cap, int ratio,
-                        const int32_t* sel, int k, const uint8_t* win_kv, int W,
-                        const int32_t* seq_len, int B, double scale, double* out, double* lse) {
+int orc_attention(const uint16_t* q, int H, const uint8_t* comp_kv, int64_t cap, int ratio,
+                  const int32_t* sel, int k, const uint8_t* win_kv, int W, int32_t seq_len,
+                  double scale, double* out, double* lse) {
+    return orc_attention_impl(q, H, comp_kv, cap, ratio, sel, k, win_kv, W, seq_len, scale, 1.0, out, lse);
+}
+
+/* Batched attention: q [B][H][512]; caches [B][cap] and [B][W]; sel [B][k] or NULL;
+ * kv_scale: scaled FP8 entries (1: the base layout). */
+int orc_attention_batch_scaled(const uint16_t* q, int H, const uint8_t* comp_kv, int64_t cap, int ratio,
+                               const int32_t* sel, int k, const uint8_t* win_kv, int W,
+                               const int32_t* seq_len, int B, double scale, double kv_scale, double* out,
+                               double* lse) {
     int rc = 0;
 #pragma omp parallel for schedule(dynamic) reduction(| : rc)
     for (int b = 0; b < B; ++b) {
-        rc |= orc_attention(q + (size_t)b * H * ORC_D, H, comp_kv + (size_t)b * cap * ORC_ENTRY_BYTES,
-                            cap, ratio, sel ? sel + (size_t)b * k : NULL, k,
-                            win_kv + (size_t)b * (W > 0 ? W : 0) * ORC_ENTRY_BYTES, W, seq_len[b],
-                            scale, out + (size_t)b * H * ORC_D, lse + (size_t)b * H);
+        rc |= orc_attention_impl(q + (size_t)b * H * ORC_D, H, comp_kv + (size_t)b * cap * ORC_ENTRY_BYTES,
+                                 cap, ratio, sel ? sel + (size_t)b * k : NULL, k,
+                                 win_kv + (size_t)b * (W > 0 ? W : 0) * ORC_ENTRY_BYTES, W, seq_len[b],
+                                 scale, kv_scale, out + (size_t)b * H * ORC_D, lse + (size_t)b * H);
     }
     return rc;
+}
+
+int orc_attention_batch(const uint16_t* q, int H, const uint8_t* comp_kv, int64_t cap, int ratio,
+                        const int32_t* sel, int k, const uint8_t* win_kv, int W,
+                        const int32_t* seq_len, int B, double scale, double* out, double* lse) {
+    return orc_attention_batch_scaled(q, H, comp_kv, cap, ratio, sel, k, win_kv, W, seq_len, B, scale, 1.0, out, lse);
 }
 
 /* ------------------------------------------------------------------------------------------
@@ -563,7 +603,7 @@ int orc_attention_batch(const uint16_t* q, int H, const uint8_t* comp_kv, int64_
 static int orc_append_impl(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, float* iscales,
                            uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate, int32_t* seq_len,
                            const float* bias, const float* w_idx, const uint16_t* x, float gate,
-                           double rope_base) {
+                           double rope_base, double kv_scale) {
     int32_t t = *seq_len;
     int complete = ((t + 1) % m) == 0;
     int64_t s = t / m;
@@ -572,7 +612,7 @@ static int orc_append_impl(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t*
         double xd[ORC_D];
         for (int d = 0; d < ORC_D; ++d) xd[d] = orc_bf16_decode(x[d]);
         if (rope_base > 0.0) orc_rope_rotate(xd, (double)t, rope_base);
-        orc_entry_encode(xd, win_kv + (size_t)(t % W) * ORC_ENTRY_BYTES);
+        orc_entry_encode_scaled(xd, kv_scale, win_kv + (size_t)(t % W) * ORC_ENTRY_BYTES);
     }
     memcpy(tail_kv + (size_t)(t % m) * ORC_D, x, sizeof(uint16_t) * ORC_D);
     tail_gate[t % m] = gate;
@@ -580,7 +620,7 @@ static int orc_append_impl(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t*
         double c[ORC_D], u[ORC_IDX_DIM];
         orc_pool_block(tail_kv, tail_gate, bias, m, c);
         if (rope_base > 0.0) orc_rope_rotate(c, (double)t, rope_base);
-        orc_entry_encode(c, comp_kv + (size_t)s * ORC_ENTRY_BYTES);
+        orc_entry_encode_scaled(c, kv_scale, comp_kv + (size_t)s * ORC_ENTRY_BYTES);
         if (w_idx) {
             orc_indexer_key_raw(c, w_idx, u);
             orc_fp4_quantize64(u, ikeys + (size_t)s * ORC_IKEY_BYTES, iscales + (size_t)s * 2);
@@ -594,14 +634,15 @@ int orc_append(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, floa
                uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate, int32_t* seq_len,
                const float* bias, const float* w_idx, const uint16_t* x, float gate) {
     return orc_append_impl(m, W, cap, comp_kv, ikeys, iscales, win_kv, tail_kv, tail_gate, seq_len, bias,
-                           w_idx, x, gate, 0.0);
+                           w_idx, x, gate, 0.0, 1.0);
 }
 
-/* The same for B sequences, one token each: x [B][512], gate [B]; rope_base as above (0: none). */
-int orc_append_batch_rope(int m, int W, int64_t cap, int B, uint8_t* comp_kv, uint8_t* ikeys,
-                          float* iscales, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
-                          int32_t* seq_len, const float* bias, const float* w_idx, const uint16_t* x,
-                          const float* gate, double rope_base) {
+/* The same for B sequences, one token each: x [B][512], gate [B]; rope_base as above (0: none);
+ * kv_scale: scaled FP8 entries (1: the base layout). */
+int orc_append_batch_variant(int m, int W, int64_t cap, int B, uint8_t* comp_kv, uint8_t* ikeys,
+                             float* iscales, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
+                             int32_t* seq_len, const float* bias, const float* w_idx, const uint16_t* x,
+                             const float* gate, double rope_base, double kv_scale) {
     int rc = 0;
     for (int b = 0; b < B; ++b) {
         rc |= orc_append_impl(m, W, cap, comp_kv + (size_t)b * cap * ORC_ENTRY_BYTES,
@@ -609,7 +650,7 @@ int orc_append_batch_rope(int m, int W, int64_t cap, int B, uint8_t* comp_kv, ui
                               iscales ? iscales + (size_t)b * cap * 2 : NULL,
                               win_kv + (size_t)b * (W > 0 ? W : 0) * ORC_ENTRY_BYTES,
                               tail_kv + (size_t)b * m * ORC_D, tail_gate + (size_t)b * m, seq_len + b,
-                              bias, w_idx, x + (size_t)b * ORC_D, gate[b], rope_base);
+                              bias, w_idx, x + (size_t)b * ORC_D, gate[b], rope_base, kv_scale);
     }
     return rc;
 }
@@ -618,8 +659,8 @@ int orc_append_batch(int m, int W, int64_t cap, int B, uint8_t* comp_kv, uint8_t
                      float* iscales, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
                      int32_t* seq_len, const float* bias, const float* w_idx, const uint16_t* x,
                      const float* gate) {
-    return orc_append_batch_rope(m, W, cap, B, comp_kv, ikeys, iscales, win_kv, tail_kv, tail_gate, seq_len,
-                                 bias, w_idx, x, gate, 0.0);
+    return orc_append_batch_variant(m, W, cap, B, comp_kv, ikeys, iscales, win_kv, tail_kv, tail_gate, seq_len,
+                                    bias, w_idx, x, gate, 0.0, 1.0);
 }
 
 int orc_num_threads(void) {
