@@ -17,7 +17,8 @@ import torch
 
 __all__ = [
     "csa_compress", "hca_compress", "compress", "compress_channel", "compress_rope", "kv_cache_append_rope",
-    "kv_cache_prefill_rope", "indexer_topk", "hybrid_decode_attention",
+    "kv_cache_prefill_rope", "compress_scaled", "kv_cache_append_scaled", "kv_cache_prefill_scaled",
+    "hybrid_decode_attention_scaled", "indexer_topk", "hybrid_decode_attention",
     "kv_cache_append", "kv_cache_prefill", "LayerCache", "CsldError", "lib", "ENTRY_BYTES",
     "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace", "DecodeStack",
     "layer_pattern", "stage", "indexer_rescore", "topk_merge", "lse_merge", "ContextParallelLayer",
@@ -66,6 +67,10 @@ def _load():
     L.csld_compress_rope.argtypes = [P, P, P, I, P, I64, I64, C.c_double, P, P, P, P]
     L.kv_cache_append_rope.argtypes = [C.POINTER(_Cache), P, P, C.c_double, P, P]
     L.kv_cache_prefill_rope.argtypes = [C.POINTER(_Cache), P, P, I64, C.c_double, P]
+    L.csld_compress_scaled.argtypes = [P, P, P, I, P, I64, F, P, P, P, P]
+    L.kv_cache_append_scaled.argtypes = [C.POINTER(_Cache), P, P, F, P, P]
+    L.kv_cache_prefill_scaled.argtypes = [C.POINTER(_Cache), P, P, I64, F, P]
+    L.hybrid_decode_attention_scaled.argtypes = [P, I, P, I64, I, P, I, P, I, P, I, F, F, P, P, P, S, P, P]
     L.csa_compress.argtypes = [P, P, P, P, I64, P, P, P, P]
     L.hca_compress.argtypes = [P, P, P, I64, P, P]
     L.kv_cache_append.argtypes = [C.POINTER(_Cache), P, P, P, P]
@@ -85,7 +90,8 @@ def _load():
     L.csld_topk_merge.argtypes = [P, P, P, I, I, I, I64, I64, P, P]
     L.csld_lse_merge.argtypes = [P, P, I, I, I, P, P, P]
     for fn in ("csld_compress", "csld_compress_channel", "csld_compress_rope", "kv_cache_append_rope",
-               "kv_cache_prefill_rope", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
+               "kv_cache_prefill_rope", "csld_compress_scaled", "kv_cache_append_scaled", "kv_cache_prefill_scaled",
+               "hybrid_decode_attention_scaled", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
                "indexer_topk", "hybrid_decode_attention", "csld_stage", "indexer_rescore", "csld_topk_merge",
                "csld_lse_merge", "indexer_topk_multi", "hybrid_decode_attention_multi"):
         getattr(L, fn).restype = I
@@ -197,6 +203,27 @@ def compress_rope(raw, gate, pos_bias, ratio, pos0, rope_base, w_idx=None, kv_ou
     return (kv_out, ikey_out, iscale_out) if w_idx is not None else kv_out
 
 
+def compress_scaled(raw, gate, pos_bias, ratio, kv_scale, w_idx=None, kv_out=None, ikey_out=None, iscale_out=None):
+    """Compression into scaled FP8 entries (csld_compress_scaled)."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    _need(pos_bias, torch.float32, "pos_bias")
+    T = raw.shape[0]
+    E = T // ratio
+    dev = raw.device
+    if kv_out is None:
+        kv_out = torch.empty((E, ENTRY_BYTES), dtype=torch.uint8, device=dev)
+    if w_idx is not None:
+        _need(w_idx, torch.float32, "w_idx")
+        if ikey_out is None:
+            ikey_out = torch.empty((E, IKEY_BYTES), dtype=torch.uint8, device=dev)
+        if iscale_out is None:
+            iscale_out = torch.empty((E, 2), dtype=torch.float32, device=dev)
+    _check(lib.csld_compress_scaled(_ptr(raw), _ptr(gate), _ptr(pos_bias), ratio, _ptr(w_idx), T, float(kv_scale),
+                                    _ptr(kv_out), _ptr(ikey_out), _ptr(iscale_out), _stream()), "csld_compress_scaled")
+    return (kv_out, ikey_out, iscale_out) if w_idx is not None else kv_out
+
+
 def csa_compress(raw, gate, pos_bias, w_idx, kv_out=None, ikey_out=None, iscale_out=None):
     return compress(raw, gate, pos_bias, 4, w_idx, kv_out, ikey_out, iscale_out)
 
@@ -258,6 +285,24 @@ def kv_cache_prefill_rope(cache: LayerCache, raw, gate, rope_base):
     s = cache.struct()
     _check(lib.kv_cache_prefill_rope(C.byref(s), _ptr(raw), _ptr(gate), raw.shape[1], float(rope_base), _stream()),
            "kv_cache_prefill_rope")
+
+
+def kv_cache_append_scaled(cache: LayerCache, kv_new, gate_new, kv_scale, err=None):
+    """kv_cache_append into scaled FP8 entries (kv_cache_append_scaled)."""
+    _bits(kv_new, "kv_new")
+    _need(gate_new, torch.float32, "gate_new")
+    s = cache.struct()
+    _check(lib.kv_cache_append_scaled(C.byref(s), _ptr(kv_new), _ptr(gate_new), float(kv_scale),
+                                      _ptr(cache.err if err is None else err), _stream()), "kv_cache_append_scaled")
+
+
+def kv_cache_prefill_scaled(cache: LayerCache, raw, gate, kv_scale):
+    """kv_cache_prefill into scaled FP8 entries (kv_cache_prefill_scaled)."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    s = cache.struct()
+    _check(lib.kv_cache_prefill_scaled(C.byref(s), _ptr(raw), _ptr(gate), raw.shape[1], float(kv_scale), _stream()),
+           "kv_cache_prefill_scaled")
 
 
 def kv_cache_prefill(cache: LayerCache, raw, gate):
@@ -326,9 +371,10 @@ def attention_workspace(B, cap, k, W, device="cuda"):
 
 
 def hybrid_decode_attention(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, out=None,
-                            lse=None, ws=None, err=None):
+                            lse=None, ws=None, err=None, kv_scale=None):
     """q [B,16,512] bf16; comp_kv [B,cap,576] u8; topk [B,k] i32 or None (dense); win_kv
-    [B,W,576] u8; seq_len [B] i32 -> (out [B,16,512] f32, lse [B,16] f32)."""
+    [B,W,576] u8; seq_len [B] i32 -> (out [B,16,512] f32, lse [B,16] f32).  kv_scale: scaled
+    FP8 entries (hybrid_decode_attention_scaled); None for the base layout."""
     _bits(q, "q")
     _need(comp_kv, torch.uint8, "comp_kv")
     _need(seq_len, torch.int32, "seq_len")
@@ -352,11 +398,22 @@ def hybrid_decode_attention(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, 
         raise CsldError(f"lse: expected shape {(B, H)}, got {tuple(lse.shape)}")
     if ws is None:
         ws = attention_workspace(B, cap, max(k, 1), W, q.device)
+    if kv_scale is not None:
+        _check(lib.hybrid_decode_attention_scaled(_ptr(q), H, _ptr(comp_kv), cap, ratio, _ptr(topk), k,
+                                                  _ptr(win_kv) if W > 0 else None, W, _ptr(seq_len), B,
+                                                  float(scale), float(kv_scale), _ptr(out), _ptr(lse), _ptr(ws),
+                                                  ws.numel(), _ptr(err), _stream()), "hybrid_decode_attention_scaled")
+        return out, lse
     _check(lib.hybrid_decode_attention(_ptr(q), H, _ptr(comp_kv), cap, ratio, _ptr(topk), k,
                                        _ptr(win_kv) if W > 0 else None, W, _ptr(seq_len), B,
                                        float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                        _ptr(err), _stream()), "hybrid_decode_attention")
     return out, lse
+
+
+def hybrid_decode_attention_scaled(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, kv_scale, **kw):
+    """hybrid_decode_attention over scaled FP8 entries (hybrid_decode_attention_scaled)."""
+    return hybrid_decode_attention(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, kv_scale=kv_scale, **kw)
 
 
 def hybrid_decode_attention_multi(q, comp_kv, ratio, topk, win_kv, W, seq_len, scale, out=None, lse=None, ws=None,

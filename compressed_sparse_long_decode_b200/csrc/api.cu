@@ -115,8 +115,8 @@ const char* csld_status_string(csld_status s) {
 
 namespace {
 csld_status compress_impl(const char* name, const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
-                          const float* w_idx, int64_t T, int64_t pos0, double rope_base, uint8_t* kv_out,
-                          uint8_t* ikey_out, float* iscale_out, void* stream) {
+                          const float* w_idx, int64_t T, int64_t pos0, double rope_base, float kv_scale,
+                          uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, void* stream) {
     if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
     if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
     if (T / ratio == 0) return CSLD_OK;
@@ -125,7 +125,8 @@ csld_status compress_impl(const char* name, const uint16_t* raw, const float* ga
     if (!aligned16(raw) || !aligned16(kv_out) || (ikey_out && !aligned16(ikey_out)))
         return fail(CSLD_ERR_ALIGN, "raw, kv_out and ikey_out must be 16-byte aligned");
     cudaError_t e = csld::launch_compress(raw, gate, pos_bias, ratio, w_idx, T, 1, T / ratio, kv_out,
-                                          ikey_out, iscale_out, num_sms(), as_stream(stream), pos0, rope_base);
+                                          ikey_out, iscale_out, num_sms(), as_stream(stream), pos0, rope_base,
+                                          kv_scale);
     if (e != cudaSuccess) return cuda_fail(e, name);
     return CSLD_OK;
 }
@@ -134,8 +135,8 @@ csld_status compress_impl(const char* name, const uint16_t* raw, const float* ga
 csld_status csld_compress(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
                           const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
                           float* iscale_out, void* stream) {
-    return compress_impl("csld_compress", raw, gate, pos_bias, ratio, w_idx, T, 0, 0.0, kv_out, ikey_out, iscale_out,
-                         stream);
+    return compress_impl("csld_compress", raw, gate, pos_bias, ratio, w_idx, T, 0, 0.0, 1.f, kv_out, ikey_out,
+                         iscale_out, stream);
 }
 
 csld_status csld_compress_rope(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
@@ -143,7 +144,19 @@ csld_status csld_compress_rope(const uint16_t* raw, const float* gate, const flo
                                uint8_t* ikey_out, float* iscale_out, void* stream) {
     if (!(rope_base > 1.0) || rope_base == INFINITY) return fail(CSLD_ERR_ARG, "rope_base must be finite and > 1");
     if (pos0 < 0 || pos0 > ((int64_t)1 << 40)) return fail(CSLD_ERR_ARG, "pos0 %lld outside 0..2^40", (long long)pos0);
-    return compress_impl("csld_compress_rope", raw, gate, pos_bias, ratio, w_idx, T, pos0, rope_base, kv_out,
+    return compress_impl("csld_compress_rope", raw, gate, pos_bias, ratio, w_idx, T, pos0, rope_base, 1.f, kv_out,
+                         ikey_out, iscale_out, stream);
+}
+
+namespace {
+bool kv_scale_ok(float kv_scale) { return kv_scale >= 0x1p-60f && kv_scale <= 0x1p60f; }
+}  // namespace
+
+csld_status csld_compress_scaled(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
+                                 const float* w_idx, int64_t T, float kv_scale, uint8_t* kv_out, uint8_t* ikey_out,
+                                 float* iscale_out, void* stream) {
+    if (!kv_scale_ok(kv_scale)) return fail(CSLD_ERR_ARG, "kv_scale %g outside 2^-60..2^60", (double)kv_scale);
+    return compress_impl("csld_compress_scaled", raw, gate, pos_bias, ratio, w_idx, T, 0, 0.0, kv_scale, kv_out,
                          ikey_out, iscale_out, stream);
 }
 
@@ -161,12 +174,12 @@ csld_status hca_compress(const uint16_t* raw, const float* gate, const float* po
 
 namespace {
 csld_status append_impl(const char* name, const csld_layer_cache* cache, const uint16_t* kv_new,
-                        const float* gate_new, int32_t* err, double rope_base, void* stream) {
+                        const float* gate_new, int32_t* err, double rope_base, float kv_scale, void* stream) {
     csld_status s = check_cache(cache);
     if (s != CSLD_OK) return s;
     if (!kv_new || !gate_new) return fail(CSLD_ERR_ARG, "kv_new / gate_new is NULL");
     if (!aligned16(kv_new)) return fail(CSLD_ERR_ALIGN, "kv_new must be 16-byte aligned");
-    cudaError_t e = csld::launch_append(*cache, kv_new, gate_new, err, as_stream(stream), rope_base);
+    cudaError_t e = csld::launch_append(*cache, kv_new, gate_new, err, as_stream(stream), rope_base, kv_scale);
     if (e != cudaSuccess) return cuda_fail(e, name);
     return CSLD_OK;
 }
@@ -174,18 +187,24 @@ csld_status append_impl(const char* name, const csld_layer_cache* cache, const u
 
 csld_status kv_cache_append(const csld_layer_cache* cache, const uint16_t* kv_new,
                             const float* gate_new, int32_t* err, void* stream) {
-    return append_impl("kv_cache_append", cache, kv_new, gate_new, err, 0.0, stream);
+    return append_impl("kv_cache_append", cache, kv_new, gate_new, err, 0.0, 1.f, stream);
 }
 
 csld_status kv_cache_append_rope(const csld_layer_cache* cache, const uint16_t* kv_new,
                                  const float* gate_new, double rope_base, int32_t* err, void* stream) {
     if (!(rope_base > 1.0) || rope_base == INFINITY) return fail(CSLD_ERR_ARG, "rope_base must be finite and > 1");
-    return append_impl("kv_cache_append_rope", cache, kv_new, gate_new, err, rope_base, stream);
+    return append_impl("kv_cache_append_rope", cache, kv_new, gate_new, err, rope_base, 1.f, stream);
+}
+
+csld_status kv_cache_append_scaled(const csld_layer_cache* cache, const uint16_t* kv_new,
+                                   const float* gate_new, float kv_scale, int32_t* err, void* stream) {
+    if (!kv_scale_ok(kv_scale)) return fail(CSLD_ERR_ARG, "kv_scale %g outside 2^-60..2^60", (double)kv_scale);
+    return append_impl("kv_cache_append_scaled", cache, kv_new, gate_new, err, 0.0, kv_scale, stream);
 }
 
 namespace {
 csld_status prefill_impl(const csld_layer_cache* cache, const uint16_t* raw, const float* gate, int64_t T,
-                         double rope_base, void* stream) {
+                         double rope_base, float kv_scale, void* stream) {
     csld_status s = check_cache(cache);
     if (s != CSLD_OK) return s;
     if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
@@ -198,10 +217,11 @@ csld_status prefill_impl(const csld_layer_cache* cache, const uint16_t* raw, con
     cudaError_t e = csld::launch_compress(raw, gate, cache->pos_bias, cache->ratio,
                                           cache->has_indexer ? cache->w_idx : nullptr, T, cache->batch,
                                           cache->capacity, cache->comp_kv, cache->ikeys,
-                                          cache->iscales, num_sms(), st, 0, rope_base);
+                                          cache->iscales, num_sms(), st, 0, rope_base, kv_scale);
     if (e != cudaSuccess) return cuda_fail(e, "kv_cache_prefill (compress)");
     e = csld::launch_prefill_state(raw, gate, T, cache->ratio, cache->window, cache->batch,
-                                   cache->win_kv, cache->tail_kv, cache->tail_gate, cache->seq_len, st, rope_base);
+                                   cache->win_kv, cache->tail_kv, cache->tail_gate, cache->seq_len, st, rope_base,
+                                   kv_scale);
     if (e != cudaSuccess) return cuda_fail(e, "kv_cache_prefill (state)");
     return CSLD_OK;
 }
@@ -209,13 +229,19 @@ csld_status prefill_impl(const csld_layer_cache* cache, const uint16_t* raw, con
 
 csld_status kv_cache_prefill(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
                              int64_t T, void* stream) {
-    return prefill_impl(cache, raw, gate, T, 0.0, stream);
+    return prefill_impl(cache, raw, gate, T, 0.0, 1.f, stream);
 }
 
 csld_status kv_cache_prefill_rope(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
                                   int64_t T, double rope_base, void* stream) {
     if (!(rope_base > 1.0) || rope_base == INFINITY) return fail(CSLD_ERR_ARG, "rope_base must be finite and > 1");
-    return prefill_impl(cache, raw, gate, T, rope_base, stream);
+    return prefill_impl(cache, raw, gate, T, rope_base, 1.f, stream);
+}
+
+csld_status kv_cache_prefill_scaled(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
+                                    int64_t T, float kv_scale, void* stream) {
+    if (!kv_scale_ok(kv_scale)) return fail(CSLD_ERR_ARG, "kv_scale %g outside 2^-60..2^60", (double)kv_scale);
+    return prefill_impl(cache, raw, gate, T, 0.0, kv_scale, stream);
 }
 
 size_t csld_indexer_workspace_size(int B, int64_t cap, int k) {
@@ -253,10 +279,11 @@ size_t csld_attention_workspace_size(int B, int heads, int64_t cap, int k, int W
     return pd.ws_bytes > ps.ws_bytes ? pd.ws_bytes : ps.ws_bytes;
 }
 
-csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t* comp_kv, int64_t cap,
-                                    int ratio, const int32_t* topk, int k, const uint8_t* win_kv, int W,
-                                    const int32_t* seq_len, int B, float scale, float* out, float* lse_out,
-                                    void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+namespace {
+csld_status attention_impl(const char* name, const uint16_t* q, int heads, const uint8_t* comp_kv, int64_t cap,
+                           int ratio, const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                           const int32_t* seq_len, int B, float scale, float kv_scale, float* out, float* lse_out,
+                           void* ws, size_t ws_bytes, int32_t* err, void* stream) {
     if (heads != CSLD_HEADS) return fail(CSLD_ERR_UNSUPPORTED, "heads = %d; the library implements %d", heads, CSLD_HEADS);
     if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
     if (cap < 1 || cap > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "cap %lld outside 1..2^31-1", (long long)cap);
@@ -273,9 +300,27 @@ csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t*
         return fail(CSLD_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, plan.ws_bytes);
     if (!aligned16(ws)) return fail(CSLD_ERR_ALIGN, "workspace must be 16-byte aligned");
     cudaError_t e = csld::launch_attention(q, comp_kv, cap, ratio, topk, topk ? k : 0, win_kv, W, W, 1, seq_len, B,
-                                           scale, out, lse_out, ws, plan, err, as_stream(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "hybrid_decode_attention");
+                                           scale, out, lse_out, ws, plan, err, as_stream(stream), kv_scale);
+    if (e != cudaSuccess) return cuda_fail(e, name);
     return CSLD_OK;
+}
+}  // namespace
+
+csld_status hybrid_decode_attention(const uint16_t* q, int heads, const uint8_t* comp_kv, int64_t cap,
+                                    int ratio, const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                                    const int32_t* seq_len, int B, float scale, float* out, float* lse_out,
+                                    void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+    return attention_impl("hybrid_decode_attention", q, heads, comp_kv, cap, ratio, topk, k, win_kv, W, seq_len, B,
+                          scale, 1.f, out, lse_out, ws, ws_bytes, err, stream);
+}
+
+csld_status hybrid_decode_attention_scaled(const uint16_t* q, int heads, const uint8_t* comp_kv, int64_t cap,
+                                           int ratio, const int32_t* topk, int k, const uint8_t* win_kv, int W,
+                                           const int32_t* seq_len, int B, float scale, float kv_scale, float* out,
+                                           float* lse_out, void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+    if (!kv_scale_ok(kv_scale)) return fail(CSLD_ERR_ARG, "kv_scale %g outside 2^-60..2^60", (double)kv_scale);
+    return attention_impl("hybrid_decode_attention_scaled", q, heads, comp_kv, cap, ratio, topk, k, win_kv, W,
+                          seq_len, B, scale, kv_scale, out, lse_out, ws, ws_bytes, err, stream);
 }
 
 csld_status csld_stage(void* dst, const void* src, size_t bytes, void* stream) {

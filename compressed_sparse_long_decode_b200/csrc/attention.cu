@@ -25,14 +25,15 @@ namespace csld {
 // largest m).  512 threads: thread t owns dims 4 (t % 128) .. +3 and adds every fourth split
 // starting at t / 128; the four partial sums are then added in a fixed order.  Every thread
 // issues its O loads before warp 0 forms the split weights, so the merge costs about one round
-// trip to L2.
+// trip to L2.  kv_scale (scaled FP8 entries; 1 for the base layout): the partials' FP8 dims
+// (0..447) are in units of the entries' codes and are multiplied by it here.
 constexpr int kMergeThreads = 512;
 constexpr int kMergeGroups = kMergeThreads / (kDim / 4);   // 4
 constexpr int kMergeU = 8;                                 // O loads a thread keeps in flight
 __global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const float* __restrict__ opart,
                                                                         const float2* __restrict__ mlpart,
                                                                         int splits, float* __restrict__ out,
-                                                                        float* __restrict__ lse_out) {
+                                                                        float* __restrict__ lse_out, float kv_scale) {
     __shared__ float fw[256];
     __shared__ float4 red[kMergeGroups - 1][kDim / 4];
     __shared__ float mlw[2];
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const fl
         }
         const float M = mlw[0], Lsum = mlw[1];
         if (Lsum > 0.f) {
-            const float inv = 1.f / Lsum;
+            const float inv = (4 * d4 < kNope) ? (1.f / Lsum) * kv_scale : 1.f / Lsum;
             acc.x *= inv;
             acc.y *= inv;
             acc.z *= inv;
@@ -133,15 +134,16 @@ cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t 
                              const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                              const int32_t* seq_len, int B, float scale, float* out,
                              float* lse_out, void* ws, const AttentionPlan& plan, int32_t* err,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, float kv_scale) {
     // B cache rows, Q query rows each: the plan and the partials count B * Q query rows
     float* opart = static_cast<float*>(ws);
     float2* mlpart = reinterpret_cast<float2*>(opart + (size_t)B * Q * plan.splits * kHeads * kDim);
     cudaError_t e = launch_attention_tc_partial(q, comp_kv, cap, ratio, topk, k, win_kv, W, Wr, Q, seq_len, B, scale,
-                                                plan.splits, opart, mlpart, err, stream);
+                                                plan.splits, opart, mlpart, err, stream, kv_scale);
     if (e != cudaSuccess) return e;
     e = launch_pdl(attention_merge_kernel, dim3(B * Q, kHeads), dim3(kMergeThreads), 0, stream,
-                   static_cast<const float*>(opart), static_cast<const float2*>(mlpart), plan.splits, out, lse_out);
+                   static_cast<const float*>(opart), static_cast<const float2*>(mlpart), plan.splits, out, lse_out,
+                   kv_scale);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

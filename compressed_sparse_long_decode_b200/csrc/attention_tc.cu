@@ -156,7 +156,10 @@ __device__ __forceinline__ void qprep_load(uint4 (&v)[4], const uint16_t* q, int
 // so it stays below 256 (E4M3 max 448); the 16 threads of a head find max|q_h| by shuffles.
 // Nope dims -> E4M3 hi and lo terms (rows h and 16 + h of the swizzled QK operand), RoPE dims
 // -> bf16; each thread writes whole 16-byte chunks.
-__device__ __forceinline__ void qprep_store(TcAttnSmem& sm, const uint4 (&v)[4], int t, float scale) {
+// kv_scale: the entries' FP8 dims stand for kv_scale times their code value (scaled FP8 entries;
+// 1 for the base layout), so the query's FP8 part is multiplied by it before it is split (the
+// output's FP8 dims are multiplied by it in the merge).
+__device__ __forceinline__ void qprep_store(TcAttnSmem& sm, const uint4 (&v)[4], int t, float scale, float kv_scale) {
     const int h = t >> 4, part = t & 15, d0 = 32 * part;
     uint32_t w[16];
 #pragma unroll
@@ -170,6 +173,7 @@ __device__ __forceinline__ void qprep_store(TcAttnSmem& sm, const uint4 (&v)[4],
 #pragma unroll
     for (int c = 0; c < 16; ++c)
         amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(w[c] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[c] >> 16))));
+    if (d0 < kNope) amax *= kv_scale;
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const int sh = amax > 0.f ? max(-100, min(100, 7 - ilogbf(amax))) : 0;
@@ -179,6 +183,7 @@ __device__ __forceinline__ void qprep_store(TcAttnSmem& sm, const uint4 (&v)[4],
         sm.c2[h] = scale * 1.4426950408889634f / sq;
     }
     if (d0 < kNope) {
+        const float sqn = sq * kv_scale;
         uint32_t hw[8], lw[8];   // bytes of dims d0 + 4c .. +3
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -186,7 +191,7 @@ __device__ __forceinline__ void qprep_store(TcAttnSmem& sm, const uint4 (&v)[4],
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const uint32_t x = w[2 * c + u];
-                const float x0 = bf16_bits_to_f32(x & 0xFFFFu) * sq, x1 = bf16_bits_to_f32(x >> 16) * sq;
+                const float x0 = bf16_bits_to_f32(x & 0xFFFFu) * sqn, x1 = bf16_bits_to_f32(x >> 16) * sqn;
                 hi2[u] = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
                 const uint32_t back = e4m3x2_to_f16x2(hi2[u]);   // exact
                 const float r0 = x0 - __half2float(__ushort_as_half(static_cast<unsigned short>(back & 0xFFFFu)));
@@ -268,7 +273,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
     const uint8_t* __restrict__ comp_kv, const uint8_t* __restrict__ win_kv,
     const uint16_t* __restrict__ q, int64_t cap, int ratio,
     const int32_t* __restrict__ topk, int k, int W, int Wr, int Q, const int32_t* __restrict__ seq_len, float scale,
-    int splits, float* __restrict__ opart, float2* __restrict__ mlpart, int32_t* err) {
+    int splits, float* __restrict__ opart, float2* __restrict__ mlpart, int32_t* err, float kv_scale) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     TcAttnSmem& sm = *reinterpret_cast<TcAttnSmem*>(smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -501,7 +506,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_partial_kernel(
             tmem_st_32x32b_x8_fill(lb + kColSFA, 0x7F7F7F7Fu);
             tmem_st_wait();
         }
-        qprep_store(sm, qv, tid - 256, scale);
+        qprep_store(sm, qv, tid - 256, scale, kv_scale);
         tc_fence_before();
         named_barrier(kReadyBar, 384);
         tc_fence_after();
@@ -725,7 +730,7 @@ int attention_tc_tile() { return kTcTile; }
 cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
                                         const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                                         const int32_t* seq_len, int B, float scale, int splits, float* opart,
-                                        float2* mlpart, int32_t* err, cudaStream_t stream) {
+                                        float2* mlpart, int32_t* err, cudaStream_t stream, float kv_scale) {
     // the caches as 2-D byte tensors [rows][576] for the box copies of whole tiles: 128-byte
     // boxes with the 128-byte swizzle, kTcTile rows tall.  B cache rows, each serving Q query
     // rows; the window ring has Wr >= W slots per cache row.  Gathered tiles read the caches
@@ -752,7 +757,7 @@ cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_k
     if (e != cudaSuccess) return e;
     e = launch_pdl(kernel, dim3(splits, B * Q), dim3(kTcThreads), smem, stream, kv_tile, win_tile,
                    comp_kv, has_win ? win_kv : nullptr, q, cap, ratio, topk, k, W, Wr, Q, seq_len,
-                   scale, splits, opart, mlpart, err);
+                   scale, splits, opart, mlpart, err, kv_scale);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -12,10 +12,12 @@
 // memory for the whole persistent CTA) on the 5th-generation tensor cores (tcgen05.mma
 // kind::f16, fp32 accumulation in tensor memory); the FP4 quantisation runs on the fp32 result.
 //
-// RoPE at compressed positions (a layout variant of the storage paragraph's bf16 RoPE dims):
-// the kernels below are also compiled with kRope, where the raw tokens' dims 448..511 are taken
-// before rotary encoding and rotated here -- a pooled entry at its block's last token, a window
-// entry at its own token (RoFormer pairs, see rope_lane).
+// Layout variants of the storage paragraph, compiled into the same kernels (kVar):
+//  - kVarRope, RoPE at compressed positions: the raw tokens' dims 448..511 are taken before
+//    rotary encoding and rotated here -- a pooled entry at its block's last token, a window
+//    entry at its own token (RoFormer pairs, see rope_lane);
+//  - kVarScaled, scaled FP8 entries: one scale sigma per layer cache, the FP8 dims stored as
+//    E4M3(x / sigma) (the kernels get 1 / sigma), the RoPE dims and the indexer key unscaled.
 #include "csld_internal.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -153,15 +155,34 @@ __device__ __forceinline__ uint2 rope_bf16x4(uint2 x, int j, int64_t pos, double
     return make_uint2(w[0], w[1]);
 }
 
-// Writes the 576-byte entry of the pooled vector held by the warp (lane l: dims 16l..16l+15).
+constexpr int kVarBase = 0, kVarRope = 1, kVarScaled = 2;
+
+// E4M3 codes of four consecutive FP8 dims of a raw token held as bf16 (a window entry's FP8
+// part); kScaled: times inv_scale first.
+template <bool kScaled>
+__device__ __forceinline__ uint32_t fp8x4_of_bf16x4(uint2 x, float inv_scale) {
+    float v[4] = {bf16_bits_to_f32(x.x), bf16_bits_to_f32(x.x >> 16), bf16_bits_to_f32(x.y), bf16_bits_to_f32(x.y >> 16)};
+    if constexpr (kScaled) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] *= inv_scale;
+    }
+    return f32_to_e4m3(v[0]) | (f32_to_e4m3(v[1]) << 8) | (f32_to_e4m3(v[2]) << 16) | (f32_to_e4m3(v[3]) << 24);
+}
+
+// Writes the 576-byte entry of the pooled vector held by the warp (lane l: dims 16l..16l+15);
+// kScaled: the FP8 dims times inv_scale (= 1 / sigma) before rounding.
+template <bool kScaled = false>
 __device__ __forceinline__ void warp_store_entry(uint8_t* __restrict__ entry, int lane,
-                                                 const float (&c)[16]) {
+                                                 const float (&c)[16], float inv_scale = 1.f) {
     if (lane < kNope / 16) {
+        float v[16];
+#pragma unroll
+        for (int d = 0; d < 16; ++d) v[d] = kScaled ? c[d] * inv_scale : c[d];
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            w[q] = f32_to_e4m3(c[4 * q]) | (f32_to_e4m3(c[4 * q + 1]) << 8) |
-                   (f32_to_e4m3(c[4 * q + 2]) << 16) | (f32_to_e4m3(c[4 * q + 3]) << 24);
+            w[q] = f32_to_e4m3(v[4 * q]) | (f32_to_e4m3(v[4 * q + 1]) << 8) |
+                   (f32_to_e4m3(v[4 * q + 2]) << 16) | (f32_to_e4m3(v[4 * q + 3]) << 24);
         *reinterpret_cast<uint4*>(entry + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
     } else {
         uint32_t w[8];
@@ -191,13 +212,14 @@ __device__ __forceinline__ void warp_store_fp4(uint8_t* __restrict__ codes, floa
 // ------------------------------------------------------------------------------------------
 // Pooling without an indexer key (HCA, or any ratio).  One warp per entry.
 // ------------------------------------------------------------------------------------------
-template <bool kRope>
+template <int kVar>
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ raw,
                                                    const float* __restrict__ gate,
                                                    const float* __restrict__ bias, int m,
                                                    int64_t T, int64_t E, int B,
                                                    int64_t out_seq_stride,
-                                                   uint8_t* __restrict__ kv_out, int64_t pos0, double rope_base) {
+                                                   uint8_t* __restrict__ kv_out, int64_t pos0, double rope_base,
+                                                   float inv_scale) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (gw >= E * B) return;
@@ -205,8 +227,8 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
     float c[16];
     warp_pool<true>(raw + ((size_t)b * T + (size_t)s * m) * kDim, gate + (size_t)b * T + (size_t)s * m,
               bias, m, lane, c);
-    if constexpr (kRope) rope_lane(c, lane, pos0 + (s + 1) * m - 1, rope_base);
-    warp_store_entry(kv_out + ((size_t)b * out_seq_stride + (size_t)s) * kEntry, lane, c);
+    if constexpr (kVar == kVarRope) rope_lane(c, lane, pos0 + (s + 1) * m - 1, rope_base);
+    warp_store_entry<kVar == kVarScaled>(kv_out + ((size_t)b * out_seq_stride + (size_t)s) * kEntry, lane, c, inv_scale);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -266,12 +288,12 @@ __device__ __forceinline__ void pool4_preloaded(const uint4 (&x)[8], const float
 }
 
 // kM4: the block ratio is 4 (two blocks' raw rows are loaded at once); otherwise any ratio.
-template <bool kM4, bool kRope>
+template <bool kM4, int kVar>
 __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
     const uint16_t* __restrict__ raw, const float* __restrict__ gate, const float* __restrict__ bias,
     int m, const float* __restrict__ w_idx, int64_t T, int64_t E, int B, int64_t out_seq_stride,
     uint8_t* __restrict__ kv_out, uint8_t* __restrict__ ikey_out, float* __restrict__ iscale_out, int64_t pos0,
-    double rope_base) {
+    double rope_base, float inv_scale) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     CompressSmem& sm = *reinterpret_cast<CompressSmem*>(smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -346,8 +368,8 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                         float w[4];
                         warp_pool_weights_pre(ga[h] + bias_l, 4, lane, w);
                         pool4_preloaded(x[h], w, c);
-                        if constexpr (kRope) rope_lane(c, lane, pos0 + (s0 + r + 1) * 4 - 1, rope_base);
-                        warp_store_entry(kvb + (size_t)(s0 + r) * kEntry, lane, c);
+                        if constexpr (kVar == kVarRope) rope_lane(c, lane, pos0 + (s0 + r + 1) * 4 - 1, rope_base);
+                        warp_store_entry<kVar == kVarScaled>(kvb + (size_t)(s0 + r) * kEntry, lane, c, inv_scale);
                     } else {
 #pragma unroll
                         for (int d = 0; d < 16; ++d) c[d] = 0.f;
@@ -363,8 +385,8 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                     float c[16];
                     if (r < n_here) {
                         warp_pool<true>(rb + (size_t)(s0 + r) * m * kDim, gb + (s0 + r) * m, bias, m, lane, c);
-                        if constexpr (kRope) rope_lane(c, lane, pos0 + (s0 + r + 1) * m - 1, rope_base);
-                        warp_store_entry(kvb + (size_t)(s0 + r) * kEntry, lane, c);
+                        if constexpr (kVar == kVarRope) rope_lane(c, lane, pos0 + (s0 + r + 1) * m - 1, rope_base);
+                        warp_store_entry<kVar == kVarScaled>(kvb + (size_t)(s0 + r) * kEntry, lane, c, inv_scale);
                     } else {
 #pragma unroll
                         for (int d = 0; d < 16; ++d) c[d] = 0.f;
@@ -468,27 +490,33 @@ size_t compress_index_smem_bytes() { return sizeof(CompressSmem) + 1024; }
 cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float* bias, int m,
                             const float* w_idx, int64_t T, int B, int64_t out_seq_stride,
                             uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, int num_sms,
-                            cudaStream_t stream, int64_t pos0, double rope_base) {
+                            cudaStream_t stream, int64_t pos0, double rope_base, float kv_scale) {
     const int64_t E = T / m;
     if (E <= 0 || B <= 0) return cudaSuccess;
-    const bool rope = rope_base > 0.0;
+    const int var = rope_base > 0.0 ? kVarRope : (kv_scale != 1.f ? kVarScaled : kVarBase);
+    const float inv_scale = 1.f / kv_scale;
     if (w_idx == nullptr) {
         const int64_t warps = E * B;
         const int64_t blocks = (warps + 7) / 8;
-        auto kernel = rope ? pool_kernel<true> : pool_kernel<false>;
+        auto kernel = var == kVarRope ? pool_kernel<kVarRope> : (var == kVarScaled ? pool_kernel<kVarScaled> : pool_kernel<kVarBase>);
         kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(raw, gate, bias, m, T, E, B, out_seq_stride, kv_out,
-                                                                  pos0, rope_base);
+                                                                  pos0, rope_base, inv_scale);
         return cudaGetLastError();
     }
     const size_t smem = compress_index_smem_bytes();
     const int64_t tiles = ((E + kCTile - 1) / kCTile) * B;
     const int64_t grid = min64(tiles, num_sms);
-    auto kernel = (m == 4) ? (rope ? pool_index_kernel<true, true> : pool_index_kernel<true, false>)
-                           : (rope ? pool_index_kernel<false, true> : pool_index_kernel<false, false>);
+    auto kernel = (m == 4) ? (var == kVarRope ? pool_index_kernel<true, kVarRope>
+                                              : (var == kVarScaled ? pool_index_kernel<true, kVarScaled>
+                                                                   : pool_index_kernel<true, kVarBase>))
+                           : (var == kVarRope ? pool_index_kernel<false, kVarRope>
+                                              : (var == kVarScaled ? pool_index_kernel<false, kVarScaled>
+                                                                   : pool_index_kernel<false, kVarBase>));
     cudaError_t e = set_smem_once(kernel, smem);
     if (e != cudaSuccess) return e;
     kernel<<<static_cast<unsigned>(grid), kCThreads, smem, stream>>>(raw, gate, bias, m, w_idx, T, E, B, out_seq_stride,
-                                                                     kv_out, ikey_out, iscale_out, pos0, rope_base);
+                                                                     kv_out, ikey_out, iscale_out, pos0, rope_base,
+                                                                     inv_scale);
     return cudaGetLastError();
 }
 
@@ -615,14 +643,15 @@ cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, cons
 // ------------------------------------------------------------------------------------------
 // Window ring + tail after a prefill of T tokens (one CTA per sequence).
 // ------------------------------------------------------------------------------------------
-template <bool kRope>
+template <int kVar>
 __global__ void __launch_bounds__(128) prefill_state_kernel(const uint16_t* __restrict__ raw,
                                                             const float* __restrict__ gate,
                                                             int64_t T, int m, int W,
                                                             uint8_t* __restrict__ win_kv,
                                                             uint16_t* __restrict__ tail_kv,
                                                             float* __restrict__ tail_gate,
-                                                            int32_t* __restrict__ seq_len, double rope_base) {
+                                                            int32_t* __restrict__ seq_len, double rope_base,
+                                                            float inv_scale) {
     const int b = blockIdx.x, tid = threadIdx.x;
     const uint16_t* rb = raw + (size_t)b * T * kDim;
     // window: tokens max(0, T-W) .. T-1; thread handles 4 dims (8 bytes of bf16)
@@ -631,13 +660,10 @@ __global__ void __launch_bounds__(128) prefill_state_kernel(const uint16_t* __re
         const uint2 x = *reinterpret_cast<const uint2*>(rb + (size_t)t * kDim + 4 * tid);
         uint8_t* e = win_kv + ((size_t)b * W + (size_t)(t % W)) * kEntry;
         if (tid < kNope / 4) {
-            const uint32_t v = f32_to_e4m3(bf16_bits_to_f32(x.x)) | (f32_to_e4m3(bf16_bits_to_f32(x.x >> 16)) << 8) |
-                               (f32_to_e4m3(bf16_bits_to_f32(x.y)) << 16) |
-                               (f32_to_e4m3(bf16_bits_to_f32(x.y >> 16)) << 24);
-            *reinterpret_cast<uint32_t*>(e + 4 * tid) = v;
+            *reinterpret_cast<uint32_t*>(e + 4 * tid) = fp8x4_of_bf16x4<kVar == kVarScaled>(x, inv_scale);
         } else {
             uint2 y = x;
-            if constexpr (kRope) y = rope_bf16x4(x, tid - kNope / 4, t, rope_base);   // at token t
+            if constexpr (kVar == kVarRope) y = rope_bf16x4(x, tid - kNope / 4, t, rope_base);   // at token t
             *reinterpret_cast<uint2*>(e + kNope + 8 * (tid - kNope / 4)) = y;
         }
     }
@@ -652,9 +678,10 @@ __global__ void __launch_bounds__(128) prefill_state_kernel(const uint16_t* __re
 
 cudaError_t launch_prefill_state(const uint16_t* raw, const float* gate, int64_t T, int m, int W,
                                  int B, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
-                                 int32_t* seq_len, cudaStream_t stream, double rope_base) {
-    auto kernel = rope_base > 0.0 ? prefill_state_kernel<true> : prefill_state_kernel<false>;
-    kernel<<<B, 128, 0, stream>>>(raw, gate, T, m, W, win_kv, tail_kv, tail_gate, seq_len, rope_base);
+                                 int32_t* seq_len, cudaStream_t stream, double rope_base, float kv_scale) {
+    auto kernel = rope_base > 0.0 ? prefill_state_kernel<kVarRope>
+                                  : (kv_scale != 1.f ? prefill_state_kernel<kVarScaled> : prefill_state_kernel<kVarBase>);
+    kernel<<<B, 128, 0, stream>>>(raw, gate, T, m, W, win_kv, tail_kv, tail_gate, seq_len, rope_base, 1.f / kv_scale);
     return cudaGetLastError();
 }
 
@@ -670,11 +697,11 @@ namespace csld {
 // ------------------------------------------------------------------------------------------
 constexpr int kAppendThreads = 256;
 
-template <bool kRope>
+template <int kVar>
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache cache,
                                                                 const uint16_t* __restrict__ kv_new,
                                                                 const float* __restrict__ gate_new,
-                                                                int32_t* err, double rope_base) {
+                                                                int32_t* err, double rope_base, float inv_scale) {
     __shared__ float cbuf[kDim];
     __shared__ float upart[kAppendThreads / 32][kIdxDim];
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -699,14 +726,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
     if (W > 0 && mover) {
         uint8_t* e = cache.win_kv + ((size_t)b * W + (size_t)(t % W)) * kEntry;
         if (tid < kNope / 4) {
-            const uint32_t v = f32_to_e4m3(bf16_bits_to_f32(x.x)) |
-                               (f32_to_e4m3(bf16_bits_to_f32(x.x >> 16)) << 8) |
-                               (f32_to_e4m3(bf16_bits_to_f32(x.y)) << 16) |
-                               (f32_to_e4m3(bf16_bits_to_f32(x.y >> 16)) << 24);
-            *reinterpret_cast<uint32_t*>(e + 4 * tid) = v;
+            *reinterpret_cast<uint32_t*>(e + 4 * tid) = fp8x4_of_bf16x4<kVar == kVarScaled>(x, inv_scale);
         } else {
             uint2 y = x;
-            if constexpr (kRope) y = rope_bf16x4(x, tid - kNope / 4, t, rope_base);   // at token t
+            if constexpr (kVar == kVarRope) y = rope_bf16x4(x, tid - kNope / 4, t, rope_base);   // at token t
             *reinterpret_cast<uint2*>(e + kNope + 8 * (tid - kNope / 4)) = y;
         }
     }
@@ -719,8 +742,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
         if (warp == 0) {
             float c[16];
             warp_pool<false>(tail, tgate, cache.pos_bias, m, lane, c);
-            if constexpr (kRope) rope_lane(c, lane, t, rope_base);   // token t ends the block
-            warp_store_entry(cache.comp_kv + ((size_t)b * cap + (size_t)s) * kEntry, lane, c);
+            if constexpr (kVar == kVarRope) rope_lane(c, lane, t, rope_base);   // token t ends the block
+            warp_store_entry<kVar == kVarScaled>(cache.comp_kv + ((size_t)b * cap + (size_t)s) * kEntry, lane, c,
+                                                 inv_scale);
 #pragma unroll
             for (int d = 0; d < 16; ++d) cbuf[16 * lane + d] = bf16_bits_to_f32(f32_to_bf16_bits(c[d]));
         }
@@ -756,12 +780,12 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
 }
 
 cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
-                          const float* gate_new, int32_t* err, cudaStream_t stream, double rope_base) {
-    cudaError_t e = rope_base > 0.0
-                        ? launch_pdl(append_kernel<true>, dim3(cache.batch), dim3(kAppendThreads), 0, stream, cache,
-                                     kv_new, gate_new, err, rope_base)
-                        : launch_pdl(append_kernel<false>, dim3(cache.batch), dim3(kAppendThreads), 0, stream, cache,
-                                     kv_new, gate_new, err, rope_base);
+                          const float* gate_new, int32_t* err, cudaStream_t stream, double rope_base,
+                          float kv_scale) {
+    auto kernel = rope_base > 0.0 ? append_kernel<kVarRope>
+                                  : (kv_scale != 1.f ? append_kernel<kVarScaled> : append_kernel<kVarBase>);
+    cudaError_t e = launch_pdl(kernel, dim3(cache.batch), dim3(kAppendThreads), 0, stream, cache, kv_new, gate_new, err,
+                               rope_base, 1.f / kv_scale);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -9,12 +9,13 @@
 
 namespace csld {
 
-// rope_base > 0: RoPE at compressed positions, raw token 0 at position pos0 (entry s rotated at
-// pos0 + (s+1) m - 1); 0: the entries' RoPE dims are pooled as given.
+// Layout variants (at most one at a time): rope_base > 0, RoPE at compressed positions with raw
+// token 0 at position pos0 (entry s rotated at pos0 + (s+1) m - 1); kv_scale != 1, scaled FP8
+// entries (E4M3(x / kv_scale)).  rope_base = 0 and kv_scale = 1: the base layout.
 cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float* bias, int m,
                             const float* w_idx, int64_t T, int B, int64_t out_seq_stride,
                             uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, int num_sms,
-                            cudaStream_t stream, int64_t pos0 = 0, double rope_base = 0.0);
+                            cudaStream_t stream, int64_t pos0 = 0, double rope_base = 0.0, float kv_scale = 1.f);
 size_t compress_index_smem_bytes();
 cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, const float* bias, int m,
                                     const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
@@ -22,10 +23,12 @@ cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, cons
 
 cudaError_t launch_prefill_state(const uint16_t* raw, const float* gate, int64_t T, int m, int W,
                                  int B, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
-                                 int32_t* seq_len, cudaStream_t stream, double rope_base = 0.0);
+                                 int32_t* seq_len, cudaStream_t stream, double rope_base = 0.0,
+                                 float kv_scale = 1.f);
 
 cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
-                          const float* gate_new, int32_t* err, cudaStream_t stream, double rope_base = 0.0);
+                          const float* gate_new, int32_t* err, cudaStream_t stream, double rope_base = 0.0,
+                          float kv_scale = 1.f);
 
 // Lightning indexer + top-k.
 struct IndexerPlan {
@@ -54,11 +57,12 @@ struct AttentionPlan {
 AttentionPlan attention_plan(int B, int64_t cap, int k, bool sparse, int W, int num_sms);
 // B cache rows with Q query rows each (query j of row b sees the first seq_len[b] - Q + 1 + j
 // tokens); the window ring has Wr >= W slots per cache row.  The plan counts B * Q rows.
+// kv_scale: the entries' FP8 dims stand for kv_scale times their code value (1: base layout).
 cudaError_t launch_attention(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
                              const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                              const int32_t* seq_len, int B, float scale, float* out,
                              float* lse_out, void* ws, const AttentionPlan& plan, int32_t* err,
-                             cudaStream_t stream);
+                             cudaStream_t stream, float kv_scale = 1.f);
 
 // Device address of the library-owned attention scratch on the current device (looked up on
 // the first call per device).
@@ -69,6 +73,6 @@ size_t attention_tc_smem_bytes();
 cudaError_t launch_attention_tc_partial(const uint16_t* q, const uint8_t* comp_kv, int64_t cap, int ratio,
                                         const int32_t* topk, int k, const uint8_t* win_kv, int W, int Wr, int Q,
                                         const int32_t* seq_len, int B, float scale, int splits, float* opart,
-                                        float2* mlpart, int32_t* err, cudaStream_t stream);
+                                        float2* mlpart, int32_t* err, cudaStream_t stream, float kv_scale);
 
 }  // namespace csld

@@ -216,6 +216,31 @@ CSLD_API csld_status kv_cache_prefill_rope(const csld_layer_cache* cache, const 
                                            const float* gate, int64_t T, double rope_base, void* stream);
 
 /* ----------------------------------------------------------------------------------------
+ * Scaled FP8 entries -- a layout variant of the storage paragraph ([HF]: entries FP8 except the
+ * RoPE dims in bf16), with one positive scale kv_scale (sigma) per layer cache: an entry's (and
+ * a window entry's) 448 FP8 dims hold E4M3(x / sigma), RNE, saturating at +-448, and stand for
+ * sigma times their code value; the 64 bf16 RoPE dims are not scaled; the indexer key is
+ * projected from the unscaled pooled vector.  A small sigma keeps values below E4M3's
+ * subnormals, a large one values above 448.  2^-60 <= kv_scale <= 2^60.
+ *   csld_compress_scaled, kv_cache_prefill_scaled, kv_cache_append_scaled: as csld_compress,
+ *     kv_cache_prefill, kv_cache_append, writing scaled entries (a cache must be filled with
+ *     one sigma throughout);
+ *   hybrid_decode_attention_scaled: as hybrid_decode_attention over such entries -- the keys
+ *     and values are the decoded entries with their FP8 dims times kv_scale.
+ * The device multiplies by 1 / sigma in fp32 before rounding, so an E4M3 code may differ by one
+ * step from the exact quotient's where that lands near a rounding midpoint.
+ * -------------------------------------------------------------------------------------- */
+CSLD_API csld_status csld_compress_scaled(const uint16_t* raw, const float* gate, const float* pos_bias,
+                                          int ratio, const float* w_idx, int64_t T, float kv_scale,
+                                          uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out,
+                                          void* stream);
+CSLD_API csld_status kv_cache_prefill_scaled(const csld_layer_cache* cache, const uint16_t* raw,
+                                             const float* gate, int64_t T, float kv_scale, void* stream);
+CSLD_API csld_status kv_cache_append_scaled(const csld_layer_cache* cache, const uint16_t* kv_new,
+                                            const float* gate_new, float kv_scale, int32_t* err,
+                                            void* stream);
+
+/* ----------------------------------------------------------------------------------------
  * Lightning indexer + top-k ([HF] CSA paragraph: "FP4, ReLU-scored multi-head dot product"
  * picks the top-k compressed blocks per query; [VEL] core technique 1).
  * For sequence b, the visible entries are s < n_b = min(seq_len[b] / ratio, cap).  The query
@@ -285,6 +310,15 @@ CSLD_API csld_status hybrid_decode_attention(const uint16_t* q, int heads, const
                                     const uint8_t* win_kv, int W, const int32_t* seq_len, int B,
                                     float scale, float* out, float* lse_out, void* ws,
                                     size_t ws_bytes, int32_t* err, void* stream);
+/* hybrid_decode_attention over scaled FP8 entries (see csld_compress_scaled): the query's FP8
+ * part is multiplied by kv_scale before it meets the codes, and the output's FP8 dims by
+ * kv_scale at the end.  2^-60 <= kv_scale <= 2^60; otherwise as hybrid_decode_attention. */
+CSLD_API csld_status hybrid_decode_attention_scaled(const uint16_t* q, int heads, const uint8_t* comp_kv,
+                                                    int64_t cap, int ratio, const int32_t* topk, int k,
+                                                    const uint8_t* win_kv, int W, const int32_t* seq_len,
+                                                    int B, float scale, float kv_scale, float* out,
+                                                    float* lse_out, void* ws, size_t ws_bytes, int32_t* err,
+                                                    void* stream);
 
 /* ----------------------------------------------------------------------------------------
  * Multi-query decode attention ([HF] layer-pattern paragraph: the multi-token-prediction block
