@@ -98,7 +98,15 @@ def _declare(L):
                                    _P, _P, _P, _P, _P]
     L.orc_append_batch_variant.restype = C.c_int
     L.orc_append_batch_variant.argtypes = [C.c_int, C.c_int, C.c_int64, C.c_int, _P, _P, _P, _P, _P, _P,
-                                           _P, _P, _P, _P, _P, C.c_double, C.c_double]
+                                           _P, _P, _P, _P, _P, C.c_double, C.c_double, C.c_int]
+    L.orc_indexer_key_raw_perhead.restype = None
+    L.orc_indexer_key_raw_perhead.argtypes = [_P, _P, _P]
+    L.orc_compress_perhead.restype = None
+    L.orc_compress_perhead.argtypes = [_P, _P, _P, _P, C.c_int64, C.c_int, _P, _P, _P]
+    L.orc_indexer_scores_perhead.restype = None
+    L.orc_indexer_scores_perhead.argtypes = [_P, _P, C.c_int64, _P, _P, _P, _P]
+    L.orc_indexer_topk_batch_perhead.restype = None
+    L.orc_indexer_topk_batch_perhead.argtypes = [_P, _P, C.c_int64, _P, C.c_int, _P, _P, C.c_int, C.c_int, _P]
     L.orc_entry_encode_scaled.restype = None
     L.orc_entry_encode_scaled.argtypes = [_P, C.c_double, _P]
     L.orc_entry_decode_scaled.restype = None
@@ -321,6 +329,60 @@ def indexer_scores(ikeys, iscales, q_idx, head_w):
     return s32[:n], s64[:n]
 
 
+def indexer_key_raw_perhead(c, w_idx):
+    """Per-head keys before quantisation: c [512] f64, w_idx [512,4,64] f32 -> u [4,64] f64."""
+    c = _c(c, np.float64)
+    w_idx = _c(w_idx, np.float32)
+    u = np.zeros((IDX_HEADS, IDX_DIM), np.float64)
+    lib().orc_indexer_key_raw_perhead(_ptr(c), _ptr(w_idx), _ptr(u))
+    return u
+
+
+def compress_perhead(raw_bits, gate, bias, m, w_idx):
+    """Prefill compression with per-head indexer keys (w_idx [512,4,64]).  Returns (kv [E,576],
+    ikeys [E,4,32], iscales [E,4,2])."""
+    raw_bits = _c(raw_bits, np.uint16)
+    gate = _c(gate, np.float32)
+    bias = _c(bias, np.float32)
+    w = _c(w_idx, np.float32)
+    T = raw_bits.shape[0]
+    E = T // m
+    kv = np.zeros((E, ENTRY_BYTES), np.uint8)
+    ik = np.zeros((E, IDX_HEADS, IKEY_BYTES), np.uint8)
+    isc = np.zeros((E, IDX_HEADS, 2), np.float32)
+    lib().orc_compress_perhead(_ptr(raw_bits), _ptr(gate), _ptr(bias), _ptr(w), T, m, _ptr(kv), _ptr(ik), _ptr(isc))
+    return kv, ik, isc
+
+
+def indexer_scores_perhead(ikeys, iscales, q_idx, head_w):
+    """ikeys [n,4,32] u8, iscales [n,4,2] f32 (per-head keys), q_idx [4,64], head_w [4] ->
+    (score32, score64)."""
+    ikeys = _c(ikeys, np.uint8)
+    iscales = _c(iscales, np.float32)
+    q_idx = _c(q_idx, np.float32)
+    head_w = _c(head_w, np.float32)
+    n = ikeys.shape[0]
+    s32 = np.zeros(max(n, 1), np.float32)
+    s64 = np.zeros(max(n, 1), np.float64)
+    lib().orc_indexer_scores_perhead(_ptr(ikeys), _ptr(iscales), n, _ptr(q_idx), _ptr(head_w), _ptr(s32),
+                                     _ptr(s64))
+    return s32[:n], s64[:n]
+
+
+def indexer_topk_batch_perhead(ikeys, iscales, seq_len, ratio, q_idx, head_w, k):
+    """ikeys [B,cap,4,32], iscales [B,cap,4,2] (per-head keys); the rest as indexer_topk_batch."""
+    ikeys = _c(ikeys, np.uint8)
+    iscales = _c(iscales, np.float32)
+    seq_len = _c(seq_len, np.int32)
+    q_idx = _c(q_idx, np.float32)
+    head_w = _c(head_w, np.float32)
+    B, cap = ikeys.shape[0], ikeys.shape[1]
+    out = np.zeros((B, k), np.int32)
+    lib().orc_indexer_topk_batch_perhead(_ptr(ikeys), _ptr(iscales), cap, _ptr(seq_len), ratio, _ptr(q_idx),
+                                         _ptr(head_w), B, k, _ptr(out))
+    return out
+
+
 def topk(score32, k):
     score32 = _c(score32, np.float32)
     out = np.zeros(k, np.int32)
@@ -379,11 +441,14 @@ def attention_batch(q_bits, comp_kv, ratio, sel, win_kv, seq_len, scale, kv_scal
 class LayerState:
     """Host copy of one layer's cache state for B sequences (same layout as the device one)."""
 
-    def __init__(self, B, cap, m, W, with_indexer):
+    def __init__(self, B, cap, m, W, with_indexer, key_heads=1):
         self.B, self.cap, self.m, self.W = B, cap, m, W
+        self.key_heads = key_heads
         self.comp_kv = np.zeros((B, cap, ENTRY_BYTES), np.uint8)
-        self.ikeys = np.zeros((B, cap, IKEY_BYTES), np.uint8) if with_indexer else None
-        self.iscales = np.zeros((B, cap, 2), np.float32) if with_indexer else None
+        kshape = (B, cap, IKEY_BYTES) if key_heads == 1 else (B, cap, key_heads, IKEY_BYTES)
+        sshape = (B, cap, 2) if key_heads == 1 else (B, cap, key_heads, 2)
+        self.ikeys = np.zeros(kshape, np.uint8) if with_indexer else None
+        self.iscales = np.zeros(sshape, np.float32) if with_indexer else None
         self.win_kv = np.zeros((B, W, ENTRY_BYTES), np.uint8)
         self.tail_kv = np.zeros((B, m, D), np.uint16)
         self.tail_gate = np.zeros((B, m), np.float32)
@@ -401,7 +466,7 @@ def append_batch(st: LayerState, bias, w_idx, x_bits, gate, rope_base=0.0, kv_sc
     rc = lib().orc_append_batch_variant(st.m, st.W, st.cap, st.B, _ptr(st.comp_kv), _ptr(st.ikeys),
                                         _ptr(st.iscales), _ptr(st.win_kv), _ptr(st.tail_kv),
                                         _ptr(st.tail_gate), _ptr(st.seq_len), _ptr(bias), _ptr(w),
-                                        _ptr(x_bits), _ptr(gate), float(rope_base), float(kv_scale))
+                                        _ptr(x_bits), _ptr(gate), float(rope_base), float(kv_scale), st.key_heads)
     if rc != 0:
         raise OverflowError("oracle append: compressed cache capacity exceeded")
 

@@ -30,7 +30,9 @@
  *  - layout variants: per-channel gating (orc_pool_block_channel), RoPE applied at
  *    compressed positions (orc_rope_rotate: RoFormer pairs (448+2i, 449+2i), angle
  *    pos * base^(-i/32); an entry at its block's last token, a window entry at its token) and
- *    scaled FP8 entries (one scale per layer cache: E4M3(x / sigma), RoPE dims unscaled).
+ *    scaled FP8 entries (one scale per layer cache: E4M3(x / sigma), RoPE dims unscaled) and
+ *    per-head indexer keys (orc_indexer_key_raw_perhead: head h projected by its own W_h and
+ *    scored against its own key).
  *
  * parity unpinned: the real model's gate form, indexer projection and FP4 scale rule are not
  * given by the pages (no weights); what is pinned is listed in the tests.
@@ -305,47 +307,74 @@ void orc_rope_rotate(double* x, double pos, double base) {
     }
 }
 
+/* O2, per-head variant (a layout variant of the indexer key: [HF] CSA paragraph scores "a
+ * multi-head dot product" against the compressed entries; in the base reading the 4 indexer
+ * heads share one 64-d key per entry).  Here every head h has its own projection W_h and its
+ * own key: u_h = c . W_h, with w_idx [512][4][64] row-major (W_h[d][j] = w_idx[d*256 + h*64 + j]),
+ * each head's key FP4-quantised as in the base (two groups of 32, power-of-two scales). */
+void orc_indexer_key_raw_perhead(const double* c, const float* w_idx, double* u) {
+    for (int h = 0; h < ORC_IDX_HEADS; ++h)
+        for (int j = 0; j < ORC_IDX_DIM; ++j) {
+            double acc = 0.0;
+            for (int d = 0; d < ORC_D; ++d)
+                acc += c[d] * (double)w_idx[(size_t)d * ORC_IDX_HEADS * ORC_IDX_DIM + h * ORC_IDX_DIM + j];
+            u[h * ORC_IDX_DIM + j] = acc;
+        }
+}
+
 /* O1 + O2 over a whole prefill: T tokens of one sequence -> floor(T/m) entries; the trailing
  * T mod m tokens form no entry.  ikey_out / iscale_out are written only when w_idx != NULL
  * (CSA; [HF] CSA paragraph: the lightning indexer runs over the 4x-compressed entries).
  * rope_base > 0: O1r, entry s rotated at position pos0 + (s+1) m - 1 after pooling. */
 static void orc_compress_impl(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
-                              int64_t T, int m, int64_t pos0, double rope_base, double kv_scale, uint8_t* kv_out,
-                              uint8_t* ikey_out, float* iscale_out) {
+                              int64_t T, int m, int64_t pos0, double rope_base, double kv_scale, int key_heads,
+                              uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
     int64_t E = T / m;
 #pragma omp parallel for schedule(static)
     for (int64_t s = 0; s < E; ++s) {
-        double c[ORC_D], u[ORC_IDX_DIM];
+        double c[ORC_D], u[ORC_IDX_HEADS * ORC_IDX_DIM];
         orc_pool_block(raw + (size_t)s * m * ORC_D, gate + (size_t)s * m, bias, m, c);
         if (rope_base > 0.0) orc_rope_rotate(c, (double)(pos0 + (s + 1) * (int64_t)m - 1), rope_base);
         if (kv_scale != 1.0)
             orc_entry_encode_scaled(c, kv_scale, kv_out + (size_t)s * ORC_ENTRY_BYTES);
         else
             orc_entry_encode(c, kv_out + (size_t)s * ORC_ENTRY_BYTES);
-        if (w_idx) {
+        if (w_idx && key_heads == 1) {
             orc_indexer_key_raw(c, w_idx, u);
             orc_fp4_quantize64(u, ikey_out + (size_t)s * ORC_IKEY_BYTES, iscale_out + (size_t)s * 2);
+        } else if (w_idx) {
+            orc_indexer_key_raw_perhead(c, w_idx, u);
+            for (int h = 0; h < ORC_IDX_HEADS; ++h)
+                orc_fp4_quantize64(u + h * ORC_IDX_DIM, ikey_out + ((size_t)s * ORC_IDX_HEADS + h) * ORC_IKEY_BYTES,
+                                   iscale_out + ((size_t)s * ORC_IDX_HEADS + h) * 2);
         }
     }
 }
 
 void orc_compress(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
                   int64_t T, int m, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
-    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, 1.0, kv_out, ikey_out, iscale_out);
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, 1.0, 1, kv_out, ikey_out, iscale_out);
 }
 
 /* O1r + O1 + O2: raw token 0 at position pos0, rotation base rope_base > 0. */
 void orc_compress_rope(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
                        int64_t T, int m, int64_t pos0, double rope_base, uint8_t* kv_out,
                        uint8_t* ikey_out, float* iscale_out) {
-    orc_compress_impl(raw, gate, bias, w_idx, T, m, pos0, rope_base, 1.0, kv_out, ikey_out, iscale_out);
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, pos0, rope_base, 1.0, 1, kv_out, ikey_out, iscale_out);
 }
 
 /* Scaled FP8 entries: as orc_compress with entries encoded by orc_entry_encode_scaled (the
  * indexer key is projected from the unscaled pooled vector). */
 void orc_compress_scaled(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
                          int64_t T, int m, double kv_scale, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
-    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, kv_scale, kv_out, ikey_out, iscale_out);
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, kv_scale, 1, kv_out, ikey_out, iscale_out);
+}
+
+/* Per-head indexer keys: as orc_compress with w_idx [512][4][64]; ikey_out [E][4][32] (each
+ * head's 32 code bytes as in the base), iscale_out [E][4][2]. */
+void orc_compress_perhead(const uint16_t* raw, const float* gate, const float* bias, const float* w_idx,
+                          int64_t T, int m, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out) {
+    orc_compress_impl(raw, gate, bias, w_idx, T, m, 0, 0.0, 1.0, ORC_IDX_HEADS, kv_out, ikey_out, iscale_out);
 }
 
 /* O1 (per-channel) + O2 over a whole prefill: gate [T][512], bias [m][512]. */
@@ -382,8 +411,8 @@ static int orc_twice_e2m1(uint8_t c) {       /* 2 * value of an E2M1 code: an in
     return (int)lrint(2.0 * orc_e2m1_decode(c));
 }
 
-void orc_indexer_scores(const uint8_t* ikeys, const float* iscales, int64_t n,
-                        const float* q_idx, const float* head_w, float* score32, double* score64) {
+static void orc_indexer_scores_impl(const uint8_t* ikeys, const float* iscales, int64_t n, int key_heads,
+                                    const float* q_idx, const float* head_w, float* score32, double* score64) {
     uint8_t qc[ORC_IDX_HEADS][ORC_IKEY_BYTES];
     float qs[ORC_IDX_HEADS][2];
     double qd[ORC_IDX_HEADS][ORC_IDX_DIM];
@@ -395,13 +424,15 @@ void orc_indexer_scores(const uint8_t* ikeys, const float* iscales, int64_t n,
     }
 #pragma omp parallel for schedule(static)
     for (int64_t s = 0; s < n; ++s) {
-        const uint8_t* kc = ikeys + (size_t)s * ORC_IKEY_BYTES;
-        const float* ks = iscales + (size_t)s * 2;
-        double kd[ORC_IDX_DIM];
-        orc_fp4_dequantize64(kc, ks, kd);
         float r32[ORC_IDX_HEADS];
         double e64 = 0.0;
         for (int h = 0; h < ORC_IDX_HEADS; ++h) {
+            /* the head's key: the entry's one key, or (per-head keys) key h of the entry */
+            const int kh = key_heads == 1 ? 0 : h;
+            const uint8_t* kc = ikeys + ((size_t)s * key_heads + kh) * ORC_IKEY_BYTES;
+            const float* ks = iscales + ((size_t)s * key_heads + kh) * 2;
+            double kd[ORC_IDX_DIM];
+            orc_fp4_dequantize64(kc, ks, kd);
             long I[2] = {0, 0};
             double dot = 0.0;
             for (int d = 0; d < ORC_IDX_DIM; ++d) {
@@ -423,6 +454,18 @@ void orc_indexer_scores(const uint8_t* ikeys, const float* iscales, int64_t n,
         if (score32) score32[s] = e;
         if (score64) score64[s] = e64;
     }
+}
+
+void orc_indexer_scores(const uint8_t* ikeys, const float* iscales, int64_t n,
+                        const float* q_idx, const float* head_w, float* score32, double* score64) {
+    orc_indexer_scores_impl(ikeys, iscales, n, 1, q_idx, head_w, score32, score64);
+}
+
+/* O3 with per-head keys: ikeys [n][4][32], iscales [n][4][2]; head h scores against key h,
+ * in the same fp32 operation order. */
+void orc_indexer_scores_perhead(const uint8_t* ikeys, const float* iscales, int64_t n,
+                                const float* q_idx, const float* head_w, float* score32, double* score64) {
+    orc_indexer_scores_impl(ikeys, iscales, n, ORC_IDX_HEADS, q_idx, head_w, score32, score64);
 }
 
 /* ------------------------------------------------------------------------------------------
@@ -469,19 +512,31 @@ void orc_topk64(const double* score64, int64_t n, int k, int32_t* out) {
 
 /* Batched indexer + top-k for B sequences: keys [B][cap], the visible count of sequence b is
  * min(seq_len[b] / ratio, cap). */
-void orc_indexer_topk_batch(const uint8_t* ikeys, const float* iscales, int64_t cap,
-                            const int32_t* seq_len, int ratio, const float* q_idx,
-                            const float* head_w, int B, int k, int32_t* out) {
+static void orc_indexer_topk_batch_impl(const uint8_t* ikeys, const float* iscales, int64_t cap, int key_heads,
+                                        const int32_t* seq_len, int ratio, const float* q_idx,
+                                        const float* head_w, int B, int k, int32_t* out) {
     for (int b = 0; b < B; ++b) {
         int64_t n = seq_len[b] / ratio;
         if (n > cap) n = cap;
         float* sc = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
-        orc_indexer_scores(ikeys + (size_t)b * cap * ORC_IKEY_BYTES, iscales + (size_t)b * cap * 2,
-                           n, q_idx + (size_t)b * ORC_IDX_HEADS * ORC_IDX_DIM,
-                           head_w + (size_t)b * ORC_IDX_HEADS, sc, NULL);
+        orc_indexer_scores_impl(ikeys + (size_t)b * cap * key_heads * ORC_IKEY_BYTES,
+                                iscales + (size_t)b * cap * key_heads * 2, n, key_heads,
+                                q_idx + (size_t)b * ORC_IDX_HEADS * ORC_IDX_DIM,
+                                head_w + (size_t)b * ORC_IDX_HEADS, sc, NULL);
         orc_topk(sc, n, k, out + (size_t)b * k);
         free(sc);
     }
+}
+void orc_indexer_topk_batch(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                            const int32_t* seq_len, int ratio, const float* q_idx,
+                            const float* head_w, int B, int k, int32_t* out) {
+    orc_indexer_topk_batch_impl(ikeys, iscales, cap, 1, seq_len, ratio, q_idx, head_w, B, k, out);
+}
+/* Per-head keys: ikeys [B][cap][4][32], iscales [B][cap][4][2]. */
+void orc_indexer_topk_batch_perhead(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                                    const int32_t* seq_len, int ratio, const float* q_idx,
+                                    const float* head_w, int B, int k, int32_t* out) {
+    orc_indexer_topk_batch_impl(ikeys, iscales, cap, ORC_IDX_HEADS, seq_len, ratio, q_idx, head_w, B, k, out);
 }
 
 /* ------------------------------------------------------------------------------------------
@@ -603,7 +658,7 @@ int orc_attention_batch(const uint16_t* q, int H, const uint8_t* comp_kv, int64_
 static int orc_append_impl(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, float* iscales,
                            uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate, int32_t* seq_len,
                            const float* bias, const float* w_idx, const uint16_t* x, float gate,
-                           double rope_base, double kv_scale) {
+                           double rope_base, double kv_scale, int key_heads) {
     int32_t t = *seq_len;
     int complete = ((t + 1) % m) == 0;
     int64_t s = t / m;
@@ -617,13 +672,18 @@ static int orc_append_impl(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t*
     memcpy(tail_kv + (size_t)(t % m) * ORC_D, x, sizeof(uint16_t) * ORC_D);
     tail_gate[t % m] = gate;
     if (complete) {
-        double c[ORC_D], u[ORC_IDX_DIM];
+        double c[ORC_D], u[ORC_IDX_HEADS * ORC_IDX_DIM];
         orc_pool_block(tail_kv, tail_gate, bias, m, c);
         if (rope_base > 0.0) orc_rope_rotate(c, (double)t, rope_base);
         orc_entry_encode_scaled(c, kv_scale, comp_kv + (size_t)s * ORC_ENTRY_BYTES);
-        if (w_idx) {
+        if (w_idx && key_heads == 1) {
             orc_indexer_key_raw(c, w_idx, u);
             orc_fp4_quantize64(u, ikeys + (size_t)s * ORC_IKEY_BYTES, iscales + (size_t)s * 2);
+        } else if (w_idx) {
+            orc_indexer_key_raw_perhead(c, w_idx, u);
+            for (int h = 0; h < ORC_IDX_HEADS; ++h)
+                orc_fp4_quantize64(u + h * ORC_IDX_DIM, ikeys + ((size_t)s * ORC_IDX_HEADS + h) * ORC_IKEY_BYTES,
+                                   iscales + ((size_t)s * ORC_IDX_HEADS + h) * 2);
         }
     }
     *seq_len = t + 1;
@@ -634,23 +694,24 @@ int orc_append(int m, int W, int64_t cap, uint8_t* comp_kv, uint8_t* ikeys, floa
                uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate, int32_t* seq_len,
                const float* bias, const float* w_idx, const uint16_t* x, float gate) {
     return orc_append_impl(m, W, cap, comp_kv, ikeys, iscales, win_kv, tail_kv, tail_gate, seq_len, bias,
-                           w_idx, x, gate, 0.0, 1.0);
+                           w_idx, x, gate, 0.0, 1.0, 1);
 }
 
 /* The same for B sequences, one token each: x [B][512], gate [B]; rope_base as above (0: none);
- * kv_scale: scaled FP8 entries (1: the base layout). */
+ * kv_scale: scaled FP8 entries (1: the base layout); key_heads: 1 (one shared indexer key) or 4
+ * (per-head keys, w_idx [512][4][64], ikeys [B][cap][4][32], iscales [B][cap][4][2]). */
 int orc_append_batch_variant(int m, int W, int64_t cap, int B, uint8_t* comp_kv, uint8_t* ikeys,
                              float* iscales, uint8_t* win_kv, uint16_t* tail_kv, float* tail_gate,
                              int32_t* seq_len, const float* bias, const float* w_idx, const uint16_t* x,
-                             const float* gate, double rope_base, double kv_scale) {
+                             const float* gate, double rope_base, double kv_scale, int key_heads) {
     int rc = 0;
     for (int b = 0; b < B; ++b) {
         rc |= orc_append_impl(m, W, cap, comp_kv + (size_t)b * cap * ORC_ENTRY_BYTES,
-                              ikeys ? ikeys + (size_t)b * cap * ORC_IKEY_BYTES : NULL,
-                              iscales ? iscales + (size_t)b * cap * 2 : NULL,
+                              ikeys ? ikeys + (size_t)b * cap * key_heads * ORC_IKEY_BYTES : NULL,
+                              iscales ? iscales + (size_t)b * cap * key_heads * 2 : NULL,
                               win_kv + (size_t)b * (W > 0 ? W : 0) * ORC_ENTRY_BYTES,
                               tail_kv + (size_t)b * m * ORC_D, tail_gate + (size_t)b * m, seq_len + b,
-                              bias, w_idx, x + (size_t)b * ORC_D, gate[b], rope_base, kv_scale);
+                              bias, w_idx, x + (size_t)b * ORC_D, gate[b], rope_base, kv_scale, key_heads);
     }
     return rc;
 }
@@ -660,7 +721,7 @@ int orc_append_batch(int m, int W, int64_t cap, int B, uint8_t* comp_kv, uint8_t
                      int32_t* seq_len, const float* bias, const float* w_idx, const uint16_t* x,
                      const float* gate) {
     return orc_append_batch_variant(m, W, cap, B, comp_kv, ikeys, iscales, win_kv, tail_kv, tail_gate, seq_len,
-                                    bias, w_idx, x, gate, 0.0, 1.0);
+                                    bias, w_idx, x, gate, 0.0, 1.0, 1);
 }
 
 int orc_num_threads(void) {
