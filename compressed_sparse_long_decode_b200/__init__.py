@@ -18,7 +18,8 @@ import torch
 __all__ = [
     "csa_compress", "hca_compress", "compress", "compress_channel", "compress_rope", "kv_cache_append_rope",
     "kv_cache_prefill_rope", "compress_scaled", "kv_cache_append_scaled", "kv_cache_prefill_scaled",
-    "hybrid_decode_attention_scaled", "indexer_topk", "hybrid_decode_attention",
+    "hybrid_decode_attention_scaled", "compress_perhead", "kv_cache_prefill_perhead", "kv_cache_append_perhead",
+    "indexer_topk_perhead", "indexer_topk", "hybrid_decode_attention",
     "kv_cache_append", "kv_cache_prefill", "LayerCache", "CsldError", "lib", "ENTRY_BYTES",
     "IKEY_BYTES", "DIM", "HEADS", "indexer_workspace", "attention_workspace", "DecodeStack",
     "layer_pattern", "stage", "indexer_rescore", "topk_merge", "lse_merge", "ContextParallelLayer",
@@ -71,6 +72,10 @@ def _load():
     L.kv_cache_append_scaled.argtypes = [C.POINTER(_Cache), P, P, F, P, P]
     L.kv_cache_prefill_scaled.argtypes = [C.POINTER(_Cache), P, P, I64, F, P]
     L.hybrid_decode_attention_scaled.argtypes = [P, I, P, I64, I, P, I, P, I, P, I, F, F, P, P, P, S, P, P]
+    L.csld_compress_perhead.argtypes = [P, P, P, I, P, I64, P, P, P, P]
+    L.kv_cache_prefill_perhead.argtypes = [C.POINTER(_Cache), P, P, I64, P]
+    L.kv_cache_append_perhead.argtypes = [C.POINTER(_Cache), P, P, P, P]
+    L.indexer_topk_perhead.argtypes = [P, P, I64, P, I, P, P, I, I, I, P, P, S, P, P]
     L.csa_compress.argtypes = [P, P, P, P, I64, P, P, P, P]
     L.hca_compress.argtypes = [P, P, P, I64, P, P]
     L.kv_cache_append.argtypes = [C.POINTER(_Cache), P, P, P, P]
@@ -91,7 +96,8 @@ def _load():
     L.csld_lse_merge.argtypes = [P, P, I, I, I, P, P, P]
     for fn in ("csld_compress", "csld_compress_channel", "csld_compress_rope", "kv_cache_append_rope",
                "kv_cache_prefill_rope", "csld_compress_scaled", "kv_cache_append_scaled", "kv_cache_prefill_scaled",
-               "hybrid_decode_attention_scaled", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
+               "hybrid_decode_attention_scaled", "csld_compress_perhead", "kv_cache_prefill_perhead",
+               "kv_cache_append_perhead", "indexer_topk_perhead", "csa_compress", "hca_compress", "kv_cache_append", "kv_cache_prefill",
                "indexer_topk", "hybrid_decode_attention", "csld_stage", "indexer_rescore", "csld_topk_merge",
                "csld_lse_merge", "indexer_topk_multi", "hybrid_decode_attention_multi"):
         getattr(L, fn).restype = I
@@ -224,6 +230,27 @@ def compress_scaled(raw, gate, pos_bias, ratio, kv_scale, w_idx=None, kv_out=Non
     return (kv_out, ikey_out, iscale_out) if w_idx is not None else kv_out
 
 
+def compress_perhead(raw, gate, pos_bias, ratio, w_idx, kv_out=None, ikey_out=None, iscale_out=None):
+    """Compression with per-head indexer keys (csld_compress_perhead): w_idx [512,4,64] f32 ->
+    (kv [E,576], ikeys [E,128] in the stored layout, iscales [E,4,2])."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    _need(pos_bias, torch.float32, "pos_bias")
+    _need(w_idx, torch.float32, "w_idx")
+    T = raw.shape[0]
+    E = T // ratio
+    dev = raw.device
+    if kv_out is None:
+        kv_out = torch.empty((E, ENTRY_BYTES), dtype=torch.uint8, device=dev)
+    if ikey_out is None:
+        ikey_out = torch.empty((E, 4 * IKEY_BYTES), dtype=torch.uint8, device=dev)
+    if iscale_out is None:
+        iscale_out = torch.empty((E, 4, 2), dtype=torch.float32, device=dev)
+    _check(lib.csld_compress_perhead(_ptr(raw), _ptr(gate), _ptr(pos_bias), ratio, _ptr(w_idx), T, _ptr(kv_out),
+                                     _ptr(ikey_out), _ptr(iscale_out), _stream()), "csld_compress_perhead")
+    return kv_out, ikey_out, iscale_out
+
+
 def csa_compress(raw, gate, pos_bias, w_idx, kv_out=None, ikey_out=None, iscale_out=None):
     return compress(raw, gate, pos_bias, 4, w_idx, kv_out, ikey_out, iscale_out)
 
@@ -236,15 +263,20 @@ def hca_compress(raw, gate, pos_bias, kv_out=None):
 class LayerCache:
     """One layer's cache state for B sequences, in device memory owned by torch."""
 
-    def __init__(self, batch, capacity, ratio, window, pos_bias, w_idx=None, device="cuda"):
+    def __init__(self, batch, capacity, ratio, window, pos_bias, w_idx=None, device="cuda", perhead=False):
+        """perhead: per-head indexer keys (w_idx [512,4,64]; ikeys [B,cap,128], iscales [B,cap,4,2]),
+        filled by the *_perhead calls."""
         if w_idx is not None and capacity % 2:
             capacity += 1
         self.batch, self.capacity, self.ratio, self.window = batch, capacity, ratio, window
         dev = torch.device(device)
         self.comp_kv = torch.zeros((batch, capacity, ENTRY_BYTES), dtype=torch.uint8, device=dev)
         self.has_indexer = w_idx is not None
-        self.ikeys = torch.zeros((batch, capacity, IKEY_BYTES), dtype=torch.uint8, device=dev) if self.has_indexer else None
-        self.iscales = torch.zeros((batch, capacity, 2), dtype=torch.float32, device=dev) if self.has_indexer else None
+        self.perhead = perhead
+        kshape = (batch, capacity, 4 * IKEY_BYTES) if perhead else (batch, capacity, IKEY_BYTES)
+        sshape = (batch, capacity, 4, 2) if perhead else (batch, capacity, 2)
+        self.ikeys = torch.zeros(kshape, dtype=torch.uint8, device=dev) if self.has_indexer else None
+        self.iscales = torch.zeros(sshape, dtype=torch.float32, device=dev) if self.has_indexer else None
         self.win_kv = torch.zeros((batch, max(window, 1), ENTRY_BYTES), dtype=torch.uint8, device=dev)
         self.tail_kv = torch.zeros((batch, ratio, DIM), dtype=torch.bfloat16, device=dev)
         self.tail_gate = torch.zeros((batch, ratio), dtype=torch.float32, device=dev)
@@ -305,6 +337,24 @@ def kv_cache_prefill_scaled(cache: LayerCache, raw, gate, kv_scale):
            "kv_cache_prefill_scaled")
 
 
+def kv_cache_append_perhead(cache: LayerCache, kv_new, gate_new, err=None):
+    """kv_cache_append with per-head indexer keys (kv_cache_append_perhead)."""
+    _bits(kv_new, "kv_new")
+    _need(gate_new, torch.float32, "gate_new")
+    s = cache.struct()
+    _check(lib.kv_cache_append_perhead(C.byref(s), _ptr(kv_new), _ptr(gate_new), _ptr(cache.err if err is None else err),
+                                       _stream()), "kv_cache_append_perhead")
+
+
+def kv_cache_prefill_perhead(cache: LayerCache, raw, gate):
+    """kv_cache_prefill with per-head indexer keys (kv_cache_prefill_perhead)."""
+    _bits(raw, "raw")
+    _need(gate, torch.float32, "gate")
+    s = cache.struct()
+    _check(lib.kv_cache_prefill_perhead(C.byref(s), _ptr(raw), _ptr(gate), raw.shape[1], _stream()),
+           "kv_cache_prefill_perhead")
+
+
 def kv_cache_prefill(cache: LayerCache, raw, gate):
     """Prefill all sequences with T tokens: raw [B,T,512] bf16, gate [B,T] f32."""
     _bits(raw, "raw")
@@ -342,6 +392,26 @@ def indexer_topk(ikeys, iscales, seq_len, ratio, q_idx, head_w, k, out=None, ws=
 def indexer_multi_workspace(B, Q, cap, device="cuda"):
     n = lib.csld_indexer_multi_workspace_size(B, Q, cap)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def indexer_topk_perhead(ikeys, iscales, seq_len, ratio, q_idx, head_w, k, out=None, ws=None, err=None):
+    """Per-head indexer keys (indexer_topk_perhead): ikeys [B,cap,128] u8 (stored layout),
+    iscales [B,cap,4,2] f32, q_idx [B,Q,4,64] f32, head_w [B,Q,4] f32 -> top-k [B,Q,k] i32."""
+    _need(ikeys, torch.uint8, "ikeys")
+    _need(iscales, torch.float32, "iscales")
+    _need(seq_len, torch.int32, "seq_len")
+    _need(q_idx, torch.float32, "q_idx")
+    _need(head_w, torch.float32, "head_w")
+    B, cap = ikeys.shape[0], ikeys.shape[1]
+    Q = q_idx.shape[1]
+    if out is None:
+        out = torch.empty((B, Q, k), dtype=torch.int32, device=ikeys.device)
+    if ws is None:
+        ws = indexer_multi_workspace(B, Q, cap, ikeys.device)
+    _check(lib.indexer_topk_perhead(_ptr(ikeys), _ptr(iscales), cap, _ptr(seq_len), ratio, _ptr(q_idx), _ptr(head_w),
+                                    B, Q, k, _ptr(out), _ptr(ws), ws.numel(), _ptr(err), _stream()),
+           "indexer_topk_perhead")
+    return out
 
 
 def indexer_topk_multi(ikeys, iscales, seq_len, ratio, q_idx, head_w, k, out=None, ws=None, err=None):

@@ -17,7 +17,8 @@ cudaError_t launch_stage(void* dst, const void* src, size_t bytes, int num_sms, 
 size_t indexer_multi_ws_bytes(int B, int Q, int64_t cap, int num_sms);
 cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
                                  int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
-                                 int32_t* topk_out, void* ws, int num_sms, int32_t* err, cudaStream_t stream);
+                                 int32_t* topk_out, void* ws, int num_sms, int32_t* err, cudaStream_t stream,
+                                 bool perhead = false);
 // cp.cu
 cudaError_t launch_indexer_rescore(const uint8_t* ikeys, const float* iscales, int64_t cap, const float* q_idx,
                                    const float* head_w, const int32_t* sel, int B, int k, float* scores,
@@ -116,7 +117,7 @@ const char* csld_status_string(csld_status s) {
 namespace {
 csld_status compress_impl(const char* name, const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
                           const float* w_idx, int64_t T, int64_t pos0, double rope_base, float kv_scale,
-                          uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, void* stream) {
+                          uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, void* stream, bool perhead = false) {
     if (ratio < 1 || ratio > CSLD_MAX_RATIO) return fail(CSLD_ERR_ARG, "ratio %d outside 1..%d", ratio, CSLD_MAX_RATIO);
     if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
     if (T / ratio == 0) return CSLD_OK;
@@ -126,7 +127,7 @@ csld_status compress_impl(const char* name, const uint16_t* raw, const float* ga
         return fail(CSLD_ERR_ALIGN, "raw, kv_out and ikey_out must be 16-byte aligned");
     cudaError_t e = csld::launch_compress(raw, gate, pos_bias, ratio, w_idx, T, 1, T / ratio, kv_out,
                                           ikey_out, iscale_out, num_sms(), as_stream(stream), pos0, rope_base,
-                                          kv_scale);
+                                          kv_scale, perhead);
     if (e != cudaSuccess) return cuda_fail(e, name);
     return CSLD_OK;
 }
@@ -152,6 +153,14 @@ namespace {
 bool kv_scale_ok(float kv_scale) { return kv_scale >= 0x1p-60f && kv_scale <= 0x1p60f; }
 }  // namespace
 
+csld_status csld_compress_perhead(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
+                                  const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out,
+                                  void* stream) {
+    if (!w_idx) return fail(CSLD_ERR_ARG, "w_idx is NULL (per-head keys need the projection)");
+    return compress_impl("csld_compress_perhead", raw, gate, pos_bias, ratio, w_idx, T, 0, 0.0, 1.f, kv_out, ikey_out,
+                         iscale_out, stream, true);
+}
+
 csld_status csld_compress_scaled(const uint16_t* raw, const float* gate, const float* pos_bias, int ratio,
                                  const float* w_idx, int64_t T, float kv_scale, uint8_t* kv_out, uint8_t* ikey_out,
                                  float* iscale_out, void* stream) {
@@ -174,12 +183,13 @@ csld_status hca_compress(const uint16_t* raw, const float* gate, const float* po
 
 namespace {
 csld_status append_impl(const char* name, const csld_layer_cache* cache, const uint16_t* kv_new,
-                        const float* gate_new, int32_t* err, double rope_base, float kv_scale, void* stream) {
+                        const float* gate_new, int32_t* err, double rope_base, float kv_scale, void* stream,
+                        bool perhead = false) {
     csld_status s = check_cache(cache);
     if (s != CSLD_OK) return s;
     if (!kv_new || !gate_new) return fail(CSLD_ERR_ARG, "kv_new / gate_new is NULL");
     if (!aligned16(kv_new)) return fail(CSLD_ERR_ALIGN, "kv_new must be 16-byte aligned");
-    cudaError_t e = csld::launch_append(*cache, kv_new, gate_new, err, as_stream(stream), rope_base, kv_scale);
+    cudaError_t e = csld::launch_append(*cache, kv_new, gate_new, err, as_stream(stream), rope_base, kv_scale, perhead);
     if (e != cudaSuccess) return cuda_fail(e, name);
     return CSLD_OK;
 }
@@ -196,6 +206,12 @@ csld_status kv_cache_append_rope(const csld_layer_cache* cache, const uint16_t* 
     return append_impl("kv_cache_append_rope", cache, kv_new, gate_new, err, rope_base, 1.f, stream);
 }
 
+csld_status kv_cache_append_perhead(const csld_layer_cache* cache, const uint16_t* kv_new,
+                                    const float* gate_new, int32_t* err, void* stream) {
+    if (!cache || !cache->has_indexer) return fail(CSLD_ERR_ARG, "per-head keys need a cache with an indexer");
+    return append_impl("kv_cache_append_perhead", cache, kv_new, gate_new, err, 0.0, 1.f, stream, true);
+}
+
 csld_status kv_cache_append_scaled(const csld_layer_cache* cache, const uint16_t* kv_new,
                                    const float* gate_new, float kv_scale, int32_t* err, void* stream) {
     if (!kv_scale_ok(kv_scale)) return fail(CSLD_ERR_ARG, "kv_scale %g outside 2^-60..2^60", (double)kv_scale);
@@ -204,7 +220,7 @@ csld_status kv_cache_append_scaled(const csld_layer_cache* cache, const uint16_t
 
 namespace {
 csld_status prefill_impl(const csld_layer_cache* cache, const uint16_t* raw, const float* gate, int64_t T,
-                         double rope_base, float kv_scale, void* stream) {
+                         double rope_base, float kv_scale, void* stream, bool perhead = false) {
     csld_status s = check_cache(cache);
     if (s != CSLD_OK) return s;
     if (T < 0 || T > (int64_t)INT32_MAX) return fail(CSLD_ERR_ARG, "T %lld outside 0..2^31-1", (long long)T);
@@ -217,7 +233,7 @@ csld_status prefill_impl(const csld_layer_cache* cache, const uint16_t* raw, con
     cudaError_t e = csld::launch_compress(raw, gate, cache->pos_bias, cache->ratio,
                                           cache->has_indexer ? cache->w_idx : nullptr, T, cache->batch,
                                           cache->capacity, cache->comp_kv, cache->ikeys,
-                                          cache->iscales, num_sms(), st, 0, rope_base, kv_scale);
+                                          cache->iscales, num_sms(), st, 0, rope_base, kv_scale, perhead);
     if (e != cudaSuccess) return cuda_fail(e, "kv_cache_prefill (compress)");
     e = csld::launch_prefill_state(raw, gate, T, cache->ratio, cache->window, cache->batch,
                                    cache->win_kv, cache->tail_kv, cache->tail_gate, cache->seq_len, st, rope_base,
@@ -236,6 +252,12 @@ csld_status kv_cache_prefill_rope(const csld_layer_cache* cache, const uint16_t*
                                   int64_t T, double rope_base, void* stream) {
     if (!(rope_base > 1.0) || rope_base == INFINITY) return fail(CSLD_ERR_ARG, "rope_base must be finite and > 1");
     return prefill_impl(cache, raw, gate, T, rope_base, 1.f, stream);
+}
+
+csld_status kv_cache_prefill_perhead(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
+                                     int64_t T, void* stream) {
+    if (!cache || !cache->has_indexer) return fail(CSLD_ERR_ARG, "per-head keys need a cache with an indexer");
+    return prefill_impl(cache, raw, gate, T, 0.0, 1.f, stream, true);
 }
 
 csld_status kv_cache_prefill_scaled(const csld_layer_cache* cache, const uint16_t* raw, const float* gate,
@@ -412,9 +434,11 @@ size_t csld_indexer_multi_workspace_size(int B, int Q, int64_t cap) {
     return csld::indexer_multi_ws_bytes(B, Q, cap, num_sms());
 }
 
-csld_status indexer_topk_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
-                               int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
-                               int32_t* topk_out, void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+namespace {
+csld_status indexer_multi_impl(const char* name, const uint8_t* ikeys, const float* iscales, int64_t cap,
+                               const int32_t* seq_len, int ratio, const float* q_idx, const float* head_w, int B, int Q,
+                               int k, int32_t* topk_out, void* ws, size_t ws_bytes, int32_t* err, void* stream,
+                               bool perhead) {
     if (B < 1 || B > 65535) return fail(CSLD_ERR_ARG, "B %d outside 1..65535", B);
     if (Q < 1 || Q > CSLD_MULTI_MAX_Q) return fail(CSLD_ERR_ARG, "Q %d outside 1..%d", Q, CSLD_MULTI_MAX_Q);
     if (k < 1 || k > CSLD_MAX_TOPK) return fail(CSLD_ERR_ARG, "k %d outside 1..%d", k, CSLD_MAX_TOPK);
@@ -428,9 +452,24 @@ csld_status indexer_topk_multi(const uint8_t* ikeys, const float* iscales, int64
     if (!ws || ws_bytes < need) return fail(CSLD_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CSLD_ERR_ALIGN, "workspace must be 256-byte aligned");
     cudaError_t e = csld::launch_indexer_multi(ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, B, Q, k, topk_out,
-                                               ws, num_sms(), err, as_stream(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_multi");
+                                               ws, num_sms(), err, as_stream(stream), perhead);
+    if (e != cudaSuccess) return cuda_fail(e, name);
     return CSLD_OK;
+}
+}  // namespace
+
+csld_status indexer_topk_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
+                               int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
+                               int32_t* topk_out, void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+    return indexer_multi_impl("indexer_topk_multi", ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, B, Q, k,
+                              topk_out, ws, ws_bytes, err, stream, false);
+}
+
+csld_status indexer_topk_perhead(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
+                                 int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
+                                 int32_t* topk_out, void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+    return indexer_multi_impl("indexer_topk_perhead", ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, B, Q, k,
+                              topk_out, ws, ws_bytes, err, stream, true);
 }
 
 csld_status hybrid_decode_attention_multi(const uint16_t* q, int heads, const uint8_t* comp_kv, int64_t cap,

@@ -17,7 +17,10 @@
 //    rotary encoding and rotated here -- a pooled entry at its block's last token, a window
 //    entry at its own token (RoFormer pairs, see rope_lane);
 //  - kVarScaled, scaled FP8 entries: one scale sigma per layer cache, the FP8 dims stored as
-//    E4M3(x / sigma) (the kernels get 1 / sigma), the RoPE dims and the indexer key unscaled.
+//    E4M3(x / sigma) (the kernels get 1 / sigma), the RoPE dims and the indexer key unscaled;
+//  - kVarPerHead, per-head indexer keys: W_I [512][4][64], one FP4 key per head and entry,
+//    stored as 128-byte rows [head][32 code bytes] pre-swizzled for a 128-byte-swizzle K-major
+//    operand (16-byte chunk c of entry s at chunk c ^ (s mod 8)), scales [entry][head][group].
 #include "csld_internal.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -155,7 +158,30 @@ __device__ __forceinline__ uint2 rope_bf16x4(uint2 x, int j, int64_t pos, double
     return make_uint2(w[0], w[1]);
 }
 
-constexpr int kVarBase = 0, kVarRope = 1, kVarScaled = 2;
+constexpr int kVarBase = 0, kVarRope = 1, kVarScaled = 2, kVarPerHead = 3;
+constexpr int kIkeyHead = kIdxHeads * kIkey;   // 128 bytes of per-head key codes per entry
+
+// FP4 codes (4 words = 16 bytes) and the power-of-two scale of one 32-element group of fp32
+// values u[0..1][0..15] (the same quantisation as the shared key).
+__device__ __forceinline__ void fp4_group_words(const uint32_t (&u)[2][16], float* sc, uint32_t (&words)[4]) {
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(u[i >> 4][i & 15])));
+    *sc = fp4_group_scale(amax);
+    const float inv = 1.0f / *sc;   // exact: a power of two
+#pragma unroll
+    for (int wq = 0; wq < 4; ++wq) {
+        uint32_t word = 0u;
+#pragma unroll
+        for (int bq = 0; bq < 4; ++bq) {
+            const int i = 8 * wq + 2 * bq;
+            const uint32_t byte = e2m1_code(__uint_as_float(u[i >> 4][i & 15]) * inv) |
+                                  (e2m1_code(__uint_as_float(u[(i + 1) >> 4][(i + 1) & 15]) * inv) << 4);
+            word |= byte << (8 * bq);
+        }
+        words[wq] = word;
+    }
+}
 
 // E4M3 codes of four consecutive FP8 dims of a raw token held as bf16 (a window entry's FP8
 // part); kScaled: times inv_scale first.
@@ -207,6 +233,22 @@ __device__ __forceinline__ void warp_store_fp4(uint8_t* __restrict__ codes, floa
     const uint32_t byte = e2m1_code(u0 * inv) | (e2m1_code(u1 * inv) << 4);
     codes[lane ^ (static_cast<int>((s >> 2) & 1) << 4)] = static_cast<uint8_t>(byte);
     if ((lane & 15) == 0) scales[lane >> 4] = sg;
+}
+
+// Per-head keys: head h's FP4 key of entry s (lane l holds u[2l], u[2l+1] of the head's 64-vector)
+// into the entry's 128-byte row (chunk 2h + g at chunk (2h + g) ^ (s mod 8)) and its two scales
+// into scales[2h], scales[2h + 1].
+__device__ __forceinline__ void warp_store_fp4_head(uint8_t* __restrict__ row, float* __restrict__ scales, int64_t s,
+                                                    int h, int lane, float u0, float u1) {
+    float amax = fmaxf(fabsf(u0), fabsf(u1));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sg = fp4_group_scale(amax);    // lanes 0..15: group 0, lanes 16..31: group 1
+    const float inv = 1.0f / sg;               // exact: sg is a power of two
+    const uint32_t byte = e2m1_code(u0 * inv) | (e2m1_code(u1 * inv) << 4);
+    const int g = lane >> 4;
+    row[16 * ((2 * h + g) ^ static_cast<int>(s & 7)) + (lane & 15)] = static_cast<uint8_t>(byte);
+    if ((lane & 15) == 0) scales[2 * h + g] = sg;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -304,13 +346,16 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
         sm.fail = 0;
         fence_barrier_init();
     }
+    // per-head keys: four 64-column accumulators (one per head)
+    constexpr uint32_t kCols = kVar == kVarPerHead ? 4 * kCTmemCols : kCTmemCols;
     if (warp == 0) {
-        tmem_alloc(&sm.tmem_base, kCTmemCols);
+        tmem_alloc(&sm.tmem_base, kCols);
         tmem_relinquish();
     }
     // W_I^T in bf16, resident for the CTA's lifetime; 32 loads per thread in flight at a time
+    // (per-head keys: each head's W_h^T is staged in turn for every tile, below)
     constexpr int kWBatch = 32;
-    for (int i0 = 0; i0 < kDim * kIdxDim; i0 += kWBatch * kCThreads) {
+    for (int i0 = 0; kVar != kVarPerHead && i0 < kDim * kIdxDim; i0 += kWBatch * kCThreads) {
         float v[kWBatch];
 #pragma unroll
         for (int u = 0; u < kWBatch; ++u) v[u] = __ldg(w_idx + i0 + u * kCThreads + tid);
@@ -417,6 +462,81 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
         tc_fence_before();
         __syncthreads();
         if (*fail) break;
+        if constexpr (kVar == kVarPerHead) {
+            // ---- 2') per head h: W_h^T staged (the previous head's MMA has ended), one MMA chain
+            //      into columns 64h..64h+63 --------------------------------------------------------
+            bool ok = true;
+            for (int h = 0; h < kIdxHeads && ok; ++h) {
+                for (int i0 = 0; i0 < kDim * kIdxDim; i0 += kWBatch * kCThreads) {
+                    float v[kWBatch];
+#pragma unroll
+                    for (int u = 0; u < kWBatch; ++u) {
+                        const int i = i0 + u * kCThreads + tid;
+                        v[u] = __ldg(w_idx + (size_t)(i / kIdxDim) * kIdxHeads * kIdxDim + h * kIdxDim + i % kIdxDim);
+                    }
+#pragma unroll
+                    for (int u = 0; u < kWBatch; ++u) {
+                        const int i = i0 + u * kCThreads + tid;
+                        const int k = i / kIdxDim, n = i % kIdxDim;
+                        *reinterpret_cast<uint16_t*>(&sm.w[k >> 6][sw128(n, 2 * (k & 63))]) =
+                            static_cast<uint16_t>(f32_to_bf16_bits(v[u]));
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kb = 0; kb < kDim / 64; ++kb)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            umma_f16(tmem + static_cast<uint32_t>(kIdxDim * h), desc_sw128(sm.a[kb], 0) + (32 * ks) / 16,
+                                     desc_sw128(sm.w[kb], 0) + (32 * ks) / 16, kIdProj, (kb | ks) != 0 ? 1u : 0u);
+                    umma_commit(&sm.mma_done);
+                }
+                ok = !__syncthreads_or(!mbar_wait(&sm.mma_done, phase));
+                phase ^= 1u;
+                tc_fence_after();
+            }
+            if (!ok) {
+                if (tid == 0) *fail = 1;
+                break;
+            }
+            // ---- 3') FP4 keys of the four heads: warps 0-3, thread = entry -------------------
+            if (warp < 4) {
+                // every lane reads tensor memory (the loads are warp-wide); only the tile's
+                // entries are stored
+                const int r = 32 * warp + lane;
+                const int64_t s = s0 + r;
+                const bool store = r < n_here;
+                uint8_t* kdst = ikey_out + ((size_t)b * out_seq_stride + (size_t)s) * kIkeyHead;
+                float* sdst = iscale_out + ((size_t)b * out_seq_stride + (size_t)s) * (2 * kIdxHeads);
+                const int sw = static_cast<int>(s & 7);
+#pragma unroll 1
+                for (int h = 0; h < kIdxHeads; ++h) {
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        uint32_t u[2][16];
+                        const uint32_t col = static_cast<uint32_t>(kIdxDim * h + 32 * g);
+                        tmem_ld_32x32b_x16(tmem + ((32u * warp) << 16) + col, u[0]);
+                        tmem_ld_32x32b_x16(tmem + ((32u * warp) << 16) + col + 16u, u[1]);
+                        tmem_ld_wait();
+                        float sc;
+                        uint32_t words[4];
+                        fp4_group_words(u, &sc, words);
+                        // chunk 2h + g of the entry's 128-byte row, at chunk (2h + g) ^ (s mod 8)
+                        if (store) {
+                            *reinterpret_cast<uint4*>(kdst + 16 * ((2 * h + g) ^ sw)) =
+                                make_uint4(words[0], words[1], words[2], words[3]);
+                            sdst[2 * h + g] = sc;
+                        }
+                    }
+                }
+                tc_fence_before();
+            }
+            continue;
+        }
         // ---- 2) projection on the tensor cores ---------------------------------------------
         if (tid == 0) {
             tc_fence_after();
@@ -481,7 +601,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kCTmemCols);
+        tmem_dealloc(tmem, kCols);
     }
 }
 
@@ -490,10 +610,10 @@ size_t compress_index_smem_bytes() { return sizeof(CompressSmem) + 1024; }
 cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float* bias, int m,
                             const float* w_idx, int64_t T, int B, int64_t out_seq_stride,
                             uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, int num_sms,
-                            cudaStream_t stream, int64_t pos0, double rope_base, float kv_scale) {
+                            cudaStream_t stream, int64_t pos0, double rope_base, float kv_scale, bool perhead) {
     const int64_t E = T / m;
     if (E <= 0 || B <= 0) return cudaSuccess;
-    const int var = rope_base > 0.0 ? kVarRope : (kv_scale != 1.f ? kVarScaled : kVarBase);
+    const int var = perhead ? kVarPerHead : (rope_base > 0.0 ? kVarRope : (kv_scale != 1.f ? kVarScaled : kVarBase));
     const float inv_scale = 1.f / kv_scale;
     if (w_idx == nullptr) {
         const int64_t warps = E * B;
@@ -508,10 +628,12 @@ cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float*
     const int64_t grid = min64(tiles, num_sms);
     auto kernel = (m == 4) ? (var == kVarRope ? pool_index_kernel<true, kVarRope>
                                               : (var == kVarScaled ? pool_index_kernel<true, kVarScaled>
-                                                                   : pool_index_kernel<true, kVarBase>))
+                                                 : (var == kVarPerHead ? pool_index_kernel<true, kVarPerHead>
+                                                                       : pool_index_kernel<true, kVarBase>)))
                            : (var == kVarRope ? pool_index_kernel<false, kVarRope>
                                               : (var == kVarScaled ? pool_index_kernel<false, kVarScaled>
-                                                                   : pool_index_kernel<false, kVarBase>));
+                                                 : (var == kVarPerHead ? pool_index_kernel<false, kVarPerHead>
+                                                                       : pool_index_kernel<false, kVarBase>)));
     cudaError_t e = set_smem_once(kernel, smem);
     if (e != cudaSuccess) return e;
     kernel<<<static_cast<unsigned>(grid), kCThreads, smem, stream>>>(raw, gate, bias, m, w_idx, T, E, B, out_seq_stride,
@@ -748,7 +870,37 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
 #pragma unroll
             for (int d = 0; d < 16; ++d) cbuf[16 * lane + d] = bf16_bits_to_f32(f32_to_bf16_bits(c[d]));
         }
-        if (cache.has_indexer) {
+        if (kVar == kVarPerHead && cache.has_indexer) {
+            // per-head keys: the same projection for each head h with W_h (W_I [512][4][64])
+            __syncthreads();
+#pragma unroll 1
+            for (int h = 0; h < kIdxHeads; ++h) {
+                float a0 = 0.f, a1 = 0.f;
+                const float* wrow = cache.w_idx + (size_t)(64 * warp) * kIdxHeads * kIdxDim + h * kIdxDim;
+#pragma unroll 16
+                for (int d = 0; d < 64; ++d) {
+                    const float cd = cbuf[64 * warp + d];
+                    const float* wr = wrow + (size_t)d * kIdxHeads * kIdxDim;
+                    a0 = fmaf(cd, bf16_bits_to_f32(f32_to_bf16_bits(__ldg(wr + lane))), a0);
+                    a1 = fmaf(cd, bf16_bits_to_f32(f32_to_bf16_bits(__ldg(wr + 32 + lane))), a1);
+                }
+                upart[warp][lane] = a0;
+                upart[warp][32 + lane] = a1;
+                __syncthreads();
+                if (warp == 0) {
+                    float u0 = 0.f, u1 = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kAppendThreads / 32; ++w) {
+                        u0 += upart[w][2 * lane];
+                        u1 += upart[w][2 * lane + 1];
+                    }
+                    warp_store_fp4_head(cache.ikeys + ((size_t)b * cap + (size_t)s) * kIkeyHead,
+                                        cache.iscales + ((size_t)b * cap + (size_t)s) * (2 * kIdxHeads), s, h, lane, u0,
+                                        u1);
+                }
+                __syncthreads();   // upart is written again for the next head
+            }
+        } else if (cache.has_indexer) {
             __syncthreads();
             // u_j = sum_d bf16(c_d) * bf16(W_I[d][j]) in fp32 (the operands the prefill
             // projection feeds its tensor cores).  Warp w takes dims 64w..64w+63, lane outputs
@@ -781,9 +933,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(csld_layer_cache
 
 cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
                           const float* gate_new, int32_t* err, cudaStream_t stream, double rope_base,
-                          float kv_scale) {
-    auto kernel = rope_base > 0.0 ? append_kernel<kVarRope>
-                                  : (kv_scale != 1.f ? append_kernel<kVarScaled> : append_kernel<kVarBase>);
+                          float kv_scale, bool perhead) {
+    auto kernel = perhead ? append_kernel<kVarPerHead>
+                          : (rope_base > 0.0 ? append_kernel<kVarRope>
+                                             : (kv_scale != 1.f ? append_kernel<kVarScaled> : append_kernel<kVarBase>));
     cudaError_t e = launch_pdl(kernel, dim3(cache.batch), dim3(kAppendThreads), 0, stream, cache, kv_new, gate_new, err,
                                rope_base, 1.f / kv_scale);
     if (e != cudaSuccess) return e;

@@ -51,7 +51,9 @@ constexpr int kMqCopyWarp = 12, kMqMmaWarp = 13;
 struct MqSmem {
     uint8_t codes[kMqStages][kMqGroup * kIkey];     // 32 KB per group, stored (pre-swizzled) layout
     float scales[kMqStages][kMqGroup * 2];          // 8 KB per group
-    alignas(256) uint8_t bq[8 * CSLD_MULTI_MAX_Q * kIkey];   // query operand, 32-byte swizzle
+    // query operand: 32-byte rows with the 32-byte swizzle (shared keys), or 128-byte rows with
+    // the 128-byte swizzle (per-head keys: head h's codes in the row's 32-byte slice h)
+    alignas(1024) uint8_t bq[8 * CSLD_MULTI_MAX_Q * kIkey * kIdxHeads];
     float qscale[CSLD_MULTI_MAX_Q][8];              // [q][group * 4 + head]
     float hw[CSLD_MULTI_MAX_Q][kIdxHeads];          // head weights of each query
     int64_t nq[CSLD_MULTI_MAX_Q];                   // entries query q sees
@@ -64,11 +66,21 @@ struct MqSmem {
 }  // namespace
 
 // Grid (chunks, B): CTA (c, b) scores tiles c, c + chunks, ... of sequence b's visible range.
+// kKeyHeads = 1: one key shared by the 4 heads (32 code bytes + 2 scales per entry, 1,024-entry
+// copy groups).  kKeyHeads = 4: per-head keys (128 code bytes in 128-byte-swizzle rows + 8
+// scales per entry, 256-entry copy groups; one MMA per head and tile, each over the head's
+// 32-byte K slice of the keys and of the query operand, whose other heads' rows are zero there,
+// so the output columns are the same exact group dots).
+template <int kKeyHeads>
 __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
     const uint8_t* __restrict__ ikeys, const float* __restrict__ iscales, int64_t cap,
     const int32_t* __restrict__ seq_len, int ratio, const float* __restrict__ q_idx,
     const float* __restrict__ head_w, int Q, uint32_t* __restrict__ keys_out, uint32_t* __restrict__ ghist,
     int32_t* err) {
+    constexpr int kKeyBytes = kIkey * kKeyHeads;           // code bytes per entry
+    constexpr int kSf = 2 * kKeyHeads;                     // scales per entry
+    constexpr int kGroupE = kMqGroup / kKeyHeads;          // entries per copy group (32 KB of codes)
+    constexpr int kGroupTiles = kGroupE / kMqTile;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     MqSmem& sm = *reinterpret_cast<MqSmem*>(smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -115,13 +127,37 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
     __syncthreads();
     const int n_tiles_all = static_cast<int>((n_max + kMqTile - 1) / kMqTile);
     // this CTA's tiles: whole copy groups g = c, c + chunks, ...
-    const int n_groups_all = (n_tiles_all + kMqGroupTiles - 1) / kMqGroupTiles;
+    const int n_groups_all = (n_tiles_all + kGroupTiles - 1) / kGroupTiles;
     const int my_groups = n_groups_all > c ? (n_groups_all - c + chunks - 1) / chunks : 0;
-    const uint8_t* cbase = ikeys + (size_t)b * cap * kIkey;
-    const float* sbase = iscales + (size_t)b * cap * 2;
+    const uint8_t* cbase = ikeys + (size_t)b * cap * kKeyBytes;
+    const float* sbase = iscales + (size_t)b * cap * kSf;
 
     // ---- query operand (warps 0-3, then handed to the MMA warp; the copy warp starts at once) --
-    if (warp < 4) {
+    if (warp < 4 && kKeyHeads > 1) {
+        // per-head keys: 8Q rows of 128 bytes, zero but for the 16 bytes of row n = 8q + 4g + h
+        // that hold group g of head h of query q, at byte 32h + 16g of the row (16-byte chunk
+        // 2h + g, stored at chunk (2h + g) ^ (n mod 8))
+        for (int i = tid; i < 8 * Q * kIkey * kIdxHeads / 4; i += 128) reinterpret_cast<uint32_t*>(sm.bq)[i] = 0u;
+        named_barrier(2, 128);
+        for (int t = tid; t < 32 * Q; t += 128) {   // thread (n, jj): bytes 4jj .. 4jj+3 of the 16
+            const int n_row = t >> 2, jj = t & 3;
+            const int q = n_row >> 3, r8 = n_row & 7, h = r8 & 3, grp = r8 >> 2;
+            const float* qv = q_idx + (((size_t)b * Q + q) * kIdxHeads + h) * kIdxDim + 32 * grp;
+            float amax = 0.f;
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(__ldg(qv + i)));
+            const float sg = fp4_group_scale(amax);
+            const float inv = 1.0f / sg;   // exact: a power of two
+            uint32_t word = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) word |= e2m1_code(__ldg(qv + 8 * jj + i) * inv) << (4 * i);
+            *reinterpret_cast<uint32_t*>(sm.bq + n_row * (kIkey * kIdxHeads) + 16 * ((2 * h + grp) ^ r8) + 4 * jj) = word;
+            if (jj == 0) sm.qscale[q][grp * 4 + h] = sg;
+        }
+        fence_proxy_async_smem();
+        tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kMqSfCol, 0x7F7F7F7Fu);
+        tmem_st_32x32b_x8_fill(tmem + ((32u * warp) << 16) + kMqSfCol + 8, 0x7F7F7F7Fu);
+        tmem_st_wait();
+    } else if (warp < 4) {
         // thread t < 8 Q writes row n = t / 8 ... one row per 8 threads: thread (n, j) writes
         // bytes 4j .. 4j+3 of row n
         for (int t = tid; t < 64 * Q; t += 128) {
@@ -162,13 +198,15 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
                     *fail = 1;
                     break;
                 }
-                const int64_t e0 = (int64_t)(c + i * chunks) * kMqGroup;
-                const int ne = static_cast<int>(min64(kMqGroup, n_max - e0));
-                const uint32_t cb = static_cast<uint32_t>(ne) * kIkey;
-                const uint32_t sb = static_cast<uint32_t>((ne + 1) & ~1) * 8u;   // cap is even
+                const int64_t e0 = (int64_t)(c + i * chunks) * kGroupE;
+                const int ne = static_cast<int>(min64(kGroupE, n_max - e0));
+                const uint32_t cb = static_cast<uint32_t>(ne) * kKeyBytes;
+                // scales: 8 bytes per entry (an even count: cap is even) or 32 per entry
+                const uint32_t sb = kKeyHeads == 1 ? static_cast<uint32_t>((ne + 1) & ~1) * 8u
+                                                   : static_cast<uint32_t>(ne) * 4u * kSf;
                 mbar_arrive_expect_tx(&sm.full[s], cb + sb);
-                bulk_g2s(sm.codes[s], cbase + (size_t)e0 * kIkey, cb, &sm.full[s]);
-                bulk_g2s(sm.scales[s], sbase + (size_t)e0 * 2, sb, &sm.full[s]);
+                bulk_g2s(sm.codes[s], cbase + (size_t)e0 * kKeyBytes, cb, &sm.full[s]);
+                bulk_g2s(sm.scales[s], sbase + (size_t)e0 * kSf, sb, &sm.full[s]);
             }
         }
     } else if (warp == kMqMmaWarp) {
@@ -184,7 +222,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
                 }
                 tc_fence_after();
                 const int g = c + i * chunks;
-                const int nt = min(kMqGroupTiles, n_tiles_all - g * kMqGroupTiles);
+                const int nt = min(kGroupTiles, n_tiles_all - g * kGroupTiles);
                 for (int tt = 0; tt < nt; ++tt, ++t) {
                     const int slot = t % kMqSlots;
                     if (t >= kMqSlots && !mbar_wait(&sm.sfree[slot], ((t / kMqSlots) - 1) & 1)) {
@@ -192,8 +230,17 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
                         break;
                     }
                     tc_fence_after();
-                    umma_mxf4(tmem + 64u * slot, smem_desc_kmajor_sw32(sm.codes[s] + tt * kMqTile * kIkey), bdesc, idesc,
-                              tmem + kMqSfCol, tmem + kMqSfCol + 8, 0u);
+                    if constexpr (kKeyHeads == 1) {
+                        umma_mxf4(tmem + 64u * slot, smem_desc_kmajor_sw32(sm.codes[s] + tt * kMqTile * kIkey), bdesc,
+                                  idesc, tmem + kMqSfCol, tmem + kMqSfCol + 8, 0u);
+                    } else {
+                        const uint64_t ad = desc_sw128(sm.codes[s] + tt * kMqTile * kKeyBytes, 0);
+                        const uint64_t bd = desc_sw128(sm.bq, 0);
+#pragma unroll
+                        for (int h = 0; h < kKeyHeads; ++h)   // head h: the 32-byte K slice h
+                            umma_mxf4(tmem + 64u * slot, ad + (32 * h) / 16, bd + (32 * h) / 16, idesc, tmem + kMqSfCol,
+                                      tmem + kMqSfCol + 8, h > 0 ? 1u : 0u);
+                    }
                     umma_commit(&sm.accf[slot]);
                 }
                 if (*fail) break;
@@ -209,7 +256,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
         for (int i = 0; i < my_groups; ++i) {
             const int s = i % kMqStages;
             const int g = c + i * chunks;
-            const int nt = min(kMqGroupTiles, n_tiles_all - g * kMqGroupTiles);
+            const int nt = min(kGroupTiles, n_tiles_all - g * kGroupTiles);
             bool ok = true;
             for (int tt = 0; tt < nt; ++tt, ++t) {
                 if (t % kMqEpi != wg) continue;
@@ -221,8 +268,9 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
                     break;
                 }
                 tc_fence_after();
-                const int64_t e = (int64_t)g * kMqGroup + tt * kMqTile + m;
-                const float2 ks = reinterpret_cast<const float2*>(sm.scales[s])[tt * kMqTile + m];
+                const int64_t e = (int64_t)g * kGroupE + tt * kMqTile + m;
+                // key scales of this entry: (group 0, group 1) of the shared key or of each head's
+                const float* ksp = sm.scales[s] + (size_t)(tt * kMqTile + m) * kSf;
                 for (int q0 = 0; q0 < Q; q0 += 2) {   // two queries (16 columns) per load
                     uint32_t r[16];
                     tmem_ld_32x32b_x16(lane_addr + 64u * slot + 8u * q0, r);
@@ -238,8 +286,9 @@ __global__ void __launch_bounds__(kMqThreads, 1) indexer_multi_score_kernel(
                             // d = fma(I1, s1, I0*s0) with s_g = (qscale_g * kscale_g) * 0.25
                             const float i0 = __fmul_rn(__uint_as_float(r[8 * qq + h]), 4.0f);
                             const float i1 = __fmul_rn(__uint_as_float(r[8 * qq + 4 + h]), 4.0f);
-                            const float s0 = __fmul_rn(__fmul_rn(sm.qscale[q][h], ks.x), 0.25f);
-                            const float s1 = __fmul_rn(__fmul_rn(sm.qscale[q][4 + h], ks.y), 0.25f);
+                            const int kh = kKeyHeads == 1 ? 0 : 2 * h;
+                            const float s0 = __fmul_rn(__fmul_rn(sm.qscale[q][h], ksp[kh]), 0.25f);
+                            const float s1 = __fmul_rn(__fmul_rn(sm.qscale[q][4 + h], ksp[kh + 1]), 0.25f);
                             const float d = __fmaf_rn(i1, s1, __fmul_rn(i0, s0));
                             rr[h] = d > 0.f ? d : 0.f;
                         }
@@ -622,7 +671,8 @@ size_t indexer_multi_ws_bytes(int B, int Q, int64_t cap, int num_sms) {
 
 cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int64_t cap, const int32_t* seq_len,
                                  int ratio, const float* q_idx, const float* head_w, int B, int Q, int k,
-                                 int32_t* topk_out, void* ws, int num_sms, int32_t* err, cudaStream_t stream) {
+                                 int32_t* topk_out, void* ws, int num_sms, int32_t* err, cudaStream_t stream,
+                                 bool perhead) {
     const int P = indexer_multi_parts(B, Q, num_sms);
     const size_t rows = (size_t)B * Q;
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -632,13 +682,15 @@ cudaError_t launch_indexer_multi(const uint8_t* ikeys, const float* iscales, int
     uint32_t* counts = reinterpret_cast<uint32_t*>(w8 + up(rows * (size_t)cap * 4) + up(rows * kMqBins * 4));
     uint2* lists = reinterpret_cast<uint2*>(w8 + up(rows * (size_t)cap * 4) + up(rows * kMqBins * 4) + up(rows * P * 4));
     const size_t smem = indexer_multi_smem_bytes();
-    cudaError_t e = set_smem_once(indexer_multi_score_kernel, smem);
+    auto score = perhead ? indexer_multi_score_kernel<kIdxHeads> : indexer_multi_score_kernel<1>;
+    cudaError_t e = set_smem_once(score, smem);
     if (e != cudaSuccess) return e;
     // copy groups of every sequence spread over about one CTA per SM
-    const int64_t groups = (cap + kMqGroup - 1) / kMqGroup;
+    const int64_t group_e = perhead ? kMqGroup / kIdxHeads : kMqGroup;
+    const int64_t groups = (cap + group_e - 1) / group_e;
     int64_t chunks = max64(1, num_sms / max(B, 1));
     chunks = min64(chunks, groups);
-    e = launch_pdl(indexer_multi_score_kernel, dim3(static_cast<unsigned>(chunks), B), dim3(kMqThreads), smem, stream,
+    e = launch_pdl(score, dim3(static_cast<unsigned>(chunks), B), dim3(kMqThreads), smem, stream,
                    ikeys, iscales, cap, seq_len, ratio, q_idx, head_w, Q, keys, ghist, err);
     if (e != cudaSuccess) return e;
     e = launch_pdl(indexer_multi_gather_kernel, dim3(P, Q, B), dim3(kMqSelThreads), 0, stream,

@@ -11,11 +11,13 @@ namespace csld {
 
 // Layout variants (at most one at a time): rope_base > 0, RoPE at compressed positions with raw
 // token 0 at position pos0 (entry s rotated at pos0 + (s+1) m - 1); kv_scale != 1, scaled FP8
-// entries (E4M3(x / kv_scale)).  rope_base = 0 and kv_scale = 1: the base layout.
+// entries (E4M3(x / kv_scale)); perhead, per-head indexer keys (w_idx [512][4][64], keys
+// [..][128 B] swizzled, scales [..][4][2]).  rope_base = 0, kv_scale = 1, !perhead: the base layout.
 cudaError_t launch_compress(const uint16_t* raw, const float* gate, const float* bias, int m,
                             const float* w_idx, int64_t T, int B, int64_t out_seq_stride,
                             uint8_t* kv_out, uint8_t* ikey_out, float* iscale_out, int num_sms,
-                            cudaStream_t stream, int64_t pos0 = 0, double rope_base = 0.0, float kv_scale = 1.f);
+                            cudaStream_t stream, int64_t pos0 = 0, double rope_base = 0.0, float kv_scale = 1.f,
+                            bool perhead = false);
 size_t compress_index_smem_bytes();
 cudaError_t launch_compress_channel(const uint16_t* raw, const float* gate, const float* bias, int m,
                                     const float* w_idx, int64_t T, uint8_t* kv_out, uint8_t* ikey_out,
@@ -28,7 +30,7 @@ cudaError_t launch_prefill_state(const uint16_t* raw, const float* gate, int64_t
 
 cudaError_t launch_append(const csld_layer_cache& cache, const uint16_t* kv_new,
                           const float* gate_new, int32_t* err, cudaStream_t stream, double rope_base = 0.0,
-                          float kv_scale = 1.f);
+                          float kv_scale = 1.f, bool perhead = false);
 
 // Lightning indexer + top-k.
 struct IndexerPlan {

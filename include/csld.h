@@ -216,6 +216,35 @@ CSLD_API csld_status kv_cache_prefill_rope(const csld_layer_cache* cache, const 
                                            const float* gate, int64_t T, double rope_base, void* stream);
 
 /* ----------------------------------------------------------------------------------------
+ * Per-head indexer keys -- a layout variant of the lightning indexer ([HF] CSA paragraph:
+ * "FP4, ReLU-scored multi-head dot product"), where every one of the 4 indexer heads has its own
+ * projection and its own key per entry, instead of one key shared by the heads:
+ *   u_h = c . W_h (bf16 operands, fp32 accumulation),  w_idx [512][4][64] f32 (W_h[d][j] at
+ *   d*256 + h*64 + j);  key h = FP4 of u_h exactly as the shared key is quantised.
+ * Stored layout: ikey_out / ikeys [entries][128] u8 -- the four heads' 32 code bytes in head
+ * order, and within each 8-entry block the 16-byte chunk c (c = 2*head + group) of entry s
+ * stored at chunk c ^ (s mod 8) (the tensor cores' 128-byte swizzle); iscale_out / iscales
+ * [entries][4][2] f32.  T/ratio entries; 16-byte alignment as for csld_compress.
+ *   csld_compress_perhead, kv_cache_prefill_perhead, kv_cache_append_perhead: as csld_compress,
+ *     kv_cache_prefill, kv_cache_append with such keys (the cache's ikeys [B][capacity][128],
+ *     iscales [B][capacity][4][2], w_idx [512][4][64]);
+ *   indexer_topk_perhead: as indexer_topk_multi (Q query tokens per sequence, 1 <= Q <=
+ *     CSLD_MULTI_MAX_Q; Q = 1 is the decode step), head h's dot taken against key h, with the
+ *     same fp32 operation order; workspace csld_indexer_multi_workspace_size(B, Q, cap).
+ * -------------------------------------------------------------------------------------- */
+CSLD_API csld_status csld_compress_perhead(const uint16_t* raw, const float* gate, const float* pos_bias,
+                                           int ratio, const float* w_idx, int64_t T, uint8_t* kv_out,
+                                           uint8_t* ikey_out, float* iscale_out, void* stream);
+CSLD_API csld_status kv_cache_prefill_perhead(const csld_layer_cache* cache, const uint16_t* raw,
+                                              const float* gate, int64_t T, void* stream);
+CSLD_API csld_status kv_cache_append_perhead(const csld_layer_cache* cache, const uint16_t* kv_new,
+                                             const float* gate_new, int32_t* err, void* stream);
+CSLD_API csld_status indexer_topk_perhead(const uint8_t* ikeys, const float* iscales, int64_t cap,
+                                          const int32_t* seq_len, int ratio, const float* q_idx,
+                                          const float* head_w, int B, int Q, int k, int32_t* topk_out,
+                                          void* ws, size_t ws_bytes, int32_t* err, void* stream);
+
+/* ----------------------------------------------------------------------------------------
  * Scaled FP8 entries -- a layout variant of the storage paragraph ([HF]: entries FP8 except the
  * RoPE dims in bf16), with one positive scale kv_scale (sigma) per layer cache: an entry's (and
  * a window entry's) 448 FP8 dims hold E4M3(x / sigma), RNE, saturating at +-448, and stand for
