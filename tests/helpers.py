@@ -208,3 +208,20 @@ def planted_near_tie(n=2048, k=10, a=500, b=600):
     q[0, 1, 32:] = 1.0
     w = torch.tensor([[1.0, 2.0 ** -30, 0.0, 0.0]])
     return ik, isc, q, w, big
+
+
+def plant_aligned(comp, q, idx, g):
+    """Overwrite entries idx[b] of comp [B,cap,576] with alpha * q[b, h] + N(0, 0.3^2) for a head h
+    cycling over the 16 heads and alpha drawn from U(0.15, 0.6): each head then has a dozen or
+    more entries whose logits stand 3-14 units above the rest, so its softmax is dominated by a
+    few entries with distinct weights and distinct values (|out| ~ 0.3, far above the 2e-2
+    absolute bar), unlike N(0,1) caches whose outputs are near-uniform averages."""
+    B = comp.shape[0]
+    qf = q.float()
+    for b in range(B):
+        n = len(idx[b])
+        heads = torch.arange(n) % 16
+        alpha = 0.15 + 0.45 * torch.rand(n, generator=g)
+        x = alpha[:, None] * qf[b, heads] + 0.3 * torch.randn((n, 512), generator=g)
+        comp[b, idx[b], :448] = x[:, :448].to(torch.float8_e4m3fn).view(torch.uint8)
+        comp[b, idx[b], 448:] = x[:, 448:].to(torch.bfloat16).view(torch.uint8).reshape(n, 128)

@@ -126,23 +126,6 @@ def test_full_workload_dense_and_sparse(csld, orc, name):
 
 
 
-def _plant_aligned(comp, q, idx, g):
-    """Overwrite entries idx[b] of comp [B,cap,576] with alpha * q[b, h] + N(0, 0.3^2) for a head h
-    cycling over the 16 heads and alpha drawn from U(0.15, 0.6): each head then has a dozen or
-    more entries whose logits stand 3-14 units above the rest, so its softmax is dominated by a
-    few entries with distinct weights and distinct values (|out| ~ 0.3, far above the 2e-2
-    absolute bar), unlike N(0,1) caches whose outputs are near-uniform averages."""
-    B = comp.shape[0]
-    qf = q.float()
-    for b in range(B):
-        n = len(idx[b])
-        heads = torch.arange(n) % 16
-        alpha = 0.15 + 0.45 * torch.rand(n, generator=g)
-        x = alpha[:, None] * qf[b, heads] + 0.3 * torch.randn((n, 512), generator=g)
-        comp[b, idx[b], :448] = x[:, :448].to(torch.float8_e4m3fn).view(torch.uint8)
-        comp[b, idx[b], 448:] = x[:, 448:].to(torch.bfloat16).view(torch.uint8).reshape(n, 128)
-
-
 @pytest.mark.parametrize("mode", ["hca", "csa"])
 def test_full_workload_peaked_softmax(csld, orc, mode):
     """The 1M-token workload (B = 8) with a peaked softmax: a few hundred entries per sequence
@@ -165,7 +148,7 @@ def test_full_workload_peaked_softmax(csld, orc, mode):
                            for _ in range(B)]).to(torch.int32)
         idx = [sel[b, torch.randperm(wl.topk, generator=g)[:256]].long() for b in range(B)]
         ratio = wl.csa_ratio
-    _plant_aligned(comp, q, idx, g)
+    H.plant_aligned(comp, q, idx, g)
     out, lse, ro, rl, err = _run(csld, orc, q, comp, ratio, sel, win, wl.window, seq)
     assert err == 0
     assert np.abs(ro).max() > 0.5 and np.median(np.abs(ro)) > 0.05   # the case really is peaked

@@ -88,3 +88,46 @@ def test_multi_query_window_only_block(csld, orc):
         ro, rl = orc.attention_batch(synth.bits16(q[:, j].contiguous()), comp.numpy(), 128, None, rings,
                                      np.full(B, n_j, np.int32), SCALE)
         H.assert_attention_close(out[:, j].cpu().numpy(), lse[:, j].cpu().numpy(), ro, rl, f"window-only query {j}")
+
+
+@pytest.mark.parametrize("mode", ["dense", "sparse"])
+def test_multi_query_full_size_peaked(csld, orc, mode):
+    """The multi-token workload at full size: 4 query tokens per sequence at 1M tokens, dense over
+    the 8,192 HCA entries of all 8 sequences (the last query alone sees entry 8,191), or sparse
+    over each query's own top-1024 of 262,144 CSA entries (2 sequences); window 128 in a ring of
+    131 slots.  128 entries per query are aligned with that query's heads, so every softmax is
+    peaked and a weight or value error of a few percent fails the bar."""
+    wl = synth.WORKLOADS["decode1m"]
+    Q, W, n = 4, wl.window, wl.context
+    W_ring = W + Q - 1
+    g = synth.gen(77)
+    B = wl.batch if mode == "dense" else 2
+    ratio = wl.hca_ratio if mode == "dense" else wl.csa_ratio
+    comp = synth.random_entries((B, wl.hca_cap if mode == "dense" else wl.csa_cap), g)
+    ring = synth.random_entries((B, W_ring), g)
+    q = synth.decode_queries(B * Q, seed=78)["q"].view(B, Q, 16, 512).contiguous()
+    seq = torch.full((B,), n, dtype=torch.int32)
+    sel = None
+    if mode == "sparse":
+        sel = torch.stack([torch.stack([torch.sort(torch.randperm((n - (Q - 1 - j)) // ratio, generator=g)[:wl.topk]).values
+                                        for j in range(Q)]) for _ in range(B)]).to(torch.int32)
+    for j in range(Q):
+        if mode == "sparse":
+            idx = [sel[b, j, torch.randperm(wl.topk, generator=g)[:128]].long() for b in range(B)]
+        else:
+            idx = [torch.randperm(wl.hca_entries, generator=g)[:128] for _ in range(B)]
+        H.plant_aligned(comp, q[:, j], idx, g)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = csld.hybrid_decode_attention_multi(q.cuda(), comp.cuda(), ratio, None if sel is None else sel.cuda(),
+                                                  ring.cuda(), W, seq.cuda(), SCALE, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for j in range(Q):
+        n_j = n - (Q - 1 - j)
+        rings = np.stack([_ring_for(ring[b].numpy(), n_j, W, W_ring) for b in range(B)])
+        ro, rl = orc.attention_batch(synth.bits16(q[:, j].contiguous()), comp.numpy(), ratio,
+                                     None if sel is None else sel[:, j].contiguous().numpy(), rings,
+                                     np.full(B, n_j, np.int32), SCALE)
+        assert np.abs(ro).max() > 0.5 and np.median(np.abs(ro)) > 0.05   # the case really is peaked
+        H.assert_attention_close(out[:, j], lse[:, j], ro, rl, f"mtp1m {mode} query {j} of {Q}")

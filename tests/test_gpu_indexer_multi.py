@@ -29,7 +29,8 @@ def _queries(B, Q, seed):
 
 @pytest.mark.parametrize("B,Q,n,k,ratio", [(2, 8, 4 * 20000 + 3, 512, 4), (3, 5, 4 * 3000, 256, 4),
                                            (1, 1, 4 * 1500 + 2, 128, 4), (4, 8, 4 * 600, 1024, 4),
-                                           (2, 3, 9 * 2000 + 4, 100, 9), (1, 8, 4 * 262144, 1024, 4)])
+                                           (2, 3, 9 * 2000 + 4, 100, 9), (1, 8, 4 * 262144, 1024, 4),
+                                           (8, 4, 4 * 262144, 1024, 4)])
 def test_multi_query_matches_oracle_and_single_query(csld, orc, B, Q, n, k, ratio):
     n_c = n // ratio
     cap = n_c + 64
