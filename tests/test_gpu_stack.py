@@ -30,16 +30,26 @@ def test_layer_pattern(csld):
     assert all(kinds[i] != kinds[i + 1] for i in range(2, 60))
 
 
-@pytest.mark.parametrize("ctx,B,k", [(65536 - 3, 2, 512), (4096 + 77, 3, 128)])
+@pytest.mark.parametrize("ctx,B,k", [(65536 - 3, 2, 512), (4096 + 77, 3, 128), (1 << 20, 8, 1024)])
 def test_stack_step_matches_oracle_on_sampled_layers(csld, orc, ctx, B, k):
+    """One decode step through all 61 layers (each prefilled from its own raw tokens), checked on
+    sampled (layer, sequence) slices.  The 1M-token, batch-8 case is the sweep's headline point in
+    the bench's launch configuration (about 40 GB of caches)."""
+    # caches (CSA entries and keys on half the layers), the raw tokens of one layer, and the fp32
+    # draws of one sequence, roughly
+    need = 61 * B * (ctx // 4) * 616 // 2 + 2 * B * ctx * 512 + 8 * ctx * 512 + (1 << 30)
+    if torch.cuda.mem_get_info()[0] < need:
+        pytest.skip(f"needs about {need / 1e9:.0f} GB of free device memory")
     kinds = csld.layer_pattern(61)
     L, W = len(kinds), 128
     inp = synth.prefill_inputs(8, seed=1)
     st = csld.DecodeStack(B, kinds, (ctx + 64) // 4, (ctx + 256) // 128, W, k, inp["bias4"], inp["bias128"],
                           inp["w_idx"])
     g = synth.gen(2, "cuda")
+    raw = torch.empty((B, ctx, 512), dtype=torch.bfloat16, device="cuda")
     for lay in st.layers:   # a distinct prefill per layer
-        raw = synth.bf16_normal((B, ctx, 512), g, "cuda")
+        for b in range(B):
+            raw[b] = synth.bf16_normal((ctx, 512), g, "cuda")
         gate = torch.randn((B, ctx), generator=g, device="cuda")
         csld.kv_cache_prefill(lay, raw, gate)
     del raw, gate
