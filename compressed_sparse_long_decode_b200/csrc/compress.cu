@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
 
 // ------------------------------------------------------------------------------------------
 // Pooling + indexer key (CSA) on the 5th-generation tensor cores.  Persistent CTAs (one per
-// SM) of 16 warps over 128-entry tiles:
+// SM) of 16 warps, each over an even share of the entries in tiles of up to 128 entries:
 //  1. every warp pools 8 entries of the tile (one warp per entry, as above; for m = 4 two
 //     entries' raw rows are loaded at once, 256 bytes per lane in flight) and writes each
 //     entry to the cache and its bf16 copy into shared memory as row r of the A operand
@@ -374,15 +374,19 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
     const uint32_t tmem = sm.tmem_base;
     volatile int32_t* fail = &sm.fail;
 
-    const int64_t tiles_per_seq = (E + kCTile - 1) / kCTile;
-    const int64_t n_tiles = tiles_per_seq * B;
+    // this CTA's entries: an even share [lo, hi) of the B x E entries, walked in tiles of up to
+    // kCTile that do not cross a sequence (an even share keeps the longest CTA at ceil(B E /
+    // grid) entries instead of two whole tiles when the tile count is not a multiple of the grid)
+    const int64_t total = E * B;
+    const int64_t lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
     const float bias_l = (kM4 && lane < 4) ? __ldg(bias + lane) : 0.f;   // slot l's positional bias
     uint32_t phase = 0;
     bool mma_pending = false;   // an MMA reading sm.a was issued and this warp has not seen it end
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t b = tile / tiles_per_seq;
-        const int64_t s0 = (tile % tiles_per_seq) * kCTile;
-        const int n_here = static_cast<int>(min64(kCTile, E - s0));
+    for (int64_t g0 = lo; g0 < hi;) {
+        const int64_t b = g0 / E;
+        const int64_t s0 = g0 % E;
+        const int n_here = static_cast<int>(min64(min64(kCTile, E - s0), hi - g0));
+        g0 += n_here;
         const uint16_t* rb = raw + (size_t)b * T * kDim;
         const float* gb = gate + (size_t)b * T;
         uint8_t* kvb = kv_out + (size_t)b * out_seq_stride * kEntry;
