@@ -172,18 +172,18 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
 
 // E2M1 code of v (|v| <= 6 expected; larger saturates): nearest grid value, ties to the even
 // mantissa (0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4).  Bit 3 = sign.
+// Branch-free: the magnitude index is the number of midpoints between grid values that lie
+// below |v|, a midpoint counting when |v| is past it (strictly, where the even index is below
+// it; from the midpoint on, where the even index is above it); NaN gives 7, as the branch
+// chain it replaces did for every input.  A chain of branches here diverges across the lanes of
+// a warp (every lane holds a different value) and serialises the FP4 quantisation of the keys.
 __device__ __forceinline__ uint32_t e2m1_code(float v) {
     const float a = fabsf(v);
-    uint32_t m;
-    if (a <= 0.25f) m = 0;
-    else if (a < 0.75f) m = 1;
-    else if (a <= 1.25f) m = 2;
-    else if (a < 1.75f) m = 3;
-    else if (a <= 2.5f) m = 4;
-    else if (a < 3.5f) m = 5;
-    else if (a <= 5.0f) m = 6;
-    else m = 7;
-    return (signbit(v) ? 8u : 0u) | m;
+    const uint32_t m = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
+                       static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
+                       static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
+                       static_cast<uint32_t>(a > 5.0f);
+    return (signbit(v) ? 8u : 0u) | (a != a ? 7u : m);
 }
 
 // Twice the value of an E2M1 magnitude index 0..7 (an integer): 0,1,2,3,4,6,8,12.
