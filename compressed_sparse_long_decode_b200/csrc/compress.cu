@@ -352,21 +352,34 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
         tmem_alloc(&sm.tmem_base, kCols);
         tmem_relinquish();
     }
-    // W_I^T in bf16, resident for the CTA's lifetime; 32 loads per thread in flight at a time
-    // (per-head keys: each head's W_h^T is staged in turn for every tile, below)
-    constexpr int kWBatch = 32;
-    for (int i0 = 0; kVar != kVarPerHead && i0 < kDim * kIdxDim; i0 += kWBatch * kCThreads) {
-        float v[kWBatch];
+    // W_I^T in bf16, resident for the CTA's lifetime.  It is first needed by the first tile's
+    // projection, so it is staged during that tile's pooling: part p (of 4) in pooling iteration
+    // p, after the iteration's row loads are issued.  Chunk c (8 per thread) = column n = c % 64
+    // and rows k0 = 8 (c / 64) .. k0 + 7 of W_I: 8 loads coalesced across the warp's columns,
+    // one 16-byte store of the 8 bf16 values (K-major, 128-byte swizzle).
+    // (Per-head keys: each head's W_h^T is staged in turn for every tile, below.)
+    constexpr int kWBatch = 32;   // per-head staging: loads per thread in flight at a time
+    auto stage_wi_part = [&](int part) {
+        if constexpr (kVar == kVarPerHead) return;
+        constexpr int kChunks = kDim * kIdxDim / 8 / kCThreads;   // 8 chunks per thread
+        constexpr int kPer = kChunks / 4;                          // per pooling iteration
+        float v[kPer][8];
 #pragma unroll
-        for (int u = 0; u < kWBatch; ++u) v[u] = __ldg(w_idx + i0 + u * kCThreads + tid);
+        for (int q = 0; q < kPer; ++q) {
+            const int c = tid + kCThreads * (kPer * part + q);
+            const int n = c % kIdxDim, k0 = 8 * (c / kIdxDim);
 #pragma unroll
-        for (int u = 0; u < kWBatch; ++u) {
-            const int i = i0 + u * kCThreads + tid;
-            const int k = i / kIdxDim, n = i % kIdxDim;
-            *reinterpret_cast<uint16_t*>(&sm.w[k >> 6][sw128(n, 2 * (k & 63))]) =
-                static_cast<uint16_t>(f32_to_bf16_bits(v[u]));
+            for (int j = 0; j < 8; ++j) v[q][j] = __ldg(w_idx + (k0 + j) * kIdxDim + n);
         }
-    }
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int c = tid + kCThreads * (kPer * part + q);
+            const int n = c % kIdxDim, k0 = 8 * (c / kIdxDim);
+            *reinterpret_cast<uint4*>(&sm.w[k0 >> 6][sw128(n, 2 * (k0 & 63))]) =
+                make_uint4(f32x2_to_bf16x2_bits(v[q][0], v[q][1]), f32x2_to_bf16x2_bits(v[q][2], v[q][3]),
+                           f32x2_to_bf16x2_bits(v[q][4], v[q][5]), f32x2_to_bf16x2_bits(v[q][6], v[q][7]));
+        }
+    };
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -382,6 +395,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
     const float bias_l = (kM4 && lane < 4) ? __ldg(bias + lane) : 0.f;   // slot l's positional bias
     uint32_t phase = 0;
     bool mma_pending = false;   // an MMA reading sm.a was issued and this warp has not seen it end
+    bool first_tile = true;
     for (int64_t g0 = lo; g0 < hi;) {
         const int64_t b = g0 / E;
         const int64_t s0 = g0 % E;
@@ -392,7 +406,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
         uint8_t* kvb = kv_out + (size_t)b * out_seq_stride * kEntry;
 
         // ---- 1) pooling: rows warp, warp + 16, ...; kRif rows at a time ------------------
-        for (int r0 = warp; r0 < kCTile; r0 += kRif * kWarps) {
+        for (int r0 = warp, it = 0; r0 < kCTile; r0 += kRif * kWarps, ++it) {
             // entries go to the cache as soon as they are pooled; their bf16 copies wait in
             // registers for the shared-memory operand to be free
             uint32_t packed[kRif][8];
@@ -409,6 +423,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                         if (lane < 4) ga[h] = __ldg(gb + (s0 + r) * 4 + lane);
                     }
                 }
+                if (first_tile) stage_wi_part(it);
 #pragma unroll
                 for (int h = 0; h < kRif; ++h) {
                     const int r = r0 + h * kWarps;
@@ -428,6 +443,7 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                         packed[h][q] = f32_to_bf16_bits(c[2 * q]) | (f32_to_bf16_bits(c[2 * q + 1]) << 16);
                 }
             } else {
+                if (first_tile) stage_wi_part(it);
 #pragma unroll 1
                 for (int h = 0; h < kRif; ++h) {
                     const int r = r0 + h * kWarps;
@@ -462,7 +478,8 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
                     make_uint4(packed[h][4], packed[h][5], packed[h][6], packed[h][7]);
             }
         }
-        fence_proxy_async_smem();
+        first_tile = false;
+        fence_proxy_async_smem();   // the pooled rows (and, after the first tile, W_I) for the MMA
         tc_fence_before();
         __syncthreads();
         if (*fail) break;
