@@ -283,8 +283,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
 //  2. one thread issues the projection U = A . W_I (tcgen05.mma kind::f16, M = 128 entries,
 //     N = 64, K = 512 in 32 steps of 16; W_I^T resident in shared memory in the same layout)
 //     into 64 fp32 columns of tensor memory;
-//  3. warps 0-3 read U back (thread = entry = TMEM lane) and FP4-quantise its two 32-value
-//     groups in registers, writing the 32 code bytes (stored layout of csld.h) and 2 scales.
+//  3. warps 0-7 read U back (thread = entry = TMEM lane; warps 0-3 the first 32-value group,
+//     warps 4-7 the second) and FP4-quantise it in registers, writing 16 code bytes (stored
+//     layout of csld.h) and a scale each.
 // Each warp's first write of the next tile's A rows waits for the MMA that read the previous
 // tile, so the pooling loads of the next tile are already in flight meanwhile.
 // ------------------------------------------------------------------------------------------
@@ -570,49 +571,47 @@ __global__ void __launch_bounds__(kCThreads, 1) pool_index_kernel(
             umma_commit(&sm.mma_done);
         }
         mma_pending = true;
-        // ---- 3) FP4 keys: warps 0-3, thread = entry ------------------------------------------
-        if (warp < 4) {
+        // ---- 3) FP4 keys: warps 0-7, thread = entry; warps 0-3 quantise group 0 (columns
+        //      0..31), warps 4-7 group 1 (columns 32..63) of their lane quarter's entries -------
+        if (warp < 8) {
             const bool ok = mbar_wait(&sm.mma_done, phase);
             mma_pending = false;
             if (!ok) *fail = 1;
             tc_fence_after();
-            const int r = 32 * warp + lane;
+            const int quarter = warp & 3, g = warp >> 2;
+            const int r = 32 * quarter + lane;
             const int64_t s = s0 + r;
             const int sw = static_cast<int>((s >> 2) & 1);
             const bool store = ok && r < n_here;
-            uint4* kdst = reinterpret_cast<uint4*>(ikey_out + ((size_t)b * out_seq_stride + (size_t)s) * kIkey);
-            float sc[2];
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {   // group g = columns 32g .. 32g+31
-                uint32_t u[2][16];
-                tmem_ld_32x32b_x16(tmem + ((32u * warp) << 16) + 32u * g, u[0]);
-                tmem_ld_32x32b_x16(tmem + ((32u * warp) << 16) + 32u * g + 16u, u[1]);
-                tmem_ld_wait();
-                float amax = 0.f;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(u[i >> 4][i & 15])));
-                sc[g] = fp4_group_scale(amax);
-                const float inv = 1.0f / sc[g];   // exact: a power of two
-                uint32_t words[4];
-#pragma unroll
-                for (int wq = 0; wq < 4; ++wq) {
-                    uint32_t word = 0u;
-#pragma unroll
-                    for (int bq = 0; bq < 4; ++bq) {
-                        const int i = 8 * wq + 2 * bq;   // elements i, i+1 of the group
-                        const uint32_t byte = e2m1_code(__uint_as_float(u[i >> 4][i & 15]) * inv) |
-                                              (e2m1_code(__uint_as_float(u[(i + 1) >> 4][(i + 1) & 15]) * inv) << 4);
-                        word |= byte << (8 * bq);
-                    }
-                    words[wq] = word;
-                }
-                // group g's 16 bytes go to half g XOR (bit 2 of s) of the stored key
-                if (store) kdst[g ^ sw] = make_uint4(words[0], words[1], words[2], words[3]);
-            }
+            uint32_t u[2][16];
+            tmem_ld_32x32b_x16(tmem + ((32u * quarter) << 16) + 32u * g, u[0]);
+            tmem_ld_32x32b_x16(tmem + ((32u * quarter) << 16) + 32u * g + 16u, u[1]);
+            tmem_ld_wait();
             tc_fence_before();
-            if (store)
-                *reinterpret_cast<float2*>(iscale_out + ((size_t)b * out_seq_stride + (size_t)s) * 2) =
-                    make_float2(sc[0], sc[1]);
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(u[i >> 4][i & 15])));
+            const float sc = fp4_group_scale(amax);
+            const float inv = 1.0f / sc;   // exact: a power of two
+            uint32_t words[4];
+#pragma unroll
+            for (int wq = 0; wq < 4; ++wq) {
+                uint32_t word = 0u;
+#pragma unroll
+                for (int bq = 0; bq < 4; ++bq) {
+                    const int i = 8 * wq + 2 * bq;   // elements i, i+1 of the group
+                    const uint32_t byte = e2m1_code(__uint_as_float(u[i >> 4][i & 15]) * inv) |
+                                          (e2m1_code(__uint_as_float(u[(i + 1) >> 4][(i + 1) & 15]) * inv) << 4);
+                    word |= byte << (8 * bq);
+                }
+                words[wq] = word;
+            }
+            // group g's 16 bytes go to half g XOR (bit 2 of s) of the stored key
+            if (store) {
+                reinterpret_cast<uint4*>(ikey_out + ((size_t)b * out_seq_stride + (size_t)s) * kIkey)[g ^ sw] =
+                    make_uint4(words[0], words[1], words[2], words[3]);
+                iscale_out[((size_t)b * out_seq_stride + (size_t)s) * 2 + g] = sc;
+            }
         }
         phase ^= 1u;
     }
