@@ -6,9 +6,9 @@ loop that must not enter the CUDA allocator between steps.  For them the library
 fixed scratch array of its own.  This test drives that entry point through the C ABI
 (ctypes on libcsld.so) and checks that, on two calls in a row, it returns what the regular
 entry point with a caller workspace returns, within the attention tolerance the other tests
-use.  It also checks that a call needing more scratch than the array holds is refused before
-anything is launched.  It must pass on its own in a fresh process as well as after the
-other tests (this file is collected last).
+use, and what the float64 oracle returns.  It also checks that a call needing more scratch
+than the array holds is refused before anything is launched.  It must pass on its own in a
+fresh process as well as after the other tests (this file is collected last).
 """
 import ctypes as C
 import math
@@ -84,15 +84,25 @@ def _run_both(lib, comp, win, q, seq, sel, ratio, W):
     return out_ws.cpu().numpy(), lse_ws.cpu().numpy(), out_st.cpu().numpy(), lse_st.cpu().numpy()
 
 
-def test_static_scratch_matches_workspace_entry_point_twice(lib):
+def _oracle(orc, comp, win, q, seq, sel, ratio):
+    return orc.attention_batch(synth.bits16(q.cpu()), comp.cpu().numpy(), ratio,
+                               None if sel is None else sel.cpu().numpy(), win.cpu().numpy(), seq.cpu().numpy(),
+                               1.0 / math.sqrt(512.0))
+
+
+def test_static_scratch_matches_workspace_entry_point_twice(lib, orc):
     # first call: dense (HCA-like), 8 sequences
     comp, win, q, seq, _ = _case(8, 700, 128, 128, 0, seed=71)
     o1, l1, o2, l2 = _run_both(lib, comp, win, q, seq, None, 128, 128)
     H.assert_attention_close(o2, l2, o1, l1, "static scratch, first call (dense)")
+    ro, rl = _oracle(orc, comp, win, q, seq, None, 128)
+    H.assert_attention_close(o2, l2, ro, rl, "static scratch, first call (dense), against the oracle")
     # second call in a row reuses the same scratch: sparse (CSA-like), different shape
     comp, win, q, seq, sel = _case(3, 5000, 4, 64, 512, seed=72)
     o1, l1, o2, l2 = _run_both(lib, comp, win, q, seq, sel, 4, 64)
     H.assert_attention_close(o2, l2, o1, l1, "static scratch, second call (sparse)")
+    ro, rl = _oracle(orc, comp, win, q, seq, sel, 4)
+    H.assert_attention_close(o2, l2, ro, rl, "static scratch, second call (sparse), against the oracle")
     assert np.isfinite(o2).all()
 
 
