@@ -24,8 +24,9 @@ replicas rotating so that no step finds its data in L2 from the step before), be
 synchronize + barrier on both sides, timed with CUDA events on the launching stream; the job time
 is the max over ranks.  Without --steps, K is chosen so the timed region lasts about 1.2 s.  The
 kernels of the timed graphs keep their programmatic (early-launch) edges; a second capture of the
-same launches with event records between the kernels gives the per-kernel times and the
-roofline of the dominant kernel.  `--impl reference` times the float64 CPU oracle instead (on
+same launches with event records between the kernels gives the per-kernel times inside the
+step, and a graph of each operation's calls alone (rotating over cache copies, so no launch finds
+its data in L2) gives the per-launch durations behind the roofline of the dominant kernel.  `--impl reference` times the float64 CPU oracle instead (on
 rank 0 only), on a bounded sample of the same workload.
 """
 import argparse
