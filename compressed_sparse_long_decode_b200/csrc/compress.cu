@@ -89,7 +89,6 @@ __device__ __forceinline__ void warp_pool(const uint16_t* rows, const float* gat
                                           const float* __restrict__ bias, int m, int lane,
                                           float (&c)[16]) {
     float w[4];
-    warp_pool_weights(gate, bias, m, lane, w);
 #pragma unroll
     for (int d = 0; d < 16; ++d) c[d] = 0.f;
     const uint4* base = reinterpret_cast<const uint4*>(rows) + 2 * lane;
@@ -109,6 +108,8 @@ __device__ __forceinline__ void warp_pool(const uint16_t* rows, const float* gat
                     x[r][1] = load_row16<kReadOnly>(base + (size_t)j * (kDim / 8) + 1);
                 }
             }
+            // the weights, once, while the first batch of rows is in flight
+            if (i == 0 && j0 == 0) warp_pool_weights(gate, bias, m, lane, w);
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 if (j0 + r >= jn) break;
